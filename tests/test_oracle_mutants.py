@@ -1,0 +1,69 @@
+"""Plant plausible mistakes in a copy of the oracle and check a pin catches each.
+
+Every mutant is the oracle's C source with one textual edit (a dropped term,
+a wrong sign, a wrong index, a transposed mapping), compiled into a temporary
+directory.  The real oracle is never modified.  A mutant that passes every
+pin would mean the pins cannot tell that mistake from the correct oracle.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle_checks import ALL_CHECKS
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTANTS = {
+    "drop_scale": ("s[j - j0] = scale * dot;", "s[j - j0] = dot;"),
+    "exp_sign": ("double w = exp(s[j - j0] - m);", "double w = exp(m - s[j - j0]);"),
+    "gqa_mapping": ("hq = (int)(r % H_q), g = hq / G;", "hq = (int)(r % H_q), g = hq % H_kv;"),
+    "no_normalise": ("for (int i = 0; i < d; ++i) o[i] /= den;", ""),
+    "row_in_page": ("ORC_PAGE_TOKENS + (j % ORC_PAGE_TOKENS)) * (size_t)d",
+                    "ORC_PAGE_TOKENS + (j / ORC_PAGE_TOKENS)) * (size_t)d"),
+    "ignore_block_table": ("int phys = block_table[(size_t)b * max_blocks + logical];\n    if (phys < 0 || phys >= num_blocks) return -1;",
+                           "int phys = logical; (void)block_table; (void)num_blocks;"),
+    "lse_without_max": ("if (lse) lse[r] = m + log(den);", "if (lse) lse[r] = log(den);"),
+    "merge_weight": ("double w = exp(L[s] - LSE);", "double w = exp(L[s] - M);"),
+    "f16_bias": ("ldexp((double)(1024 + frac), expo - 25)", "ldexp((double)(1024 + frac), expo - 24)"),
+    "f16_subnormal": ("ldexp((double)frac, -24)", "ldexp((double)frac, -25)"),
+    "bf16_shift": ("((uint32_t)b) << 16", "((uint32_t)b) << 15"),
+    "append_row": ("int row = pos % ORC_PAGE_TOKENS;", "int row = pos / ORC_PAGE_TOKENS;"),
+    "append_head_stride": ("size_t src = ((size_t)b * H_kv + h) * (size_t)d;",
+                           "size_t src = ((size_t)h * B + b) * (size_t)d;"),
+    "tiled_no_rescale": ("ssum = ssum * exp_old + tile_sum;", "ssum = ssum + tile_sum;"),
+    "kv_bytes_no_kv_factor": ("return 2LL * (long long)dtype_size * layers * heads * d_head;",
+                              "return (long long)dtype_size * layers * heads * d_head;"),
+    "max_skips_first": ("for (int t = 0; t < n; ++t) if (s[t] > m) m = s[t];",
+                        "for (int t = 1; t < n; ++t) if (s[t] > m) m = s[t];"),
+}
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(SRC, encoding="utf-8") as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, source, tmp_path):
+    old, new = MUTANTS[name]
+    assert source.count(old) == 1, f"mutation site for {name} not unique in oracle.c"
+    src = tmp_path / "mutant.c"
+    src.write_text(source.replace(old, new), encoding="utf-8")
+    lib = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                    "-ffp-contract=off", str(src), "-o", str(lib), "-lm"], check=True)
+    caught = []
+    with oracle.using_library(str(lib)):
+        for check in ALL_CHECKS:
+            try:
+                check()
+            except AssertionError:
+                caught.append(check.__name__)
+                break
+            except oracle.OracleError:
+                caught.append(check.__name__ + " (error)")
+                break
+    assert caught, f"no pin detects the planted mistake {name!r}"
