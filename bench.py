@@ -1,0 +1,420 @@
+"""Benchmark of one paged-KV decode step (append + decode attention + merge).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mha7b]
+    python bench.py --impl reference ...     # the CPU oracle, timed on host cores
+
+Prints ONE JSON line (rank 0).  Metric: achieved HBM GB/s of the decode step
+= algorithmic bytes of one step (K/V pages of every (sequence, KV head) pair,
+q, out, and the appended K/V rows read and written) / device time of one step.
+Inputs are resident in HBM when timing starts; the KV pool (2.1 GB for the
+7B-shape workload) is far larger than the 126 MB L2, so no flush is needed
+between steps.
+
+Multi-GPU (torchrun): every rank runs the same workload on its own GPU with no
+data-path collective (the decode step of independent sequences shards by
+batch); value = bytes of all ranks / slowest rank's time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from synth import build_workload, config_spec, named_config, step_inputs, to_words  # noqa: E402
+
+METRIC = "paged decode-attention achieved HBM GB/s (% of B200 peak); us per decode step"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_mha7b_ncu.md")
+DECODE_SOURCE = os.path.join(ROOT, "kv_cache_decode_scatters_b200", "csrc", "decode.cu")
+
+
+# ------------------------------------------------------------------ helpers
+
+def attention_bytes(w, seq_lens) -> int:
+    """K/V pages read + q read + out written (algorithmic, per step)."""
+    s = 2  # fp16 / bf16 bytes
+    kv = int(seq_lens.to(torch.int64).sum().item()) * w.H_kv * 2 * w.d * s
+    return kv + 2 * w.B * w.H_q * w.d * s
+
+
+def append_bytes(w, slot) -> int:
+    rows = int((slot >= 0).sum().item()) * w.H_kv
+    return rows * w.d * 2 * 2 * 2          # K and V rows, read from k_new/v_new and written
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash() -> str:
+    with open(DECODE_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profile_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current decode kernel source for this workload."""
+    try:
+        text = open(PROFILE_SUMMARY, encoding="utf-8").read()
+    except OSError:
+        return None
+    m_src = re.search(r"decode_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_wl = re.search(r"workload:\s*(\S+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not (m_src and m_b and m_wl) or m_src.group(1) != source_hash() or m_wl.group(1) != workload:
+        return None
+    return int(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"]
+        except Exception:
+            sel = []
+        self.cmd = ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                    "-lms", "100"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist, dist.get_rank(), world, local
+    if n_gpus > 1:
+        raise SystemExit("--gpus N > 1 must be launched with torchrun (one rank per GPU)")
+    return None, 0, 1, 0
+
+
+def max_over_ranks(dist, x: float) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+# ------------------------------------------------------------ CPU (oracle)
+
+def oracle_sample(w_name, budget_s=12.0, min_seqs=1):
+    """Time the fp64 CPU oracle (append + attend) on whole sequences of the
+    workload's shape, one after another, until about budget_s seconds are spent.
+    Returns (GB/s, seconds, sequences, threads, description)."""
+    import oracle
+    spec = config_spec(w_name)
+    threads = oracle.max_threads()
+    done, spent, nbytes = 0, 0.0, 0
+    while (spent < budget_s or done < min_seqs) and done < spec["B"]:
+        n = spec["lens"][done]
+        w = build_workload("cpu_sample", 1, spec["H_q"], spec["H_kv"], spec["d"], spec["dtype"], [n],
+                           seed=4242 + done, placement="shuffle")
+        si = step_inputs(w, 0)
+        kc, vc = to_words(w.k_cache).copy(), to_words(w.v_cache).copy()
+        bt = w.block_table.numpy()
+        q, kn, vn = to_words(si["q"]), to_words(si["k_new"]), to_words(si["v_new"])
+        sl, slot = si["seq_lens"].numpy(), si["slot"].numpy()
+        dt = oracle.BF16 if w.dtype == torch.bfloat16 else oracle.F16
+        t0 = time.perf_counter()
+        oracle.append(kc, vc, bt, slot, kn, vn)
+        oracle.attend(q, kc, vc, bt, sl, w.scale, dt, nthreads=threads)
+        spent += time.perf_counter() - t0
+        nbytes += attention_bytes(w, si["seq_lens"]) + append_bytes(w, si["slot"])
+        done += 1
+    desc = (f"{done} of {spec['B']} sequences of the {w_name} shape (all {spec['H_q']} query heads, "
+            f"lengths {spec['lens'][:done]}), one append+attend each, fp64 oracle, "
+            f"{threads} OpenMP threads")
+    return nbytes / spent / 1e9, spent, done, threads, desc
+
+
+def run_reference(args):
+    dist, rank, world, local = (None, int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0)
+    if rank != 0:
+        return 0
+    vals = []
+    desc = threads = None
+    for i in range(args.warmup + args.steps):
+        gbs, spent, done, threads, desc = oracle_sample(args.workload, budget_s=args.ref_budget)
+        if i >= args.warmup:
+            vals.append((gbs, spent))
+    gbs = sum(v for v, _ in vals) / len(vals)
+    spec = config_spec(args.workload)
+    line = {
+        "metric": METRIC, "value": round(gbs, 6), "unit": "GB/s", "impl": "reference",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sum(s for _, s in vals) / len(vals), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, **{k: spec[k] for k in ("B", "H_q", "H_kv", "d")},
+                   "kv_dtype": spec["dtype"], "sample": "whole sequences, see cpu_baseline"},
+        "cpu_baseline": {"value": round(gbs, 6), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(gbs, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU path
+
+def run_ours(args):
+    import kv_cache_decode_scatters_b200 as kvd
+
+    dist, rank, world, local = dist_setup(args.gpus)
+    if world != args.gpus and dist is not None:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    w = named_config(args.workload, device="cuda", gen_device="cuda")
+    si = step_inputs(w, 0)
+    kc, vc, bt = w.k_cache, w.v_cache, w.block_table.to(dev)
+    q, k_new, v_new = si["q"], si["k_new"], si["v_new"]
+    slot, seq_lens = si["slot"].to(dev), si["seq_lens"].to(dev)
+    out = torch.empty_like(q)
+    ws = kvd.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, args.partitions, dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev_a=None, ev_b=None):
+        kvd.kvd_append(kc, vc, bt, slot, k_new, v_new, stream=stream)
+        if ev_a is not None:
+            ev_a.record(stream)
+        kvd.kvd_decode_attention(q, kc, vc, bt, seq_lens, w.scale, out=out,
+                                 num_partitions=args.partitions, workspace=ws, stream=stream)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    a_bytes = attention_bytes(w, si["seq_lens"])
+    p_bytes = append_bytes(w, si["slot"])
+    step_bytes = a_bytes + p_bytes
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all(), "non-finite output"
+    assert kvd.kvd_read_device_error() == 0, "device error flagged during warm-up"
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.__enter__()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(*evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.__exit__(None, None, None)
+    barrier(dist)
+    total_ms = t_start.elapsed_time(t_end)
+    attn_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    total_ms = max_over_ranks(dist, total_ms)
+    attn_ms = max_over_ranks(dist, attn_ms)
+    ms_step = total_ms / args.steps
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+
+    # ---- end to end through the public API with pinned host buffers
+    h_in = {n: t.cpu().pin_memory() for n, t in
+            (("q", q), ("k_new", k_new), ("v_new", v_new), ("slot", slot), ("seq_lens", seq_lens))}
+    d_in = {n: torch.empty_like(t, device=dev) for n, t in h_in.items()}
+    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+
+    def e2e_step():
+        for n in h_in:
+            d_in[n].copy_(h_in[n], non_blocking=True)
+        kvd.kvd_append(kc, vc, bt, d_in["slot"], d_in["k_new"], d_in["v_new"], stream=stream)
+        kvd.kvd_decode_attention(d_in["q"], kc, vc, bt, d_in["seq_lens"], w.scale, out=out,
+                                 num_partitions=args.partitions, workspace=ws, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    barrier(dist)
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e2e_s = max_over_ranks(dist, time.perf_counter() - t0)
+    barrier(dist)
+    e2e_val = world * step_bytes * e2e_steps / e2e_s / 1e9
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+
+    peak, peak_kind = peaks()
+    achieved = a_bytes / (attn_ms * 1e-3) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        gbs, spent, done, threads, desc = oracle_sample(args.workload, budget_s=args.cpu_budget)
+        cpu = {"value": round(gbs, 6), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": desc}
+    clocks = sampler.summary() if sampler else None
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype_name,
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
+            "seq_lens": _lens_desc(w), "page_tokens": 16, "pages_in_pool": w.num_blocks,
+            "placement": "shuffled pages", "partitions": args.partitions or kvd.kvd_auto_partitions(),
+            "bytes_per_step": step_bytes, "attention_bytes": a_bytes, "append_bytes": p_bytes,
+            "l2": "inputs larger than L2 (KV pool %.2f GB >> 126 MB); no flush" % (
+                2 * w.k_cache.numel() * 2 / 1e9),
+            "step": "kvd_append + kvd_decode_attention (decode + merge kernels)",
+        },
+        "us_per_step": round(ms_step * 1e3, 2),
+        "attention_us": round(attn_ms * 1e3, 2),
+        "roofline": {
+            "bound": "hbm",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "peak_kind": peak_kind,
+            "kernel": "kvd_decode_attention call (decode_kernel + decode_merge_kernel), CUDA events",
+            "traffic": profile_traffic(w.name),
+        },
+        "frac_of_8000_spec": round(achieved / 8000.0, 4),
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "us_per_step": round(e2e_s / e2e_steps * 1e6, 2),
+                "how": "pinned host inputs -> H2D, append, decode, D2H of out, stream sync; wall clock"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def _lens_desc(w):
+    l = w.seq_lens0
+    if bool((l == l[0]).all()):
+        return int(l[0])
+    return {"min": int(l.min()), "max": int(l.max()), "mean": round(float(l.float().mean()), 1)}
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="mha7b",
+                   choices=["tiny", "mha7b", "gqa70b", "long", "cbatch"])
+    p.add_argument("--partitions", type=int, default=0, help="0 = automatic")
+    p.add_argument("--e2e-steps", type=int, default=300)
+    p.add_argument("--cpu-budget", type=float, default=12.0,
+                   help="seconds of oracle work for the CPU baseline sample")
+    p.add_argument("--ref-budget", type=float, default=8.0,
+                   help="seconds of oracle work per reference-arm step")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    args = p.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,181 @@
+/*
+ * kvdecode.h -- C interface of libkvdecode.so: one autoregressive decode step of
+ * attention over a paged KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The method these calls implement is described on three web pages:
+ *   [KVF]  "推理速度慢怎么办？KV Cache与Flash Attention如何加速大模型推理" (ipipp.com)
+ *   [LES]  "KV缓存与Flash注意力" (FANDEX course lesson)
+ *   [BLOG] "KV Cache:推理慢的真正原因" (cybercheems.top)
+ *
+ * A decode step is: kvd_append (write the new token's K/V into its page), then
+ * kvd_decode_attention (the new query attends over every cached token).
+ * kvd_merge_lse combines partial results of a context split into partitions.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers named as device memory must be CUDA device (or managed) memory
+ *    of the current device, 16-byte aligned; the caller owns every buffer.
+ *    The library allocates no device memory.
+ *  - Page size is fixed at KVD_PAGE_TOKENS = 16 tokens ([BLOG] section
+ *    "工程优化手段 / PagedAttention": fixed blocks of 16 tokens and a block table
+ *    mapping logical to physical blocks).
+ *  - KV pool layout, row-major: k_cache, v_cache [num_blocks][H_kv][16][d];
+ *    token t of sequence b, KV head g is row (t % 16) of page
+ *    block_table[b * max_blocks_per_seq + t / 16], head g.
+ *  - block_table: int32 [B][max_blocks_per_seq]; entries past a sequence's
+ *    last page are never read.  seq_lens: int32 [B] tokens to attend,
+ *    including the one appended in the same step.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = legacy default stream).  They never synchronise the device.
+ *  - Host-side argument errors return before any launch.  Errors found on
+ *    the device (a block-table entry outside [0, num_blocks), a sequence
+ *    length outside [0, 16 * max_blocks_per_seq], a slot outside the table,
+ *    a pipeline wait that ran out) set bits of a device error word that
+ *    kvd_read_device_error returns; the offending page or row is skipped,
+ *    never read or written out of bounds.
+ *  - Supported: dtype fp16 or bf16; d in {64, 128}; H_q % H_kv == 0 with a
+ *    group size H_q / H_kv <= 16; B <= KVD_MAX_BATCH;
+ *    num_blocks * H_kv * 16 < 2^31.
+ */
+#ifndef KVDECODE_H
+#define KVDECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVD_PAGE_TOKENS 16
+#define KVD_MAX_BATCH 4096
+#define KVD_MAX_GROUP 16
+
+typedef enum {
+    KVD_OK = 0,
+    KVD_ERR_INVALID = 1,      /* bad pointer, shape, alignment or size */
+    KVD_ERR_UNSUPPORTED = 2,  /* valid arguments outside the supported set */
+    KVD_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    KVD_ERR_WORKSPACE = 4     /* workspace missing or smaller than required */
+} kvd_status;
+
+typedef enum { KVD_F16 = 0, KVD_BF16 = 1 } kvd_dtype;
+
+/* Device error word bits (kvd_read_device_error). */
+#define KVD_DEVERR_BLOCK_TABLE 0x1u   /* block_table entry outside [0, num_blocks) */
+#define KVD_DEVERR_SEQ_LEN     0x2u   /* seq_lens entry outside [0, 16 * max_blocks_per_seq] */
+#define KVD_DEVERR_SLOT        0x4u   /* append slot outside the block table */
+#define KVD_DEVERR_TIMEOUT     0x8u   /* a pipeline wait gave up */
+
+/*
+ * kvd_append -- write the new token's K and V into the paged cache.
+ * [BLOG] section "缓存的是什么" (KVCache.append writes the step's K/V at
+ * position `length`), made paged by section "PagedAttention"; [KVF] section
+ * "一、KV Cache" (append the new K/V behind the cache, then attend).
+ *
+ *   k_cache, v_cache  device, [num_blocks][H_kv][16][d], written in place
+ *   block_table       device, int32 [B][max_blocks_per_seq]
+ *   slot              device, int32 [B]: logical position of the new token of
+ *                     sequence b (its seq_len - 1); slot < 0 skips b
+ *   k_new, v_new      device, [B][H_kv][d]
+ * For each b with slot[b] >= 0 and each head h, the d storage words of
+ * k_new[b][h] are copied verbatim to row slot % 16 of page
+ * block_table[b][slot / 16], head h (same for V).  Nothing else changes.
+ * The target page must not be shared with another sequence appending in the
+ * same call.  Returns KVD_OK or an error; device-side range errors set
+ * KVD_DEVERR_SLOT / KVD_DEVERR_BLOCK_TABLE and skip that sequence.
+ */
+kvd_status kvd_append(void *k_cache, void *v_cache, const int32_t *block_table,
+                      const int32_t *slot, const void *k_new, const void *v_new,
+                      int B, int H_kv, int d, int num_blocks, int max_blocks_per_seq,
+                      kvd_dtype dtype, void *stream);
+
+/*
+ * kvd_decode_attention -- the new query of every sequence attends over all of
+ * its cached keys and values.
+ * [KVF] section "一、KV Cache" (forward_with_kv_cache: softmax(q K^T * scale) V
+ * over the whole cache including the appended token, no causal mask);
+ * [LES] section "Flash Attention — 分块技巧" and "步骤2:分块softmax" (tiles of K/V
+ * with a running (max, sum), so no score matrix is ever written to memory);
+ * [BLOG] section "工程优化手段 / GQA" (query head hq reads KV head hq / (H_q/H_kv)).
+ *
+ *   q          device, [B][H_q][d]
+ *   out        device, [B][H_q][d], same dtype as the cache; written for every
+ *              row (a sequence of length 0 gets zeros)
+ *   scale      score multiplier (usually 1/sqrt(d))
+ *   num_partitions
+ *              0: automatic (one partition per resident worker warp of the
+ *              device).  n >= 1: the concatenated page list of all (sequence,
+ *              KV head) pairs is cut into n equal contiguous partitions; a
+ *              pair that spans several partitions is finished by an LSE merge
+ *              launched by this call on the same stream.
+ *   workspace  device scratch of at least
+ *              kvd_workspace_size(B, H_q, H_kv, d, num_partitions) bytes,
+ *              256-byte aligned; contents need no initialisation.
+ *   lse_out    nullable device float [B][H_q]: natural-log sum of exp of the
+ *              scaled scores (-inf for an empty sequence)
+ * Output rounding: fp32 accumulation, one round-to-nearest to the dtype.
+ */
+kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *block_table, const int32_t *seq_lens,
+                                float scale, void *out,
+                                int B, int H_q, int H_kv, int d, int num_blocks,
+                                int max_blocks_per_seq, int num_partitions,
+                                void *workspace, size_t workspace_bytes,
+                                float *lse_out, kvd_dtype dtype, void *stream);
+
+/*
+ * kvd_merge_lse -- combine S partial attention results of each query row.
+ * Not printed on the pages as such: it is the running-state rescale of [LES]
+ * "步骤2:分块softmax" applied to whole partitions.  With M = max_s lse_s:
+ *   LSE = M + ln sum_s exp(lse_s - M),   out = sum_s exp(lse_s - LSE) o_s.
+ *
+ *   part_o             device float [B][H_q][S][d], each partial normalised
+ *   part_lse           device float [B][H_q][S]; -inf marks an empty partial
+ *                      (its part_o is ignored)
+ *   num_splits_per_seq nullable device int32 [B]: sequence b uses its first
+ *                      num_splits_per_seq[b] partials (0..S); NULL = all S
+ *   out                device [B][H_q][d] in dtype; lse_out nullable float [B][H_q]
+ * A row whose partials are all empty gets out = 0 and lse = -inf.
+ */
+kvd_status kvd_merge_lse(const float *part_o, const float *part_lse,
+                         const int32_t *num_splits_per_seq, int B, int H_q, int d, int S,
+                         void *out, float *lse_out, kvd_dtype dtype, void *stream);
+
+/*
+ * Bytes of workspace kvd_decode_attention needs for this shape.
+ * num_partitions = 0 means the automatic count of the current device (this
+ * queries the device; with no usable device it returns 0 and records the
+ * reason for kvd_last_error).
+ */
+size_t kvd_workspace_size(int B, int H_q, int H_kv, int d, int num_partitions);
+
+/*
+ * Partition count used when num_partitions = 0 on the current device, or 0
+ * if no device is usable.
+ */
+int kvd_auto_partitions(void);
+
+/*
+ * KV-cache bytes per token over all layers:
+ *   2 (K and V) x dtype_size x layers x heads x d_head
+ * ([BLOG] section "显存账"; [LES] section "KV缓存数学"; [KVF] section "一、KV Cache").
+ * Pure arithmetic, no device access.  Returns 0 for a negative argument.
+ */
+size_t kvd_kv_bytes_per_token(int layers, int heads, int d_head, int dtype_size);
+
+/*
+ * Copy the device error word of the current device into *flags (bitwise OR
+ * of KVD_DEVERR_* since the last clear) and, if clear != 0, reset it.  This
+ * call synchronises the device; it is a diagnostic, not part of a step.
+ */
+kvd_status kvd_read_device_error(unsigned int *flags, int clear);
+
+/* Text of the last error recorded by a call on this host thread ("" if none). */
+const char *kvd_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVDECODE_H */

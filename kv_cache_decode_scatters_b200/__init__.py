@@ -1,0 +1,203 @@
+"""Python binding of libkvdecode.so: one decode step over a paged KV cache.
+
+The functions here carry the C names of ``include/kvdecode.h`` and do argument
+marshalling only (tensor checks, pointers, the current CUDA stream).  Every
+step of the computation runs in the library's sm_100a kernels; there is no
+Python or CPU fallback.  If the shared library is missing, importing this
+package raises ImportError.
+
+PyTorch supplies device memory and streams.  All tensors must be CUDA,
+contiguous, on the current device.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "KVD_OK", "KVD_ERR_INVALID", "KVD_ERR_UNSUPPORTED", "KVD_ERR_CUDA", "KVD_ERR_WORKSPACE",
+    "KVD_F16", "KVD_BF16", "KVD_PAGE_TOKENS", "KvdError",
+    "kvd_append", "kvd_decode_attention", "kvd_merge_lse", "kvd_workspace_size",
+    "kvd_auto_partitions", "kvd_kv_bytes_per_token", "kvd_read_device_error",
+    "kvd_last_error", "alloc_workspace", "library_path", "lib",
+]
+
+KVD_OK, KVD_ERR_INVALID, KVD_ERR_UNSUPPORTED, KVD_ERR_CUDA, KVD_ERR_WORKSPACE = 0, 1, 2, 3, 4
+KVD_F16, KVD_BF16 = 0, 1
+KVD_PAGE_TOKENS = 16
+KVD_DEVERR_BLOCK_TABLE, KVD_DEVERR_SEQ_LEN, KVD_DEVERR_SLOT, KVD_DEVERR_TIMEOUT = 1, 2, 4, 8
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libkvdecode.so")
+
+
+def _load():
+    path = library_path()
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with `python -m kv_cache_decode_scatters_b200.build`")
+    L = ctypes.CDLL(path)
+    P, I, S, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    L.kvd_append.restype = I
+    L.kvd_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
+    L.kvd_decode_attention.restype = I
+    L.kvd_decode_attention.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, I, P, S, P, I, P]
+    L.kvd_merge_lse.restype = I
+    L.kvd_merge_lse.argtypes = [P, P, P, I, I, I, I, P, P, I, P]
+    L.kvd_workspace_size.restype = S
+    L.kvd_workspace_size.argtypes = [I, I, I, I, I]
+    L.kvd_auto_partitions.restype = I
+    L.kvd_auto_partitions.argtypes = []
+    L.kvd_kv_bytes_per_token.restype = S
+    L.kvd_kv_bytes_per_token.argtypes = [I, I, I, I]
+    L.kvd_read_device_error.restype = I
+    L.kvd_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), I]
+    L.kvd_last_error.restype = ctypes.c_char_p
+    L.kvd_last_error.argtypes = []
+    return L
+
+
+_lib = _load()
+
+
+def lib():
+    """The loaded ctypes library (raw C entry points)."""
+    return _lib
+
+
+class KvdError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where} failed with status {status}: {kvd_last_error()}")
+
+
+def kvd_last_error() -> str:
+    return _lib.kvd_last_error().decode("utf-8", "replace")
+
+
+def _check(status: int, where: str):
+    if status != KVD_OK:
+        raise KvdError(status, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return KVD_F16
+    if t.dtype == torch.bfloat16:
+        return KVD_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (fp16 or bf16)")
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def kvd_kv_bytes_per_token(layers: int, heads: int, d_head: int, dtype_size: int) -> int:
+    return int(_lib.kvd_kv_bytes_per_token(layers, heads, d_head, dtype_size))
+
+
+def kvd_auto_partitions() -> int:
+    return int(_lib.kvd_auto_partitions())
+
+
+def kvd_workspace_size(B: int, H_q: int, H_kv: int, d: int, num_partitions: int = 0) -> int:
+    n = int(_lib.kvd_workspace_size(B, H_q, H_kv, d, num_partitions))
+    if n == 0 and B > 0:
+        raise KvdError(KVD_ERR_INVALID, "kvd_workspace_size")
+    return n
+
+
+def alloc_workspace(B, H_q, H_kv, d, num_partitions=0, device=None) -> torch.Tensor:
+    """A uint8 device buffer of kvd_workspace_size bytes (torch's allocator
+    returns 256-byte aligned blocks)."""
+    n = kvd_workspace_size(B, H_q, H_kv, d, num_partitions)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def kvd_append(k_cache, v_cache, block_table, slot, k_new, v_new, stream=None):
+    """Scatter k_new/v_new [B,H_kv,d] into row slot%16 of page
+    block_table[b, slot//16] of k_cache/v_cache [NB,H_kv,16,d] (in place)."""
+    NB, H_kv, P, d = k_cache.shape
+    if P != KVD_PAGE_TOKENS:
+        raise ValueError("cache pages must hold 16 tokens")
+    B = k_new.shape[0]
+    if v_cache.shape != k_cache.shape or tuple(k_new.shape) != (B, H_kv, d) or v_new.shape != k_new.shape:
+        raise ValueError("shape mismatch between caches and new K/V")
+    dt = k_cache.dtype
+    _check(_lib.kvd_append(_dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+                           _dev(block_table, "block_table", torch.int32),
+                           _dev(slot, "slot", torch.int32), _dev(k_new, "k_new", dt),
+                           _dev(v_new, "v_new", dt), B, H_kv, d, NB, block_table.shape[1],
+                           _dtype_code(k_cache), _stream(stream)),
+           "kvd_append")
+
+
+def kvd_decode_attention(q, k_cache, v_cache, block_table, seq_lens, scale=None, out=None,
+                         num_partitions=0, workspace=None, lse_out=None, stream=None):
+    """out[b, hq] = softmax(scale * q[b, hq] K_b^T) V_b over the seq_lens[b]
+    cached tokens of sequence b (KV head hq // (H_q // H_kv)).  Returns out."""
+    B, H_q, d = q.shape
+    NB, H_kv, P, d2 = k_cache.shape
+    if P != KVD_PAGE_TOKENS or d2 != d:
+        raise ValueError("q / cache shape mismatch")
+    dt = k_cache.dtype
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(B, H_q, H_kv, d, num_partitions, q.device)
+    lse_ptr = None if lse_out is None else _dev(lse_out, "lse_out", torch.float32)
+    _check(_lib.kvd_decode_attention(
+        _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
+        float(scale), _dev(out, "out", dt), B, H_q, H_kv, d, NB, block_table.shape[1],
+        int(num_partitions), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        lse_ptr, _dtype_code(k_cache), _stream(stream)),
+        "kvd_decode_attention")
+    return out
+
+
+def kvd_merge_lse(part_o, part_lse, num_splits_per_seq=None, out=None, lse_out=None,
+                  dtype=torch.float16, stream=None):
+    """Merge partials part_o [B,H_q,S,d] (fp32), part_lse [B,H_q,S] into out [B,H_q,d]."""
+    B, H_q, S, d = part_o.shape
+    if out is None:
+        out = torch.empty((B, H_q, d), dtype=dtype, device=part_o.device)
+    cnt = None if num_splits_per_seq is None else _dev(num_splits_per_seq, "num_splits_per_seq", torch.int32)
+    lse_ptr = None if lse_out is None else _dev(lse_out, "lse_out", torch.float32)
+    _check(_lib.kvd_merge_lse(_dev(part_o, "part_o", torch.float32),
+                              _dev(part_lse, "part_lse", torch.float32), cnt, B, H_q, d, S,
+                              _dev(out, "out"), lse_ptr, _dtype_code(out), _stream(stream)),
+           "kvd_merge_lse")
+    return out
+
+
+def kvd_read_device_error(clear: bool = True) -> int:
+    """Device error bits (KVD_DEVERR_*) since the last clear; synchronises."""
+    flags = ctypes.c_uint(0)
+    _check(_lib.kvd_read_device_error(ctypes.byref(flags), 1 if clear else 0),
+           "kvd_read_device_error")
+    return int(flags.value)

@@ -1,0 +1,327 @@
+// api.cu -- the C interface of libkvdecode.so (declared in include/kvdecode.h):
+// argument validation, workspace carving, TMA descriptor encoding, launches,
+// error reporting.  Every call is asynchronous on the caller's stream except
+// kvd_read_device_error.
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/kvdecode.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+// Device error word of each device that loads the library (bits KVD_DEVERR_*).
+__device__ unsigned g_device_error = 0u;
+
+thread_local std::string g_last_error;
+
+kvd_status fail(kvd_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+kvd_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(KVD_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+// Average pages per partition below which the automatic split stops cutting
+// (keeps tiny problems from producing more partials than pages).
+constexpr int kAutoMinPages = 8;
+
+std::mutex g_mu;
+int g_sms[kMaxDevices];
+unsigned *g_err_ptr[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+kvd_status current_device(int *dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (*dev < 0 || *dev >= kMaxDevices) return fail(KVD_ERR_UNSUPPORTED, "device ordinal %d", *dev);
+  return KVD_OK;
+}
+
+kvd_status sm_count(int dev, int *sms) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sms[dev]) {
+    int v = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+    g_sms[dev] = v;
+  }
+  *sms = g_sms[dev];
+  return KVD_OK;
+}
+
+// Device address of this device's error word (looked up once per device,
+// with that device current).
+kvd_status error_word(int dev, unsigned **p) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void *a = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&a, g_device_error);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+    g_err_ptr[dev] = static_cast<unsigned *>(a);
+  }
+  *p = g_err_ptr[dev];
+  return KVD_OK;
+}
+
+kvd_status encoder(PFN_cuTensorMapEncodeTiled_v12000 *fn) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                                     cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+      return fail(KVD_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  *fn = g_encode;
+  return KVD_OK;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t cum, lse, o, total;
+};
+
+WsLayout ws_layout(int B, int G, int d, long long slots) {
+  WsLayout L;
+  L.cum = 0;
+  L.lse = round_up(static_cast<size_t>(B + 1) * 4, 256);
+  L.o = L.lse + round_up(static_cast<size_t>(slots) * G * 4, 256);
+  L.total = L.o + static_cast<size_t>(slots) * G * d * 4;
+  return L;
+}
+
+kvd_status resolve_parts(int d, int num_partitions, int *N) {
+  if (num_partitions < 0) return fail(KVD_ERR_INVALID, "num_partitions < 0");
+  if (num_partitions > 0) {
+    *N = num_partitions;
+    return KVD_OK;
+  }
+  int dev, sms;
+  kvd_status st = current_device(&dev);
+  if (st) return st;
+  st = sm_count(dev, &sms);
+  if (st) return st;
+  *N = kvd::decode_auto_parts(d, sms);
+  return KVD_OK;
+}
+
+kvd_status check_heads(int B, int H_q, int H_kv, int d) {
+  if (B < 0) return fail(KVD_ERR_INVALID, "B = %d < 0", B);
+  if (B > KVD_MAX_BATCH) return fail(KVD_ERR_UNSUPPORTED, "B = %d > %d", B, KVD_MAX_BATCH);
+  if (H_q <= 0 || H_kv <= 0) return fail(KVD_ERR_INVALID, "head counts must be positive");
+  if (H_q % H_kv) return fail(KVD_ERR_UNSUPPORTED, "H_q = %d not a multiple of H_kv = %d", H_q, H_kv);
+  if (H_q / H_kv > KVD_MAX_GROUP)
+    return fail(KVD_ERR_UNSUPPORTED, "group size %d > %d", H_q / H_kv, KVD_MAX_GROUP);
+  if (d != 64 && d != 128) return fail(KVD_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", d);
+  return KVD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kvd_last_error(void) { return g_last_error.c_str(); }
+
+size_t kvd_kv_bytes_per_token(int layers, int heads, int d_head, int dtype_size) {
+  if (layers < 0 || heads < 0 || d_head < 0 || dtype_size < 0) return 0;
+  return 2ull * static_cast<size_t>(dtype_size) * layers * heads * d_head;
+}
+
+int kvd_auto_partitions(void) {
+  int N = 0;
+  if (resolve_parts(128, 0, &N) != KVD_OK) return 0;
+  return N;
+}
+
+size_t kvd_workspace_size(int B, int H_q, int H_kv, int d, int num_partitions) {
+  if (check_heads(B, H_q, H_kv, d) != KVD_OK) return 0;
+  int N = 0;
+  if (resolve_parts(d, num_partitions, &N) != KVD_OK) return 0;
+  const long long slots = static_cast<long long>(N) + static_cast<long long>(B) * H_kv;
+  return ws_layout(B, H_q / H_kv, d, slots).total;
+}
+
+kvd_status kvd_read_device_error(unsigned int *flags, int clear) {
+  if (!flags) return fail(KVD_ERR_INVALID, "flags is NULL");
+  int dev;
+  unsigned *p;
+  kvd_status st = current_device(&dev);
+  if (st) return st;
+  st = error_word(dev, &p);
+  if (st) return st;
+  cudaError_t e = cudaMemcpy(flags, p, sizeof(unsigned), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (clear) {
+    e = cudaMemset(p, 0, sizeof(unsigned));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  }
+  return KVD_OK;
+}
+
+kvd_status kvd_append(void *k_cache, void *v_cache, const int32_t *block_table,
+                      const int32_t *slot, const void *k_new, const void *v_new, int B, int H_kv,
+                      int d, int num_blocks, int max_blocks_per_seq, kvd_dtype dtype,
+                      void *stream) {
+  if (B < 0) return fail(KVD_ERR_INVALID, "B = %d < 0", B);
+  if (H_kv <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+    return fail(KVD_ERR_INVALID, "H_kv, num_blocks and max_blocks_per_seq must be positive");
+  if (d <= 0 || d % 8 || d > 128) return fail(KVD_ERR_UNSUPPORTED, "head dim %d (need a multiple of 8, <= 128)", d);
+  if (dtype != KVD_F16 && dtype != KVD_BF16) return fail(KVD_ERR_INVALID, "unknown dtype %d", (int)dtype);
+  if (B == 0) return KVD_OK;
+  if (!k_cache || !v_cache || !block_table || !slot || !k_new || !v_new)
+    return fail(KVD_ERR_INVALID, "a required pointer is NULL");
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(k_new, 16) || !aligned(v_new, 16))
+    return fail(KVD_ERR_INVALID, "K/V buffers must be 16-byte aligned");
+  if (static_cast<long long>(max_blocks_per_seq) * KVD_PAGE_TOKENS > 0x7fffffffLL)
+    return fail(KVD_ERR_UNSUPPORTED, "max_blocks_per_seq too large");
+  int dev;
+  unsigned *err;
+  kvd_status st = current_device(&dev);
+  if (st) return st;
+  st = error_word(dev, &err);
+  if (st) return st;
+  kvd::AppendArgs a{k_cache, v_cache, block_table, slot, k_new, v_new, err,
+                    B, H_kv, d, num_blocks, max_blocks_per_seq};
+  cudaError_t e = kvd::launch_append(a, dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16,
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  return KVD_OK;
+}
+
+kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *block_table, const int32_t *seq_lens, float scale,
+                                void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                                int max_blocks_per_seq, int num_partitions, void *workspace,
+                                size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+                                void *stream) {
+  kvd_status st = check_heads(B, H_q, H_kv, d);
+  if (st) return st;
+  if (num_blocks <= 0 || max_blocks_per_seq <= 0)
+    return fail(KVD_ERR_INVALID, "num_blocks and max_blocks_per_seq must be positive");
+  if (dtype != KVD_F16 && dtype != KVD_BF16) return fail(KVD_ERR_INVALID, "unknown dtype %d", (int)dtype);
+  if (static_cast<long long>(num_blocks) * H_kv * KVD_PAGE_TOKENS >= 0x80000000LL)
+    return fail(KVD_ERR_UNSUPPORTED, "num_blocks * H_kv * 16 must be < 2^31");
+  if (static_cast<long long>(max_blocks_per_seq) * KVD_PAGE_TOKENS > 0x7fffffffLL)
+    return fail(KVD_ERR_UNSUPPORTED, "max_blocks_per_seq too large");
+  if (!(scale == scale)) return fail(KVD_ERR_INVALID, "scale is NaN");
+  if (num_partitions < 0) return fail(KVD_ERR_INVALID, "num_partitions < 0");
+  if (B == 0) return KVD_OK;
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out)
+    return fail(KVD_ERR_INVALID, "a required pointer is NULL");
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
+    return fail(KVD_ERR_INVALID, "q, caches and out must be 16-byte aligned");
+  if (lse_out && !aligned(lse_out, 4)) return fail(KVD_ERR_INVALID, "lse_out misaligned");
+
+  int N = 0;
+  st = resolve_parts(d, num_partitions, &N);
+  if (st) return st;
+  const int G = H_q / H_kv;
+  const long long slots = static_cast<long long>(N) + static_cast<long long>(B) * H_kv;
+  const WsLayout L = ws_layout(B, G, d, slots);
+  if (!workspace) return fail(KVD_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", L.total);
+  if (!aligned(workspace, 256)) return fail(KVD_ERR_INVALID, "workspace must be 256-byte aligned");
+  if (workspace_bytes < L.total)
+    return fail(KVD_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, L.total);
+
+  int dev;
+  unsigned *err;
+  st = current_device(&dev);
+  if (st) return st;
+  st = error_word(dev, &err);
+  if (st) return st;
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  st = encoder(&encode);
+  if (st) return st;
+
+  // K and V pools as 3-D tensors {64 elements, d/64 units, num_blocks*H_kv*16
+  // rows}; one box = one page of one head (16 rows x d), 128-byte swizzled.
+  CUtensorMap tm[2];
+  const void *pools[2] = {k_cache, v_cache};
+  for (int i = 0; i < 2; ++i) {
+    cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(d / 64),
+                          static_cast<cuuint64_t>(num_blocks) * H_kv * KVD_PAGE_TOKENS};
+    cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(d) * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(d / 64), KVD_PAGE_TOKENS};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = encode(&tm[i],
+                        dtype == KVD_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        3, const_cast<void *>(pools[i]), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KVD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  }
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  kvd::DecodeArgs a;
+  a.q = q;
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.out = out;
+  a.lse_out = lse_out;
+  a.part_o = reinterpret_cast<float *>(ws + L.o);
+  a.part_lse = reinterpret_cast<float *>(ws + L.lse);
+  a.ws_cum = reinterpret_cast<int32_t *>(ws + L.cum);
+  a.err = err;
+  a.scale_log2 = scale * kvd::kLog2e;
+  a.B = B;
+  a.H_q = H_q;
+  a.H_kv = H_kv;
+  a.G = G;
+  a.num_blocks = num_blocks;
+  a.maxb = max_blocks_per_seq;
+  a.nparts = N;
+  a.min_pages = num_partitions > 0 ? 1 : kAutoMinPages;
+  a.evict_first = 0;
+
+  const kvd::DType dt = dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int W = kvd::decode_warps_per_cta(d);
+  const int grid = (N + W - 1) / W;
+  cudaError_t e = kvd::launch_decode(a, d, dt, tm[0], tm[1], s, grid);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  e = kvd::launch_decode_merge(a, d, dt, s);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return KVD_OK;
+}
+
+kvd_status kvd_merge_lse(const float *part_o, const float *part_lse,
+                         const int32_t *num_splits_per_seq, int B, int H_q, int d, int S,
+                         void *out, float *lse_out, kvd_dtype dtype, void *stream) {
+  if (B < 0 || H_q <= 0 || S <= 0) return fail(KVD_ERR_INVALID, "need B >= 0, H_q > 0, S > 0");
+  if (d != 64 && d != 128) return fail(KVD_ERR_UNSUPPORTED, "head dim %d not in {64, 128}", d);
+  if (dtype != KVD_F16 && dtype != KVD_BF16) return fail(KVD_ERR_INVALID, "unknown dtype %d", (int)dtype);
+  if (static_cast<long long>(B) * H_q > 0x7fffffffLL) return fail(KVD_ERR_UNSUPPORTED, "B * H_q too large");
+  if (B == 0) return KVD_OK;
+  if (!part_o || !part_lse || !out) return fail(KVD_ERR_INVALID, "a required pointer is NULL");
+  if (!aligned(part_o, 16) || !aligned(part_lse, 4) || !aligned(out, 2))
+    return fail(KVD_ERR_INVALID, "misaligned buffer");
+  kvd::GenericMergeArgs a{part_o, part_lse, num_splits_per_seq, out, lse_out, B, H_q, d, S};
+  cudaError_t e = kvd::launch_generic_merge(a, dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16,
+                                            static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return KVD_OK;
+}
+
+}  // extern "C"

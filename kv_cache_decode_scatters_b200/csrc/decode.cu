@@ -1,0 +1,660 @@
+// decode.cu -- paged decode attention for sm_100a.
+//
+// What it computes ("推理速度慢怎么办？KV Cache与Flash Attention如何加速大模型推理",
+// section 一、KV Cache; "KV缓存与Flash注意力", sections "Flash Attention — 分块技巧"
+// and "步骤2:分块softmax"; "KV Cache:推理慢的真正原因", sections PagedAttention and
+// GQA): for every sequence b and query head hq, out = softmax(scale * q K^T) V
+// over the sequence's cached tokens, read through the block table, with query
+// head hq using KV head hq / G.  Scores never leave registers: each 16-token
+// page updates a running (max, sum, output) state.
+//
+// How it is laid out on the B200:
+//  * Work split (stream-K).  The pages of all (sequence, KV head) pairs,
+//    concatenated, form one list of P pages; it is cut into N equal
+//    contiguous partitions, one per worker warp (N = resident warps of the
+//    GPU).  Every worker streams the same number of pages whatever the
+//    sequence lengths are.  A pair that lies inside one partition is written
+//    straight to `out`; a pair cut by partition edges leaves one normalised
+//    partial (o, lse) per piece, at slot (worker + pair), and the merge
+//    kernel combines them.
+//  * Each worker warp owns an S-stage ring in shared memory.  Lane 0 issues
+//    two TMA tile loads per page (K and V, 16 x d each, 128-byte swizzle)
+//    that complete on the stage's mbarrier; the whole warp waits, computes,
+//    and hands the stage back to the next page.  No other warp is involved,
+//    so there is no block-level synchronisation in the main loop.
+//  * Every KV byte is read once per GQA group: the G query rows of a KV head
+//    ride along as the N dimension of the tensor-core tile.  Per page,
+//    S^T[16 tokens x 8 rows] = K[16 x d] . Q^T uses mma.m16n8k16 with the K
+//    page as the A operand (ldmatrix from the swizzled stage); the
+//    probabilities are transposed in registers (movmatrix) into the B
+//    operand of O^T[d x 8] += V^T[d x 16] . P^T[16 x 8] (ldmatrix.trans).
+//    G <= 8 uses one n-tile, G <= 16 two.
+//  * Softmax in base 2: scores are scaled by scale * log2(e) in fp32 and
+//    exponentiated with ex2.approx.  Probabilities are rounded once to the
+//    storage dtype for the PV product and the running sum uses the same
+//    rounded values, so the output is an exact weighted mean of V up to fp32
+//    accumulation.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kvd {
+
+namespace {
+
+template <int D, int W, int S>
+struct Geo {
+  static constexpr int kPageBytes = kPage * D * 2;      // one K (or V) page of one head
+  static constexpr int kStageBytes = 2 * kPageBytes;    // K page then V page
+  static constexpr int kThreads = 32 * W;
+  static constexpr int kSteps = D / 16;                 // k-steps of S, m-tiles of O
+  static size_t smem(int B) {
+    return 1024 + (size_t)W * S * kStageBytes + (size_t)W * S * 16 + (size_t)(B + 1) * 4;
+  }
+};
+
+// Byte offset of element column `col` (a multiple of 8) of token row t inside
+// a page stored by a 128B-swizzled TMA box of 64-element units.
+template <int D>
+__device__ __forceinline__ uint32_t swz(int t, int col) {
+  const int u = t * (D / 64) + (col >> 6);
+  const int chunk = (col & 63) >> 3;
+  return static_cast<uint32_t>(u * 128 + ((chunk ^ (u & 7)) << 4));
+}
+
+__device__ __forceinline__ int clamp_len(int n, int cap) { return n < 0 ? 0 : (n > cap ? cap : n); }
+
+template <typename T>
+struct Stor;
+template <>
+struct Stor<__half> {
+  static __device__ __forceinline__ void zero_row(__half *p, int d) {
+    for (int i = 0; i < d; i += 8) *reinterpret_cast<uint4 *>(p + i) = make_uint4(0, 0, 0, 0);
+  }
+};
+template <>
+struct Stor<__nv_bfloat16> {
+  static __device__ __forceinline__ void zero_row(__nv_bfloat16 *p, int d) {
+    for (int i = 0; i < d; i += 8) *reinterpret_cast<uint4 *>(p + i) = make_uint4(0, 0, 0, 0);
+  }
+};
+
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  return v;
+}
+
+}  // namespace
+
+template <int D, int NT, typename T, int W, int S>
+__global__ void __launch_bounds__(32 * W, 1)
+    decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV) {
+  using Gm = Geo<D, W, S>;
+  using M = Mma<T>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int warp_tot[32];
+
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *stages = smem;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)W * S * Gm::kStageBytes);
+  int2 *meta = reinterpret_cast<int2 *>(bars + W * S);
+  int *cum = reinterpret_cast<int *>(meta + W * S);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cap = a.maxb * kPage;
+
+  grid_dependency_wait();
+  if (tid == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+  }
+
+  // ---- 1. pages per sequence, exclusive prefix sum into cum[0..B]
+  {
+    const int per = (a.B + Gm::kThreads - 1) / Gm::kThreads;
+    const int b0 = tid * per;
+    const int b1 = min(a.B, b0 + per);
+    int local = 0;
+    for (int b = b0; b < b1; ++b) {
+      const int raw = __ldg(a.seq_lens + b);
+      if (raw < 0 || raw > cap) flag_error(a.err, kErrSeqLen);
+      local += (clamp_len(raw, cap) + kPage - 1) / kPage;
+    }
+    const int incl = warp_incl_scan(local, lane);
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int v = lane < W ? warp_tot[lane] : 0;
+      v = warp_incl_scan(v, lane);
+      if (lane < W) warp_tot[lane] = v;
+    }
+    __syncthreads();
+    int run = (warp ? warp_tot[warp - 1] : 0) + incl - local;
+    for (int b = b0; b < b1; ++b) {
+      cum[b] = run;
+      run += (clamp_len(__ldg(a.seq_lens + b), cap) + kPage - 1) / kPage;
+    }
+    if (tid == 0) cum[a.B] = warp_tot[W - 1];
+    __syncthreads();
+  }
+  const long long P = static_cast<long long>(cum[a.B]) * a.H_kv;
+  const int N = effective_parts(P, a.nparts, a.min_pages);
+  if (blockIdx.x == 0)
+    for (int i = tid; i <= a.B; i += Gm::kThreads) a.ws_cum[i] = cum[i];
+
+  // ---- 2. empty sequences: zero output rows (their pairs own no pages)
+  {
+    const long long rows = static_cast<long long>(a.B) * a.H_q;
+    for (long long r = static_cast<long long>(blockIdx.x) * Gm::kThreads + tid; r < rows;
+         r += static_cast<long long>(gridDim.x) * Gm::kThreads) {
+      const int b = static_cast<int>(r / a.H_q);
+      if (cum[b + 1] == cum[b]) {
+        Stor<T>::zero_row(reinterpret_cast<T *>(a.out) + r * D, D);
+        if (a.lse_out) a.lse_out[r] = -INFINITY;
+      }
+    }
+  }
+
+  // ---- 3. this warp's partition of the page list
+  const int w = blockIdx.x * W + warp;
+  if (w >= N) return;
+  const long long p0 = part_begin(w, P, N), p1 = part_begin(w + 1, P, N);
+  if (p0 >= p1) return;
+
+  const uint32_t stage0 = smem_u32(stages + (size_t)warp * S * Gm::kStageBytes);
+  const uint32_t bar0 = smem_u32(bars + warp * S);
+  int2 *meta_w = meta + warp * S;
+  const uint64_t policy = a.evict_first ? l2_policy_evict_first() : l2_policy_evict_normal();
+
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < S; ++s) mbar_init(bar0 + 8 * s, 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+
+  // Fetch-side page descriptors, one fetch position per lane, in windows of
+  // 32 positions.  `nx*` is the next window, computed one window early so its
+  // block-table loads are long done when it is promoted.
+  const int H = a.H_kv;
+  auto describe = [&](long long wb, int &pb, int &h, int &seg, int &ntok) {
+    pb = -1;
+    h = 0;
+    seg = -1;
+    ntok = 0;
+    const long long pos = wb + lane;
+    if (pos < p1) {
+      int lo = 0, hi = a.B;  // largest b with cum[b] * H <= pos
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (static_cast<long long>(cum[mid]) * H <= pos) lo = mid; else hi = mid;
+      }
+      const int b = lo;
+      const int np = cum[b + 1] - cum[b];
+      const long long off = pos - static_cast<long long>(cum[b]) * H;
+      h = static_cast<int>(off / np);
+      const int i = static_cast<int>(off - static_cast<long long>(h) * np);
+      pb = __ldg(a.block_table + static_cast<size_t>(b) * a.maxb + i);
+      ntok = min(kPage, clamp_len(__ldg(a.seq_lens + b), cap) - i * kPage);
+      seg = b * H + h;
+    }
+  };
+  auto promote = [&](int pb, int h, int seg) -> int {
+    if (seg < 0) return -1;
+    if (pb < 0 || pb >= a.num_blocks) {
+      flag_error(a.err, kErrBlockTable);
+      return -1;
+    }
+    return (pb * H + h) * kPage;  // TMA row coordinate of this page's 16 rows
+  };
+
+  long long wb = p0;
+  int cur_row, cur_seg, cur_ntok;
+  int nx_pb, nx_h, nx_seg, nx_ntok;
+  {
+    int pb, h;
+    describe(wb, pb, h, cur_seg, cur_ntok);
+    cur_row = promote(pb, h, cur_seg);
+    describe(wb + 32, nx_pb, nx_h, nx_seg, nx_ntok);
+  }
+
+  long long f = p0;  // next page to fetch
+  int fst = 0;       // its stage
+  auto issue = [&]() {
+    int j = static_cast<int>(f - wb);
+    if (j >= 32) {
+      cur_row = promote(nx_pb, nx_h, nx_seg);
+      cur_seg = nx_seg;
+      cur_ntok = nx_ntok;
+      wb += 32;
+      describe(wb + 32, nx_pb, nx_h, nx_seg, nx_ntok);
+      j -= 32;
+    }
+    const int row = __shfl_sync(0xffffffffu, cur_row, j);
+    const int seg = __shfl_sync(0xffffffffu, cur_seg, j);
+    const int ntok = __shfl_sync(0xffffffffu, cur_ntok, j);
+    if (lane == 0) {
+      meta_w[fst] = make_int2(seg, row >= 0 ? ntok : 0);
+      const uint32_t bar = bar0 + 8 * fst;
+      if (row >= 0) {
+        const uint32_t dst = stage0 + fst * Gm::kStageBytes;
+        mbar_arrive_expect_tx(bar, Gm::kStageBytes);
+        tma_load_3d(dst, &tmK, 0, 0, row, bar, policy);
+        tma_load_3d(dst + Gm::kPageBytes, &tmV, 0, 0, row, bar, policy);
+      } else {
+        mbar_arrive(bar);
+      }
+    }
+    ++f;
+    if (++fst == S) fst = 0;
+  };
+
+#pragma unroll 1
+  for (int s = 0; s < S; ++s)
+    if (f < p1) issue();
+
+  // ---- per-lane fragment geometry
+  const int g8 = lane >> 2, tig = lane & 3;
+  const int tK = (lane & 7) | (((lane >> 3) & 1) << 3);
+  const int cK = ((lane >> 4) & 1) << 3;
+  const int tV = (lane & 7) | (((lane >> 4) & 1) << 3);
+  const int cV = ((lane >> 3) & 1) << 3;
+
+  // ---- running state of the current (sequence, KV head) pair
+  uint32_t qf[NT][Gm::kSteps][2];
+  float acc[NT][Gm::kSteps][4];
+  float m_run[NT][2], l_run[NT][2];
+  int cur = -1;  // pair being accumulated
+
+  auto begin_pair = [&](int seg) {
+    const int b = seg / H, h = seg - (seg / H) * H;
+    const uint32_t *qw = reinterpret_cast<const uint32_t *>(a.q) +
+                         (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G) * (D / 2);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int r = nt * 8 + g8;
+#pragma unroll
+      for (int ks = 0; ks < Gm::kSteps; ++ks) {
+        if (r < a.G) {
+          qf[nt][ks][0] = __ldg(qw + r * (D / 2) + ks * 8 + tig);
+          qf[nt][ks][1] = __ldg(qw + r * (D / 2) + ks * 8 + 4 + tig);
+        } else {
+          qf[nt][ks][0] = 0u;
+          qf[nt][ks][1] = 0u;
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < Gm::kSteps; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
+      m_run[nt][0] = m_run[nt][1] = -INFINITY;
+      l_run[nt][0] = l_run[nt][1] = 0.f;
+    }
+  };
+
+  auto finish_pair = [&](int seg) {
+    const int b = seg / H, h = seg - (seg / H) * H;
+    const int np = cum[b + 1] - cum[b];
+    const long long s0 = static_cast<long long>(cum[b]) * H + static_cast<long long>(h) * np;
+    const bool whole = s0 >= p0 && s0 + np <= p1;
+    const size_t row0 = static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        float l = l_run[nt][i];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        const int r = nt * 8 + 2 * tig + i;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float lse = l > 0.f ? (m_run[nt][i] + fast_log2(l)) * kLn2 : -INFINITY;
+        if (r < a.G) {
+          if (whole) {
+            T *o = reinterpret_cast<T *>(a.out) + (row0 + r) * D;
+#pragma unroll
+            for (int mt = 0; mt < Gm::kSteps; ++mt) {
+              o[mt * 16 + g8] = M::from_float(acc[nt][mt][i] * inv);
+              o[mt * 16 + 8 + g8] = M::from_float(acc[nt][mt][2 + i] * inv);
+            }
+            if (a.lse_out && g8 == 0) a.lse_out[row0 + r] = lse;
+          } else {
+            const size_t slot = static_cast<size_t>(w) + seg;
+            float *o = a.part_o + (slot * a.G + r) * D;
+#pragma unroll
+            for (int mt = 0; mt < Gm::kSteps; ++mt) {
+              o[mt * 16 + g8] = acc[nt][mt][i] * inv;
+              o[mt * 16 + 8 + g8] = acc[nt][mt][2 + i] * inv;
+            }
+            if (g8 == 0) a.part_lse[slot * a.G + r] = lse;
+          }
+        }
+      }
+    }
+  };
+
+  // ---- main loop over this partition's pages
+  const long long nmy = p1 - p0;
+  int cst = 0;
+  uint32_t cph = 0;
+  bool failed = false;
+  long long c = 0;
+#pragma unroll 1
+  for (; c < nmy; ++c) {
+    const uint32_t bar = bar0 + 8 * cst;
+    const bool ok = mbar_wait_bounded(bar, cph);
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) flag_error(a.err, kErrTimeout);
+      failed = true;
+      break;
+    }
+    const int2 md = meta_w[cst];
+    if (md.x != cur) {
+      if (cur >= 0) finish_pair(cur);
+      cur = md.x;
+      begin_pair(cur);
+    }
+    const int ntok = md.y;
+    if (ntok > 0) {
+      uint8_t *kp = stages + ((size_t)warp * S + cst) * Gm::kStageBytes;
+      uint8_t *vp = kp + Gm::kPageBytes;
+      if (ntok < kPage) {
+        // rows past the sequence end may hold anything (even NaN): clear V's
+        // so the zero weights of masked tokens cannot turn into NaN
+        uint4 *z = reinterpret_cast<uint4 *>(vp + ntok * D * 2);
+        const int n16 = (kPage - ntok) * D * 2 / 16;
+        for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      const uint32_t kb = smem_u32(kp), vb = smem_u32(vp);
+
+      // S^T = K Q^T, two independent accumulator chains over d
+      float s[NT][4], s2[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < Gm::kSteps; ++ks) {
+        uint32_t fa[4];
+        ldmatrix_x4(fa, kb + swz<D>(tK, ks * 16 + cK));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          if (ks & 1) M::run(s2[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
+          else M::run(s[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
+        }
+      }
+
+      // online softmax update (base 2), probabilities rounded to T
+      const bool v0 = g8 < ntok, v1 = g8 + 8 < ntok;
+      uint32_t pb0[NT], pb1[NT];
+      float alpha[NT][2];
+      bool rescale = false;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float x0 = v0 ? (s[nt][0] + s2[nt][0]) * a.scale_log2 : -INFINITY;
+        const float x1 = v0 ? (s[nt][1] + s2[nt][1]) * a.scale_log2 : -INFINITY;
+        const float x2 = v1 ? (s[nt][2] + s2[nt][2]) * a.scale_log2 : -INFINITY;
+        const float x3 = v1 ? (s[nt][3] + s2[nt][3]) * a.scale_log2 : -INFINITY;
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+        alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
+        alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
+        rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
+        m_run[nt][0] = mn0;
+        m_run[nt][1] = mn1;
+        const uint32_t lo = M::pack(fast_exp2(x0 - mn0), fast_exp2(x1 - mn1));
+        const uint32_t hi = M::pack(fast_exp2(x2 - mn0), fast_exp2(x3 - mn1));
+        const float2 fl = M::unpack(lo), fh = M::unpack(hi);
+        l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (fl.x + fh.x);
+        l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (fl.y + fh.y);
+        pb0[nt] = movmatrix_trans(lo);
+        pb1[nt] = movmatrix_trans(hi);
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int mt = 0; mt < Gm::kSteps; ++mt) {
+            acc[nt][mt][0] *= alpha[nt][0];
+            acc[nt][mt][1] *= alpha[nt][1];
+            acc[nt][mt][2] *= alpha[nt][0];
+            acc[nt][mt][3] *= alpha[nt][1];
+          }
+      }
+
+      // O^T += V^T P^T
+#pragma unroll
+      for (int mt = 0; mt < Gm::kSteps; ++mt) {
+        uint32_t fa[4];
+        ldmatrix_x4_trans(fa, vb + swz<D>(tV, mt * 16 + cV));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) M::run(acc[nt][mt], fa, pb0[nt], pb1[nt]);
+      }
+    }
+    __syncwarp();
+    if (f < p1) issue();
+    if (++cst == S) {
+      cst = 0;
+      cph ^= 1u;
+    }
+  }
+
+  if (failed) {
+    // let every copy still in flight land before the CTA's shared memory goes away
+    for (; c < f - p0; ++c) {
+      mbar_wait_bounded(bar0 + 8 * cst, cph);
+      if (++cst == S) {
+        cst = 0;
+        cph ^= 1u;
+      }
+    }
+    return;
+  }
+  if (cur >= 0) finish_pair(cur);
+}
+
+// ------------------------------------------------------------------ merge
+
+// One CTA (256 threads) merges `count` partial results of one output row:
+// partial k has log-sum-exp lse[k * lse_stride] and normalised output
+// o[k * o_stride .. + D).  LSE = M + ln sum_k exp(lse_k - M);
+// out = sum_k exp(lse_k - LSE) o_k, one rounding to T.
+template <int D, typename T>
+__device__ __forceinline__ void merge_row(const float *lse, long long lse_stride, const float *o,
+                                          long long o_stride, int count, T *out, float *lse_out) {
+  constexpr int kV = D / 32;
+  __shared__ float red[8];
+  __shared__ __align__(16) float part[8][D];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  float mx = -INFINITY;
+  for (int k = tid; k < count; k += 256) mx = fmaxf(mx, lse[k * lse_stride]);
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  mx = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) mx = fmaxf(mx, red[i]);
+  __syncthreads();
+  if (mx == -INFINITY) {
+    for (int t = tid; t < D; t += 256) out[t] = Mma<T>::from_float(0.f);
+    if (tid == 0 && lse_out) *lse_out = -INFINITY;
+    return;
+  }
+  const float mx2 = mx * kLog2e;
+  float sum = 0.f;
+  for (int k = tid; k < count; k += 256) sum += fast_exp2(lse[k * lse_stride] * kLog2e - mx2);
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, s);
+  if (lane == 0) red[warp] = sum;
+  __syncthreads();
+  sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sum += red[i];
+  const float lse2 = mx2 + fast_log2(sum);
+
+  float accv[kV];
+#pragma unroll
+  for (int e = 0; e < kV; ++e) accv[e] = 0.f;
+#pragma unroll 4
+  for (int k = warp; k < count; k += 8) {
+    const float wk = fast_exp2(lse[k * lse_stride] * kLog2e - lse2);
+    const float *src = o + k * o_stride + lane * kV;
+    if (wk > 0.f) {
+      if constexpr (kV == 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(src);
+        accv[0] += wk * v.x;
+        accv[1] += wk * v.y;
+        accv[2] += wk * v.z;
+        accv[3] += wk * v.w;
+      } else {
+        const float2 v = *reinterpret_cast<const float2 *>(src);
+        accv[0] += wk * v.x;
+        accv[1] += wk * v.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < kV; ++e) part[warp][lane * kV + e] = accv[e];
+  __syncthreads();
+  for (int t = tid; t < D; t += 256) {
+    float v = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v += part[i][t];
+    out[t] = Mma<T>::from_float(v);
+  }
+  if (tid == 0 && lse_out) *lse_out = lse2 * kLn2;
+}
+
+// Merge of the pieces of every (sequence, KV head) pair that partition edges
+// cut; grid = (B * H_kv pairs, G rows).
+template <int D, typename T>
+__global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeArgs a) {
+  grid_dependency_wait();
+  const int seg = blockIdx.x, r = blockIdx.y;
+  const int b = seg / a.H_kv, h = seg - b * a.H_kv;
+  const int c0 = a.ws_cum[b], np = a.ws_cum[b + 1] - c0;
+  if (np == 0) return;
+  const long long P = static_cast<long long>(a.ws_cum[a.B]) * a.H_kv;
+  const int N = effective_parts(P, a.nparts, a.min_pages);
+  const long long s0 = static_cast<long long>(c0) * a.H_kv + static_cast<long long>(h) * np;
+  const long long wf = part_of(s0, P, N), wl = part_of(s0 + np - 1, P, N);
+  if (wf == wl) return;  // written directly by its only worker
+  const long long slot0 = wf + seg;
+  const size_t row = (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + r);
+  merge_row<D, T>(a.part_lse + slot0 * a.G + r, a.G, a.part_o + (slot0 * a.G + r) * D,
+                  static_cast<long long>(a.G) * D, static_cast<int>(wl - wf + 1),
+                  reinterpret_cast<T *>(a.out) + row * D, a.lse_out ? a.lse_out + row : nullptr);
+}
+
+// Merge of caller-provided partials [B][H_q][S][D]; grid = B * H_q rows.
+template <int D, typename T>
+__global__ void __launch_bounds__(256) generic_merge_kernel(const GenericMergeArgs a) {
+  const long long row = blockIdx.x;
+  const int b = static_cast<int>(row / a.H_q);
+  int count = a.S;
+  if (a.counts) count = clamp_len(__ldg(a.counts + b), a.S);
+  merge_row<D, T>(a.part_lse + row * a.S, 1, a.part_o + row * a.S * D, D, count,
+                  reinterpret_cast<T *>(a.out) + row * D, a.lse_out ? a.lse_out + row : nullptr);
+}
+
+// ------------------------------------------------------------- launchers
+
+namespace {
+
+template <int D>
+struct Tune;
+// d = 128: 8 KB per stage; 4 worker warps x 6 stages = 192 KB of ring per SM.
+template <>
+struct Tune<128> {
+  static constexpr int W = 4, S = 6;
+};
+// d = 64: 4 KB per stage; 4 x 10 stages.
+template <>
+struct Tune<64> {
+  static constexpr int W = 4, S = 10;
+};
+
+template <int D, int NT, typename T>
+cudaError_t launch_decode_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                            cudaStream_t st, int grid) {
+  constexpr int W = Tune<D>::W, S = Tune<D>::S;
+  auto kern = decode_kernel<D, NT, T, W, S>;
+  const size_t smem = Geo<D, W, S>::smem(a.B);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, 32 * W, smem, st>>>(a, tmK, tmV);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_decode_dt(const DecodeArgs &a, int d, const CUtensorMap &tmK,
+                             const CUtensorMap &tmV, cudaStream_t st, int grid) {
+  const bool two = a.G > 8;
+  if (d == 128)
+    return two ? launch_decode_t<128, 2, T>(a, tmK, tmV, st, grid)
+               : launch_decode_t<128, 1, T>(a, tmK, tmV, st, grid);
+  return two ? launch_decode_t<64, 2, T>(a, tmK, tmV, st, grid)
+             : launch_decode_t<64, 1, T>(a, tmK, tmV, st, grid);
+}
+
+template <typename T>
+cudaError_t launch_merge_dt(const DecodeArgs &a, int d, cudaStream_t st) {
+  dim3 grid(a.B * a.H_kv, a.G);
+  if (d == 128) decode_merge_kernel<128, T><<<grid, 256, 0, st>>>(a);
+  else decode_merge_kernel<64, T><<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_generic_dt(const GenericMergeArgs &a, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>(static_cast<long long>(a.B) * a.H_q);
+  if (a.d == 128) generic_merge_kernel<128, T><<<grid, 256, 0, st>>>(a);
+  else generic_merge_kernel<64, T><<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int decode_warps_per_cta(int d) { return d == 128 ? Tune<128>::W : Tune<64>::W; }
+
+size_t decode_smem_bytes(int d, int B) {
+  return d == 128 ? Geo<128, Tune<128>::W, Tune<128>::S>::smem(B)
+                  : Geo<64, Tune<64>::W, Tune<64>::S>::smem(B);
+}
+
+int decode_auto_parts(int d, int sms) { return sms * decode_warps_per_cta(d); }
+
+cudaError_t launch_decode(const DecodeArgs &a, int d, DType dt, const CUtensorMap &tmK,
+                          const CUtensorMap &tmV, cudaStream_t s, int grid) {
+  return dt == DType::BF16 ? launch_decode_dt<__nv_bfloat16>(a, d, tmK, tmV, s, grid)
+                           : launch_decode_dt<__half>(a, d, tmK, tmV, s, grid);
+}
+
+cudaError_t launch_decode_merge(const DecodeArgs &a, int d, DType dt, cudaStream_t s) {
+  if (a.B == 0) return cudaSuccess;
+  return dt == DType::BF16 ? launch_merge_dt<__nv_bfloat16>(a, d, s)
+                           : launch_merge_dt<__half>(a, d, s);
+}
+
+cudaError_t launch_generic_merge(const GenericMergeArgs &a, DType dt, cudaStream_t s) {
+  if (a.B == 0) return cudaSuccess;
+  return dt == DType::BF16 ? launch_generic_dt<__nv_bfloat16>(a, s)
+                           : launch_generic_dt<__half>(a, s);
+}
+
+}  // namespace kvd

@@ -1,0 +1,68 @@
+// kernels.h -- launchers of the decode-step kernels (internal to libkvdecode).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kvd {
+
+enum class DType { F16 = 0, BF16 = 1 };
+
+struct AppendArgs {
+  void *k_cache;
+  void *v_cache;
+  const int32_t *block_table;
+  const int32_t *slot;
+  const void *k_new;
+  const void *v_new;
+  unsigned *err;
+  int B, H_kv, d, num_blocks, maxb;
+};
+
+struct DecodeArgs {
+  const void *q;
+  const int32_t *block_table;
+  const int32_t *seq_lens;
+  void *out;
+  float *lse_out;
+  float *part_o;      // [slots][G][d]
+  float *part_lse;    // [slots][G]
+  int32_t *ws_cum;    // [B + 1] pages per sequence, exclusive prefix sum
+  unsigned *err;
+  float scale_log2;   // scale * log2(e)
+  int B, H_q, H_kv, G, num_blocks, maxb;
+  int nparts;         // N: partitions of the concatenated page list
+  int min_pages;      // lower bound on average pages per used partition
+  int evict_first;    // 1: stream K/V with an L2 evict-first hint
+};
+
+struct GenericMergeArgs {
+  const float *part_o;
+  const float *part_lse;
+  const int32_t *counts;
+  void *out;
+  float *lse_out;
+  int B, H_q, d, S;
+};
+
+// Decode-kernel launch geometry for head dim d (warps per CTA, ring stages).
+struct DecodeGeometry {
+  int warps;
+  int stages;
+  size_t smem_bytes;  // dynamic shared memory for batch B (see decode_smem_bytes)
+};
+
+int decode_warps_per_cta(int d);
+size_t decode_smem_bytes(int d, int B);
+// Partitions = resident worker warps of a device with `sms` SMs.
+int decode_auto_parts(int d, int sms);
+
+cudaError_t launch_append(const AppendArgs &a, DType dt, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs &a, int d, DType dt, const CUtensorMap &tmK,
+                          const CUtensorMap &tmV, cudaStream_t s, int grid);
+cudaError_t launch_decode_merge(const DecodeArgs &a, int d, DType dt, cudaStream_t s);
+cudaError_t launch_generic_merge(const GenericMergeArgs &a, DType dt, cudaStream_t s);
+
+}  // namespace kvd

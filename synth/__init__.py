@@ -10,6 +10,7 @@ from .workloads import (  # noqa: F401
     PAGE_TOKENS,
     Workload,
     build_workload,
+    config_spec,
     named_config,
     NAMED_CONFIGS,
     step_inputs,

@@ -232,36 +232,33 @@ def _lognormal_suffix(B, g, median=1000.0, sigma=1.0):
     return torch.round(x).to(torch.int64)
 
 
-def named_config(name: str, device="cpu", gen_device=None, scale_down: int = 1) -> Workload:
-    """The five synthetic workloads of this method's decode-step benchmark.
+def config_spec(name: str, scale_down: int = 1) -> dict:
+    """Shapes, lengths and build options of a named workload (no pool).
 
-    scale_down > 1 shrinks batch and lengths (same structure) for quick tests.
-    Seeds are 1000 + config index.
+    The five synthetic decode workloads of this method's benchmark; seeds are
+    1000 + config index.  scale_down > 1 shrinks batch and lengths with the
+    same structure, for quick tests.
     """
     s = max(1, int(scale_down))
     if name == "tiny":
         # 1 sequence, 8 heads, d=64, fp16, 1023 cached + 1 appended = 1024
         # tokens on pages 0..63 in order.
-        n = max(1, 1024 // s)
-        return build_workload("tiny", 1, 8, 8, 64, "f16", [n], seed=1001,
-                              placement="identity", device=device, gen_device=gen_device)
+        return dict(B=1, H_q=8, H_kv=8, d=64, dtype="f16", lens=[max(1, 1024 // s)], seed=1001,
+                    opts=dict(placement="identity"))
     if name == "mha7b":
         B = max(1, 32 // s)
-        n = max(1, 4096 // s)
-        return build_workload("mha7b", B, 32, 32, 128, "f16", [n] * B, seed=1002,
-                              placement="shuffle", device=device, gen_device=gen_device)
+        return dict(B=B, H_q=32, H_kv=32, d=128, dtype="f16", lens=[max(1, 4096 // s)] * B,
+                    seed=1002, opts=dict(placement="shuffle"))
     if name == "gqa70b":
         B = max(1, 64 // s)
         g = _gen(1003, "cpu")
         lo, hi = 512 // s, 32768 // s
-        lens = torch.randint(max(1, lo), hi + 1, (B,), generator=g)
-        return build_workload("gqa70b", B, 64, 8, 128, "bf16", lens.tolist(), seed=1003,
-                              placement="shuffle", outlier_frac=0.01, outlier_scale=20.0,
-                              device=device, gen_device=gen_device)
+        lens = torch.randint(max(1, lo), hi + 1, (B,), generator=g).tolist()
+        return dict(B=B, H_q=64, H_kv=8, d=128, dtype="bf16", lens=lens, seed=1003,
+                    opts=dict(placement="shuffle", outlier_frac=0.01, outlier_scale=20.0))
     if name == "long":
-        n = max(1, 131072 // s)
-        return build_workload("long", 1, 64, 8, 128, "bf16", [n], seed=1004,
-                              placement="shuffle", device=device, gen_device=gen_device)
+        return dict(B=1, H_q=64, H_kv=8, d=128, dtype="bf16", lens=[max(1, 131072 // s)],
+                    seed=1004, opts=dict(placement="shuffle"))
     if name == "cbatch":
         groups, per = 8, max(1, 32 // s)
         B = groups * per
@@ -270,11 +267,17 @@ def named_config(name: str, device="cpu", gen_device=None, scale_down: int = 1) 
         g = _gen(1005, "cpu")
         suf = _lognormal_suffix(B, g, median=1000.0 / s)
         suf = suf.clamp(min=1, max=max(1, cap - prefix))
-        lens = (prefix + suf).tolist()
-        return build_workload("cbatch", B, 32, 8, 128, "f16", lens, seed=1005, steps=16,
-                              placement="shuffle", prefix_groups=groups, prefix_tokens=prefix,
-                              device=device, gen_device=gen_device)
+        return dict(B=B, H_q=32, H_kv=8, d=128, dtype="f16", lens=(prefix + suf).tolist(),
+                    seed=1005, opts=dict(placement="shuffle", steps=16, prefix_groups=groups,
+                                         prefix_tokens=prefix))
     raise KeyError(name)
+
+
+def named_config(name: str, device="cpu", gen_device=None, scale_down: int = 1) -> Workload:
+    """Build the named workload's pool, block table and lengths (see config_spec)."""
+    c = config_spec(name, scale_down)
+    return build_workload(name, c["B"], c["H_q"], c["H_kv"], c["d"], c["dtype"], c["lens"],
+                          seed=c["seed"], device=device, gen_device=gen_device, **c["opts"])
 
 
 NAMED_CONFIGS = ("tiny", "mha7b", "gqa70b", "long", "cbatch")

@@ -1,0 +1,241 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Append must be bit-exact over the whole pool; attention must be within the
+max-abs tolerance (2e-3 fp16, 1e-2 bf16) of the oracle.  Inputs are seeded
+synthetic workloads whose unused pool slots hold NaN canaries.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import (LSE_TOL, TOL, gpu_state, gpu_step, max_err, max_lse_err, oracle_step,
+                         words)
+from synth import CANARY_WORD, build_workload, step_inputs, to_words
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kvd():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import kv_cache_decode_scatters_b200 as m
+    m.kvd_read_device_error(clear=True)
+    return m
+
+
+def run_case(kvd, w, step=0, num_partitions=0):
+    si = step_inputs(w, step)
+    kc, vc, bt = gpu_state(w)
+    out, lse = gpu_step(kvd, w, si, kc, vc, bt, num_partitions=num_partitions)
+    okc, ovc, ref = oracle_step(w, si)
+    return si, kc, vc, out, lse, okc, ovc, ref
+
+
+# ------------------------------------------------------------------ append
+
+@pytest.mark.parametrize("d,dtype", [(64, "f16"), (128, "bf16"), (128, "f16")])
+def test_append_bit_exact_whole_pool(kvd, d, dtype):
+    w = build_workload("app", 6, 8, 4, d, dtype, [1, 15, 16, 17, 33, 0], seed=501, spare_pages=5)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    kvd.kvd_append(kc, vc, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    torch.cuda.synchronize()
+    okc, ovc = to_words(w.k_cache).copy(), to_words(w.v_cache).copy()
+    oracle.append(okc, ovc, w.block_table.numpy(), si["slot"].numpy(), to_words(si["k_new"]),
+                  to_words(si["v_new"]))
+    assert np.array_equal(to_words(kc), okc)
+    assert np.array_equal(to_words(vc), ovc)
+    assert kvd.kvd_read_device_error() == 0
+
+
+def test_append_out_of_range_is_flagged_not_written(kvd):
+    w = build_workload("app", 3, 4, 4, 128, "f16", [5, 9, 20], seed=502)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    slot = si["slot"].clone()
+    slot[1] = 16 * w.max_blocks + 3          # beyond the table
+    bt_bad = bt.clone()
+    bt_bad[2, 1] = w.num_blocks + 100        # page outside the pool
+    before_k = to_words(kc).copy()
+    kvd.kvd_append(kc, vc, bt_bad, slot.cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    flags = kvd.kvd_read_device_error(clear=True)
+    assert flags & kvd.KVD_DEVERR_SLOT and flags & kvd.KVD_DEVERR_BLOCK_TABLE
+    okc = before_k.copy()
+    ovc = to_words(w.v_cache).copy()
+    s0 = si["slot"].numpy().copy()
+    s0[1:] = -1
+    oracle.append(okc, ovc, w.block_table.numpy(), s0, to_words(si["k_new"]), to_words(si["v_new"]))
+    assert np.array_equal(to_words(kc), okc), "only sequence 0 may have been written"
+
+
+# --------------------------------------------------------------- attention
+
+CASES = [
+    # B, H_q, H_kv, d, dtype, lens
+    (1, 8, 8, 64, "f16", [1024]),                  # the pages' (1, 8, 1024, 64) example
+    (3, 4, 4, 128, "f16", [1, 15, 16]),
+    (4, 8, 8, 128, "f16", [17, 31, 32, 33]),
+    (2, 8, 1, 128, "bf16", [100, 257]),            # MQA, group 8
+    (2, 16, 1, 128, "bf16", [40, 130]),            # MQA, group 16
+    (3, 16, 8, 64, "f16", [64, 1, 300]),           # group 2
+    (3, 32, 8, 128, "bf16", [500, 77, 1000]),      # group 4
+    (4, 64, 8, 128, "bf16", [513, 2049, 16, 999]), # group 8 (70B shape)
+    (2, 32, 2, 128, "f16", [1500, 31]),            # group 16
+    (2, 12, 4, 64, "bf16", [48, 95]),              # group 3 (padded n-tile)
+    (5, 8, 2, 128, "f16", [3, 0, 45, 0, 200]),     # empty sequences in the batch
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_d{c[3]}_{c[4]}")
+def test_decode_matches_oracle(kvd, case):
+    B, H_q, H_kv, d, dtype, lens = case
+    w = build_workload("par", B, H_q, H_kv, d, dtype, lens, seed=700 + CASES.index(case), spare_pages=3)
+    si, kc, vc, out, lse, okc, ovc, ref = run_case(kvd, w)
+    assert np.array_equal(to_words(kc), okc) and np.array_equal(to_words(vc), ovc)
+    err = max_err(out, ref)
+    assert err <= TOL[w.dtype], f"max abs error {err}"
+    assert max_lse_err(lse, ref) <= LSE_TOL
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert torch.all(out[b] == 0) and torch.all(torch.isneginf(lse[b]))
+    assert kvd.kvd_read_device_error() == 0
+
+
+@pytest.mark.parametrize("parts", [1, 2, 3, 7, 64, 1000, 0])
+def test_partition_counts_agree(kvd, parts):
+    w = build_workload("parts", 3, 32, 8, 128, "bf16", [700, 33, 1200], seed=601)
+    si, kc, vc, out, lse, okc, ovc, ref = run_case(kvd, w, num_partitions=parts)
+    assert max_err(out, ref) <= TOL[w.dtype]
+    assert max_lse_err(lse, ref) <= LSE_TOL
+
+
+def test_single_token_returns_v0_exactly(kvd):
+    w = build_workload("one", 3, 8, 2, 128, "f16", [1, 1, 1], seed=611)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    out, _ = gpu_step(kvd, w, si, kc, vc, bt)
+    v = si["v_new"].cuda().repeat_interleave(4, dim=1)
+    assert torch.equal(out, v)
+
+
+def test_constant_values_give_that_constant(kvd):
+    w = build_workload("const", 2, 4, 4, 64, "bf16", [200, 17], seed=612)
+    si = step_inputs(w, 0)
+    c = torch.randn(4, 64, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    vw = w.v_cache
+    for b, n in enumerate([200, 17]):
+        for j in range(n - 1):
+            vw[int(w.block_table[b, j // 16]), :, j % 16, :] = c
+    si["v_new"][:] = c
+    kc, vc, bt = gpu_state(w)
+    out, _ = gpu_step(kvd, w, si, kc, vc, bt)
+    ref = c.float().cuda()[None].expand(2, 4, 64)
+    assert torch.max(torch.abs(out.float() - ref)).item() <= 2 ** -7 * ref.abs().max().item()
+
+
+def test_paged_equals_contiguous_placement(kvd):
+    lens = [300, 47, 129]
+    a = build_workload("pl", 3, 16, 4, 128, "f16", lens, seed=621, placement="shuffle")
+    si = step_inputs(a, 0)
+    # same logical content, pages handed out in logical order
+    b = build_workload("pl", 3, 16, 4, 128, "f16", lens, seed=621, placement="identity")
+    kb = b.k_cache.clone()
+    vb = b.v_cache.clone()
+    for s in range(3):
+        for i in range((lens[s] + 15) // 16):
+            kb[int(b.block_table[s, i])] = a.k_cache[int(a.block_table[s, i])]
+            vb[int(b.block_table[s, i])] = a.v_cache[int(a.block_table[s, i])]
+    b.k_cache, b.v_cache = kb, vb
+    outs = []
+    for w in (a, b):
+        kc, vc, bt = gpu_state(w)
+        o, _ = gpu_step(kvd, w, si, kc, vc, bt, num_partitions=37)
+        outs.append(o)
+    assert torch.equal(outs[0], outs[1]), "physical placement changed the result"
+
+
+def test_shared_prefix_equals_private_copies(kvd):
+    lens = [90, 130, 70, 64 + 1]
+    w = build_workload("pre", 4, 8, 2, 128, "bf16", lens, seed=631, prefix_groups=2, prefix_tokens=64)
+    assert w.block_table[0, 0] == w.block_table[1, 0]
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    o1, _ = gpu_step(kvd, w, si, kc, vc, bt, num_partitions=5)
+    pages, rows = [], torch.full_like(w.block_table, -1)
+    for b, n in enumerate(lens):
+        for i in range((n + 15) // 16):
+            rows[b, i] = len(pages)
+            pages.append(int(w.block_table[b, i]))
+    idx = torch.tensor(pages)
+    kc2, vc2 = w.k_cache[idx].cuda(), w.v_cache[idx].cuda()
+    o2, _ = gpu_step(kvd, w, si, kc2, vc2, rows.cuda(), num_partitions=5)
+    assert torch.equal(o1, o2)
+
+
+def test_bad_block_table_entry_is_flagged_and_contained(kvd):
+    w = build_workload("bad", 3, 8, 8, 128, "f16", [64, 64, 64], seed=641)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    kvd.kvd_append(kc, vc, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    bt_bad = bt.clone()
+    bt_bad[1, 2] = -5
+    out = kvd.kvd_decode_attention(si["q"].cuda(), kc, vc, bt_bad, si["seq_lens"].cuda(), w.scale,
+                                   num_partitions=3)
+    flags = kvd.kvd_read_device_error(clear=True)
+    assert flags & kvd.KVD_DEVERR_BLOCK_TABLE
+    _, _, ref = oracle_step(w, si)
+    g = out.float().cpu().double().numpy()
+    for b in (0, 2):
+        assert np.max(np.abs(g[b] - ref[b][0])) <= TOL[w.dtype]
+    assert np.all(np.isfinite(g[1]))
+
+
+def test_bad_seq_len_is_flagged(kvd):
+    w = build_workload("badlen", 2, 4, 4, 64, "f16", [20, 20], seed=651)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    sl = si["seq_lens"].clone()
+    sl[0] = 16 * w.max_blocks + 1
+    sl[1] = -4
+    kvd.kvd_decode_attention(si["q"].cuda(), kc, vc, bt, sl.cuda(), w.scale)
+    assert kvd.kvd_read_device_error(clear=True) & kvd.KVD_DEVERR_SEQ_LEN
+
+
+def test_generic_merge_matches_oracle(kvd):
+    rng = np.random.default_rng(5)
+    for d, dt in ((128, torch.float16), (64, torch.bfloat16)):
+        B, H_q, S = 3, 4, 6
+        po = rng.standard_normal((B, H_q, S, d))
+        pl = rng.standard_normal((B, H_q, S)) * 3
+        pl[0, 1, 2] = -np.inf
+        pl[2, :, :] = -np.inf                     # sequence 2: everything empty
+        counts = np.array([6, 4, 5], np.int32)
+        po32, pl32 = po.astype(np.float32), pl.astype(np.float32)
+        ref, ref_lse = oracle.merge(po32.astype(np.float64), pl32.astype(np.float64), counts)
+        lse = torch.empty((B, H_q), dtype=torch.float32, device="cuda")
+        out = kvd.kvd_merge_lse(torch.from_numpy(po32).cuda(), torch.from_numpy(pl32).cuda(),
+                                torch.from_numpy(counts).cuda(), lse_out=lse, dtype=dt)
+        torch.cuda.synchronize()
+        err = np.max(np.abs(out.float().cpu().double().numpy() - ref))
+        assert err <= TOL[dt] * 2, err
+        fin = np.isfinite(ref_lse)
+        got = lse.cpu().double().numpy()
+        assert np.array_equal(np.isfinite(got), fin)
+        assert np.max(np.abs(got[fin] - ref_lse[fin])) <= LSE_TOL
+        assert torch.all(out[2] == 0)
+
+
+def test_repeated_calls_are_deterministic(kvd):
+    w = build_workload("det", 4, 32, 8, 128, "bf16", [900, 40, 1500, 333], seed=661)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    kvd.kvd_append(kc, vc, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    q, sl = si["q"].cuda(), si["seq_lens"].cuda()
+    a = kvd.kvd_decode_attention(q, kc, vc, bt, sl, w.scale)
+    b = kvd.kvd_decode_attention(q, kc, vc, bt, sl, w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
