@@ -245,7 +245,7 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    w = named_config(args.workload, device="cuda", gen_device="cuda")
+    w = named_config(args.workload, device="cuda", gen_device="cuda", scale_down=args.scale_down)
     si = step_inputs(w, 0)
     kc, vc, bt = w.k_cache, w.v_cache, w.block_table.to(dev)
     q, k_new, v_new = si["q"], si["k_new"], si["v_new"]
@@ -351,7 +351,8 @@ def run_ours(args):
         "dtype": w.dtype_name,
         "data": "synthetic",
         "config": {
-            "workload": w.name, "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
+            "workload": w.name if args.scale_down == 1 else f"{w.name}/scale_down={args.scale_down}",
+            "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
             "seq_lens": _lens_desc(w), "page_tokens": 16, "pages_in_pool": w.num_blocks,
             "placement": "shuffled pages", "partitions": args.partitions or kvd.kvd_auto_partitions(),
             "bytes_per_step": step_bytes, "attention_bytes": a_bytes, "append_bytes": p_bytes,
@@ -408,6 +409,8 @@ def main(argv=None):
     p.add_argument("--ref-budget", type=float, default=8.0,
                    help="seconds of oracle work per reference-arm step")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--scale-down", type=int, default=1,
+                   help="shrink batch and lengths by this factor (profiling small cases only)")
     args = p.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

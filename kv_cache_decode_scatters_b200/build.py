@@ -1,6 +1,8 @@
 """Build libkvdecode.so in-tree with nvcc for sm_100a (B200).
 
-    python -m kv_cache_decode_scatters_b200.build [--force] [--verbose-ptxas]
+    python kv_cache_decode_scatters_b200/build.py [--force] [--verbose-ptxas]
+
+(run it as a script: importing the package loads the library it builds)
 
 The library is written next to this file so it travels with the source tree;
 it is rebuilt when any source or the public header is newer than it.
