@@ -160,11 +160,23 @@ def dist_setup(n_gpus):
 
 
 def max_over_ranks(dist, x: float) -> float:
+    """Largest x over all ranks (host timing bookkeeping, not a data-path collective)."""
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate(dist, world, steps, total_ms, attn_ms, step_bytes):
+    """Whole-job numbers from per-rank device times: the slowest rank sets the
+    step time; value counts the bytes every rank processed (weak scaling)."""
+    total_ms = max_over_ranks(dist, total_ms)
+    attn_ms = max_over_ranks(dist, attn_ms)
+    ms_step = total_ms / steps
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    return ms_step, attn_ms, value
 
 
 def barrier(dist):
@@ -245,7 +257,9 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    w = named_config(args.workload, device="cuda", gen_device="cuda", scale_down=args.scale_down)
+    # each rank decodes its own batch of the workload (rank 0: the standard one)
+    w = named_config(args.workload, device="cuda", gen_device="cuda", scale_down=args.scale_down,
+                     shard=rank)
     si = step_inputs(w, 0)
     kc, vc, bt = w.k_cache, w.v_cache, w.block_table.to(dev)
     q, k_new, v_new = si["q"], si["k_new"], si["v_new"]
@@ -289,12 +303,9 @@ def run_ours(args):
     if sampler:
         sampler.__exit__(None, None, None)
     barrier(dist)
-    total_ms = t_start.elapsed_time(t_end)
-    attn_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
-    total_ms = max_over_ranks(dist, total_ms)
-    attn_ms = max_over_ranks(dist, attn_ms)
-    ms_step = total_ms / args.steps
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    ms_step, attn_ms, value = aggregate(dist, world, args.steps, t_start.elapsed_time(t_end),
+                                        sum(a.elapsed_time(b) for a, b in evs) / args.steps,
+                                        step_bytes)
 
     # ---- end to end through the public API with pinned host buffers
     h_in = {n: t.cpu().pin_memory() for n, t in

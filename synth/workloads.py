@@ -232,14 +232,26 @@ def _lognormal_suffix(B, g, median=1000.0, sigma=1.0):
     return torch.round(x).to(torch.int64)
 
 
-def config_spec(name: str, scale_down: int = 1) -> dict:
+def config_spec(name: str, scale_down: int = 1, shard: int = 0) -> dict:
     """Shapes, lengths and build options of a named workload (no pool).
 
     The five synthetic decode workloads of this method's benchmark; seeds are
     1000 + config index.  scale_down > 1 shrinks batch and lengths with the
-    same structure, for quick tests.
+    same structure, for quick tests.  shard > 0 draws another batch of the
+    same workload (other seeds), e.g. the sequences of another GPU.
     """
     s = max(1, int(scale_down))
+    spec = _config_spec(name, s)
+    if shard:
+        off = 7919 * int(shard)
+        spec["seed"] += off
+        if name in ("gqa70b", "cbatch"):
+            spec = _config_spec(name, s, seed_offset=off)
+            spec["seed"] += off
+    return spec
+
+
+def _config_spec(name: str, s: int, seed_offset: int = 0) -> dict:
     if name == "tiny":
         # 1 sequence, 8 heads, d=64, fp16, 1023 cached + 1 appended = 1024
         # tokens on pages 0..63 in order.
@@ -251,7 +263,7 @@ def config_spec(name: str, scale_down: int = 1) -> dict:
                     seed=1002, opts=dict(placement="shuffle"))
     if name == "gqa70b":
         B = max(1, 64 // s)
-        g = _gen(1003, "cpu")
+        g = _gen(1003 + seed_offset, "cpu")
         lo, hi = 512 // s, 32768 // s
         lens = torch.randint(max(1, lo), hi + 1, (B,), generator=g).tolist()
         return dict(B=B, H_q=64, H_kv=8, d=128, dtype="bf16", lens=lens, seed=1003,
@@ -264,7 +276,7 @@ def config_spec(name: str, scale_down: int = 1) -> dict:
         B = groups * per
         prefix = max(PAGE_TOKENS, (4096 // s) // PAGE_TOKENS * PAGE_TOKENS)
         cap = 16384 // s - 16
-        g = _gen(1005, "cpu")
+        g = _gen(1005 + seed_offset, "cpu")
         suf = _lognormal_suffix(B, g, median=1000.0 / s)
         suf = suf.clamp(min=1, max=max(1, cap - prefix))
         return dict(B=B, H_q=32, H_kv=8, d=128, dtype="f16", lens=(prefix + suf).tolist(),
@@ -273,9 +285,10 @@ def config_spec(name: str, scale_down: int = 1) -> dict:
     raise KeyError(name)
 
 
-def named_config(name: str, device="cpu", gen_device=None, scale_down: int = 1) -> Workload:
+def named_config(name: str, device="cpu", gen_device=None, scale_down: int = 1,
+                 shard: int = 0) -> Workload:
     """Build the named workload's pool, block table and lengths (see config_spec)."""
-    c = config_spec(name, scale_down)
+    c = config_spec(name, scale_down, shard)
     return build_workload(name, c["B"], c["H_q"], c["H_kv"], c["d"], c["dtype"], c["lens"],
                           seed=c["seed"], device=device, gen_device=gen_device, **c["opts"])
 
