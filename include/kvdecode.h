@@ -124,6 +124,42 @@ kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *
                                 void *workspace, size_t workspace_bytes,
                                 float *lse_out, kvd_dtype dtype, void *stream);
 
+/* Bytes of the library's fixed scratch array used by kvd_decode_attention_static. */
+#define KVD_STATIC_WORKSPACE_BYTES (8u << 20)
+
+/*
+ * kvd_decode_attention_static -- kvd_decode_attention for callers that cannot
+ * allocate device memory.  The pages have no counterpart of this call: it is
+ * an interface convenience, computing exactly what kvd_decode_attention
+ * computes with num_partitions = 0.
+ *
+ * Some callers are not allowed to allocate: a plugin inside an inference
+ * server that is given only its input and output buffers, a runtime that
+ * plans all device memory up front, or a decode loop that cannot pay for
+ * cudaMalloc / cudaFree, which may synchronise the device.  This entry point
+ * takes no workspace argument; its scratch is a fixed array of
+ * KVD_STATIC_WORKSPACE_BYTES (8 MiB) compiled into the library, which every
+ * GPU that loads the library keeps until the process exits.  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *
+ *   Arguments: as kvd_decode_attention (q, caches, block table, lengths,
+ *   scale, out, shape, optional lse_out, dtype, stream).
+ *   Returns KVD_ERR_UNSUPPORTED, with the needed size in kvd_last_error(),
+ *   when the shape needs more scratch than the fixed array holds (the needed
+ *   size is kvd_workspace_size(B, H_q, H_kv, d, 0)).
+ *   The first call on a device looks up the array's device address with that
+ *   device current; make that first call before any stream capture.
+ *   All calls on one device share the array: calls that overlap on the GPU
+ *   (on streams not ordered with each other) race and corrupt each other's
+ *   results.  No part of the array needs to start at zero; it keeps the last
+ *   call's contents.
+ */
+kvd_status kvd_decode_attention_static(const void *q, const void *k_cache, const void *v_cache,
+                                       const int32_t *block_table, const int32_t *seq_lens,
+                                       float scale, void *out, int B, int H_q, int H_kv, int d,
+                                       int num_blocks, int max_blocks_per_seq, float *lse_out,
+                                       kvd_dtype dtype, void *stream);
+
 /*
  * kvd_merge_lse -- combine S partial attention results of each query row.
  * Not printed on the pages as such: it is the running-state rescale of [LES]

@@ -20,7 +20,8 @@ import torch
 __all__ = [
     "KVD_OK", "KVD_ERR_INVALID", "KVD_ERR_UNSUPPORTED", "KVD_ERR_CUDA", "KVD_ERR_WORKSPACE",
     "KVD_F16", "KVD_BF16", "KVD_PAGE_TOKENS", "KvdError",
-    "kvd_append", "kvd_decode_attention", "kvd_merge_lse", "kvd_workspace_size",
+    "kvd_append", "kvd_decode_attention", "kvd_decode_attention_static", "kvd_merge_lse",
+    "kvd_workspace_size", "KVD_STATIC_WORKSPACE_BYTES",
     "kvd_auto_partitions", "kvd_kv_bytes_per_token", "kvd_read_device_error",
     "kvd_last_error", "alloc_workspace", "library_path", "lib",
 ]
@@ -28,6 +29,7 @@ __all__ = [
 KVD_OK, KVD_ERR_INVALID, KVD_ERR_UNSUPPORTED, KVD_ERR_CUDA, KVD_ERR_WORKSPACE = 0, 1, 2, 3, 4
 KVD_F16, KVD_BF16 = 0, 1
 KVD_PAGE_TOKENS = 16
+KVD_STATIC_WORKSPACE_BYTES = 8 << 20
 KVD_DEVERR_BLOCK_TABLE, KVD_DEVERR_SEQ_LEN, KVD_DEVERR_SLOT, KVD_DEVERR_TIMEOUT = 1, 2, 4, 8
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -41,13 +43,15 @@ def _load():
     path = library_path()
     if not os.path.exists(path):
         raise ImportError(
-            f"{path} is missing: build it with `python -m kv_cache_decode_scatters_b200.build`")
+            f"{path} is missing: build it with `python kv_cache_decode_scatters_b200/build.py`")
     L = ctypes.CDLL(path)
     P, I, S, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
     L.kvd_append.restype = I
     L.kvd_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
     L.kvd_decode_attention.restype = I
     L.kvd_decode_attention.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, I, P, S, P, I, P]
+    L.kvd_decode_attention_static.restype = I
+    L.kvd_decode_attention_static.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, P, I, P]
     L.kvd_merge_lse.restype = I
     L.kvd_merge_lse.argtypes = [P, P, P, I, I, I, I, P, P, I, P]
     L.kvd_workspace_size.restype = S
@@ -177,6 +181,32 @@ def kvd_decode_attention(q, k_cache, v_cache, block_table, seq_lens, scale=None,
         int(num_partitions), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         lse_ptr, _dtype_code(k_cache), _stream(stream)),
         "kvd_decode_attention")
+    return out
+
+
+def kvd_decode_attention_static(q, k_cache, v_cache, block_table, seq_lens, scale=None, out=None,
+                                lse_out=None, stream=None):
+    """kvd_decode_attention without a workspace argument, for callers that
+    cannot allocate device memory: the scratch is the library's fixed
+    KVD_STATIC_WORKSPACE_BYTES array (shared by every call on a device, so
+    calls overlapping on the GPU race).  `out` must be given by such callers;
+    when it is None this wrapper allocates it with torch for convenience."""
+    B, H_q, d = q.shape
+    NB, H_kv, P, d2 = k_cache.shape
+    if P != KVD_PAGE_TOKENS or d2 != d:
+        raise ValueError("q / cache shape mismatch")
+    dt = k_cache.dtype
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    lse_ptr = None if lse_out is None else _dev(lse_out, "lse_out", torch.float32)
+    _check(_lib.kvd_decode_attention_static(
+        _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
+        float(scale), _dev(out, "out", dt), B, H_q, H_kv, d, NB, block_table.shape[1],
+        lse_ptr, _dtype_code(k_cache), _stream(stream)),
+        "kvd_decode_attention_static")
     return out
 
 

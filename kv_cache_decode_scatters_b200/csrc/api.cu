@@ -138,6 +138,11 @@ kvd_status check_heads(int B, int H_q, int H_kv, int d) {
 
 }  // namespace
 
+namespace kvd {
+// Lets other translation units of the library set the text kvd_last_error returns.
+void record_error(const char *msg) { g_last_error = msg; }
+}  // namespace kvd
+
 extern "C" {
 
 const char *kvd_last_error(void) { return g_last_error.c_str(); }

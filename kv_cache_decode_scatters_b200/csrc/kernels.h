@@ -59,6 +59,9 @@ size_t decode_smem_bytes(int d, int B);
 // Partitions = resident worker warps of a device with `sms` SMs.
 int decode_auto_parts(int d, int sms);
 
+// Set the text returned by kvd_last_error on this host thread.
+void record_error(const char *msg);
+
 cudaError_t launch_append(const AppendArgs &a, DType dt, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, int d, DType dt, const CUtensorMap &tmK,
                           const CUtensorMap &tmV, cudaStream_t s, int grid);
