@@ -36,9 +36,9 @@ kvd_status cuda_fail(cudaError_t e, const char *what) {
 }
 
 constexpr int kMaxDevices = 64;
-// Average pages per partition below which the automatic split stops cutting
-// (keeps tiny problems from producing more partials than pages).
-constexpr int kAutoMinPages = 8;
+// Average pages per partition (CTA) below which the automatic split stops
+// cutting, so each of a CTA's worker warps gets a couple of pages at least.
+constexpr int kAutoMinPages = 32;
 
 std::mutex g_mu;
 int g_sms[kMaxDevices];
@@ -121,7 +121,8 @@ kvd_status resolve_parts(int d, int num_partitions, int *N) {
   if (st) return st;
   st = sm_count(dev, &sms);
   if (st) return st;
-  *N = kvd::decode_auto_parts(d, sms);
+  (void)d;
+  *N = kvd::decode_auto_parts(sms);
   return KVD_OK;
 }
 
@@ -260,14 +261,15 @@ kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *
   if (st) return st;
 
   // K and V pools as 3-D tensors {64 elements, d/64 units, num_blocks*H_kv*16
-  // rows}; one box = one page of one head (16 rows x d), 128-byte swizzled.
+  // rows}; one box = one 64-element half of one page of one head (16 rows x
+  // 64), 128-byte swizzled.
   CUtensorMap tm[2];
   const void *pools[2] = {k_cache, v_cache};
   for (int i = 0; i < 2; ++i) {
     cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(d / 64),
                           static_cast<cuuint64_t>(num_blocks) * H_kv * KVD_PAGE_TOKENS};
     cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(d) * 2};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(d / 64), KVD_PAGE_TOKENS};
+    cuuint32_t box[3] = {64, 1, KVD_PAGE_TOKENS};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = encode(&tm[i],
                         dtype == KVD_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -302,9 +304,7 @@ kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *
 
   const kvd::DType dt = dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int W = kvd::decode_warps_per_cta(d);
-  const int grid = (N + W - 1) / W;
-  cudaError_t e = kvd::launch_decode(a, d, dt, tm[0], tm[1], s, grid);
+  cudaError_t e = kvd::launch_decode(a, d, dt, tm[0], tm[1], s, N);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   e = kvd::launch_decode_merge(a, d, dt, s);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");

@@ -16,6 +16,9 @@
 namespace kvd {
 
 __global__ void __launch_bounds__(256) append_kernel(const AppendArgs a) {
+  // let the decode grid that usually follows be scheduled early; it waits for
+  // this grid's writes before it reads anything
+  grid_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long pair = static_cast<long long>(blockIdx.x) * 8 + warp;
   if (pair >= static_cast<long long>(a.B) * a.H_kv) return;

@@ -11,17 +11,22 @@
 // How it is laid out on the B200:
 //  * Work split (stream-K).  The pages of all (sequence, KV head) pairs,
 //    concatenated, form one list of P pages; it is cut into N equal
-//    contiguous partitions, one per worker warp (N = resident warps of the
-//    GPU).  Every worker streams the same number of pages whatever the
-//    sequence lengths are.  A pair that lies inside one partition is written
-//    straight to `out`; a pair cut by partition edges leaves one normalised
-//    partial (o, lse) per piece, at slot (worker + pair), and the merge
-//    kernel combines them.
+//    contiguous partitions, one per CTA (N = SM count by default), and each
+//    CTA's partition into equal contiguous shares, one per worker warp.  Every
+//    warp streams the same number of pages whatever the sequence lengths are,
+//    and warps never synchronise while streaming.
+//  * A pair inside one warp's share is written straight to `out`.  A pair
+//    several warps of the CTA hold pieces of is combined once, at the end, in
+//    shared memory (each piece parks its unnormalised accumulators, row max
+//    and row sum).  A pair that crosses CTA partitions leaves one normalised
+//    partial (o, lse) per CTA at slot (CTA + pair), and the merge kernel
+//    combines those.
 //  * Each worker warp owns an S-stage ring in shared memory.  Lane 0 issues
-//    two TMA tile loads per page (K and V, 16 x d each, 128-byte swizzle)
-//    that complete on the stage's mbarrier; the whole warp waits, computes,
-//    and hands the stage back to the next page.  No other warp is involved,
-//    so there is no block-level synchronisation in the main loop.
+//    TMA tile loads for each page (K and V, each as d/64 boxes of 16 x 64
+//    elements with the 128-byte swizzle) that complete on the stage's
+//    mbarrier; the whole warp waits, computes, and hands the stage back to
+//    the next page.  Latency is hidden by many warps (12-16 per SM) rather
+//    than by deep per-warp rings.
 //  * Every KV byte is read once per GQA group: the G query rows of a KV head
 //    ride along as the N dimension of the tensor-core tile.  Per page,
 //    S^T[16 tokens x 8 rows] = K[16 x d] . Q^T uses mma.m16n8k16 with the K
@@ -30,35 +35,48 @@
 //    operand of O^T[d x 8] += V^T[d x 16] . P^T[16 x 8] (ldmatrix.trans).
 //    G <= 8 uses one n-tile, G <= 16 two.
 //  * Softmax in base 2: scores are scaled by scale * log2(e) in fp32 and
-//    exponentiated with ex2.approx.  Probabilities are rounded once to the
-//    storage dtype for the PV product and the running sum uses the same
-//    rounded values, so the output is an exact weighted mean of V up to fp32
-//    accumulation.
+//    exponentiated with ex2.approx.  For fp16 the probabilities are rounded
+//    once for the PV product and the running sum uses the same rounded
+//    values; for bf16 (8 significant bits) each probability is carried as a
+//    rounded head plus a rounded remainder in two PV products.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
+
+#ifndef KVD_BF16_SPLIT_P
+#define KVD_BF16_SPLIT_P 1
+#endif
 
 namespace kvd {
 
 namespace {
 
-template <int D, int W, int S>
+template <int D, int NT, int W, int S>
 struct Geo {
   static constexpr int kPageBytes = kPage * D * 2;      // one K (or V) page of one head
   static constexpr int kStageBytes = 2 * kPageBytes;    // K page then V page
   static constexpr int kThreads = 32 * W;
   static constexpr int kSteps = D / 16;                 // k-steps of S, m-tiles of O
+  static constexpr int kEdgeFloats = 8 * NT * D;        // one parked accumulator tile
+  static_assert(kEdgeFloats * 4 <= kStageBytes, "a parked tile must fit in one stage");
   static size_t smem(int B) {
-    return 1024 + (size_t)W * S * kStageBytes + (size_t)W * S * 16 + (size_t)(B + 1) * 4;
+    return 1024 + (size_t)W * S * kStageBytes + (size_t)W * kEdgeFloats * 4 + (size_t)W * S * 16 +
+           (size_t)W * 2 * 2 * 8 * NT * 4 + (size_t)W * 2 * 4 + (size_t)(B + 1) * 4;
   }
 };
 
 // Byte offset of element column `col` (a multiple of 8) of token row t inside
-// a page stored by a 128B-swizzled TMA box of 64-element units.
+// a page staged as d/64 boxes of [16 tokens][64 elements], each box one
+// 2 KB run of 128-byte rows with the TMA 128-byte swizzle (16-byte chunk
+// index XOR row % 8).  Keeping each 64-column half in its own 2 KB run puts 8
+// consecutive tokens on 8 different chunk positions, so every 8-row ldmatrix
+// phase is free of bank conflicts.
 template <int D>
 __device__ __forceinline__ uint32_t swz(int t, int col) {
-  const int u = t * (D / 64) + (col >> 6);
+  const int half = col >> 6;
   const int chunk = (col & 63) >> 3;
-  return static_cast<uint32_t>(u * 128 + ((chunk ^ (u & 7)) << 4));
+  return static_cast<uint32_t>(half * (kPage * 128) + t * 128 + ((chunk ^ (t & 7)) << 4));
 }
 
 __device__ __forceinline__ int clamp_len(int n, int cap) { return n < 0 ? 0 : (n > cap ? cap : n); }
@@ -93,22 +111,34 @@ template <int D, int NT, typename T, int W, int S>
 __global__ void __launch_bounds__(32 * W, 1)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV) {
-  using Gm = Geo<D, W, S>;
+  using Gm = Geo<D, NT, W, S>;
   using M = Mma<T>;
+  constexpr int kRows = 8 * NT;  // query rows per tile (G padded)
+  // bf16 keeps only 8 significant bits of each probability; carrying the
+  // rounding remainder in a second PV product restores ~16 bits for the cost
+  // of d/16 extra MMAs per page (free while the kernel waits on HBM).
+  constexpr bool kSplitP = KVD_BF16_SPLIT_P && std::is_same<T, __nv_bfloat16>::value;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int warp_tot[32];
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *stages = smem;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)W * S * Gm::kStageBytes);
+  float *edge_acc = reinterpret_cast<float *>(smem + (size_t)W * S * Gm::kStageBytes);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(edge_acc + (size_t)W * Gm::kEdgeFloats);
   int2 *meta = reinterpret_cast<int2 *>(bars + W * S);
-  int *cum = reinterpret_cast<int *>(meta + W * S);
+  float *edge_ml = reinterpret_cast<float *>(meta + W * S);  // [W][2][2][kRows]: m, l
+  int *edge_id = reinterpret_cast<int *>(edge_ml + W * 2 * 2 * kRows);  // [W][2]
+  int *cum = edge_id + 2 * W;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cap = a.maxb * kPage;
 
+  // Launched as a programmatic dependent: nothing is read before the
+  // preceding grid has completed and its writes are visible.  Dependents (the
+  // merge) may be scheduled at once; they wait for this grid the same way.
   grid_dependency_wait();
+  grid_launch_dependents();
   if (tid == 0) {
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
@@ -140,6 +170,7 @@ __global__ void __launch_bounds__(32 * W, 1)
       run += (clamp_len(__ldg(a.seq_lens + b), cap) + kPage - 1) / kPage;
     }
     if (tid == 0) cum[a.B] = warp_tot[W - 1];
+    if (tid < 2 * W) edge_id[tid] = -1;
     __syncthreads();
   }
   const long long P = static_cast<long long>(cum[a.B]) * a.H_kv;
@@ -160,157 +191,37 @@ __global__ void __launch_bounds__(32 * W, 1)
     }
   }
 
-  // ---- 3. this warp's partition of the page list
-  const int w = blockIdx.x * W + warp;
-  if (w >= N) return;
-  const long long p0 = part_begin(w, P, N), p1 = part_begin(w + 1, P, N);
-  if (p0 >= p1) return;
-
-  const uint32_t stage0 = smem_u32(stages + (size_t)warp * S * Gm::kStageBytes);
-  const uint32_t bar0 = smem_u32(bars + warp * S);
-  int2 *meta_w = meta + warp * S;
-  const uint64_t policy = a.evict_first ? l2_policy_evict_first() : l2_policy_evict_normal();
-
-  if (lane == 0) {
-#pragma unroll
-    for (int s = 0; s < S; ++s) mbar_init(bar0 + 8 * s, 1);
-    mbar_init_fence();
-  }
-  __syncwarp();
-
-  // Fetch-side page descriptors, one fetch position per lane, in windows of
-  // 32 positions.  `nx*` is the next window, computed one window early so its
-  // block-table loads are long done when it is promoted.
+  // ---- 3. this CTA's partition, and this warp's contiguous share of it
+  const int cta = blockIdx.x;
+  if (cta >= N) return;  // the whole CTA: no block-level sync follows for it
+  const long long c0 = part_begin(cta, P, N), c1 = part_begin(cta + 1, P, N);
+  const long long p0 = c0 + ((c1 - c0) * warp) / W, p1 = c0 + ((c1 - c0) * (warp + 1)) / W;
   const int H = a.H_kv;
-  auto describe = [&](long long wb, int &pb, int &h, int &seg, int &ntok) {
-    pb = -1;
-    h = 0;
-    seg = -1;
-    ntok = 0;
-    const long long pos = wb + lane;
-    if (pos < p1) {
-      int lo = 0, hi = a.B;  // largest b with cum[b] * H <= pos
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (static_cast<long long>(cum[mid]) * H <= pos) lo = mid; else hi = mid;
-      }
-      const int b = lo;
-      const int np = cum[b + 1] - cum[b];
-      const long long off = pos - static_cast<long long>(cum[b]) * H;
-      h = static_cast<int>(off / np);
-      const int i = static_cast<int>(off - static_cast<long long>(h) * np);
-      pb = __ldg(a.block_table + static_cast<size_t>(b) * a.maxb + i);
-      ntok = min(kPage, clamp_len(__ldg(a.seq_lens + b), cap) - i * kPage);
-      seg = b * H + h;
-    }
-  };
-  auto promote = [&](int pb, int h, int seg) -> int {
-    if (seg < 0) return -1;
-    if (pb < 0 || pb >= a.num_blocks) {
-      flag_error(a.err, kErrBlockTable);
-      return -1;
-    }
-    return (pb * H + h) * kPage;  // TMA row coordinate of this page's 16 rows
-  };
-
-  long long wb = p0;
-  int cur_row, cur_seg, cur_ntok;
-  int nx_pb, nx_h, nx_seg, nx_ntok;
-  {
-    int pb, h;
-    describe(wb, pb, h, cur_seg, cur_ntok);
-    cur_row = promote(pb, h, cur_seg);
-    describe(wb + 32, nx_pb, nx_h, nx_seg, nx_ntok);
-  }
-
-  long long f = p0;  // next page to fetch
-  int fst = 0;       // its stage
-  auto issue = [&]() {
-    int j = static_cast<int>(f - wb);
-    if (j >= 32) {
-      cur_row = promote(nx_pb, nx_h, nx_seg);
-      cur_seg = nx_seg;
-      cur_ntok = nx_ntok;
-      wb += 32;
-      describe(wb + 32, nx_pb, nx_h, nx_seg, nx_ntok);
-      j -= 32;
-    }
-    const int row = __shfl_sync(0xffffffffu, cur_row, j);
-    const int seg = __shfl_sync(0xffffffffu, cur_seg, j);
-    const int ntok = __shfl_sync(0xffffffffu, cur_ntok, j);
-    if (lane == 0) {
-      meta_w[fst] = make_int2(seg, row >= 0 ? ntok : 0);
-      const uint32_t bar = bar0 + 8 * fst;
-      if (row >= 0) {
-        const uint32_t dst = stage0 + fst * Gm::kStageBytes;
-        mbar_arrive_expect_tx(bar, Gm::kStageBytes);
-        tma_load_3d(dst, &tmK, 0, 0, row, bar, policy);
-        tma_load_3d(dst + Gm::kPageBytes, &tmV, 0, 0, row, bar, policy);
-      } else {
-        mbar_arrive(bar);
-      }
-    }
-    ++f;
-    if (++fst == S) fst = 0;
-  };
-
-#pragma unroll 1
-  for (int s = 0; s < S; ++s)
-    if (f < p1) issue();
-
-  // ---- per-lane fragment geometry
   const int g8 = lane >> 2, tig = lane & 3;
-  const int tK = (lane & 7) | (((lane >> 3) & 1) << 3);
-  const int cK = ((lane >> 4) & 1) << 3;
-  const int tV = (lane & 7) | (((lane >> 4) & 1) << 3);
-  const int cV = ((lane >> 3) & 1) << 3;
 
-  // ---- running state of the current (sequence, KV head) pair
+  // running state of the current (sequence, KV head) pair
   uint32_t qf[NT][Gm::kSteps][2];
   float acc[NT][Gm::kSteps][4];
   float m_run[NT][2], l_run[NT][2];
-  int cur = -1;  // pair being accumulated
 
-  auto begin_pair = [&](int seg) {
-    const int b = seg / H, h = seg - (seg / H) * H;
-    const uint32_t *qw = reinterpret_cast<const uint32_t *>(a.q) +
-                         (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G) * (D / 2);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int r = nt * 8 + g8;
-#pragma unroll
-      for (int ks = 0; ks < Gm::kSteps; ++ks) {
-        if (r < a.G) {
-          qf[nt][ks][0] = __ldg(qw + r * (D / 2) + ks * 8 + tig);
-          qf[nt][ks][1] = __ldg(qw + r * (D / 2) + ks * 8 + 4 + tig);
-        } else {
-          qf[nt][ks][0] = 0u;
-          qf[nt][ks][1] = 0u;
-        }
-      }
-#pragma unroll
-      for (int mt = 0; mt < Gm::kSteps; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
-      m_run[nt][0] = m_run[nt][1] = -INFINITY;
-      l_run[nt][0] = l_run[nt][1] = 0.f;
-    }
-  };
-
-  auto finish_pair = [&](int seg) {
+  auto pair_range = [&](int seg, long long &s0, long long &s1) {
     const int b = seg / H, h = seg - (seg / H) * H;
     const int np = cum[b + 1] - cum[b];
-    const long long s0 = static_cast<long long>(cum[b]) * H + static_cast<long long>(h) * np;
-    const bool whole = s0 >= p0 && s0 + np <= p1;
+    s0 = static_cast<long long>(cum[b]) * H + static_cast<long long>(h) * np;
+    s1 = s0 + np;
+  };
+
+  // Write a finished pair from register state (l_run already summed over the
+  // 8 token lanes): the final rows if `whole`, else a normalised partial
+  // (o, lse) at slot cta + seg for the cross-CTA merge.
+  auto emit = [&](int seg, bool whole) {
+    const int b = seg / H, h = seg - (seg / H) * H;
     const size_t row0 = static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        float l = l_run[nt][i];
-        l += __shfl_xor_sync(0xffffffffu, l, 4);
-        l += __shfl_xor_sync(0xffffffffu, l, 8);
-        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        const float l = l_run[nt][i];
         const int r = nt * 8 + 2 * tig + i;
         const float inv = l > 0.f ? 1.f / l : 0.f;
         const float lse = l > 0.f ? (m_run[nt][i] + fast_log2(l)) * kLn2 : -INFINITY;
@@ -324,7 +235,7 @@ __global__ void __launch_bounds__(32 * W, 1)
             }
             if (a.lse_out && g8 == 0) a.lse_out[row0 + r] = lse;
           } else {
-            const size_t slot = static_cast<size_t>(w) + seg;
+            const size_t slot = static_cast<size_t>(cta) + seg;
             float *o = a.part_o + (slot * a.G + r) * D;
 #pragma unroll
             for (int mt = 0; mt < Gm::kSteps; ++mt) {
@@ -338,131 +249,399 @@ __global__ void __launch_bounds__(32 * W, 1)
     }
   };
 
-  // ---- main loop over this partition's pages
-  const long long nmy = p1 - p0;
-  int cst = 0;
-  uint32_t cph = 0;
-  bool failed = false;
-  long long c = 0;
-#pragma unroll 1
-  for (; c < nmy; ++c) {
-    const uint32_t bar = bar0 + 8 * cst;
-    const bool ok = mbar_wait_bounded(bar, cph);
-    if (!__all_sync(0xffffffffu, ok)) {
-      if (lane == 0) flag_error(a.err, kErrTimeout);
-      failed = true;
-      break;
-    }
-    const int2 md = meta_w[cst];
-    if (md.x != cur) {
-      if (cur >= 0) finish_pair(cur);
-      cur = md.x;
-      begin_pair(cur);
-    }
-    const int ntok = md.y;
-    if (ntok > 0) {
-      uint8_t *kp = stages + ((size_t)warp * S + cst) * Gm::kStageBytes;
-      uint8_t *vp = kp + Gm::kPageBytes;
-      if (ntok < kPage) {
-        // rows past the sequence end may hold anything (even NaN): clear V's
-        // so the zero weights of masked tokens cannot turn into NaN
-        uint4 *z = reinterpret_cast<uint4 *>(vp + ntok * D * 2);
-        const int n16 = (kPage - ntok) * D * 2 / 16;
-        for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
-        fence_proxy_async_smem();
-        __syncwarp();
+  auto sum_l = [&]() {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        float l = l_run[nt][i];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        l_run[nt][i] = l;
       }
-      const uint32_t kb = smem_u32(kp), vb = smem_u32(vp);
+  };
 
-      // S^T = K Q^T, two independent accumulator chains over d
-      float s[NT][4], s2[NT][4];
+  // Park a pair this warp holds only a piece of: unnormalised accumulators
+  // (lane-major, conflict-free) plus per-row max and sum, for the combine step.
+  auto park = [&](int seg, int which, float *dst) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int mt = 0; mt < Gm::kSteps; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[((nt * Gm::kSteps + mt) * 4 + e) * 32 + lane] = acc[nt][mt][e];
+    float *ml = edge_ml + (warp * 2 + which) * 2 * kRows;
+    if (g8 == 0) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
+        for (int i = 0; i < 2; ++i) {
+          ml[nt * 8 + 2 * tig + i] = m_run[nt][i];
+          ml[kRows + nt * 8 + 2 * tig + i] = l_run[nt][i];
+        }
+    }
+    if (lane == 0) edge_id[warp * 2 + which] = seg;
+  };
+
+  auto finish_pair = [&](int seg, bool last) {
+    sum_l();
+    long long s0, s1;
+    pair_range(seg, s0, s1);
+    if (s0 >= p0 && s1 <= p1) {
+      emit(seg, true);          // entirely inside this warp's share
+    } else if (s0 < p0) {
+      park(seg, 0, edge_acc + (size_t)warp * Gm::kEdgeFloats);  // continues from an earlier warp
+    } else {
+      // continues into a later warp; this is the warp's last pair, so its
+      // ring is idle and stage 0 holds the parked state
+      park(seg, 1, reinterpret_cast<float *>(stages + (size_t)warp * S * Gm::kStageBytes));
+    }
+    (void)last;
+  };
+
+  bool failed = false;
+  if (p0 < p1) {
+    const uint32_t stage0 = smem_u32(stages + (size_t)warp * S * Gm::kStageBytes);
+    const uint32_t bar0 = smem_u32(bars + warp * S);
+    int2 *meta_w = meta + warp * S;
+    const uint64_t policy = a.evict_first ? l2_policy_evict_first() : l2_policy_evict_normal();
+
+    if (lane == 0) {
 #pragma unroll
-      for (int ks = 0; ks < Gm::kSteps; ++ks) {
-        uint32_t fa[4];
-        ldmatrix_x4(fa, kb + swz<D>(tK, ks * 16 + cK));
+      for (int s = 0; s < S; ++s) mbar_init(bar0 + 8 * s, 1);
+      mbar_init_fence();
+    }
+    __syncwarp();
+
+    // Fetch-side page descriptors, one fetch position per lane, in windows of
+    // 32 positions.  `nx*` is the next window, computed one window early so
+    // its block-table loads are long done when it is promoted.
+    auto describe = [&](long long wb, int &pb, int &h, int &seg, int &ntok) {
+      pb = -1;
+      h = 0;
+      seg = -1;
+      ntok = 0;
+      const long long pos = wb + lane;
+      if (pos < p1) {
+        int lo = 0, hi = a.B;  // largest b with cum[b] * H <= pos
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (static_cast<long long>(cum[mid]) * H <= pos) lo = mid; else hi = mid;
+        }
+        const int b = lo;
+        const int np = cum[b + 1] - cum[b];
+        const long long off = pos - static_cast<long long>(cum[b]) * H;
+        h = static_cast<int>(off / np);
+        const int i = static_cast<int>(off - static_cast<long long>(h) * np);
+        pb = __ldg(a.block_table + static_cast<size_t>(b) * a.maxb + i);
+        ntok = min(kPage, clamp_len(__ldg(a.seq_lens + b), cap) - i * kPage);
+        seg = b * H + h;
+      }
+    };
+    auto promote = [&](int pb, int h, int seg) -> int {
+      if (seg < 0) return -1;
+      if (pb < 0 || pb >= a.num_blocks) {
+        flag_error(a.err, kErrBlockTable);
+        return -1;
+      }
+      return (pb * H + h) * kPage;  // TMA row coordinate of this page's 16 rows
+    };
+
+    long long wb = p0;
+    int cur_row, cur_seg, cur_ntok;
+    int nx_pb, nx_h, nx_seg, nx_ntok;
+    {
+      int pb, h;
+      describe(wb, pb, h, cur_seg, cur_ntok);
+      cur_row = promote(pb, h, cur_seg);
+      describe(wb + 32, nx_pb, nx_h, nx_seg, nx_ntok);
+    }
+
+    long long f = p0;  // next page to fetch
+    int fst = 0;       // its stage
+    auto issue = [&]() {
+      int j = static_cast<int>(f - wb);
+      if (j >= 32) {
+        cur_row = promote(nx_pb, nx_h, nx_seg);
+        cur_seg = nx_seg;
+        cur_ntok = nx_ntok;
+        wb += 32;
+        describe(wb + 32, nx_pb, nx_h, nx_seg, nx_ntok);
+        j -= 32;
+      }
+      const int row = __shfl_sync(0xffffffffu, cur_row, j);
+      const int seg = __shfl_sync(0xffffffffu, cur_seg, j);
+      const int ntok = __shfl_sync(0xffffffffu, cur_ntok, j);
+      if (lane == 0) {
+        meta_w[fst] = make_int2(seg, row >= 0 ? ntok : 0);
+        const uint32_t bar = bar0 + 8 * fst;
+        if (row >= 0) {
+          const uint32_t dst = stage0 + fst * Gm::kStageBytes;
+          mbar_arrive_expect_tx(bar, Gm::kStageBytes);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          if (ks & 1) M::run(s2[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
-          else M::run(s[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
+          for (int hf = 0; hf < D / 64; ++hf) {
+            tma_load_3d(dst + hf * kPage * 128, &tmK, 0, hf, row, bar, policy);
+            tma_load_3d(dst + Gm::kPageBytes + hf * kPage * 128, &tmV, 0, hf, row, bar, policy);
+          }
+        } else {
+          mbar_arrive(bar);
         }
       }
+      ++f;
+      if (++fst == S) fst = 0;
+    };
 
-      // online softmax update (base 2), probabilities rounded to T
-      const bool v0 = g8 < ntok, v1 = g8 + 8 < ntok;
-      uint32_t pb0[NT], pb1[NT];
-      float alpha[NT][2];
-      bool rescale = false;
+#pragma unroll 1
+    for (int s = 0; s < S; ++s)
+      if (f < p1) issue();
+
+    // ---- per-lane fragment geometry
+    const int tK = (lane & 7) | (((lane >> 3) & 1) << 3);
+    const int cK = ((lane >> 4) & 1) << 3;
+    const int tV = (lane & 7) | (((lane >> 4) & 1) << 3);
+    const int cV = ((lane >> 3) & 1) << 3;
+
+    int cur = -1;  // pair being accumulated
+
+    auto begin_pair = [&](int seg) {
+      const int b = seg / H, h = seg - (seg / H) * H;
+      const uint32_t *qw = reinterpret_cast<const uint32_t *>(a.q) +
+                           (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G) * (D / 2);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const float x0 = v0 ? (s[nt][0] + s2[nt][0]) * a.scale_log2 : -INFINITY;
-        const float x1 = v0 ? (s[nt][1] + s2[nt][1]) * a.scale_log2 : -INFINITY;
-        const float x2 = v1 ? (s[nt][2] + s2[nt][2]) * a.scale_log2 : -INFINITY;
-        const float x3 = v1 ? (s[nt][3] + s2[nt][3]) * a.scale_log2 : -INFINITY;
-        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+        const int r = nt * 8 + g8;
 #pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        for (int ks = 0; ks < Gm::kSteps; ++ks) {
+          if (r < a.G) {
+            qf[nt][ks][0] = __ldg(qw + r * (D / 2) + ks * 8 + tig);
+            qf[nt][ks][1] = __ldg(qw + r * (D / 2) + ks * 8 + 4 + tig);
+          } else {
+            qf[nt][ks][0] = 0u;
+            qf[nt][ks][1] = 0u;
+          }
         }
-        const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-        alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
-        alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
-        rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
-        m_run[nt][0] = mn0;
-        m_run[nt][1] = mn1;
-        const uint32_t lo = M::pack(fast_exp2(x0 - mn0), fast_exp2(x1 - mn1));
-        const uint32_t hi = M::pack(fast_exp2(x2 - mn0), fast_exp2(x3 - mn1));
-        const float2 fl = M::unpack(lo), fh = M::unpack(hi);
-        l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (fl.x + fh.x);
-        l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (fl.y + fh.y);
-        pb0[nt] = movmatrix_trans(lo);
-        pb1[nt] = movmatrix_trans(hi);
+#pragma unroll
+        for (int mt = 0; mt < Gm::kSteps; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
+        m_run[nt][0] = m_run[nt][1] = -INFINITY;
+        l_run[nt][0] = l_run[nt][1] = 0.f;
       }
-      if (__any_sync(0xffffffffu, rescale)) {
+    };
+
+    // ---- main loop over this warp's pages
+    const long long nmy = p1 - p0;
+    int cst = 0;
+    uint32_t cph = 0;
+    long long c = 0;
+#pragma unroll 1
+    for (; c < nmy; ++c) {
+      const uint32_t bar = bar0 + 8 * cst;
+      const bool ok = mbar_wait_bounded(bar, cph);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) flag_error(a.err, kErrTimeout);
+        failed = true;
+        break;
+      }
+      const int2 md = meta_w[cst];
+      if (md.x != cur) {
+        if (cur >= 0) finish_pair(cur, false);
+        cur = md.x;
+        begin_pair(cur);
+      }
+      const int ntok = md.y;
+      if (ntok > 0) {
+        uint8_t *kp = stages + ((size_t)warp * S + cst) * Gm::kStageBytes;
+        uint8_t *vp = kp + Gm::kPageBytes;
+        if (ntok < kPage) {
+          // rows past the sequence end may hold anything (even NaN): clear V's
+          // so the zero weights of masked tokens cannot turn into NaN
+          const int n16 = (kPage - ntok) * 128 / 16;  // 16-byte chunks per half
+#pragma unroll
+          for (int hf = 0; hf < D / 64; ++hf) {
+            uint4 *z = reinterpret_cast<uint4 *>(vp + hf * kPage * 128 + ntok * 128);
+            for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        const uint32_t kb = smem_u32(kp), vb = smem_u32(vp);
+
+        // S^T = K Q^T, two independent accumulator chains over d
+        float s[NT][4], s2[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int mt = 0; mt < Gm::kSteps; ++mt) {
-            acc[nt][mt][0] *= alpha[nt][0];
-            acc[nt][mt][1] *= alpha[nt][1];
-            acc[nt][mt][2] *= alpha[nt][0];
-            acc[nt][mt][3] *= alpha[nt][1];
+          for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < Gm::kSteps; ++ks) {
+          uint32_t fa[4];
+          ldmatrix_x4(fa, kb + swz<D>(tK, ks * 16 + cK));
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            if (ks & 1) M::run(s2[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
+            else M::run(s[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
           }
-      }
+        }
 
-      // O^T += V^T P^T
+        // online softmax update (base 2), probabilities rounded to T (bf16:
+        // split into a rounded head and a rounded remainder, see kSplitP)
+        const bool v0 = g8 < ntok, v1 = g8 + 8 < ntok;
+        uint32_t pb0[NT], pb1[NT], pc0[NT], pc1[NT];
+        float alpha[NT][2];
+        bool rescale = false;
 #pragma unroll
-      for (int mt = 0; mt < Gm::kSteps; ++mt) {
-        uint32_t fa[4];
-        ldmatrix_x4_trans(fa, vb + swz<D>(tV, mt * 16 + cV));
+        for (int nt = 0; nt < NT; ++nt) {
+          const float x0 = v0 ? (s[nt][0] + s2[nt][0]) * a.scale_log2 : -INFINITY;
+          const float x1 = v0 ? (s[nt][1] + s2[nt][1]) * a.scale_log2 : -INFINITY;
+          const float x2 = v1 ? (s[nt][2] + s2[nt][2]) * a.scale_log2 : -INFINITY;
+          const float x3 = v1 ? (s[nt][3] + s2[nt][3]) * a.scale_log2 : -INFINITY;
+          float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) M::run(acc[nt][mt], fa, pb0[nt], pb1[nt]);
-      }
-    }
-    __syncwarp();
-    if (f < p1) issue();
-    if (++cst == S) {
-      cst = 0;
-      cph ^= 1u;
-    }
-  }
+          for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+          }
+          const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+          alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
+          alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
+          rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
+          m_run[nt][0] = mn0;
+          m_run[nt][1] = mn1;
+          const float e0 = fast_exp2(x0 - mn0), e1 = fast_exp2(x1 - mn1);
+          const float e2 = fast_exp2(x2 - mn0), e3 = fast_exp2(x3 - mn1);
+          const uint32_t lo = M::pack(e0, e1), hi = M::pack(e2, e3);
+          const float2 fl = M::unpack(lo), fh = M::unpack(hi);
+          if constexpr (kSplitP) {
+            // p = head + remainder, both bf16: ~16 significant bits in the PV
+            // product; the running sum uses the unrounded p to match
+            const uint32_t lo2 = M::pack(e0 - fl.x, e1 - fl.y);
+            const uint32_t hi2 = M::pack(e2 - fh.x, e3 - fh.y);
+            l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (e0 + e2);
+            l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (e1 + e3);
+            pc0[nt] = movmatrix_trans(lo2);
+            pc1[nt] = movmatrix_trans(hi2);
+          } else {
+            // the running sum uses the same rounded p as the PV product, so
+            // the output is an exact weighted mean of V up to fp32 sums
+            l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (fl.x + fh.x);
+            l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (fl.y + fh.y);
+            pc0[nt] = pc1[nt] = 0u;
+          }
+          pb0[nt] = movmatrix_trans(lo);
+          pb1[nt] = movmatrix_trans(hi);
+        }
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int mt = 0; mt < Gm::kSteps; ++mt) {
+              acc[nt][mt][0] *= alpha[nt][0];
+              acc[nt][mt][1] *= alpha[nt][1];
+              acc[nt][mt][2] *= alpha[nt][0];
+              acc[nt][mt][3] *= alpha[nt][1];
+            }
+        }
 
-  if (failed) {
-    // let every copy still in flight land before the CTA's shared memory goes away
-    for (; c < f - p0; ++c) {
-      mbar_wait_bounded(bar0 + 8 * cst, cph);
+        // O^T += V^T P^T
+#pragma unroll
+        for (int mt = 0; mt < Gm::kSteps; ++mt) {
+          uint32_t fa[4];
+          ldmatrix_x4_trans(fa, vb + swz<D>(tV, mt * 16 + cV));
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            M::run(acc[nt][mt], fa, pb0[nt], pb1[nt]);
+            if constexpr (kSplitP) M::run(acc[nt][mt], fa, pc0[nt], pc1[nt]);
+          }
+        }
+      }
+      __syncwarp();
+      if (f < p1) issue();
       if (++cst == S) {
         cst = 0;
         cph ^= 1u;
       }
     }
-    return;
+
+    if (failed) {
+      // let every copy still in flight land before shared memory is reused or freed
+      for (; c < f - p0; ++c) {
+        mbar_wait_bounded(bar0 + 8 * cst, cph);
+        if (++cst == S) {
+          cst = 0;
+          cph ^= 1u;
+        }
+      }
+    } else if (cur >= 0) {
+      __syncwarp();
+      finish_pair(cur, true);
+    }
   }
-  if (cur >= 0) finish_pair(cur);
+
+  // ---- 4. combine the pieces of pairs that several warps of this CTA hold
+  __syncthreads();
+  if (failed) return;
+#pragma unroll 1
+  for (int which = 0; which < 2; ++which) {
+    const int seg = edge_id[warp * 2 + which];
+    if (seg < 0) continue;
+    bool owner = true;  // lowest warp holding a piece of seg
+    for (int w2 = 0; w2 < warp; ++w2)
+      if (edge_id[w2 * 2] == seg || edge_id[w2 * 2 + 1] == seg) owner = false;
+    if (!owner) continue;
+    // gather: new maximum per row, then rescaled sums of l and accumulators
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        m_run[nt][i] = -INFINITY;
+        l_run[nt][i] = 0.f;
+      }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int mt = 0; mt < Gm::kSteps; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
+    for (int w2 = warp; w2 < W; ++w2)
+      for (int k = 0; k < 2; ++k)
+        if (edge_id[w2 * 2 + k] == seg) {
+          const float *ml = edge_ml + (w2 * 2 + k) * 2 * kRows;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) m_run[nt][i] = fmaxf(m_run[nt][i], ml[nt * 8 + 2 * tig + i]);
+        }
+    for (int w2 = warp; w2 < W; ++w2)
+      for (int k = 0; k < 2; ++k)
+        if (edge_id[w2 * 2 + k] == seg) {
+          const float *ml = edge_ml + (w2 * 2 + k) * 2 * kRows;
+          const float *src = k == 0 ? edge_acc + (size_t)w2 * Gm::kEdgeFloats
+                                    : reinterpret_cast<const float *>(
+                                          stages + (size_t)w2 * S * Gm::kStageBytes);
+          float sc[NT][2];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int r = nt * 8 + 2 * tig + i;
+              const float mi = ml[r];
+              sc[nt][i] = mi == -INFINITY ? 0.f : fast_exp2(mi - m_run[nt][i]);
+              l_run[nt][i] += ml[kRows + r] * sc[nt][i];
+            }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int mt = 0; mt < Gm::kSteps; ++mt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                acc[nt][mt][e] += src[((nt * Gm::kSteps + mt) * 4 + e) * 32 + lane] * sc[nt][e & 1];
+        }
+    long long s0, s1;
+    pair_range(seg, s0, s1);
+    emit(seg, s0 >= c0 && s1 <= c1);
+  }
 }
 
 // ------------------------------------------------------------------ merge
@@ -575,30 +754,64 @@ __global__ void __launch_bounds__(256) generic_merge_kernel(const GenericMergeAr
 
 namespace {
 
-template <int D>
+// Worker warps per CTA (one CTA per SM) and ring stages per warp, per head
+// dim D and n-tiles NT (G <= 8: 1, G <= 16: 2).  Shared memory per warp is
+// S * 64 * D bytes of ring plus one parked accumulator tile.  Defaults can
+// be overridden at build time (-DKVD_TUNE_W128_1=... etc.).
+#ifndef KVD_TUNE_W128_1
+#define KVD_TUNE_W128_1 16
+#endif
+#ifndef KVD_TUNE_S128_1
+#define KVD_TUNE_S128_1 1
+#endif
+#ifndef KVD_TUNE_W128_2
+#define KVD_TUNE_W128_2 12
+#endif
+#ifndef KVD_TUNE_S128_2
+#define KVD_TUNE_S128_2 1
+#endif
+#ifndef KVD_TUNE_W64_1
+#define KVD_TUNE_W64_1 16
+#endif
+#ifndef KVD_TUNE_S64_1
+#define KVD_TUNE_S64_1 2
+#endif
+#ifndef KVD_TUNE_W64_2
+#define KVD_TUNE_W64_2 12
+#endif
+#ifndef KVD_TUNE_S64_2
+#define KVD_TUNE_S64_2 2
+#endif
+
+template <int D, int NT>
 struct Tune;
-// d = 128: 8 KB per stage; 4 worker warps x 6 stages = 192 KB of ring per SM.
 template <>
-struct Tune<128> {
-  static constexpr int W = 4, S = 6;
+struct Tune<128, 1> {
+  static constexpr int W = KVD_TUNE_W128_1, S = KVD_TUNE_S128_1;
 };
-// d = 64: 4 KB per stage; 4 x 10 stages.
 template <>
-struct Tune<64> {
-  static constexpr int W = 4, S = 10;
+struct Tune<128, 2> {
+  static constexpr int W = KVD_TUNE_W128_2, S = KVD_TUNE_S128_2;
+};
+template <>
+struct Tune<64, 1> {
+  static constexpr int W = KVD_TUNE_W64_1, S = KVD_TUNE_S64_1;
+};
+template <>
+struct Tune<64, 2> {
+  static constexpr int W = KVD_TUNE_W64_2, S = KVD_TUNE_S64_2;
 };
 
 template <int D, int NT, typename T>
 cudaError_t launch_decode_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                             cudaStream_t st, int grid) {
-  constexpr int W = Tune<D>::W, S = Tune<D>::S;
+  constexpr int W = Tune<D, NT>::W, S = Tune<D, NT>::S;
   auto kern = decode_kernel<D, NT, T, W, S>;
-  const size_t smem = Geo<D, W, S>::smem(a.B);
+  const size_t smem = Geo<D, NT, W, S>::smem(a.B);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, 32 * W, smem, st>>>(a, tmK, tmV);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(32 * W), smem, st, a, tmK, tmV);
 }
 
 template <typename T>
@@ -615,9 +828,8 @@ cudaError_t launch_decode_dt(const DecodeArgs &a, int d, const CUtensorMap &tmK,
 template <typename T>
 cudaError_t launch_merge_dt(const DecodeArgs &a, int d, cudaStream_t st) {
   dim3 grid(a.B * a.H_kv, a.G);
-  if (d == 128) decode_merge_kernel<128, T><<<grid, 256, 0, st>>>(a);
-  else decode_merge_kernel<64, T><<<grid, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  if (d == 128) return launch_pdl(decode_merge_kernel<128, T>, grid, dim3(256), 0, st, a);
+  return launch_pdl(decode_merge_kernel<64, T>, grid, dim3(256), 0, st, a);
 }
 
 template <typename T>
@@ -630,14 +842,7 @@ cudaError_t launch_generic_dt(const GenericMergeArgs &a, cudaStream_t st) {
 
 }  // namespace
 
-int decode_warps_per_cta(int d) { return d == 128 ? Tune<128>::W : Tune<64>::W; }
-
-size_t decode_smem_bytes(int d, int B) {
-  return d == 128 ? Geo<128, Tune<128>::W, Tune<128>::S>::smem(B)
-                  : Geo<64, Tune<64>::W, Tune<64>::S>::smem(B);
-}
-
-int decode_auto_parts(int d, int sms) { return sms * decode_warps_per_cta(d); }
+int decode_auto_parts(int sms) { return sms; }
 
 cudaError_t launch_decode(const DecodeArgs &a, int d, DType dt, const CUtensorMap &tmK,
                           const CUtensorMap &tmV, cudaStream_t s, int grid) {

@@ -33,7 +33,7 @@ struct DecodeArgs {
   unsigned *err;
   float scale_log2;   // scale * log2(e)
   int B, H_q, H_kv, G, num_blocks, maxb;
-  int nparts;         // N: partitions of the concatenated page list
+  int nparts;         // N: partitions (CTAs) of the concatenated page list
   int min_pages;      // lower bound on average pages per used partition
   int evict_first;    // 1: stream K/V with an L2 evict-first hint
 };
@@ -47,17 +47,9 @@ struct GenericMergeArgs {
   int B, H_q, d, S;
 };
 
-// Decode-kernel launch geometry for head dim d (warps per CTA, ring stages).
-struct DecodeGeometry {
-  int warps;
-  int stages;
-  size_t smem_bytes;  // dynamic shared memory for batch B (see decode_smem_bytes)
-};
-
-int decode_warps_per_cta(int d);
-size_t decode_smem_bytes(int d, int B);
-// Partitions = resident worker warps of a device with `sms` SMs.
-int decode_auto_parts(int d, int sms);
+// Partitions used when the caller asks for the automatic count: one CTA per
+// SM of a device with `sms` SMs (each CTA runs 12-16 worker warps).
+int decode_auto_parts(int sms);
 
 // Set the text returned by kvd_last_error on this host thread.
 void record_error(const char *msg);
