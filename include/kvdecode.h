@@ -124,6 +124,28 @@ kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *
                                 void *workspace, size_t workspace_bytes,
                                 float *lse_out, kvd_dtype dtype, void *stream);
 
+/*
+ * kvd_decode_step -- one whole decode step in one launch: the append of
+ * kvd_append followed by the attention of kvd_decode_attention.
+ * [KVF] section "一、KV Cache" (the step appends the new token's K/V, then the
+ * new query attends over the whole cache including it); [BLOG] "缓存的是什么".
+ *
+ *   k_new, v_new   device, [B][H_kv][d]: the step's new keys and values
+ *   k_cache, v_cache written in place
+ *   other arguments as kvd_decode_attention
+ * Every sequence b with seq_lens[b] >= 1 appends its new token at position
+ * seq_lens[b] - 1 (row (n-1) % 16 of page block_table[b][(n-1) / 16]); a
+ * sequence with seq_lens[b] = 0 appends nothing.  The result -- the cache
+ * and out -- is bit-identical to kvd_append (slot = seq_lens - 1) followed
+ * by kvd_decode_attention with the same num_partitions.  The page that
+ * receives the new token must not be shared with another sequence.
+ */
+kvd_status kvd_decode_step(const void *q, const void *k_new, const void *v_new, void *k_cache,
+                           void *v_cache, const int32_t *block_table, const int32_t *seq_lens,
+                           float scale, void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                           int max_blocks_per_seq, int num_partitions, void *workspace,
+                           size_t workspace_bytes, float *lse_out, kvd_dtype dtype, void *stream);
+
 /* Bytes of the library's fixed scratch array used by kvd_decode_attention_static. */
 #define KVD_STATIC_WORKSPACE_BYTES (8u << 20)
 

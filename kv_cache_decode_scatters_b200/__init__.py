@@ -20,7 +20,8 @@ import torch
 __all__ = [
     "KVD_OK", "KVD_ERR_INVALID", "KVD_ERR_UNSUPPORTED", "KVD_ERR_CUDA", "KVD_ERR_WORKSPACE",
     "KVD_F16", "KVD_BF16", "KVD_PAGE_TOKENS", "KvdError",
-    "kvd_append", "kvd_decode_attention", "kvd_decode_attention_static", "kvd_merge_lse",
+    "kvd_append", "kvd_decode_attention", "kvd_decode_step", "kvd_decode_attention_static",
+    "kvd_merge_lse",
     "kvd_workspace_size", "KVD_STATIC_WORKSPACE_BYTES",
     "kvd_auto_partitions", "kvd_kv_bytes_per_token", "kvd_read_device_error",
     "kvd_last_error", "alloc_workspace", "library_path", "lib",
@@ -50,6 +51,8 @@ def _load():
     L.kvd_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P]
     L.kvd_decode_attention.restype = I
     L.kvd_decode_attention.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, I, P, S, P, I, P]
+    L.kvd_decode_step.restype = I
+    L.kvd_decode_step.argtypes = [P, P, P, P, P, P, P, F, P, I, I, I, I, I, I, I, P, S, P, I, P]
     L.kvd_decode_attention_static.restype = I
     L.kvd_decode_attention_static.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, P, I, P]
     L.kvd_merge_lse.restype = I
@@ -181,6 +184,36 @@ def kvd_decode_attention(q, k_cache, v_cache, block_table, seq_lens, scale=None,
         int(num_partitions), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         lse_ptr, _dtype_code(k_cache), _stream(stream)),
         "kvd_decode_attention")
+    return out
+
+
+def kvd_decode_step(q, k_new, v_new, k_cache, v_cache, block_table, seq_lens, scale=None,
+                    out=None, num_partitions=0, workspace=None, lse_out=None, stream=None):
+    """Append k_new/v_new [B,H_kv,d] at position seq_lens[b]-1 of every
+    non-empty sequence, then attend (kvd_append + kvd_decode_attention in one
+    launch).  Returns out."""
+    B, H_q, d = q.shape
+    NB, H_kv, P, d2 = k_cache.shape
+    if P != KVD_PAGE_TOKENS or d2 != d:
+        raise ValueError("q / cache shape mismatch")
+    if tuple(k_new.shape) != (B, H_kv, d) or v_new.shape != k_new.shape:
+        raise ValueError("k_new / v_new must be [B, H_kv, d]")
+    dt = k_cache.dtype
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(B, H_q, H_kv, d, num_partitions, q.device)
+    lse_ptr = None if lse_out is None else _dev(lse_out, "lse_out", torch.float32)
+    _check(_lib.kvd_decode_step(
+        _dev(q, "q", dt), _dev(k_new, "k_new", dt), _dev(v_new, "v_new", dt),
+        _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
+        float(scale), _dev(out, "out", dt), B, H_q, H_kv, d, NB, block_table.shape[1],
+        int(num_partitions), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        lse_ptr, _dtype_code(k_cache), _stream(stream)),
+        "kvd_decode_step")
     return out
 
 

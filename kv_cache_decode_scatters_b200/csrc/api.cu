@@ -215,12 +215,14 @@ kvd_status kvd_append(void *k_cache, void *v_cache, const int32_t *block_table,
   return KVD_OK;
 }
 
-kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *v_cache,
-                                const int32_t *block_table, const int32_t *seq_lens, float scale,
-                                void *out, int B, int H_q, int H_kv, int d, int num_blocks,
-                                int max_blocks_per_seq, int num_partitions, void *workspace,
-                                size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
-                                void *stream) {
+}  // extern "C"
+
+static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *block_table, const int32_t *seq_lens, float scale,
+                              void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                              int max_blocks_per_seq, int num_partitions, void *workspace,
+                              size_t workspace_bytes, float *lse_out, kvd_dtype dtype, void *stream,
+                              const void *k_new, const void *v_new) {
   kvd_status st = check_heads(B, H_q, H_kv, d);
   if (st) return st;
   if (num_blocks <= 0 || max_blocks_per_seq <= 0)
@@ -301,6 +303,10 @@ kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *
   a.nparts = N;
   a.min_pages = num_partitions > 0 ? 1 : kAutoMinPages;
   a.evict_first = 0;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.k_cache = const_cast<void *>(k_cache);
+  a.v_cache = const_cast<void *>(v_cache);
 
   const kvd::DType dt = dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -309,6 +315,34 @@ kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *
   e = kvd::launch_decode_merge(a, d, dt, s);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return KVD_OK;
+}
+
+extern "C" {
+
+kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *block_table, const int32_t *seq_lens, float scale,
+                                void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                                int max_blocks_per_seq, int num_partitions, void *workspace,
+                                size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+                                void *stream) {
+  return decode_impl(q, k_cache, v_cache, block_table, seq_lens, scale, out, B, H_q, H_kv, d,
+                     num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
+                     lse_out, dtype, stream, nullptr, nullptr);
+}
+
+kvd_status kvd_decode_step(const void *q, const void *k_new, const void *v_new, void *k_cache,
+                           void *v_cache, const int32_t *block_table, const int32_t *seq_lens,
+                           float scale, void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                           int max_blocks_per_seq, int num_partitions, void *workspace,
+                           size_t workspace_bytes, float *lse_out, kvd_dtype dtype, void *stream) {
+  if (B > 0) {
+    if (!k_new || !v_new) return fail(KVD_ERR_INVALID, "k_new / v_new is NULL");
+    if (!aligned(k_new, 16) || !aligned(v_new, 16))
+      return fail(KVD_ERR_INVALID, "k_new / v_new must be 16-byte aligned");
+  }
+  return decode_impl(q, k_cache, v_cache, block_table, seq_lens, scale, out, B, H_q, H_kv, d,
+                     num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
+                     lse_out, dtype, stream, k_new, v_new);
 }
 
 kvd_status kvd_merge_lse(const float *part_o, const float *part_lse,

@@ -61,7 +61,7 @@ struct Geo {
   static constexpr int kEdgeFloats = 8 * NT * D;        // one parked accumulator tile
   static_assert(kEdgeFloats * 4 <= kStageBytes, "a parked tile must fit in one stage");
   static size_t smem(int B) {
-    return 1024 + (size_t)W * S * kStageBytes + (size_t)W * kEdgeFloats * 4 + (size_t)W * S * 16 +
+    return 1024 + (size_t)W * S * kStageBytes + (size_t)W * kEdgeFloats * 4 + (size_t)W * S * 24 +
            (size_t)W * 2 * 2 * 8 * NT * 4 + (size_t)W * 2 * 4 + (size_t)(B + 1) * 4;
   }
 };
@@ -114,6 +114,8 @@ __global__ void __launch_bounds__(32 * W, 1)
   using Gm = Geo<D, NT, W, S>;
   using M = Mma<T>;
   constexpr int kRows = 8 * NT;  // query rows per tile (G padded)
+  constexpr int kPatch = 32;     // page-meta flag: fused append writes a row of this page
+  const bool fused = a.k_new != nullptr;
   // bf16 keeps only 8 significant bits of each probability; carrying the
   // rounding remainder in a second PV product restores ~16 bits for the cost
   // of d/16 extra MMAs per page (free while the kernel waits on HBM).
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(32 * W, 1)
   uint8_t *stages = smem;
   float *edge_acc = reinterpret_cast<float *>(smem + (size_t)W * S * Gm::kStageBytes);
   uint64_t *bars = reinterpret_cast<uint64_t *>(edge_acc + (size_t)W * Gm::kEdgeFloats);
-  int2 *meta = reinterpret_cast<int2 *>(bars + W * S);
+  int4 *meta = reinterpret_cast<int4 *>(bars + W * S);
   float *edge_ml = reinterpret_cast<float *>(meta + W * S);  // [W][2][2][kRows]: m, l
   int *edge_id = reinterpret_cast<int *>(edge_ml + W * 2 * 2 * kRows);  // [W][2]
   int *cum = edge_id + 2 * W;
@@ -304,7 +306,7 @@ __global__ void __launch_bounds__(32 * W, 1)
   if (p0 < p1) {
     const uint32_t stage0 = smem_u32(stages + (size_t)warp * S * Gm::kStageBytes);
     const uint32_t bar0 = smem_u32(bars + warp * S);
-    int2 *meta_w = meta + warp * S;
+    int4 *meta_w = meta + warp * S;
     const uint64_t policy = a.evict_first ? l2_policy_evict_first() : l2_policy_evict_normal();
 
     if (lane == 0) {
@@ -336,6 +338,8 @@ __global__ void __launch_bounds__(32 * W, 1)
         const int i = static_cast<int>(off - static_cast<long long>(h) * np);
         pb = __ldg(a.block_table + static_cast<size_t>(b) * a.maxb + i);
         ntok = min(kPage, clamp_len(__ldg(a.seq_lens + b), cap) - i * kPage);
+        // fused append: the pair's last page holds the step's new token
+        if (fused && i == np - 1) ntok |= kPatch;
         seg = b * H + h;
       }
     };
@@ -374,7 +378,7 @@ __global__ void __launch_bounds__(32 * W, 1)
       const int seg = __shfl_sync(0xffffffffu, cur_seg, j);
       const int ntok = __shfl_sync(0xffffffffu, cur_ntok, j);
       if (lane == 0) {
-        meta_w[fst] = make_int2(seg, row >= 0 ? ntok : 0);
+        meta_w[fst] = make_int4(seg, row >= 0 ? ntok : 0, row, 0);
         const uint32_t bar = bar0 + 8 * fst;
         if (row >= 0) {
           const uint32_t dst = stage0 + fst * Gm::kStageBytes;
@@ -444,16 +448,34 @@ __global__ void __launch_bounds__(32 * W, 1)
         failed = true;
         break;
       }
-      const int2 md = meta_w[cst];
+      const int4 md = meta_w[cst];
       if (md.x != cur) {
         if (cur >= 0) finish_pair(cur, false);
         cur = md.x;
         begin_pair(cur);
       }
-      const int ntok = md.y;
+      const int ntok = md.y & (kPatch - 1);
       if (ntok > 0) {
         uint8_t *kp = stages + ((size_t)warp * S + cst) * Gm::kStageBytes;
         uint8_t *vp = kp + Gm::kPageBytes;
+        if (md.y & kPatch) {
+          // fused append: the new token is row ntok - 1 of this page.  Put
+          // k_new / v_new into the staged page (the copy just read may
+          // predate it) and write them to the cache -- no other CTA reads
+          // this row in this launch.
+          const int b = cur / H, h = cur - (cur / H) * H;
+          const int half = lane >> 4, ch = lane & 15;
+          if (ch < D / 8) {
+            const size_t src = (static_cast<size_t>(b) * H + h) * D;
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
+                                      static_cast<const uint16_t *>(half ? a.v_new : a.k_new) + src) + ch);
+            *reinterpret_cast<uint4 *>((half ? vp : kp) + swz<D>(ntok - 1, ch * 8)) = v;
+            const size_t dst = (static_cast<size_t>(md.z) + (ntok - 1)) * D;
+            *(reinterpret_cast<uint4 *>(static_cast<uint16_t *>(half ? a.v_cache : a.k_cache) + dst) + ch) = v;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
         if (ntok < kPage) {
           // rows past the sequence end may hold anything (even NaN): clear V's
           // so the zero weights of masked tokens cannot turn into NaN
@@ -646,76 +668,92 @@ __global__ void __launch_bounds__(32 * W, 1)
 
 // ------------------------------------------------------------------ merge
 
-// One CTA (256 threads) merges `count` partial results of one output row:
-// partial k has log-sum-exp lse[k * lse_stride] and normalised output
-// o[k * o_stride .. + D).  LSE = M + ln sum_k exp(lse_k - M);
-// out = sum_k exp(lse_k - LSE) o_k, one rounding to T.
+// One CTA (256 threads, 8 warps) merges `count` partial results of one
+// output row: partial k has log-sum-exp lse[k * lse_stride] and normalised
+// output o[k * o_stride .. + D).  Each warp folds its partials k = warp,
+// warp + 8, ... into a running (max, sum, output) state -- the rescale of
+// the online softmax applied to whole partials -- loading four partials'
+// lse and o at once; the 8 warp states are then combined in shared memory.
+// Result: LSE = M + ln sum_k exp(lse_k - M), out = sum_k exp(lse_k - LSE) o_k,
+// one rounding to T.  Partials with lse = -inf carry no weight (their o is
+// never read); if all are empty, out = 0 and LSE = -inf.
 template <int D, typename T>
 __device__ __forceinline__ void merge_row(const float *lse, long long lse_stride, const float *o,
                                           long long o_stride, int count, T *out, float *lse_out) {
   constexpr int kV = D / 32;
-  __shared__ float red[8];
-  __shared__ __align__(16) float part[8][D];
+  constexpr int kBatch = 4;
+  __shared__ float wm[8], wl[8];
+  __shared__ __align__(16) float wo[8][D];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  float mx = -INFINITY;
-  for (int k = tid; k < count; k += 256) mx = fmaxf(mx, lse[k * lse_stride]);
+  float m = -INFINITY, l = 0.f;
+  float acc[kV];
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
-  if (lane == 0) red[warp] = mx;
-  __syncthreads();
-  mx = red[0];
+  for (int e = 0; e < kV; ++e) acc[e] = 0.f;
+  for (int k0 = warp; k0 < count; k0 += 8 * kBatch) {
+    float lk[kBatch];
+    float ov[kBatch][kV];
 #pragma unroll
-  for (int i = 1; i < 8; ++i) mx = fmaxf(mx, red[i]);
+    for (int j = 0; j < kBatch; ++j) {
+      const int k = k0 + 8 * j;
+      lk[j] = k < count ? lse[k * lse_stride] * kLog2e : -INFINITY;
+      // o is loaded with lse (not after it) so both are in flight together;
+      // an empty partial's o is read but never used
+      if (k < count) {
+        const float *src = o + k * o_stride + lane * kV;
+        if constexpr (kV == 4) {
+          const float4 v = *reinterpret_cast<const float4 *>(src);
+          ov[j][0] = v.x;
+          ov[j][1] = v.y;
+          ov[j][2] = v.z;
+          ov[j][3] = v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2 *>(src);
+          ov[j][0] = v.x;
+          ov[j][1] = v.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      if (lk[j] == -INFINITY) continue;
+      const float mn = fmaxf(m, lk[j]);
+      const float a = fast_exp2(m - mn), b = fast_exp2(lk[j] - mn);
+#pragma unroll
+      for (int e = 0; e < kV; ++e) acc[e] = acc[e] * a + ov[j][e] * b;
+      l = l * a + b;
+      m = mn;
+    }
+  }
+  if (lane == 0) {
+    wm[warp] = m;
+    wl[warp] = l;
+  }
+#pragma unroll
+  for (int e = 0; e < kV; ++e) wo[warp][lane * kV + e] = acc[e];
   __syncthreads();
-  if (mx == -INFINITY) {
+  float M = wm[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) M = fmaxf(M, wm[i]);
+  if (M == -INFINITY) {
     for (int t = tid; t < D; t += 256) out[t] = Mma<T>::from_float(0.f);
     if (tid == 0 && lse_out) *lse_out = -INFINITY;
     return;
   }
-  const float mx2 = mx * kLog2e;
-  float sum = 0.f;
-  for (int k = tid; k < count; k += 256) sum += fast_exp2(lse[k * lse_stride] * kLog2e - mx2);
+  float sc[8], L = 0.f;
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, s);
-  if (lane == 0) red[warp] = sum;
-  __syncthreads();
-  sum = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) sum += red[i];
-  const float lse2 = mx2 + fast_log2(sum);
-
-  float accv[kV];
-#pragma unroll
-  for (int e = 0; e < kV; ++e) accv[e] = 0.f;
-#pragma unroll 4
-  for (int k = warp; k < count; k += 8) {
-    const float wk = fast_exp2(lse[k * lse_stride] * kLog2e - lse2);
-    const float *src = o + k * o_stride + lane * kV;
-    if (wk > 0.f) {
-      if constexpr (kV == 4) {
-        const float4 v = *reinterpret_cast<const float4 *>(src);
-        accv[0] += wk * v.x;
-        accv[1] += wk * v.y;
-        accv[2] += wk * v.z;
-        accv[3] += wk * v.w;
-      } else {
-        const float2 v = *reinterpret_cast<const float2 *>(src);
-        accv[0] += wk * v.x;
-        accv[1] += wk * v.y;
-      }
-    }
+  for (int i = 0; i < 8; ++i) {
+    sc[i] = wm[i] == -INFINITY ? 0.f : fast_exp2(wm[i] - M);
+    L += wl[i] * sc[i];
   }
-#pragma unroll
-  for (int e = 0; e < kV; ++e) part[warp][lane * kV + e] = accv[e];
-  __syncthreads();
+  const float inv = 1.f / L;
   for (int t = tid; t < D; t += 256) {
     float v = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v += part[i][t];
-    out[t] = Mma<T>::from_float(v);
+    for (int i = 0; i < 8; ++i) v += wo[i][t] * sc[i];
+    out[t] = Mma<T>::from_float(v * inv);
   }
-  if (tid == 0 && lse_out) *lse_out = lse2 * kLn2;
+  if (tid == 0 && lse_out) *lse_out = (M + fast_log2(L)) * kLn2;
 }
 
 // Merge of the pieces of every (sequence, KV head) pair that partition edges

@@ -36,6 +36,12 @@ struct DecodeArgs {
   int nparts;         // N: partitions (CTAs) of the concatenated page list
   int min_pages;      // lower bound on average pages per used partition
   int evict_first;    // 1: stream K/V with an L2 evict-first hint
+  // fused append (all null for attention only): every sequence with
+  // seq_lens[b] >= 1 writes k_new[b], v_new[b] at position seq_lens[b] - 1
+  const void *k_new;
+  const void *v_new;
+  void *k_cache;
+  void *v_cache;
 };
 
 struct GenericMergeArgs {

@@ -93,6 +93,15 @@ def test_decode_validation(kw, status):
     assert kvd.kvd_last_error() != ""
 
 
+def test_step_requires_new_rows():
+    a = (DUMMY, NULL, DUMMY, DUMMY, DUMMY, DUMMY, DUMMY, 0.125, DUMMY, 2, 8, 2, 128, 16, 4, 4,
+         DUMMY, 1 << 30, NULL, kvd.KVD_F16, NULL)
+    assert L.kvd_decode_step(*a) == kvd.KVD_ERR_INVALID
+    b = list(a)
+    b[1], b[2] = MISALIGNED, DUMMY
+    assert L.kvd_decode_step(*b) == kvd.KVD_ERR_INVALID
+
+
 def test_decode_empty_batch_is_a_no_op():
     assert decode(B=0, q=NULL, out=NULL, ws=NULL) == kvd.KVD_OK
 

@@ -239,3 +239,52 @@ def test_repeated_calls_are_deterministic(kvd):
     b = kvd.kvd_decode_attention(q, kc, vc, bt, sl, w.scale)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+# ------------------------------------------------------- fused decode step
+
+STEP_CASES = [
+    (4, 32, 8, 128, "bf16", [700, 33, 1200, 0], 0),
+    (5, 8, 8, 64, "f16", [1, 16, 17, 300, 47], 0),
+    (3, 16, 1, 128, "bf16", [200, 64, 129], 7),
+    (2, 32, 2, 128, "f16", [513, 31], 3),
+]
+
+
+@pytest.mark.parametrize("case", STEP_CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_d{c[3]}_{c[4]}_N{c[6]}")
+def test_fused_step_equals_append_then_attend(kvd, case):
+    B, H_q, H_kv, d, dtype, lens, parts = case
+    w = build_workload("step", B, H_q, H_kv, d, dtype, lens, seed=800 + STEP_CASES.index(case),
+                       spare_pages=2)
+    si = step_inputs(w, 0)
+    kc1, vc1, bt = gpu_state(w)
+    o1, l1 = gpu_step(kvd, w, si, kc1, vc1, bt, num_partitions=parts)
+    kc2, vc2, _ = gpu_state(w)
+    l2 = torch.empty_like(l1)
+    o2 = kvd.kvd_decode_step(si["q"].cuda(), si["k_new"].cuda(), si["v_new"].cuda(), kc2, vc2, bt,
+                             si["seq_lens"].cuda(), w.scale, num_partitions=parts, lse_out=l2)
+    torch.cuda.synchronize()
+    assert torch.equal(kc1.view(torch.int16), kc2.view(torch.int16))
+    assert torch.equal(vc1.view(torch.int16), vc2.view(torch.int16))
+    assert torch.equal(o1, o2)
+    assert torch.equal(l1, l2)
+    _, _, ref = oracle_step(w, si)
+    assert max_err(o2, ref) <= TOL[w.dtype]
+    assert kvd.kvd_read_device_error() == 0
+
+
+def test_fused_steps_continuous_batching(kvd):
+    # 4 consecutive fused steps with a shared prefix, against the oracle
+    lens = [40, 47, 33, 64 + 5]
+    w = build_workload("steps", 4, 8, 2, 128, "f16", lens, seed=851, steps=4, prefix_groups=2,
+                       prefix_tokens=32)
+    kc, vc, bt = gpu_state(w)
+    okc, ovc = to_words(w.k_cache).copy(), to_words(w.v_cache).copy()
+    for step in range(4):
+        si = step_inputs(w, step)
+        out = kvd.kvd_decode_step(si["q"].cuda(), si["k_new"].cuda(), si["v_new"].cuda(), kc, vc,
+                                  bt, si["seq_lens"].cuda(), w.scale)
+        torch.cuda.synchronize()
+        okc, ovc, ref = oracle_step(w, si, okc, ovc)
+        assert max_err(out, ref) <= TOL[w.dtype]
+    assert np.array_equal(to_words(kc), okc) and np.array_equal(to_words(vc), ovc)
