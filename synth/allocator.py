@@ -68,7 +68,12 @@ class BlockAllocator:
             raise KeyError(f"sequence {seq_id} already present")
         self.tables[seq_id] = []
         self.lengths[seq_id] = 0
-        self.grow(seq_id, tokens)
+        try:
+            self.grow(seq_id, tokens)
+        except OutOfPages:
+            del self.tables[seq_id]
+            del self.lengths[seq_id]
+            raise
         return self.tables[seq_id]
 
     def grow(self, seq_id: int, tokens: int) -> list[int]:
