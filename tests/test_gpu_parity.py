@@ -288,3 +288,43 @@ def test_fused_steps_continuous_batching(kvd):
         okc, ovc, ref = oracle_step(w, si, okc, ovc)
         assert max_err(out, ref) <= TOL[w.dtype]
     assert np.array_equal(to_words(kc), okc) and np.array_equal(to_words(vc), ovc)
+
+
+def test_cuda_graph_of_16_steps_matches_eager(kvd):
+    # continuous batching: 16 fused append+attend steps captured once in a CUDA
+    # graph; replaying it must give the eager steps' caches and outputs exactly
+    lens = [40, 47, 33, 69, 52, 38, 90, 61]
+    w = build_workload("graph", 8, 16, 4, 128, "bf16", lens, seed=871, steps=16, prefix_groups=2,
+                       prefix_tokens=32)
+    steps = [step_inputs(w, s) for s in range(16)]
+    dev = [{k: v.cuda() for k, v in si.items()} for si in steps]
+    ws = kvd.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, 0)
+
+    kc_e, vc_e, bt = gpu_state(w)
+    outs_e = [torch.empty_like(d["q"]) for d in dev]
+    for d, o in zip(dev, outs_e):
+        kvd.kvd_decode_step(d["q"], d["k_new"], d["v_new"], kc_e, vc_e, bt, d["seq_lens"], w.scale,
+                            out=o, workspace=ws)
+    torch.cuda.synchronize()
+
+    kc_g, vc_g, _ = gpu_state(w)
+    outs_g = [torch.empty_like(d["q"]) for d in dev]
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for d, o in zip(dev, outs_g):
+                kvd.kvd_decode_step(d["q"], d["k_new"], d["v_new"], kc_g, vc_g, bt, d["seq_lens"],
+                                    w.scale, out=o, workspace=ws, stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(outs_e, outs_g):
+        assert torch.equal(a, b)
+    assert torch.equal(kc_e.view(torch.int16), kc_g.view(torch.int16))
+    assert torch.equal(vc_e.view(torch.int16), vc_g.view(torch.int16))
+    # a second replay rewrites the same rows and recomputes the same outputs
+    g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(outs_e, outs_g):
+        assert torch.equal(a, b)
+    del g
