@@ -297,7 +297,28 @@ def run_ours(args):
     ws = kvd.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, args.partitions, dev)
     stream = torch.cuda.current_stream()
 
+    sp = None
+    if args.shared_prefix:
+        if not w.groups:
+            raise SystemExit("--shared-prefix needs a workload with prefix groups (cbatch)")
+        per = w.B // w.groups
+        sp = {"start": torch.arange(0, w.B + 1, per, dtype=torch.int32, device=dev),
+              "pages": torch.full((w.groups,), w.prefix_tokens // 16, dtype=torch.int32, device=dev),
+              "max": per}
+        n = kvd.kvd_shared_prefix_workspace_size(w.B, w.H_q, w.H_kv, w.d, w.groups, per, args.partitions)
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+
     def step(ev_a=None, ev_b=None):
+        if sp is not None:
+            if ev_a is not None:
+                ev_a.record(stream)
+            kvd.kvd_decode_attention_shared_prefix(q, kc, vc, bt, seq_lens, sp["start"], sp["pages"],
+                                                   sp["max"], w.scale, out=out, k_new=k_new,
+                                                   v_new=v_new, num_partitions=args.partitions,
+                                                   workspace=ws, stream=stream)
+            if ev_b is not None:
+                ev_b.record(stream)
+            return
         if args.separate_append:
             kvd.kvd_append(kc, vc, bt, slot, k_new, v_new, stream=stream)
         if ev_a is not None:
@@ -390,7 +411,13 @@ def run_ours(args):
     def e2e_step():
         for n in h_in:
             d_in[n].copy_(h_in[n], non_blocking=True)
-        if args.separate_append:
+        if sp is not None:
+            kvd.kvd_decode_attention_shared_prefix(d_in["q"], kc, vc, bt, d_in["seq_lens"], sp["start"],
+                                                   sp["pages"], sp["max"], w.scale, out=out,
+                                                   k_new=d_in["k_new"], v_new=d_in["v_new"],
+                                                   num_partitions=args.partitions, workspace=ws,
+                                                   stream=stream)
+        elif args.separate_append:
             kvd.kvd_append(kc, vc, bt, d_in["slot"], d_in["k_new"], d_in["v_new"], stream=stream)
             kvd.kvd_decode_attention(d_in["q"], kc, vc, bt, d_in["seq_lens"], w.scale, out=out,
                                      num_partitions=args.partitions, workspace=ws, stream=stream)
@@ -446,7 +473,9 @@ def run_ours(args):
             "bytes_per_step": step_bytes, "attention_bytes": a_bytes, "append_bytes": p_bytes,
             "l2": "inputs larger than L2 (KV pool %.2f GB >> 126 MB); no flush" % (
                 2 * w.k_cache.numel() * 2 / 1e9),
-            "step": ("kvd_append + kvd_decode_attention (append, decode, merge kernels)"
+            "step": ("kvd_decode_attention_shared_prefix with fused append (prefix, decode, merge kernels)"
+                     if sp is not None else
+                     "kvd_append + kvd_decode_attention (append, decode, merge kernels)"
                      if args.separate_append else
                      "kvd_decode_step (decode kernel with fused append, merge kernel)"),
         },
@@ -481,7 +510,7 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "us_per_step": round(e2e_s / e2e_steps * 1e6, 2),
                 "how": "pinned host inputs -> H2D, append, decode, D2H of out, stream sync; wall clock"},
-        "gpu_launches": (3 if args.separate_append else 2) * args.steps * per,
+        "gpu_launches": (3 if (args.separate_append or sp is not None) else 2) * args.steps * per,
         "graph": ({"steps_per_graph": args.graph_steps, "replays": args.steps} if graph is not None
                   else None),
         "clocks": clocks,
@@ -511,6 +540,8 @@ def main(argv=None):
     p.add_argument("--separate-append", action="store_true",
                    help="time kvd_append + kvd_decode_attention instead of the fused kvd_decode_step")
     p.add_argument("--e2e-steps", type=int, default=300)
+    p.add_argument("--shared-prefix", action="store_true",
+                   help="read each group's shared prefix pages once (kvd_decode_attention_shared_prefix)")
     p.add_argument("--graph", action="store_true",
                    help="capture --graph-steps fused steps in one CUDA graph and time its replays")
     p.add_argument("--graph-steps", type=int, default=16)
@@ -524,7 +555,7 @@ def main(argv=None):
     args = p.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.graph and args.separate_append:
+    if args.graph and (args.separate_append or args.shared_prefix):
         raise SystemExit("--graph times the fused step only")
     if args.impl == "reference":
         return run_reference(args)

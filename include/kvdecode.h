@@ -146,6 +146,40 @@ kvd_status kvd_decode_step(const void *q, const void *k_new, const void *v_new, 
                            int max_blocks_per_seq, int num_partitions, void *workspace,
                            size_t workspace_bytes, float *lse_out, kvd_dtype dtype, void *stream);
 
+/*
+ * kvd_decode_attention_shared_prefix -- decode attention (optionally with the
+ * fused append of kvd_decode_step) for batches whose sequences share prefix
+ * pages, reading each shared page once per group instead of once per member.
+ * "KV缓存与Flash注意力", sections 实际应用 and 练习 (prefix caching: requests with
+ * the same system prompt or document reuse its KV); [BLOG] "PagedAttention"
+ * (members' block tables point at the same physical pages).
+ *
+ *   group_start   device int32 [n_groups + 1]: group g is the contiguous
+ *                 sequences group_start[g] .. group_start[g+1]-1
+ *   group_pages   device int32 [n_groups]: the first group_pages[g] pages of
+ *                 every member are the same physical pages, namely
+ *                 block_table[group_start[g]][0 .. group_pages[g]-1]
+ *   n_groups      0 makes this call kvd_decode_attention / kvd_decode_step
+ *   max_group_size  upper bound on members per group (sizes the launch)
+ *   k_new, v_new  nullable; when given, the step's new token is appended as
+ *                 in kvd_decode_step (it must land in a private page)
+ *   workspace     kvd_shared_prefix_workspace_size(...) bytes, 256-aligned
+ *   other arguments as kvd_decode_attention.
+ * The result equals kvd_decode_attention's up to fp32 rounding order (the
+ * shared tokens are summed in a separate pass and merged by log-sum-exp).
+ * A member shorter than its group's shared pages is attended whole.
+ */
+kvd_status kvd_decode_attention_shared_prefix(
+    const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+    const int32_t *block_table, const int32_t *seq_lens, float scale, void *out, int B, int H_q,
+    int H_kv, int d, int num_blocks, int max_blocks_per_seq, const int32_t *group_start,
+    const int32_t *group_pages, int n_groups, int max_group_size, int num_partitions,
+    void *workspace, size_t workspace_bytes, float *lse_out, kvd_dtype dtype, void *stream);
+
+/* Workspace bytes of kvd_decode_attention_shared_prefix (0 if the shape is rejected). */
+size_t kvd_shared_prefix_workspace_size(int B, int H_q, int H_kv, int d, int n_groups,
+                                        int max_group_size, int num_partitions);
+
 /* Bytes of the library's fixed scratch array used by kvd_decode_attention_static. */
 #define KVD_STATIC_WORKSPACE_BYTES (8u << 20)
 

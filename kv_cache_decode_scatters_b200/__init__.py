@@ -21,6 +21,7 @@ __all__ = [
     "KVD_OK", "KVD_ERR_INVALID", "KVD_ERR_UNSUPPORTED", "KVD_ERR_CUDA", "KVD_ERR_WORKSPACE",
     "KVD_F16", "KVD_BF16", "KVD_PAGE_TOKENS", "KvdError",
     "kvd_append", "kvd_decode_attention", "kvd_decode_step", "kvd_decode_attention_static",
+    "kvd_decode_attention_shared_prefix", "kvd_shared_prefix_workspace_size",
     "kvd_merge_lse",
     "kvd_workspace_size", "KVD_STATIC_WORKSPACE_BYTES",
     "kvd_auto_partitions", "kvd_kv_bytes_per_token", "kvd_read_device_error",
@@ -53,6 +54,11 @@ def _load():
     L.kvd_decode_attention.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, I, P, S, P, I, P]
     L.kvd_decode_step.restype = I
     L.kvd_decode_step.argtypes = [P, P, P, P, P, P, P, F, P, I, I, I, I, I, I, I, P, S, P, I, P]
+    L.kvd_decode_attention_shared_prefix.restype = I
+    L.kvd_decode_attention_shared_prefix.argtypes = [P, P, P, P, P, P, P, F, P, I, I, I, I, I, I,
+                                                     P, P, I, I, I, P, S, P, I, P]
+    L.kvd_shared_prefix_workspace_size.restype = S
+    L.kvd_shared_prefix_workspace_size.argtypes = [I, I, I, I, I, I, I]
     L.kvd_decode_attention_static.restype = I
     L.kvd_decode_attention_static.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, P, I, P]
     L.kvd_merge_lse.restype = I
@@ -214,6 +220,52 @@ def kvd_decode_step(q, k_new, v_new, k_cache, v_cache, block_table, seq_lens, sc
         int(num_partitions), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         lse_ptr, _dtype_code(k_cache), _stream(stream)),
         "kvd_decode_step")
+    return out
+
+
+def kvd_shared_prefix_workspace_size(B, H_q, H_kv, d, n_groups, max_group_size, num_partitions=0):
+    n = int(_lib.kvd_shared_prefix_workspace_size(B, H_q, H_kv, d, n_groups, max_group_size,
+                                                  num_partitions))
+    if n == 0 and B > 0:
+        raise KvdError(KVD_ERR_INVALID, "kvd_shared_prefix_workspace_size")
+    return n
+
+
+def kvd_decode_attention_shared_prefix(q, k_cache, v_cache, block_table, seq_lens, group_start,
+                                       group_pages, max_group_size, scale=None, out=None,
+                                       k_new=None, v_new=None, num_partitions=0, workspace=None,
+                                       lse_out=None, stream=None):
+    """Decode attention over a batch whose groups of consecutive sequences
+    share their first group_pages[g] pages (read once per group).  With
+    k_new/v_new it also appends the step's token as kvd_decode_step does."""
+    B, H_q, d = q.shape
+    NB, H_kv, P, d2 = k_cache.shape
+    if P != KVD_PAGE_TOKENS or d2 != d:
+        raise ValueError("q / cache shape mismatch")
+    n_groups = group_pages.shape[0]
+    if group_start.shape[0] != n_groups + 1:
+        raise ValueError("group_start must have n_groups + 1 entries")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new or neither")
+    dt = k_cache.dtype
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        n = kvd_shared_prefix_workspace_size(B, H_q, H_kv, d, n_groups, max_group_size, num_partitions)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    kn = None if k_new is None else _dev(k_new, "k_new", dt)
+    vn = None if v_new is None else _dev(v_new, "v_new", dt)
+    lse_ptr = None if lse_out is None else _dev(lse_out, "lse_out", torch.float32)
+    _check(_lib.kvd_decode_attention_shared_prefix(
+        _dev(q, "q", dt), kn, vn, _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
+        float(scale), _dev(out, "out", dt), B, H_q, H_kv, d, NB, block_table.shape[1],
+        _dev(group_start, "group_start", torch.int32), _dev(group_pages, "group_pages", torch.int32),
+        n_groups, int(max_group_size), int(num_partitions), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), lse_ptr, _dtype_code(k_cache), _stream(stream)),
+        "kvd_decode_attention_shared_prefix")
     return out
 
 

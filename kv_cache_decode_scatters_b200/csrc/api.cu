@@ -110,6 +110,42 @@ WsLayout ws_layout(int B, int G, int d, long long slots) {
   return L;
 }
 
+// Shared-prefix scratch after the decode workspace: per-sequence skipped
+// pages, then the prefix chunks' partial lse and o.
+struct PrefixLayout {
+  size_t skip, pre_lse, pre_o, total;
+  int chunks, row_blocks;
+};
+
+kvd_status prefix_layout(int B, int H_kv, int G, int d, int n_groups, int max_group_size,
+                         size_t base, PrefixLayout *out) {
+  int dev, sms;
+  kvd_status st = current_device(&dev);
+  if (st) return st;
+  st = sm_count(dev, &sms);
+  if (st) return st;
+  const long long rows = static_cast<long long>(max_group_size) * G;
+  const int rpc = kvd::prefix_rows_per_cta();
+  const long long rb = (rows + rpc - 1) / rpc;
+  if (rb > 65535) return fail(KVD_ERR_UNSUPPORTED, "group of %d sequences too large", max_group_size);
+  // about four prefix CTAs per SM in all, each over a contiguous chunk of pages
+  const long long units = static_cast<long long>(n_groups) * H_kv * rb;
+  long long chunks = (4LL * sms + units - 1) / units;
+  chunks = chunks < 1 ? 1 : (chunks > 64 ? 64 : chunks);
+  if (static_cast<long long>(n_groups) * chunks > 0x7fffffffLL)
+    return fail(KVD_ERR_UNSUPPORTED, "too many groups");
+  PrefixLayout L;
+  L.chunks = static_cast<int>(chunks);
+  L.row_blocks = static_cast<int>(rb);
+  L.skip = round_up(base, 256);
+  L.pre_lse = L.skip + round_up(static_cast<size_t>(B) * 4, 256);
+  const size_t n = static_cast<size_t>(chunks) * H_kv * B * G;
+  L.pre_o = L.pre_lse + round_up(n * 4, 256);
+  L.total = L.pre_o + n * d * 4;
+  *out = L;
+  return KVD_OK;
+}
+
 kvd_status resolve_parts(int d, int num_partitions, int *N) {
   if (num_partitions < 0) return fail(KVD_ERR_INVALID, "num_partitions < 0");
   if (num_partitions > 0) {
@@ -222,7 +258,10 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
                               void *out, int B, int H_q, int H_kv, int d, int num_blocks,
                               int max_blocks_per_seq, int num_partitions, void *workspace,
                               size_t workspace_bytes, float *lse_out, kvd_dtype dtype, void *stream,
-                              const void *k_new, const void *v_new) {
+                              const void *k_new, const void *v_new,
+                              const int32_t *group_start = nullptr,
+                              const int32_t *group_pages = nullptr, int n_groups = 0,
+                              int max_group_size = 0) {
   kvd_status st = check_heads(B, H_q, H_kv, d);
   if (st) return st;
   if (num_blocks <= 0 || max_blocks_per_seq <= 0)
@@ -246,7 +285,16 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   if (st) return st;
   const int G = H_q / H_kv;
   const long long slots = static_cast<long long>(N) + static_cast<long long>(B) * H_kv;
-  const WsLayout L = ws_layout(B, G, d, slots);
+  const WsLayout L0 = ws_layout(B, G, d, slots);
+  PrefixLayout PL{};
+  if (n_groups > 0) {
+    if (!group_start || !group_pages) return fail(KVD_ERR_INVALID, "group_start / group_pages is NULL");
+    if (max_group_size <= 0) return fail(KVD_ERR_INVALID, "max_group_size must be positive");
+    st = prefix_layout(B, H_kv, G, d, n_groups, max_group_size, L0.total, &PL);
+    if (st) return st;
+  }
+  WsLayout L = L0;
+  if (n_groups > 0) L.total = PL.total;
   if (!workspace) return fail(KVD_ERR_WORKSPACE, "workspace is NULL (need %zu bytes)", L.total);
   if (!aligned(workspace, 256)) return fail(KVD_ERR_INVALID, "workspace must be 256-byte aligned");
   if (workspace_bytes < L.total)
@@ -307,10 +355,43 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   a.v_new = v_new;
   a.k_cache = const_cast<void *>(k_cache);
   a.v_cache = const_cast<void *>(v_cache);
+  a.skip = nullptr;
+  a.pre_o = nullptr;
+  a.pre_lse = nullptr;
+  a.pre_chunks = 0;
 
   const kvd::DType dt = dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = kvd::launch_decode(a, d, dt, tm[0], tm[1], s, N);
+  cudaError_t e;
+  if (n_groups > 0) {
+    kvd::PrefixArgs pa;
+    pa.q = q;
+    pa.block_table = block_table;
+    pa.seq_lens = seq_lens;
+    pa.group_start = group_start;
+    pa.group_pages = group_pages;
+    pa.skip = reinterpret_cast<int32_t *>(ws + PL.skip);
+    pa.pre_o = reinterpret_cast<float *>(ws + PL.pre_o);
+    pa.pre_lse = reinterpret_cast<float *>(ws + PL.pre_lse);
+    pa.err = err;
+    pa.scale_log2 = a.scale_log2;
+    pa.B = B;
+    pa.H_q = H_q;
+    pa.H_kv = H_kv;
+    pa.G = G;
+    pa.num_blocks = num_blocks;
+    pa.maxb = max_blocks_per_seq;
+    pa.n_groups = n_groups;
+    pa.chunks = PL.chunks;
+    pa.fused = k_new != nullptr;
+    e = kvd::launch_prefix(pa, d, dt, tm[0], tm[1], PL.row_blocks, s);
+    if (e != cudaSuccess) return cuda_fail(e, "prefix launch");
+    a.skip = pa.skip;
+    a.pre_o = pa.pre_o;
+    a.pre_lse = pa.pre_lse;
+    a.pre_chunks = PL.chunks;
+  }
+  e = kvd::launch_decode(a, d, dt, tm[0], tm[1], s, N);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   e = kvd::launch_decode_merge(a, d, dt, s);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
@@ -328,6 +409,41 @@ kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *
   return decode_impl(q, k_cache, v_cache, block_table, seq_lens, scale, out, B, H_q, H_kv, d,
                      num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
                      lse_out, dtype, stream, nullptr, nullptr);
+}
+
+size_t kvd_shared_prefix_workspace_size(int B, int H_q, int H_kv, int d, int n_groups,
+                                        int max_group_size, int num_partitions) {
+  if (check_heads(B, H_q, H_kv, d) != KVD_OK) return 0;
+  if (n_groups < 0 || max_group_size <= 0) {
+    fail(KVD_ERR_INVALID, "n_groups >= 0 and max_group_size > 0 required");
+    return 0;
+  }
+  int N = 0;
+  if (resolve_parts(d, num_partitions, &N) != KVD_OK) return 0;
+  const long long slots = static_cast<long long>(N) + static_cast<long long>(B) * H_kv;
+  const WsLayout L0 = ws_layout(B, H_q / H_kv, d, slots);
+  if (n_groups == 0) return L0.total;
+  PrefixLayout PL;
+  if (prefix_layout(B, H_kv, H_q / H_kv, d, n_groups, max_group_size, L0.total, &PL) != KVD_OK)
+    return 0;
+  return PL.total;
+}
+
+kvd_status kvd_decode_attention_shared_prefix(
+    const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+    const int32_t *block_table, const int32_t *seq_lens, float scale, void *out, int B, int H_q,
+    int H_kv, int d, int num_blocks, int max_blocks_per_seq, const int32_t *group_start,
+    const int32_t *group_pages, int n_groups, int max_group_size, int num_partitions,
+    void *workspace, size_t workspace_bytes, float *lse_out, kvd_dtype dtype, void *stream) {
+  if (n_groups < 0) return fail(KVD_ERR_INVALID, "n_groups < 0");
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return fail(KVD_ERR_INVALID, "k_new and v_new must both be given or both be NULL");
+  if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16)))
+    return fail(KVD_ERR_INVALID, "k_new / v_new must be 16-byte aligned");
+  return decode_impl(q, k_cache, v_cache, block_table, seq_lens, scale, out, B, H_q, H_kv, d,
+                     num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
+                     lse_out, dtype, stream, k_new, v_new, group_start, group_pages, n_groups,
+                     max_group_size);
 }
 
 kvd_status kvd_decode_step(const void *q, const void *k_new, const void *v_new, void *k_cache,

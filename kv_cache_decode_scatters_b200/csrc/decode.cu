@@ -43,10 +43,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
-
-#ifndef KVD_BF16_SPLIT_P
-#define KVD_BF16_SPLIT_P 1
-#endif
+#include "tile.cuh"
 
 namespace kvd {
 
@@ -66,20 +63,6 @@ struct Geo {
   }
 };
 
-// Byte offset of element column `col` (a multiple of 8) of token row t inside
-// a page staged as d/64 boxes of [16 tokens][64 elements], each box one
-// 2 KB run of 128-byte rows with the TMA 128-byte swizzle (16-byte chunk
-// index XOR row % 8).  Keeping each 64-column half in its own 2 KB run puts 8
-// consecutive tokens on 8 different chunk positions, so every 8-row ldmatrix
-// phase is free of bank conflicts.
-template <int D>
-__device__ __forceinline__ uint32_t swz(int t, int col) {
-  const int half = col >> 6;
-  const int chunk = (col & 63) >> 3;
-  return static_cast<uint32_t>(half * (kPage * 128) + t * 128 + ((chunk ^ (t & 7)) << 4));
-}
-
-__device__ __forceinline__ int clamp_len(int n, int cap) { return n < 0 ? 0 : (n > cap ? cap : n); }
 
 template <typename T>
 struct Stor;
@@ -116,10 +99,6 @@ __global__ void __launch_bounds__(32 * W, 1)
   constexpr int kRows = 8 * NT;  // query rows per tile (G padded)
   constexpr int kPatch = 32;     // page-meta flag: fused append writes a row of this page
   const bool fused = a.k_new != nullptr;
-  // bf16 keeps only 8 significant bits of each probability; carrying the
-  // rounding remainder in a second PV product restores ~16 bits for the cost
-  // of d/16 extra MMAs per page (free while the kernel waits on HBM).
-  constexpr bool kSplitP = KVD_BF16_SPLIT_P && std::is_same<T, __nv_bfloat16>::value;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int warp_tot[32];
 
@@ -146,6 +125,14 @@ __global__ void __launch_bounds__(32 * W, 1)
     prefetch_tensormap(&tmV);
   }
 
+  // pages of sequence b this kernel streams: all of them, minus the leading
+  // shared pages a prefix pass already attended (shared-prefix mode)
+  auto skip_of = [&](int b) -> int { return a.skip ? __ldg(a.skip + b) : 0; };
+  auto pages_of = [&](int b) -> int {
+    const int np = (clamp_len(__ldg(a.seq_lens + b), cap) + kPage - 1) / kPage;
+    return max(0, np - skip_of(b));
+  };
+
   // ---- 1. pages per sequence, exclusive prefix sum into cum[0..B]
   {
     const int per = (a.B + Gm::kThreads - 1) / Gm::kThreads;
@@ -155,7 +142,7 @@ __global__ void __launch_bounds__(32 * W, 1)
     for (int b = b0; b < b1; ++b) {
       const int raw = __ldg(a.seq_lens + b);
       if (raw < 0 || raw > cap) flag_error(a.err, kErrSeqLen);
-      local += (clamp_len(raw, cap) + kPage - 1) / kPage;
+      local += pages_of(b);
     }
     const int incl = warp_incl_scan(local, lane);
     if (lane == 31) warp_tot[warp] = incl;
@@ -169,7 +156,7 @@ __global__ void __launch_bounds__(32 * W, 1)
     int run = (warp ? warp_tot[warp - 1] : 0) + incl - local;
     for (int b = b0; b < b1; ++b) {
       cum[b] = run;
-      run += (clamp_len(__ldg(a.seq_lens + b), cap) + kPage - 1) / kPage;
+      run += pages_of(b);
     }
     if (tid == 0) cum[a.B] = warp_tot[W - 1];
     if (tid < 2 * W) edge_id[tid] = -1;
@@ -186,7 +173,7 @@ __global__ void __launch_bounds__(32 * W, 1)
     for (long long r = static_cast<long long>(blockIdx.x) * Gm::kThreads + tid; r < rows;
          r += static_cast<long long>(gridDim.x) * Gm::kThreads) {
       const int b = static_cast<int>(r / a.H_q);
-      if (cum[b + 1] == cum[b]) {
+      if (cum[b + 1] == cum[b] && skip_of(b) == 0) {
         Stor<T>::zero_row(reinterpret_cast<T *>(a.out) + r * D, D);
         if (a.lse_out) a.lse_out[r] = -INFINITY;
       }
@@ -205,6 +192,9 @@ __global__ void __launch_bounds__(32 * W, 1)
   uint32_t qf[NT][Gm::kSteps][2];
   float acc[NT][Gm::kSteps][4];
   float m_run[NT][2], l_run[NT][2];
+
+  // a pair whose sequence also has prefix partials always leaves a partial
+  auto forced_partial = [&](int seg) -> bool { return a.skip && skip_of(seg / H) > 0; };
 
   auto pair_range = [&](int seg, long long &s0, long long &s1) {
     const int b = seg / H, h = seg - (seg / H) * H;
@@ -291,7 +281,9 @@ __global__ void __launch_bounds__(32 * W, 1)
     long long s0, s1;
     pair_range(seg, s0, s1);
     if (s0 >= p0 && s1 <= p1) {
-      emit(seg, true);          // entirely inside this warp's share
+      // entirely inside this warp's share: final rows, or the one partial of
+      // this CTA when the sequence also has prefix partials to merge
+      emit(seg, !forced_partial(seg));
     } else if (s0 < p0) {
       park(seg, 0, edge_acc + (size_t)warp * Gm::kEdgeFloats);  // continues from an earlier warp
     } else {
@@ -336,8 +328,9 @@ __global__ void __launch_bounds__(32 * W, 1)
         const long long off = pos - static_cast<long long>(cum[b]) * H;
         h = static_cast<int>(off / np);
         const int i = static_cast<int>(off - static_cast<long long>(h) * np);
-        pb = __ldg(a.block_table + static_cast<size_t>(b) * a.maxb + i);
-        ntok = min(kPage, clamp_len(__ldg(a.seq_lens + b), cap) - i * kPage);
+        const int li = i + skip_of(b);  // logical page index in the sequence
+        pb = __ldg(a.block_table + static_cast<size_t>(b) * a.maxb + li);
+        ntok = min(kPage, clamp_len(__ldg(a.seq_lens + b), cap) - li * kPage);
         // fused append: the pair's last page holds the step's new token
         if (fused && i == np - 1) ntok |= kPatch;
         seg = b * H + h;
@@ -399,12 +392,6 @@ __global__ void __launch_bounds__(32 * W, 1)
 #pragma unroll 1
     for (int s = 0; s < S; ++s)
       if (f < p1) issue();
-
-    // ---- per-lane fragment geometry
-    const int tK = (lane & 7) | (((lane >> 3) & 1) << 3);
-    const int cK = ((lane >> 4) & 1) << 3;
-    const int tV = (lane & 7) | (((lane >> 4) & 1) << 3);
-    const int cV = ((lane >> 3) & 1) << 3;
 
     int cur = -1;  // pair being accumulated
 
@@ -488,95 +475,8 @@ __global__ void __launch_bounds__(32 * W, 1)
           fence_proxy_async_smem();
           __syncwarp();
         }
-        const uint32_t kb = smem_u32(kp), vb = smem_u32(vp);
-
-        // S^T = K Q^T, two independent accumulator chains over d
-        float s[NT][4], s2[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < Gm::kSteps; ++ks) {
-          uint32_t fa[4];
-          ldmatrix_x4(fa, kb + swz<D>(tK, ks * 16 + cK));
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            if (ks & 1) M::run(s2[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
-            else M::run(s[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
-          }
-        }
-
-        // online softmax update (base 2), probabilities rounded to T (bf16:
-        // split into a rounded head and a rounded remainder, see kSplitP)
-        const bool v0 = g8 < ntok, v1 = g8 + 8 < ntok;
-        uint32_t pb0[NT], pb1[NT], pc0[NT], pc1[NT];
-        float alpha[NT][2];
-        bool rescale = false;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const float x0 = v0 ? (s[nt][0] + s2[nt][0]) * a.scale_log2 : -INFINITY;
-          const float x1 = v0 ? (s[nt][1] + s2[nt][1]) * a.scale_log2 : -INFINITY;
-          const float x2 = v1 ? (s[nt][2] + s2[nt][2]) * a.scale_log2 : -INFINITY;
-          const float x3 = v1 ? (s[nt][3] + s2[nt][3]) * a.scale_log2 : -INFINITY;
-          float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-          for (int o = 4; o < 32; o <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-          }
-          const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-          alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
-          alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
-          rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
-          m_run[nt][0] = mn0;
-          m_run[nt][1] = mn1;
-          const float e0 = fast_exp2(x0 - mn0), e1 = fast_exp2(x1 - mn1);
-          const float e2 = fast_exp2(x2 - mn0), e3 = fast_exp2(x3 - mn1);
-          const uint32_t lo = M::pack(e0, e1), hi = M::pack(e2, e3);
-          const float2 fl = M::unpack(lo), fh = M::unpack(hi);
-          if constexpr (kSplitP) {
-            // p = head + remainder, both bf16: ~16 significant bits in the PV
-            // product; the running sum uses the unrounded p to match
-            const uint32_t lo2 = M::pack(e0 - fl.x, e1 - fl.y);
-            const uint32_t hi2 = M::pack(e2 - fh.x, e3 - fh.y);
-            l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (e0 + e2);
-            l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (e1 + e3);
-            pc0[nt] = movmatrix_trans(lo2);
-            pc1[nt] = movmatrix_trans(hi2);
-          } else {
-            // the running sum uses the same rounded p as the PV product, so
-            // the output is an exact weighted mean of V up to fp32 sums
-            l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (fl.x + fh.x);
-            l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (fl.y + fh.y);
-            pc0[nt] = pc1[nt] = 0u;
-          }
-          pb0[nt] = movmatrix_trans(lo);
-          pb1[nt] = movmatrix_trans(hi);
-        }
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int mt = 0; mt < Gm::kSteps; ++mt) {
-              acc[nt][mt][0] *= alpha[nt][0];
-              acc[nt][mt][1] *= alpha[nt][1];
-              acc[nt][mt][2] *= alpha[nt][0];
-              acc[nt][mt][3] *= alpha[nt][1];
-            }
-        }
-
-        // O^T += V^T P^T
-#pragma unroll
-        for (int mt = 0; mt < Gm::kSteps; ++mt) {
-          uint32_t fa[4];
-          ldmatrix_x4_trans(fa, vb + swz<D>(tV, mt * 16 + cV));
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            M::run(acc[nt][mt], fa, pb0[nt], pb1[nt]);
-            if constexpr (kSplitP) M::run(acc[nt][mt], fa, pc0[nt], pc1[nt]);
-          }
-        }
+        tile_page<D, NT, T>(smem_u32(kp), smem_u32(vp), ntok, a.scale_log2, lane, qf, acc, m_run,
+                            l_run);
       }
       __syncwarp();
       if (f < p1) issue();
@@ -662,14 +562,14 @@ __global__ void __launch_bounds__(32 * W, 1)
         }
     long long s0, s1;
     pair_range(seg, s0, s1);
-    emit(seg, s0 >= c0 && s1 <= c1);
+    emit(seg, s0 >= c0 && s1 <= c1 && !forced_partial(seg));
   }
 }
 
 // ------------------------------------------------------------------ merge
 
-// One CTA (256 threads, 8 warps) merges `count` partial results of one
-// output row: partial k has log-sum-exp lse[k * lse_stride] and normalised
+// One CTA (256 threads, 8 warps) merges `count` (+ `count2` from a second
+// set laid out the same way) partial results of one output row: partial k has log-sum-exp lse[k * lse_stride] and normalised
 // output o[k * o_stride .. + D).  Each warp folds its partials k = warp,
 // warp + 8, ... into a running (max, sum, output) state -- the rescale of
 // the online softmax applied to whole partials -- loading four partials'
@@ -679,7 +579,10 @@ __global__ void __launch_bounds__(32 * W, 1)
 // never read); if all are empty, out = 0 and LSE = -inf.
 template <int D, typename T>
 __device__ __forceinline__ void merge_row(const float *lse, long long lse_stride, const float *o,
-                                          long long o_stride, int count, T *out, float *lse_out) {
+                                          long long o_stride, int count, T *out, float *lse_out,
+                                          const float *lse2 = nullptr, long long lse2_stride = 0,
+                                          const float *o2 = nullptr, long long o2_stride = 0,
+                                          int count2 = 0) {
   constexpr int kV = D / 32;
   constexpr int kBatch = 4;
   __shared__ float wm[8], wl[8];
@@ -690,17 +593,21 @@ __device__ __forceinline__ void merge_row(const float *lse, long long lse_stride
   float acc[kV];
 #pragma unroll
   for (int e = 0; e < kV; ++e) acc[e] = 0.f;
-  for (int k0 = warp; k0 < count; k0 += 8 * kBatch) {
+  const int total = count + count2;
+  for (int k0 = warp; k0 < total; k0 += 8 * kBatch) {
     float lk[kBatch];
     float ov[kBatch][kV];
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
       const int k = k0 + 8 * j;
-      lk[j] = k < count ? lse[k * lse_stride] * kLog2e : -INFINITY;
+      const bool first = k < count;
+      const long long kk = first ? k : k - count;
+      lk[j] = k < total ? (first ? lse[kk * lse_stride] : lse2[kk * lse2_stride]) * kLog2e
+                        : -INFINITY;
       // o is loaded with lse (not after it) so both are in flight together;
       // an empty partial's o is read but never used
-      if (k < count) {
-        const float *src = o + k * o_stride + lane * kV;
+      if (k < total) {
+        const float *src = (first ? o + kk * o_stride : o2 + kk * o2_stride) + lane * kV;
         if constexpr (kV == 4) {
           const float4 v = *reinterpret_cast<const float4 *>(src);
           ov[j][0] = v.x;
@@ -756,25 +663,118 @@ __device__ __forceinline__ void merge_row(const float *lse, long long lse_stride
   if (tid == 0 && lse_out) *lse_out = (M + fast_log2(L)) * kLn2;
 }
 
+// One warp merges the partials of one output row (two sets laid out like
+// merge_row's): the same running fold, four partials' loads in flight at a
+// time, no shared memory.  Used when rows have few partials each.
+template <int D, typename T>
+__device__ __forceinline__ void merge_row_warp(const float *lse, long long lse_stride,
+                                               const float *o, long long o_stride, int count,
+                                               T *out, float *lse_out, const float *lse2,
+                                               long long lse2_stride, const float *o2,
+                                               long long o2_stride, int count2, int lane) {
+  constexpr int kV = D / 32;
+  constexpr int kBatch = 4;
+  float m = -INFINITY, l = 0.f;
+  float acc[kV];
+#pragma unroll
+  for (int e = 0; e < kV; ++e) acc[e] = 0.f;
+  const int total = count + count2;
+  for (int k0 = 0; k0 < total; k0 += kBatch) {
+    float lk[kBatch];
+    float ov[kBatch][kV];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int k = k0 + j;
+      const bool first = k < count;
+      const long long kk = first ? k : k - count;
+      lk[j] = k < total ? (first ? lse[kk * lse_stride] : lse2[kk * lse2_stride]) * kLog2e
+                        : -INFINITY;
+      if (k < total) {
+        const float *src = (first ? o + kk * o_stride : o2 + kk * o2_stride) + lane * kV;
+        if constexpr (kV == 4) {
+          const float4 v = *reinterpret_cast<const float4 *>(src);
+          ov[j][0] = v.x;
+          ov[j][1] = v.y;
+          ov[j][2] = v.z;
+          ov[j][3] = v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2 *>(src);
+          ov[j][0] = v.x;
+          ov[j][1] = v.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      if (lk[j] == -INFINITY) continue;
+      const float mn = fmaxf(m, lk[j]);
+      const float a = fast_exp2(m - mn), b = fast_exp2(lk[j] - mn);
+#pragma unroll
+      for (int e = 0; e < kV; ++e) acc[e] = acc[e] * a + ov[j][e] * b;
+      l = l * a + b;
+      m = mn;
+    }
+  }
+  if (m == -INFINITY) {
+#pragma unroll
+    for (int e = 0; e < kV; ++e) out[lane * kV + e] = Mma<T>::from_float(0.f);
+    if (lane == 0 && lse_out) *lse_out = -INFINITY;
+    return;
+  }
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int e = 0; e < kV; ++e) out[lane * kV + e] = Mma<T>::from_float(acc[e] * inv);
+  if (lane == 0 && lse_out) *lse_out = (m + fast_log2(l)) * kLn2;
+}
+
 // Merge of the pieces of every (sequence, KV head) pair that partition edges
 // cut; grid = (B * H_kv pairs, G rows).
-template <int D, typename T>
+// Rows with many partials (long contexts cut by many CTAs) get a whole CTA
+// each (kWide); otherwise each warp of a CTA takes one row.
+template <int D, typename T, bool kWide>
 __global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeArgs a) {
   grid_dependency_wait();
-  const int seg = blockIdx.x, r = blockIdx.y;
+  grid_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row_id = kWide ? static_cast<long long>(blockIdx.x)
+                                 : static_cast<long long>(blockIdx.x) * 8 + warp;
+  if (row_id >= static_cast<long long>(a.B) * a.H_q) return;  // whole warp (or CTA)
+  const int seg = static_cast<int>(row_id / a.G), r = static_cast<int>(row_id - (row_id / a.G) * a.G);
   const int b = seg / a.H_kv, h = seg - b * a.H_kv;
   const int c0 = a.ws_cum[b], np = a.ws_cum[b + 1] - c0;
-  if (np == 0) return;
+  const int skip = a.skip ? __ldg(a.skip + b) : 0;
+  if (np == 0 && skip == 0) return;  // empty sequence: zeroed by the decode kernel
   const long long P = static_cast<long long>(a.ws_cum[a.B]) * a.H_kv;
-  const int N = effective_parts(P, a.nparts, a.min_pages);
-  const long long s0 = static_cast<long long>(c0) * a.H_kv + static_cast<long long>(h) * np;
-  const long long wf = part_of(s0, P, N), wl = part_of(s0 + np - 1, P, N);
-  if (wf == wl) return;  // written directly by its only worker
-  const long long slot0 = wf + seg;
   const size_t row = (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + r);
-  merge_row<D, T>(a.part_lse + slot0 * a.G + r, a.G, a.part_o + (slot0 * a.G + r) * D,
-                  static_cast<long long>(a.G) * D, static_cast<int>(wl - wf + 1),
-                  reinterpret_cast<T *>(a.out) + row * D, a.lse_out ? a.lse_out + row : nullptr);
+  long long slot0 = 0;
+  int count = 0;
+  if (np > 0) {
+    const int N = effective_parts(P, a.nparts, a.min_pages);
+    const long long s0 = static_cast<long long>(c0) * a.H_kv + static_cast<long long>(h) * np;
+    const long long wf = part_of(s0, P, N), wl = part_of(s0 + np - 1, P, N);
+    if (wf == wl && skip == 0) return;  // written directly by its only CTA
+    slot0 = wf + seg;
+    count = static_cast<int>(wl - wf + 1);
+  }
+  const float *pl = nullptr, *po = nullptr;
+  long long pls = 0, pos = 0;
+  int pc = 0;
+  if (skip > 0) {  // the prefix pass's chunk partials of this row
+    const size_t i0 = (static_cast<size_t>(h) * a.B + b) * a.G + r;
+    pls = static_cast<long long>(a.H_kv) * a.B * a.G;
+    pos = pls * D;
+    pl = a.pre_lse + i0;
+    po = a.pre_o + i0 * D;
+    pc = a.pre_chunks;
+  }
+  T *out = reinterpret_cast<T *>(a.out) + row * D;
+  float *lo = a.lse_out ? a.lse_out + row : nullptr;
+  if constexpr (kWide)
+    merge_row<D, T>(a.part_lse + slot0 * a.G + r, a.G, a.part_o + (slot0 * a.G + r) * D,
+                    static_cast<long long>(a.G) * D, count, out, lo, pl, pls, po, pos, pc);
+  else
+    merge_row_warp<D, T>(a.part_lse + slot0 * a.G + r, a.G, a.part_o + (slot0 * a.G + r) * D,
+                         static_cast<long long>(a.G) * D, count, out, lo, pl, pls, po, pos, pc, lane);
 }
 
 // Merge of caller-provided partials [B][H_q][S][D]; grid = B * H_q rows.
@@ -865,9 +865,18 @@ cudaError_t launch_decode_dt(const DecodeArgs &a, int d, const CUtensorMap &tmK,
 
 template <typename T>
 cudaError_t launch_merge_dt(const DecodeArgs &a, int d, cudaStream_t st) {
-  dim3 grid(a.B * a.H_kv, a.G);
-  if (d == 128) return launch_pdl(decode_merge_kernel<128, T>, grid, dim3(256), 0, st, a);
-  return launch_pdl(decode_merge_kernel<64, T>, grid, dim3(256), 0, st, a);
+  // expected partials per row: CTA partitions per pair, plus prefix chunks
+  const long long pairs = static_cast<long long>(a.B) * a.H_kv;
+  const long long per_row = a.nparts / (pairs > 0 ? pairs : 1) + 1 + a.pre_chunks;
+  const long long rows = static_cast<long long>(a.B) * a.H_q;
+  if (per_row >= 16) {
+    const dim3 grid(static_cast<unsigned>(rows));
+    if (d == 128) return launch_pdl(decode_merge_kernel<128, T, true>, grid, dim3(256), 0, st, a);
+    return launch_pdl(decode_merge_kernel<64, T, true>, grid, dim3(256), 0, st, a);
+  }
+  const dim3 grid(static_cast<unsigned>((rows + 7) / 8));
+  if (d == 128) return launch_pdl(decode_merge_kernel<128, T, false>, grid, dim3(256), 0, st, a);
+  return launch_pdl(decode_merge_kernel<64, T, false>, grid, dim3(256), 0, st, a);
 }
 
 template <typename T>

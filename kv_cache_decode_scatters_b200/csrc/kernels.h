@@ -42,6 +42,28 @@ struct DecodeArgs {
   const void *v_new;
   void *k_cache;
   void *v_cache;
+  // shared-prefix mode (all null otherwise): skip[b] leading pages of
+  // sequence b were attended by the prefix kernel; those pairs always leave
+  // partials, and the merge adds the prefix partials pre_o / pre_lse
+  // ([pre_chunks][H_kv][B][G][d] and [pre_chunks][H_kv][B][G])
+  const int32_t *skip;
+  const float *pre_o;
+  const float *pre_lse;
+  int pre_chunks;
+};
+
+struct PrefixArgs {
+  const void *q;
+  const int32_t *block_table;
+  const int32_t *seq_lens;
+  const int32_t *group_start;  // [n_groups + 1]: group g = sequences [start[g], start[g+1])
+  const int32_t *group_pages;  // [n_groups]: leading pages every member shares
+  int32_t *skip;               // [B] out: shared pages attended here per sequence (0 = none)
+  float *pre_o;                // [chunks][H_kv][B][G][d] normalised partial outputs
+  float *pre_lse;              // [chunks][H_kv][B][G]
+  unsigned *err;
+  float scale_log2;
+  int B, H_q, H_kv, G, num_blocks, maxb, n_groups, chunks, fused;
 };
 
 struct GenericMergeArgs {
@@ -65,5 +87,10 @@ cudaError_t launch_decode(const DecodeArgs &a, int d, DType dt, const CUtensorMa
                           const CUtensorMap &tmV, cudaStream_t s, int grid);
 cudaError_t launch_decode_merge(const DecodeArgs &a, int d, DType dt, cudaStream_t s);
 cudaError_t launch_generic_merge(const GenericMergeArgs &a, DType dt, cudaStream_t s);
+// Prefix pass of the shared-prefix decode: grid (n_groups * chunks, H_kv, row blocks).
+cudaError_t launch_prefix(const PrefixArgs &a, int d, DType dt, const CUtensorMap &tmK,
+                          const CUtensorMap &tmV, int row_blocks, cudaStream_t s);
+// Query rows one prefix CTA handles.
+int prefix_rows_per_cta();
 
 }  // namespace kvd

@@ -1,0 +1,264 @@
+// tile.cuh -- the per-page tensor-core tile shared by the decode and
+// shared-prefix kernels: swizzled page addressing and one 16-token step of
+// the online softmax for the query rows a warp holds.
+#pragma once
+
+#include <type_traits>
+
+#include "common.cuh"
+
+#ifndef KVD_BF16_SPLIT_P
+#define KVD_BF16_SPLIT_P 1
+#endif
+
+namespace kvd {
+
+// Byte offset of element column `col` (a multiple of 8) of token row t inside
+// a page staged as d/64 boxes of [16 tokens][64 elements], each box one
+// 2 KB run of 128-byte rows with the TMA 128-byte swizzle (16-byte chunk
+// index XOR row % 8).  Keeping each 64-column half in its own 2 KB run puts 8
+// consecutive tokens on 8 different chunk positions, so every 8-row ldmatrix
+// phase is free of bank conflicts.
+template <int D>
+__device__ __forceinline__ uint32_t swz(int t, int col) {
+  const int half = col >> 6;
+  const int chunk = (col & 63) >> 3;
+  return static_cast<uint32_t>(half * (kPage * 128) + t * 128 + ((chunk ^ (t & 7)) << 4));
+}
+
+__device__ __forceinline__ int clamp_len(int n, int cap) { return n < 0 ? 0 : (n > cap ? cap : n); }
+
+// One 16-token page of the online softmax for 8*NT query rows held by one
+// warp: S^T = K Q^T (K page as the A operand), base-2 running max / sum per
+// row, probabilities to the B operand via movmatrix, O^T += V^T P^T.  kb, vb:
+// shared addresses of the staged K and V pages (d/64 swizzled 2 KB boxes);
+// tokens >= ntok are masked.  The state arrays are the warp's registers.
+template <int D, int NT, typename T>
+__device__ __forceinline__ void tile_page(uint32_t kb, uint32_t vb, int ntok, float scale_log2,
+                                          int lane, const uint32_t (&qf)[NT][D / 16][2],
+                                          float (&acc)[NT][D / 16][4], float (&m_run)[NT][2],
+                                          float (&l_run)[NT][2]) {
+  using M = Mma<T>;
+  constexpr int kSteps = D / 16;
+  // bf16 keeps only 8 significant bits of each probability; carrying the
+  // rounding remainder in a second PV product restores ~16 bits for the cost
+  // of d/16 extra MMAs per page (free while the kernel waits on HBM).
+  constexpr bool kSplitP = KVD_BF16_SPLIT_P && std::is_same<T, __nv_bfloat16>::value;
+  const int g8 = lane >> 2;
+  const int tK = (lane & 7) | (((lane >> 3) & 1) << 3);
+  const int cK = ((lane >> 4) & 1) << 3;
+  const int tV = (lane & 7) | (((lane >> 4) & 1) << 3);
+  const int cV = ((lane >> 3) & 1) << 3;
+
+  // S^T = K Q^T, two independent accumulator chains over d
+  float s[NT][4], s2[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < kSteps; ++ks) {
+    uint32_t fa[4];
+    ldmatrix_x4(fa, kb + swz<D>(tK, ks * 16 + cK));
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      if (ks & 1) M::run(s2[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
+      else M::run(s[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
+    }
+  }
+
+  // online softmax update (base 2), probabilities rounded to T (bf16:
+  // split into a rounded head and a rounded remainder, see kSplitP)
+  const bool v0 = g8 < ntok, v1 = g8 + 8 < ntok;
+  uint32_t pb0[NT], pb1[NT], pc0[NT], pc1[NT];
+  float alpha[NT][2];
+  bool rescale = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const float x0 = v0 ? (s[nt][0] + s2[nt][0]) * scale_log2 : -INFINITY;
+    const float x1 = v0 ? (s[nt][1] + s2[nt][1]) * scale_log2 : -INFINITY;
+    const float x2 = v1 ? (s[nt][2] + s2[nt][2]) * scale_log2 : -INFINITY;
+    const float x3 = v1 ? (s[nt][3] + s2[nt][3]) * scale_log2 : -INFINITY;
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+    alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
+    alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
+    rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
+    m_run[nt][0] = mn0;
+    m_run[nt][1] = mn1;
+    const float e0 = fast_exp2(x0 - mn0), e1 = fast_exp2(x1 - mn1);
+    const float e2 = fast_exp2(x2 - mn0), e3 = fast_exp2(x3 - mn1);
+    const uint32_t lo = M::pack(e0, e1), hi = M::pack(e2, e3);
+    const float2 fl = M::unpack(lo), fh = M::unpack(hi);
+    if constexpr (kSplitP) {
+      // p = head + remainder, both bf16: ~16 significant bits in the PV
+      // product; the running sum uses the unrounded p to match
+      const uint32_t lo2 = M::pack(e0 - fl.x, e1 - fl.y);
+      const uint32_t hi2 = M::pack(e2 - fh.x, e3 - fh.y);
+      l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (e0 + e2);
+      l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (e1 + e3);
+      pc0[nt] = movmatrix_trans(lo2);
+      pc1[nt] = movmatrix_trans(hi2);
+    } else {
+      // the running sum uses the same rounded p as the PV product, so
+      // the output is an exact weighted mean of V up to fp32 sums
+      l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (fl.x + fh.x);
+      l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (fl.y + fh.y);
+      pc0[nt] = pc1[nt] = 0u;
+    }
+    pb0[nt] = movmatrix_trans(lo);
+    pb1[nt] = movmatrix_trans(hi);
+  }
+  if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int mt = 0; mt < kSteps; ++mt) {
+        acc[nt][mt][0] *= alpha[nt][0];
+        acc[nt][mt][1] *= alpha[nt][1];
+        acc[nt][mt][2] *= alpha[nt][0];
+        acc[nt][mt][3] *= alpha[nt][1];
+      }
+  }
+
+  // O^T += V^T P^T
+#pragma unroll
+  for (int mt = 0; mt < kSteps; ++mt) {
+    uint32_t fa[4];
+    ldmatrix_x4_trans(fa, vb + swz<D>(tV, mt * 16 + cV));
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      M::run(acc[nt][mt], fa, pb0[nt], pb1[nt]);
+      if constexpr (kSplitP) M::run(acc[nt][mt], fa, pc0[nt], pc1[nt]);
+    }
+  }
+}
+
+}  // namespace kvd
+
+namespace kvd {
+
+// Two full 16-token pages (A then B, in token order) in one step: both
+// pages' S^T chains run independently, one max/sum update covers the 32
+// tokens, and both PV products accumulate into the same tile.  Same result as
+// two tile_page calls up to fp32 rounding order; more independent work per
+// step for warps that are short of latency hiding.
+template <int D, int NT, typename T>
+__device__ __forceinline__ void tile_page2(uint32_t kbA, uint32_t vbA, uint32_t kbB, uint32_t vbB,
+                                           float scale_log2, int lane,
+                                           const uint32_t (&qf)[NT][D / 16][2],
+                                           float (&acc)[NT][D / 16][4], float (&m_run)[NT][2],
+                                           float (&l_run)[NT][2]) {
+  using M = Mma<T>;
+  constexpr int kSteps = D / 16;
+  constexpr bool kSplitP = KVD_BF16_SPLIT_P && std::is_same<T, __nv_bfloat16>::value;
+  const int tK = (lane & 7) | (((lane >> 3) & 1) << 3);
+  const int cK = ((lane >> 4) & 1) << 3;
+  const int tV = (lane & 7) | (((lane >> 4) & 1) << 3);
+  const int cV = ((lane >> 3) & 1) << 3;
+
+  float sa[NT][4], sb[NT][4], sa2[NT][4], sb2[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sa[nt][e] = sb[nt][e] = sa2[nt][e] = sb2[nt][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < kSteps; ++ks) {
+    uint32_t fa[4], fb[4];
+    ldmatrix_x4(fa, kbA + swz<D>(tK, ks * 16 + cK));
+    ldmatrix_x4(fb, kbB + swz<D>(tK, ks * 16 + cK));
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      if (ks & 1) {
+        M::run(sa2[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
+        M::run(sb2[nt], fb, qf[nt][ks][0], qf[nt][ks][1]);
+      } else {
+        M::run(sa[nt], fa, qf[nt][ks][0], qf[nt][ks][1]);
+        M::run(sb[nt], fb, qf[nt][ks][0], qf[nt][ks][1]);
+      }
+    }
+  }
+
+  uint32_t pa0[NT], pa1[NT], pb0[NT], pb1[NT];
+  uint32_t ra0[NT], ra1[NT], rb0[NT], rb1[NT];  // bf16 remainders
+  float alpha[NT][2];
+  bool rescale = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float x[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[e] = (sa[nt][e] + sa2[nt][e]) * scale_log2;
+      x[4 + e] = (sb[nt][e] + sb2[nt][e]) * scale_log2;
+    }
+    // row r0 = elements 0, 2 (page A), 4, 6 (page B); row r1 = 1, 3, 5, 7
+    float mx0 = fmaxf(fmaxf(x[0], x[2]), fmaxf(x[4], x[6]));
+    float mx1 = fmaxf(fmaxf(x[1], x[3]), fmaxf(x[5], x[7]));
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+    alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
+    alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
+    rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
+    m_run[nt][0] = mn0;
+    m_run[nt][1] = mn1;
+    float e[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) e[i] = fast_exp2(x[i] - ((i & 1) ? mn1 : mn0));
+    const uint32_t w0 = M::pack(e[0], e[1]), w1 = M::pack(e[2], e[3]);
+    const uint32_t w2 = M::pack(e[4], e[5]), w3 = M::pack(e[6], e[7]);
+    const float2 f0 = M::unpack(w0), f1 = M::unpack(w1), f2 = M::unpack(w2), f3 = M::unpack(w3);
+    if constexpr (kSplitP) {
+      ra0[nt] = movmatrix_trans(M::pack(e[0] - f0.x, e[1] - f0.y));
+      ra1[nt] = movmatrix_trans(M::pack(e[2] - f1.x, e[3] - f1.y));
+      rb0[nt] = movmatrix_trans(M::pack(e[4] - f2.x, e[5] - f2.y));
+      rb1[nt] = movmatrix_trans(M::pack(e[6] - f3.x, e[7] - f3.y));
+      l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + ((e[0] + e[2]) + (e[4] + e[6]));
+      l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + ((e[1] + e[3]) + (e[5] + e[7]));
+    } else {
+      ra0[nt] = ra1[nt] = rb0[nt] = rb1[nt] = 0u;
+      l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + ((f0.x + f1.x) + (f2.x + f3.x));
+      l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + ((f0.y + f1.y) + (f2.y + f3.y));
+    }
+    pa0[nt] = movmatrix_trans(w0);
+    pa1[nt] = movmatrix_trans(w1);
+    pb0[nt] = movmatrix_trans(w2);
+    pb1[nt] = movmatrix_trans(w3);
+  }
+  if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int mt = 0; mt < kSteps; ++mt) {
+        acc[nt][mt][0] *= alpha[nt][0];
+        acc[nt][mt][1] *= alpha[nt][1];
+        acc[nt][mt][2] *= alpha[nt][0];
+        acc[nt][mt][3] *= alpha[nt][1];
+      }
+  }
+#pragma unroll
+  for (int mt = 0; mt < kSteps; ++mt) {
+    uint32_t fa[4], fb[4];
+    ldmatrix_x4_trans(fa, vbA + swz<D>(tV, mt * 16 + cV));
+    ldmatrix_x4_trans(fb, vbB + swz<D>(tV, mt * 16 + cV));
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      M::run(acc[nt][mt], fa, pa0[nt], pa1[nt]);
+      M::run(acc[nt][mt], fb, pb0[nt], pb1[nt]);
+      if constexpr (kSplitP) {
+        M::run(acc[nt][mt], fa, ra0[nt], ra1[nt]);
+        M::run(acc[nt][mt], fb, rb0[nt], rb1[nt]);
+      }
+    }
+  }
+}
+
+}  // namespace kvd

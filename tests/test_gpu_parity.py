@@ -328,3 +328,90 @@ def test_cuda_graph_of_16_steps_matches_eager(kvd):
     for a, b in zip(outs_e, outs_g):
         assert torch.equal(a, b)
     del g
+
+
+# --------------------------------------------------- shared-prefix decode
+
+def groups_of(w):
+    per = w.B // w.groups
+    start = torch.arange(0, w.B + 1, per, dtype=torch.int32)
+    pages = torch.full((w.groups,), w.prefix_tokens // 16, dtype=torch.int32)
+    return start.cuda(), pages.cuda(), per
+
+
+SP_CASES = [
+    # B, H_q, H_kv, d, dtype, lens, groups, prefix tokens, partitions
+    (8, 32, 8, 128, "f16", [300, 257, 520, 999, 290, 400, 700, 266], 2, 256, 0),
+    (6, 64, 8, 128, "bf16", [40, 33, 90, 49, 34, 70], 3, 32, 0),
+    (4, 8, 8, 64, "f16", [600, 513, 530, 1000], 1, 512, 5),
+    (4, 16, 1, 128, "bf16", [200, 145, 160, 300], 2, 144, 0),   # MQA, group 16
+]
+
+
+@pytest.mark.parametrize("case", SP_CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_d{c[3]}_{c[4]}_g{c[6]}")
+def test_shared_prefix_matches_oracle_and_plain_decode(kvd, case):
+    B, H_q, H_kv, d, dtype, lens, groups, prefix, parts = case
+    w = build_workload("sp", B, H_q, H_kv, d, dtype, lens, seed=900 + SP_CASES.index(case),
+                       prefix_groups=groups, prefix_tokens=prefix)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    ref_gpu, _ = gpu_step(kvd, w, si, kc, vc, bt, num_partitions=parts)   # append + plain decode
+    gs, gp, per = groups_of(w)
+    lse = torch.empty((B, H_q), dtype=torch.float32, device="cuda")
+    out = kvd.kvd_decode_attention_shared_prefix(si["q"].cuda(), kc, vc, bt, si["seq_lens"].cuda(),
+                                                 gs, gp, per, w.scale, num_partitions=parts,
+                                                 lse_out=lse)
+    torch.cuda.synchronize()
+    _, _, ref = oracle_step(w, si)
+    assert max_err(out, ref) <= TOL[w.dtype]
+    assert max_lse_err(lse, ref) <= LSE_TOL
+    assert torch.max(torch.abs(out.float() - ref_gpu.float())).item() <= TOL[w.dtype]
+    assert kvd.kvd_read_device_error() == 0
+
+
+def test_shared_prefix_fused_append_matches_decode_step(kvd):
+    lens = [300, 257, 520, 999, 290, 400, 700, 266]
+    w = build_workload("spf", 8, 32, 8, 128, "bf16", lens, seed=951, steps=3, prefix_groups=4,
+                       prefix_tokens=256)
+    gs, gp, per = groups_of(w)
+    kc1, vc1, bt = gpu_state(w)
+    kc2, vc2, _ = gpu_state(w)
+    okc, ovc = to_words(w.k_cache).copy(), to_words(w.v_cache).copy()
+    for step in range(3):
+        si = step_inputs(w, step)
+        d = {k: v.cuda() for k, v in si.items()}
+        o1 = kvd.kvd_decode_step(d["q"], d["k_new"], d["v_new"], kc1, vc1, bt, d["seq_lens"], w.scale)
+        o2 = kvd.kvd_decode_attention_shared_prefix(d["q"], kc2, vc2, bt, d["seq_lens"], gs, gp, per,
+                                                    w.scale, k_new=d["k_new"], v_new=d["v_new"])
+        torch.cuda.synchronize()
+        okc, ovc, ref = oracle_step(w, si, okc, ovc)
+        assert max_err(o2, ref) <= TOL[w.dtype]
+        assert torch.max(torch.abs(o1.float() - o2.float())).item() <= TOL[w.dtype]
+    assert torch.equal(kc1.view(torch.int16), kc2.view(torch.int16))
+    assert torch.equal(vc1.view(torch.int16), vc2.view(torch.int16))
+    assert np.array_equal(to_words(kc2), okc)
+    assert kvd.kvd_read_device_error() == 0
+
+
+def test_shared_prefix_member_shorter_than_prefix_is_attended_whole(kvd):
+    # group claims 4 shared pages, but member 1 has only 40 tokens: it must
+    # fall back to plain attention and still match the oracle
+    lens = [90, 40, 100, 120]
+    w = build_workload("spshort", 4, 8, 2, 128, "f16", lens, seed=961)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    kvd.kvd_append(kc, vc, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    # make sequences 0 and 1 share sequence 0's first 4 pages in the table
+    bt2 = bt.clone()
+    bt2[1, :3] = bt[0, :3]
+    kc_h, vc_h = kc.cpu(), vc.cpu()
+    gs = torch.tensor([0, 2, 4], dtype=torch.int32).cuda()
+    gp = torch.tensor([4, 0], dtype=torch.int32).cuda()
+    out = kvd.kvd_decode_attention_shared_prefix(si["q"].cuda(), kc, vc, bt2, si["seq_lens"].cuda(),
+                                                 gs, gp, 2, w.scale)
+    torch.cuda.synchronize()
+    q = to_words(si["q"])
+    ref, _ = oracle.attend(q, to_words(kc_h), to_words(vc_h), bt2.cpu().numpy(),
+                           si["seq_lens"].numpy(), w.scale, oracle.F16)
+    err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
+    assert err <= TOL[w.dtype]
