@@ -52,6 +52,17 @@ def load(path):
     L.orc_merge.argtypes = [P, P, P, i32, i32, i32, i32, P, P]
     L.orc_max_threads.restype = i32
     L.orc_max_threads.argtypes = []
+    L.orc_e4m3_decode.restype = ctypes.c_double
+    L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.orc_e4m3_encode.restype = ctypes.c_uint8
+    L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+    L.orc_quantize_fp8.restype = i32
+    L.orc_quantize_fp8.argtypes = [P, i32, i32, i32, P, P]
+    L.orc_append_fp8.restype = i32
+    L.orc_append_fp8.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32]
+    L.orc_attend_fp8.restype = i32
+    L.orc_attend_fp8.argtypes = [P, P, P, P, P, P, P, ctypes.c_double, i32, i32, i32, i32, i32,
+                                 i32, i32, P, P, i32]
     return L
 
 
@@ -175,3 +186,59 @@ def merge(part_o, part_lse, counts=None):
 
 def max_threads():
     return int(lib().orc_max_threads())
+
+
+# ------------------------------------------------------------ 8-bit KV cache
+
+FP8_GROUP = 32
+
+
+def e4m3_decode(code):
+    return lib().orc_e4m3_decode(int(code))
+
+
+def e4m3_encode(x):
+    return int(lib().orc_e4m3_encode(float(x)))
+
+
+def quantize_fp8(rows, dtype):
+    """rows [..., d] storage words -> (codes uint8 [..., d], scales float32 [..., d/32])."""
+    rows = _words(rows)
+    d = rows.shape[-1]
+    n = rows.size // d
+    codes = np.zeros(rows.shape, dtype=np.uint8)
+    scales = np.zeros(rows.shape[:-1] + (d // FP8_GROUP,), dtype=np.float32)
+    _check(lib().orc_quantize_fp8(_ptr(rows), n, d, dtype, _ptr(codes), _ptr(scales)),
+           "orc_quantize_fp8")
+    return codes, scales
+
+
+def append_fp8(k8, v8, ks, vs, block_table, slot, k_new, v_new, dtype):
+    """In-place quantised scatter into codes [NB,H_kv,16,d] and scales [NB,H_kv,16,d/32]."""
+    for a in (k8, v8):
+        assert a.dtype == np.uint8 and a.flags.c_contiguous
+    for a in (ks, vs):
+        assert a.dtype == np.float32 and a.flags.c_contiguous
+    k_new, v_new = _words(k_new), _words(v_new)
+    bt, sl = _i32(block_table), _i32(slot)
+    NB, H_kv, P, d = k8.shape
+    _check(lib().orc_append_fp8(_ptr(k8), _ptr(v8), _ptr(ks), _ptr(vs), _ptr(bt), _ptr(sl),
+                                _ptr(k_new), _ptr(v_new), k_new.shape[0], H_kv, d, NB,
+                                bt.shape[1], dtype),
+           "orc_append_fp8")
+
+
+def attend_fp8(q, k8, v8, ks, vs, block_table, seq_lens, scale, dtype, nthreads=0):
+    """Attention (binary64) over the dequantised 8-bit cache -> (out, lse)."""
+    q = _words(q)
+    bt, sl = _i32(block_table), _i32(seq_lens)
+    B, H_q, d = q.shape
+    NB, H_kv, P, _ = k8.shape
+    out = np.zeros((B, H_q, d), dtype=np.float64)
+    lse = np.zeros((B, H_q), dtype=np.float64)
+    _check(lib().orc_attend_fp8(_ptr(q), _ptr(np.ascontiguousarray(k8)), _ptr(np.ascontiguousarray(v8)),
+                                _ptr(np.ascontiguousarray(ks)), _ptr(np.ascontiguousarray(vs)),
+                                _ptr(bt), _ptr(sl), float(scale), B, H_q, H_kv, d, NB,
+                                bt.shape[1], dtype, _ptr(out), _ptr(lse), int(nthreads)),
+           "orc_attend_fp8")
+    return out, lse

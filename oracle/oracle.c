@@ -23,6 +23,10 @@
  *                                        closed forms, GQA == repeated-head MHA
  *   orc_attend_tiled                  -- equals orc_attend (flash is exact)
  *   orc_merge                         -- merge of disjoint partitions == one shot
+ *   orc_e4m3_decode / orc_e4m3_encode -- torch float8_e4m3fn (all codes; RN ties)
+ *   orc_quantize_fp8 / orc_append_fp8 -- round-trip bound, per-group scales,
+ *                                        outlier isolation, == numpy re-derivation
+ *   orc_attend_fp8                    -- CPU float64 SDPA on the dequantised cache
  */
 #include <math.h>
 #include <stdint.h>
@@ -307,6 +311,172 @@ int orc_merge(const double *part_o, const double *part_lse, const int32_t *count
         }
     }
     return ORC_OK;
+}
+
+/* ------------------------------------------------------- 8-bit KV cache */
+
+/* "KV Cache:推理慢的真正原因", section "工程优化手段 / 量化": the cache is stored in
+ * 8 bits; because a few keys are very large, the scale is taken per channel
+ * group rather than one for the whole tensor.  "KV缓存与Flash注意力", section
+ * "实际应用" (serving with an fp8 KV cache).  Reading taken here: FP8 E4M3
+ * codes with one fp32 scale per (token, KV head, group of 32 channels);
+ * s = max|x| / 448 (448 = largest E4M3 value), code = E4M3(x / s) rounded to
+ * nearest (ties to even), saturating at +-448; both divisions are IEEE fp32
+ * (the precision the kernels use, since the fp32 quotient decides the code).
+ * A group of zeros gets s = 0 and codes 0.  Dequantised value: s * E4M3(code). */
+#define ORC_FP8_GROUP 32
+
+/* E4M3 ("fn" variant): 1 sign, 4 exponent bits (bias 7), 3 fraction bits; no
+ * infinities; exponent 15 with fraction 7 is NaN; subnormals fraction * 2^-9. */
+double orc_e4m3_decode(uint8_t c)
+{
+    int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp((double)(8 + m), e - 10);
+    return sign ? -v : v;
+}
+
+uint8_t orc_e4m3_encode(float x)
+{
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a < ldexp(1.0, -6)) {                 /* subnormal range: multiples of 2^-9 */
+        double r = rint(a / ldexp(1.0, -9));  /* nearest, ties to even; 8 = smallest normal */
+        return sign | (uint8_t)r;
+    }
+    int e2;
+    frexp(a, &e2);                            /* a = f * 2^e2, f in [0.5, 1) */
+    int E = e2 - 1;                           /* a = 1.xxx * 2^E */
+    double r = rint(a / ldexp(1.0, E - 3));   /* in [8, 16] */
+    if (r == 16.0) { r = 8.0; E += 1; }
+    int biased = E + 7;
+    int frac = (int)r - 8;
+    if (biased > 15 || (biased == 15 && frac == 7)) return sign | 0x7E;   /* saturate at 448 */
+    return sign | (uint8_t)((biased << 3) | frac);
+}
+
+/* Quantise n rows of d storage words (fp16/bf16) into codes [n][d] and
+ * scales [n][d / 32]. */
+int orc_quantize_fp8(const uint16_t *rows, int n, int d, int dtype, uint8_t *codes, float *scales)
+{
+    if (!rows || !codes || !scales || n < 0 || d <= 0 || d % ORC_FP8_GROUP) return ORC_ERR_ARGS;
+    const int ng = d / ORC_FP8_GROUP;
+    for (long long r = 0; r < n; ++r) {
+        for (int g = 0; g < ng; ++g) {
+            const uint16_t *x = rows + r * d + g * ORC_FP8_GROUP;
+            float mx = 0.0f;
+            for (int i = 0; i < ORC_FP8_GROUP; ++i) {
+                float v = (float)fabs(decode_elem(x[i], dtype));
+                if (v > mx) mx = v;
+            }
+            volatile float s = mx / 448.0f;
+            scales[r * ng + g] = s;
+            for (int i = 0; i < ORC_FP8_GROUP; ++i) {
+                float v = (float)decode_elem(x[i], dtype);
+                volatile float q = s == 0.0f ? 0.0f : v / s;
+                codes[r * d + g * ORC_FP8_GROUP + i] = s == 0.0f ? 0 : orc_e4m3_encode(q);
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* Append for the 8-bit cache: quantise k_new/v_new [B][H_kv][d] and write the
+ * codes and scales of row slot[b] % 16 of page block_table[b][slot[b] / 16]
+ * (codes [NB][H_kv][16][d], scales [NB][H_kv][16][d/32]). */
+int orc_append_fp8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t *block_table,
+                   const int32_t *slot, const uint16_t *k_new, const uint16_t *v_new, int B,
+                   int H_kv, int d, int num_blocks, int max_blocks, int dtype)
+{
+    if (!k8 || !v8 || !ks || !vs || !block_table || !slot || !k_new || !v_new) return ORC_ERR_ARGS;
+    if (d % ORC_FP8_GROUP) return ORC_ERR_ARGS;
+    const int ng = d / ORC_FP8_GROUP;
+    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    float *sc = (float *)malloc((size_t)ng * sizeof(float));
+    if (!code || !sc) { free(code); free(sc); return ORC_ERR_NOMEM; }
+    int rc = ORC_OK;
+    for (int b = 0; b < B && rc == ORC_OK; ++b) {
+        int pos = slot[b];
+        if (pos < 0) continue;
+        int logical = pos / ORC_PAGE_TOKENS, row = pos % ORC_PAGE_TOKENS;
+        if (logical >= max_blocks) { rc = ORC_ERR_RANGE; break; }
+        int phys = block_table[(size_t)b * max_blocks + logical];
+        if (phys < 0 || phys >= num_blocks) { rc = ORC_ERR_RANGE; break; }
+        for (int h = 0; h < H_kv; ++h) {
+            size_t r = ((size_t)phys * H_kv + h) * ORC_PAGE_TOKENS + row;
+            size_t src = ((size_t)b * H_kv + h) * (size_t)d;
+            orc_quantize_fp8(k_new + src, 1, d, dtype, code, sc);
+            memcpy(k8 + r * d, code, (size_t)d);
+            memcpy(ks + r * ng, sc, (size_t)ng * sizeof(float));
+            orc_quantize_fp8(v_new + src, 1, d, dtype, code, sc);
+            memcpy(v8 + r * d, code, (size_t)d);
+            memcpy(vs + r * ng, sc, (size_t)ng * sizeof(float));
+        }
+    }
+    free(code);
+    free(sc);
+    return rc;
+}
+
+/* Attention over the 8-bit cache: exactly orc_attend's definition applied to
+ * the dequantised values s * E4M3(code) (binary64).  q is fp16/bf16 words. */
+int orc_attend_fp8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, const float *ks,
+                   const float *vs, const int32_t *block_table, const int32_t *seq_lens,
+                   double scale, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks,
+                   int dtype, double *out, double *lse, int nthreads)
+{
+    if (!q || !k8 || !v8 || !ks || !vs || !block_table || !seq_lens || !out) return ORC_ERR_ARGS;
+    if (B < 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv || d <= 0 || d % ORC_FP8_GROUP) return ORC_ERR_ARGS;
+    for (int b = 0; b < B; ++b)
+        if (seq_lens[b] < 0 || seq_lens[b] > max_blocks * ORC_PAGE_TOKENS) return ORC_ERR_RANGE;
+    const int G = H_q / H_kv, ng = d / ORC_FP8_GROUP;
+    int status = ORC_OK;
+    long long rows = (long long)B * H_q;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (long long r = 0; r < rows; ++r) {
+        int b = (int)(r / H_q), hq = (int)(r % H_q), g = hq / G;
+        int n = seq_lens[b];
+        double *o = out + (size_t)r * d;
+        for (int i = 0; i < d; ++i) o[i] = 0.0;
+        if (n == 0) { if (lse) lse[r] = -INFINITY; continue; }
+        double *s = (double *)malloc((size_t)n * sizeof(double));
+        double *qv = (double *)malloc((size_t)d * sizeof(double));
+        if (!s || !qv) { free(s); free(qv); status = ORC_ERR_NOMEM; continue; }
+        for (int i = 0; i < d; ++i) qv[i] = decode_elem(q[(size_t)r * d + i], dtype);
+        int bad = 0;
+        for (int j = 0; j < n; ++j) {
+            long long off = token_offset(block_table, b, j, g, H_kv, d, num_blocks, max_blocks);
+            if (off < 0) { bad = 1; break; }
+            const float *sk = ks + off / d * ng;
+            double dot = 0.0;
+            for (int i = 0; i < d; ++i)
+                dot += qv[i] * ((double)sk[i / ORC_FP8_GROUP] * orc_e4m3_decode(k8[off + i]));
+            s[j] = scale * dot;
+        }
+        if (bad) { free(s); free(qv); status = ORC_ERR_RANGE; continue; }
+        double m = -INFINITY;
+        for (int t = 0; t < n; ++t) if (s[t] > m) m = s[t];
+        double den = 0.0;
+        for (int j = 0; j < n; ++j) {
+            double w = exp(s[j] - m);
+            den += w;
+            long long off = token_offset(block_table, b, j, g, H_kv, d, num_blocks, max_blocks);
+            const float *sv = vs + off / d * ng;
+            for (int i = 0; i < d; ++i)
+                o[i] += w * ((double)sv[i / ORC_FP8_GROUP] * orc_e4m3_decode(v8[off + i]));
+        }
+        for (int i = 0; i < d; ++i) o[i] /= den;
+        if (lse) lse[r] = m + log(den);
+        free(s);
+        free(qv);
+    }
+    return status;
 }
 
 int orc_max_threads(void)

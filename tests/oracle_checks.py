@@ -352,6 +352,130 @@ def check_append():
     assert np.array_equal(got, contiguous[:, :n]), "paged append != contiguous append"
 
 
+# ------------------------------------------------------------ 8-bit cache
+
+def _torch_e4m3(x32):
+    """float32 array -> E4M3 codes via torch's float8_e4m3fn conversion."""
+    return torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32)).to(
+        torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def _torch_e4m3_value(codes):
+    return torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).view(
+        torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def check_e4m3_decoder():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = _torch_e4m3_value(codes)
+    got = np.array([oracle.e4m3_decode(c) for c in codes])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan), "E4M3 NaN codes differ"
+    assert np.array_equal(got[~nan], ref[~nan]), "E4M3 decoding differs from torch"
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9
+
+
+def check_e4m3_encoder():
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal(20000) * np.exp(rng.uniform(-12, 6, 20000))).astype(np.float32)
+    x = np.clip(x, -448, 448)
+    # every midpoint between neighbouring finite values: ties go to the even code
+    vals = np.unique(np.abs(_torch_e4m3_value(np.arange(0x7F, dtype=np.uint8))))
+    mids = ((vals[1:] + vals[:-1]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, -mids, vals.astype(np.float32)])
+    got = np.array([oracle.e4m3_encode(v) for v in x], dtype=np.uint8)
+    ref = _torch_e4m3(x)
+    assert np.array_equal(got, ref), f"{int(np.sum(got != ref))} E4M3 encodings differ from torch"
+    # saturation (torch turns these into NaN; the kernels' conversion saturates)
+    assert oracle.e4m3_encode(449.0) == 0x7E and oracle.e4m3_encode(-1000.0) == 0xFE
+
+
+def _quantize_numpy(rows_f32):
+    """Independent re-derivation: fp32 scale max|x|/448 per 32 channels, codes by torch."""
+    n, d = rows_f32.shape
+    g = rows_f32.reshape(n, d // 32, 32)
+    mx = np.abs(g).max(axis=2).astype(np.float32)
+    s = (mx / np.float32(448.0)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        qv = np.where(s[..., None] > 0, g / s[..., None], 0).astype(np.float32)
+    codes = _torch_e4m3(qv.reshape(n, d)).reshape(n, d)
+    return codes, s
+
+
+def check_quantize_fp8():
+    rng = np.random.default_rng(12)
+    for dt, tdt in ((oracle.F16, torch.float16), (oracle.BF16, torch.bfloat16)):
+        x = torch.from_numpy(rng.standard_normal((64, 128)).astype(np.float32))
+        x[3, 17] = 40.0                        # an outlier channel in group 0 of row 3
+        x[5, 64:96] = 0.0                      # an all-zero group
+        xq = x.to(tdt)
+        words = to_words(xq)
+        codes, scales = oracle.quantize_fp8(words, dt)
+        rows32 = xq.to(torch.float32).numpy()
+        rc, rs = _quantize_numpy(rows32)
+        assert np.array_equal(codes, rc), "codes differ from the numpy/torch re-derivation"
+        assert np.array_equal(scales, rs), "scales differ from the numpy re-derivation"
+        deq = _torch_e4m3_value(codes).reshape(64, 4, 32) * scales[..., None]
+        err = np.abs(deq.reshape(64, 128) - rows32)
+        # half an E4M3 ulp at the largest binade (448 -> ulp 32), in units of s;
+        # the tiny slack covers ties landing exactly on the half ulp
+        bound = scales.repeat(32, axis=1).astype(np.float64) * 16.0 * (1 + 1e-6) + 1e-30
+        assert np.all(err <= bound), "round trip exceeds half an E4M3 ulp"
+        assert scales[5, 2] == 0 and np.all(codes[5, 64:96] == 0)
+        # the outlier only coarsens its own group
+        assert scales[3, 0] > 10 * np.median(scales[:, 0]) and scales[3, 1] < 3 * np.median(scales[:, 1])
+
+
+def _fp8_case(B, H_q, H_kv, d, dt, lens, seed):
+    c = case(B, H_q, H_kv, d, dt, lens, seed)
+    k8, ks = oracle.quantize_fp8(c["kc"], c["dt"])
+    v8, vs = oracle.quantize_fp8(c["vc"], c["dt"])
+    c.update(k8=k8, ks=ks, v8=v8, vs=vs)
+    return c
+
+
+def check_attend_fp8_against_sdpa():
+    for (B, H_q, H_kv, d, dt, lens, seed) in [(2, 8, 2, 128, "bf16", [40, 77], 31),
+                                              (1, 4, 4, 64, "f16", [33], 32)]:
+        c = _fp8_case(B, H_q, H_kv, d, dt, lens, seed)
+        out, lse = oracle.attend_fp8(c["q"], c["k8"], c["v8"], c["ks"], c["vs"], c["bt"], c["sl"],
+                                     c["scale"], c["dt"])
+        G = H_q // H_kv
+        for b in range(B):
+            n = int(c["sl"][b])
+            j = np.arange(n)
+            pages, rows = c["bt"][b, j // 16], j % 16
+            Kd = _torch_e4m3_value(c["k8"][pages, :, rows, :]) * np.repeat(c["ks"][pages, :, rows, :], 32, axis=-1)
+            Vd = _torch_e4m3_value(c["v8"][pages, :, rows, :]) * np.repeat(c["vs"][pages, :, rows, :], 32, axis=-1)
+            K = torch.from_numpy(Kd.transpose(1, 0, 2)).repeat_interleave(G, dim=0)[None]
+            V = torch.from_numpy(Vd.transpose(1, 0, 2)).repeat_interleave(G, dim=0)[None]
+            q = torch.from_numpy(f64(c["q"][b], c["dt"]))[None, :, None, :]
+            ref = F.scaled_dot_product_attention(q, K, V, scale=c["scale"])[0, :, 0, :].numpy()
+            close(out[b], ref, 1e-12, 1e-12, "fp8 attention vs SDPA on dequantised K/V")
+        # quantisation error against the unquantised cache stays small
+        full, _ = run(c)
+        assert np.max(np.abs(out - full)) < 0.1, "fp8 attention far from fp16/bf16 attention"
+
+
+def check_append_fp8():
+    w = build_workload("pin8", 4, 4, 2, 128, "bf16", [1, 16, 17, 40], seed=83)
+    si = step_inputs(w, 0)
+    kc, vc = to_words(w.k_cache), to_words(w.v_cache)
+    k8, ks = oracle.quantize_fp8(kc, oracle.BF16)
+    v8, vs = oracle.quantize_fp8(vc, oracle.BF16)
+    k8_0, ks_0 = k8.copy(), ks.copy()
+    oracle.append_fp8(k8, v8, ks, vs, w.block_table.numpy(), si["slot"].numpy(),
+                      to_words(si["k_new"]), to_words(si["v_new"]), oracle.BF16)
+    kn8, kns = oracle.quantize_fp8(to_words(si["k_new"]), oracle.BF16)
+    bt = w.block_table.numpy()
+    changed = np.any(k8 != k8_0, axis=(1, 3))
+    for b, pos in enumerate(si["slot"].numpy()):
+        p, r = bt[b, pos // 16], pos % 16
+        assert np.array_equal(k8[p, :, r, :], kn8[b]) and np.array_equal(ks[p, :, r, :], kns[b])
+        changed[p, r] = False
+    assert not changed.any(), "fp8 append touched other rows"
+
+
 ALL_CHECKS = [
     check_f16_decoder,
     check_bf16_decoder,
@@ -366,4 +490,9 @@ ALL_CHECKS = [
     check_paging_invariance,
     check_shared_prefix_equals_private,
     check_append,
+    check_e4m3_decoder,
+    check_e4m3_encoder,
+    check_quantize_fp8,
+    check_attend_fp8_against_sdpa,
+    check_append_fp8,
 ]

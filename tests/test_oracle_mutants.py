@@ -35,6 +35,10 @@ MUTANTS = {
     "tiled_no_rescale": ("ssum = ssum * exp_old + tile_sum;", "ssum = ssum + tile_sum;"),
     "kv_bytes_no_kv_factor": ("return 2LL * (long long)dtype_size * layers * heads * d_head;",
                               "return (long long)dtype_size * layers * heads * d_head;"),
+    "fp8_scale_max": ("volatile float s = mx / 448.0f;", "volatile float s = mx / 240.0f;"),
+    "fp8_group_index": ("const float *sk = ks + off / d * ng;", "const float *sk = ks + off / d;"),
+    "fp8_round_down": ("double r = rint(a / ldexp(1.0, E - 3));", "double r = floor(a / ldexp(1.0, E - 3));"),
+    "fp8_decode_bias": ("else v = ldexp((double)(8 + m), e - 10);", "else v = ldexp((double)(8 + m), e - 9);"),
     "max_skips_first": ("for (int t = 0; t < n; ++t) if (s[t] > m) m = s[t];",
                         "for (int t = 1; t < n; ++t) if (s[t] > m) m = s[t];"),
 }
@@ -49,9 +53,11 @@ def source():
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_mutant_is_caught(name, source, tmp_path):
     old, new = MUTANTS[name]
-    assert source.count(old) == 1, f"mutation site for {name} not unique in oracle.c"
+    # the first occurrence is the plain attention's (the 8-bit path repeats a
+    # few lines after it); one planted mistake per mutant
+    assert source.count(old) >= 1, f"mutation site for {name} not found in oracle.c"
     src = tmp_path / "mutant.c"
-    src.write_text(source.replace(old, new), encoding="utf-8")
+    src.write_text(source.replace(old, new, 1), encoding="utf-8")
     lib = tmp_path / "libmutant.so"
     subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
                     "-ffp-contract=off", str(src), "-o", str(lib), "-lm"], check=True)
