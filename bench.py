@@ -58,6 +58,12 @@ def unique_attention_bytes(w, seq_lens) -> int:
     return toks * w.H_kv * 2 * w.d * s + 2 * w.B * w.H_q * w.d * s
 
 
+def fp8_attention_bytes(w, seq_lens) -> int:
+    """Attention bytes over the 8-bit cache: codes + fp32 group scales + q + out."""
+    per_tok = w.H_kv * 2 * (w.d + (w.d // 32) * 4)
+    return int(seq_lens.to(torch.int64).sum().item()) * per_tok + 2 * w.B * w.H_q * w.d * 2
+
+
 def append_bytes(w, slot) -> int:
     rows = int((slot >= 0).sum().item()) * w.H_kv
     return rows * w.d * 2 * 2 * 2          # K and V rows, read from k_new/v_new and written
@@ -297,6 +303,13 @@ def run_ours(args):
     ws = kvd.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, args.partitions, dev)
     stream = torch.cuda.current_stream()
 
+    f8 = None
+    if args.kv_fp8:
+        # the pool stored as E4M3 codes + per-32-channel fp32 scales
+        k8, ks = kvd.kvd_quantize_fp8(kc)
+        v8, vs = kvd.kvd_quantize_fp8(vc)
+        f8 = {"k8": k8, "v8": v8, "ks": ks, "vs": vs}
+
     sp = None
     if args.shared_prefix:
         if not w.groups:
@@ -309,6 +322,17 @@ def run_ours(args):
         ws = torch.empty(n, dtype=torch.uint8, device=dev)
 
     def step(ev_a=None, ev_b=None):
+        if f8 is not None:
+            kvd.kvd_append_fp8(f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, slot, k_new, v_new,
+                               stream=stream)
+            if ev_a is not None:
+                ev_a.record(stream)
+            kvd.kvd_decode_attention_fp8(q, f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, seq_lens,
+                                         w.scale, out=out, num_partitions=args.partitions,
+                                         workspace=ws, stream=stream)
+            if ev_b is not None:
+                ev_b.record(stream)
+            return
         if sp is not None:
             if ev_a is not None:
                 ev_a.record(stream)
@@ -334,9 +358,12 @@ def run_ours(args):
 
     a_bytes = attention_bytes(w, si["seq_lens"])
     p_bytes = append_bytes(w, si["slot"])
+    if f8 is not None:
+        a_bytes = fp8_attention_bytes(w, si["seq_lens"])
+        p_bytes = int((si["slot"] >= 0).sum().item()) * w.H_kv * 2 * (w.d * 2 + w.d + (w.d // 32) * 4)
     step_bytes = a_bytes + p_bytes
     # bytes of the call the roofline times (events bracket it)
-    timed_bytes = a_bytes if args.separate_append else step_bytes
+    timed_bytes = a_bytes if (args.separate_append or f8 is not None) else step_bytes
 
     graph = None
     if args.graph:
@@ -399,7 +426,7 @@ def run_ours(args):
 
     # ---- end to end through the public API with pinned host buffers
     inputs = [("q", q), ("k_new", k_new), ("v_new", v_new), ("seq_lens", seq_lens)]
-    if args.separate_append:
+    if args.separate_append or f8 is not None:
         inputs.append(("slot", slot))
     h_in = {n: t.cpu().pin_memory() for n, t in inputs}
     d_in = {n: torch.empty_like(t, device=dev) for n, t in h_in.items()}
@@ -411,7 +438,14 @@ def run_ours(args):
     def e2e_step():
         for n in h_in:
             d_in[n].copy_(h_in[n], non_blocking=True)
-        if sp is not None:
+        if f8 is not None:
+            kvd.kvd_append_fp8(f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, d_in["slot"],
+                               d_in["k_new"], d_in["v_new"], stream=stream)
+            kvd.kvd_decode_attention_fp8(d_in["q"], f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt,
+                                         d_in["seq_lens"], w.scale, out=out,
+                                         num_partitions=args.partitions, workspace=ws,
+                                         stream=stream)
+        elif sp is not None:
             kvd.kvd_decode_attention_shared_prefix(d_in["q"], kc, vc, bt, d_in["seq_lens"], sp["start"],
                                                    sp["pages"], sp["max"], w.scale, out=out,
                                                    k_new=d_in["k_new"], v_new=d_in["v_new"],
@@ -463,7 +497,7 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": w.dtype_name,
+        "dtype": ("e4m3 cache, " + w.dtype_name + " q/out") if f8 is not None else w.dtype_name,
         "data": "synthetic",
         "config": {
             "workload": w.name if args.scale_down == 1 else f"{w.name}/scale_down={args.scale_down}",
@@ -473,7 +507,9 @@ def run_ours(args):
             "bytes_per_step": step_bytes, "attention_bytes": a_bytes, "append_bytes": p_bytes,
             "l2": "inputs larger than L2 (KV pool %.2f GB >> 126 MB); no flush" % (
                 2 * w.k_cache.numel() * 2 / 1e9),
-            "step": ("kvd_decode_attention_shared_prefix with fused append (prefix, decode, merge kernels)"
+            "step": ("kvd_append_fp8 + kvd_decode_attention_fp8 over an E4M3 cache "
+                     "(2 quantise, decode, merge kernels)" if f8 is not None else
+                     "kvd_decode_attention_shared_prefix with fused append (prefix, decode, merge kernels)"
                      if sp is not None else
                      "kvd_append + kvd_decode_attention (append, decode, merge kernels)"
                      if args.separate_append else
@@ -488,7 +524,9 @@ def run_ours(args):
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "peak_kind": peak_kind,
-            "kernel": ("kvd_decode_attention call (decode_kernel + decode_merge_kernel)"
+            "kernel": ("kvd_decode_attention_fp8 call (decode_kernel over E4M3 pages + merge)"
+                       if f8 is not None else
+                       "kvd_decode_attention call (decode_kernel + decode_merge_kernel)"
                        if args.separate_append else
                        "kvd_decode_step call (decode_kernel with fused append + decode_merge_kernel)")
                       + ", CUDA events on the launching stream; achieved = its algorithmic bytes / mean duration",
@@ -510,7 +548,8 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "us_per_step": round(e2e_s / e2e_steps * 1e6, 2),
                 "how": "pinned host inputs -> H2D, append, decode, D2H of out, stream sync; wall clock"},
-        "gpu_launches": (3 if (args.separate_append or sp is not None) else 2) * args.steps * per,
+        "gpu_launches": (4 if f8 is not None else 3 if (args.separate_append or sp is not None)
+                         else 2) * args.steps * per,
         "graph": ({"steps_per_graph": args.graph_steps, "replays": args.steps} if graph is not None
                   else None),
         "clocks": clocks,
@@ -540,6 +579,8 @@ def main(argv=None):
     p.add_argument("--separate-append", action="store_true",
                    help="time kvd_append + kvd_decode_attention instead of the fused kvd_decode_step")
     p.add_argument("--e2e-steps", type=int, default=300)
+    p.add_argument("--kv-fp8", action="store_true",
+                   help="store the cache as FP8 E4M3 codes with per-32-channel scales (d=128)")
     p.add_argument("--shared-prefix", action="store_true",
                    help="read each group's shared prefix pages once (kvd_decode_attention_shared_prefix)")
     p.add_argument("--graph", action="store_true",
@@ -555,7 +596,7 @@ def main(argv=None):
     args = p.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.graph and (args.separate_append or args.shared_prefix):
+    if args.graph and (args.separate_append or args.shared_prefix or args.kv_fp8):
         raise SystemExit("--graph times the fused step only")
     if args.impl == "reference":
         return run_reference(args)

@@ -180,6 +180,41 @@ kvd_status kvd_decode_attention_shared_prefix(
 size_t kvd_shared_prefix_workspace_size(int B, int H_q, int H_kv, int d, int n_groups,
                                         int max_group_size, int num_partitions);
 
+/*
+ * 8-bit (FP8 E4M3) KV cache.
+ * [BLOG] section "工程优化手段 / 量化" (store the cache in 8 bits; a few very large
+ * keys would swamp one tensor-wide scale, so scale per channel group); [LES]
+ * section "实际应用" (serving with an fp8 KV cache).
+ * Format: codes uint8 [num_blocks][H_kv][16][d]; scales float [num_blocks]
+ * [H_kv][16][d/32]: one per (token, KV head, group of 32 channels), with
+ * s = max|x| / 448 over the group and code = E4M3(x / s) (round to nearest
+ * even, saturating; both divisions IEEE fp32); value = s * E4M3(code).
+ *
+ * kvd_quantize_fp8   n_rows rows of d fp16/bf16 values (device [n_rows][d])
+ *                    -> codes [n_rows][d] and scales [n_rows][d/32]
+ *                    (e.g. to fill a cache after prefill).  d in {32..128}, step 32.
+ * kvd_append_fp8     the append of kvd_append for the 8-bit cache: quantise
+ *                    k_new/v_new [B][H_kv][d] into row slot % 16 of page
+ *                    block_table[b][slot / 16] of codes and scales.
+ * kvd_decode_attention_fp8
+ *                    kvd_decode_attention over the 8-bit cache (d = 128):
+ *                    softmax(scale q K^T) V with K, V the dequantised values;
+ *                    q and out in dtype; workspace as kvd_decode_attention.
+ */
+kvd_status kvd_quantize_fp8(const void *src, uint8_t *codes, float *scales, long long n_rows,
+                            int d, kvd_dtype dtype, void *stream);
+kvd_status kvd_append_fp8(uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
+                          const int32_t *block_table, const int32_t *slot, const void *k_new,
+                          const void *v_new, int B, int H_kv, int d, int num_blocks,
+                          int max_blocks_per_seq, kvd_dtype dtype, void *stream);
+kvd_status kvd_decode_attention_fp8(const void *q, const uint8_t *k_codes, const uint8_t *v_codes,
+                                    const float *k_scale, const float *v_scale,
+                                    const int32_t *block_table, const int32_t *seq_lens,
+                                    float scale, void *out, int B, int H_q, int H_kv, int d,
+                                    int num_blocks, int max_blocks_per_seq, int num_partitions,
+                                    void *workspace, size_t workspace_bytes, float *lse_out,
+                                    kvd_dtype dtype, void *stream);
+
 /* Bytes of the library's fixed scratch array used by kvd_decode_attention_static. */
 #define KVD_STATIC_WORKSPACE_BYTES (8u << 20)
 

@@ -22,6 +22,7 @@ __all__ = [
     "KVD_F16", "KVD_BF16", "KVD_PAGE_TOKENS", "KvdError",
     "kvd_append", "kvd_decode_attention", "kvd_decode_step", "kvd_decode_attention_static",
     "kvd_decode_attention_shared_prefix", "kvd_shared_prefix_workspace_size",
+    "kvd_quantize_fp8", "kvd_append_fp8", "kvd_decode_attention_fp8",
     "kvd_merge_lse",
     "kvd_workspace_size", "KVD_STATIC_WORKSPACE_BYTES",
     "kvd_auto_partitions", "kvd_kv_bytes_per_token", "kvd_read_device_error",
@@ -59,6 +60,14 @@ def _load():
                                                      P, P, I, I, I, P, S, P, I, P]
     L.kvd_shared_prefix_workspace_size.restype = S
     L.kvd_shared_prefix_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    LL = ctypes.c_longlong
+    L.kvd_quantize_fp8.restype = I
+    L.kvd_quantize_fp8.argtypes = [P, P, P, LL, I, I, P]
+    L.kvd_append_fp8.restype = I
+    L.kvd_append_fp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+    L.kvd_decode_attention_fp8.restype = I
+    L.kvd_decode_attention_fp8.argtypes = [P, P, P, P, P, P, P, F, P, I, I, I, I, I, I, I, P, S, P,
+                                           I, P]
     L.kvd_decode_attention_static.restype = I
     L.kvd_decode_attention_static.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, P, I, P]
     L.kvd_merge_lse.restype = I
@@ -266,6 +275,59 @@ def kvd_decode_attention_shared_prefix(q, k_cache, v_cache, block_table, seq_len
         n_groups, int(max_group_size), int(num_partitions), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), lse_ptr, _dtype_code(k_cache), _stream(stream)),
         "kvd_decode_attention_shared_prefix")
+    return out
+
+
+def kvd_quantize_fp8(src, codes=None, scales=None, stream=None):
+    """Quantise rows src [..., d] (fp16/bf16) into E4M3 codes (uint8 [..., d])
+    and fp32 scales [..., d/32], one per 32 channels.  Returns (codes, scales)."""
+    d = src.shape[-1]
+    n = src.numel() // d
+    if codes is None:
+        codes = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+    if scales is None:
+        scales = torch.empty(src.shape[:-1] + (d // 32,), dtype=torch.float32, device=src.device)
+    _check(_lib.kvd_quantize_fp8(_dev(src, "src"), _dev(codes, "codes", torch.uint8),
+                                 _dev(scales, "scales", torch.float32), n, d, _dtype_code(src),
+                                 _stream(stream)),
+           "kvd_quantize_fp8")
+    return codes, scales
+
+
+def kvd_append_fp8(k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, stream=None):
+    """kvd_append for the 8-bit cache (codes [NB,H_kv,16,d], scales [NB,H_kv,16,d/32])."""
+    NB, H_kv, P, d = k_codes.shape
+    B = k_new.shape[0]
+    _check(_lib.kvd_append_fp8(_dev(k_codes, "k_codes", torch.uint8), _dev(v_codes, "v_codes", torch.uint8),
+                               _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+                               _dev(block_table, "block_table", torch.int32), _dev(slot, "slot", torch.int32),
+                               _dev(k_new, "k_new", k_new.dtype), _dev(v_new, "v_new", k_new.dtype),
+                               B, H_kv, d, NB, block_table.shape[1], _dtype_code(k_new), _stream(stream)),
+           "kvd_append_fp8")
+
+
+def kvd_decode_attention_fp8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale=None,
+                             out=None, num_partitions=0, workspace=None, lse_out=None, stream=None):
+    """kvd_decode_attention over the 8-bit cache (d = 128).  Returns out (q's dtype)."""
+    B, H_q, d = q.shape
+    NB, H_kv, P, d2 = k_codes.shape
+    if P != KVD_PAGE_TOKENS or d2 != d:
+        raise ValueError("q / cache shape mismatch")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(B, H_q, H_kv, d, num_partitions, q.device)
+    lse_ptr = None if lse_out is None else _dev(lse_out, "lse_out", torch.float32)
+    _check(_lib.kvd_decode_attention_fp8(
+        _dev(q, "q", q.dtype), _dev(k_codes, "k_codes", torch.uint8), _dev(v_codes, "v_codes", torch.uint8),
+        _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+        _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
+        float(scale), _dev(out, "out", q.dtype), B, H_q, H_kv, d, NB, block_table.shape[1],
+        int(num_partitions), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        lse_ptr, _dtype_code(q), _stream(stream)),
+        "kvd_decode_attention_fp8")
     return out
 
 

@@ -261,7 +261,9 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
                               const void *k_new, const void *v_new,
                               const int32_t *group_start = nullptr,
                               const int32_t *group_pages = nullptr, int n_groups = 0,
-                              int max_group_size = 0) {
+                              int max_group_size = 0, const float *k_scale = nullptr,
+                              const float *v_scale = nullptr) {
+  const bool fp8 = k_scale != nullptr;
   kvd_status st = check_heads(B, H_q, H_kv, d);
   if (st) return st;
   if (num_blocks <= 0 || max_blocks_per_seq <= 0)
@@ -273,6 +275,14 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
     return fail(KVD_ERR_UNSUPPORTED, "max_blocks_per_seq too large");
   if (!(scale == scale)) return fail(KVD_ERR_INVALID, "scale is NaN");
   if (num_partitions < 0) return fail(KVD_ERR_INVALID, "num_partitions < 0");
+  if (fp8) {
+    if (d != 128) return fail(KVD_ERR_UNSUPPORTED, "the 8-bit cache supports d = 128 only");
+    if (!v_scale) return fail(KVD_ERR_INVALID, "v_scale is NULL");
+    if (k_new || n_groups > 0)
+      return fail(KVD_ERR_UNSUPPORTED, "the 8-bit cache has no fused append or shared-prefix mode");
+    if (!aligned(k_scale, 16) || !aligned(v_scale, 16))
+      return fail(KVD_ERR_INVALID, "scale pools must be 16-byte aligned");
+  }
   if (B == 0) return KVD_OK;
   if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out)
     return fail(KVD_ERR_INVALID, "a required pointer is NULL");
@@ -310,23 +320,35 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   st = encoder(&encode);
   if (st) return st;
 
-  // K and V pools as 3-D tensors {64 elements, d/64 units, num_blocks*H_kv*16
-  // rows}; one box = one 64-element half of one page of one head (16 rows x
-  // 64), 128-byte swizzled.
   CUtensorMap tm[2];
   const void *pools[2] = {k_cache, v_cache};
   for (int i = 0; i < 2; ++i) {
-    cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(d / 64),
-                          static_cast<cuuint64_t>(num_blocks) * H_kv * KVD_PAGE_TOKENS};
-    cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(d) * 2};
-    cuuint32_t box[3] = {64, 1, KVD_PAGE_TOKENS};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = encode(&tm[i],
-                        dtype == KVD_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                        3, const_cast<void *>(pools[i]), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r;
+    if (fp8) {
+      // E4M3 code pools as 2-D byte tensors {128, num_blocks*H_kv*16 rows};
+      // one box = the 16 rows of one page of one head, 128-byte swizzled.
+      cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(num_blocks) * H_kv * KVD_PAGE_TOKENS};
+      cuuint64_t strides[1] = {128};
+      cuuint32_t box[2] = {128, KVD_PAGE_TOKENS};
+      cuuint32_t estr[2] = {1, 1};
+      r = encode(&tm[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(pools[i]), dims,
+                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+      // K and V pools as 3-D tensors {64 elements, d/64 units, num_blocks*H_kv*16
+      // rows}; one box = one 64-element half of one page of one head (16 rows x
+      // 64), 128-byte swizzled.
+      cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(d / 64),
+                            static_cast<cuuint64_t>(num_blocks) * H_kv * KVD_PAGE_TOKENS};
+      cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(d) * 2};
+      cuuint32_t box[3] = {64, 1, KVD_PAGE_TOKENS};
+      cuuint32_t estr[3] = {1, 1, 1};
+      r = encode(&tm[i],
+                 dtype == KVD_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                 3, const_cast<void *>(pools[i]), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
     if (r != CUDA_SUCCESS) return fail(KVD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   }
 
@@ -359,6 +381,8 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   a.pre_o = nullptr;
   a.pre_lse = nullptr;
   a.pre_chunks = 0;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
 
   const kvd::DType dt = dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -391,7 +415,8 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
     a.pre_lse = pa.pre_lse;
     a.pre_chunks = PL.chunks;
   }
-  e = kvd::launch_decode(a, d, dt, tm[0], tm[1], s, N);
+  e = fp8 ? kvd::launch_decode_fp8(a, dt, tm[0], tm[1], s, N)
+          : kvd::launch_decode(a, d, dt, tm[0], tm[1], s, N);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   e = kvd::launch_decode_merge(a, d, dt, s);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
@@ -409,6 +434,73 @@ kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *
   return decode_impl(q, k_cache, v_cache, block_table, seq_lens, scale, out, B, H_q, H_kv, d,
                      num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
                      lse_out, dtype, stream, nullptr, nullptr);
+}
+
+kvd_status kvd_quantize_fp8(const void *src, uint8_t *codes, float *scales, long long n_rows,
+                            int d, kvd_dtype dtype, void *stream) {
+  if (n_rows < 0) return fail(KVD_ERR_INVALID, "n_rows < 0");
+  if (d <= 0 || d % 32 || d > 128) return fail(KVD_ERR_UNSUPPORTED, "d must be 32, 64, 96 or 128");
+  if (dtype != KVD_F16 && dtype != KVD_BF16) return fail(KVD_ERR_INVALID, "unknown dtype %d", (int)dtype);
+  if (n_rows == 0) return KVD_OK;
+  if (!src || !codes || !scales) return fail(KVD_ERR_INVALID, "a required pointer is NULL");
+  if (!aligned(src, 8) || !aligned(codes, 4) || !aligned(scales, 4))
+    return fail(KVD_ERR_INVALID, "misaligned buffer");
+  kvd::QuantArgs q{src, codes, scales, nullptr, nullptr, nullptr, n_rows, d, 1, 1, 1, 0};
+  cudaError_t e = kvd::launch_quantize_fp8(q, dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16,
+                                           static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return KVD_OK;
+}
+
+kvd_status kvd_append_fp8(uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
+                          const int32_t *block_table, const int32_t *slot, const void *k_new,
+                          const void *v_new, int B, int H_kv, int d, int num_blocks,
+                          int max_blocks_per_seq, kvd_dtype dtype, void *stream) {
+  if (B < 0) return fail(KVD_ERR_INVALID, "B = %d < 0", B);
+  if (H_kv <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+    return fail(KVD_ERR_INVALID, "H_kv, num_blocks and max_blocks_per_seq must be positive");
+  if (d <= 0 || d % 32 || d > 128) return fail(KVD_ERR_UNSUPPORTED, "d must be 32, 64, 96 or 128");
+  if (dtype != KVD_F16 && dtype != KVD_BF16) return fail(KVD_ERR_INVALID, "unknown dtype %d", (int)dtype);
+  if (B == 0) return KVD_OK;
+  if (!k_codes || !v_codes || !k_scale || !v_scale || !block_table || !slot || !k_new || !v_new)
+    return fail(KVD_ERR_INVALID, "a required pointer is NULL");
+  if (!aligned(k_new, 8) || !aligned(v_new, 8) || !aligned(k_codes, 4) || !aligned(v_codes, 4) ||
+      !aligned(k_scale, 4) || !aligned(v_scale, 4))
+    return fail(KVD_ERR_INVALID, "misaligned buffer");
+  int dev;
+  unsigned *err;
+  kvd_status st = current_device(&dev);
+  if (st) return st;
+  st = error_word(dev, &err);
+  if (st) return st;
+  const kvd::DType dt = dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long n = static_cast<long long>(B) * H_kv;
+  kvd::QuantArgs qk{k_new, k_codes, k_scale, block_table, slot, err, n, d, H_kv, num_blocks,
+                    max_blocks_per_seq, 1};
+  cudaError_t e = kvd::launch_quantize_fp8(qk, dt, s);
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  kvd::QuantArgs qv = qk;
+  qv.src = v_new;
+  qv.codes = v_codes;
+  qv.scales = v_scale;
+  e = kvd::launch_quantize_fp8(qv, dt, s);
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  return KVD_OK;
+}
+
+kvd_status kvd_decode_attention_fp8(const void *q, const uint8_t *k_codes, const uint8_t *v_codes,
+                                    const float *k_scale, const float *v_scale,
+                                    const int32_t *block_table, const int32_t *seq_lens,
+                                    float scale, void *out, int B, int H_q, int H_kv, int d,
+                                    int num_blocks, int max_blocks_per_seq, int num_partitions,
+                                    void *workspace, size_t workspace_bytes, float *lse_out,
+                                    kvd_dtype dtype, void *stream) {
+  if (!k_scale) return fail(KVD_ERR_INVALID, "k_scale is NULL");
+  return decode_impl(q, k_codes, v_codes, block_table, seq_lens, scale, out, B, H_q, H_kv, d,
+                     num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
+                     lse_out, dtype, stream, nullptr, nullptr, nullptr, nullptr, 0, 0, k_scale,
+                     v_scale);
 }
 
 size_t kvd_shared_prefix_workspace_size(int B, int H_q, int H_kv, int d, int n_groups,

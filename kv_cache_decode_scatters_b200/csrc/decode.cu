@@ -49,35 +49,135 @@ namespace kvd {
 
 namespace {
 
-template <int D, int NT, int W, int S>
+template <int D, int NT, int W, int S, int kStride>
 struct Geo {
-  static constexpr int kPageBytes = kPage * D * 2;      // one K (or V) page of one head
-  static constexpr int kStageBytes = 2 * kPageBytes;    // K page then V page
+  static constexpr int kStageBytes = kStride;           // smem stride of one ring stage
   static constexpr int kThreads = 32 * W;
   static constexpr int kSteps = D / 16;                 // k-steps of S, m-tiles of O
   static constexpr int kEdgeFloats = 8 * NT * D;        // one parked accumulator tile
-  static_assert(kEdgeFloats * 4 <= kStageBytes, "a parked tile must fit in one stage");
+  static_assert(kEdgeFloats * 4 <= S * kStageBytes, "a parked tile must fit in a warp's ring");
+  static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
   static size_t smem(int B) {
     return 1024 + (size_t)W * S * kStageBytes + (size_t)W * kEdgeFloats * 4 + (size_t)W * S * 24 +
            (size_t)W * 2 * 2 * 8 * NT * 4 + (size_t)W * 2 * 4 + (size_t)(B + 1) * 4;
   }
 };
 
+}  // namespace
 
+// ---------------------------------------------------------- page formats
+//
+// What the decode kernel needs to know about a page format: how to copy a
+// page of one KV head into a ring stage, how to clear the rows past the
+// sequence end, the tensor-core step over a staged page, how q feeds it, and
+// which output channel each accumulator element holds.
+
+// fp16 / bf16 pages: [16 tokens][d] per (page, head), d/64 swizzled boxes.
+template <int D, int NT, typename T>
+struct Page16 {
+  using Out = T;
+  static constexpr bool kPatchable = true;  // supports the fused append
+  static constexpr int kPageBytes = kPage * D * 2;
+  static constexpr int kCopyBytes = 2 * kPageBytes;
+  static constexpr int kStride = kCopyBytes;
+  static __device__ __forceinline__ void issue(uint32_t dst, uint32_t bar, const CUtensorMap *tmK,
+                                               const CUtensorMap *tmV, int row, uint64_t policy,
+                                               const DecodeArgs &) {
+    mbar_arrive_expect_tx(bar, kCopyBytes);
+#pragma unroll
+    for (int hf = 0; hf < D / 64; ++hf) {
+      tma_load_3d(dst + hf * kPage * 128, tmK, 0, hf, row, bar, policy);
+      tma_load_3d(dst + kPageBytes + hf * kPage * 128, tmV, 0, hf, row, bar, policy);
+    }
+  }
+  static __device__ __forceinline__ void zero_tail(uint8_t *st, int ntok, int lane) {
+    const int n16 = (kPage - ntok) * 128 / 16;  // 16-byte chunks per half
+#pragma unroll
+    for (int hf = 0; hf < D / 64; ++hf) {
+      uint4 *z = reinterpret_cast<uint4 *>(st + kPageBytes + hf * kPage * 128 + ntok * 128);
+      for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  static __device__ __forceinline__ void tile(uint8_t *st, int ntok, float sl2, int lane,
+                                              const uint32_t (&qf)[NT][D / 16][2],
+                                              float (&acc)[NT][D / 16][4], float (&m)[NT][2],
+                                              float (&l)[NT][2]) {
+    tile_page<D, NT, T>(smem_u32(st), smem_u32(st + kPageBytes), ntok, sl2, lane, qf, acc, m, l);
+  }
+  static __device__ __forceinline__ void q_words(const uint32_t *qrow, int ks, int tig,
+                                                 uint32_t &w0, uint32_t &w1) {
+    w0 = __ldg(qrow + ks * 8 + tig);
+    w1 = __ldg(qrow + ks * 8 + 4 + tig);
+  }
+  static __device__ __forceinline__ int dim(int mt, int e, int g8) {
+    return mt * 16 + g8 + ((e >> 1) << 3);
+  }
+};
+
+// E4M3 pages (d = 128): codes [16][128] per (page, head) in one swizzled box,
+// fp32 scales [16][4] per (page, head) copied alongside; output dtype T.
+template <int NT, typename T>
+struct Page8 {
+  using Out = T;
+  static constexpr bool kPatchable = false;
+  static constexpr int kPageBytes = kPage * 128;             // codes of K (or V)
+  static constexpr int kScaleBytes = kPage * 4 * 4;          // scales of K (or V)
+  static constexpr int kCopyBytes = 2 * kPageBytes + 2 * kScaleBytes;
+  static constexpr int kStride = 5120;
+  static __device__ __forceinline__ void issue(uint32_t dst, uint32_t bar, const CUtensorMap *tmK,
+                                               const CUtensorMap *tmV, int row, uint64_t policy,
+                                               const DecodeArgs &a) {
+    mbar_arrive_expect_tx(bar, kCopyBytes);
+    tma_load_2d(dst, tmK, 0, row, bar, policy);
+    tma_load_2d(dst + kPageBytes, tmV, 0, row, bar, policy);
+    bulk_load(dst + 2 * kPageBytes, a.k_scale + static_cast<size_t>(row) * 4, kScaleBytes, bar);
+    bulk_load(dst + 2 * kPageBytes + kScaleBytes, a.v_scale + static_cast<size_t>(row) * 4,
+              kScaleBytes, bar);
+  }
+  static __device__ __forceinline__ void zero_tail(uint8_t *st, int ntok, int lane) {
+    // V codes and V scales of masked rows (their zero weights times a NaN
+    // scale would otherwise poison the PV product)
+    const int n16 = (kPage - ntok) * 128 / 16;
+    uint4 *z = reinterpret_cast<uint4 *>(st + kPageBytes + ntok * 128);
+    for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
+    uint4 *zs = reinterpret_cast<uint4 *>(st + 2 * kPageBytes + kScaleBytes + ntok * 16);
+    for (int i = lane; i < kPage - ntok; i += 32) zs[i] = make_uint4(0, 0, 0, 0);
+  }
+  static __device__ __forceinline__ void tile(uint8_t *st, int ntok, float sl2, int lane,
+                                              const uint32_t (&qf)[NT][8][2],
+                                              float (&acc)[NT][8][4], float (&m)[NT][2],
+                                              float (&l)[NT][2]) {
+    const float *ks = reinterpret_cast<const float *>(st + 2 * kPageBytes);
+    tile_page_fp8<NT>(smem_u32(st), smem_u32(st + kPageBytes), ks, ks + kPage * 4, ntok, sl2, lane,
+                      qf, acc, m, l);
+  }
+  // q in f16, channel order of the E4M3 tile: k-slots 2t, 2t+1 <- channels
+  // 4t, 4t+1 and k-slots 2t+8, 2t+9 <- channels 4t+2, 4t+3 of each 16
+  static __device__ __forceinline__ uint32_t to_f16x2(uint32_t w) {
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w));
+      return f16pack(f.x, f.y);
+    } else {
+      return w;
+    }
+  }
+  static __device__ __forceinline__ void q_words(const uint32_t *qrow, int ks, int tig,
+                                                 uint32_t &w0, uint32_t &w1) {
+    w0 = to_f16x2(__ldg(qrow + ks * 8 + 2 * tig));
+    w1 = to_f16x2(__ldg(qrow + ks * 8 + 2 * tig + 1));
+  }
+  static __device__ __forceinline__ int dim(int mt, int e, int g8) {
+    return mt * 16 + 2 * g8 + (e >> 1);
+  }
+};
+
+namespace {
+
+// Zero one output row of d elements (16-byte stores).
 template <typename T>
-struct Stor;
-template <>
-struct Stor<__half> {
-  static __device__ __forceinline__ void zero_row(__half *p, int d) {
-    for (int i = 0; i < d; i += 8) *reinterpret_cast<uint4 *>(p + i) = make_uint4(0, 0, 0, 0);
-  }
-};
-template <>
-struct Stor<__nv_bfloat16> {
-  static __device__ __forceinline__ void zero_row(__nv_bfloat16 *p, int d) {
-    for (int i = 0; i < d; i += 8) *reinterpret_cast<uint4 *>(p + i) = make_uint4(0, 0, 0, 0);
-  }
-};
+__device__ __forceinline__ void zero_row(T *p, int d) {
+  for (int i = 0; i < d; i += 8) *reinterpret_cast<uint4 *>(p + i) = make_uint4(0, 0, 0, 0);
+}
 
 __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 #pragma unroll
@@ -90,11 +190,12 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 
 }  // namespace
 
-template <int D, int NT, typename T, int W, int S>
+template <int D, int NT, class Pol, int W, int S>
 __global__ void __launch_bounds__(32 * W, 1)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV) {
-  using Gm = Geo<D, NT, W, S>;
+  using T = typename Pol::Out;
+  using Gm = Geo<D, NT, W, S, Pol::kStride>;
   using M = Mma<T>;
   constexpr int kRows = 8 * NT;  // query rows per tile (G padded)
   constexpr int kPatch = 32;     // page-meta flag: fused append writes a row of this page
@@ -174,7 +275,7 @@ __global__ void __launch_bounds__(32 * W, 1)
          r += static_cast<long long>(gridDim.x) * Gm::kThreads) {
       const int b = static_cast<int>(r / a.H_q);
       if (cum[b + 1] == cum[b] && skip_of(b) == 0) {
-        Stor<T>::zero_row(reinterpret_cast<T *>(a.out) + r * D, D);
+        zero_row(reinterpret_cast<T *>(a.out) + r * D, D);
         if (a.lse_out) a.lse_out[r] = -INFINITY;
       }
     }
@@ -222,8 +323,8 @@ __global__ void __launch_bounds__(32 * W, 1)
             T *o = reinterpret_cast<T *>(a.out) + (row0 + r) * D;
 #pragma unroll
             for (int mt = 0; mt < Gm::kSteps; ++mt) {
-              o[mt * 16 + g8] = M::from_float(acc[nt][mt][i] * inv);
-              o[mt * 16 + 8 + g8] = M::from_float(acc[nt][mt][2 + i] * inv);
+              o[Pol::dim(mt, i, g8)] = M::from_float(acc[nt][mt][i] * inv);
+              o[Pol::dim(mt, 2 + i, g8)] = M::from_float(acc[nt][mt][2 + i] * inv);
             }
             if (a.lse_out && g8 == 0) a.lse_out[row0 + r] = lse;
           } else {
@@ -231,8 +332,8 @@ __global__ void __launch_bounds__(32 * W, 1)
             float *o = a.part_o + (slot * a.G + r) * D;
 #pragma unroll
             for (int mt = 0; mt < Gm::kSteps; ++mt) {
-              o[mt * 16 + g8] = acc[nt][mt][i] * inv;
-              o[mt * 16 + 8 + g8] = acc[nt][mt][2 + i] * inv;
+              o[Pol::dim(mt, i, g8)] = acc[nt][mt][i] * inv;
+              o[Pol::dim(mt, 2 + i, g8)] = acc[nt][mt][2 + i] * inv;
             }
             if (g8 == 0) a.part_lse[slot * a.G + r] = lse;
           }
@@ -374,13 +475,7 @@ __global__ void __launch_bounds__(32 * W, 1)
         meta_w[fst] = make_int4(seg, row >= 0 ? ntok : 0, row, 0);
         const uint32_t bar = bar0 + 8 * fst;
         if (row >= 0) {
-          const uint32_t dst = stage0 + fst * Gm::kStageBytes;
-          mbar_arrive_expect_tx(bar, Gm::kStageBytes);
-#pragma unroll
-          for (int hf = 0; hf < D / 64; ++hf) {
-            tma_load_3d(dst + hf * kPage * 128, &tmK, 0, hf, row, bar, policy);
-            tma_load_3d(dst + Gm::kPageBytes + hf * kPage * 128, &tmV, 0, hf, row, bar, policy);
-          }
+          Pol::issue(stage0 + fst * Gm::kStageBytes, bar, &tmK, &tmV, row, policy, a);
         } else {
           mbar_arrive(bar);
         }
@@ -405,8 +500,7 @@ __global__ void __launch_bounds__(32 * W, 1)
 #pragma unroll
         for (int ks = 0; ks < Gm::kSteps; ++ks) {
           if (r < a.G) {
-            qf[nt][ks][0] = __ldg(qw + r * (D / 2) + ks * 8 + tig);
-            qf[nt][ks][1] = __ldg(qw + r * (D / 2) + ks * 8 + 4 + tig);
+            Pol::q_words(qw + r * (D / 2), ks, tig, qf[nt][ks][0], qf[nt][ks][1]);
           } else {
             qf[nt][ks][0] = 0u;
             qf[nt][ks][1] = 0u;
@@ -444,7 +538,8 @@ __global__ void __launch_bounds__(32 * W, 1)
       const int ntok = md.y & (kPatch - 1);
       if (ntok > 0) {
         uint8_t *kp = stages + ((size_t)warp * S + cst) * Gm::kStageBytes;
-        uint8_t *vp = kp + Gm::kPageBytes;
+        if constexpr (Pol::kPatchable) {
+        uint8_t *vp = kp + Pol::kPageBytes;
         if (md.y & kPatch) {
           // fused append: the new token is row ntok - 1 of this page.  Put
           // k_new / v_new into the staged page (the copy just read may
@@ -463,20 +558,15 @@ __global__ void __launch_bounds__(32 * W, 1)
           fence_proxy_async_smem();
           __syncwarp();
         }
+        }
         if (ntok < kPage) {
           // rows past the sequence end may hold anything (even NaN): clear V's
           // so the zero weights of masked tokens cannot turn into NaN
-          const int n16 = (kPage - ntok) * 128 / 16;  // 16-byte chunks per half
-#pragma unroll
-          for (int hf = 0; hf < D / 64; ++hf) {
-            uint4 *z = reinterpret_cast<uint4 *>(vp + hf * kPage * 128 + ntok * 128);
-            for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
-          }
+          Pol::zero_tail(kp, ntok, lane);
           fence_proxy_async_smem();
           __syncwarp();
         }
-        tile_page<D, NT, T>(smem_u32(kp), smem_u32(vp), ntok, a.scale_log2, lane, qf, acc, m_run,
-                            l_run);
+        Pol::tile(kp, ntok, a.scale_log2, lane, qf, acc, m_run, l_run);
       }
       __syncwarp();
       if (f < p1) issue();
@@ -844,8 +934,9 @@ template <int D, int NT, typename T>
 cudaError_t launch_decode_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                             cudaStream_t st, int grid) {
   constexpr int W = Tune<D, NT>::W, S = Tune<D, NT>::S;
-  auto kern = decode_kernel<D, NT, T, W, S>;
-  const size_t smem = Geo<D, NT, W, S>::smem(a.B);
+  using Pol = Page16<D, NT, T>;
+  auto kern = decode_kernel<D, NT, Pol, W, S>;
+  const size_t smem = Geo<D, NT, W, S, Pol::kStride>::smem(a.B);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -890,6 +981,41 @@ cudaError_t launch_generic_dt(const GenericMergeArgs &a, cudaStream_t st) {
 }  // namespace
 
 int decode_auto_parts(int sms) { return sms; }
+
+// 8-bit cache (d = 128): each page-stage is 4.5 KB, so fewer warps with
+// deeper rings keep enough bytes in flight.
+#ifndef KVD_TUNE_W8
+#define KVD_TUNE_W8 8
+#endif
+#ifndef KVD_TUNE_S8
+#define KVD_TUNE_S8 4
+#endif
+
+namespace {
+template <int NT, typename T>
+cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                             cudaStream_t st, int grid) {
+  constexpr int W = KVD_TUNE_W8;
+  constexpr int S = (NT == 2 && KVD_TUNE_S8 > 3) ? 3 : KVD_TUNE_S8;  // NT=2 parks 8 KB tiles
+  using Pol = Page8<NT, T>;
+  auto kern = decode_kernel<128, NT, Pol, W, S>;
+  const size_t smem = Geo<128, NT, W, S, Pol::kStride>::smem(a.B);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(grid), dim3(32 * W), smem, st, a, tmK, tmV);
+}
+}  // namespace
+
+cudaError_t launch_decode_fp8(const DecodeArgs &a, DType dt, const CUtensorMap &tmK,
+                              const CUtensorMap &tmV, cudaStream_t s, int grid) {
+  const bool two = a.G > 8;
+  if (dt == DType::BF16)
+    return two ? launch_decode8_t<2, __nv_bfloat16>(a, tmK, tmV, s, grid)
+               : launch_decode8_t<1, __nv_bfloat16>(a, tmK, tmV, s, grid);
+  return two ? launch_decode8_t<2, __half>(a, tmK, tmV, s, grid)
+             : launch_decode8_t<1, __half>(a, tmK, tmV, s, grid);
+}
 
 cudaError_t launch_decode(const DecodeArgs &a, int d, DType dt, const CUtensorMap &tmK,
                           const CUtensorMap &tmV, cudaStream_t s, int grid) {

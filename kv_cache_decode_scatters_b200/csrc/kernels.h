@@ -50,6 +50,23 @@ struct DecodeArgs {
   const float *pre_o;
   const float *pre_lse;
   int pre_chunks;
+  // 8-bit cache (null for 16-bit pages): fp32 scales [num_blocks][H_kv][16][d/32]
+  const float *k_scale;
+  const float *v_scale;
+};
+
+// Quantise rows of d fp16/bf16 words into E4M3 codes + fp32 per-32-channel
+// scales; `dst_rows` (nullable) maps source row r to destination row.
+struct QuantArgs {
+  const void *src;        // [n][d]
+  uint8_t *codes;         // [rows][d]
+  float *scales;          // [rows][d / 32]
+  const int32_t *block_table;  // append mode: destination of k_new/v_new rows
+  const int32_t *slot;
+  unsigned *err;
+  long long n;            // source rows
+  int d, H_kv, num_blocks, maxb;
+  int append;             // 1: src is [B][H_kv][d] and goes to page rows per slot
 };
 
 struct PrefixArgs {
@@ -87,6 +104,9 @@ cudaError_t launch_decode(const DecodeArgs &a, int d, DType dt, const CUtensorMa
                           const CUtensorMap &tmV, cudaStream_t s, int grid);
 cudaError_t launch_decode_merge(const DecodeArgs &a, int d, DType dt, cudaStream_t s);
 cudaError_t launch_generic_merge(const GenericMergeArgs &a, DType dt, cudaStream_t s);
+cudaError_t launch_decode_fp8(const DecodeArgs &a, DType dt, const CUtensorMap &tmK,
+                              const CUtensorMap &tmV, cudaStream_t s, int grid);
+cudaError_t launch_quantize_fp8(const QuantArgs &a, DType dt, cudaStream_t s);
 // Prefix pass of the shared-prefix decode: grid (n_groups * chunks, H_kv, row blocks).
 cudaError_t launch_prefix(const PrefixArgs &a, int d, DType dt, const CUtensorMap &tmK,
                           const CUtensorMap &tmV, int row_blocks, cudaStream_t s);

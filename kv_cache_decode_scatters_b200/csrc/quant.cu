@@ -1,0 +1,74 @@
+// quant.cu -- FP8 (E4M3) quantisation of K/V rows for the 8-bit cache.
+//
+// "KV Cache:推理慢的真正原因", section 工程优化手段 / 量化: store the cache in 8 bits
+// with scales per channel group, so a few very large key channels do not
+// swamp the scale of the others.  Each row (one token of one KV head) is
+// split into groups of 32 channels; group scale s = max|x| / 448 (448 is the
+// largest E4M3 value) and code = E4M3(x / s), rounded to nearest even and
+// saturated; both divisions are IEEE fp32 (__fdiv_rn), so the codes are the
+// same on every run and every machine.  A group of zeros gets s = 0.
+//
+// One warp per row: lane l holds channels 4l..4l+3, a group is 8 lanes and
+// its maximum is three shuffles.  In append mode the source rows are the
+// step's k_new (or v_new) [B][H_kv][d] and each goes to row slot % 16 of page
+// block_table[b][slot / 16] of the code and scale pools.
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kvd {
+
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_fp8_kernel(const QuantArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long r = static_cast<long long>(blockIdx.x) * 8 + warp;
+  if (r >= a.n) return;
+  long long dst = r;
+  if (a.append) {
+    const int b = static_cast<int>(r / a.H_kv), h = static_cast<int>(r % a.H_kv);
+    const int pos = __ldg(a.slot + b);
+    if (pos < 0) return;
+    if (pos >= a.maxb * kPage) {
+      if (lane == 0 && h == 0) flag_error(a.err, kErrSlot);
+      return;
+    }
+    const int pb = __ldg(a.block_table + static_cast<size_t>(b) * a.maxb + pos / kPage);
+    if (pb < 0 || pb >= a.num_blocks) {
+      if (lane == 0 && h == 0) flag_error(a.err, kErrBlockTable);
+      return;
+    }
+    dst = (static_cast<long long>(pb) * a.H_kv + h) * kPage + pos % kPage;
+  }
+  const bool live = lane * 4 < a.d;
+  float x[4] = {0.f, 0.f, 0.f, 0.f};
+  if (live) {
+    const uint2 w = *reinterpret_cast<const uint2 *>(static_cast<const T *>(a.src) + r * a.d + lane * 4);
+    const T *v = reinterpret_cast<const T *>(&w);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = static_cast<float>(v[i]);
+  }
+  float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+  const float s = __fdiv_rn(mx, 448.0f);
+  float q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) q[i] = s == 0.0f ? 0.0f : __fdiv_rn(x[i], s);
+  if (!live) return;
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(q[0], q[1]), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(q[2], q[3]), __NV_SATFINITE, __NV_E4M3);
+  *reinterpret_cast<uint32_t *>(a.codes + dst * a.d + lane * 4) = (lo & 0xffffu) | (hi << 16);
+  if ((lane & 7) == 0) a.scales[dst * (a.d / 32) + (lane >> 3)] = s;
+}
+
+cudaError_t launch_quantize_fp8(const QuantArgs &a, DType dt, cudaStream_t s) {
+  if (a.n == 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>((a.n + 7) / 8);
+  if (dt == DType::BF16) quantize_fp8_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
+  else quantize_fp8_kernel<__half><<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace kvd

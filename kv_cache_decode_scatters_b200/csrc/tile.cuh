@@ -262,3 +262,153 @@ __device__ __forceinline__ void tile_page2(uint32_t kbA, uint32_t vbA, uint32_t 
 }
 
 }  // namespace kvd
+
+// ------------------------------------------------------------ 8-bit pages
+#include <cuda_fp8.h>
+
+namespace kvd {
+
+// Two E4M3 codes (low byte first) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+__device__ __forceinline__ uint32_t f16pack(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Byte offset of 16-byte chunk c of token row t in a 16-row page of 128-byte
+// rows staged by one 128B-swizzled TMA box.
+__device__ __forceinline__ uint32_t swz8(int t, int c) {
+  return static_cast<uint32_t>(t * 128 + ((c ^ (t & 7)) << 4));
+}
+
+// One 16-token page of an E4M3 cache (d = 128) for 8*NT query rows of one
+// warp.  Codes are exact in f16, so the tensor-core tile runs in f16:
+//  * K: ldmatrix on the code bytes gives each lane four consecutive channels
+//    of a token per register; converted in pairs they fill the A fragment
+//    with the channel order permuted inside each 16-channel k-step (the q
+//    fragments, `qf`, use the same order).  Scores are summed per 32-channel
+//    group and then weighted by the token's group scales.
+//  * V: ldmatrix.trans on the code bytes gives (channel pair) x (token pair);
+//    a byte permute splits it into the A fragments of V^T, with output slot
+//    g8 <-> channel 2*g8 and slot g8+8 <-> channel 2*g8+1 of each m-tile.
+//    The V group scales ride on the probabilities (one P^T operand per group).
+// ks, vs: the page's fp32 scales in shared memory, [16 tokens][4 groups].
+template <int NT>
+__device__ __forceinline__ void tile_page_fp8(uint32_t kb, uint32_t vb, const float *ks,
+                                              const float *vs, int ntok, float scale_log2,
+                                              int lane, const uint32_t (&qf)[NT][8][2],
+                                              float (&acc)[NT][8][4], float (&m_run)[NT][2],
+                                              float (&l_run)[NT][2]) {
+  using M = Mma<__half>;
+  const int g8 = lane >> 2;
+  const int mi = lane >> 3, r8 = lane & 7;
+  const int tok = r8 + ((mi & 1) << 3);  // row this lane addresses for ldmatrix
+  const int hi16 = mi >> 1;              // second 16 bytes of a 32-channel group
+
+  float sg[4][NT][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sg[j][nt][e] = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t R[4];
+    ldmatrix_x4(R, kb + swz8(tok, 2 * j + hi16));
+    const uint32_t A0[4] = {e4m3x2_to_f16x2(R[0] & 0xffff), e4m3x2_to_f16x2(R[1] & 0xffff),
+                            e4m3x2_to_f16x2(R[0] >> 16), e4m3x2_to_f16x2(R[1] >> 16)};
+    const uint32_t A1[4] = {e4m3x2_to_f16x2(R[2] & 0xffff), e4m3x2_to_f16x2(R[3] & 0xffff),
+                            e4m3x2_to_f16x2(R[2] >> 16), e4m3x2_to_f16x2(R[3] >> 16)};
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      M::run(sg[j][nt], A0, qf[nt][2 * j][0], qf[nt][2 * j][1]);
+      M::run(sg[j][nt], A1, qf[nt][2 * j + 1][0], qf[nt][2 * j + 1][1]);
+    }
+  }
+  const float4 kA = *reinterpret_cast<const float4 *>(ks + g8 * 4);
+  const float4 kB = *reinterpret_cast<const float4 *>(ks + (g8 + 8) * 4);
+  const float4 vA = *reinterpret_cast<const float4 *>(vs + g8 * 4);
+  const float4 vB = *reinterpret_cast<const float4 *>(vs + (g8 + 8) * 4);
+  const float kAs[4] = {kA.x, kA.y, kA.z, kA.w}, kBs[4] = {kB.x, kB.y, kB.z, kB.w};
+  const float vAs[4] = {vA.x, vA.y, vA.z, vA.w}, vBs[4] = {vB.x, vB.y, vB.z, vB.w};
+
+  const bool v0 = g8 < ntok, v1 = g8 + 8 < ntok;
+  uint32_t pj0[4][NT], pj1[4][NT];
+  float alpha[NT][2];
+  bool rescale = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      s4[0] += sg[j][nt][0] * kAs[j];
+      s4[1] += sg[j][nt][1] * kAs[j];
+      s4[2] += sg[j][nt][2] * kBs[j];
+      s4[3] += sg[j][nt][3] * kBs[j];
+    }
+    const float x0 = v0 ? s4[0] * scale_log2 : -INFINITY;
+    const float x1 = v0 ? s4[1] * scale_log2 : -INFINITY;
+    const float x2 = v1 ? s4[2] * scale_log2 : -INFINITY;
+    const float x3 = v1 ? s4[3] * scale_log2 : -INFINITY;
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+    alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
+    alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
+    rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
+    m_run[nt][0] = mn0;
+    m_run[nt][1] = mn1;
+    const float e0 = fast_exp2(x0 - mn0), e1 = fast_exp2(x1 - mn1);
+    const float e2 = fast_exp2(x2 - mn0), e3 = fast_exp2(x3 - mn1);
+    l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (e0 + e2);
+    l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (e1 + e3);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      // masked tokens have e = 0 and a V scale of 0 (cleared by the caller)
+      pj0[j][nt] = movmatrix_trans(f16pack(e0 * vAs[j], e1 * vAs[j]));
+      pj1[j][nt] = movmatrix_trans(f16pack(e2 * vBs[j], e3 * vBs[j]));
+    }
+  }
+  if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        acc[nt][mt][0] *= alpha[nt][0];
+        acc[nt][mt][1] *= alpha[nt][1];
+        acc[nt][mt][2] *= alpha[nt][0];
+        acc[nt][mt][3] *= alpha[nt][1];
+      }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t R[4];
+    ldmatrix_x4_trans(R, vb + swz8(tok, 2 * j + hi16));
+    // R[0]: tokens 0-7, R[1]: tokens 8-15 (channels 32j..+15); R[2], R[3]: +16
+    uint32_t A[2][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t lo = R[2 * h], hi = R[2 * h + 1];
+      A[h][0] = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(lo, 0, 0x0020)));
+      A[h][1] = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(lo, 0, 0x0031)));
+      A[h][2] = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(hi, 0, 0x0020)));
+      A[h][3] = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(hi, 0, 0x0031)));
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      M::run(acc[nt][2 * j], A[0], pj0[j][nt], pj1[j][nt]);
+      M::run(acc[nt][2 * j + 1], A[1], pj0[j][nt], pj1[j][nt]);
+    }
+  }
+}
+
+}  // namespace kvd

@@ -1,0 +1,146 @@
+"""GPU parity of the 8-bit (FP8 E4M3) KV cache against the oracle.
+
+Quantisation and append must be bit-exact (codes and scales); attention over
+the 8-bit cache must be within the dtype tolerance of the oracle's attention
+over the same dequantised values.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import LSE_TOL, TOL
+from synth import build_workload, named_config, step_inputs, to_words
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kvd():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import kv_cache_decode_scatters_b200 as m
+    m.kvd_read_device_error(clear=True)
+    return m
+
+
+def odt(w):
+    return oracle.BF16 if w.dtype == torch.bfloat16 else oracle.F16
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("d", [128, 64])
+def test_quantize_bit_exact(kvd, dtype, d):
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(1000, d, generator=g)
+    x[3, 17] = 40.0            # outlier channel
+    x[5, 32:64] = 0.0          # all-zero group
+    x[7] *= 1e-3               # small row
+    x = x.to(dtype)
+    codes, scales = kvd.kvd_quantize_fp8(x.cuda())
+    torch.cuda.synchronize()
+    oc, os_ = oracle.quantize_fp8(to_words(x), oracle.BF16 if dtype == torch.bfloat16 else oracle.F16)
+    assert np.array_equal(codes.cpu().numpy(), oc)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+
+
+def fp8_state(kvd, w):
+    """Quantise the workload's 16-bit pools on the GPU; also return host copies."""
+    k8, ks = kvd.kvd_quantize_fp8(w.k_cache.cuda())
+    v8, vs = kvd.kvd_quantize_fp8(w.v_cache.cuda())
+    torch.cuda.synchronize()
+    return k8, v8, ks, vs
+
+
+def host(t):
+    return t.cpu().numpy().copy()
+
+
+def test_append_fp8_bit_exact_whole_pool(kvd):
+    w = build_workload("a8", 5, 8, 4, 128, "bf16", [1, 16, 17, 40, 0], seed=1201, spare_pages=3)
+    si = step_inputs(w, 0)
+    k8, v8, ks, vs = fp8_state(kvd, w)
+    hk8, hv8, hks, hvs = host(k8), host(v8), host(ks), host(vs)
+    bt = w.block_table.cuda()
+    kvd.kvd_append_fp8(k8, v8, ks, vs, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    torch.cuda.synchronize()
+    oracle.append_fp8(hk8, hv8, hks, hvs, w.block_table.numpy(), si["slot"].numpy(),
+                      to_words(si["k_new"]), to_words(si["v_new"]), oracle.BF16)
+    assert np.array_equal(host(k8), hk8) and np.array_equal(host(v8), hv8)
+    assert np.array_equal(host(ks).view(np.uint32), hks.view(np.uint32))
+    assert np.array_equal(host(vs).view(np.uint32), hvs.view(np.uint32))
+    assert kvd.kvd_read_device_error() == 0
+
+
+CASES = [
+    # B, H_q, H_kv, dtype, lens, partitions
+    (4, 32, 32, "f16", [1, 15, 16, 300], 0),
+    (3, 64, 8, "bf16", [513, 77, 1000], 0),
+    (2, 16, 1, "bf16", [40, 130], 0),          # MQA, group 16
+    (5, 32, 8, "f16", [3, 0, 45, 0, 200], 7),  # empty sequences, fixed partitions
+    (2, 24, 8, "bf16", [700, 31], 1),          # group 3, one partition
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_{c[3]}_N{c[5]}")
+def test_decode_fp8_matches_oracle(kvd, case):
+    B, H_q, H_kv, dtype, lens, parts = case
+    w = build_workload("d8", B, H_q, H_kv, 128, dtype, lens, seed=1300 + CASES.index(case),
+                       spare_pages=2)
+    si = step_inputs(w, 0)
+    k8, v8, ks, vs = fp8_state(kvd, w)
+    bt = w.block_table.cuda()
+    kvd.kvd_append_fp8(k8, v8, ks, vs, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    lse = torch.empty((B, H_q), dtype=torch.float32, device="cuda")
+    out = kvd.kvd_decode_attention_fp8(si["q"].cuda(), k8, v8, ks, vs, bt, si["seq_lens"].cuda(),
+                                       w.scale, num_partitions=parts, lse_out=lse)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle.attend_fp8(to_words(si["q"]), host(k8), host(v8), host(ks), host(vs),
+                                     w.block_table.numpy(), si["seq_lens"].numpy(), w.scale, odt(w))
+    g = out.float().cpu().double().numpy()
+    err = float(np.max(np.abs(g - ref)))
+    assert err <= TOL[w.dtype], f"max abs error {err}"
+    fin = np.isfinite(ref_lse)
+    gl = lse.cpu().double().numpy()
+    assert np.array_equal(np.isfinite(gl), fin)
+    assert np.max(np.abs(gl[fin] - ref_lse[fin])) <= LSE_TOL
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert torch.all(out[b] == 0)
+    # against the 16-bit cache, the error is the quantisation's: every value
+    # is within half an E4M3 ulp (2^-4 relative) and out is a weighted mean of
+    # values, so |out_fp8 - out_16| <= 2^-4 max|v| plus what the changed
+    # scores move (checked loosely)
+    kc, vc = to_words(w.k_cache).copy(), to_words(w.v_cache).copy()
+    oracle.append(kc, vc, w.block_table.numpy(), si["slot"].numpy(), to_words(si["k_new"]),
+                  to_words(si["v_new"]))
+    full, _ = oracle.attend(to_words(si["q"]), kc, vc, w.block_table.numpy(), si["seq_lens"].numpy(),
+                            w.scale, odt(w))
+    vmax = float(np.nanmax(np.abs(si["v_new"].float().numpy())))
+    assert np.max(np.abs(g - full)) <= 2 * 2 ** -4 * max(vmax, 4.0)
+    assert kvd.kvd_read_device_error() == 0
+
+
+def test_decode_fp8_full_size_gqa70b(kvd):
+    w = named_config("gqa70b", device="cuda", gen_device="cuda")
+    si = step_inputs(w, 0)
+    k8, v8, ks, vs = fp8_state(kvd, w)
+    bt = w.block_table.cuda()
+    kvd.kvd_append_fp8(k8, v8, ks, vs, bt, si["slot"], si["k_new"], si["v_new"])
+    out = kvd.kvd_decode_attention_fp8(si["q"], k8, v8, ks, vs, bt, si["seq_lens"], w.scale)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    lens = w.seq_lens0.numpy()
+    rows = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 5, 40})
+    hk8, hv8, hks, hvs = host(k8), host(v8), host(ks), host(vs)
+    q = to_words(si["q"])
+    sl = si["seq_lens"].cpu().numpy()
+    btn = w.block_table.numpy()
+    worst = 0.0
+    for b in rows:
+        ref, _ = oracle.attend_fp8(q[b:b + 1], hk8, hv8, hks, hvs, btn[b:b + 1], sl[b:b + 1], w.scale,
+                                   oracle.BF16)
+        worst = max(worst, float(np.max(np.abs(out[b].float().cpu().double().numpy() - ref[0]))))
+    print(f"gqa70b fp8: max abs error {worst:.3e} over sequences {rows}")
+    assert worst <= TOL[w.dtype]
+    assert kvd.kvd_read_device_error() == 0
