@@ -35,8 +35,9 @@ from synth import build_workload, config_spec, named_config, step_inputs, to_wor
 
 METRIC = "paged decode-attention achieved HBM GB/s (% of B200 peak); us per decode step"
 FALLBACK_HBM_GBS = 6650.0
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_mha7b_ncu.md")
-DECODE_SOURCE = os.path.join(ROOT, "kv_cache_decode_scatters_b200", "csrc", "decode.cu")
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+DECODE_SOURCES = [os.path.join(ROOT, "kv_cache_decode_scatters_b200", "csrc", f)
+                  for f in ("decode.cu", "tile.cuh", "common.cuh")]
 
 
 # ------------------------------------------------------------------ helpers
@@ -99,23 +100,38 @@ def read_only_peak_gbs(nbytes=4 << 30, reps=5):
 
 
 def source_hash() -> str:
-    with open(DECODE_SOURCE, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the decode kernel's sources (kernel, tile, shared helpers)."""
+    h = hashlib.sha256()
+    for path in DECODE_SOURCES:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
-def profile_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current decode kernel source for this workload."""
+def profile_traffic(workload: str, mode: str):
+    """DRAM bytes per decode launch from a committed ncu summary under
+    profiles/, if one was taken on the current decode kernel sources for this
+    workload and step mode ("fused", "separate_append", "shared_prefix" or
+    "fp8")."""
     try:
-        text = open(PROFILE_SUMMARY, encoding="utf-8").read()
+        names = sorted(os.listdir(PROFILE_DIR))
     except OSError:
         return None
-    m_src = re.search(r"decode_source_sha256_16:\s*([0-9a-f]+)", text)
-    m_wl = re.search(r"workload:\s*(\S+)", text)
-    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not (m_src and m_b and m_wl) or m_src.group(1) != source_hash() or m_wl.group(1) != workload:
-        return None
-    return int(m_b.group(1))
+    want = source_hash()
+    for name in names:
+        if not (name.startswith("decode_kernel") and name.endswith(".md")):
+            continue
+        with open(os.path.join(PROFILE_DIR, name), encoding="utf-8") as f:
+            text = f.read()
+        m_src = re.search(r"decode_source_sha256_16:\s*([0-9a-f]+)", text)
+        m_wl = re.search(r"workload:\s*(\S+)", text)
+        m_mode = re.search(r"cache_mode:\s*(\S+)", text)
+        m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+        if not (m_src and m_b and m_wl and m_mode):
+            continue
+        if m_src.group(1) == want and m_wl.group(1) == workload and m_mode.group(1) == mode:
+            return int(m_b.group(1))
+    return None
 
 
 class ClockSampler:
@@ -508,7 +524,7 @@ def run_ours(args):
             "l2": "inputs larger than L2 (KV pool %.2f GB >> 126 MB); no flush" % (
                 2 * w.k_cache.numel() * 2 / 1e9),
             "step": ("kvd_append_fp8 + kvd_decode_attention_fp8 over an E4M3 cache "
-                     "(2 quantise, decode, merge kernels)" if f8 is not None else
+                     "(quantising append, decode, merge kernels)" if f8 is not None else
                      "kvd_decode_attention_shared_prefix with fused append (prefix, decode, merge kernels)"
                      if sp is not None else
                      "kvd_append + kvd_decode_attention (append, decode, merge kernels)"
@@ -526,12 +542,15 @@ def run_ours(args):
             "peak_kind": peak_kind,
             "kernel": ("kvd_decode_attention_fp8 call (decode_kernel over E4M3 pages + merge)"
                        if f8 is not None else
+                       "kvd_decode_attention_shared_prefix call (prefix_kernel + decode_kernel with fused "
+                       "append + merge)" if sp is not None else
                        "kvd_decode_attention call (decode_kernel + decode_merge_kernel)"
                        if args.separate_append else
                        "kvd_decode_step call (decode_kernel with fused append + decode_merge_kernel)")
                       + ", CUDA events on the launching stream; achieved = its algorithmic bytes / mean duration",
             "bytes_per_launch": timed_bytes,
-            "traffic": profile_traffic(w.name),
+            "traffic": profile_traffic(w.name, "fp8" if f8 is not None else "shared_prefix" if sp is not None
+                                      else "separate_append" if args.separate_append else "fused"),
         },
         "frac_of_8000_spec": round(achieved / 8000.0, 4),
         "shared_prefix": ({"unique_attention_bytes": unique_attention_bytes(w, si["seq_lens"]),

@@ -49,16 +49,18 @@ namespace kvd {
 
 namespace {
 
-template <int D, int NT, int W, int S, int kStride>
+template <int D, int NT, int W, int S, int kStride, int kAux>
 struct Geo {
   static constexpr int kStageBytes = kStride;           // smem stride of one ring stage
+  static constexpr int kAuxBytes = kAux;                // per-stage side data (scales), own area
   static constexpr int kThreads = 32 * W;
   static constexpr int kSteps = D / 16;                 // k-steps of S, m-tiles of O
   static constexpr int kEdgeFloats = 8 * NT * D;        // one parked accumulator tile
   static_assert(kEdgeFloats * 4 <= S * kStageBytes, "a parked tile must fit in a warp's ring");
   static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
   static size_t smem(int B) {
-    return 1024 + (size_t)W * S * kStageBytes + (size_t)W * kEdgeFloats * 4 + (size_t)W * S * 24 +
+    return 1024 + (size_t)W * S * kStageBytes + (size_t)W * kEdgeFloats * 4 + (size_t)W * S * kAux +
+           (size_t)W * S * 24 +
            (size_t)W * 2 * 2 * 8 * NT * 4 + (size_t)W * 2 * 4 + (size_t)(B + 1) * 4;
   }
 };
@@ -80,9 +82,10 @@ struct Page16 {
   static constexpr int kPageBytes = kPage * D * 2;
   static constexpr int kCopyBytes = 2 * kPageBytes;
   static constexpr int kStride = kCopyBytes;
-  static __device__ __forceinline__ void issue(uint32_t dst, uint32_t bar, const CUtensorMap *tmK,
-                                               const CUtensorMap *tmV, int row, uint64_t policy,
-                                               const DecodeArgs &) {
+  static constexpr int kAuxBytes = 0;
+  static __device__ __forceinline__ void issue(uint32_t dst, uint32_t, uint32_t bar,
+                                               const CUtensorMap *tmK, const CUtensorMap *tmV,
+                                               int row, uint64_t policy, const DecodeArgs &) {
     mbar_arrive_expect_tx(bar, kCopyBytes);
 #pragma unroll
     for (int hf = 0; hf < D / 64; ++hf) {
@@ -90,7 +93,7 @@ struct Page16 {
       tma_load_3d(dst + kPageBytes + hf * kPage * 128, tmV, 0, hf, row, bar, policy);
     }
   }
-  static __device__ __forceinline__ void zero_tail(uint8_t *st, int ntok, int lane) {
+  static __device__ __forceinline__ void zero_tail(uint8_t *st, uint8_t *, int ntok, int lane) {
     const int n16 = (kPage - ntok) * 128 / 16;  // 16-byte chunks per half
 #pragma unroll
     for (int hf = 0; hf < D / 64; ++hf) {
@@ -98,7 +101,7 @@ struct Page16 {
       for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
     }
   }
-  static __device__ __forceinline__ void tile(uint8_t *st, int ntok, float sl2, int lane,
+  static __device__ __forceinline__ void tile(uint8_t *st, uint8_t *, int ntok, float sl2, int lane,
                                               const uint32_t (&qf)[NT][D / 16][2],
                                               float (&acc)[NT][D / 16][4], float (&m)[NT][2],
                                               float (&l)[NT][2]) {
@@ -123,31 +126,31 @@ struct Page8 {
   static constexpr int kPageBytes = kPage * 128;             // codes of K (or V)
   static constexpr int kScaleBytes = kPage * 4 * 4;          // scales of K (or V)
   static constexpr int kCopyBytes = 2 * kPageBytes + 2 * kScaleBytes;
-  static constexpr int kStride = 5120;
-  static __device__ __forceinline__ void issue(uint32_t dst, uint32_t bar, const CUtensorMap *tmK,
-                                               const CUtensorMap *tmV, int row, uint64_t policy,
-                                               const DecodeArgs &a) {
+  static constexpr int kStride = 2 * kPageBytes;             // codes only: 1024-aligned stages
+  static constexpr int kAuxBytes = 2 * kScaleBytes;          // scales, in their own area
+  static __device__ __forceinline__ void issue(uint32_t dst, uint32_t aux, uint32_t bar,
+                                               const CUtensorMap *tmK, const CUtensorMap *tmV,
+                                               int row, uint64_t policy, const DecodeArgs &a) {
     mbar_arrive_expect_tx(bar, kCopyBytes);
     tma_load_2d(dst, tmK, 0, row, bar, policy);
     tma_load_2d(dst + kPageBytes, tmV, 0, row, bar, policy);
-    bulk_load(dst + 2 * kPageBytes, a.k_scale + static_cast<size_t>(row) * 4, kScaleBytes, bar);
-    bulk_load(dst + 2 * kPageBytes + kScaleBytes, a.v_scale + static_cast<size_t>(row) * 4,
-              kScaleBytes, bar);
+    bulk_load(aux, a.k_scale + static_cast<size_t>(row) * 4, kScaleBytes, bar);
+    bulk_load(aux + kScaleBytes, a.v_scale + static_cast<size_t>(row) * 4, kScaleBytes, bar);
   }
-  static __device__ __forceinline__ void zero_tail(uint8_t *st, int ntok, int lane) {
+  static __device__ __forceinline__ void zero_tail(uint8_t *st, uint8_t *aux, int ntok, int lane) {
     // V codes and V scales of masked rows (their zero weights times a NaN
     // scale would otherwise poison the PV product)
     const int n16 = (kPage - ntok) * 128 / 16;
     uint4 *z = reinterpret_cast<uint4 *>(st + kPageBytes + ntok * 128);
     for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
-    uint4 *zs = reinterpret_cast<uint4 *>(st + 2 * kPageBytes + kScaleBytes + ntok * 16);
+    uint4 *zs = reinterpret_cast<uint4 *>(aux + kScaleBytes + ntok * 16);
     for (int i = lane; i < kPage - ntok; i += 32) zs[i] = make_uint4(0, 0, 0, 0);
   }
-  static __device__ __forceinline__ void tile(uint8_t *st, int ntok, float sl2, int lane,
+  static __device__ __forceinline__ void tile(uint8_t *st, uint8_t *aux, int ntok, float sl2, int lane,
                                               const uint32_t (&qf)[NT][8][2],
                                               float (&acc)[NT][8][4], float (&m)[NT][2],
                                               float (&l)[NT][2]) {
-    const float *ks = reinterpret_cast<const float *>(st + 2 * kPageBytes);
+    const float *ks = reinterpret_cast<const float *>(aux);
     tile_page_fp8<NT>(smem_u32(st), smem_u32(st + kPageBytes), ks, ks + kPage * 4, ntok, sl2, lane,
                       qf, acc, m, l);
   }
@@ -195,7 +198,7 @@ __global__ void __launch_bounds__(32 * W, 1)
     decode_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV) {
   using T = typename Pol::Out;
-  using Gm = Geo<D, NT, W, S, Pol::kStride>;
+  using Gm = Geo<D, NT, W, S, Pol::kStride, Pol::kAuxBytes>;
   using M = Mma<T>;
   constexpr int kRows = 8 * NT;  // query rows per tile (G padded)
   constexpr int kPatch = 32;     // page-meta flag: fused append writes a row of this page
@@ -207,7 +210,8 @@ __global__ void __launch_bounds__(32 * W, 1)
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *stages = smem;
   float *edge_acc = reinterpret_cast<float *>(smem + (size_t)W * S * Gm::kStageBytes);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(edge_acc + (size_t)W * Gm::kEdgeFloats);
+  uint8_t *aux = reinterpret_cast<uint8_t *>(edge_acc + (size_t)W * Gm::kEdgeFloats);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(aux + (size_t)W * S * Gm::kAuxBytes);
   int4 *meta = reinterpret_cast<int4 *>(bars + W * S);
   float *edge_ml = reinterpret_cast<float *>(meta + W * S);  // [W][2][2][kRows]: m, l
   int *edge_id = reinterpret_cast<int *>(edge_ml + W * 2 * 2 * kRows);  // [W][2]
@@ -398,6 +402,7 @@ __global__ void __launch_bounds__(32 * W, 1)
   bool failed = false;
   if (p0 < p1) {
     const uint32_t stage0 = smem_u32(stages + (size_t)warp * S * Gm::kStageBytes);
+    const uint32_t aux0 = smem_u32(aux + (size_t)warp * S * Gm::kAuxBytes);
     const uint32_t bar0 = smem_u32(bars + warp * S);
     int4 *meta_w = meta + warp * S;
     const uint64_t policy = a.evict_first ? l2_policy_evict_first() : l2_policy_evict_normal();
@@ -475,7 +480,8 @@ __global__ void __launch_bounds__(32 * W, 1)
         meta_w[fst] = make_int4(seg, row >= 0 ? ntok : 0, row, 0);
         const uint32_t bar = bar0 + 8 * fst;
         if (row >= 0) {
-          Pol::issue(stage0 + fst * Gm::kStageBytes, bar, &tmK, &tmV, row, policy, a);
+          Pol::issue(stage0 + fst * Gm::kStageBytes, aux0 + fst * Gm::kAuxBytes, bar, &tmK, &tmV, row,
+                     policy, a);
         } else {
           mbar_arrive(bar);
         }
@@ -538,6 +544,7 @@ __global__ void __launch_bounds__(32 * W, 1)
       const int ntok = md.y & (kPatch - 1);
       if (ntok > 0) {
         uint8_t *kp = stages + ((size_t)warp * S + cst) * Gm::kStageBytes;
+        uint8_t *ap = aux + ((size_t)warp * S + cst) * Gm::kAuxBytes;
         if constexpr (Pol::kPatchable) {
         uint8_t *vp = kp + Pol::kPageBytes;
         if (md.y & kPatch) {
@@ -562,11 +569,11 @@ __global__ void __launch_bounds__(32 * W, 1)
         if (ntok < kPage) {
           // rows past the sequence end may hold anything (even NaN): clear V's
           // so the zero weights of masked tokens cannot turn into NaN
-          Pol::zero_tail(kp, ntok, lane);
+          Pol::zero_tail(kp, ap, ntok, lane);
           fence_proxy_async_smem();
           __syncwarp();
         }
-        Pol::tile(kp, ntok, a.scale_log2, lane, qf, acc, m_run, l_run);
+        Pol::tile(kp, ap, ntok, a.scale_log2, lane, qf, acc, m_run, l_run);
       }
       __syncwarp();
       if (f < p1) issue();
@@ -936,7 +943,7 @@ cudaError_t launch_decode_t(const DecodeArgs &a, const CUtensorMap &tmK, const C
   constexpr int W = Tune<D, NT>::W, S = Tune<D, NT>::S;
   using Pol = Page16<D, NT, T>;
   auto kern = decode_kernel<D, NT, Pol, W, S>;
-  const size_t smem = Geo<D, NT, W, S, Pol::kStride>::smem(a.B);
+  const size_t smem = Geo<D, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -982,24 +989,30 @@ cudaError_t launch_generic_dt(const GenericMergeArgs &a, cudaStream_t st) {
 
 int decode_auto_parts(int sms) { return sms; }
 
-// 8-bit cache (d = 128): each page-stage is 4.5 KB, so fewer warps with
-// deeper rings keep enough bytes in flight.
-#ifndef KVD_TUNE_W8
-#define KVD_TUNE_W8 8
+// 8-bit cache (d = 128): 4 KB code stages plus 512 B of scales; as for the
+// 16-bit pages, many warps with a short ring each keep the copies in flight.
+#ifndef KVD_TUNE_W8_1
+#define KVD_TUNE_W8_1 16
 #endif
-#ifndef KVD_TUNE_S8
-#define KVD_TUNE_S8 4
+#ifndef KVD_TUNE_S8_1
+#define KVD_TUNE_S8_1 2
+#endif
+#ifndef KVD_TUNE_W8_2
+#define KVD_TUNE_W8_2 10
+#endif
+#ifndef KVD_TUNE_S8_2
+#define KVD_TUNE_S8_2 2
 #endif
 
 namespace {
 template <int NT, typename T>
 cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                              cudaStream_t st, int grid) {
-  constexpr int W = KVD_TUNE_W8;
-  constexpr int S = (NT == 2 && KVD_TUNE_S8 > 3) ? 3 : KVD_TUNE_S8;  // NT=2 parks 8 KB tiles
+  constexpr int W = NT == 1 ? KVD_TUNE_W8_1 : KVD_TUNE_W8_2;
+  constexpr int S = NT == 1 ? KVD_TUNE_S8_1 : KVD_TUNE_S8_2;
   using Pol = Page8<NT, T>;
   auto kern = decode_kernel<128, NT, Pol, W, S>;
-  const size_t smem = Geo<128, NT, W, S, Pol::kStride>::smem(a.B);
+  const size_t smem = Geo<128, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

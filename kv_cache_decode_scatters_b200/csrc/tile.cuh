@@ -268,10 +268,15 @@ __device__ __forceinline__ void tile_page2(uint32_t kbA, uint32_t vbA, uint32_t 
 
 namespace kvd {
 
-// Two E4M3 codes (low byte first) -> f16x2, exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
-  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// Four E4M3 codes (bytes 0..3 of `four`) -> f16x2 of bytes (0, 1) and of
+// bytes (2, 3), exact (every E4M3 value is an f16 value).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t four, uint32_t &lo, uint32_t &hi) {
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(four));
 }
 
 __device__ __forceinline__ uint32_t f16pack(float lo, float hi) {
@@ -320,10 +325,11 @@ __device__ __forceinline__ void tile_page_fp8(uint32_t kb, uint32_t vb, const fl
   for (int j = 0; j < 4; ++j) {
     uint32_t R[4];
     ldmatrix_x4(R, kb + swz8(tok, 2 * j + hi16));
-    const uint32_t A0[4] = {e4m3x2_to_f16x2(R[0] & 0xffff), e4m3x2_to_f16x2(R[1] & 0xffff),
-                            e4m3x2_to_f16x2(R[0] >> 16), e4m3x2_to_f16x2(R[1] >> 16)};
-    const uint32_t A1[4] = {e4m3x2_to_f16x2(R[2] & 0xffff), e4m3x2_to_f16x2(R[3] & 0xffff),
-                            e4m3x2_to_f16x2(R[2] >> 16), e4m3x2_to_f16x2(R[3] >> 16)};
+    uint32_t A0[4], A1[4];
+    e4m3x4_to_f16x2x2(R[0], A0[0], A0[2]);
+    e4m3x4_to_f16x2x2(R[1], A0[1], A0[3]);
+    e4m3x4_to_f16x2x2(R[2], A1[0], A1[2]);
+    e4m3x4_to_f16x2x2(R[3], A1[1], A1[3]);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       M::run(sg[j][nt], A0, qf[nt][2 * j][0], qf[nt][2 * j][1]);
@@ -397,11 +403,9 @@ __device__ __forceinline__ void tile_page_fp8(uint32_t kb, uint32_t vb, const fl
     uint32_t A[2][4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const uint32_t lo = R[2 * h], hi = R[2 * h + 1];
-      A[h][0] = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(lo, 0, 0x0020)));
-      A[h][1] = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(lo, 0, 0x0031)));
-      A[h][2] = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(hi, 0, 0x0020)));
-      A[h][3] = e4m3x2_to_f16x2(static_cast<uint16_t>(__byte_perm(hi, 0, 0x0031)));
+      // bytes (0, 2) and (1, 3) of each word: the two channels of a pair
+      e4m3x4_to_f16x2x2(__byte_perm(R[2 * h], 0, 0x3120), A[h][0], A[h][1]);
+      e4m3x4_to_f16x2x2(__byte_perm(R[2 * h + 1], 0, 0x3120), A[h][2], A[h][3]);
     }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {

@@ -345,6 +345,10 @@ SP_CASES = [
     (6, 64, 8, 128, "bf16", [40, 33, 90, 49, 34, 70], 3, 32, 0),
     (4, 8, 8, 64, "f16", [600, 513, 530, 1000], 1, 512, 5),
     (4, 16, 1, 128, "bf16", [200, 145, 160, 300], 2, 144, 0),   # MQA, group 16
+    # one group of 40 members x 4 rows = 160 query rows: two 128-row blocks
+    (40, 32, 8, 128, "f16", [530 + 7 * i for i in range(40)], 1, 512, 0),
+    # a long shared prefix: several 64-token steps per chunk and a ragged last step
+    (16, 64, 8, 128, "bf16", [2100 + 13 * i for i in range(16)], 2, 2048, 0),
 ]
 
 
@@ -367,6 +371,28 @@ def test_shared_prefix_matches_oracle_and_plain_decode(kvd, case):
     assert max_lse_err(lse, ref) <= LSE_TOL
     assert torch.max(torch.abs(out.float() - ref_gpu.float())).item() <= TOL[w.dtype]
     assert kvd.kvd_read_device_error() == 0
+
+
+def test_shared_prefix_bad_page_is_flagged_and_contained(kvd):
+    # a block-table entry of group 0's shared prefix points outside the pool:
+    # the error word says so and group 1 is still exact
+    lens = [300, 257, 520, 999, 290, 400, 700, 266]
+    w = build_workload("spbad", 8, 32, 8, 128, "f16", lens, seed=971, prefix_groups=2,
+                       prefix_tokens=256)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    kvd.kvd_append(kc, vc, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    gs, gp, per = groups_of(w)
+    bt_bad = bt.clone()
+    bt_bad[0, 5] = w.num_blocks + 3
+    kvd.kvd_read_device_error(clear=True)
+    out = kvd.kvd_decode_attention_shared_prefix(si["q"].cuda(), kc, vc, bt_bad, si["seq_lens"].cuda(),
+                                                 gs, gp, per, w.scale)
+    torch.cuda.synchronize()
+    assert kvd.kvd_read_device_error(clear=True) & kvd.KVD_DEVERR_BLOCK_TABLE
+    _, _, ref = oracle_step(w, si)
+    for b in range(per, w.B):
+        assert np.max(np.abs(out[b].float().cpu().double().numpy() - ref[b][0])) <= TOL[w.dtype]
 
 
 def test_shared_prefix_fused_append_matches_decode_step(kvd):
