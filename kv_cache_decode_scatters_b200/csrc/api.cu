@@ -128,9 +128,11 @@ kvd_status prefix_layout(int B, int H_kv, int G, int d, int n_groups, int max_gr
   const int rpc = kvd::prefix_rows_per_cta();
   const long long rb = (rows + rpc - 1) / rpc;
   if (rb > 65535) return fail(KVD_ERR_UNSUPPORTED, "group of %d sequences too large", max_group_size);
-  // about four prefix CTAs per SM in all, each over a contiguous chunk of pages
+  // each (group, KV head, row block) unit's pages are cut into contiguous
+  // chunks, one CTA each: at d = 128 (tensor-memory pass, two CTAs per SM)
+  // about two per SM so that all are resident at once; otherwise about four
   const long long units = static_cast<long long>(n_groups) * H_kv * rb;
-  long long chunks = (4LL * sms + units - 1) / units;
+  long long chunks = d == 128 ? (2LL * sms) / units : (4LL * sms + units - 1) / units;
   chunks = chunks < 1 ? 1 : (chunks > 64 ? 64 : chunks);
   if (static_cast<long long>(n_groups) * chunks > 0x7fffffffLL)
     return fail(KVD_ERR_UNSUPPORTED, "too many groups");

@@ -23,7 +23,10 @@
 // it, and the producer waits for that before refilling the stage.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 #include "tile.cuh"
+
+#include <type_traits>
 
 namespace kvd {
 
@@ -39,6 +42,29 @@ struct PGeo {
   static constexpr int kStageBytes = 2 * kPageBytes;
   static constexpr size_t smem() { return 1024 + (size_t)kStages * kStageBytes + 2 * kStages * 8; }
 };
+
+// Per-sequence shared pages for the suffix pass (CTA (0,0,0) of the prefix
+// launch writes them, all its threads).  A member whose length does not cover
+// the group's pages keeps no shared pages and is attended whole by the decode
+// kernel.
+__device__ void write_skip(const PrefixArgs &a, int cap) {
+  const int tid = threadIdx.x;
+  for (int b = tid; b < a.B; b += blockDim.x) a.skip[b] = 0;
+  __syncthreads();
+  for (int g = 0; g < a.n_groups; ++g) {
+    const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
+    const int gp = __ldg(a.group_pages + g);
+    for (int b = s0 + tid; b < s1; b += blockDim.x) {
+      if (b < 0 || b >= a.B) continue;
+      const int n = clamp_len(__ldg(a.seq_lens + b), cap);
+      if (gp > 0 && gp * kPage <= n) {
+        a.skip[b] = gp;
+        // the step's new token must land in a private page
+        if (a.fused && gp * kPage == n) flag_error(a.err, kErrSlot);
+      }
+    }
+  }
+}
 
 }  // namespace
 
@@ -62,26 +88,7 @@ __global__ void __launch_bounds__(32 * kWarps, 1)
   grid_dependency_wait();
   grid_launch_dependents();
 
-  // Per-sequence shared pages for the suffix pass (one CTA writes them).  A
-  // member whose length does not cover the group's pages keeps no shared
-  // pages and is attended whole by the decode kernel.
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {
-    for (int b = tid; b < a.B; b += blockDim.x) a.skip[b] = 0;
-    __syncthreads();
-    for (int g = 0; g < a.n_groups; ++g) {
-      const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
-      const int gp = __ldg(a.group_pages + g);
-      for (int b = s0 + tid; b < s1; b += blockDim.x) {
-        if (b < 0 || b >= a.B) continue;
-        const int n = clamp_len(__ldg(a.seq_lens + b), cap);
-        if (gp > 0 && gp * kPage <= n) {
-          a.skip[b] = gp;
-          // the step's new token must land in a private page
-          if (a.fused && gp * kPage == n) flag_error(a.err, kErrSlot);
-        }
-      }
-    }
-  }
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) write_skip(a, cap);
 
   const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
   const int h = blockIdx.y;
@@ -236,9 +243,454 @@ __global__ void __launch_bounds__(32 * kWarps, 1)
   }
 }
 
+// ------------------------------------------------------------------------
+// The same pass on the 5th-generation tensor cores (d = 128).
+//
+// The 128 query rows of a CTA are the M dimension of tcgen05.mma, so every
+// staged K/V byte is read from shared memory once by the tensor core for all
+// rows (the warp-level tile above re-reads each page once per warp).  Per
+// step of kTcPages pages (N = 64 tokens):
+//   S[128 x N]  = Q[128 x d] . K^T      Q and K page rows in smem
+//   softmax     one thread per row reads its S row from TMEM, keeps the
+//               running (max, sum) and writes P (16-bit) over that S in TMEM
+//   O[128 x d] += P[128 x N] . V         P in TMEM (A), V rows in smem (B)
+// with fp32 accumulators S and O in TMEM.  The running max is a reference
+// that only moves when a row's maximum exceeds it by more than 2^8; below
+// that the probabilities stay <= 256 (exact enough in f16/bf16 and fp32), so
+// O is rescaled in TMEM only on the rare steps that move it.
+//
+// Each CTA takes half of TMEM (O and two S/P buffers, 256 columns) and about
+// 100 KB of shared memory, so two CTAs share an SM and one's softmax overlaps
+// the other's MMAs and copies.
+//
+// Roles (192 threads): warp 0 allocates TMEM and its lane 0 issues the TMA
+// loads of K/V into a kTcStages-deep ring; warp 1 lane 0 issues the MMAs;
+// warps 2-5 (TMEM lane quarters 2, 3, 0, 1) do the softmax, the O
+// corrections and the epilogue.  Hand-offs are mbarriers: TMA -> MMA (one
+// "full" barrier for the K half and one for the V half of a stage), MMA ->
+// TMA ("empty": a stage's K is released once QK^T has read it, its V after
+// the PV product, so the next K copy starts a whole step earlier), MMA ->
+// softmax (s_full), softmax -> MMA (p_full), and o_done (one phase per PV
+// product) before the softmax touches O.  The S/P buffers are double
+// buffered so QK^T of step j+1 runs during the softmax of step j; QK^T of
+// step j+2 overwrites the P of step j only after the PV product reading it
+// (MMAs of one thread run in issue order).
+// Every wait is bounded; a timed-out role flags the error word and the CTA
+// still releases its TMEM after the MMAs it issued have completed.
+namespace {
+constexpr int kTcPages = 4;                       // pages per step
+constexpr int kTcTok = kTcPages * kPage;          // N of QK^T: 64 tokens
+constexpr int kTcStages = 2;                      // steps of K/V in flight per CTA
+constexpr int kTcWarps = 6;
+constexpr int kTcHalf = kTcPages * kPage * 128;   // one 64-column half of a step's K (or V): 8 KB
+constexpr int kTcStage = 4 * kTcHalf;             // K half 0, K half 1, V half 0, V half 1
+constexpr int kTcQBytes = kRowsPerCta * 128 * 2;  // Q tile, two 64-column halves: 32 KB
+constexpr uint32_t kColO = 0;                     // O: 128 fp32 columns
+constexpr uint32_t kColS = 128;                   // S: 2 x 64 fp32 columns; P overwrites S
+constexpr uint32_t kTmemCols = 256;
+constexpr float kRefSlack = 8.f;                  // log2 of the largest probability kept
+constexpr int kTcBars = 4 * kTcStages + 7;
+constexpr size_t kTcSmem = 1024 + kTcQBytes + (size_t)kTcStages * kTcStage + kTcBars * 8 + 64;
+// two CTAs per SM share its 512 TMEM columns; a third never fits beside them
+static_assert(2 * kTcSmem <= 227 * 1024 && 3 * kTcSmem > 228 * 1024,
+              "exactly two CTAs per SM: each allocates half of TMEM");
+}  // namespace
+
+template <typename T>
+__global__ void __launch_bounds__(32 * kTcWarps, 2)
+    prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV) {
+  constexpr int D = 128;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  using M = Mma<T>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *qs = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  uint8_t *ring = qs + kTcQBytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ring + (size_t)kTcStages * kTcStage);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kTcBars);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cap = a.maxb * kPage;
+
+  grid_dependency_wait();
+  grid_launch_dependents();
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) write_skip(a, cap);
+
+  const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
+  const int h = blockIdx.y;
+  const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
+  const int gp = __ldg(a.group_pages + g);
+  if (s0 < 0 || s1 > a.B || s1 < s0 || gp < 0 || gp > a.maxb) {
+    if (tid == 0) flag_error(a.err, kErrSeqLen);
+    return;
+  }
+  const int rows = (s1 - s0) * a.G;
+  const int r0 = blockIdx.z * kRowsPerCta;
+  if (r0 >= rows || gp == 0) return;
+  const int p_begin = static_cast<int>((static_cast<long long>(chunk) * gp) / a.chunks);
+  const int p_end = static_cast<int>((static_cast<long long>(chunk + 1) * gp) / a.chunks);
+  const int nsteps = (p_end - p_begin + kTcPages - 1) / kTcPages;
+  if (nsteps == 0) {  // an empty chunk leaves empty partials
+    for (int r = tid; r < kRowsPerCta; r += blockDim.x) {
+      const int row = r0 + r;
+      if (row >= rows) continue;
+      const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + s0 + row / a.G) * a.G +
+                         row % a.G;
+      for (int c = 0; c < D; ++c) a.pre_o[idx * D + c] = 0.f;
+      a.pre_lse[idx] = -INFINITY;
+    }
+    return;
+  }
+  const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
+  auto step_pages = [&](int j) { return min(kTcPages, p_end - (p_begin + j * kTcPages)); };
+  // pages of step j that exist (bit p: page p of the step)
+  auto step_mask = [&](int j) -> uint32_t {
+    uint32_t m = 0;
+    if (j < nsteps) {
+      const int p0 = p_begin + j * kTcPages, np = step_pages(j);
+#pragma unroll
+      for (int p = 0; p < kTcPages; ++p) {
+        const int pb = p < np ? __ldg(bt + p0 + p) : -1;
+        if (pb >= 0 && pb < a.num_blocks) m |= 1u << p;
+      }
+    }
+    return m;
+  };
+
+  const uint32_t q0 = smem_u32(qs), ring0 = smem_u32(ring), bar0 = smem_u32(bars);
+  // K and V halves of a stage have their own barriers: K is released as soon
+  // as QK^T has read it, V after the PV product
+  auto FULL_K = [&](int s) { return bar0 + 8 * s; };
+  auto FULL_V = [&](int s) { return bar0 + 8 * (kTcStages + s); };
+  auto EMPTY_K = [&](int s) { return bar0 + 8 * (2 * kTcStages + s); };
+  auto EMPTY_V = [&](int s) { return bar0 + 8 * (3 * kTcStages + s); };
+  const uint32_t S_FULL = bar0 + 8 * (4 * kTcStages);  // + 8 * buffer
+  const uint32_t P_FULL = S_FULL + 16;                 // + 8 * buffer
+  const uint32_t O_DONE = S_FULL + 32, Q_FULL = S_FULL + 40, DRAIN = S_FULL + 48;
+
+  if (warp == 0) {
+    __syncwarp();
+    tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  if (tid == 32) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(FULL_K(s), 1);
+      mbar_init(FULL_V(s), 1);
+      mbar_init(EMPTY_K(s), 1);
+      mbar_init(EMPTY_V(s), 1);
+    }
+    mbar_init(S_FULL, 1);
+    mbar_init(S_FULL + 8, 1);
+    mbar_init(P_FULL, 4);
+    mbar_init(P_FULL + 8, 4);
+    mbar_init(O_DONE, 1);
+    mbar_init(Q_FULL, 4);
+    mbar_init(DRAIN, 1);
+    mbar_init_fence();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      const uint64_t policy = l2_policy_evict_normal();
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < nsteps; ++j) {
+        const int s = j % kTcStages;
+        const uint32_t rel = ((j / kTcStages) - 1) & 1;  // phase of step j - kTcStages
+        const int p0 = p_begin + j * kTcPages, np = step_pages(j);
+        int prow[kTcPages];
+        int good = 0;
+#pragma unroll
+        for (int p = 0; p < kTcPages; ++p) {
+          prow[p] = -1;
+          if (p < np) {
+            const int pb = __ldg(bt + p0 + p);
+            if (pb >= 0 && pb < a.num_blocks) {
+              prow[p] = (pb * a.H_kv + h) * kPage;
+              ++good;
+            } else {
+              flag_error(a.err, kErrBlockTable);
+            }
+          }
+        }
+        const uint32_t st = ring0 + s * kTcStage;
+        const uint32_t bytes = static_cast<uint32_t>(good) * 2 * kPage * 128;
+        // K of step j, once QK^T of step j - kTcStages has read the stage's K
+        if (j >= kTcStages && !mbar_wait_bounded(EMPTY_K(s), rel)) {
+          flag_error(a.err, kErrTimeout);
+          break;
+        }
+        mbar_arrive_expect_tx(FULL_K(s), bytes);
+#pragma unroll
+        for (int p = 0; p < kTcPages; ++p) {
+          if (prow[p] < 0) continue;
+          tma_load_3d(st + p * kPage * 128, &tmK, 0, 0, prow[p], FULL_K(s), policy);
+          tma_load_3d(st + kTcHalf + p * kPage * 128, &tmK, 0, 1, prow[p], FULL_K(s), policy);
+        }
+        issued_k = j + 1;
+        // V of step j, once the PV product of step j - kTcStages has read its V
+        if (j >= kTcStages && !mbar_wait_bounded(EMPTY_V(s), rel)) {
+          flag_error(a.err, kErrTimeout);
+          break;
+        }
+        mbar_arrive_expect_tx(FULL_V(s), bytes);
+#pragma unroll
+        for (int p = 0; p < kTcPages; ++p) {
+          if (prow[p] < 0) continue;
+          tma_load_3d(st + 2 * kTcHalf + p * kPage * 128, &tmV, 0, 0, prow[p], FULL_V(s), policy);
+          tma_load_3d(st + 3 * kTcHalf + p * kPage * 128, &tmV, 0, 1, prow[p], FULL_V(s), policy);
+        }
+        issued_v = j + 1;
+      }
+      // the copies of the last stages have landed before the CTA exits
+      for (int j = max(0, issued_k - kTcStages); j < issued_k; ++j)
+        mbar_wait_bounded(FULL_K(j % kTcStages), (j / kTcStages) & 1);
+      for (int j = max(0, issued_v - kTcStages); j < issued_v; ++j)
+        mbar_wait_bounded(FULL_V(j % kTcStages), (j / kTcStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t fmt = kBf16 ? 1u : 0u;
+      bool ok = mbar_wait_bounded(Q_FULL, 0);
+      tc::fence_after_sync();
+      bool o_started = false;
+      auto issue_qk = [&](int j) {
+        const int b = j & 1;
+        const uint32_t idesc = tc::idesc_f16(fmt, static_cast<uint32_t>(step_pages(j) * kPage), false);
+        const uint32_t kst = ring0 + (j % kTcStages) * kTcStage;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t kaddr = kst + (k >> 2) * kTcHalf + (k & 3) * 32;
+          const uint32_t qaddr = q0 + (k >> 2) * (kTcQBytes / 2) + (k & 3) * 32;
+          tc::mma_ss(tbase + kColS + b * kTcTok, tc::smem_desc(qaddr, 16, 1024),
+                     tc::smem_desc(kaddr, 16, 1024), idesc, k > 0);
+        }
+        tc::commit(EMPTY_K(j % kTcStages));
+        tc::commit(S_FULL + 8 * b);
+      };
+      uint32_t pv_mask0 = 0u, pv_mask1 = 0u;  // loaded one step before the PV product uses it
+      auto issue_pv = [&](int j) {
+        const int b = j & 1, s = j % kTcStages;
+        const int np = step_pages(j);
+        const uint32_t mask = (j & 1) ? pv_mask1 : pv_mask0;
+        const uint32_t idesc = tc::idesc_f16(fmt, D, true);
+        const uint32_t vst = ring0 + s * kTcStage + 2 * kTcHalf;
+        for (int kk = 0; kk < np; ++kk) {
+          if (!((mask >> kk) & 1u)) continue;  // (its scores are masked; its stage bytes are stale)
+          const uint64_t vd = tc::smem_desc(vst + kk * kPage * 128, kTcHalf, 1024);
+          const uint32_t pa = tbase + kColS + b * kTcTok + kk * 8;  // P over S; remainder at +32
+          tc::mma_ts(tbase + kColO, pa, vd, idesc, o_started);
+          o_started = true;
+          if (kBf16) tc::mma_ts(tbase + kColO, pa + kTcTok / 2, vd, idesc, true);
+        }
+        tc::commit(EMPTY_V(s));
+        tc::commit(O_DONE);
+      };
+      // the PV product of step j waits for its probabilities and its V pages
+      auto wait_pv = [&](int j) {
+        return mbar_wait_bounded(P_FULL + 8 * (j & 1), (j >> 1) & 1) &&
+               mbar_wait_bounded(FULL_V(j % kTcStages), (j / kTcStages) & 1);
+      };
+      for (int j = 0; ok && j < nsteps; ++j) {
+        if (j & 1) pv_mask1 = step_mask(j); else pv_mask0 = step_mask(j);
+        if (!mbar_wait_bounded(FULL_K(j % kTcStages), (j / kTcStages) & 1)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        issue_qk(j);
+        if (j >= 1) {
+          if (!wait_pv(j - 1)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          issue_pv(j - 1);
+        }
+      }
+      if (ok) {
+        const int j = nsteps - 1;
+        if (wait_pv(j)) {
+          tc::fence_after_sync();
+          issue_pv(j);
+        } else {
+          ok = false;
+        }
+      }
+      if (!ok) flag_error(a.err, kErrTimeout);
+      // every MMA issued here completes before TMEM is released
+      tc::commit(DRAIN);
+      mbar_wait_bounded(DRAIN, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
+    const int row = r0 + quarter * 32 + lane;  // row of the group: member row / G, head row % G
+    const bool live = row < rows;
+    const int b = s0 + (live ? row / a.G : 0), jr = live ? row % a.G : 0;
+    {
+      // this row of Q into the K-major, 128-byte-swizzled tile the MMA reads
+      const int r = quarter * 32 + lane;
+      const uint4 *qv = reinterpret_cast<const uint4 *>(
+          static_cast<const T *>(a.q) +
+          (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + jr) * D);
+#pragma unroll
+      for (int c = 0; c < 2 * 8; ++c) {
+        const uint4 v = live ? __ldg(qv + c) : make_uint4(0u, 0u, 0u, 0u);
+        const int half = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4 *>(qs + half * (kTcQBytes / 2) + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();  // visible to the tensor core's reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(Q_FULL);
+    }
+
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    uint32_t next_mask = step_mask(0);  // loaded one step before use
+    for (int j = 0; j < nsteps; ++j) {
+      const int bs = j & 1;
+      const uint32_t pm = next_mask;
+      next_mask = step_mask(j + 1);
+      const bool got = mbar_wait_bounded(S_FULL + 8 * bs, (j >> 1) & 1);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      float x[kTcTok];
+      {
+        uint32_t r0v[32], r1v[32];
+        tc::ld32(tbase + lanes + kColS + bs * kTcTok, r0v);
+        tc::ld32(tbase + lanes + kColS + bs * kTcTok + 32, r1v);
+        tc::wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          x[i] = __uint_as_float(r0v[i]);
+          x[32 + i] = __uint_as_float(r1v[i]);
+        }
+      }
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int i = 0; i < kTcTok; ++i) {
+        x[i] = ((pm >> (i / kPage)) & 1u) ? x[i] * a.scale_log2 : -INFINITY;
+        mx4[i & 3] = fmaxf(mx4[i & 3], x[i]);
+      }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      const float m_new = mx > m_ref + kRefSlack ? mx : m_ref;
+      const float alpha = m_new == m_ref ? 1.f : fast_exp2(m_ref - m_new);
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      uint32_t ph[kTcTok / 2], pl[kTcTok / 2];
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < kTcTok; i += 2) {
+        const float e0 = fast_exp2(x[i] - m_use), e1 = fast_exp2(x[i + 1] - m_use);
+        ph[i / 2] = M::pack(e0, e1);
+        const float2 r = M::unpack(ph[i / 2]);
+        if constexpr (kBf16) {
+          pl[i / 2] = M::pack(e0 - r.x, e1 - r.y);
+          sum4[(i / 2) & 3] += e0 + e1;
+        } else {
+          sum4[(i / 2) & 3] += r.x + r.y;  // the sum of the values the PV product uses
+        }
+      }
+      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      l = l * alpha + sum;
+      tc::st32(tbase + lanes + kColS + bs * kTcTok, ph);
+      if constexpr (kBf16) tc::st32(tbase + lanes + kColS + bs * kTcTok + kTcTok / 2, pl);
+      if (j >= 1) {
+        // O holds the product of step j-1 once its o_done phase completes
+        const bool got2 = mbar_wait_bounded(O_DONE, (j - 1) & 1);
+        if (!__all_sync(0xffffffffu, got2)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tc::ld32(tbase + lanes + kColO + c * 32, r);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tc::st32(tbase + lanes + kColO + c * 32, r);
+          }
+        }
+      }
+      m_ref = m_new;
+      tc::wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(P_FULL + 8 * bs);
+    }
+    if (ok) {
+      const bool got = mbar_wait_bounded(O_DONE, (nsteps - 1) & 1);
+      ok = __all_sync(0xffffffffu, got);
+    }
+    if (!ok) {
+      if (lane == 0) flag_error(a.err, kErrTimeout);
+    } else {
+      tc::fence_after_sync();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float lse = l > 0.f ? (m_ref + fast_log2(l)) * kLn2 : -INFINITY;
+      const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + b) * a.G + jr;
+      float4 *o = reinterpret_cast<float4 *>(a.pre_o + idx * D);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tc::ld32(tbase + lanes + kColO + c * 32, r);
+        tc::wait_ld();
+        if (live) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 v = l > 0.f ? make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
+                                                   __uint_as_float(r[i + 2]) * inv,
+                                                   __uint_as_float(r[i + 3]) * inv)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+            o[c * 8 + i / 4] = v;
+          }
+        }
+        __syncwarp();
+      }
+      if (live) a.pre_lse[idx] = lse;
+    }
+  }
+
+  // release TMEM once every role is done with it
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
 int prefix_rows_per_cta() { return kRowsPerCta; }
 
 namespace {
+template <typename T>
+cudaError_t launch_prefix_tc_t(const PrefixArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                               int row_blocks, cudaStream_t st) {
+  auto kern = prefix_tc_kernel<T>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kTcSmem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.n_groups * a.chunks, a.H_kv, row_blocks);
+  return launch_pdl(kern, grid, dim3(32 * kTcWarps), kTcSmem, st, a, tmK, tmV);
+}
+
 template <int D, typename T>
 cudaError_t launch_prefix_t(const PrefixArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                             int row_blocks, cudaStream_t st) {
@@ -255,6 +707,11 @@ cudaError_t launch_prefix_t(const PrefixArgs &a, const CUtensorMap &tmK, const C
 cudaError_t launch_prefix(const PrefixArgs &a, int d, DType dt, const CUtensorMap &tmK,
                           const CUtensorMap &tmV, int row_blocks, cudaStream_t s) {
   if (a.n_groups == 0 || a.B == 0) return cudaSuccess;
+#ifndef KVD_PREFIX_MMA_SYNC
+  if (d == 128)
+    return dt == DType::BF16 ? launch_prefix_tc_t<__nv_bfloat16>(a, tmK, tmV, row_blocks, s)
+                             : launch_prefix_tc_t<__half>(a, tmK, tmV, row_blocks, s);
+#endif
   if (dt == DType::BF16)
     return d == 128 ? launch_prefix_t<128, __nv_bfloat16>(a, tmK, tmV, row_blocks, s)
                     : launch_prefix_t<64, __nv_bfloat16>(a, tmK, tmV, row_blocks, s);
