@@ -478,15 +478,9 @@ kvd_status kvd_append_fp8(uint8_t *k_codes, uint8_t *v_codes, float *k_scale, fl
   const kvd::DType dt = dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long long n = static_cast<long long>(B) * H_kv;
-  kvd::QuantArgs qk{k_new, k_codes, k_scale, block_table, slot, err, n, d, H_kv, num_blocks,
-                    max_blocks_per_seq, 1};
-  cudaError_t e = kvd::launch_quantize_fp8(qk, dt, s);
-  if (e != cudaSuccess) return cuda_fail(e, "append launch");
-  kvd::QuantArgs qv = qk;
-  qv.src = v_new;
-  qv.codes = v_codes;
-  qv.scales = v_scale;
-  e = kvd::launch_quantize_fp8(qv, dt, s);
+  kvd::QuantArgs qa{k_new, k_codes, k_scale, block_table, slot, err, n, d, H_kv, num_blocks,
+                    max_blocks_per_seq, 1, v_new, v_codes, v_scale};
+  cudaError_t e = kvd::launch_quantize_fp8(qa, dt, s);
   if (e != cudaSuccess) return cuda_fail(e, "append launch");
   return KVD_OK;
 }

@@ -67,6 +67,11 @@ struct QuantArgs {
   long long n;            // source rows
   int d, H_kv, num_blocks, maxb;
   int append;             // 1: src is [B][H_kv][d] and goes to page rows per slot
+  // optional second tensor (append mode): rows n..2n-1 of the launch quantise
+  // src2 into codes2 / scales2 (the V rows of an append next to the K rows)
+  const void *src2;
+  uint8_t *codes2;
+  float *scales2;
 };
 
 struct PrefixArgs {

@@ -580,30 +580,56 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
           x[32 + i] = __uint_as_float(r1v[i]);
         }
       }
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // row maximum of the scaled scores (in log2 units): the scale is folded
+      // into the exponent below, so the raw scores are compared (their
+      // minimum when the scale is negative); masked columns are -inf
+      const float c = a.scale_log2;
+      const bool full_step = pm == (1u << kTcPages) - 1u;  // warp-uniform
+      if (!full_step) {
 #pragma unroll
-      for (int i = 0; i < kTcTok; ++i) {
-        x[i] = ((pm >> (i / kPage)) & 1u) ? x[i] * a.scale_log2 : -INFINITY;
-        mx4[i & 3] = fmaxf(mx4[i & 3], x[i]);
+        for (int i = 0; i < kTcTok; ++i)
+          if (!((pm >> (i / kPage)) & 1u)) x[i] = c >= 0.f ? -INFINITY : INFINITY;
       }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      float e4[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) e4[k] = x[k];
+      if (c >= 0.f) {
+#pragma unroll
+        for (int i = 4; i < kTcTok; ++i) e4[i & 3] = fmaxf(e4[i & 3], x[i]);
+      } else {
+#pragma unroll
+        for (int i = 4; i < kTcTok; ++i) e4[i & 3] = fminf(e4[i & 3], x[i]);
+      }
+      const float ext = c >= 0.f ? fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]))
+                                 : fminf(fminf(e4[0], e4[1]), fminf(e4[2], e4[3]));
+      // an all-masked row keeps -inf; otherwise the largest scaled score
+      const float mx = (ext == INFINITY || ext == -INFINITY) ? -INFINITY : ext * c;
       const float m_new = mx > m_ref + kRefSlack ? mx : m_ref;
       const float alpha = m_new == m_ref ? 1.f : fast_exp2(m_ref - m_new);
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
       uint32_t ph[kTcTok / 2], pl[kTcTok / 2];
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      // exp2(s * c - m) per column; masked columns (partial steps only) are 0
+      auto exps = [&](auto masked) {
 #pragma unroll
-      for (int i = 0; i < kTcTok; i += 2) {
-        const float e0 = fast_exp2(x[i] - m_use), e1 = fast_exp2(x[i + 1] - m_use);
-        ph[i / 2] = M::pack(e0, e1);
-        const float2 r = M::unpack(ph[i / 2]);
-        if constexpr (kBf16) {
-          pl[i / 2] = M::pack(e0 - r.x, e1 - r.y);
+        for (int i = 0; i < kTcTok; i += 2) {
+          float e0 = fast_exp2(fmaf(x[i], c, -m_use));
+          float e1 = fast_exp2(fmaf(x[i + 1], c, -m_use));
+          if constexpr (decltype(masked)::value) {
+            const bool v = (pm >> (i / kPage)) & 1u;  // both columns are in one page
+            e0 = v ? e0 : 0.f;
+            e1 = v ? e1 : 0.f;
+          }
+          ph[i / 2] = M::pack(e0, e1);
+          if constexpr (kBf16) {
+            const float2 r = M::unpack(ph[i / 2]);
+            pl[i / 2] = M::pack(e0 - r.x, e1 - r.y);
+          }
           sum4[(i / 2) & 3] += e0 + e1;
-        } else {
-          sum4[(i / 2) & 3] += r.x + r.y;  // the sum of the values the PV product uses
         }
-      }
+      };
+      if (full_step) exps(std::false_type{});
+      else exps(std::true_type{});
       const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l = l * alpha + sum;
       tc::st32(tbase + lanes + kColS + bs * kTcTok, ph);

@@ -10,8 +10,9 @@
 //
 // One warp per row: lane l holds channels 4l..4l+3, a group is 8 lanes and
 // its maximum is three shuffles.  In append mode the source rows are the
-// step's k_new (or v_new) [B][H_kv][d] and each goes to row slot % 16 of page
-// block_table[b][slot / 16] of the code and scale pools.
+// step's k_new and v_new [B][H_kv][d] (one launch, K rows then V rows) and
+// each goes to row slot % 16 of page block_table[b][slot / 16] of its code
+// and scale pools.
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -21,9 +22,17 @@ namespace kvd {
 
 template <typename T>
 __global__ void __launch_bounds__(256) quantize_fp8_kernel(const QuantArgs a) {
+  // programmatic dependent launch: wait for the preceding grid's writes
+  grid_dependency_wait();
+  grid_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long r = static_cast<long long>(blockIdx.x) * 8 + warp;
+  long long r = static_cast<long long>(blockIdx.x) * 8 + warp;
+  const bool second = a.src2 != nullptr && r >= a.n;
+  if (second) r -= a.n;
   if (r >= a.n) return;
+  const void *src = second ? a.src2 : a.src;
+  uint8_t *codes = second ? a.codes2 : a.codes;
+  float *scales = second ? a.scales2 : a.scales;
   long long dst = r;
   if (a.append) {
     const int b = static_cast<int>(r / a.H_kv), h = static_cast<int>(r % a.H_kv);
@@ -43,7 +52,7 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(const QuantArgs a) {
   const bool live = lane * 4 < a.d;
   float x[4] = {0.f, 0.f, 0.f, 0.f};
   if (live) {
-    const uint2 w = *reinterpret_cast<const uint2 *>(static_cast<const T *>(a.src) + r * a.d + lane * 4);
+    const uint2 w = *reinterpret_cast<const uint2 *>(static_cast<const T *>(src) + r * a.d + lane * 4);
     const T *v = reinterpret_cast<const T *>(&w);
 #pragma unroll
     for (int i = 0; i < 4; ++i) x[i] = static_cast<float>(v[i]);
@@ -59,16 +68,16 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(const QuantArgs a) {
   if (!live) return;
   const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(q[0], q[1]), __NV_SATFINITE, __NV_E4M3);
   const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(q[2], q[3]), __NV_SATFINITE, __NV_E4M3);
-  *reinterpret_cast<uint32_t *>(a.codes + dst * a.d + lane * 4) = (lo & 0xffffu) | (hi << 16);
-  if ((lane & 7) == 0) a.scales[dst * (a.d / 32) + (lane >> 3)] = s;
+  *reinterpret_cast<uint32_t *>(codes + dst * a.d + lane * 4) = (lo & 0xffffu) | (hi << 16);
+  if ((lane & 7) == 0) scales[dst * (a.d / 32) + (lane >> 3)] = s;
 }
 
 cudaError_t launch_quantize_fp8(const QuantArgs &a, DType dt, cudaStream_t s) {
   if (a.n == 0) return cudaSuccess;
-  const unsigned grid = static_cast<unsigned>((a.n + 7) / 8);
-  if (dt == DType::BF16) quantize_fp8_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
-  else quantize_fp8_kernel<__half><<<grid, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  const long long rows = a.src2 ? 2 * a.n : a.n;
+  const dim3 grid(static_cast<unsigned>((rows + 7) / 8));
+  if (dt == DType::BF16) return launch_pdl(quantize_fp8_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, a);
+  return launch_pdl(quantize_fp8_kernel<__half>, grid, dim3(256), 0, s, a);
 }
 
 }  // namespace kvd

@@ -373,6 +373,27 @@ def test_shared_prefix_matches_oracle_and_plain_decode(kvd, case):
     assert kvd.kvd_read_device_error() == 0
 
 
+@pytest.mark.parametrize("scale", [-0.09, 0.0])
+def test_shared_prefix_any_scale(kvd, scale):
+    # a negative scale turns the row maximum into a minimum of the raw scores;
+    # a zero scale gives uniform weights (the mean of V over the sequence)
+    lens = [300, 257, 520, 999, 290, 400, 700, 266]
+    w = build_workload("spscale", 8, 32, 8, 128, "f16", lens, seed=981, prefix_groups=2,
+                       prefix_tokens=256, scale=scale)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    gs, gp, per = groups_of(w)
+    lse = torch.empty((w.B, w.H_q), dtype=torch.float32, device="cuda")
+    out = kvd.kvd_decode_attention_shared_prefix(si["q"].cuda(), kc, vc, bt, si["seq_lens"].cuda(),
+                                                 gs, gp, per, w.scale, k_new=si["k_new"].cuda(),
+                                                 v_new=si["v_new"].cuda(), lse_out=lse)
+    torch.cuda.synchronize()
+    _, _, ref = oracle_step(w, si)
+    assert max_err(out, ref) <= TOL[w.dtype]
+    assert max_lse_err(lse, ref) <= LSE_TOL
+    assert kvd.kvd_read_device_error() == 0
+
+
 def test_shared_prefix_bad_page_is_flagged_and_contained(kvd):
     # a block-table entry of group 0's shared prefix points outside the pool:
     # the error word says so and group 1 is still exact
