@@ -63,6 +63,17 @@ def load(path):
     L.orc_attend_fp8.restype = i32
     L.orc_attend_fp8.argtypes = [P, P, P, P, P, P, P, ctypes.c_double, i32, i32, i32, i32, i32,
                                  i32, i32, P, P, i32]
+    L.orc_int8_decode.restype = ctypes.c_double
+    L.orc_int8_decode.argtypes = [ctypes.c_uint8]
+    L.orc_int8_encode.restype = ctypes.c_uint8
+    L.orc_int8_encode.argtypes = [ctypes.c_float]
+    L.orc_quantize_int8.restype = i32
+    L.orc_quantize_int8.argtypes = [P, i32, i32, i32, P, P]
+    L.orc_append_int8.restype = i32
+    L.orc_append_int8.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32]
+    L.orc_attend_int8.restype = i32
+    L.orc_attend_int8.argtypes = [P, P, P, P, P, P, P, ctypes.c_double, i32, i32, i32, i32, i32,
+                                  i32, i32, P, P, i32]
     return L
 
 
@@ -201,20 +212,17 @@ def e4m3_encode(x):
     return int(lib().orc_e4m3_encode(float(x)))
 
 
-def quantize_fp8(rows, dtype):
-    """rows [..., d] storage words -> (codes uint8 [..., d], scales float32 [..., d/32])."""
+def _quantize8(fn, rows, dtype):
     rows = _words(rows)
     d = rows.shape[-1]
     n = rows.size // d
     codes = np.zeros(rows.shape, dtype=np.uint8)
     scales = np.zeros(rows.shape[:-1] + (d // FP8_GROUP,), dtype=np.float32)
-    _check(lib().orc_quantize_fp8(_ptr(rows), n, d, dtype, _ptr(codes), _ptr(scales)),
-           "orc_quantize_fp8")
+    _check(getattr(lib(), fn)(_ptr(rows), n, d, dtype, _ptr(codes), _ptr(scales)), fn)
     return codes, scales
 
 
-def append_fp8(k8, v8, ks, vs, block_table, slot, k_new, v_new, dtype):
-    """In-place quantised scatter into codes [NB,H_kv,16,d] and scales [NB,H_kv,16,d/32]."""
+def _append8(fn, k8, v8, ks, vs, block_table, slot, k_new, v_new, dtype):
     for a in (k8, v8):
         assert a.dtype == np.uint8 and a.flags.c_contiguous
     for a in (ks, vs):
@@ -222,23 +230,60 @@ def append_fp8(k8, v8, ks, vs, block_table, slot, k_new, v_new, dtype):
     k_new, v_new = _words(k_new), _words(v_new)
     bt, sl = _i32(block_table), _i32(slot)
     NB, H_kv, P, d = k8.shape
-    _check(lib().orc_append_fp8(_ptr(k8), _ptr(v8), _ptr(ks), _ptr(vs), _ptr(bt), _ptr(sl),
-                                _ptr(k_new), _ptr(v_new), k_new.shape[0], H_kv, d, NB,
-                                bt.shape[1], dtype),
-           "orc_append_fp8")
+    _check(getattr(lib(), fn)(_ptr(k8), _ptr(v8), _ptr(ks), _ptr(vs), _ptr(bt), _ptr(sl),
+                              _ptr(k_new), _ptr(v_new), k_new.shape[0], H_kv, d, NB,
+                              bt.shape[1], dtype), fn)
 
 
-def attend_fp8(q, k8, v8, ks, vs, block_table, seq_lens, scale, dtype, nthreads=0):
-    """Attention (binary64) over the dequantised 8-bit cache -> (out, lse)."""
+def _attend8(fn, q, k8, v8, ks, vs, block_table, seq_lens, scale, dtype, nthreads):
     q = _words(q)
     bt, sl = _i32(block_table), _i32(seq_lens)
     B, H_q, d = q.shape
     NB, H_kv, P, _ = k8.shape
     out = np.zeros((B, H_q, d), dtype=np.float64)
     lse = np.zeros((B, H_q), dtype=np.float64)
-    _check(lib().orc_attend_fp8(_ptr(q), _ptr(np.ascontiguousarray(k8)), _ptr(np.ascontiguousarray(v8)),
-                                _ptr(np.ascontiguousarray(ks)), _ptr(np.ascontiguousarray(vs)),
-                                _ptr(bt), _ptr(sl), float(scale), B, H_q, H_kv, d, NB,
-                                bt.shape[1], dtype, _ptr(out), _ptr(lse), int(nthreads)),
-           "orc_attend_fp8")
+    _check(getattr(lib(), fn)(_ptr(q), _ptr(np.ascontiguousarray(k8)), _ptr(np.ascontiguousarray(v8)),
+                              _ptr(np.ascontiguousarray(ks)), _ptr(np.ascontiguousarray(vs)),
+                              _ptr(bt), _ptr(sl), float(scale), B, H_q, H_kv, d, NB,
+                              bt.shape[1], dtype, _ptr(out), _ptr(lse), int(nthreads)), fn)
     return out, lse
+
+
+def quantize_fp8(rows, dtype):
+    """rows [..., d] storage words -> (codes uint8 [..., d], scales float32 [..., d/32])."""
+    return _quantize8("orc_quantize_fp8", rows, dtype)
+
+
+def append_fp8(k8, v8, ks, vs, block_table, slot, k_new, v_new, dtype):
+    """In-place quantised scatter into codes [NB,H_kv,16,d] and scales [NB,H_kv,16,d/32]."""
+    _append8("orc_append_fp8", k8, v8, ks, vs, block_table, slot, k_new, v_new, dtype)
+
+
+def attend_fp8(q, k8, v8, ks, vs, block_table, seq_lens, scale, dtype, nthreads=0):
+    """Attention (binary64) over the dequantised 8-bit cache -> (out, lse)."""
+    return _attend8("orc_attend_fp8", q, k8, v8, ks, vs, block_table, seq_lens, scale, dtype,
+                    nthreads)
+
+
+def int8_decode(code):
+    return lib().orc_int8_decode(int(code))
+
+
+def int8_encode(x):
+    return int(lib().orc_int8_encode(float(x)))
+
+
+def quantize_int8(rows, dtype):
+    """rows [..., d] storage words -> (codes as uint8 bytes of int8 [..., d], scales [..., d/32])."""
+    return _quantize8("orc_quantize_int8", rows, dtype)
+
+
+def append_int8(k8, v8, ks, vs, block_table, slot, k_new, v_new, dtype):
+    """In-place INT8 quantised scatter (same layout as append_fp8)."""
+    _append8("orc_append_int8", k8, v8, ks, vs, block_table, slot, k_new, v_new, dtype)
+
+
+def attend_int8(q, k8, v8, ks, vs, block_table, seq_lens, scale, dtype, nthreads=0):
+    """Attention (binary64) over the dequantised INT8 cache -> (out, lse)."""
+    return _attend8("orc_attend_int8", q, k8, v8, ks, vs, block_table, seq_lens, scale, dtype,
+                    nthreads)

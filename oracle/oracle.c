@@ -27,6 +27,10 @@
  *   orc_quantize_fp8 / orc_append_fp8 -- round-trip bound, per-group scales,
  *                                        outlier isolation, == numpy re-derivation
  *   orc_attend_fp8                    -- CPU float64 SDPA on the dequantised cache
+ *   orc_int8_decode / orc_int8_encode -- numpy int8 view; closed-form roundings
+ *   orc_quantize_int8 / orc_append_int8 / orc_attend_int8
+ *                                     -- half-step round trip, extreme -> +-127,
+ *                                        CPU float64 SDPA on the dequantised cache
  */
 #include <math.h>
 #include <stdint.h>
@@ -384,12 +388,15 @@ int orc_quantize_fp8(const uint16_t *rows, int n, int d, int dtype, uint8_t *cod
     return ORC_OK;
 }
 
-/* Append for the 8-bit cache: quantise k_new/v_new [B][H_kv][d] and write the
- * codes and scales of row slot[b] % 16 of page block_table[b][slot[b] / 16]
- * (codes [NB][H_kv][16][d], scales [NB][H_kv][16][d/32]). */
-int orc_append_fp8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t *block_table,
-                   const int32_t *slot, const uint16_t *k_new, const uint16_t *v_new, int B,
-                   int H_kv, int d, int num_blocks, int max_blocks, int dtype)
+/* Append for an 8-bit cache: quantise k_new/v_new [B][H_kv][d] with `quant`
+ * and write the codes and scales of row slot[b] % 16 of page
+ * block_table[b][slot[b] / 16] (codes [NB][H_kv][16][d], scales
+ * [NB][H_kv][16][d/32]). */
+typedef int (*orc_quant_fn)(const uint16_t *, int, int, int, uint8_t *, float *);
+
+static int append_kv8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t *block_table,
+                      const int32_t *slot, const uint16_t *k_new, const uint16_t *v_new, int B,
+                      int H_kv, int d, int num_blocks, int max_blocks, int dtype, orc_quant_fn quant)
 {
     if (!k8 || !v8 || !ks || !vs || !block_table || !slot || !k_new || !v_new) return ORC_ERR_ARGS;
     if (d % ORC_FP8_GROUP) return ORC_ERR_ARGS;
@@ -408,10 +415,10 @@ int orc_append_fp8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t
         for (int h = 0; h < H_kv; ++h) {
             size_t r = ((size_t)phys * H_kv + h) * ORC_PAGE_TOKENS + row;
             size_t src = ((size_t)b * H_kv + h) * (size_t)d;
-            orc_quantize_fp8(k_new + src, 1, d, dtype, code, sc);
+            quant(k_new + src, 1, d, dtype, code, sc);
             memcpy(k8 + r * d, code, (size_t)d);
             memcpy(ks + r * ng, sc, (size_t)ng * sizeof(float));
-            orc_quantize_fp8(v_new + src, 1, d, dtype, code, sc);
+            quant(v_new + src, 1, d, dtype, code, sc);
             memcpy(v8 + r * d, code, (size_t)d);
             memcpy(vs + r * ng, sc, (size_t)ng * sizeof(float));
         }
@@ -421,12 +428,22 @@ int orc_append_fp8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t
     return rc;
 }
 
-/* Attention over the 8-bit cache: exactly orc_attend's definition applied to
- * the dequantised values s * E4M3(code) (binary64).  q is fp16/bf16 words. */
-int orc_attend_fp8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, const float *ks,
-                   const float *vs, const int32_t *block_table, const int32_t *seq_lens,
-                   double scale, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks,
-                   int dtype, double *out, double *lse, int nthreads)
+int orc_append_fp8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t *block_table,
+                   const int32_t *slot, const uint16_t *k_new, const uint16_t *v_new, int B,
+                   int H_kv, int d, int num_blocks, int max_blocks, int dtype)
+{
+    return append_kv8(k8, v8, ks, vs, block_table, slot, k_new, v_new, B, H_kv, d, num_blocks,
+                      max_blocks, dtype, orc_quantize_fp8);
+}
+
+/* Attention over an 8-bit cache: exactly orc_attend's definition applied to
+ * the dequantised values s * dec(code) (binary64).  q is fp16/bf16 words. */
+typedef double (*orc_dec_fn)(uint8_t);
+
+static int attend_kv8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, const float *ks,
+                      const float *vs, const int32_t *block_table, const int32_t *seq_lens,
+                      double scale, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks,
+                      int dtype, double *out, double *lse, int nthreads, orc_dec_fn dec)
 {
     if (!q || !k8 || !v8 || !ks || !vs || !block_table || !seq_lens || !out) return ORC_ERR_ARGS;
     if (B < 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv || d <= 0 || d % ORC_FP8_GROUP) return ORC_ERR_ARGS;
@@ -456,7 +473,7 @@ int orc_attend_fp8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, cons
             const float *sk = ks + off / d * ng;
             double dot = 0.0;
             for (int i = 0; i < d; ++i)
-                dot += qv[i] * ((double)sk[i / ORC_FP8_GROUP] * orc_e4m3_decode(k8[off + i]));
+                dot += qv[i] * ((double)sk[i / ORC_FP8_GROUP] * dec(k8[off + i]));
             s[j] = scale * dot;
         }
         if (bad) { free(s); free(qv); status = ORC_ERR_RANGE; continue; }
@@ -469,7 +486,7 @@ int orc_attend_fp8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, cons
             long long off = token_offset(block_table, b, j, g, H_kv, d, num_blocks, max_blocks);
             const float *sv = vs + off / d * ng;
             for (int i = 0; i < d; ++i)
-                o[i] += w * ((double)sv[i / ORC_FP8_GROUP] * orc_e4m3_decode(v8[off + i]));
+                o[i] += w * ((double)sv[i / ORC_FP8_GROUP] * dec(v8[off + i]));
         }
         for (int i = 0; i < d; ++i) o[i] /= den;
         if (lse) lse[r] = m + log(den);
@@ -477,6 +494,79 @@ int orc_attend_fp8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, cons
         free(qv);
     }
     return status;
+}
+
+int orc_attend_fp8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, const float *ks,
+                   const float *vs, const int32_t *block_table, const int32_t *seq_lens,
+                   double scale, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks,
+                   int dtype, double *out, double *lse, int nthreads)
+{
+    return attend_kv8(q, k8, v8, ks, vs, block_table, seq_lens, scale, B, H_q, H_kv, d, num_blocks,
+                      max_blocks, dtype, out, lse, nthreads, orc_e4m3_decode);
+}
+
+/* Symmetric INT8 codes.  "KV Cache:推理慢的真正原因", section "工程优化手段 /
+ * 量化" (int8 or int4 storage, scales per channel group because of outlier
+ * keys); "推理速度慢怎么办？KV Cache与Flash Attention如何加速大模型推理", section
+ * "三、实际落地" (the cache kept in INT8 or even INT4).  Reading taken here:
+ * the same per-(token, KV head, 32-channel group) fp32 scale as the E4M3
+ * cache with s = max|x| / 127 (fp32 division), code = x / s (fp32 division)
+ * rounded to the nearest integer, ties to even, clamped to [-127, 127]; a
+ * NaN quotient gives code 0; a group of zeros gets s = 0 and codes 0.
+ * Dequantised value: s * code. */
+double orc_int8_decode(uint8_t c)
+{
+    return (double)(int8_t)c;
+}
+
+uint8_t orc_int8_encode(float x)
+{
+    if (isnan(x)) return 0;
+    double r = rint((double)x);               /* nearest, ties to even */
+    if (r > 127.0) r = 127.0;
+    if (r < -127.0) r = -127.0;
+    return (uint8_t)(int8_t)r;
+}
+
+int orc_quantize_int8(const uint16_t *rows, int n, int d, int dtype, uint8_t *codes, float *scales)
+{
+    if (!rows || !codes || !scales || n < 0 || d <= 0 || d % ORC_FP8_GROUP) return ORC_ERR_ARGS;
+    const int ng = d / ORC_FP8_GROUP;
+    for (long long r = 0; r < n; ++r) {
+        for (int g = 0; g < ng; ++g) {
+            const uint16_t *x = rows + r * d + g * ORC_FP8_GROUP;
+            float mx = 0.0f;
+            for (int i = 0; i < ORC_FP8_GROUP; ++i) {
+                float v = (float)fabs(decode_elem(x[i], dtype));
+                if (v > mx) mx = v;
+            }
+            volatile float s = mx / 127.0f;
+            scales[r * ng + g] = s;
+            for (int i = 0; i < ORC_FP8_GROUP; ++i) {
+                float v = (float)decode_elem(x[i], dtype);
+                volatile float qt = s == 0.0f ? 0.0f : v / s;
+                codes[r * d + g * ORC_FP8_GROUP + i] = s == 0.0f ? 0 : orc_int8_encode(qt);
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+int orc_append_int8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t *block_table,
+                    const int32_t *slot, const uint16_t *k_new, const uint16_t *v_new, int B,
+                    int H_kv, int d, int num_blocks, int max_blocks, int dtype)
+{
+    return append_kv8(k8, v8, ks, vs, block_table, slot, k_new, v_new, B, H_kv, d, num_blocks,
+                      max_blocks, dtype, orc_quantize_int8);
+}
+
+int orc_attend_int8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, const float *ks,
+                    const float *vs, const int32_t *block_table, const int32_t *seq_lens,
+                    double scale, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks,
+                    int dtype, double *out, double *lse, int nthreads)
+{
+    return attend_kv8(q, k8, v8, ks, vs, block_table, seq_lens, scale, B, H_q, H_kv, d, num_blocks,
+                      max_blocks, dtype, out, lse, nthreads, orc_int8_decode);
 }
 
 int orc_max_threads(void)

@@ -476,6 +476,107 @@ def check_append_fp8():
     assert not changed.any(), "fp8 append touched other rows"
 
 
+# ------------------------------------------------------------ INT8 cache
+
+def _i8(codes):
+    return np.ascontiguousarray(codes, dtype=np.uint8).view(np.int8).astype(np.float64)
+
+
+def check_int8_decoder():
+    codes = np.arange(256, dtype=np.uint8)
+    got = np.array([oracle.int8_decode(c) for c in codes])
+    assert np.array_equal(got, codes.view(np.int8).astype(np.float64)), "INT8 decoding differs"
+
+
+def check_int8_encoder():
+    # closed forms: nearest integer, ties to the even one, clamp at +-127, NaN -> 0
+    cases = {2.5: 2, 3.5: 4, -2.5: -2, 0.5: 0, 1.5: 2, -0.5: 0, 126.5: 126, 127.4: 127,
+             127.5: 127, 200.0: 127, -1e9: -127, -127.6: -127, 63.49: 63, -63.51: -64, 0.0: 0}
+    for x, want in cases.items():
+        got = np.uint8(oracle.int8_encode(x)).view(np.int8)
+        assert got == want, f"INT8 encode({x}) = {got}, expected {want}"
+    assert oracle.int8_encode(float("nan")) == 0
+    rng = np.random.default_rng(14)
+    x = rng.uniform(-127.4, 127.4, 5000).astype(np.float32)
+    got = _i8(np.array([oracle.int8_encode(v) for v in x], dtype=np.uint8))
+    assert np.all(np.abs(got - x.astype(np.float64)) <= 0.5), "INT8 encode is not the nearest integer"
+
+
+def check_quantize_int8():
+    rng = np.random.default_rng(15)
+    for dt, tdt in ((oracle.F16, torch.float16), (oracle.BF16, torch.bfloat16)):
+        x = torch.from_numpy(rng.standard_normal((64, 128)).astype(np.float32))
+        x[3, 17] = 40.0                        # an outlier channel in group 0 of row 3
+        x[5, 64:96] = 0.0                      # an all-zero group
+        x[9, 40] = float("nan")                # a NaN element (group 1 of row 9)
+        xq = x.to(tdt)
+        codes, scales = oracle.quantize_int8(to_words(xq), dt)
+        rows32 = xq.to(torch.float32).numpy().astype(np.float64)
+        deq = (_i8(codes).reshape(64, 4, 32) * scales[..., None]).reshape(64, 128)
+        fin = np.isfinite(rows32)
+        # every value within half a quantisation step of its group, plus the
+        # rounding of the fp32 quotient x / s the code is taken from (at most
+        # 127 * 2^-24 of a step: a quotient just below a half can round onto it)
+        step = scales.repeat(32, axis=1).astype(np.float64)
+        bound = step * (0.5 + 128 * 2.0 ** -24)
+        assert np.all(np.abs(deq - rows32)[fin] <= bound[fin]), "INT8 round trip exceeds half a step"
+        # the largest magnitude of each group is the extreme code, with its sign
+        g = np.where(fin, rows32, 0).reshape(64, 4, 32)
+        i = np.abs(g).argmax(axis=2)
+        ext = np.take_along_axis(_i8(codes).reshape(64, 4, 32), i[..., None], 2)[..., 0]
+        sgn = np.sign(np.take_along_axis(g, i[..., None], 2)[..., 0])
+        nz = scales > 0
+        assert np.array_equal(ext[nz], 127 * sgn[nz]), "a group's extreme is not +-127"
+        assert scales[5, 2] == 0 and np.all(codes[5, 64:96] == 0)
+        assert codes[9, 40] == 0 and np.isfinite(scales[9, 1]) and scales[9, 1] > 0
+        # the outlier only coarsens its own group
+        assert scales[3, 0] > 10 * np.median(scales[:, 0]) and scales[3, 1] < 3 * np.median(scales[:, 1])
+
+
+def check_attend_int8_against_sdpa():
+    for (B, H_q, H_kv, d, dt, lens, seed) in [(2, 8, 2, 128, "bf16", [40, 77], 41),
+                                              (1, 4, 4, 64, "f16", [33], 42)]:
+        c = case(B, H_q, H_kv, d, dt, lens, seed)
+        k8, ks = oracle.quantize_int8(c["kc"], c["dt"])
+        v8, vs = oracle.quantize_int8(c["vc"], c["dt"])
+        out, lse = oracle.attend_int8(c["q"], k8, v8, ks, vs, c["bt"], c["sl"], c["scale"], c["dt"])
+        G = H_q // H_kv
+        for b in range(B):
+            n = int(c["sl"][b])
+            j = np.arange(n)
+            pages, rows = c["bt"][b, j // 16], j % 16
+            Kd = _i8(k8[pages, :, rows, :]) * np.repeat(ks[pages, :, rows, :], 32, axis=-1)
+            Vd = _i8(v8[pages, :, rows, :]) * np.repeat(vs[pages, :, rows, :], 32, axis=-1)
+            K = torch.from_numpy(Kd.transpose(1, 0, 2)).repeat_interleave(G, dim=0)[None]
+            V = torch.from_numpy(Vd.transpose(1, 0, 2)).repeat_interleave(G, dim=0)[None]
+            q = torch.from_numpy(f64(c["q"][b], c["dt"]))[None, :, None, :]
+            ref = F.scaled_dot_product_attention(q, K, V, scale=c["scale"])[0, :, 0, :].numpy()
+            close(out[b], ref, 1e-12, 1e-12, "int8 attention vs SDPA on dequantised K/V")
+        full, _ = run(c)
+        assert np.max(np.abs(out - full)) < 0.05, "int8 attention far from fp16/bf16 attention"
+
+
+def check_append_int8():
+    w = build_workload("pin8i", 4, 4, 2, 128, "bf16", [1, 16, 17, 40], seed=84)
+    si = step_inputs(w, 0)
+    kc, vc = to_words(w.k_cache), to_words(w.v_cache)
+    k8, ks = oracle.quantize_int8(kc, oracle.BF16)
+    v8, vs = oracle.quantize_int8(vc, oracle.BF16)
+    k8_0, v8_0 = k8.copy(), v8.copy()
+    oracle.append_int8(k8, v8, ks, vs, w.block_table.numpy(), si["slot"].numpy(),
+                       to_words(si["k_new"]), to_words(si["v_new"]), oracle.BF16)
+    kn8, kns = oracle.quantize_int8(to_words(si["k_new"]), oracle.BF16)
+    vn8, vns = oracle.quantize_int8(to_words(si["v_new"]), oracle.BF16)
+    bt = w.block_table.numpy()
+    changed = np.any(k8 != k8_0, axis=(1, 3)) | np.any(v8 != v8_0, axis=(1, 3))
+    for b, pos in enumerate(si["slot"].numpy()):
+        p, r = bt[b, pos // 16], pos % 16
+        assert np.array_equal(k8[p, :, r, :], kn8[b]) and np.array_equal(ks[p, :, r, :], kns[b])
+        assert np.array_equal(v8[p, :, r, :], vn8[b]) and np.array_equal(vs[p, :, r, :], vns[b])
+        changed[p, r] = False
+    assert not changed.any(), "int8 append touched other rows"
+
+
 ALL_CHECKS = [
     check_f16_decoder,
     check_bf16_decoder,
@@ -495,4 +596,9 @@ ALL_CHECKS = [
     check_quantize_fp8,
     check_attend_fp8_against_sdpa,
     check_append_fp8,
+    check_int8_decoder,
+    check_int8_encoder,
+    check_quantize_int8,
+    check_attend_int8_against_sdpa,
+    check_append_int8,
 ]

@@ -39,6 +39,11 @@ MUTANTS = {
     "fp8_group_index": ("const float *sk = ks + off / d * ng;", "const float *sk = ks + off / d;"),
     "fp8_round_down": ("double r = rint(a / ldexp(1.0, E - 3));", "double r = floor(a / ldexp(1.0, E - 3));"),
     "fp8_decode_bias": ("else v = ldexp((double)(8 + m), e - 10);", "else v = ldexp((double)(8 + m), e - 9);"),
+    "int8_scale_max": ("volatile float s = mx / 127.0f;", "volatile float s = mx / 128.0f;"),
+    "int8_round_floor": ("double r = rint((double)x);", "double r = floor((double)x);"),
+    "int8_decode_unsigned": ("return (double)(int8_t)c;", "return (double)c;"),
+    "int8_clamp": ("if (r > 127.0) r = 127.0;", "if (r > 128.0) r = 128.0;"),
+    "int8_nan_code": ("if (isnan(x)) return 0;", "if (isnan(x)) return 0x7F;"),
     "max_skips_first": ("for (int t = 0; t < n; ++t) if (s[t] > m) m = s[t];",
                         "for (int t = 1; t < n; ++t) if (s[t] > m) m = s[t];"),
 }
