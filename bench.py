@@ -49,16 +49,6 @@ def attention_bytes(w, seq_lens) -> int:
     return kv + 2 * w.B * w.H_q * w.d * s
 
 
-def unique_attention_bytes(w, seq_lens) -> int:
-    """Like attention_bytes, but counting each shared prefix page once per group."""
-    s = 2
-    toks = int(seq_lens.to(torch.int64).sum().item())
-    if w.groups:
-        per = w.B // w.groups
-        toks -= w.groups * (per - 1) * w.prefix_tokens
-    return toks * w.H_kv * 2 * w.d * s + 2 * w.B * w.H_q * w.d * s
-
-
 def fp8_attention_bytes(w, seq_lens) -> int:
     """Attention bytes over the 8-bit cache: codes + fp32 group scales + q + out."""
     per_tok = w.H_kv * 2 * (w.d + (w.d // 32) * 4)
@@ -111,8 +101,8 @@ def source_hash() -> str:
 def profile_traffic(workload: str, mode: str):
     """DRAM bytes per decode launch from a committed ncu summary under
     profiles/, if one was taken on the current decode kernel sources for this
-    workload and step mode ("fused", "separate_append", "shared_prefix" or
-    "fp8")."""
+    workload and step mode ("fused", "separate_append", "shared_prefix", "fp8"
+    or "int8")."""
     try:
         names = sorted(os.listdir(PROFILE_DIR))
     except OSError:
@@ -320,11 +310,15 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     f8 = None
-    if args.kv_fp8:
-        # the pool stored as E4M3 codes + per-32-channel fp32 scales
-        k8, ks = kvd.kvd_quantize_fp8(kc)
-        v8, vs = kvd.kvd_quantize_fp8(vc)
-        f8 = {"k8": k8, "v8": v8, "ks": ks, "vs": vs}
+    if args.kv_fp8 or args.kv_int8:
+        # the pool stored as 8-bit codes (E4M3 or INT8) + per-32-channel fp32 scales
+        fmt = "fp8" if args.kv_fp8 else "int8"
+        k8, ks = getattr(kvd, "kvd_quantize_" + fmt)(kc)
+        v8, vs = getattr(kvd, "kvd_quantize_" + fmt)(vc)
+        f8 = {"fmt": fmt, "k8": k8, "v8": v8, "ks": ks, "vs": vs,
+              "append": getattr(kvd, "kvd_append_" + fmt),
+              "decode": getattr(kvd, "kvd_decode_attention_" + fmt),
+              "name": "E4M3" if fmt == "fp8" else "INT8"}
 
     sp = None
     if args.shared_prefix:
@@ -339,13 +333,11 @@ def run_ours(args):
 
     def step(ev_a=None, ev_b=None):
         if f8 is not None:
-            kvd.kvd_append_fp8(f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, slot, k_new, v_new,
-                               stream=stream)
+            f8["append"](f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, slot, k_new, v_new, stream=stream)
             if ev_a is not None:
                 ev_a.record(stream)
-            kvd.kvd_decode_attention_fp8(q, f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, seq_lens,
-                                         w.scale, out=out, num_partitions=args.partitions,
-                                         workspace=ws, stream=stream)
+            f8["decode"](q, f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, seq_lens, w.scale, out=out,
+                         num_partitions=args.partitions, workspace=ws, stream=stream)
             if ev_b is not None:
                 ev_b.record(stream)
             return
@@ -374,9 +366,17 @@ def run_ours(args):
 
     a_bytes = attention_bytes(w, si["seq_lens"])
     p_bytes = append_bytes(w, si["slot"])
+    kv_tok = w.H_kv * 2 * w.d * 2  # K and V bytes per token of one sequence
     if f8 is not None:
         a_bytes = fp8_attention_bytes(w, si["seq_lens"])
         p_bytes = int((si["slot"] >= 0).sum().item()) * w.H_kv * 2 * (w.d * 2 + w.d + (w.d // 32) * 4)
+        kv_tok = w.H_kv * 2 * (w.d + (w.d // 32) * 4)
+    # with shared prefixes the HBM bytes count each shared page once per group
+    # (the metric's bytes); the logical bytes (every member's own view) are
+    # reported beside them
+    a_bytes_logical = a_bytes
+    if w.groups:
+        a_bytes -= w.groups * (w.B // w.groups - 1) * w.prefix_tokens * kv_tok
     step_bytes = a_bytes + p_bytes
     # bytes of the call the roofline times (events bracket it)
     timed_bytes = a_bytes if (args.separate_append or f8 is not None) else step_bytes
@@ -455,9 +455,9 @@ def run_ours(args):
         for n in h_in:
             d_in[n].copy_(h_in[n], non_blocking=True)
         if f8 is not None:
-            kvd.kvd_append_fp8(f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, d_in["slot"],
+            f8["append"](f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, d_in["slot"],
                                d_in["k_new"], d_in["v_new"], stream=stream)
-            kvd.kvd_decode_attention_fp8(d_in["q"], f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt,
+            f8["decode"](d_in["q"], f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt,
                                          d_in["seq_lens"], w.scale, out=out,
                                          num_partitions=args.partitions, workspace=ws,
                                          stream=stream)
@@ -513,7 +513,7 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": ("e4m3 cache, " + w.dtype_name + " q/out") if f8 is not None else w.dtype_name,
+        "dtype": (f8["fmt"] + " cache, " + w.dtype_name + " q/out") if f8 is not None else w.dtype_name,
         "data": "synthetic",
         "config": {
             "workload": w.name if args.scale_down == 1 else f"{w.name}/scale_down={args.scale_down}",
@@ -523,8 +523,9 @@ def run_ours(args):
             "bytes_per_step": step_bytes, "attention_bytes": a_bytes, "append_bytes": p_bytes,
             "l2": "inputs larger than L2 (KV pool %.2f GB >> 126 MB); no flush" % (
                 2 * w.k_cache.numel() * 2 / 1e9),
-            "step": ("kvd_append_fp8 + kvd_decode_attention_fp8 over an E4M3 cache "
-                     "(quantising append, decode, merge kernels)" if f8 is not None else
+            "step": ("kvd_append_%s + kvd_decode_attention_%s over an %s cache "
+                     "(quantising append, decode, merge kernels)" % (f8["fmt"], f8["fmt"], f8["name"])
+                     if f8 is not None else
                      "kvd_decode_attention_shared_prefix with fused append (prefix, decode, merge kernels)"
                      if sp is not None else
                      "kvd_append + kvd_decode_attention (append, decode, merge kernels)"
@@ -540,8 +541,8 @@ def run_ours(args):
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "peak_kind": peak_kind,
-            "kernel": ("kvd_decode_attention_fp8 call (decode_kernel over E4M3 pages + merge)"
-                       if f8 is not None else
+            "kernel": ("kvd_decode_attention_%s call (decode_kernel over %s pages + merge)"
+                       % (f8["fmt"], f8["name"]) if f8 is not None else
                        "kvd_decode_attention_shared_prefix call (prefix_kernel + decode_kernel with fused "
                        "append + merge)" if sp is not None else
                        "kvd_decode_attention call (decode_kernel + decode_merge_kernel)"
@@ -549,15 +550,17 @@ def run_ours(args):
                        "kvd_decode_step call (decode_kernel with fused append + decode_merge_kernel)")
                       + ", CUDA events on the launching stream; achieved = its algorithmic bytes / mean duration",
             "bytes_per_launch": timed_bytes,
-            "traffic": profile_traffic(w.name, "fp8" if f8 is not None else "shared_prefix" if sp is not None
+            "traffic": profile_traffic(w.name, f8["fmt"] if f8 is not None else "shared_prefix" if sp is not None
                                       else "separate_append" if args.separate_append else "fused"),
         },
         "frac_of_8000_spec": round(achieved / 8000.0, 4),
-        "shared_prefix": ({"unique_attention_bytes": unique_attention_bytes(w, si["seq_lens"]),
-                           "achieved_unique_gbs": round(
-                               (unique_attention_bytes(w, si["seq_lens"]) + (timed_bytes - a_bytes))
-                               / (attn_ms * 1e-3) / 1e9, 2),
-                           "note": "shared prefix pages counted once per group"}
+        "shared_prefix": ({"logical_attention_bytes": a_bytes_logical,
+                           "value_logical_gbs": round(
+                               world * (step_bytes + a_bytes_logical - a_bytes) / (ms_step * 1e-3) / 1e9, 2),
+                           "achieved_logical_gbs": round(
+                               (timed_bytes + a_bytes_logical - a_bytes) / (attn_ms * 1e-3) / 1e9, 2),
+                           "note": ("value, roofline and e2e count each shared prefix page once per "
+                                    "group; the logical figures count it once per member")}
                           if w.groups else None),
         "read_only_peak": {"value": round(read_peak, 1), "unit": "GB/s",
                            "frac": round(achieved / read_peak, 4),
@@ -567,7 +570,7 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "us_per_step": round(e2e_s / e2e_steps * 1e6, 2),
                 "how": "pinned host inputs -> H2D, append, decode, D2H of out, stream sync; wall clock"},
-        "gpu_launches": (4 if f8 is not None else 3 if (args.separate_append or sp is not None)
+        "gpu_launches": (3 if (f8 is not None or args.separate_append or sp is not None)
                          else 2) * args.steps * per,
         "graph": ({"steps_per_graph": args.graph_steps, "replays": args.steps} if graph is not None
                   else None),
@@ -600,6 +603,8 @@ def main(argv=None):
     p.add_argument("--e2e-steps", type=int, default=300)
     p.add_argument("--kv-fp8", action="store_true",
                    help="store the cache as FP8 E4M3 codes with per-32-channel scales (d=128)")
+    p.add_argument("--kv-int8", action="store_true",
+                   help="store the cache as INT8 codes with per-32-channel scales (d=128)")
     p.add_argument("--shared-prefix", action="store_true",
                    help="read each group's shared prefix pages once (kvd_decode_attention_shared_prefix)")
     p.add_argument("--graph", action="store_true",
@@ -615,8 +620,10 @@ def main(argv=None):
     args = p.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.graph and (args.separate_append or args.shared_prefix or args.kv_fp8):
+    if args.graph and (args.separate_append or args.shared_prefix or args.kv_fp8 or args.kv_int8):
         raise SystemExit("--graph times the fused step only")
+    if args.kv_fp8 and args.kv_int8:
+        raise SystemExit("--kv-fp8 and --kv-int8 are exclusive")
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

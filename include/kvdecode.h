@@ -215,6 +215,32 @@ kvd_status kvd_decode_attention_fp8(const void *q, const uint8_t *k_codes, const
                                     void *workspace, size_t workspace_bytes, float *lse_out,
                                     kvd_dtype dtype, void *stream);
 
+/*
+ * 8-bit (INT8) KV cache: the same layout, scales and calls as the E4M3 cache
+ * above, with symmetric integer codes.
+ * [BLOG] section "工程优化手段 / 量化" (quantise the cache from fp16 to int8 or
+ * int4, with scales per channel group because of outlier keys); [KVF] section
+ * "三、实际落地" (keys and values kept in INT8 or even INT4).
+ * Format: codes int8 [num_blocks][H_kv][16][d]; scales float [num_blocks]
+ * [H_kv][16][d/32] with s = max|x| / 127 over the group and code = x / s
+ * rounded to the nearest integer (ties to even) and clamped to [-127, 127]
+ * (a NaN quotient gives 0; both divisions IEEE fp32); value = s * code.
+ * Arguments, ownership, validation and errors are those of the _fp8 calls.
+ */
+kvd_status kvd_quantize_int8(const void *src, int8_t *codes, float *scales, long long n_rows,
+                             int d, kvd_dtype dtype, void *stream);
+kvd_status kvd_append_int8(int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale,
+                           const int32_t *block_table, const int32_t *slot, const void *k_new,
+                           const void *v_new, int B, int H_kv, int d, int num_blocks,
+                           int max_blocks_per_seq, kvd_dtype dtype, void *stream);
+kvd_status kvd_decode_attention_int8(const void *q, const int8_t *k_codes, const int8_t *v_codes,
+                                     const float *k_scale, const float *v_scale,
+                                     const int32_t *block_table, const int32_t *seq_lens,
+                                     float scale, void *out, int B, int H_q, int H_kv, int d,
+                                     int num_blocks, int max_blocks_per_seq, int num_partitions,
+                                     void *workspace, size_t workspace_bytes, float *lse_out,
+                                     kvd_dtype dtype, void *stream);
+
 /* Bytes of the library's fixed scratch array used by kvd_decode_attention_static. */
 #define KVD_STATIC_WORKSPACE_BYTES (8u << 20)
 

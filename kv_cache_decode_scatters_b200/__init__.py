@@ -23,6 +23,7 @@ __all__ = [
     "kvd_append", "kvd_decode_attention", "kvd_decode_step", "kvd_decode_attention_static",
     "kvd_decode_attention_shared_prefix", "kvd_shared_prefix_workspace_size",
     "kvd_quantize_fp8", "kvd_append_fp8", "kvd_decode_attention_fp8",
+    "kvd_quantize_int8", "kvd_append_int8", "kvd_decode_attention_int8",
     "kvd_merge_lse",
     "kvd_workspace_size", "KVD_STATIC_WORKSPACE_BYTES",
     "kvd_auto_partitions", "kvd_kv_bytes_per_token", "kvd_read_device_error",
@@ -61,13 +62,14 @@ def _load():
     L.kvd_shared_prefix_workspace_size.restype = S
     L.kvd_shared_prefix_workspace_size.argtypes = [I, I, I, I, I, I, I]
     LL = ctypes.c_longlong
-    L.kvd_quantize_fp8.restype = I
-    L.kvd_quantize_fp8.argtypes = [P, P, P, LL, I, I, P]
-    L.kvd_append_fp8.restype = I
-    L.kvd_append_fp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
-    L.kvd_decode_attention_fp8.restype = I
-    L.kvd_decode_attention_fp8.argtypes = [P, P, P, P, P, P, P, F, P, I, I, I, I, I, I, I, P, S, P,
-                                           I, P]
+    for fmt in ("fp8", "int8"):
+        getattr(L, "kvd_quantize_" + fmt).restype = I
+        getattr(L, "kvd_quantize_" + fmt).argtypes = [P, P, P, LL, I, I, P]
+        getattr(L, "kvd_append_" + fmt).restype = I
+        getattr(L, "kvd_append_" + fmt).argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+        getattr(L, "kvd_decode_attention_" + fmt).restype = I
+        getattr(L, "kvd_decode_attention_" + fmt).argtypes = [P, P, P, P, P, P, P, F, P, I, I, I, I,
+                                                              I, I, I, P, S, P, I, P]
     L.kvd_decode_attention_static.restype = I
     L.kvd_decode_attention_static.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, P, I, P]
     L.kvd_merge_lse.restype = I
@@ -278,37 +280,38 @@ def kvd_decode_attention_shared_prefix(q, k_cache, v_cache, block_table, seq_len
     return out
 
 
-def kvd_quantize_fp8(src, codes=None, scales=None, stream=None):
-    """Quantise rows src [..., d] (fp16/bf16) into E4M3 codes (uint8 [..., d])
-    and fp32 scales [..., d/32], one per 32 channels.  Returns (codes, scales)."""
+# 8-bit KV caches: E4M3 codes (torch.uint8 storage) or INT8 codes (torch.int8),
+# one fp32 scale per (token, KV head, 32 channels).
+_CODE8 = {"fp8": torch.uint8, "int8": torch.int8}
+
+
+def _quantize8(fmt, src, codes, scales, stream):
     d = src.shape[-1]
     n = src.numel() // d
     if codes is None:
-        codes = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+        codes = torch.empty(src.shape, dtype=_CODE8[fmt], device=src.device)
     if scales is None:
         scales = torch.empty(src.shape[:-1] + (d // 32,), dtype=torch.float32, device=src.device)
-    _check(_lib.kvd_quantize_fp8(_dev(src, "src"), _dev(codes, "codes", torch.uint8),
-                                 _dev(scales, "scales", torch.float32), n, d, _dtype_code(src),
-                                 _stream(stream)),
-           "kvd_quantize_fp8")
+    _check(getattr(_lib, "kvd_quantize_" + fmt)(
+        _dev(src, "src"), _dev(codes, "codes", _CODE8[fmt]), _dev(scales, "scales", torch.float32), n, d,
+        _dtype_code(src), _stream(stream)), "kvd_quantize_" + fmt)
     return codes, scales
 
 
-def kvd_append_fp8(k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, stream=None):
-    """kvd_append for the 8-bit cache (codes [NB,H_kv,16,d], scales [NB,H_kv,16,d/32])."""
+def _append8(fmt, k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, stream):
     NB, H_kv, P, d = k_codes.shape
     B = k_new.shape[0]
-    _check(_lib.kvd_append_fp8(_dev(k_codes, "k_codes", torch.uint8), _dev(v_codes, "v_codes", torch.uint8),
-                               _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
-                               _dev(block_table, "block_table", torch.int32), _dev(slot, "slot", torch.int32),
-                               _dev(k_new, "k_new", k_new.dtype), _dev(v_new, "v_new", k_new.dtype),
-                               B, H_kv, d, NB, block_table.shape[1], _dtype_code(k_new), _stream(stream)),
-           "kvd_append_fp8")
+    c = _CODE8[fmt]
+    _check(getattr(_lib, "kvd_append_" + fmt)(
+        _dev(k_codes, "k_codes", c), _dev(v_codes, "v_codes", c),
+        _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+        _dev(block_table, "block_table", torch.int32), _dev(slot, "slot", torch.int32),
+        _dev(k_new, "k_new", k_new.dtype), _dev(v_new, "v_new", k_new.dtype),
+        B, H_kv, d, NB, block_table.shape[1], _dtype_code(k_new), _stream(stream)), "kvd_append_" + fmt)
 
 
-def kvd_decode_attention_fp8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale=None,
-                             out=None, num_partitions=0, workspace=None, lse_out=None, stream=None):
-    """kvd_decode_attention over the 8-bit cache (d = 128).  Returns out (q's dtype)."""
+def _decode8(fmt, q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
+             num_partitions, workspace, lse_out, stream):
     B, H_q, d = q.shape
     NB, H_kv, P, d2 = k_codes.shape
     if P != KVD_PAGE_TOKENS or d2 != d:
@@ -320,15 +323,51 @@ def kvd_decode_attention_fp8(q, k_codes, v_codes, k_scale, v_scale, block_table,
     if workspace is None:
         workspace = alloc_workspace(B, H_q, H_kv, d, num_partitions, q.device)
     lse_ptr = None if lse_out is None else _dev(lse_out, "lse_out", torch.float32)
-    _check(_lib.kvd_decode_attention_fp8(
-        _dev(q, "q", q.dtype), _dev(k_codes, "k_codes", torch.uint8), _dev(v_codes, "v_codes", torch.uint8),
+    c = _CODE8[fmt]
+    _check(getattr(_lib, "kvd_decode_attention_" + fmt)(
+        _dev(q, "q", q.dtype), _dev(k_codes, "k_codes", c), _dev(v_codes, "v_codes", c),
         _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
         _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
         float(scale), _dev(out, "out", q.dtype), B, H_q, H_kv, d, NB, block_table.shape[1],
         int(num_partitions), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-        lse_ptr, _dtype_code(q), _stream(stream)),
-        "kvd_decode_attention_fp8")
+        lse_ptr, _dtype_code(q), _stream(stream)), "kvd_decode_attention_" + fmt)
     return out
+
+
+def kvd_quantize_fp8(src, codes=None, scales=None, stream=None):
+    """Quantise rows src [..., d] (fp16/bf16) into E4M3 codes (uint8 [..., d])
+    and fp32 scales [..., d/32], one per 32 channels.  Returns (codes, scales)."""
+    return _quantize8("fp8", src, codes, scales, stream)
+
+
+def kvd_append_fp8(k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, stream=None):
+    """kvd_append for the 8-bit cache (codes [NB,H_kv,16,d], scales [NB,H_kv,16,d/32])."""
+    _append8("fp8", k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, stream)
+
+
+def kvd_decode_attention_fp8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale=None,
+                             out=None, num_partitions=0, workspace=None, lse_out=None, stream=None):
+    """kvd_decode_attention over the 8-bit cache (d = 128).  Returns out (q's dtype)."""
+    return _decode8("fp8", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
+                    num_partitions, workspace, lse_out, stream)
+
+
+def kvd_quantize_int8(src, codes=None, scales=None, stream=None):
+    """Quantise rows src [..., d] (fp16/bf16) into INT8 codes (int8 [..., d])
+    and fp32 scales [..., d/32], one per 32 channels.  Returns (codes, scales)."""
+    return _quantize8("int8", src, codes, scales, stream)
+
+
+def kvd_append_int8(k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, stream=None):
+    """kvd_append for the INT8 cache (codes [NB,H_kv,16,d], scales [NB,H_kv,16,d/32])."""
+    _append8("int8", k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, stream)
+
+
+def kvd_decode_attention_int8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale=None,
+                              out=None, num_partitions=0, workspace=None, lse_out=None, stream=None):
+    """kvd_decode_attention over the INT8 cache (d = 128).  Returns out (q's dtype)."""
+    return _decode8("int8", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
+                    num_partitions, workspace, lse_out, stream)
 
 
 def kvd_decode_attention_static(q, k_cache, v_cache, block_table, seq_lens, scale=None, out=None,

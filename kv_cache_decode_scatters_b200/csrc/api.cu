@@ -264,8 +264,8 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
                               const int32_t *group_start = nullptr,
                               const int32_t *group_pages = nullptr, int n_groups = 0,
                               int max_group_size = 0, const float *k_scale = nullptr,
-                              const float *v_scale = nullptr) {
-  const bool fp8 = k_scale != nullptr;
+                              const float *v_scale = nullptr, kvd::Code8 fmt = kvd::Code8::E4M3) {
+  const bool q8 = k_scale != nullptr;  // 8-bit cache (codes + scales)
   kvd_status st = check_heads(B, H_q, H_kv, d);
   if (st) return st;
   if (num_blocks <= 0 || max_blocks_per_seq <= 0)
@@ -277,7 +277,7 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
     return fail(KVD_ERR_UNSUPPORTED, "max_blocks_per_seq too large");
   if (!(scale == scale)) return fail(KVD_ERR_INVALID, "scale is NaN");
   if (num_partitions < 0) return fail(KVD_ERR_INVALID, "num_partitions < 0");
-  if (fp8) {
+  if (q8) {
     if (d != 128) return fail(KVD_ERR_UNSUPPORTED, "the 8-bit cache supports d = 128 only");
     if (!v_scale) return fail(KVD_ERR_INVALID, "v_scale is NULL");
     if (k_new || n_groups > 0)
@@ -326,7 +326,7 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   const void *pools[2] = {k_cache, v_cache};
   for (int i = 0; i < 2; ++i) {
     CUresult r;
-    if (fp8) {
+    if (q8) {
       // E4M3 code pools as 2-D byte tensors {128, num_blocks*H_kv*16 rows};
       // one box = the 16 rows of one page of one head, 128-byte swizzled.
       cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(num_blocks) * H_kv * KVD_PAGE_TOKENS};
@@ -417,7 +417,7 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
     a.pre_lse = pa.pre_lse;
     a.pre_chunks = PL.chunks;
   }
-  e = fp8 ? kvd::launch_decode_fp8(a, dt, tm[0], tm[1], s, N)
+  e = q8 ? kvd::launch_decode_q8(a, dt, fmt, tm[0], tm[1], s, N)
           : kvd::launch_decode(a, d, dt, tm[0], tm[1], s, N);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   e = kvd::launch_decode_merge(a, d, dt, s);
@@ -438,8 +438,8 @@ kvd_status kvd_decode_attention(const void *q, const void *k_cache, const void *
                      lse_out, dtype, stream, nullptr, nullptr);
 }
 
-kvd_status kvd_quantize_fp8(const void *src, uint8_t *codes, float *scales, long long n_rows,
-                            int d, kvd_dtype dtype, void *stream) {
+static kvd_status quantize_q8(const void *src, uint8_t *codes, float *scales, long long n_rows,
+                              int d, kvd_dtype dtype, void *stream, kvd::Code8 fmt) {
   if (n_rows < 0) return fail(KVD_ERR_INVALID, "n_rows < 0");
   if (d <= 0 || d % 32 || d > 128) return fail(KVD_ERR_UNSUPPORTED, "d must be 32, 64, 96 or 128");
   if (dtype != KVD_F16 && dtype != KVD_BF16) return fail(KVD_ERR_INVALID, "unknown dtype %d", (int)dtype);
@@ -448,16 +448,16 @@ kvd_status kvd_quantize_fp8(const void *src, uint8_t *codes, float *scales, long
   if (!aligned(src, 8) || !aligned(codes, 4) || !aligned(scales, 4))
     return fail(KVD_ERR_INVALID, "misaligned buffer");
   kvd::QuantArgs q{src, codes, scales, nullptr, nullptr, nullptr, n_rows, d, 1, 1, 1, 0};
-  cudaError_t e = kvd::launch_quantize_fp8(q, dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16,
-                                           static_cast<cudaStream_t>(stream));
+  cudaError_t e = kvd::launch_quantize_q8(q, dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16,
+                                          fmt, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return KVD_OK;
 }
 
-kvd_status kvd_append_fp8(uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
-                          const int32_t *block_table, const int32_t *slot, const void *k_new,
-                          const void *v_new, int B, int H_kv, int d, int num_blocks,
-                          int max_blocks_per_seq, kvd_dtype dtype, void *stream) {
+static kvd_status append_q8(uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
+                            const int32_t *block_table, const int32_t *slot, const void *k_new,
+                            const void *v_new, int B, int H_kv, int d, int num_blocks,
+                            int max_blocks_per_seq, kvd_dtype dtype, void *stream, kvd::Code8 fmt) {
   if (B < 0) return fail(KVD_ERR_INVALID, "B = %d < 0", B);
   if (H_kv <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
     return fail(KVD_ERR_INVALID, "H_kv, num_blocks and max_blocks_per_seq must be positive");
@@ -480,9 +480,35 @@ kvd_status kvd_append_fp8(uint8_t *k_codes, uint8_t *v_codes, float *k_scale, fl
   const long long n = static_cast<long long>(B) * H_kv;
   kvd::QuantArgs qa{k_new, k_codes, k_scale, block_table, slot, err, n, d, H_kv, num_blocks,
                     max_blocks_per_seq, 1, v_new, v_codes, v_scale};
-  cudaError_t e = kvd::launch_quantize_fp8(qa, dt, s);
+  cudaError_t e = kvd::launch_quantize_q8(qa, dt, fmt, s);
   if (e != cudaSuccess) return cuda_fail(e, "append launch");
   return KVD_OK;
+}
+
+static kvd_status decode_q8(const void *q, const uint8_t *k_codes, const uint8_t *v_codes,
+                            const float *k_scale, const float *v_scale, const int32_t *block_table,
+                            const int32_t *seq_lens, float scale, void *out, int B, int H_q, int H_kv,
+                            int d, int num_blocks, int max_blocks_per_seq, int num_partitions,
+                            void *workspace, size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+                            void *stream, kvd::Code8 fmt) {
+  if (!k_scale) return fail(KVD_ERR_INVALID, "k_scale is NULL");
+  return decode_impl(q, k_codes, v_codes, block_table, seq_lens, scale, out, B, H_q, H_kv, d,
+                     num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
+                     lse_out, dtype, stream, nullptr, nullptr, nullptr, nullptr, 0, 0, k_scale,
+                     v_scale, fmt);
+}
+
+kvd_status kvd_quantize_fp8(const void *src, uint8_t *codes, float *scales, long long n_rows,
+                            int d, kvd_dtype dtype, void *stream) {
+  return quantize_q8(src, codes, scales, n_rows, d, dtype, stream, kvd::Code8::E4M3);
+}
+
+kvd_status kvd_append_fp8(uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
+                          const int32_t *block_table, const int32_t *slot, const void *k_new,
+                          const void *v_new, int B, int H_kv, int d, int num_blocks,
+                          int max_blocks_per_seq, kvd_dtype dtype, void *stream) {
+  return append_q8(k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, B, H_kv, d,
+                   num_blocks, max_blocks_per_seq, dtype, stream, kvd::Code8::E4M3);
 }
 
 kvd_status kvd_decode_attention_fp8(const void *q, const uint8_t *k_codes, const uint8_t *v_codes,
@@ -492,11 +518,38 @@ kvd_status kvd_decode_attention_fp8(const void *q, const uint8_t *k_codes, const
                                     int num_blocks, int max_blocks_per_seq, int num_partitions,
                                     void *workspace, size_t workspace_bytes, float *lse_out,
                                     kvd_dtype dtype, void *stream) {
-  if (!k_scale) return fail(KVD_ERR_INVALID, "k_scale is NULL");
-  return decode_impl(q, k_codes, v_codes, block_table, seq_lens, scale, out, B, H_q, H_kv, d,
-                     num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
-                     lse_out, dtype, stream, nullptr, nullptr, nullptr, nullptr, 0, 0, k_scale,
-                     v_scale);
+  return decode_q8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out, B, H_q,
+                   H_kv, d, num_blocks, max_blocks_per_seq, num_partitions, workspace,
+                   workspace_bytes, lse_out, dtype, stream, kvd::Code8::E4M3);
+}
+
+kvd_status kvd_quantize_int8(const void *src, int8_t *codes, float *scales, long long n_rows,
+                             int d, kvd_dtype dtype, void *stream) {
+  return quantize_q8(src, reinterpret_cast<uint8_t *>(codes), scales, n_rows, d, dtype, stream,
+                     kvd::Code8::INT8);
+}
+
+kvd_status kvd_append_int8(int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale,
+                           const int32_t *block_table, const int32_t *slot, const void *k_new,
+                           const void *v_new, int B, int H_kv, int d, int num_blocks,
+                           int max_blocks_per_seq, kvd_dtype dtype, void *stream) {
+  return append_q8(reinterpret_cast<uint8_t *>(k_codes), reinterpret_cast<uint8_t *>(v_codes),
+                   k_scale, v_scale, block_table, slot, k_new, v_new, B, H_kv, d, num_blocks,
+                   max_blocks_per_seq, dtype, stream, kvd::Code8::INT8);
+}
+
+kvd_status kvd_decode_attention_int8(const void *q, const int8_t *k_codes, const int8_t *v_codes,
+                                     const float *k_scale, const float *v_scale,
+                                     const int32_t *block_table, const int32_t *seq_lens,
+                                     float scale, void *out, int B, int H_q, int H_kv, int d,
+                                     int num_blocks, int max_blocks_per_seq, int num_partitions,
+                                     void *workspace, size_t workspace_bytes, float *lse_out,
+                                     kvd_dtype dtype, void *stream) {
+  return decode_q8(q, reinterpret_cast<const uint8_t *>(k_codes),
+                   reinterpret_cast<const uint8_t *>(v_codes), k_scale, v_scale, block_table,
+                   seq_lens, scale, out, B, H_q, H_kv, d, num_blocks, max_blocks_per_seq,
+                   num_partitions, workspace, workspace_bytes, lse_out, dtype, stream,
+                   kvd::Code8::INT8);
 }
 
 size_t kvd_shared_prefix_workspace_size(int B, int H_q, int H_kv, int d, int n_groups,

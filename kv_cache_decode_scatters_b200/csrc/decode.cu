@@ -117,9 +117,10 @@ struct Page16 {
   }
 };
 
-// E4M3 pages (d = 128): codes [16][128] per (page, head) in one swizzled box,
-// fp32 scales [16][4] per (page, head) copied alongside; output dtype T.
-template <int NT, typename T>
+// 8-bit pages (d = 128; E4M3 or INT8 codes): codes [16][128] per (page, head)
+// in one swizzled box, fp32 scales [16][4] per (page, head) copied alongside;
+// output dtype T.
+template <int NT, typename T, Code8 kFmt>
 struct Page8 {
   using Out = T;
   static constexpr bool kPatchable = false;
@@ -151,8 +152,8 @@ struct Page8 {
                                               float (&acc)[NT][8][4], float (&m)[NT][2],
                                               float (&l)[NT][2]) {
     const float *ks = reinterpret_cast<const float *>(aux);
-    tile_page_fp8<NT>(smem_u32(st), smem_u32(st + kPageBytes), ks, ks + kPage * 4, ntok, sl2, lane,
-                      qf, acc, m, l);
+    tile_page_q8<NT, kFmt>(smem_u32(st), smem_u32(st + kPageBytes), ks, ks + kPage * 4, ntok, sl2,
+                           lane, qf, acc, m, l);
   }
   // q in f16, channel order of the E4M3 tile: k-slots 2t, 2t+1 <- channels
   // 4t, 4t+1 and k-slots 2t+8, 2t+9 <- channels 4t+2, 4t+3 of each 16
@@ -998,19 +999,19 @@ int decode_auto_parts(int sms) { return sms; }
 #define KVD_TUNE_S8_1 2
 #endif
 #ifndef KVD_TUNE_W8_2
-#define KVD_TUNE_W8_2 10
+#define KVD_TUNE_W8_2 8
 #endif
 #ifndef KVD_TUNE_S8_2
 #define KVD_TUNE_S8_2 2
 #endif
 
 namespace {
-template <int NT, typename T>
+template <int NT, typename T, Code8 kFmt>
 cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                              cudaStream_t st, int grid) {
   constexpr int W = NT == 1 ? KVD_TUNE_W8_1 : KVD_TUNE_W8_2;
   constexpr int S = NT == 1 ? KVD_TUNE_S8_1 : KVD_TUNE_S8_2;
-  using Pol = Page8<NT, T>;
+  using Pol = Page8<NT, T, kFmt>;
   auto kern = decode_kernel<128, NT, Pol, W, S>;
   const size_t smem = Geo<128, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1020,14 +1021,23 @@ cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const 
 }
 }  // namespace
 
-cudaError_t launch_decode_fp8(const DecodeArgs &a, DType dt, const CUtensorMap &tmK,
-                              const CUtensorMap &tmV, cudaStream_t s, int grid) {
+namespace {
+template <Code8 kFmt>
+cudaError_t launch_decode_q8_fmt(const DecodeArgs &a, DType dt, const CUtensorMap &tmK,
+                                 const CUtensorMap &tmV, cudaStream_t s, int grid) {
   const bool two = a.G > 8;
   if (dt == DType::BF16)
-    return two ? launch_decode8_t<2, __nv_bfloat16>(a, tmK, tmV, s, grid)
-               : launch_decode8_t<1, __nv_bfloat16>(a, tmK, tmV, s, grid);
-  return two ? launch_decode8_t<2, __half>(a, tmK, tmV, s, grid)
-             : launch_decode8_t<1, __half>(a, tmK, tmV, s, grid);
+    return two ? launch_decode8_t<2, __nv_bfloat16, kFmt>(a, tmK, tmV, s, grid)
+               : launch_decode8_t<1, __nv_bfloat16, kFmt>(a, tmK, tmV, s, grid);
+  return two ? launch_decode8_t<2, __half, kFmt>(a, tmK, tmV, s, grid)
+             : launch_decode8_t<1, __half, kFmt>(a, tmK, tmV, s, grid);
+}
+}  // namespace
+
+cudaError_t launch_decode_q8(const DecodeArgs &a, DType dt, Code8 fmt, const CUtensorMap &tmK,
+                             const CUtensorMap &tmV, cudaStream_t s, int grid) {
+  return fmt == Code8::INT8 ? launch_decode_q8_fmt<Code8::INT8>(a, dt, tmK, tmV, s, grid)
+                            : launch_decode_q8_fmt<Code8::E4M3>(a, dt, tmK, tmV, s, grid);
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, int d, DType dt, const CUtensorMap &tmK,

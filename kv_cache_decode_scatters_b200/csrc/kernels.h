@@ -10,6 +10,9 @@ namespace kvd {
 
 enum class DType { F16 = 0, BF16 = 1 };
 
+// formats of an 8-bit KV cache
+enum class Code8 { E4M3 = 0, INT8 = 1 };
+
 struct AppendArgs {
   void *k_cache;
   void *v_cache;
@@ -109,9 +112,9 @@ cudaError_t launch_decode(const DecodeArgs &a, int d, DType dt, const CUtensorMa
                           const CUtensorMap &tmV, cudaStream_t s, int grid);
 cudaError_t launch_decode_merge(const DecodeArgs &a, int d, DType dt, cudaStream_t s);
 cudaError_t launch_generic_merge(const GenericMergeArgs &a, DType dt, cudaStream_t s);
-cudaError_t launch_decode_fp8(const DecodeArgs &a, DType dt, const CUtensorMap &tmK,
+cudaError_t launch_decode_q8(const DecodeArgs &a, DType dt, Code8 fmt, const CUtensorMap &tmK,
                               const CUtensorMap &tmV, cudaStream_t s, int grid);
-cudaError_t launch_quantize_fp8(const QuantArgs &a, DType dt, cudaStream_t s);
+cudaError_t launch_quantize_q8(const QuantArgs &a, DType dt, Code8 fmt, cudaStream_t s);
 // Prefix pass of the shared-prefix decode: grid (n_groups * chunks, H_kv, row blocks).
 cudaError_t launch_prefix(const PrefixArgs &a, int d, DType dt, const CUtensorMap &tmK,
                           const CUtensorMap &tmV, int row_blocks, cudaStream_t s);

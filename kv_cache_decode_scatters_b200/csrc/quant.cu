@@ -1,12 +1,17 @@
-// quant.cu -- FP8 (E4M3) quantisation of K/V rows for the 8-bit cache.
+// quant.cu -- 8-bit quantisation of K/V rows (FP8 E4M3 or INT8 codes).
 //
 // "KV Cache:推理慢的真正原因", section 工程优化手段 / 量化: store the cache in 8 bits
 // with scales per channel group, so a few very large key channels do not
-// swamp the scale of the others.  Each row (one token of one KV head) is
-// split into groups of 32 channels; group scale s = max|x| / 448 (448 is the
-// largest E4M3 value) and code = E4M3(x / s), rounded to nearest even and
-// saturated; both divisions are IEEE fp32 (__fdiv_rn), so the codes are the
-// same on every run and every machine.  A group of zeros gets s = 0.
+// swamp the scale of the others ("推理速度慢怎么办？KV Cache与Flash Attention如何加速
+// 大模型推理", section 三、实际落地, names INT8; serving with an fp8 cache is the
+// other common form).  Each row (one token of one KV head) is split into
+// groups of 32 channels with one fp32 scale s each:
+//  * E4M3: s = max|x| / 448 (448 is the largest E4M3 value), code = E4M3(x / s)
+//    rounded to nearest even and saturated;
+//  * INT8: s = max|x| / 127, code = x / s rounded to the nearest integer (ties
+//    to even) and clamped to +-127; a NaN quotient gives 0.
+// Both divisions are IEEE fp32 (__fdiv_rn), so the codes are the same on
+// every run and every machine.  A group of zeros gets s = 0.
 //
 // One warp per row: lane l holds channels 4l..4l+3, a group is 8 lanes and
 // its maximum is three shuffles.  In append mode the source rows are the
@@ -20,8 +25,9 @@
 
 namespace kvd {
 
-template <typename T>
-__global__ void __launch_bounds__(256) quantize_fp8_kernel(const QuantArgs a) {
+template <typename T, Code8 kFmt>
+__global__ void __launch_bounds__(256) quantize_q8_kernel(const QuantArgs a) {
+  constexpr float kMax = kFmt == Code8::E4M3 ? 448.0f : 127.0f;
   // programmatic dependent launch: wait for the preceding grid's writes
   grid_dependency_wait();
   grid_launch_dependents();
@@ -61,23 +67,40 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(const QuantArgs a) {
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-  const float s = __fdiv_rn(mx, 448.0f);
+  const float s = __fdiv_rn(mx, kMax);
   float q[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) q[i] = s == 0.0f ? 0.0f : __fdiv_rn(x[i], s);
   if (!live) return;
-  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(q[0], q[1]), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(q[2], q[3]), __NV_SATFINITE, __NV_E4M3);
-  *reinterpret_cast<uint32_t *>(codes + dst * a.d + lane * 4) = (lo & 0xffffu) | (hi << 16);
+  uint32_t word;
+  if constexpr (kFmt == Code8::E4M3) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(q[0], q[1]), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(q[2], q[3]), __NV_SATFINITE, __NV_E4M3);
+    word = (lo & 0xffffu) | (hi << 16);
+  } else {
+    word = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float r = q[i] != q[i] ? 0.f : fminf(fmaxf(rintf(q[i]), -127.f), 127.f);
+      word |= (static_cast<uint32_t>(static_cast<int>(r)) & 0xffu) << (8 * i);
+    }
+  }
+  *reinterpret_cast<uint32_t *>(codes + dst * a.d + lane * 4) = word;
   if ((lane & 7) == 0) scales[dst * (a.d / 32) + (lane >> 3)] = s;
 }
 
-cudaError_t launch_quantize_fp8(const QuantArgs &a, DType dt, cudaStream_t s) {
+cudaError_t launch_quantize_q8(const QuantArgs &a, DType dt, Code8 fmt, cudaStream_t s) {
   if (a.n == 0) return cudaSuccess;
   const long long rows = a.src2 ? 2 * a.n : a.n;
   const dim3 grid(static_cast<unsigned>((rows + 7) / 8));
-  if (dt == DType::BF16) return launch_pdl(quantize_fp8_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, a);
-  return launch_pdl(quantize_fp8_kernel<__half>, grid, dim3(256), 0, s, a);
+  if (fmt == Code8::INT8) {
+    if (dt == DType::BF16)
+      return launch_pdl(quantize_q8_kernel<__nv_bfloat16, Code8::INT8>, grid, dim3(256), 0, s, a);
+    return launch_pdl(quantize_q8_kernel<__half, Code8::INT8>, grid, dim3(256), 0, s, a);
+  }
+  if (dt == DType::BF16)
+    return launch_pdl(quantize_q8_kernel<__nv_bfloat16, Code8::E4M3>, grid, dim3(256), 0, s, a);
+  return launch_pdl(quantize_q8_kernel<__half, Code8::E4M3>, grid, dim3(256), 0, s, a);
 }
 
 }  // namespace kvd

@@ -6,6 +6,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "kernels.h"
 
 #ifndef KVD_BF16_SPLIT_P
 #define KVD_BF16_SPLIT_P 1
@@ -268,15 +269,29 @@ __device__ __forceinline__ void tile_page2(uint32_t kbA, uint32_t vbA, uint32_t 
 
 namespace kvd {
 
-// Four E4M3 codes (bytes 0..3 of `four`) -> f16x2 of bytes (0, 1) and of
-// bytes (2, 3), exact (every E4M3 value is an f16 value).
-__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t four, uint32_t &lo, uint32_t &hi) {
-  asm("{\n\t.reg .b16 a, b;\n\t"
-      "mov.b32 {a, b}, %2;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
-      : "=r"(lo), "=r"(hi)
-      : "r"(four));
+// Four 8-bit codes (bytes 0..3 of `four`) -> f16x2 of bytes (0, 1) and of
+// bytes (2, 3), exact (every E4M3 value and every integer in [-128, 127] is an
+// f16 value).
+//  * E4M3: the hardware conversion, two codes per instruction.
+//  * INT8: each signed byte b becomes the f16 with bits 0x64 | (b + 128), that
+//    is 1024 + (b + 128), and 1152 is subtracted (exact: |result| <= 128).
+template <Code8 kFmt>
+__device__ __forceinline__ void code8x4_to_f16x2x2(uint32_t four, uint32_t &lo, uint32_t &hi) {
+  if constexpr (kFmt == Code8::E4M3) {
+    asm("{\n\t.reg .b16 a, b;\n\t"
+        "mov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(four));
+  } else {
+    const uint32_t u = four ^ 0x80808080u;  // b + 128, unsigned
+    const uint32_t l = __byte_perm(u, 0x64646464u, 0x4140);
+    const uint32_t h = __byte_perm(u, 0x64646464u, 0x4342);
+    const uint32_t bias = 0x64806480u;      // f16x2 (1152, 1152)
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(l), "r"(bias));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(h), "r"(bias));
+  }
 }
 
 __device__ __forceinline__ uint32_t f16pack(float lo, float hi) {
@@ -290,8 +305,9 @@ __device__ __forceinline__ uint32_t swz8(int t, int c) {
   return static_cast<uint32_t>(t * 128 + ((c ^ (t & 7)) << 4));
 }
 
-// One 16-token page of an E4M3 cache (d = 128) for 8*NT query rows of one
-// warp.  Codes are exact in f16, so the tensor-core tile runs in f16:
+// One 16-token page of an 8-bit cache (d = 128; E4M3 or INT8 codes) for 8*NT
+// query rows of one warp.  Codes are exact in f16, so the tensor-core tile
+// runs in f16:
 //  * K: ldmatrix on the code bytes gives each lane four consecutive channels
 //    of a token per register; converted in pairs they fill the A fragment
 //    with the channel order permuted inside each 16-channel k-step (the q
@@ -302,8 +318,8 @@ __device__ __forceinline__ uint32_t swz8(int t, int c) {
 //    g8 <-> channel 2*g8 and slot g8+8 <-> channel 2*g8+1 of each m-tile.
 //    The V group scales ride on the probabilities (one P^T operand per group).
 // ks, vs: the page's fp32 scales in shared memory, [16 tokens][4 groups].
-template <int NT>
-__device__ __forceinline__ void tile_page_fp8(uint32_t kb, uint32_t vb, const float *ks,
+template <int NT, Code8 kFmt>
+__device__ __forceinline__ void tile_page_q8(uint32_t kb, uint32_t vb, const float *ks,
                                               const float *vs, int ntok, float scale_log2,
                                               int lane, const uint32_t (&qf)[NT][8][2],
                                               float (&acc)[NT][8][4], float (&m_run)[NT][2],
@@ -326,10 +342,10 @@ __device__ __forceinline__ void tile_page_fp8(uint32_t kb, uint32_t vb, const fl
     uint32_t R[4];
     ldmatrix_x4(R, kb + swz8(tok, 2 * j + hi16));
     uint32_t A0[4], A1[4];
-    e4m3x4_to_f16x2x2(R[0], A0[0], A0[2]);
-    e4m3x4_to_f16x2x2(R[1], A0[1], A0[3]);
-    e4m3x4_to_f16x2x2(R[2], A1[0], A1[2]);
-    e4m3x4_to_f16x2x2(R[3], A1[1], A1[3]);
+    code8x4_to_f16x2x2<kFmt>(R[0], A0[0], A0[2]);
+    code8x4_to_f16x2x2<kFmt>(R[1], A0[1], A0[3]);
+    code8x4_to_f16x2x2<kFmt>(R[2], A1[0], A1[2]);
+    code8x4_to_f16x2x2<kFmt>(R[3], A1[1], A1[3]);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       M::run(sg[j][nt], A0, qf[nt][2 * j][0], qf[nt][2 * j][1]);
@@ -404,8 +420,8 @@ __device__ __forceinline__ void tile_page_fp8(uint32_t kb, uint32_t vb, const fl
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       // bytes (0, 2) and (1, 3) of each word: the two channels of a pair
-      e4m3x4_to_f16x2x2(__byte_perm(R[2 * h], 0, 0x3120), A[h][0], A[h][1]);
-      e4m3x4_to_f16x2x2(__byte_perm(R[2 * h + 1], 0, 0x3120), A[h][2], A[h][3]);
+      code8x4_to_f16x2x2<kFmt>(__byte_perm(R[2 * h], 0, 0x3120), A[h][0], A[h][1]);
+      code8x4_to_f16x2x2<kFmt>(__byte_perm(R[2 * h + 1], 0, 0x3120), A[h][2], A[h][3]);
     }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {

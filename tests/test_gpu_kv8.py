@@ -1,4 +1,4 @@
-"""GPU parity of the 8-bit (FP8 E4M3) KV cache against the oracle.
+"""GPU parity of the 8-bit KV caches (FP8 E4M3 and INT8 codes) against the oracle.
 
 Quantisation and append must be bit-exact (codes and scales); attention over
 the 8-bit cache must be within the dtype tolerance of the oracle's attention
@@ -28,44 +28,67 @@ def odt(w):
     return oracle.BF16 if w.dtype == torch.bfloat16 else oracle.F16
 
 
+FORMATS = ["fp8", "int8"]
+
+
+@pytest.fixture(params=FORMATS)
+def fmt(request):
+    return request.param
+
+
+def gpu_fn(kvd, what, fmt):
+    return getattr(kvd, f"kvd_{what}_{fmt}")
+
+
+def orc_fn(what, fmt):
+    return getattr(oracle, f"{what}_{fmt}")
+
+
+def host(t):
+    """Device tensor -> numpy copy; 8-bit codes as their bytes (uint8)."""
+    a = t.cpu().numpy().copy()
+    return a.view(np.uint8) if a.dtype == np.int8 else a
+
+
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("d", [128, 64])
-def test_quantize_bit_exact(kvd, dtype, d):
+def test_quantize_bit_exact(kvd, fmt, dtype, d):
     g = torch.Generator().manual_seed(5)
     x = torch.randn(1000, d, generator=g)
     x[3, 17] = 40.0            # outlier channel
     x[5, 32:64] = 0.0          # all-zero group
     x[7] *= 1e-3               # small row
+    x[9, 40] = float("nan")    # a NaN element
+    x[11, 0:32] = 2.5          # a group with max 127: INT8 scale 1.0, quotients on exact ties
+    x[11, 0], x[11, 1], x[11, 2], x[11, 3] = 127.0, 3.5, -2.5, 0.5
+    x[13, 5] = -2.0 ** -20     # a value far below its group's step
     x = x.to(dtype)
-    codes, scales = kvd.kvd_quantize_fp8(x.cuda())
+    codes, scales = gpu_fn(kvd, "quantize", fmt)(x.cuda())
     torch.cuda.synchronize()
-    oc, os_ = oracle.quantize_fp8(to_words(x), oracle.BF16 if dtype == torch.bfloat16 else oracle.F16)
-    assert np.array_equal(codes.cpu().numpy(), oc)
-    assert np.array_equal(scales.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+    oc, os_ = orc_fn("quantize", fmt)(to_words(x), oracle.BF16 if dtype == torch.bfloat16 else oracle.F16)
+    assert np.array_equal(host(codes), oc)
+    assert np.array_equal(host(scales).view(np.uint32), os_.view(np.uint32))
 
 
-def fp8_state(kvd, w):
-    """Quantise the workload's 16-bit pools on the GPU; also return host copies."""
-    k8, ks = kvd.kvd_quantize_fp8(w.k_cache.cuda())
-    v8, vs = kvd.kvd_quantize_fp8(w.v_cache.cuda())
+def q8_state(kvd, w, fmt):
+    """Quantise the workload's 16-bit pools on the GPU."""
+    k8, ks = gpu_fn(kvd, "quantize", fmt)(w.k_cache.cuda())
+    v8, vs = gpu_fn(kvd, "quantize", fmt)(w.v_cache.cuda())
     torch.cuda.synchronize()
     return k8, v8, ks, vs
 
 
-def host(t):
-    return t.cpu().numpy().copy()
-
-
-def test_append_fp8_bit_exact_whole_pool(kvd):
+def test_append_bit_exact_whole_pool(kvd, fmt):
     w = build_workload("a8", 5, 8, 4, 128, "bf16", [1, 16, 17, 40, 0], seed=1201, spare_pages=3)
     si = step_inputs(w, 0)
-    k8, v8, ks, vs = fp8_state(kvd, w)
+    k8, v8, ks, vs = q8_state(kvd, w, fmt)
     hk8, hv8, hks, hvs = host(k8), host(v8), host(ks), host(vs)
     bt = w.block_table.cuda()
-    kvd.kvd_append_fp8(k8, v8, ks, vs, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    gpu_fn(kvd, "append", fmt)(k8, v8, ks, vs, bt, si["slot"].cuda(), si["k_new"].cuda(),
+                               si["v_new"].cuda())
     torch.cuda.synchronize()
-    oracle.append_fp8(hk8, hv8, hks, hvs, w.block_table.numpy(), si["slot"].numpy(),
-                      to_words(si["k_new"]), to_words(si["v_new"]), oracle.BF16)
+    orc_fn("append", fmt)(hk8, hv8, hks, hvs, w.block_table.numpy(), si["slot"].numpy(),
+                          to_words(si["k_new"]), to_words(si["v_new"]), oracle.BF16)
     assert np.array_equal(host(k8), hk8) and np.array_equal(host(v8), hv8)
     assert np.array_equal(host(ks).view(np.uint32), hks.view(np.uint32))
     assert np.array_equal(host(vs).view(np.uint32), hvs.view(np.uint32))
@@ -83,20 +106,21 @@ CASES = [
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_{c[3]}_N{c[5]}")
-def test_decode_fp8_matches_oracle(kvd, case):
+def test_decode_matches_oracle(kvd, fmt, case):
     B, H_q, H_kv, dtype, lens, parts = case
     w = build_workload("d8", B, H_q, H_kv, 128, dtype, lens, seed=1300 + CASES.index(case),
                        spare_pages=2)
     si = step_inputs(w, 0)
-    k8, v8, ks, vs = fp8_state(kvd, w)
+    k8, v8, ks, vs = q8_state(kvd, w, fmt)
     bt = w.block_table.cuda()
-    kvd.kvd_append_fp8(k8, v8, ks, vs, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    gpu_fn(kvd, "append", fmt)(k8, v8, ks, vs, bt, si["slot"].cuda(), si["k_new"].cuda(),
+                               si["v_new"].cuda())
     lse = torch.empty((B, H_q), dtype=torch.float32, device="cuda")
-    out = kvd.kvd_decode_attention_fp8(si["q"].cuda(), k8, v8, ks, vs, bt, si["seq_lens"].cuda(),
-                                       w.scale, num_partitions=parts, lse_out=lse)
+    out = gpu_fn(kvd, "decode_attention", fmt)(si["q"].cuda(), k8, v8, ks, vs, bt, si["seq_lens"].cuda(),
+                                               w.scale, num_partitions=parts, lse_out=lse)
     torch.cuda.synchronize()
-    ref, ref_lse = oracle.attend_fp8(to_words(si["q"]), host(k8), host(v8), host(ks), host(vs),
-                                     w.block_table.numpy(), si["seq_lens"].numpy(), w.scale, odt(w))
+    ref, ref_lse = orc_fn("attend", fmt)(to_words(si["q"]), host(k8), host(v8), host(ks), host(vs),
+                                         w.block_table.numpy(), si["seq_lens"].numpy(), w.scale, odt(w))
     g = out.float().cpu().double().numpy()
     err = float(np.max(np.abs(g - ref)))
     assert err <= TOL[w.dtype], f"max abs error {err}"
@@ -121,13 +145,13 @@ def test_decode_fp8_matches_oracle(kvd, case):
     assert kvd.kvd_read_device_error() == 0
 
 
-def test_decode_fp8_full_size_gqa70b(kvd):
+def test_decode_full_size_gqa70b(kvd, fmt):
     w = named_config("gqa70b", device="cuda", gen_device="cuda")
     si = step_inputs(w, 0)
-    k8, v8, ks, vs = fp8_state(kvd, w)
+    k8, v8, ks, vs = q8_state(kvd, w, fmt)
     bt = w.block_table.cuda()
-    kvd.kvd_append_fp8(k8, v8, ks, vs, bt, si["slot"], si["k_new"], si["v_new"])
-    out = kvd.kvd_decode_attention_fp8(si["q"], k8, v8, ks, vs, bt, si["seq_lens"], w.scale)
+    gpu_fn(kvd, "append", fmt)(k8, v8, ks, vs, bt, si["slot"], si["k_new"], si["v_new"])
+    out = gpu_fn(kvd, "decode_attention", fmt)(si["q"], k8, v8, ks, vs, bt, si["seq_lens"], w.scale)
     torch.cuda.synchronize()
     assert torch.isfinite(out.float()).all()
     lens = w.seq_lens0.numpy()
@@ -138,9 +162,9 @@ def test_decode_fp8_full_size_gqa70b(kvd):
     btn = w.block_table.numpy()
     worst = 0.0
     for b in rows:
-        ref, _ = oracle.attend_fp8(q[b:b + 1], hk8, hv8, hks, hvs, btn[b:b + 1], sl[b:b + 1], w.scale,
-                                   oracle.BF16)
+        ref, _ = orc_fn("attend", fmt)(q[b:b + 1], hk8, hv8, hks, hvs, btn[b:b + 1], sl[b:b + 1],
+                                       w.scale, oracle.BF16)
         worst = max(worst, float(np.max(np.abs(out[b].float().cpu().double().numpy() - ref[0]))))
-    print(f"gqa70b fp8: max abs error {worst:.3e} over sequences {rows}")
+    print(f"gqa70b {fmt}: max abs error {worst:.3e} over sequences {rows}")
     assert worst <= TOL[w.dtype]
     assert kvd.kvd_read_device_error() == 0
