@@ -277,10 +277,15 @@ __global__ void __launch_bounds__(32 * kWarps, 1)
 // (MMAs of one thread run in issue order).
 // Every wait is bounded; a timed-out role flags the error word and the CTA
 // still releases its TMEM after the MMAs it issued have completed.
+// pages per step (N = 16 x pages), settable at build time for tuning
+#ifndef KVD_TC_PAGES
+#define KVD_TC_PAGES 4
+#endif
 namespace {
-constexpr int kTcPages = 4;                       // pages per step
+constexpr int kTcPages = KVD_TC_PAGES;            // pages per step
+static_assert(kTcPages == 2 || kTcPages == 4, "steps of 2 or 4 pages");
 constexpr int kTcTok = kTcPages * kPage;          // N of QK^T: 64 tokens
-constexpr int kTcStages = 2;                      // steps of K/V in flight per CTA
+constexpr int kTcStages = 8 / kTcPages;          // steps of K/V in flight per CTA (8 pages)
 constexpr int kTcWarps = 6;
 constexpr int kTcHalf = kTcPages * kPage * 128;   // one 64-column half of a step's K (or V): 8 KB
 constexpr int kTcStage = 4 * kTcHalf;             // K half 0, K half 1, V half 0, V half 1
@@ -570,15 +575,14 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
       tc::fence_after_sync();
       float x[kTcTok];
       {
-        uint32_t r0v[32], r1v[32];
-        tc::ld32(tbase + lanes + kColS + bs * kTcTok, r0v);
-        tc::ld32(tbase + lanes + kColS + bs * kTcTok + 32, r1v);
+        uint32_t rv[kTcTok / 32][32];
+#pragma unroll
+        for (int c = 0; c < kTcTok / 32; ++c) tc::ld32(tbase + lanes + kColS + bs * kTcTok + c * 32, rv[c]);
         tc::wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          x[i] = __uint_as_float(r0v[i]);
-          x[32 + i] = __uint_as_float(r1v[i]);
-        }
+        for (int c = 0; c < kTcTok / 32; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(rv[c][i]);
       }
       // row maximum of the scaled scores (in log2 units): the scale is folded
       // into the exponent below, so the raw scores are compared (their
@@ -632,8 +636,8 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
       else exps(std::true_type{});
       const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l = l * alpha + sum;
-      tc::st32(tbase + lanes + kColS + bs * kTcTok, ph);
-      if constexpr (kBf16) tc::st32(tbase + lanes + kColS + bs * kTcTok + kTcTok / 2, pl);
+      tc::st_cols<kTcTok / 2>(tbase + lanes + kColS + bs * kTcTok, ph);
+      if constexpr (kBf16) tc::st_cols<kTcTok / 2>(tbase + lanes + kColS + bs * kTcTok + kTcTok / 2, pl);
       if (j >= 1) {
         // O holds the product of step j-1 once its o_done phase completes
         const bool got2 = mbar_wait_bounded(O_DONE, (j - 1) & 1);

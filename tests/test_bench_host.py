@@ -1,0 +1,67 @@
+"""Host-side pieces of bench.py that need no GPU: the hash-keyed lookup of a
+profile's DRAM traffic and the bounded CPU-oracle sampler of the reference arm."""
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _summary(tmp, name, workload, mode, digest, nbytes):
+    (tmp / name).write_text(
+        f"# test\n\nworkload: {workload}\ncache_mode: {mode}\n"
+        f"decode_source_sha256_16: {digest}\ndram_bytes_per_launch: {nbytes}\n", encoding="utf-8")
+
+
+def test_profile_traffic_is_keyed_by_source_hash_workload_and_mode(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "PROFILE_DIR", str(tmp_path))
+    now = bench.source_hash()
+    _summary(tmp_path, "decode_kernel_a.md", "mha7b", "fused", now, 111)
+    _summary(tmp_path, "decode_kernel_b.md", "mha7b", "fp8", now, 222)
+    _summary(tmp_path, "decode_kernel_c.md", "gqa70b", "fused", "0" * 16, 333)  # stale source
+    _summary(tmp_path, "other_kernel.md", "gqa70b", "fused", now, 444)          # not a decode summary
+    assert bench.profile_traffic("mha7b", "fused") == 111
+    assert bench.profile_traffic("mha7b", "fp8") == 222
+    assert bench.profile_traffic("mha7b", "int8") is None
+    assert bench.profile_traffic("gqa70b", "fused") is None
+
+
+def test_committed_profiles_parse():
+    # every committed decode summary carries the machine-readable lines
+    for name in sorted(os.listdir(os.path.join(ROOT, "profiles"))):
+        if not (name.startswith("decode_kernel") and name.endswith(".md")):
+            continue
+        text = open(os.path.join(ROOT, "profiles", name), encoding="utf-8").read()
+        if "dram_bytes_per_launch:" in text:
+            for key in ("workload:", "cache_mode:", "decode_source_sha256_16:"):
+                assert key in text, f"{name} lacks {key}"
+
+
+def test_oracle_sampler_bounds_and_reuses_inputs():
+    smp = bench.OracleSampler("tiny")
+    gbs, spent, done = smp.run(0.0)             # at least one unit even with no budget
+    assert done == 1 and gbs > 0 and spent > 0
+    gbs2, _, done2 = smp.run(0.0, min_units=3)
+    assert done2 == 3 and gbs2 > 0
+    assert len(smp.cache) == 1                  # one sequence in the tiny shape, built once
+    assert "4 append+attend units over 1 of the 1 sequences of the tiny shape" in smp.describe()
+
+
+def test_long_sequences_are_sampled_by_kv_head():
+    smp = bench.OracleSampler("long")
+    c = smp._inputs(0)
+    # 131072 tokens x 2 x 128 x 2 B = 64 MiB per KV head: one KV head and its 8 query heads
+    assert c["heads"] == (8, 1)
+
+
+def test_reference_arm_prints_one_json_line(capsys):
+    args = bench.parse_args(["--impl", "reference", "--workload", "tiny", "--steps", "4",
+                             "--warmup", "3", "--ref-budget", "0.5"])
+    assert bench.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["steps"] == 4 and line["warmup"] == 3
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
