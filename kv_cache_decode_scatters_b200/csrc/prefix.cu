@@ -281,7 +281,7 @@ namespace {
 constexpr int kTcPages = 4;                       // pages per step
 constexpr int kTcTok = kTcPages * kPage;          // N of QK^T: 64 tokens
 constexpr int kTcStages = 2;                      // steps of K/V in flight per CTA
-constexpr int kTcWarps = 10;                     // TMA, MMA, 8 softmax warps
+constexpr int kTcWarps = 6;
 constexpr int kTcHalf = kTcPages * kPage * 128;   // one 64-column half of a step's K (or V): 8 KB
 constexpr int kTcStage = 4 * kTcHalf;             // K half 0, K half 1, V half 0, V half 1
 constexpr int kTcQBytes = kRowsPerCta * 128 * 2;  // Q tile, two 64-column halves: 32 KB
@@ -289,9 +289,8 @@ constexpr uint32_t kColO = 0;                     // O: 128 fp32 columns
 constexpr uint32_t kColS = 128;                   // S: 2 x 64 fp32 columns; P overwrites S
 constexpr uint32_t kTmemCols = 256;
 constexpr float kRefSlack = 8.f;                  // log2 of the largest probability kept
-constexpr int kTcBars = 4 * kTcStages + 7 + 12;   // + score exchanges (4 x 2) and sums (4)
-constexpr int kTcXch = (2 * 2 + 2) * kRowsPerCta * 4;  // score extremes [2 parities][2 halves], sums [2]
-constexpr size_t kTcSmem = 1024 + kTcQBytes + (size_t)kTcStages * kTcStage + kTcXch + kTcBars * 8 + 64;
+constexpr int kTcBars = 4 * kTcStages + 7;
+constexpr size_t kTcSmem = 1024 + kTcQBytes + (size_t)kTcStages * kTcStage + kTcBars * 8 + 64;
 // two CTAs per SM share its 512 TMEM columns; a third never fits beside them
 static_assert(2 * kTcSmem <= 227 * 1024 && 3 * kTcSmem > 228 * 1024,
               "exactly two CTAs per SM: each allocates half of TMEM");
@@ -308,9 +307,7 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
   uint8_t *qs = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   uint8_t *ring = qs + kTcQBytes;
-  float *xmax = reinterpret_cast<float *>(ring + (size_t)kTcStages * kTcStage);  // [2][2][rows]
-  float *lsum = xmax + 2 * 2 * kRowsPerCta;                                       // [2][rows]
-  uint64_t *bars = reinterpret_cast<uint64_t *>(lsum + 2 * kRowsPerCta);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ring + (size_t)kTcStages * kTcStage);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kTcBars);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -371,8 +368,6 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
   const uint32_t S_FULL = bar0 + 8 * (4 * kTcStages);  // + 8 * buffer
   const uint32_t P_FULL = S_FULL + 16;                 // + 8 * buffer
   const uint32_t O_DONE = S_FULL + 32, Q_FULL = S_FULL + 40, DRAIN = S_FULL + 48;
-  const uint32_t XCH = S_FULL + 56;  // + 16 * quarter + 8 * parity: score exchange of a row pair
-  const uint32_t LBAR = XCH + 64;    // + 8 * quarter: row-sum exchange
 
   if (warp == 0) {
     __syncwarp();
@@ -388,13 +383,11 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
     }
     mbar_init(S_FULL, 1);
     mbar_init(S_FULL + 8, 1);
-    mbar_init(P_FULL, 8);
-    mbar_init(P_FULL + 8, 8);
+    mbar_init(P_FULL, 4);
+    mbar_init(P_FULL + 8, 4);
     mbar_init(O_DONE, 1);
-    mbar_init(Q_FULL, 8);
+    mbar_init(Q_FULL, 4);
     mbar_init(DRAIN, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(XCH + 8 * i, 2);
-    for (int i = 0; i < 4; ++i) mbar_init(LBAR + 8 * i, 2);
     mbar_init_fence();
   }
   tc::fence_before_sync();
@@ -540,51 +533,34 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    // Two warps per TMEM lane quarter: warp w handles rows quarter*32 + lane
-    // and the columns of its half of each step (half = (w - 2) / 4).  The two
-    // halves of a row exchange their score extremes through shared memory
-    // every step (mbarrier of count 2, bounded wait), so both take the same
-    // reference max; each keeps its own part of the row sum, O's columns of
-    // its half, and the two parts of l meet once at the end.
-    const int quarter = warp & 3, half = (warp - 2) >> 2;
+    const int quarter = warp & 3;
     const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
-    const int rc = quarter * 32 + lane;        // row of this CTA
-    const int row = r0 + rc;                   // row of the group: member row / G, head row % G
+    const int row = r0 + quarter * 32 + lane;  // row of the group: member row / G, head row % G
     const bool live = row < rows;
     const int b = s0 + (live ? row / a.G : 0), jr = live ? row % a.G : 0;
-    constexpr int kHalfTok = kTcTok / 2;       // columns of S per warp and step
-    constexpr int kHalfPages = kTcPages / 2;
     {
-      // this row's half of Q into the K-major, 128-byte-swizzled tile the MMA reads
+      // this row of Q into the K-major, 128-byte-swizzled tile the MMA reads
+      const int r = quarter * 32 + lane;
       const uint4 *qv = reinterpret_cast<const uint4 *>(
           static_cast<const T *>(a.q) +
           (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + jr) * D);
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        const uint4 v = live ? __ldg(qv + half * 8 + cc) : make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4 *>(qs + half * (kTcQBytes / 2) + rc * 128 + ((cc ^ (rc & 7)) << 4)) = v;
+      for (int c = 0; c < 2 * 8; ++c) {
+        const uint4 v = live ? __ldg(qv + c) : make_uint4(0u, 0u, 0u, 0u);
+        const int half = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4 *>(qs + half * (kTcQBytes / 2) + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
       }
       fence_proxy_async_smem();  // visible to the tensor core's reads
       __syncwarp();
       if (lane == 0) mbar_arrive(Q_FULL);
     }
-    const uint32_t XBAR = XCH + 16 * quarter;  // + 8 * (step parity)
-    auto exchange = [&](float *slot, float mine, uint32_t bar, uint32_t parity, float &other) -> bool {
-      slot[half * kRowsPerCta + rc] = mine;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar);
-      const bool got = mbar_wait_bounded(bar, parity);
-      if (!__all_sync(0xffffffffu, got)) return false;
-      other = slot[(1 - half) * kRowsPerCta + rc];
-      return true;
-    };
 
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     uint32_t next_mask = step_mask(0);  // loaded one step before use
     for (int j = 0; j < nsteps; ++j) {
       const int bs = j & 1;
-      const uint32_t pm = (next_mask >> (half * kHalfPages)) & ((1u << kHalfPages) - 1u);
+      const uint32_t pm = next_mask;
       next_mask = step_mask(j + 1);
       const bool got = mbar_wait_bounded(S_FULL + 8 * bs, (j >> 1) & 1);
       if (!__all_sync(0xffffffffu, got)) {
@@ -592,22 +568,26 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
         break;
       }
       tc::fence_after_sync();
-      float x[kHalfTok];
+      float x[kTcTok];
       {
-        uint32_t rv[kHalfTok];
-        tc::ld_cols<kHalfTok>(tbase + lanes + kColS + bs * kTcTok + half * kHalfTok, rv);
+        uint32_t r0v[32], r1v[32];
+        tc::ld32(tbase + lanes + kColS + bs * kTcTok, r0v);
+        tc::ld32(tbase + lanes + kColS + bs * kTcTok + 32, r1v);
         tc::wait_ld();
 #pragma unroll
-        for (int i = 0; i < kHalfTok; ++i) x[i] = __uint_as_float(rv[i]);
+        for (int i = 0; i < 32; ++i) {
+          x[i] = __uint_as_float(r0v[i]);
+          x[32 + i] = __uint_as_float(r1v[i]);
+        }
       }
       // row maximum of the scaled scores (in log2 units): the scale is folded
       // into the exponent below, so the raw scores are compared (their
       // minimum when the scale is negative); masked columns are -inf
       const float c = a.scale_log2;
-      const bool full_step = pm == (1u << kHalfPages) - 1u;  // warp-uniform
+      const bool full_step = pm == (1u << kTcPages) - 1u;  // warp-uniform
       if (!full_step) {
 #pragma unroll
-        for (int i = 0; i < kHalfTok; ++i)
+        for (int i = 0; i < kTcTok; ++i)
           if (!((pm >> (i / kPage)) & 1u)) x[i] = c >= 0.f ? -INFINITY : INFINITY;
       }
       float e4[4];
@@ -615,30 +595,24 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
       for (int k = 0; k < 4; ++k) e4[k] = x[k];
       if (c >= 0.f) {
 #pragma unroll
-        for (int i = 4; i < kHalfTok; ++i) e4[i & 3] = fmaxf(e4[i & 3], x[i]);
+        for (int i = 4; i < kTcTok; ++i) e4[i & 3] = fmaxf(e4[i & 3], x[i]);
       } else {
 #pragma unroll
-        for (int i = 4; i < kHalfTok; ++i) e4[i & 3] = fminf(e4[i & 3], x[i]);
+        for (int i = 4; i < kTcTok; ++i) e4[i & 3] = fminf(e4[i & 3], x[i]);
       }
-      float ext = c >= 0.f ? fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]))
-                           : fminf(fminf(e4[0], e4[1]), fminf(e4[2], e4[3]));
-      float ext_other;
-      if (!exchange(xmax + bs * 2 * kRowsPerCta, ext, XBAR + 8 * bs, (j >> 1) & 1, ext_other)) {
-        ok = false;
-        break;
-      }
-      ext = c >= 0.f ? fmaxf(ext, ext_other) : fminf(ext, ext_other);
+      const float ext = c >= 0.f ? fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]))
+                                 : fminf(fminf(e4[0], e4[1]), fminf(e4[2], e4[3]));
       // an all-masked row keeps -inf; otherwise the largest scaled score
       const float mx = (ext == INFINITY || ext == -INFINITY) ? -INFINITY : ext * c;
       const float m_new = mx > m_ref + kRefSlack ? mx : m_ref;
       const float alpha = m_new == m_ref ? 1.f : fast_exp2(m_ref - m_new);
       const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      uint32_t ph[kHalfTok / 2], pl[kHalfTok / 2];
+      uint32_t ph[kTcTok / 2], pl[kTcTok / 2];
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
       // exp2(s * c - m) per column; masked columns (partial steps only) are 0
       auto exps = [&](auto masked) {
 #pragma unroll
-        for (int i = 0; i < kHalfTok; i += 2) {
+        for (int i = 0; i < kTcTok; i += 2) {
           float e0 = fast_exp2(fmaf(x[i], c, -m_use));
           float e1 = fast_exp2(fmaf(x[i + 1], c, -m_use));
           if constexpr (decltype(masked)::value) {
@@ -658,11 +632,8 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
       else exps(std::true_type{});
       const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l = l * alpha + sum;
-      // P over this half's part of S: tokens half*kHalfTok.. -> 16-bit pairs
-      tc::st_cols<kHalfTok / 2>(tbase + lanes + kColS + bs * kTcTok + half * (kHalfTok / 2), ph);
-      if constexpr (kBf16)
-        tc::st_cols<kHalfTok / 2>(tbase + lanes + kColS + bs * kTcTok + kTcTok / 2 + half * (kHalfTok / 2),
-                                  pl);
+      tc::st32(tbase + lanes + kColS + bs * kTcTok, ph);
+      if constexpr (kBf16) tc::st32(tbase + lanes + kColS + bs * kTcTok + kTcTok / 2, pl);
       if (j >= 1) {
         // O holds the product of step j-1 once its o_done phase completes
         const bool got2 = mbar_wait_bounded(O_DONE, (j - 1) & 1);
@@ -673,14 +644,13 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
         tc::fence_after_sync();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-          for (int cq = 0; cq < D / 64; ++cq) {  // this half's 64 columns of O
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t r[32];
-            const uint32_t oc = tbase + lanes + kColO + half * (D / 2) + cq * 32;
-            tc::ld32(oc, r);
+            tc::ld32(tbase + lanes + kColO + c * 32, r);
             tc::wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tc::st32(oc, r);
+            tc::st32(tbase + lanes + kColO + c * 32, r);
           }
         }
       }
@@ -694,35 +664,32 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
       const bool got = mbar_wait_bounded(O_DONE, (nsteps - 1) & 1);
       ok = __all_sync(0xffffffffu, got);
     }
-    float l_other = 0.f;
-    if (ok) ok = exchange(lsum, l, LBAR + 8 * quarter, 0, l_other);
     if (!ok) {
       if (lane == 0) flag_error(a.err, kErrTimeout);
     } else {
       tc::fence_after_sync();
-      const float lt = l + l_other;
-      const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      const float lse = lt > 0.f ? (m_ref + fast_log2(lt)) * kLn2 : -INFINITY;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float lse = l > 0.f ? (m_ref + fast_log2(l)) * kLn2 : -INFINITY;
       const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + b) * a.G + jr;
-      float4 *o = reinterpret_cast<float4 *>(a.pre_o + idx * D + half * (D / 2));
+      float4 *o = reinterpret_cast<float4 *>(a.pre_o + idx * D);
 #pragma unroll 1
-      for (int cq = 0; cq < D / 64; ++cq) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
-        tc::ld32(tbase + lanes + kColO + half * (D / 2) + cq * 32, r);
+        tc::ld32(tbase + lanes + kColO + c * 32, r);
         tc::wait_ld();
         if (live) {
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
-            const float4 v = lt > 0.f ? make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
-                                                    __uint_as_float(r[i + 2]) * inv,
-                                                    __uint_as_float(r[i + 3]) * inv)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-            o[cq * 8 + i / 4] = v;
+            const float4 v = l > 0.f ? make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
+                                                   __uint_as_float(r[i + 2]) * inv,
+                                                   __uint_as_float(r[i + 3]) * inv)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+            o[c * 8 + i / 4] = v;
           }
         }
         __syncwarp();
       }
-      if (live && half == 0) a.pre_lse[idx] = lse;
+      if (live) a.pre_lse[idx] = lse;
     }
   }
 
