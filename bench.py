@@ -37,7 +37,7 @@ METRIC = "paged decode-attention achieved HBM GB/s (% of B200 peak); us per deco
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 DECODE_SOURCES = [os.path.join(ROOT, "kv_cache_decode_scatters_b200", "csrc", f)
-                  for f in ("decode.cu", "tile.cuh", "common.cuh")]
+                  for f in ("decode.cu", "tile.cuh", "common.cuh", "quant.cuh")]
 
 
 # ------------------------------------------------------------------ helpers
@@ -101,8 +101,8 @@ def source_hash() -> str:
 def profile_traffic(workload: str, mode: str):
     """DRAM bytes per decode launch from a committed ncu summary under
     profiles/, if one was taken on the current decode kernel sources for this
-    workload and step mode ("fused", "separate_append", "shared_prefix", "fp8"
-    or "int8")."""
+    workload and step mode ("fused", "separate_append", "shared_prefix", "fp8",
+    "int8", "fp8_separate_append" or "int8_separate_append")."""
     try:
         names = sorted(os.listdir(PROFILE_DIR))
     except OSError:
@@ -368,6 +368,7 @@ def run_ours(args):
         f8 = {"fmt": fmt, "k8": k8, "v8": v8, "ks": ks, "vs": vs,
               "append": getattr(kvd, "kvd_append_" + fmt),
               "decode": getattr(kvd, "kvd_decode_attention_" + fmt),
+              "step": getattr(kvd, "kvd_decode_step_" + fmt),
               "name": "E4M3" if fmt == "fp8" else "INT8"}
 
     sp = None
@@ -382,6 +383,14 @@ def run_ours(args):
         ws = torch.empty(n, dtype=torch.uint8, device=dev)
 
     def step(ev_a=None, ev_b=None):
+        if f8 is not None and not args.separate_append:
+            if ev_a is not None:
+                ev_a.record(stream)
+            f8["step"](q, k_new, v_new, f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, seq_lens, w.scale,
+                       out=out, num_partitions=args.partitions, workspace=ws, stream=stream)
+            if ev_b is not None:
+                ev_b.record(stream)
+            return
         if f8 is not None:
             f8["append"](f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, slot, k_new, v_new, stream=stream)
             if ev_a is not None:
@@ -429,7 +438,7 @@ def run_ours(args):
         a_bytes -= w.groups * (w.B // w.groups - 1) * w.prefix_tokens * kv_tok
     step_bytes = a_bytes + p_bytes
     # bytes of the call the roofline times (events bracket it)
-    timed_bytes = a_bytes if (args.separate_append or f8 is not None) else step_bytes
+    timed_bytes = a_bytes if args.separate_append else step_bytes
 
     graph = None
     if args.graph:
@@ -492,7 +501,7 @@ def run_ours(args):
 
     # ---- end to end through the public API with pinned host buffers
     inputs = [("q", q), ("k_new", k_new), ("v_new", v_new), ("seq_lens", seq_lens)]
-    if args.separate_append or f8 is not None:
+    if args.separate_append:
         inputs.append(("slot", slot))
     h_in = {n: t.cpu().pin_memory() for n, t in inputs}
     d_in = {n: torch.empty_like(t, device=dev) for n, t in h_in.items()}
@@ -504,7 +513,11 @@ def run_ours(args):
     def e2e_step():
         for n in h_in:
             d_in[n].copy_(h_in[n], non_blocking=True)
-        if f8 is not None:
+        if f8 is not None and not args.separate_append:
+            f8["step"](d_in["q"], d_in["k_new"], d_in["v_new"], f8["k8"], f8["v8"], f8["ks"], f8["vs"],
+                       bt, d_in["seq_lens"], w.scale, out=out, num_partitions=args.partitions,
+                       workspace=ws, stream=stream)
+        elif f8 is not None:
             f8["append"](f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, d_in["slot"],
                                d_in["k_new"], d_in["v_new"], stream=stream)
             f8["decode"](d_in["q"], f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt,
@@ -575,6 +588,9 @@ def run_ours(args):
                 2 * w.k_cache.numel() * 2 / 1e9),
             "step": ("kvd_append_%s + kvd_decode_attention_%s over an %s cache "
                      "(quantising append, decode, merge kernels)" % (f8["fmt"], f8["fmt"], f8["name"])
+                     if f8 is not None and args.separate_append else
+                     "kvd_decode_step_%s over an %s cache (decode kernel with fused quantising "
+                     "append, merge kernel)" % (f8["fmt"], f8["name"])
                      if f8 is not None else
                      "kvd_decode_attention_shared_prefix with fused append (prefix, decode, merge kernels)"
                      if sp is not None else
@@ -592,7 +608,9 @@ def run_ours(args):
             "frac": round(achieved / peak, 4),
             "peak_kind": peak_kind,
             "kernel": ("kvd_decode_attention_%s call (decode_kernel over %s pages + merge)"
-                       % (f8["fmt"], f8["name"]) if f8 is not None else
+                       % (f8["fmt"], f8["name"]) if f8 is not None and args.separate_append else
+                       "kvd_decode_step_%s call (decode_kernel over %s pages with fused quantising "
+                       "append + merge)" % (f8["fmt"], f8["name"]) if f8 is not None else
                        "kvd_decode_attention_shared_prefix call (prefix_kernel + decode_kernel with fused "
                        "append + merge)" if sp is not None else
                        "kvd_decode_attention call (decode_kernel + decode_merge_kernel)"
@@ -600,7 +618,8 @@ def run_ours(args):
                        "kvd_decode_step call (decode_kernel with fused append + decode_merge_kernel)")
                       + ", CUDA events on the launching stream; achieved = its algorithmic bytes / mean duration",
             "bytes_per_launch": timed_bytes,
-            "traffic": profile_traffic(w.name, f8["fmt"] if f8 is not None else "shared_prefix" if sp is not None
+            "traffic": profile_traffic(w.name, (f8["fmt"] + ("_separate_append" if args.separate_append else ""))
+                                      if f8 is not None else "shared_prefix" if sp is not None
                                       else "separate_append" if args.separate_append else "fused"),
         },
         "frac_of_8000_spec": round(achieved / 8000.0, 4),
@@ -620,8 +639,7 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "us_per_step": round(e2e_s / e2e_steps * 1e6, 2),
                 "how": "pinned host inputs -> H2D, append, decode, D2H of out, stream sync; wall clock"},
-        "gpu_launches": (3 if (f8 is not None or args.separate_append or sp is not None)
-                         else 2) * args.steps * per,
+        "gpu_launches": (3 if (args.separate_append or sp is not None) else 2) * args.steps * per,
         "graph": ({"steps_per_graph": args.graph_steps, "replays": args.steps} if graph is not None
                   else None),
         "clocks": clocks,
@@ -649,7 +667,8 @@ def parse_args(argv=None):
                    choices=["tiny", "mha7b", "gqa70b", "long", "cbatch"])
     p.add_argument("--partitions", type=int, default=0, help="0 = automatic")
     p.add_argument("--separate-append", action="store_true",
-                   help="time kvd_append + kvd_decode_attention instead of the fused kvd_decode_step")
+                   help="time kvd_append[_fp8|_int8] + kvd_decode_attention[_fp8|_int8] instead of "
+                        "the fused kvd_decode_step[_fp8|_int8]")
     p.add_argument("--e2e-steps", type=int, default=300)
     p.add_argument("--kv-fp8", action="store_true",
                    help="store the cache as FP8 E4M3 codes with per-32-channel scales (d=128)")

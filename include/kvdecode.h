@@ -241,6 +241,40 @@ kvd_status kvd_decode_attention_int8(const void *q, const int8_t *k_codes, const
                                      void *workspace, size_t workspace_bytes, float *lse_out,
                                      kvd_dtype dtype, void *stream);
 
+/*
+ * kvd_decode_step_fp8, kvd_decode_step_int8 -- kvd_decode_step over an 8-bit
+ * cache: the quantising append of kvd_append_{fp8,int8} followed by the
+ * attention of kvd_decode_attention_{fp8,int8}, in one decode launch.
+ * [KVF] section "一、KV Cache" (a decode step appends the new token's K/V,
+ * then attends over the whole cache including it); [BLOG] section
+ * "工程优化手段 / 量化" (the cache those steps read and write holds 8-bit codes
+ * with per-group scales).
+ *
+ *   k_new, v_new     device, [B][H_kv][d] in dtype, 16-byte aligned
+ *   k_codes, v_codes, k_scale, v_scale  the 8-bit cache, written in place
+ *   other arguments as kvd_decode_attention_{fp8,int8} (d = 128)
+ * Every sequence b with seq_lens[b] >= 1 appends its new token at position
+ * seq_lens[b] - 1; seq_lens[b] = 0 appends nothing.  The codes and scales
+ * written are bit-identical to kvd_append_{fp8,int8} with slot =
+ * seq_lens - 1, and out to that append followed by
+ * kvd_decode_attention_{fp8,int8} with the same num_partitions.  The page that
+ * receives the new token must not be shared with another sequence.
+ */
+kvd_status kvd_decode_step_fp8(const void *q, const void *k_new, const void *v_new,
+                               uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
+                               const int32_t *block_table, const int32_t *seq_lens, float scale,
+                               void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                               int max_blocks_per_seq, int num_partitions, void *workspace,
+                               size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+                               void *stream);
+kvd_status kvd_decode_step_int8(const void *q, const void *k_new, const void *v_new,
+                                int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale,
+                                const int32_t *block_table, const int32_t *seq_lens, float scale,
+                                void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                                int max_blocks_per_seq, int num_partitions, void *workspace,
+                                size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+                                void *stream);
+
 /* Bytes of the library's fixed scratch array used by kvd_decode_attention_static. */
 #define KVD_STATIC_WORKSPACE_BYTES (8u << 20)
 

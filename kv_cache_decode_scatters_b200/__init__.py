@@ -22,8 +22,8 @@ __all__ = [
     "KVD_F16", "KVD_BF16", "KVD_PAGE_TOKENS", "KvdError",
     "kvd_append", "kvd_decode_attention", "kvd_decode_step", "kvd_decode_attention_static",
     "kvd_decode_attention_shared_prefix", "kvd_shared_prefix_workspace_size",
-    "kvd_quantize_fp8", "kvd_append_fp8", "kvd_decode_attention_fp8",
-    "kvd_quantize_int8", "kvd_append_int8", "kvd_decode_attention_int8",
+    "kvd_quantize_fp8", "kvd_append_fp8", "kvd_decode_attention_fp8", "kvd_decode_step_fp8",
+    "kvd_quantize_int8", "kvd_append_int8", "kvd_decode_attention_int8", "kvd_decode_step_int8",
     "kvd_merge_lse",
     "kvd_workspace_size", "KVD_STATIC_WORKSPACE_BYTES",
     "kvd_auto_partitions", "kvd_kv_bytes_per_token", "kvd_read_device_error",
@@ -70,6 +70,9 @@ def _load():
         getattr(L, "kvd_decode_attention_" + fmt).restype = I
         getattr(L, "kvd_decode_attention_" + fmt).argtypes = [P, P, P, P, P, P, P, F, P, I, I, I, I,
                                                               I, I, I, P, S, P, I, P]
+        getattr(L, "kvd_decode_step_" + fmt).restype = I
+        getattr(L, "kvd_decode_step_" + fmt).argtypes = [P, P, P, P, P, P, P, P, P, F, P, I, I, I,
+                                                         I, I, I, I, P, S, P, I, P]
     L.kvd_decode_attention_static.restype = I
     L.kvd_decode_attention_static.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, P, I, P]
     L.kvd_merge_lse.restype = I
@@ -311,11 +314,14 @@ def _append8(fmt, k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, 
 
 
 def _decode8(fmt, q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
-             num_partitions, workspace, lse_out, stream):
+             num_partitions, workspace, lse_out, stream, k_new=None, v_new=None):
     B, H_q, d = q.shape
     NB, H_kv, P, d2 = k_codes.shape
     if P != KVD_PAGE_TOKENS or d2 != d:
         raise ValueError("q / cache shape mismatch")
+    step = k_new is not None
+    if step and (tuple(k_new.shape) != (B, H_kv, d) or v_new is None or v_new.shape != k_new.shape):
+        raise ValueError("k_new / v_new must be [B, H_kv, d]")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
@@ -324,13 +330,15 @@ def _decode8(fmt, q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, 
         workspace = alloc_workspace(B, H_q, H_kv, d, num_partitions, q.device)
     lse_ptr = None if lse_out is None else _dev(lse_out, "lse_out", torch.float32)
     c = _CODE8[fmt]
-    _check(getattr(_lib, "kvd_decode_attention_" + fmt)(
-        _dev(q, "q", q.dtype), _dev(k_codes, "k_codes", c), _dev(v_codes, "v_codes", c),
+    name = ("kvd_decode_step_" if step else "kvd_decode_attention_") + fmt
+    new = (_dev(k_new, "k_new", q.dtype), _dev(v_new, "v_new", q.dtype)) if step else ()
+    _check(getattr(_lib, name)(
+        _dev(q, "q", q.dtype), *new, _dev(k_codes, "k_codes", c), _dev(v_codes, "v_codes", c),
         _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
         _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
         float(scale), _dev(out, "out", q.dtype), B, H_q, H_kv, d, NB, block_table.shape[1],
         int(num_partitions), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
-        lse_ptr, _dtype_code(q), _stream(stream)), "kvd_decode_attention_" + fmt)
+        lse_ptr, _dtype_code(q), _stream(stream)), name)
     return out
 
 
@@ -352,6 +360,16 @@ def kvd_decode_attention_fp8(q, k_codes, v_codes, k_scale, v_scale, block_table,
                     num_partitions, workspace, lse_out, stream)
 
 
+def kvd_decode_step_fp8(q, k_new, v_new, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                        scale=None, out=None, num_partitions=0, workspace=None, lse_out=None,
+                        stream=None):
+    """kvd_decode_step over the E4M3 cache: quantise k_new/v_new [B,H_kv,d] into
+    position seq_lens[b]-1 of every non-empty sequence, then attend
+    (kvd_append_fp8 + kvd_decode_attention_fp8 in one launch).  Returns out."""
+    return _decode8("fp8", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
+                    num_partitions, workspace, lse_out, stream, k_new, v_new)
+
+
 def kvd_quantize_int8(src, codes=None, scales=None, stream=None):
     """Quantise rows src [..., d] (fp16/bf16) into INT8 codes (int8 [..., d])
     and fp32 scales [..., d/32], one per 32 channels.  Returns (codes, scales)."""
@@ -368,6 +386,15 @@ def kvd_decode_attention_int8(q, k_codes, v_codes, k_scale, v_scale, block_table
     """kvd_decode_attention over the INT8 cache (d = 128).  Returns out (q's dtype)."""
     return _decode8("int8", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
                     num_partitions, workspace, lse_out, stream)
+
+
+def kvd_decode_step_int8(q, k_new, v_new, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                         scale=None, out=None, num_partitions=0, workspace=None, lse_out=None,
+                         stream=None):
+    """kvd_decode_step over the INT8 cache (kvd_append_int8 + kvd_decode_attention_int8
+    in one launch).  Returns out."""
+    return _decode8("int8", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
+                    num_partitions, workspace, lse_out, stream, k_new, v_new)
 
 
 def kvd_decode_attention_static(q, k_cache, v_cache, block_table, seq_lens, scale=None, out=None,

@@ -280,8 +280,7 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   if (q8) {
     if (d != 128) return fail(KVD_ERR_UNSUPPORTED, "the 8-bit cache supports d = 128 only");
     if (!v_scale) return fail(KVD_ERR_INVALID, "v_scale is NULL");
-    if (k_new || n_groups > 0)
-      return fail(KVD_ERR_UNSUPPORTED, "the 8-bit cache has no fused append or shared-prefix mode");
+    if (n_groups > 0) return fail(KVD_ERR_UNSUPPORTED, "the 8-bit cache has no shared-prefix mode");
     if (!aligned(k_scale, 16) || !aligned(v_scale, 16))
       return fail(KVD_ERR_INVALID, "scale pools must be 16-byte aligned");
   }
@@ -383,8 +382,10 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   a.pre_o = nullptr;
   a.pre_lse = nullptr;
   a.pre_chunks = 0;
-  a.k_scale = k_scale;
-  a.v_scale = v_scale;
+  // the scale pools are written only when k_new is given (the _step calls,
+  // which take them writable)
+  a.k_scale = const_cast<float *>(k_scale);
+  a.v_scale = const_cast<float *>(v_scale);
 
   const kvd::DType dt = dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -490,12 +491,33 @@ static kvd_status decode_q8(const void *q, const uint8_t *k_codes, const uint8_t
                             const int32_t *seq_lens, float scale, void *out, int B, int H_q, int H_kv,
                             int d, int num_blocks, int max_blocks_per_seq, int num_partitions,
                             void *workspace, size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
-                            void *stream, kvd::Code8 fmt) {
+                            void *stream, kvd::Code8 fmt, const void *k_new = nullptr,
+                            const void *v_new = nullptr) {
   if (!k_scale) return fail(KVD_ERR_INVALID, "k_scale is NULL");
   return decode_impl(q, k_codes, v_codes, block_table, seq_lens, scale, out, B, H_q, H_kv, d,
                      num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
-                     lse_out, dtype, stream, nullptr, nullptr, nullptr, nullptr, 0, 0, k_scale,
+                     lse_out, dtype, stream, k_new, v_new, nullptr, nullptr, 0, 0, k_scale,
                      v_scale, fmt);
+}
+
+// The fused step over an 8-bit cache: kvd_append_{fp8,int8} (slot =
+// seq_lens - 1) and kvd_decode_attention_{fp8,int8} in one decode launch.
+static kvd_status step_q8(const void *q, const void *k_new, const void *v_new, uint8_t *k_codes,
+                          uint8_t *v_codes, float *k_scale, float *v_scale,
+                          const int32_t *block_table, const int32_t *seq_lens, float scale,
+                          void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                          int max_blocks_per_seq, int num_partitions, void *workspace,
+                          size_t workspace_bytes, float *lse_out, kvd_dtype dtype, void *stream,
+                          kvd::Code8 fmt) {
+  if (B > 0) {
+    if (!k_new || !v_new) return fail(KVD_ERR_INVALID, "k_new / v_new is NULL");
+    if (!aligned(k_new, 16) || !aligned(v_new, 16))
+      return fail(KVD_ERR_INVALID, "k_new / v_new must be 16-byte aligned");
+  }
+  return decode_q8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out, B, H_q,
+                   H_kv, d, num_blocks, max_blocks_per_seq, num_partitions, workspace,
+                   workspace_bytes, lse_out, dtype, stream, fmt, B > 0 ? k_new : nullptr,
+                   B > 0 ? v_new : nullptr);
 }
 
 kvd_status kvd_quantize_fp8(const void *src, uint8_t *codes, float *scales, long long n_rows,
@@ -521,6 +543,18 @@ kvd_status kvd_decode_attention_fp8(const void *q, const uint8_t *k_codes, const
   return decode_q8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out, B, H_q,
                    H_kv, d, num_blocks, max_blocks_per_seq, num_partitions, workspace,
                    workspace_bytes, lse_out, dtype, stream, kvd::Code8::E4M3);
+}
+
+kvd_status kvd_decode_step_fp8(const void *q, const void *k_new, const void *v_new,
+                               uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
+                               const int32_t *block_table, const int32_t *seq_lens, float scale,
+                               void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                               int max_blocks_per_seq, int num_partitions, void *workspace,
+                               size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+                               void *stream) {
+  return step_q8(q, k_new, v_new, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale,
+                 out, B, H_q, H_kv, d, num_blocks, max_blocks_per_seq, num_partitions, workspace,
+                 workspace_bytes, lse_out, dtype, stream, kvd::Code8::E4M3);
 }
 
 kvd_status kvd_quantize_int8(const void *src, int8_t *codes, float *scales, long long n_rows,
@@ -550,6 +584,19 @@ kvd_status kvd_decode_attention_int8(const void *q, const int8_t *k_codes, const
                    seq_lens, scale, out, B, H_q, H_kv, d, num_blocks, max_blocks_per_seq,
                    num_partitions, workspace, workspace_bytes, lse_out, dtype, stream,
                    kvd::Code8::INT8);
+}
+
+kvd_status kvd_decode_step_int8(const void *q, const void *k_new, const void *v_new,
+                                int8_t *k_codes, int8_t *v_codes, float *k_scale, float *v_scale,
+                                const int32_t *block_table, const int32_t *seq_lens, float scale,
+                                void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                                int max_blocks_per_seq, int num_partitions, void *workspace,
+                                size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+                                void *stream) {
+  return step_q8(q, k_new, v_new, reinterpret_cast<uint8_t *>(k_codes),
+                 reinterpret_cast<uint8_t *>(v_codes), k_scale, v_scale, block_table, seq_lens,
+                 scale, out, B, H_q, H_kv, d, num_blocks, max_blocks_per_seq, num_partitions,
+                 workspace, workspace_bytes, lse_out, dtype, stream, kvd::Code8::INT8);
 }
 
 size_t kvd_shared_prefix_workspace_size(int B, int H_q, int H_kv, int d, int n_groups,

@@ -43,6 +43,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "quant.cuh"
 #include "tile.cuh"
 
 namespace kvd {
@@ -78,7 +79,6 @@ struct Geo {
 template <int D, int NT, typename T>
 struct Page16 {
   using Out = T;
-  static constexpr bool kPatchable = true;  // supports the fused append
   static constexpr int kPageBytes = kPage * D * 2;
   static constexpr int kCopyBytes = 2 * kPageBytes;
   static constexpr int kStride = kCopyBytes;
@@ -99,6 +99,20 @@ struct Page16 {
     for (int hf = 0; hf < D / 64; ++hf) {
       uint4 *z = reinterpret_cast<uint4 *>(st + kPageBytes + hf * kPage * 128 + ntok * 128);
       for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  // fused append: put the new token of pair (b, h) into row t of the staged
+  // page and write it to the cache at pool row `row` + t
+  static __device__ __forceinline__ void patch(uint8_t *st, uint8_t *, int t, int lane,
+                                               const DecodeArgs &a, int b, int h, int row) {
+    const int half = lane >> 4, ch = lane & 15;
+    if (ch < D / 8) {
+      const size_t src = (static_cast<size_t>(b) * a.H_kv + h) * D;
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
+                                static_cast<const uint16_t *>(half ? a.v_new : a.k_new) + src) + ch);
+      *reinterpret_cast<uint4 *>(st + (half ? kPageBytes : 0) + swz<D>(t, ch * 8)) = v;
+      const size_t dst = (static_cast<size_t>(row) + t) * D;
+      *(reinterpret_cast<uint4 *>(static_cast<uint16_t *>(half ? a.v_cache : a.k_cache) + dst) + ch) = v;
     }
   }
   static __device__ __forceinline__ void tile(uint8_t *st, uint8_t *, int ntok, float sl2, int lane,
@@ -123,7 +137,6 @@ struct Page16 {
 template <int NT, typename T, Code8 kFmt>
 struct Page8 {
   using Out = T;
-  static constexpr bool kPatchable = false;
   static constexpr int kPageBytes = kPage * 128;             // codes of K (or V)
   static constexpr int kScaleBytes = kPage * 4 * 4;          // scales of K (or V)
   static constexpr int kCopyBytes = 2 * kPageBytes + 2 * kScaleBytes;
@@ -146,6 +159,27 @@ struct Page8 {
     for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
     uint4 *zs = reinterpret_cast<uint4 *>(aux + kScaleBytes + ntok * 16);
     for (int i = lane; i < kPage - ntok; i += 32) zs[i] = make_uint4(0, 0, 0, 0);
+  }
+  // fused append: encode the new token of pair (b, h) exactly as the
+  // quantising append does (encode_row4), put its codes and scales into row t
+  // of the staged page and write them to the pools at row `row` + t
+  static __device__ __forceinline__ void patch(uint8_t *st, uint8_t *aux, int t, int lane,
+                                               const DecodeArgs &a, int b, int h, int row) {
+    const size_t src = (static_cast<size_t>(b) * a.H_kv + h) * 128;
+    const size_t dst = static_cast<size_t>(row) + t;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float sc;
+      const uint32_t w =
+          encode_row4<T, kFmt>(static_cast<const T *>(half ? a.v_new : a.k_new) + src, true, lane, sc);
+      *reinterpret_cast<uint32_t *>(st + half * kPageBytes + swz8(t, lane >> 2) + (lane & 3) * 4) = w;
+      *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(half ? a.v_cache : a.k_cache) + dst * 128 +
+                                    lane * 4) = w;
+      if ((lane & 7) == 0) {
+        reinterpret_cast<float *>(aux + half * kScaleBytes)[t * 4 + (lane >> 3)] = sc;
+        (half ? a.v_scale : a.k_scale)[dst * 4 + (lane >> 3)] = sc;
+      }
+    }
   }
   static __device__ __forceinline__ void tile(uint8_t *st, uint8_t *aux, int ntok, float sl2, int lane,
                                               const uint32_t (&qf)[NT][8][2],
@@ -546,26 +580,13 @@ __global__ void __launch_bounds__(32 * W, 1)
       if (ntok > 0) {
         uint8_t *kp = stages + ((size_t)warp * S + cst) * Gm::kStageBytes;
         uint8_t *ap = aux + ((size_t)warp * S + cst) * Gm::kAuxBytes;
-        if constexpr (Pol::kPatchable) {
-        uint8_t *vp = kp + Pol::kPageBytes;
         if (md.y & kPatch) {
-          // fused append: the new token is row ntok - 1 of this page.  Put
-          // k_new / v_new into the staged page (the copy just read may
-          // predate it) and write them to the cache -- no other CTA reads
-          // this row in this launch.
-          const int b = cur / H, h = cur - (cur / H) * H;
-          const int half = lane >> 4, ch = lane & 15;
-          if (ch < D / 8) {
-            const size_t src = (static_cast<size_t>(b) * H + h) * D;
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
-                                      static_cast<const uint16_t *>(half ? a.v_new : a.k_new) + src) + ch);
-            *reinterpret_cast<uint4 *>((half ? vp : kp) + swz<D>(ntok - 1, ch * 8)) = v;
-            const size_t dst = (static_cast<size_t>(md.z) + (ntok - 1)) * D;
-            *(reinterpret_cast<uint4 *>(static_cast<uint16_t *>(half ? a.v_cache : a.k_cache) + dst) + ch) = v;
-          }
+          // fused append: the new token is row ntok - 1 of this page.  Put it
+          // into the staged page (the copy just read may predate it) and
+          // write it to the cache -- no other CTA reads this row in this launch.
+          Pol::patch(kp, ap, ntok - 1, lane, a, cur / H, cur - (cur / H) * H, md.z);
           fence_proxy_async_smem();
           __syncwarp();
-        }
         }
         if (ntok < kPage) {
           // rows past the sequence end may hold anything (even NaN): clear V's

@@ -54,8 +54,9 @@ struct DecodeArgs {
   const float *pre_lse;
   int pre_chunks;
   // 8-bit cache (null for 16-bit pages): fp32 scales [num_blocks][H_kv][16][d/32]
-  const float *k_scale;
-  const float *v_scale;
+  // (k_cache / v_cache are then the code pools); written only by the fused append
+  float *k_scale;
+  float *v_scale;
 };
 
 // Quantise rows of d fp16/bf16 words into E4M3 codes + fp32 per-32-channel

@@ -13,21 +13,18 @@
 // Both divisions are IEEE fp32 (__fdiv_rn), so the codes are the same on
 // every run and every machine.  A group of zeros gets s = 0.
 //
-// One warp per row: lane l holds channels 4l..4l+3, a group is 8 lanes and
-// its maximum is three shuffles.  In append mode the source rows are the
-// step's k_new and v_new [B][H_kv][d] (one launch, K rows then V rows) and
-// each goes to row slot % 16 of page block_table[b][slot / 16] of its code
-// and scale pools.
-#include <cuda_fp8.h>
-
+// One warp per row (encode_row4, shared with the decode kernel's fused
+// append).  In append mode the source rows are the step's k_new and v_new
+// [B][H_kv][d] (one launch, K rows then V rows) and each goes to row
+// slot % 16 of page block_table[b][slot / 16] of its code and scale pools.
 #include "common.cuh"
 #include "kernels.h"
+#include "quant.cuh"
 
 namespace kvd {
 
 template <typename T, Code8 kFmt>
 __global__ void __launch_bounds__(256) quantize_q8_kernel(const QuantArgs a) {
-  constexpr float kMax = kFmt == Code8::E4M3 ? 448.0f : 127.0f;
   // programmatic dependent launch: wait for the preceding grid's writes
   grid_dependency_wait();
   grid_launch_dependents();
@@ -56,37 +53,11 @@ __global__ void __launch_bounds__(256) quantize_q8_kernel(const QuantArgs a) {
     dst = (static_cast<long long>(pb) * a.H_kv + h) * kPage + pos % kPage;
   }
   const bool live = lane * 4 < a.d;
-  float x[4] = {0.f, 0.f, 0.f, 0.f};
-  if (live) {
-    const uint2 w = *reinterpret_cast<const uint2 *>(static_cast<const T *>(src) + r * a.d + lane * 4);
-    const T *v = reinterpret_cast<const T *>(&w);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = static_cast<float>(v[i]);
-  }
-  float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-  const float s = __fdiv_rn(mx, kMax);
-  float q[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) q[i] = s == 0.0f ? 0.0f : __fdiv_rn(x[i], s);
+  float sc;
+  const uint32_t word = encode_row4<T, kFmt>(static_cast<const T *>(src) + r * a.d, live, lane, sc);
   if (!live) return;
-  uint32_t word;
-  if constexpr (kFmt == Code8::E4M3) {
-    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(q[0], q[1]), __NV_SATFINITE, __NV_E4M3);
-    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(q[2], q[3]), __NV_SATFINITE, __NV_E4M3);
-    word = (lo & 0xffffu) | (hi << 16);
-  } else {
-    word = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float r = q[i] != q[i] ? 0.f : fminf(fmaxf(rintf(q[i]), -127.f), 127.f);
-      word |= (static_cast<uint32_t>(static_cast<int>(r)) & 0xffu) << (8 * i);
-    }
-  }
   *reinterpret_cast<uint32_t *>(codes + dst * a.d + lane * 4) = word;
-  if ((lane & 7) == 0) scales[dst * (a.d / 32) + (lane >> 3)] = s;
+  if ((lane & 7) == 0) scales[dst * (a.d / 32) + (lane >> 3)] = sc;
 }
 
 cudaError_t launch_quantize_q8(const QuantArgs &a, DType dt, Code8 fmt, cudaStream_t s) {

@@ -168,3 +168,99 @@ def test_decode_full_size_gqa70b(kvd, fmt):
     print(f"gqa70b {fmt}: max abs error {worst:.3e} over sequences {rows}")
     assert worst <= TOL[w.dtype]
     assert kvd.kvd_read_device_error() == 0
+
+
+def _bits(t):
+    """A tensor's raw bits (int16 view for 16-bit floats, int32 for fp32), on the host."""
+    t = t.detach().cpu()
+    return t.view(torch.int16) if t.element_size() == 2 else (t.view(torch.int32) if t.element_size() == 4 else t)
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_{c[3]}_N{c[5]}")
+def test_fused_step_matches_oracle_and_two_calls(kvd, fmt, case):
+    # kvd_decode_step_<fmt>: the pools after the call are the oracle's append
+    # (slot = seq_lens - 1) bit for bit, out is within tolerance of the
+    # oracle's attention over them, and both are bit-identical to the
+    # two-call path (append, then attention with the same partitions)
+    B, H_q, H_kv, dtype, lens, parts = case
+    w = build_workload("s8", B, H_q, H_kv, 128, dtype, lens, seed=1400 + CASES.index(case),
+                       spare_pages=2)
+    si = step_inputs(w, 0)
+    k8, v8, ks, vs = q8_state(kvd, w, fmt)
+    two = [t.clone() for t in (k8, v8, ks, vs)]
+    hk8, hv8, hks, hvs = host(k8), host(v8), host(ks), host(vs)
+    bt = w.block_table.cuda()
+    q, kn, vn, sl = si["q"].cuda(), si["k_new"].cuda(), si["v_new"].cuda(), si["seq_lens"].cuda()
+    lse = torch.empty((B, H_q), dtype=torch.float32, device="cuda")
+    out = gpu_fn(kvd, "decode_step", fmt)(q, kn, vn, k8, v8, ks, vs, bt, sl, w.scale,
+                                          num_partitions=parts, lse_out=lse)
+    gpu_fn(kvd, "append", fmt)(*two, bt, si["slot"].cuda(), kn, vn)
+    lse2 = torch.empty_like(lse)
+    out2 = gpu_fn(kvd, "decode_attention", fmt)(q, *two, bt, sl, w.scale, num_partitions=parts,
+                                                lse_out=lse2)
+    torch.cuda.synchronize()
+    orc_fn("append", fmt)(hk8, hv8, hks, hvs, w.block_table.numpy(), si["slot"].numpy(),
+                          to_words(si["k_new"]), to_words(si["v_new"]), odt(w))
+    assert np.array_equal(host(k8), hk8) and np.array_equal(host(v8), hv8)
+    assert np.array_equal(host(ks).view(np.uint32), hks.view(np.uint32))
+    assert np.array_equal(host(vs).view(np.uint32), hvs.view(np.uint32))
+    ref, ref_lse = orc_fn("attend", fmt)(to_words(si["q"]), hk8, hv8, hks, hvs, w.block_table.numpy(),
+                                         si["seq_lens"].numpy(), w.scale, odt(w))
+    err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
+    assert err <= TOL[w.dtype], f"max abs error {err}"
+    fin = np.isfinite(ref_lse)
+    gl = lse.cpu().double().numpy()
+    assert np.array_equal(np.isfinite(gl), fin)
+    assert np.max(np.abs(gl[fin] - ref_lse[fin])) <= LSE_TOL
+    for a, b in zip((k8, v8, ks, vs), two):
+        assert torch.equal(_bits(a), _bits(b))
+    assert torch.equal(_bits(out), _bits(out2)) and torch.equal(_bits(lse), _bits(lse2))
+    assert kvd.kvd_read_device_error() == 0
+
+
+def test_fused_step_full_size_gqa70b(kvd, fmt):
+    # the benchmark's 70B-shape GQA step over the 8-bit cache: pools and out
+    # bit-identical to the two-call path, sampled sequences against the oracle
+    w = named_config("gqa70b", device="cuda", gen_device="cuda")
+    si = step_inputs(w, 0)
+    k8, v8, ks, vs = q8_state(kvd, w, fmt)
+    two = [t.clone() for t in (k8, v8, ks, vs)]
+    bt = w.block_table.cuda()
+    out = gpu_fn(kvd, "decode_step", fmt)(si["q"], si["k_new"], si["v_new"], k8, v8, ks, vs, bt,
+                                          si["seq_lens"], w.scale)
+    gpu_fn(kvd, "append", fmt)(*two, bt, si["slot"], si["k_new"], si["v_new"])
+    out2 = gpu_fn(kvd, "decode_attention", fmt)(si["q"], *two, bt, si["seq_lens"], w.scale)
+    torch.cuda.synchronize()
+    for a, b in zip((k8, v8, ks, vs), two):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+    del two
+    lens = w.seq_lens0.numpy()
+    rows = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 7, 33})
+    hk8, hv8, hks, hvs = host(k8), host(v8), host(ks), host(vs)
+    q = to_words(si["q"])
+    sl = si["seq_lens"].cpu().numpy()
+    btn = w.block_table.numpy()
+    worst = 0.0
+    for b in rows:
+        ref, _ = orc_fn("attend", fmt)(q[b:b + 1], hk8, hv8, hks, hvs, btn[b:b + 1], sl[b:b + 1],
+                                       w.scale, oracle.BF16)
+        worst = max(worst, float(np.max(np.abs(out[b].float().cpu().double().numpy() - ref[0]))))
+    assert worst <= TOL[w.dtype], f"max abs error {worst}"
+    assert kvd.kvd_read_device_error() == 0
+
+
+def test_fused_step_rejects_missing_new_rows(kvd, fmt):
+    w = build_workload("r8", 2, 8, 8, 128, "f16", [5, 9], seed=1499, spare_pages=1)
+    si = step_inputs(w, 0)
+    k8, v8, ks, vs = q8_state(kvd, w, fmt)
+    lib = kvd.lib()
+    ws = kvd.alloc_workspace(2, 8, 8, 128, 0, torch.device("cuda"))
+    out = torch.empty_like(si["q"]).cuda()
+    st = getattr(lib, "kvd_decode_step_" + fmt)(
+        si["q"].cuda().data_ptr(), None, None, k8.data_ptr(), v8.data_ptr(), ks.data_ptr(),
+        vs.data_ptr(), w.block_table.cuda().data_ptr(), si["seq_lens"].cuda().data_ptr(), w.scale,
+        out.data_ptr(), 2, 8, 8, 128, w.num_blocks, w.block_table.shape[1], 0, ws.data_ptr(),
+        ws.numel(), None, kvd.KVD_F16, None)
+    assert st == kvd.KVD_ERR_INVALID
+    assert "k_new" in kvd.kvd_last_error()
