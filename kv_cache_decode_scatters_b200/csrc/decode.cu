@@ -620,68 +620,123 @@ __global__ void __launch_bounds__(32 * W, 1)
     }
   }
 
-  // ---- 4. combine the pieces of pairs that several warps of this CTA hold
+  // ---- 4. combine the pieces of pairs that several warps of this CTA hold.
+  // A job is one such pair.  Its accumulator slots (kSlots per lane) are cut
+  // into `parts` equal ranges of PER slots -- as many as keep every warp busy:
+  // one part when the CTA has many split pairs, down to one slot pair per
+  // part when it has one or two -- and the (job, part) units go round-robin
+  // over the warps.  Each unit folds the pair's pieces in ascending (warp,
+  // slot) order: new row maxima, then rescaled sums of l and of its slots,
+  // the arithmetic and order of one warp folding them all.
   __syncthreads();
   if (failed) return;
-#pragma unroll 1
-  for (int which = 0; which < 2; ++which) {
-    const int seg = edge_id[warp * 2 + which];
-    if (seg < 0) continue;
-    bool owner = true;  // lowest warp holding a piece of seg
-    for (int w2 = 0; w2 < warp; ++w2)
-      if (edge_id[w2 * 2] == seg || edge_id[w2 * 2 + 1] == seg) owner = false;
-    if (!owner) continue;
-    // gather: new maximum per row, then rescaled sums of l and accumulators
+  {
+    constexpr int kRowSlots = Gm::kSteps * 4;  // slots of one n-tile
+    constexpr int kSlots = NT * kRowSlots;
+    static_assert((kSlots & (kSlots - 1)) == 0, "slot count must be a power of two");
+    const int e_id = lane < 2 * W ? edge_id[lane] : -1;  // piece slot w2 * 2 + k -> its pair
+    bool first = e_id >= 0;
+    for (int j = 0; j < 2 * W; ++j) {
+      const int ej = __shfl_sync(0xffffffffu, e_id, j);
+      if (j < lane && ej == e_id) first = false;
+    }
+    const unsigned firsts = __ballot_sync(0xffffffffu, first);  // one bit per job
+    const int jobs = __popc(firsts);
+    int parts = 1;
+    while (parts * 2 * jobs <= W && parts * 2 <= kSlots / 2) parts *= 2;
+
+    auto unit = [&](auto per_c, int u) {
+      constexpr int PER = decltype(per_c)::value;
+      constexpr int kParts = kSlots / PER;
+      const int jj = u / kParts, pp = u - jj * kParts;
+      unsigned fb = firsts;
+      for (int i = 0; i < jj; ++i) fb &= fb - 1;
+      const int seg = __shfl_sync(0xffffffffu, e_id, __ffs(fb) - 1);
+      const unsigned pieces = __ballot_sync(0xffffffffu, e_id == seg);
+      const int sl0 = pp * PER;  // first slot of this unit
+      // n-tile of slot k of the unit (uniform over the unit unless it spans n-tiles)
+      auto nt_of = [&](int k) { return PER > kRowSlots ? k / kRowSlots : sl0 / kRowSlots; };
+      float mr[NT][2], lr[NT][2], av[PER];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        m_run[nt][i] = -INFINITY;
-        l_run[nt][i] = 0.f;
+        for (int i = 0; i < 2; ++i) {
+          mr[nt][i] = -INFINITY;
+          lr[nt][i] = 0.f;
+        }
+#pragma unroll
+      for (int k = 0; k < PER; ++k) av[k] = 0.f;
+      for (unsigned pc = pieces; pc; pc &= pc - 1) {
+        const float *ml = edge_ml + (__ffs(pc) - 1) * 2 * kRows;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 2; ++i) mr[nt][i] = fmaxf(mr[nt][i], ml[nt * 8 + 2 * tig + i]);
       }
+      for (unsigned pc = pieces; pc; pc &= pc - 1) {
+        const int idx = __ffs(pc) - 1, w2 = idx >> 1;
+        const float *ml = edge_ml + idx * 2 * kRows;
+        const float *src = ((idx & 1) == 0 ? edge_acc + (size_t)w2 * Gm::kEdgeFloats
+                                           : reinterpret_cast<const float *>(
+                                                 stages + (size_t)w2 * S * Gm::kStageBytes)) +
+                           sl0 * 32 + lane;
+        float sc[NT][2];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int mt = 0; mt < Gm::kSteps; ++mt)
+          for (int i = 0; i < 2; ++i) {
+            const int r = nt * 8 + 2 * tig + i;
+            const float mi = ml[r];
+            sc[nt][i] = mi == -INFINITY ? 0.f : fast_exp2(mi - mr[nt][i]);
+            lr[nt][i] += ml[kRows + r] * sc[nt][i];
+          }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
-    for (int w2 = warp; w2 < W; ++w2)
-      for (int k = 0; k < 2; ++k)
-        if (edge_id[w2 * 2 + k] == seg) {
-          const float *ml = edge_ml + (w2 * 2 + k) * 2 * kRows;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 2; ++i) m_run[nt][i] = fmaxf(m_run[nt][i], ml[nt * 8 + 2 * tig + i]);
+        for (int k = 0; k < PER; ++k) {
+          const int nt = nt_of(k);
+          const float s_k = NT == 1 || nt == 0 ? sc[0][k & 1] : sc[NT - 1][k & 1];
+          av[k] += src[k * 32] * s_k;
         }
-    for (int w2 = warp; w2 < W; ++w2)
-      for (int k = 0; k < 2; ++k)
-        if (edge_id[w2 * 2 + k] == seg) {
-          const float *ml = edge_ml + (w2 * 2 + k) * 2 * kRows;
-          const float *src = k == 0 ? edge_acc + (size_t)w2 * Gm::kEdgeFloats
-                                    : reinterpret_cast<const float *>(
-                                          stages + (size_t)w2 * S * Gm::kStageBytes);
-          float sc[NT][2];
+      }
+      // write the unit's slots: final rows, or the CTA's partial
+      long long s0, s1;
+      pair_range(seg, s0, s1);
+      const bool whole = s0 >= c0 && s1 <= c1 && !forced_partial(seg);
+      const int b = seg / H, h = seg - (seg / H) * H;
+      const size_t row0 = static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G;
+      const size_t slot = static_cast<size_t>(cta) + seg;
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const int r = nt * 8 + 2 * tig + i;
-              const float mi = ml[r];
-              sc[nt][i] = mi == -INFINITY ? 0.f : fast_exp2(mi - m_run[nt][i]);
-              l_run[nt][i] += ml[kRows + r] * sc[nt][i];
-            }
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int mt = 0; mt < Gm::kSteps; ++mt)
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                acc[nt][mt][e] += src[((nt * Gm::kSteps + mt) * 4 + e) * 32 + lane] * sc[nt][e & 1];
+      for (int k = 0; k < PER; ++k) {
+        const int sl = sl0 + k, nt = nt_of(k), i = k & 1;
+        const int mt = (sl - nt * kRowSlots) >> 2, e = sl & 3;
+        const int r = nt * 8 + 2 * tig + i;
+        if (r >= a.G) continue;
+        const float l = NT == 1 || nt == 0 ? lr[0][i] : lr[NT - 1][i];
+        const float m = NT == 1 || nt == 0 ? mr[0][i] : mr[NT - 1][i];
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const bool lse_slot = g8 == 0 && (sl - nt * kRowSlots) < 2;  // the row's first slot
+        if (whole) {
+          reinterpret_cast<T *>(a.out)[(row0 + r) * D + Pol::dim(mt, e, g8)] = M::from_float(av[k] * inv);
+          if (lse_slot && a.lse_out)
+            a.lse_out[row0 + r] = l > 0.f ? (m + fast_log2(l)) * kLn2 : -INFINITY;
+        } else {
+          a.part_o[(slot * a.G + r) * D + Pol::dim(mt, e, g8)] = av[k] * inv;
+          if (lse_slot) a.part_lse[slot * a.G + r] = l > 0.f ? (m + fast_log2(l)) * kLn2 : -INFINITY;
         }
-    long long s0, s1;
-    pair_range(seg, s0, s1);
-    emit(seg, s0 >= c0 && s1 <= c1 && !forced_partial(seg));
+      }
+    };
+
+    const int units = jobs * parts;
+#pragma unroll 1
+    for (int u = warp; u < units; u += W) {
+      switch (kSlots / parts) {
+        case 2: unit(std::integral_constant<int, 2>{}, u); break;
+        case 4: unit(std::integral_constant<int, 4>{}, u); break;
+        case 8: unit(std::integral_constant<int, 8>{}, u); break;
+        case 16: unit(std::integral_constant<int, (kSlots >= 16 ? 16 : 2)>{}, u); break;
+        case 32: unit(std::integral_constant<int, (kSlots >= 32 ? 32 : 2)>{}, u); break;
+        default: unit(std::integral_constant<int, (kSlots >= 64 ? 64 : 2)>{}, u); break;
+      }
+    }
   }
 }
 
