@@ -237,12 +237,12 @@ class OracleSampler:
     UNIT_BYTES = 64 << 20
     MAX_SEQS = 16  # distinct sequences prepared (cycled; bounds host memory)
 
-    def __init__(self, w_name):
+    def __init__(self, w_name, threads=0):
         import oracle
         self.oracle = oracle
         self.name = w_name
         self.spec = config_spec(w_name)
-        self.threads = oracle.max_threads()
+        self.threads = threads if threads > 0 else oracle.max_threads()
         self.cache = {}
         self.next = 0
         self.units = []
@@ -295,10 +295,14 @@ class OracleSampler:
                 f"fp64 oracle, {self.threads} OpenMP threads")
 
 
-def oracle_sample(w_name, budget_s=12.0):
-    """The CPU baseline: the oracle timed for about budget_s seconds.
+ONE_THREAD_WORKLOADS = ("tiny", "long")
+
+
+def oracle_sample(w_name, budget_s=12.0, threads=0):
+    """The CPU baseline: the oracle timed for about budget_s seconds, on all
+    host threads (threads=0) or on `threads`.
     Returns (GB/s, seconds, units, threads, description)."""
-    smp = OracleSampler(w_name)
+    smp = OracleSampler(w_name, threads)
     gbs, spent, done = smp.run(budget_s)
     return gbs, spent, done, smp.threads, smp.describe()
 
@@ -423,19 +427,24 @@ def run_ours(args):
         if ev_b is not None:
             ev_b.record(stream)
 
-    a_bytes = attention_bytes(w, si["seq_lens"])
-    p_bytes = append_bytes(w, si["slot"])
-    kv_tok = w.H_kv * 2 * w.d * 2  # K and V bytes per token of one sequence
-    if f8 is not None:
-        a_bytes = fp8_attention_bytes(w, si["seq_lens"])
-        p_bytes = int((si["slot"] >= 0).sum().item()) * w.H_kv * 2 * (w.d * 2 + w.d + (w.d // 32) * 4)
-        kv_tok = w.H_kv * 2 * (w.d + (w.d // 32) * 4)
-    # with shared prefixes the HBM bytes count each shared page once per group
-    # (the metric's bytes); the logical bytes (every member's own view) are
-    # reported beside them
-    a_bytes_logical = a_bytes
-    if w.groups:
-        a_bytes -= w.groups * (w.B // w.groups - 1) * w.prefix_tokens * kv_tok
+    def bytes_of(x):
+        """(attention bytes, logical attention bytes, append bytes) of a step.
+        With shared prefixes the HBM bytes count each shared page once per
+        group (the metric's bytes); the logical bytes (every member's own
+        view) are reported beside them."""
+        a_b = attention_bytes(w, x["seq_lens"])
+        p_b = append_bytes(w, x["slot"])
+        kv_tok = w.H_kv * 2 * w.d * 2  # K and V bytes per token of one sequence
+        if f8 is not None:
+            a_b = fp8_attention_bytes(w, x["seq_lens"])
+            p_b = int((x["slot"] >= 0).sum().item()) * w.H_kv * 2 * (w.d * 2 + w.d + (w.d // 32) * 4)
+            kv_tok = w.H_kv * 2 * (w.d + (w.d // 32) * 4)
+        a_logical = a_b
+        if w.groups:
+            a_b -= w.groups * (w.B // w.groups - 1) * w.prefix_tokens * kv_tok
+        return a_b, a_logical, p_b
+
+    a_bytes, a_bytes_logical, p_bytes = bytes_of(si)
     step_bytes = a_bytes + p_bytes
     # bytes of the call the roofline times (events bracket it)
     timed_bytes = a_bytes if args.separate_append else step_bytes
@@ -495,9 +504,61 @@ def run_ours(args):
         sampler.__exit__(None, None, None)
     barrier(dist)
     per = args.graph_steps if graph is not None else 1      # decode steps per timed iteration
+    call_median_us = sorted(a.elapsed_time(b) for a, b in evs)[args.steps // 2] * 1e3 / per
     ms_step, attn_ms, value = aggregate(dist, world, args.steps * per, t_start.elapsed_time(t_end),
                                         sum(a.elapsed_time(b) for a, b in evs) / (args.steps * per),
                                         step_bytes)
+
+    def run_step(x):
+        """One step of the selected mode on the inputs x (q, k_new, v_new,
+        seq_lens and, for the two-call paths, slot)."""
+        if f8 is not None and not args.separate_append:
+            f8["step"](x["q"], x["k_new"], x["v_new"], f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt,
+                       x["seq_lens"], w.scale, out=out, num_partitions=args.partitions, workspace=ws,
+                       stream=stream)
+        elif f8 is not None:
+            f8["append"](f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, x["slot"], x["k_new"], x["v_new"],
+                         stream=stream)
+            f8["decode"](x["q"], f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, x["seq_lens"], w.scale,
+                         out=out, num_partitions=args.partitions, workspace=ws, stream=stream)
+        elif sp is not None:
+            kvd.kvd_decode_attention_shared_prefix(x["q"], kc, vc, bt, x["seq_lens"], sp["start"],
+                                                   sp["pages"], sp["max"], w.scale, out=out,
+                                                   k_new=x["k_new"], v_new=x["v_new"],
+                                                   num_partitions=args.partitions, workspace=ws,
+                                                   stream=stream)
+        elif args.separate_append:
+            kvd.kvd_append(kc, vc, bt, x["slot"], x["k_new"], x["v_new"], stream=stream)
+            kvd.kvd_decode_attention(x["q"], kc, vc, bt, x["seq_lens"], w.scale, out=out,
+                                     num_partitions=args.partitions, workspace=ws, stream=stream)
+        else:
+            kvd.kvd_decode_step(x["q"], x["k_new"], x["v_new"], kc, vc, bt, x["seq_lens"], w.scale,
+                                out=out, num_partitions=args.partitions, workspace=ws, stream=stream)
+
+    # ---- a workload's consecutive steps (continuous batching: every length
+    # grows by one per step), each with its own inputs, back to back
+    multi = None
+    if w.steps > 1 and graph is None:
+        sets = [step_inputs(w, s, device=dev) for s in range(w.steps)]
+        for x in sets:
+            run_step(x)
+        reps = 5
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        m0.record(stream)
+        for _ in range(reps):
+            for x in sets:
+                run_step(x)
+        m1.record(stream)
+        torch.cuda.synchronize()
+        tot_ms = m0.elapsed_time(m1) / reps
+        nb = sum(sum(bytes_of({k: v.cpu() for k, v in x.items()})[::2]) for x in sets)
+        multi = {"steps": w.steps, "total_us": round(tot_ms * 1e3, 2),
+                 "us_per_step": round(tot_ms * 1e3 / w.steps, 2),
+                 "gbs": round(nb / (tot_ms * 1e-3) / 1e9, 2), "repeats": reps,
+                 "how": "the workload's consecutive steps (lengths +1 per step, own inputs), "
+                        "back to back on one stream, CUDA events; mean over the repeats"}
+        del sets
 
     # ---- end to end through the public API with pinned host buffers
     inputs = [("q", q), ("k_new", k_new), ("v_new", v_new), ("seq_lens", seq_lens)]
@@ -513,31 +574,7 @@ def run_ours(args):
     def e2e_step():
         for n in h_in:
             d_in[n].copy_(h_in[n], non_blocking=True)
-        if f8 is not None and not args.separate_append:
-            f8["step"](d_in["q"], d_in["k_new"], d_in["v_new"], f8["k8"], f8["v8"], f8["ks"], f8["vs"],
-                       bt, d_in["seq_lens"], w.scale, out=out, num_partitions=args.partitions,
-                       workspace=ws, stream=stream)
-        elif f8 is not None:
-            f8["append"](f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, d_in["slot"],
-                               d_in["k_new"], d_in["v_new"], stream=stream)
-            f8["decode"](d_in["q"], f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt,
-                                         d_in["seq_lens"], w.scale, out=out,
-                                         num_partitions=args.partitions, workspace=ws,
-                                         stream=stream)
-        elif sp is not None:
-            kvd.kvd_decode_attention_shared_prefix(d_in["q"], kc, vc, bt, d_in["seq_lens"], sp["start"],
-                                                   sp["pages"], sp["max"], w.scale, out=out,
-                                                   k_new=d_in["k_new"], v_new=d_in["v_new"],
-                                                   num_partitions=args.partitions, workspace=ws,
-                                                   stream=stream)
-        elif args.separate_append:
-            kvd.kvd_append(kc, vc, bt, d_in["slot"], d_in["k_new"], d_in["v_new"], stream=stream)
-            kvd.kvd_decode_attention(d_in["q"], kc, vc, bt, d_in["seq_lens"], w.scale, out=out,
-                                     num_partitions=args.partitions, workspace=ws, stream=stream)
-        else:
-            kvd.kvd_decode_step(d_in["q"], d_in["k_new"], d_in["v_new"], kc, vc, bt,
-                                d_in["seq_lens"], w.scale, out=out,
-                                num_partitions=args.partitions, workspace=ws, stream=stream)
+        run_step(d_in)
         h_out.copy_(out, non_blocking=True)
         stream.synchronize()
 
@@ -564,6 +601,10 @@ def run_ours(args):
         gbs, spent, done, threads, desc = oracle_sample(args.workload, budget_s=args.cpu_budget)
         cpu = {"value": round(gbs, 6), "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": desc}
+        if args.workload in ONE_THREAD_WORKLOADS:
+            # the single-thread figure of the smallest and the longest shapes
+            g1, _, _, _, d1 = oracle_sample(args.workload, budget_s=args.cpu_budget / 3, threads=1)
+            cpu["one_thread"] = {"value": round(g1, 6), "unit": "GB/s", "cores": 1, "sample": d1}
     clocks = sampler.summary() if sampler else None
     line = {
         "metric": METRIC,
@@ -600,6 +641,8 @@ def run_ours(args):
         },
         "us_per_step": round(ms_step * 1e3, 2),
         "timed_call_us": round(attn_ms * 1e3, 2),
+        "timed_call_us_median": round(call_median_us, 2),
+        "consecutive_steps": multi,
         "roofline": {
             "bound": "hbm",
             "achieved": round(achieved, 2),
