@@ -1082,11 +1082,13 @@ int decode_auto_parts(int sms) { return sms; }
 #endif
 
 namespace {
-template <int NT, typename T, Code8 kFmt>
-cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
-                             cudaStream_t st, int grid) {
-  constexpr int W = NT == 1 ? KVD_TUNE_W8_1 : KVD_TUNE_W8_2;
-  constexpr int S = NT == 1 ? KVD_TUNE_S8_1 : KVD_TUNE_S8_2;
+// Largest shared memory one CTA may opt into on sm_100 (227 KB); 1 KB of it is
+// left for the kernels' static shared variables.
+constexpr size_t kMaxCtaSmem = 232448;
+
+template <int NT, typename T, Code8 kFmt, int W, int S>
+cudaError_t launch_decode8_ws(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                              cudaStream_t st, int grid) {
   using Pol = Page8<NT, T, kFmt>;
   auto kern = decode_kernel<128, NT, Pol, W, S>;
   const size_t smem = Geo<128, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B);
@@ -1094,6 +1096,23 @@ cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const 
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(32 * W), smem, st, a, tmK, tmV);
+}
+
+// The tuned ring depth, or one stage per warp when the batch's prefix sums
+// (4 bytes per sequence) would push the tuned layout past the CTA limit.
+template <int NT, typename T, Code8 kFmt>
+cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                             cudaStream_t st, int grid) {
+  constexpr int W = NT == 1 ? KVD_TUNE_W8_1 : KVD_TUNE_W8_2;
+  constexpr int S = NT == 1 ? KVD_TUNE_S8_1 : KVD_TUNE_S8_2;
+  using Pol = Page8<NT, T, kFmt>;
+  // one stage must still hold a parked accumulator tile
+  constexpr bool kCanShrink = S > 1 && 8 * NT * 128 * 4 <= Pol::kStride;
+  if constexpr (kCanShrink) {
+    if (Geo<128, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B) + 1024 > kMaxCtaSmem)
+      return launch_decode8_ws<NT, T, kFmt, W, 1>(a, tmK, tmV, st, grid);
+  }
+  return launch_decode8_ws<NT, T, kFmt, W, S>(a, tmK, tmV, st, grid);
 }
 }  // namespace
 

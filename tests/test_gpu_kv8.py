@@ -264,3 +264,31 @@ def test_fused_step_rejects_missing_new_rows(kvd, fmt):
         ws.numel(), None, kvd.KVD_F16, None)
     assert st == kvd.KVD_ERR_INVALID
     assert "k_new" in kvd.kvd_last_error()
+
+
+def test_fused_step_maximum_batch(kvd, fmt):
+    # B = KVD_MAX_BATCH ragged sequences: the per-sequence prefix sums push the
+    # tuned two-stage layout past the CTA's shared memory, so the kernel runs
+    # with one stage per warp; pools and out must still match the oracle
+    B = 4096
+    g = np.random.default_rng(4321)
+    lens = g.integers(0, 81, size=B)
+    lens[::101] = 0
+    w = build_workload("max8", B, 8, 2, 128, "bf16", [int(x) for x in lens], seed=1501, spare_pages=4)
+    si = step_inputs(w, 0)
+    k8, v8, ks, vs = q8_state(kvd, w, fmt)
+    hk8, hv8, hks, hvs = host(k8), host(v8), host(ks), host(vs)
+    bt = w.block_table.cuda()
+    out = gpu_fn(kvd, "decode_step", fmt)(si["q"].cuda(), si["k_new"].cuda(), si["v_new"].cuda(), k8, v8,
+                                          ks, vs, bt, si["seq_lens"].cuda(), w.scale)
+    torch.cuda.synchronize()
+    orc_fn("append", fmt)(hk8, hv8, hks, hvs, w.block_table.numpy(), si["slot"].numpy(),
+                          to_words(si["k_new"]), to_words(si["v_new"]), odt(w))
+    assert np.array_equal(host(k8), hk8) and np.array_equal(host(v8), hv8)
+    assert np.array_equal(host(ks).view(np.uint32), hks.view(np.uint32))
+    assert np.array_equal(host(vs).view(np.uint32), hvs.view(np.uint32))
+    ref, _ = orc_fn("attend", fmt)(to_words(si["q"]), hk8, hv8, hks, hvs, w.block_table.numpy(),
+                                   si["seq_lens"].numpy(), w.scale, odt(w))
+    err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
+    assert err <= TOL[w.dtype], f"max abs error {err}"
+    assert kvd.kvd_read_device_error() == 0

@@ -90,6 +90,23 @@ CASES = [
 ]
 
 
+def test_maximum_batch(kvd):
+    # B = KVD_MAX_BATCH ragged sequences (0..80 tokens, some empty): eight
+    # sequences per prologue thread in the prefix sums, thousands of short
+    # pairs per partition, every partition edge inside a short pair
+    B = 4096
+    g = np.random.default_rng(1234)
+    lens = g.integers(0, 81, size=B)
+    lens[::97] = 0
+    w = build_workload("maxb", B, 8, 2, 128, "f16", [int(x) for x in lens], seed=705, spare_pages=4)
+    si, kc, vc, out, lse, okc, ovc, ref = run_case(kvd, w)
+    assert np.array_equal(to_words(kc), okc) and np.array_equal(to_words(vc), ovc)
+    assert max_err(out, ref) <= TOL[w.dtype]
+    for b in np.flatnonzero(lens == 0):
+        assert torch.all(out[b] == 0)
+    assert kvd.kvd_read_device_error() == 0
+
+
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_d{c[3]}_{c[4]}")
 def test_decode_matches_oracle(kvd, case):
     B, H_q, H_kv, d, dtype, lens = case
