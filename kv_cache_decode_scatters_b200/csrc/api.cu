@@ -39,6 +39,9 @@ constexpr int kMaxDevices = 64;
 // Average pages per partition (CTA) below which the automatic split stops
 // cutting, so each of a CTA's worker warps gets a couple of pages at least.
 constexpr int kAutoMinPages = 32;
+// Launches with at most this many (sequence, KV head) pairs stream K/V with
+// an L2 evict-first hint.
+constexpr long long kEvictFirstPairs = 64;
 
 std::mutex g_mu;
 int g_sms[kMaxDevices];
@@ -373,7 +376,9 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   a.maxb = max_blocks_per_seq;
   a.nparts = N;
   a.min_pages = num_partitions > 0 ? 1 : kAutoMinPages;
-  a.evict_first = 0;
+  // few (sequence, KV head) pairs (long contexts): stream K/V with the
+  // evict-first hint, measured faster there; many pairs keep evict-normal
+  a.evict_first = static_cast<long long>(B) * H_kv <= kEvictFirstPairs ? 1 : 0;
   a.k_new = k_new;
   a.v_new = v_new;
   a.k_cache = const_cast<void *>(k_cache);

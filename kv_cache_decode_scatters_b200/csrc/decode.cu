@@ -369,12 +369,13 @@ __global__ void __launch_bounds__(32 * W, 1)
           } else {
             const size_t slot = static_cast<size_t>(cta) + seg;
             float *o = a.part_o + (slot * a.G + r) * D;
+            const uint64_t keep = l2_policy_evict_last();
 #pragma unroll
             for (int mt = 0; mt < Gm::kSteps; ++mt) {
-              o[Pol::dim(mt, i, g8)] = acc[nt][mt][i] * inv;
-              o[Pol::dim(mt, 2 + i, g8)] = acc[nt][mt][2 + i] * inv;
+              st_keep(o + Pol::dim(mt, i, g8), acc[nt][mt][i] * inv, keep);
+              st_keep(o + Pol::dim(mt, 2 + i, g8), acc[nt][mt][2 + i] * inv, keep);
             }
-            if (g8 == 0) a.part_lse[slot * a.G + r] = lse;
+            if (g8 == 0) st_keep(a.part_lse + slot * a.G + r, lse, keep);
           }
         }
       }
@@ -719,8 +720,10 @@ __global__ void __launch_bounds__(32 * W, 1)
           if (lse_slot && a.lse_out)
             a.lse_out[row0 + r] = l > 0.f ? (m + fast_log2(l)) * kLn2 : -INFINITY;
         } else {
-          a.part_o[(slot * a.G + r) * D + Pol::dim(mt, e, g8)] = av[k] * inv;
-          if (lse_slot) a.part_lse[slot * a.G + r] = l > 0.f ? (m + fast_log2(l)) * kLn2 : -INFINITY;
+          const uint64_t keep = l2_policy_evict_last();
+          st_keep(a.part_o + (slot * a.G + r) * D + Pol::dim(mt, e, g8), av[k] * inv, keep);
+          if (lse_slot)
+            st_keep(a.part_lse + slot * a.G + r, l > 0.f ? (m + fast_log2(l)) * kLn2 : -INFINITY, keep);
         }
       }
     };
