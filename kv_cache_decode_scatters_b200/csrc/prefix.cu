@@ -233,12 +233,13 @@ __global__ void __launch_bounds__(32 * kWarps, 1)
       const float lse = l > 0.f ? (m_run[nt][i] + fast_log2(l)) * kLn2 : -INFINITY;
       const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + b) * a.G + j;
       float *o = a.pre_o + idx * D;
+      const uint64_t keep = l2_policy_evict_last();  // read again by the merge
 #pragma unroll
       for (int mt = 0; mt < kSteps; ++mt) {
-        o[mt * 16 + g8] = acc[nt][mt][i] * inv;
-        o[mt * 16 + 8 + g8] = acc[nt][mt][2 + i] * inv;
+        st_keep(o + mt * 16 + g8, acc[nt][mt][i] * inv, keep);
+        st_keep(o + mt * 16 + 8 + g8, acc[nt][mt][2 + i] * inv, keep);
       }
-      if (g8 == 0) a.pre_lse[idx] = lse;
+      if (g8 == 0) st_keep(a.pre_lse + idx, lse, keep);
     }
   }
 }
@@ -672,6 +673,7 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
       const float lse = l > 0.f ? (m_ref + fast_log2(l)) * kLn2 : -INFINITY;
       const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + b) * a.G + jr;
       float4 *o = reinterpret_cast<float4 *>(a.pre_o + idx * D);
+      const uint64_t keep = l2_policy_evict_last();  // read again by the merge
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
@@ -684,12 +686,12 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
                                                    __uint_as_float(r[i + 2]) * inv,
                                                    __uint_as_float(r[i + 3]) * inv)
                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-            o[c * 8 + i / 4] = v;
+            st_keep4(o + c * 8 + i / 4, v, keep);
           }
         }
         __syncwarp();
       }
-      if (live) a.pre_lse[idx] = lse;
+      if (live) st_keep(a.pre_lse + idx, lse, keep);
     }
   }
 
