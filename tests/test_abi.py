@@ -147,6 +147,76 @@ def test_merge_validation(kw, status):
                            a["out"], a["lse"], a["dt"], a["stream"]) == status
 
 
+# ----------------------------------------------------------- 8-bit caches
+
+def decode8(fmt, step=False, **kw):
+    a = dict(q=DUMMY, kn=DUMMY, vn=DUMMY, k=DUMMY, v=DUMMY, ks=DUMMY, vs=DUMMY, bt=DUMMY, sl=DUMMY,
+             scale=0.125, out=DUMMY, B=2, H_q=8, H_kv=2, d=128, NB=16, maxb=4, parts=4, ws=DUMMY,
+             wsb=1 << 30, lse=NULL, dt=kvd.KVD_BF16, stream=NULL)
+    a.update(kw)
+    tail = (a["k"], a["v"], a["ks"], a["vs"], a["bt"], a["sl"], a["scale"], a["out"], a["B"], a["H_q"],
+            a["H_kv"], a["d"], a["NB"], a["maxb"], a["parts"], a["ws"], a["wsb"], a["lse"], a["dt"],
+            a["stream"])
+    if step:
+        return getattr(L, "kvd_decode_step_" + fmt)(a["q"], a["kn"], a["vn"], *tail)
+    return getattr(L, "kvd_decode_attention_" + fmt)(a["q"], *tail)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("step", [False, True])
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=64), kvd.KVD_ERR_UNSUPPORTED),                 # the 8-bit tile is d = 128 only
+    (dict(ks=NULL), kvd.KVD_ERR_INVALID),
+    (dict(vs=NULL), kvd.KVD_ERR_INVALID),
+    (dict(ks=ctypes.c_void_p(256 + 8)), kvd.KVD_ERR_INVALID),   # scale pools 16-byte aligned
+    (dict(k=MISALIGNED), kvd.KVD_ERR_INVALID),
+    (dict(H_q=34, H_kv=2), kvd.KVD_ERR_UNSUPPORTED),
+    (dict(wsb=16), kvd.KVD_ERR_WORKSPACE),
+])
+def test_decode8_validation(fmt, step, kw, status):
+    assert decode8(fmt, step, **kw) == status
+    assert kvd.kvd_last_error() != ""
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+def test_step8_requires_aligned_new_rows(fmt):
+    assert decode8(fmt, True, kn=NULL) == kvd.KVD_ERR_INVALID
+    assert decode8(fmt, True, vn=MISALIGNED) == kvd.KVD_ERR_INVALID
+    assert decode8(fmt, True, B=0, q=NULL, kn=NULL, vn=NULL, out=NULL, ws=NULL) == kvd.KVD_OK
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=48), kvd.KVD_ERR_UNSUPPORTED),
+    (dict(d=160), kvd.KVD_ERR_UNSUPPORTED),
+    (dict(B=-1), kvd.KVD_ERR_INVALID),
+    (dict(ks=NULL), kvd.KVD_ERR_INVALID),
+    (dict(kn=MISALIGNED), kvd.KVD_ERR_INVALID),
+    (dict(dt=5), kvd.KVD_ERR_INVALID),
+])
+def test_append8_validation(fmt, kw, status):
+    a = dict(k=DUMMY, v=DUMMY, ks=DUMMY, vs=DUMMY, bt=DUMMY, slot=DUMMY, kn=DUMMY, vn=DUMMY, B=2,
+             H_kv=2, d=128, NB=16, maxb=4, dt=kvd.KVD_F16, stream=NULL)
+    a.update(kw)
+    assert getattr(L, "kvd_append_" + fmt)(a["k"], a["v"], a["ks"], a["vs"], a["bt"], a["slot"], a["kn"],
+                                            a["vn"], a["B"], a["H_kv"], a["d"], a["NB"], a["maxb"],
+                                            a["dt"], a["stream"]) == status
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=40), kvd.KVD_ERR_UNSUPPORTED),
+    (dict(n=-1), kvd.KVD_ERR_INVALID),
+    (dict(src=NULL), kvd.KVD_ERR_INVALID),
+    (dict(n=0, src=NULL), kvd.KVD_OK),
+])
+def test_quantize8_validation(fmt, kw, status):
+    a = dict(src=DUMMY, codes=DUMMY, scales=DUMMY, n=4, d=128, dt=kvd.KVD_BF16, stream=NULL)
+    a.update(kw)
+    assert getattr(L, "kvd_quantize_" + fmt)(a["src"], a["codes"], a["scales"], a["n"], a["d"], a["dt"],
+                                              a["stream"]) == status
+
+
 def test_workspace_size_with_explicit_partitions():
     # layout: (B+1) int32 -> 256-byte rounded; slots*G floats -> rounded; slots*G*d floats
     B, H_q, H_kv, d, N = 3, 8, 2, 128, 10
