@@ -217,6 +217,31 @@ def test_quantize8_validation(fmt, kw, status):
                                               a["stream"]) == status
 
 
+# -------------------------------------------------- shared-prefix decode
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(ng=-1), kvd.KVD_ERR_INVALID),
+    (dict(kn=DUMMY, vn=NULL), kvd.KVD_ERR_INVALID),       # both or neither
+    (dict(kn=MISALIGNED, vn=DUMMY), kvd.KVD_ERR_INVALID),
+    (dict(gs=NULL), kvd.KVD_ERR_INVALID),
+    (dict(gp=NULL), kvd.KVD_ERR_INVALID),
+    (dict(mg=0), kvd.KVD_ERR_INVALID),
+    (dict(d=96), kvd.KVD_ERR_UNSUPPORTED),
+    (dict(q=NULL), kvd.KVD_ERR_INVALID),
+])
+def test_shared_prefix_validation(kw, status):
+    a = dict(q=DUMMY, kn=NULL, vn=NULL, k=DUMMY, v=DUMMY, bt=DUMMY, sl=DUMMY, scale=0.125, out=DUMMY,
+             B=4, H_q=8, H_kv=2, d=128, NB=16, maxb=4, gs=DUMMY, gp=DUMMY, ng=2, mg=2, parts=4,
+             ws=DUMMY, wsb=1 << 30, lse=NULL, dt=kvd.KVD_F16, stream=NULL)
+    a.update(kw)
+    st = L.kvd_decode_attention_shared_prefix(
+        a["q"], a["kn"], a["vn"], a["k"], a["v"], a["bt"], a["sl"], a["scale"], a["out"], a["B"],
+        a["H_q"], a["H_kv"], a["d"], a["NB"], a["maxb"], a["gs"], a["gp"], a["ng"], a["mg"], a["parts"],
+        a["ws"], a["wsb"], a["lse"], a["dt"], a["stream"])
+    assert st == status
+    assert kvd.kvd_last_error() != ""
+
+
 def test_workspace_size_with_explicit_partitions():
     # layout: (B+1) int32 -> 256-byte rounded; slots*G floats -> rounded; slots*G*d floats
     B, H_q, H_kv, d, N = 3, 8, 2, 128, 10
