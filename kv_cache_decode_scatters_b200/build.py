@@ -7,6 +7,7 @@
 The library is written next to this file so it travels with the source tree;
 it is rebuilt when any source or the public header is newer than it.
 """
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -53,11 +54,14 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if verbose_ptxas:
         flags += ["-Xptxas", "-v"]
     with tempfile.TemporaryDirectory(dir=HERE, prefix="_build_") as tmp:
-        objs = []
-        for src in sources():
-            obj = os.path.join(tmp, os.path.basename(src) + ".o")
-            subprocess.run([nvcc(), *flags, "-c", src, "-o", obj], check=True)
-            objs.append(obj)
+        objs = [os.path.join(tmp, os.path.basename(src) + ".o") for src in sources()]
+        # the translation units are independent: compile them concurrently
+        jobs = max(1, min(len(objs), os.cpu_count() or 1))
+        with concurrent.futures.ThreadPoolExecutor(jobs) as pool:
+            runs = [pool.submit(subprocess.run, [nvcc(), *flags, "-c", src, "-o", obj], check=True)
+                    for src, obj in zip(sources(), objs)]
+            for r in runs:
+                r.result()  # re-raises a failed compile
         out = os.path.join(tmp, "libkvdecode.so")
         subprocess.run([nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", out, *objs], check=True)
         os.replace(out, LIB)
