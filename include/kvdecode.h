@@ -104,8 +104,10 @@ kvd_status kvd_append(void *k_cache, void *v_cache, const int32_t *block_table,
  *              row (a sequence of length 0 gets zeros)
  *   scale      score multiplier (usually 1/sqrt(d))
  *   num_partitions
- *              0: automatic (one partition per resident worker warp of the
- *              device).  n >= 1: the concatenated page list of all (sequence,
+ *              0: automatic (one partition per streaming multiprocessor of
+ *              the device, each a CTA of worker warps that share its pages
+ *              equally; small problems use fewer).  n >= 1: the concatenated
+ *              page list of all (sequence,
  *              KV head) pairs is cut into n equal contiguous partitions; a
  *              pair that spans several partitions is finished by an LSE merge
  *              launched by this call on the same stream.

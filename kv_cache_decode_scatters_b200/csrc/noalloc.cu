@@ -42,9 +42,15 @@ extern "C" kvd_status kvd_decode_attention_static(
     const int32_t *seq_lens, float scale, void *out, int B, int H_q, int H_kv, int d,
     int num_blocks, int max_blocks_per_seq, float *lse_out, kvd_dtype dtype, void *stream) {
   char msg[256];
-  if (B == 0) return KVD_OK;
   const size_t need = kvd_workspace_size(B, H_q, H_kv, d, 0);
-  if (need == 0) return KVD_ERR_UNSUPPORTED;  // shape rejected; kvd_last_error says why
+  if (need == 0) {
+    // The shape (or the device query) was rejected.  Let the workspace entry
+    // point validate the same call, so both return the same status and the
+    // same kvd_last_error text; it fails before it would need a workspace.
+    return kvd_decode_attention(q, k_cache, v_cache, block_table, seq_lens, scale, out, B, H_q,
+                                H_kv, d, num_blocks, max_blocks_per_seq, 0, nullptr, 0, lse_out,
+                                dtype, stream);
+  }
   if (need > kStaticWorkspaceBytes) {
     snprintf(msg, sizeof msg,
              "kvd_decode_attention_static: this shape needs %zu bytes of scratch, more than the "

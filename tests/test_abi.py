@@ -106,6 +106,44 @@ def test_decode_empty_batch_is_a_no_op():
     assert decode(B=0, q=NULL, out=NULL, ws=NULL) == kvd.KVD_OK
 
 
+def static(**kw):
+    a = dict(q=DUMMY, k=DUMMY, v=DUMMY, bt=DUMMY, sl=DUMMY, scale=0.125, out=DUMMY,
+             B=2, H_q=8, H_kv=2, d=128, NB=16, maxb=4, lse=NULL, dt=kvd.KVD_F16, stream=NULL)
+    a.update(kw)
+    return L.kvd_decode_attention_static(a["q"], a["k"], a["v"], a["bt"], a["sl"], a["scale"],
+                                         a["out"], a["B"], a["H_q"], a["H_kv"], a["d"], a["NB"],
+                                         a["maxb"], a["lse"], a["dt"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), kvd.KVD_ERR_UNSUPPORTED),
+    (dict(H_q=6, H_kv=4), kvd.KVD_ERR_UNSUPPORTED),
+    (dict(B=5000), kvd.KVD_ERR_UNSUPPORTED),
+    (dict(B=-1), kvd.KVD_ERR_INVALID),
+    (dict(H_q=0), kvd.KVD_ERR_INVALID),
+    (dict(dt=7), kvd.KVD_ERR_INVALID),
+    (dict(scale=float("nan")), kvd.KVD_ERR_INVALID),
+    (dict(q=MISALIGNED), kvd.KVD_ERR_INVALID),
+    # an empty batch is still validated
+    (dict(B=0, dt=7), kvd.KVD_ERR_INVALID),
+    (dict(B=0, d=96), kvd.KVD_ERR_UNSUPPORTED),
+    (dict(B=0, H_q=6, H_kv=4), kvd.KVD_ERR_UNSUPPORTED),
+    (dict(B=0, scale=float("nan")), kvd.KVD_ERR_INVALID),
+])
+def test_static_validation_matches_workspace_entry_point(kw, status):
+    # the fixed-scratch entry point rejects a bad call with the status (and
+    # the message) of kvd_decode_attention, before any device work
+    assert static(**kw) == status
+    msg = kvd.kvd_last_error()
+    assert msg != ""
+    assert decode(parts=0, **kw) == status
+    assert kvd.kvd_last_error() == msg
+
+
+def test_static_empty_batch_is_a_no_op():
+    assert static(B=0, q=NULL, out=NULL) == kvd.KVD_OK
+
+
 def append(**kw):
     a = dict(k=DUMMY, v=DUMMY, bt=DUMMY, slot=DUMMY, kn=DUMMY, vn=DUMMY, B=2, H_kv=2, d=128,
              NB=16, maxb=4, dt=kvd.KVD_BF16, stream=NULL)
