@@ -25,6 +25,7 @@ import subprocess
 import sys
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -70,23 +71,30 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def read_only_peak_gbs(nbytes=4 << 30, reps=5):
-    """Best-of-reps read bandwidth of a torch reduction over a large buffer
-    (a read-only reference next to the copy-based peak)."""
-    x = torch.zeros(nbytes // 4, dtype=torch.float32, device="cuda")
-    x.sum()
-    torch.cuda.synchronize()
-    best = float("inf")
-    for _ in range(reps):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        x.sum()
-        b.record()
+def read_only_peak_gbs(kvd, nbytes=4 << 30, reps=5):
+    """Read-only HBM bandwidth of this device, measured by the library's
+    streaming kernels (kvd_read_stream) over a buffer far larger than L2:
+    best of `reps` launches of each form, CUDA events on the launching
+    stream.  Returns {form: GB/s}."""
+    x = torch.ones(nbytes // 4, dtype=torch.int32, device="cuda")
+    sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    res = {}
+    for name, mode in (("vector", kvd.KVD_READ_VECTOR), ("bulk", kvd.KVD_READ_BULK)):
+        kvd.kvd_read_stream(x, mode, sink=sink, stream=stream)
         torch.cuda.synchronize()
-        best = min(best, a.elapsed_time(b))
+        best = float("inf")
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            kvd.kvd_read_stream(x, mode, sink=sink, stream=stream)
+            b.record(stream)
+            torch.cuda.synchronize()
+            best = min(best, a.elapsed_time(b))
+        res[name] = nbytes / (best * 1e-3) / 1e9
     del x
     torch.cuda.empty_cache()
-    return nbytes / (best * 1e-3) / 1e9
+    return res
 
 
 def source_hash() -> str:
@@ -122,6 +130,54 @@ def profile_traffic(workload: str, mode: str):
         if m_src.group(1) == want and m_wl.group(1) == workload and m_mode.group(1) == mode:
             return int(m_b.group(1))
     return None
+
+
+def sample_sequences(w, k, seed):
+    """k seeded random sequences of w plus its longest and its shortest."""
+    g = torch.Generator().manual_seed(seed)
+    pick = set(torch.randperm(w.B, generator=g)[:min(k, w.B)].tolist())
+    pick.add(int(torch.argmax(w.seq_lens0)))
+    pick.add(int(torch.argmin(w.seq_lens0)))
+    return sorted(pick)
+
+
+class RowSnapshot:
+    """Host copy of what a few sequences of a workload read -- their pages
+    (renumbered compactly, storage words) and their step inputs -- taken
+    before any kernel writes the pool.  It is the input of the CPU-baseline
+    leg's oracle run, whose result the GPU's output rows are compared with."""
+
+    def __init__(self, w, si, rows):
+        bt = w.block_table.cpu()
+        n = si["seq_lens"].cpu()
+        npg = [(int(n[b]) + 15) // 16 for b in rows]
+        pages = sorted({int(p) for b, m in zip(rows, npg) for p in bt[b, :m].tolist()})
+        idx = torch.tensor(pages or [0], dtype=torch.long, device=w.k_cache.device)
+        self.k = to_words(w.k_cache.index_select(0, idx)).copy()
+        self.v = to_words(w.v_cache.index_select(0, idx)).copy()
+        remap = {p: i for i, p in enumerate(pages)}
+        self.bt = np.zeros((len(rows), max(npg + [1])), dtype=np.int32)
+        for i, (b, m) in enumerate(zip(rows, npg)):
+            self.bt[i, :m] = [remap[p] for p in bt[b, :m].tolist()]
+        sel = torch.tensor(rows, dtype=torch.long)
+        self.rows = rows
+        self.q = to_words(si["q"].cpu()[sel])
+        self.k_new = to_words(si["k_new"].cpu()[sel])
+        self.v_new = to_words(si["v_new"].cpu()[sel])
+        self.seq_lens = n[sel].numpy().astype(np.int32)
+        self.slot = si["slot"].cpu()[sel].numpy().astype(np.int32)
+        self.scale = w.scale
+        self.bf16 = w.dtype == torch.bfloat16
+        tokens = int(self.seq_lens.astype(np.int64).sum())
+        self.nbytes = (tokens * w.H_kv * 2 * w.d * 2 + 2 * len(rows) * w.H_q * w.d * 2
+                       + int((self.slot >= 0).sum()) * w.H_kv * w.d * 2 * 2 * 2)
+
+    def describe(self, w):
+        return (f"sequences {self.rows} of {w.B} (lengths {self.seq_lens.tolist()}), all "
+                f"{w.H_q} query heads each")
+
+    def describe_short(self):
+        return f"sequences {self.rows} (lengths {self.seq_lens.tolist()}), all query heads"
 
 
 class ClockSampler:
@@ -295,6 +351,32 @@ class OracleSampler:
                 f"fp64 oracle, {self.threads} OpenMP threads")
 
 
+def oracle_parity(snap, gpu_rows, threads=0, fmt=None):
+    """CPU-baseline leg: the oracle's append + attend on a RowSnapshot (for an
+    8-bit cache, after the oracle's own quantisation of the snapshot's pages),
+    timed, and the largest |GPU - oracle| over the snapshot's output rows.
+    gpu_rows: float64 [rows, H_q, d] of the GPU's output for those sequences.
+    Returns (max_abs_err, seconds, GB/s of the oracle, threads)."""
+    import oracle
+    dt = oracle.BF16 if snap.bf16 else oracle.F16
+    threads = threads if threads > 0 else oracle.max_threads()
+    t0 = time.perf_counter()
+    if fmt is None:
+        kc, vc = snap.k.copy(), snap.v.copy()
+        oracle.append(kc, vc, snap.bt, snap.slot, snap.k_new, snap.v_new)
+        ref, _ = oracle.attend(snap.q, kc, vc, snap.bt, snap.seq_lens, snap.scale, dt, nthreads=threads)
+    else:
+        quant = getattr(oracle, "quantize_" + fmt)
+        k8, ks = quant(snap.k, dt)
+        v8, vs = quant(snap.v, dt)
+        getattr(oracle, "append_" + fmt)(k8, v8, ks, vs, snap.bt, snap.slot, snap.k_new, snap.v_new, dt)
+        ref, _ = getattr(oracle, "attend_" + fmt)(snap.q, k8, v8, ks, vs, snap.bt, snap.seq_lens,
+                                                  snap.scale, dt, nthreads=threads)
+    spent = time.perf_counter() - t0
+    err = float(np.max(np.abs(gpu_rows - ref))) if ref.size else 0.0
+    return err, spent, snap.nbytes / spent / 1e9, threads
+
+
 ONE_THREAD_WORKLOADS = ("tiny", "long")
 
 
@@ -343,6 +425,103 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ GPU path
 
+# The workloads reported beside the headline one in a default run (workload,
+# shared-prefix mode): every synthetic configuration of the method's benchmark.
+PER_WORKLOADS = (("tiny", False), ("gqa70b", False), ("long", False), ("cbatch", False),
+                 ("cbatch", True))
+
+
+def measure_workload(kvd, name, shared_prefix, dev, steps, warmup):
+    """Time one workload's decode step through the call the headline uses
+    (kvd_decode_step, or the shared-prefix call with its fused append) with
+    automatic partitions: `warmup` untimed steps, then `steps` calls each
+    bracketed by CUDA events on the launching stream.  Returns (report dict,
+    RowSnapshot of sampled sequences taken before any kernel ran, the GPU's
+    output rows of those sequences as float64)."""
+    w = named_config(name, device="cuda", gen_device="cuda")
+    si = step_inputs(w, 0)
+    snap = RowSnapshot(w, si, sample_sequences(w, 3, 77))
+    kc, vc, bt = w.k_cache, w.v_cache, w.block_table.to(dev)
+    q, k_new, v_new, seq_lens = si["q"], si["k_new"], si["v_new"], si["seq_lens"].to(dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    sp = None
+    if shared_prefix:
+        per = w.B // w.groups
+        sp = {"start": torch.arange(0, w.B + 1, per, dtype=torch.int32, device=dev),
+              "pages": torch.full((w.groups,), w.prefix_tokens // 16, dtype=torch.int32, device=dev),
+              "max": per}
+        n = kvd.kvd_shared_prefix_workspace_size(w.B, w.H_q, w.H_kv, w.d, w.groups, per, 0)
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    else:
+        ws = kvd.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, 0, dev)
+
+    def call(x_q, x_k, x_v, x_len):
+        if sp is not None:
+            kvd.kvd_decode_attention_shared_prefix(x_q, kc, vc, bt, x_len, sp["start"], sp["pages"],
+                                                   sp["max"], w.scale, out=out, k_new=x_k, v_new=x_v,
+                                                   workspace=ws, stream=stream)
+        else:
+            kvd.kvd_decode_step(x_q, x_k, x_v, kc, vc, bt, x_len, w.scale, out=out, workspace=ws,
+                                stream=stream)
+
+    for _ in range(warmup):
+        call(q, k_new, v_new, seq_lens)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for a, b in evs:
+        a.record(stream)
+        call(q, k_new, v_new, seq_lens)
+        b.record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    flags = kvd.kvd_read_device_error()
+    gpu_rows = out[snap.rows].float().cpu().double().numpy()
+    times = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)
+    call_us = sum(times) / len(times)
+    step_us = t0.elapsed_time(t1) * 1e3 / steps
+
+    a_b = attention_bytes(w, si["seq_lens"].cpu())
+    a_logical = a_b
+    if sp is not None:
+        a_b -= w.groups * (w.B // w.groups - 1) * w.prefix_tokens * w.H_kv * 2 * w.d * 2
+    nbytes = a_b + append_bytes(w, si["slot"].cpu())
+    rep = {
+        "workload": name + (" --shared-prefix" if shared_prefix else ""),
+        "call": ("kvd_decode_attention_shared_prefix (fused append)" if sp is not None
+                 else "kvd_decode_step"),
+        "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "kv_dtype": w.dtype_name,
+        "seq_lens": _lens_desc(w), "steps": steps, "warmup": warmup,
+        "bytes_per_step": nbytes,
+        "us_per_step": round(step_us, 2),
+        "timed_call_us": round(call_us, 2),
+        "timed_call_us_median": round(times[len(times) // 2], 2),
+        "gbs": round(nbytes / (call_us * 1e-6) / 1e9, 2),
+        "device_error_flags": flags,
+    }
+    if sp is not None:
+        rep["logical_attention_bytes"] = a_logical
+    if w.steps > 1:
+        # the workload's consecutive steps, each with its own inputs (lengths
+        # +1 per step), back to back; one warm pass, then one timed pass
+        sets = [step_inputs(w, i, device=dev) for i in range(w.steps)]
+        for x in sets:
+            call(x["q"], x["k_new"], x["v_new"], x["seq_lens"])
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for x in sets:
+            call(x["q"], x["k_new"], x["v_new"], x["seq_lens"])
+        c1.record(stream)
+        torch.cuda.synchronize()
+        rep["consecutive_steps"] = {"steps": w.steps,
+                                    "us_per_step": round(c0.elapsed_time(c1) * 1e3 / w.steps, 2)}
+        del sets
+    return rep, snap, gpu_rows
+
+
 def run_ours(args):
     import kv_cache_decode_scatters_b200 as kvd
 
@@ -356,6 +535,10 @@ def run_ours(args):
     w = named_config(args.workload, device="cuda", gen_device="cuda", scale_down=args.scale_down,
                      shard=rank)
     si = step_inputs(w, 0)
+    # the parity sample: host copy of a few sequences' pages before any kernel runs
+    snap = None
+    if world == 1 and not args.no_cpu_baseline and not args.graph:
+        snap = RowSnapshot(w, si, sample_sequences(w, 3, 77))
     kc, vc, bt = w.k_cache, w.v_cache, w.block_table.to(dev)
     q, k_new, v_new = si["q"], si["k_new"], si["v_new"]
     slot, seq_lens = si["slot"].to(dev), si["seq_lens"].to(dev)
@@ -503,6 +686,7 @@ def run_ours(args):
     if sampler:
         sampler.__exit__(None, None, None)
     barrier(dist)
+    head_rows = out[snap.rows].float().cpu().double().numpy() if snap is not None else None
     per = args.graph_steps if graph is not None else 1      # decode steps per timed iteration
     call_median_us = sorted(a.elapsed_time(b) for a, b in evs)[args.steps // 2] * 1e3 / per
     ms_step, attn_ms, value = aggregate(dist, world, args.steps * per, t_start.elapsed_time(t_end),
@@ -593,9 +777,19 @@ def run_ours(args):
             dist.destroy_process_group()
         return 0
 
+    # ---- every other configuration of the benchmark, through the same call
+    per_wl = []
+    default_run = (args.workload == "mha7b" and f8 is None and sp is None and not args.separate_append
+                   and graph is None and args.scale_down == 1)
+    if world == 1 and (args.per_workload == "on" or (args.per_workload == "auto" and default_run)):
+        for name, shared in PER_WORKLOADS:
+            per_wl.append(measure_workload(kvd, name, shared, dev, args.per_workload_steps, 5))
+            torch.cuda.empty_cache()
+
     peak, peak_kind = peaks()
     achieved = timed_bytes / (attn_ms * 1e-3) / 1e9
-    read_peak = read_only_peak_gbs()
+    read_peaks = read_only_peak_gbs(kvd)
+    read_peak = max(read_peaks.values())
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         gbs, spent, done, threads, desc = oracle_sample(args.workload, budget_s=args.cpu_budget)
@@ -605,6 +799,28 @@ def run_ours(args):
             # the single-thread figure of the smallest and the longest shapes
             g1, _, _, _, d1 = oracle_sample(args.workload, budget_s=args.cpu_budget / 3, threads=1)
             cpu["one_thread"] = {"value": round(g1, 6), "unit": "GB/s", "cores": 1, "sample": d1}
+    # ---- parity of the timed call against the oracle (CPU-baseline leg)
+    tol = 1e-2 if w.dtype == torch.bfloat16 else 2e-3
+    parity = None
+    if snap is not None:
+        err, spent, ogbs, othr = oracle_parity(snap, head_rows, fmt=f8["fmt"] if f8 else None)
+        parity = {"max_abs_err": err, "tol": tol, "ok": err <= tol, "sample": snap.describe(w),
+                  "against": "fp64 oracle" + (" over the oracle's own %s quantisation" % f8["name"]
+                                               if f8 else "")}
+    per_report = []
+    for rep, psnap, prows in per_wl:
+        ptol = 1e-2 if psnap.bf16 else 2e-3
+        perr, pspent, pgbs, pthr = oracle_parity(psnap, prows)
+        ach = rep["bytes_per_step"] / (rep["timed_call_us"] * 1e-6) / 1e9
+        rep["roofline"] = {"achieved": round(ach, 2), "frac": round(ach / peak, 4),
+                           "frac_of_read_only_peak": round(ach / read_peak, 4)}
+        rep["max_abs_err"] = perr
+        rep["tol"] = ptol
+        rep["parity_ok"] = perr <= ptol
+        rep["parity_sample"] = psnap.describe_short()
+        rep["cpu_baseline"] = {"value": round(pgbs, 4), "unit": "GB/s", "cores": pthr, "kind": "oracle",
+                               "sample": "append + attend of the parity sample, one run"}
+        per_report.append(rep)
     clocks = sampler.summary() if sampler else None
     line = {
         "metric": METRIC,
@@ -676,7 +892,12 @@ def run_ours(args):
                           if w.groups else None),
         "read_only_peak": {"value": round(read_peak, 1), "unit": "GB/s",
                            "frac": round(achieved / read_peak, 4),
-                           "how": "torch sum over 4 GiB float32, best of 5, this run"},
+                           "forms": {k: round(v, 1) for k, v in read_peaks.items()},
+                           "how": "kvd_read_stream over 4 GiB (vector: 16-byte loads; bulk: the decode "
+                                  "kernel's 16-warp bulk-copy pipeline with no arithmetic), best of 5 "
+                                  "each, CUDA events, this run; value = the faster form"},
+        "parity": parity,
+        "per_workload": per_report or None,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
@@ -727,6 +948,10 @@ def parse_args(argv=None):
     p.add_argument("--ref-budget", type=float, default=90.0,
                    help="seconds of oracle work for the whole reference-arm run")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--per-workload", choices=["auto", "on", "off"], default="auto",
+                   help="also time (and parity-check) every other configuration; auto = only in the "
+                        "default single-GPU run")
+    p.add_argument("--per-workload-steps", type=int, default=50)
     p.add_argument("--scale-down", type=int, default=1,
                    help="shrink batch and lengths by this factor (profiling small cases only)")
     args = p.parse_args(argv)

@@ -332,6 +332,31 @@ kvd_status kvd_merge_lse(const float *part_o, const float *part_lse,
                          void *out, float *lse_out, kvd_dtype dtype, void *stream);
 
 /*
+ * kvd_read_stream -- read `bytes` of device memory once and fold them into a
+ * checksum: the read-only HBM bandwidth ceiling of this device, measured with
+ * the memory pipelines the decode kernel uses.  Not a step of the method: the
+ * pages only state that decode attention is bound by memory traffic
+ * ([LES] section "问题所在"), and this call measures the bandwidth that bounds
+ * it, next to the copy (read + write) bandwidth.
+ *
+ *   src    device, 16-byte aligned, `bytes` readable bytes
+ *   bytes  a multiple of 16 (0 is a no-op)
+ *   mode   KVD_READ_VECTOR: every thread keeps eight 16-byte loads in flight
+ *          over a grid of 4 CTAs per SM;
+ *          KVD_READ_BULK: one CTA per SM of 16 warps, each streaming an equal
+ *          contiguous share in 8 KB bulk copies (cp.async.bulk) into its own
+ *          shared-memory stage, completed on an mbarrier -- the decode
+ *          kernel's pipeline without its arithmetic
+ *   sink   device uint32: XOR of every 32-bit word of the buffer is XORed into
+ *          *sink (zero it first to read the checksum)
+ * Asynchronous on `stream`; time it with events on that stream.  A bulk wait
+ * that runs out sets KVD_DEVERR_TIMEOUT.
+ */
+#define KVD_READ_VECTOR 0
+#define KVD_READ_BULK 1
+kvd_status kvd_read_stream(const void *src, size_t bytes, int mode, uint32_t *sink, void *stream);
+
+/*
  * Bytes of workspace kvd_decode_attention needs for this shape.
  * num_partitions = 0 means the automatic count of the current device (this
  * queries the device; with no usable device it returns 0 and records the
@@ -359,6 +384,24 @@ size_t kvd_kv_bytes_per_token(int layers, int heads, int d_head, int dtype_size)
  * call synchronises the device; it is a diagnostic, not part of a step.
  */
 kvd_status kvd_read_device_error(unsigned int *flags, int clear);
+
+/*
+ * kvd_set_decode_wait_limit -- testing hook for the failure path of the
+ * decode kernel; not for production use.
+ * Each worker warp of the decode kernel waits on a shared-memory barrier for
+ * every page it streams.  Such a wait polls at most 2^22 times; past that the
+ * warp gives up, sets KVD_DEVERR_TIMEOUT, lets every copy it has in flight
+ * land (with the full limit) and leaves the launch, whose output is then
+ * undefined.  This call sets the poll limit of those page waits for every
+ * later decode launch of the process (kvd_decode_attention, kvd_decode_step,
+ * the shared-prefix call's decode pass and the 8-bit calls): 0 makes every
+ * first wait give up at once, a negative value restores the default.  The
+ * waits that drain copies in flight always keep the full limit, so a lowered
+ * limit ends the launch early and never leaves a copy behind.  Always returns
+ * KVD_OK.  (No page of the method corresponds: it exists so that tests can
+ * reach the timeout path without a copy that never lands.)
+ */
+kvd_status kvd_set_decode_wait_limit(long long polls);
 
 /* Text of the last error recorded by a call on this host thread ("" if none). */
 const char *kvd_last_error(void);

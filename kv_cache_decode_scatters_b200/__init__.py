@@ -35,6 +35,7 @@ KVD_F16, KVD_BF16 = 0, 1
 KVD_PAGE_TOKENS = 16
 KVD_STATIC_WORKSPACE_BYTES = 8 << 20
 KVD_DEVERR_BLOCK_TABLE, KVD_DEVERR_SEQ_LEN, KVD_DEVERR_SLOT, KVD_DEVERR_TIMEOUT = 1, 2, 4, 8
+KVD_READ_VECTOR, KVD_READ_BULK = 0, 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -87,6 +88,10 @@ def _load():
     L.kvd_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint), I]
     L.kvd_last_error.restype = ctypes.c_char_p
     L.kvd_last_error.argtypes = []
+    L.kvd_read_stream.restype = I
+    L.kvd_read_stream.argtypes = [P, S, I, P, P]
+    L.kvd_set_decode_wait_limit.restype = I
+    L.kvd_set_decode_wait_limit.argtypes = [LL]
     return L
 
 
@@ -444,3 +449,23 @@ def kvd_read_device_error(clear: bool = True) -> int:
     _check(_lib.kvd_read_device_error(ctypes.byref(flags), 1 if clear else 0),
            "kvd_read_device_error")
     return int(flags.value)
+
+
+def kvd_set_decode_wait_limit(polls: int) -> None:
+    """Testing hook: poll limit of the decode kernel's page waits for later
+    launches (0 = give up at once and flag KVD_DEVERR_TIMEOUT; negative =
+    the default).  Copies in flight are always drained with the full limit."""
+    _check(_lib.kvd_set_decode_wait_limit(int(polls)), "kvd_set_decode_wait_limit")
+
+
+def kvd_read_stream(buf: torch.Tensor, mode: int = KVD_READ_BULK, sink=None, stream=None):
+    """Read every byte of the contiguous device tensor `buf` once (mode
+    KVD_READ_VECTOR or KVD_READ_BULK), XOR-folding its 32-bit words into
+    `sink` (a 1-element int32 device tensor, zeroed here if not given).
+    Returns sink."""
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int32, device=buf.device)
+    nbytes = buf.numel() * buf.element_size()
+    _check(_lib.kvd_read_stream(_dev(buf, "buf"), nbytes, int(mode), _dev(sink, "sink", torch.int32),
+                                _stream(stream)), "kvd_read_stream")
+    return sink

@@ -4,6 +4,7 @@
 // kvd_read_device_error.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -42,6 +43,10 @@ constexpr int kAutoMinPages = 32;
 // Launches with at most this many (sequence, KV head) pairs stream K/V with
 // an L2 evict-first hint.
 constexpr long long kEvictFirstPairs = 64;
+
+// Poll limit of the decode kernel's streaming waits; negative = kWaitPolls.
+// Lowered only through kvd_set_decode_wait_limit (a test hook).
+std::atomic<long long> g_wait_polls{-1};
 
 std::mutex g_mu;
 int g_sms[kMaxDevices];
@@ -188,6 +193,11 @@ void record_error(const char *msg) { g_last_error = msg; }
 extern "C" {
 
 const char *kvd_last_error(void) { return g_last_error.c_str(); }
+
+kvd_status kvd_set_decode_wait_limit(long long polls) {
+  g_wait_polls.store(polls < 0 ? -1 : polls, std::memory_order_relaxed);
+  return KVD_OK;
+}
 
 size_t kvd_kv_bytes_per_token(int layers, int heads, int d_head, int dtype_size) {
   if (layers < 0 || heads < 0 || d_head < 0 || dtype_size < 0) return 0;
@@ -379,6 +389,10 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   // few (sequence, KV head) pairs (long contexts): stream K/V with the
   // evict-first hint, measured faster there; many pairs keep evict-normal
   a.evict_first = static_cast<long long>(B) * H_kv <= kEvictFirstPairs ? 1 : 0;
+  {
+    const long long wp = g_wait_polls.load(std::memory_order_relaxed);
+    a.wait_polls = wp < 0 || wp > kvd::kWaitPolls ? kvd::kWaitPolls : static_cast<uint32_t>(wp);
+  }
   a.k_new = k_new;
   a.v_new = v_new;
   a.k_cache = const_cast<void *>(k_cache);
@@ -652,6 +666,27 @@ kvd_status kvd_decode_step(const void *q, const void *k_new, const void *v_new, 
   return decode_impl(q, k_cache, v_cache, block_table, seq_lens, scale, out, B, H_q, H_kv, d,
                      num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
                      lse_out, dtype, stream, k_new, v_new);
+}
+
+kvd_status kvd_read_stream(const void *src, size_t bytes, int mode, uint32_t *sink, void *stream) {
+  if (mode != KVD_READ_VECTOR && mode != KVD_READ_BULK)
+    return fail(KVD_ERR_INVALID, "unknown read mode %d", mode);
+  if (bytes % 16) return fail(KVD_ERR_INVALID, "bytes = %zu is not a multiple of 16", bytes);
+  if (bytes == 0) return KVD_OK;
+  if (!src || !sink) return fail(KVD_ERR_INVALID, "a required pointer is NULL");
+  if (!aligned(src, 16) || !aligned(sink, 4)) return fail(KVD_ERR_INVALID, "misaligned buffer");
+  int dev, sms;
+  unsigned *err;
+  kvd_status st = current_device(&dev);
+  if (st) return st;
+  st = sm_count(dev, &sms);
+  if (st) return st;
+  st = error_word(dev, &err);
+  if (st) return st;
+  cudaError_t e = kvd::launch_read_stream(src, bytes, mode, sink, err, sms,
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "read-stream launch");
+  return KVD_OK;
 }
 
 kvd_status kvd_merge_lse(const float *part_o, const float *part_lse,

@@ -565,7 +565,7 @@ __global__ void __launch_bounds__(32 * W, 1)
 #pragma unroll 1
     for (; c < nmy; ++c) {
       const uint32_t bar = bar0 + 8 * cst;
-      const bool ok = mbar_wait_bounded(bar, cph);
+      const bool ok = mbar_wait_bounded(bar, cph, a.wait_polls);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) flag_error(a.err, kErrTimeout);
         failed = true;
@@ -607,7 +607,8 @@ __global__ void __launch_bounds__(32 * W, 1)
     }
 
     if (failed) {
-      // let every copy still in flight land before shared memory is reused or freed
+      // let every copy still in flight land before shared memory is reused or
+      // freed (with the full poll limit, whatever the streaming waits used)
       for (; c < f - p0; ++c) {
         mbar_wait_bounded(bar0 + 8 * cst, cph);
         if (++cst == S) {

@@ -39,6 +39,9 @@ struct DecodeArgs {
   int nparts;         // N: partitions (CTAs) of the concatenated page list
   int min_pages;      // lower bound on average pages per used partition
   int evict_first;    // 1: stream K/V with an L2 evict-first hint
+  // poll limit of each page wait of the streaming loop (kWaitPolls unless a
+  // test lowers it); the waits that drain copies in flight keep kWaitPolls
+  uint32_t wait_polls;
   // fused append (all null for attention only): every sequence with
   // seq_lens[b] >= 1 writes k_new[b], v_new[b] at position seq_lens[b] - 1
   const void *k_new;
@@ -116,6 +119,10 @@ cudaError_t launch_generic_merge(const GenericMergeArgs &a, DType dt, cudaStream
 cudaError_t launch_decode_q8(const DecodeArgs &a, DType dt, Code8 fmt, const CUtensorMap &tmK,
                               const CUtensorMap &tmV, cudaStream_t s, int grid);
 cudaError_t launch_quantize_q8(const QuantArgs &a, DType dt, Code8 fmt, cudaStream_t s);
+// Read-only streaming of `bytes` (a multiple of 16) from src: mode
+// KVD_READ_VECTOR or KVD_READ_BULK; XOR of every 32-bit word into *sink.
+cudaError_t launch_read_stream(const void *src, size_t bytes, int mode, unsigned *sink,
+                               unsigned *err, int sms, cudaStream_t s);
 // Prefix pass of the shared-prefix decode: grid (n_groups * chunks, H_kv, row blocks).
 cudaError_t launch_prefix(const PrefixArgs &a, int d, DType dt, const CUtensorMap &tmK,
                           const CUtensorMap &tmV, int row_blocks, cudaStream_t s);

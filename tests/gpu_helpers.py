@@ -9,6 +9,14 @@ from synth import step_inputs, to_words
 TOL = {torch.float16: 2e-3, torch.bfloat16: 1e-2}   # max-abs error vs the fp64 oracle
 LSE_TOL = 1e-3
 
+# (workload, call, rows checked, max-abs error, lse error, tolerance) of the
+# full-size parity tests; the session prints them (see conftest.py)
+ERROR_REPORT = []
+
+
+def record_error(workload, call, rows, err, lse_err, tol):
+    ERROR_REPORT.append((workload, call, rows, err, lse_err, tol))
+
 
 def odt(w):
     return oracle.BF16 if w.dtype == torch.bfloat16 else oracle.F16
@@ -73,5 +81,5 @@ def words(t):
     return to_words(t)
 
 
-__all__ = ["TOL", "LSE_TOL", "gpu_state", "gpu_step", "oracle_step", "max_err", "max_lse_err",
+__all__ = ["TOL", "LSE_TOL", "ERROR_REPORT", "record_error", "gpu_state", "gpu_step", "oracle_step", "max_err", "max_lse_err",
            "words", "step_inputs"]

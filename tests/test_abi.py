@@ -280,6 +280,25 @@ def test_shared_prefix_validation(kw, status):
     assert kvd.kvd_last_error() != ""
 
 
+@pytest.mark.parametrize("kw,status", [
+    (dict(mode=2), kvd.KVD_ERR_INVALID),
+    (dict(nbytes=24), kvd.KVD_ERR_INVALID),
+    (dict(src=NULL), kvd.KVD_ERR_INVALID),
+    (dict(sink=NULL), kvd.KVD_ERR_INVALID),
+    (dict(src=ctypes.c_void_p(256 + 8)), kvd.KVD_ERR_INVALID),
+    (dict(nbytes=0, src=NULL), kvd.KVD_OK),
+])
+def test_read_stream_validation(kw, status):
+    a = dict(src=DUMMY, nbytes=4096, mode=kvd.KVD_READ_BULK, sink=DUMMY, stream=NULL)
+    a.update(kw)
+    assert L.kvd_read_stream(a["src"], a["nbytes"], a["mode"], a["sink"], a["stream"]) == status
+
+
+def test_wait_limit_hook_accepts_any_value():
+    for v in (0, 5, -1, 1 << 40, -7):
+        assert L.kvd_set_decode_wait_limit(v) == kvd.KVD_OK
+
+
 def test_workspace_size_with_explicit_partitions():
     # layout: (B+1) int32 -> 256-byte rounded; slots*G floats -> rounded; slots*G*d floats
     B, H_q, H_kv, d, N = 3, 8, 2, 128, 10

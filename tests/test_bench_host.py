@@ -65,3 +65,50 @@ def test_reference_arm_prints_one_json_line(capsys):
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["steps"] == 4 and line["warmup"] == 3
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _full_oracle(w, si):
+    import oracle
+    from synth import to_words
+    kc, vc = to_words(w.k_cache).copy(), to_words(w.v_cache).copy()
+    oracle.append(kc, vc, w.block_table.numpy(), si["slot"].numpy(), to_words(si["k_new"]),
+                  to_words(si["v_new"]))
+    dt = oracle.BF16 if w.dtype.is_floating_point and w.dtype == bench.torch.bfloat16 else oracle.F16
+    out, _ = oracle.attend(to_words(si["q"]), kc, vc, w.block_table.numpy(), si["seq_lens"].numpy(),
+                           w.scale, dt)
+    return out
+
+
+def test_row_snapshot_renumbers_pages_and_feeds_the_oracle():
+    # the parity sample's compact copy (shared prefix pages, shuffled pool,
+    # sampled rows) must give the oracle exactly the rows of the whole batch
+    from synth import build_workload, step_inputs
+    w = build_workload("snap", 8, 8, 2, 64, "f16", [70, 33, 90, 37, 64, 65, 100, 34], seed=31,
+                       prefix_groups=2, prefix_tokens=32, spare_pages=3)
+    si = step_inputs(w, 0)
+    rows = bench.sample_sequences(w, 3, 5)
+    assert 1 in rows and 6 in rows            # shortest and longest are always sampled
+    snap = bench.RowSnapshot(w, si, rows)
+    assert snap.k.shape[0] < w.num_blocks      # only the sampled sequences' pages
+    full = _full_oracle(w, si)
+    err, spent, gbs, threads = bench.oracle_parity(snap, full[rows])
+    assert err == 0.0 and spent > 0 and threads >= 1
+    # a wrong row is seen
+    wrong = full[rows].copy()
+    wrong[-1, 0, 0] += 0.01
+    assert abs(bench.oracle_parity(snap, wrong)[0] - 0.01) < 1e-9
+
+
+def test_row_snapshot_8bit_parity_uses_the_oracles_quantisation():
+    import oracle
+    from synth import build_workload, step_inputs, to_words
+    w = build_workload("snap8", 3, 8, 2, 128, "bf16", [40, 17, 33], seed=32, spare_pages=2)
+    si = step_inputs(w, 0)
+    snap = bench.RowSnapshot(w, si, [0, 1, 2])
+    k8, ks = oracle.quantize_fp8(to_words(w.k_cache), oracle.BF16)
+    v8, vs = oracle.quantize_fp8(to_words(w.v_cache), oracle.BF16)
+    oracle.append_fp8(k8, v8, ks, vs, w.block_table.numpy(), si["slot"].numpy(), to_words(si["k_new"]),
+                      to_words(si["v_new"]), oracle.BF16)
+    ref, _ = oracle.attend_fp8(to_words(si["q"]), k8, v8, ks, vs, w.block_table.numpy(),
+                               si["seq_lens"].numpy(), w.scale, oracle.BF16)
+    assert bench.oracle_parity(snap, ref, fmt="fp8")[0] == 0.0
