@@ -162,7 +162,10 @@ kvd_status kvd_decode_step(const void *q, const void *k_new, const void *v_new, 
  *                 every member are the same physical pages, namely
  *                 block_table[group_start[g]][0 .. group_pages[g]-1]
  *   n_groups      0 makes this call kvd_decode_attention / kvd_decode_step
- *   max_group_size  upper bound on members per group (sizes the launch)
+ *   max_group_size  upper bound on members per group (sizes the launch); a
+ *                 larger group, or one whose bounds leave [0, B], is invalid:
+ *                 it sets KVD_DEVERR_SEQ_LEN and its members are attended
+ *                 whole, without the shared pass
  *   k_new, v_new  nullable; when given, the step's new token is appended as
  *                 in kvd_decode_step (it must land in a private page)
  *   workspace     kvd_shared_prefix_workspace_size(...) bytes, 256-aligned

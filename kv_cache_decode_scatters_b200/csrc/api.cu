@@ -430,6 +430,7 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
     pa.n_groups = n_groups;
     pa.chunks = PL.chunks;
     pa.fused = k_new != nullptr;
+    pa.maxg = max_group_size;
     e = kvd::launch_prefix(pa, d, dt, tm[0], tm[1], PL.row_blocks, s);
     if (e != cudaSuccess) return cuda_fail(e, "prefix launch");
     a.skip = pa.skip;

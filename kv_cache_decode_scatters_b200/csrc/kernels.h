@@ -93,6 +93,7 @@ struct PrefixArgs {
   unsigned *err;
   float scale_log2;
   int B, H_q, H_kv, G, num_blocks, maxb, n_groups, chunks, fused;
+  int maxg;                    // members per group at most: a larger group is invalid
 };
 
 struct GenericMergeArgs {

@@ -43,10 +43,17 @@ struct PGeo {
   static constexpr size_t smem() { return 1024 + (size_t)kStages * kStageBytes + 2 * kStages * 8; }
 };
 
+// A group whose bounds leave [0, B], that has more members than the
+// launch was sized for (maxg) or a shared page count outside the table is
+// invalid: the prefix pass skips it and its members are attended whole.
+__device__ __forceinline__ bool group_ok(const PrefixArgs &a, int s0, int s1, int gp) {
+  return s0 >= 0 && s1 <= a.B && s1 >= s0 && s1 - s0 <= a.maxg && gp >= 0 && gp <= a.maxb;
+}
+
 // Per-sequence shared pages for the suffix pass (CTA (0,0,0) of the prefix
 // launch writes them, all its threads).  A member whose length does not cover
 // the group's pages keeps no shared pages and is attended whole by the decode
-// kernel.
+// kernel; so do the members of an invalid group.
 __device__ void write_skip(const PrefixArgs &a, int cap) {
   const int tid = threadIdx.x;
   for (int b = tid; b < a.B; b += blockDim.x) a.skip[b] = 0;
@@ -54,6 +61,7 @@ __device__ void write_skip(const PrefixArgs &a, int cap) {
   for (int g = 0; g < a.n_groups; ++g) {
     const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
     const int gp = __ldg(a.group_pages + g);
+    if (!group_ok(a, s0, s1, gp)) continue;  // flagged by the group's CTAs
     for (int b = s0 + tid; b < s1; b += blockDim.x) {
       if (b < 0 || b >= a.B) continue;
       const int n = clamp_len(__ldg(a.seq_lens + b), cap);
@@ -94,7 +102,7 @@ __global__ void __launch_bounds__(32 * kWarps, 1)
   const int h = blockIdx.y;
   const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
   int gp = __ldg(a.group_pages + g);
-  if (s0 < 0 || s1 > a.B || s1 < s0 || gp < 0 || gp > a.maxb) {
+  if (!group_ok(a, s0, s1, gp)) {
     if (tid == 0) flag_error(a.err, kErrSeqLen);
     return;
   }
@@ -322,7 +330,7 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
   const int h = blockIdx.y;
   const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
   const int gp = __ldg(a.group_pages + g);
-  if (s0 < 0 || s1 > a.B || s1 < s0 || gp < 0 || gp > a.maxb) {
+  if (!group_ok(a, s0, s1, gp)) {
     if (tid == 0) flag_error(a.err, kErrSeqLen);
     return;
   }

@@ -479,3 +479,68 @@ def test_shared_prefix_member_shorter_than_prefix_is_attended_whole(kvd):
                            si["seq_lens"].numpy(), w.scale, oracle.F16)
     err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
     assert err <= TOL[w.dtype]
+
+
+def uneven_groups_case(d, dtype, H_q, H_kv, seed):
+    """Groups of different sizes and shared page counts, made by pointing
+    each member's first pages at its group's first member's pages."""
+    sizes = [5, 40, 1, 3, 7]
+    gpages = [4, 10, 2, 0, 6]
+    rng = np.random.default_rng(seed)
+    lens, starts = [], [0]
+    for sz, gp in zip(sizes, gpages):
+        for i in range(sz):
+            lens.append(int(gp * 16 + 1 + rng.integers(0, 90)))
+        starts.append(starts[-1] + sz)
+    lens[starts[1] + 3] = 10 * 16      # exactly the shared prefix: no private page
+    lens[starts[4] + 2] = 40           # shorter than its group's 6 shared pages
+    w = build_workload("spu", len(lens), H_q, H_kv, d, dtype, lens, seed=seed, spare_pages=4)
+    bt2 = w.block_table.clone()
+    for g, gp in enumerate(gpages):
+        s0, s1 = starts[g], starts[g + 1]
+        for b in range(s0 + 1, s1):
+            bt2[b, :gp] = w.block_table[s0, :gp]
+    gs = torch.tensor(starts, dtype=torch.int32)
+    gpg = torch.tensor(gpages, dtype=torch.int32)
+    return w, bt2, gs, gpg, max(sizes)
+
+
+@pytest.mark.parametrize("d,dtype,H_q,H_kv", [(128, "f16", 32, 8), (128, "bf16", 64, 8), (64, "f16", 16, 4)])
+def test_shared_prefix_uneven_groups(kvd, d, dtype, H_q, H_kv):
+    # groups of 5, 40, 1, 3 and 7 members sharing 4, 10, 2, 0 and 6 pages:
+    # units of different page counts and row blocks, one member exactly as
+    # long as its prefix, one shorter than it
+    w, bt2, gs, gpg, maxg = uneven_groups_case(d, dtype, H_q, H_kv, seed=1401)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    kvd.kvd_append(kc, vc, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    kvd.kvd_read_device_error(clear=True)
+    lse = torch.empty((w.B, w.H_q), dtype=torch.float32, device="cuda")
+    out = kvd.kvd_decode_attention_shared_prefix(si["q"].cuda(), kc, vc, bt2.cuda(), si["seq_lens"].cuda(),
+                                                 gs.cuda(), gpg.cuda(), maxg, w.scale, lse_out=lse)
+    torch.cuda.synchronize()
+    assert kvd.kvd_read_device_error() == 0
+    ref, ref_lse = oracle.attend(to_words(si["q"]), to_words(kc), to_words(vc), bt2.numpy(),
+                                 si["seq_lens"].numpy(), w.scale,
+                                 oracle.BF16 if w.dtype == torch.bfloat16 else oracle.F16)
+    err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
+    assert err <= TOL[w.dtype], f"max abs error {err}"
+    assert float(np.max(np.abs(lse.cpu().double().numpy() - ref_lse))) <= LSE_TOL
+
+
+def test_shared_prefix_group_larger_than_declared_is_flagged_and_attended_whole(kvd):
+    # max_group_size below the 40-member group: that group is invalid (its
+    # members are attended whole, the error word says so), the others share
+    w, bt2, gs, gpg, maxg = uneven_groups_case(128, "f16", 32, 8, seed=1402)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    kvd.kvd_append(kc, vc, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    kvd.kvd_read_device_error(clear=True)
+    out = kvd.kvd_decode_attention_shared_prefix(si["q"].cuda(), kc, vc, bt2.cuda(), si["seq_lens"].cuda(),
+                                                 gs.cuda(), gpg.cuda(), 8, w.scale)
+    torch.cuda.synchronize()
+    assert kvd.kvd_read_device_error(clear=True) & kvd.KVD_DEVERR_SEQ_LEN
+    ref, _ = oracle.attend(to_words(si["q"]), to_words(kc), to_words(vc), bt2.numpy(),
+                           si["seq_lens"].numpy(), w.scale, oracle.F16)
+    err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
+    assert err <= TOL[w.dtype], f"max abs error {err}"
