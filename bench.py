@@ -548,6 +548,7 @@ def run_ours(args):
     out = torch.empty_like(q)
     ws = kvd.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, args.partitions, dev)
     stream = torch.cuda.current_stream()
+    stream0 = stream
 
     f8 = None
     if args.kv_fp8 or args.kv_int8:
@@ -696,9 +697,11 @@ def run_ours(args):
                                         sum(a.elapsed_time(b) for a, b in evs) / (args.steps * per),
                                         step_bytes)
 
-    def run_step(x):
+    def run_step(x, st=None):
         """One step of the selected mode on the inputs x (q, k_new, v_new,
-        seq_lens and, for the two-call paths, slot)."""
+        seq_lens and, for the two-call paths, slot), on stream st (default:
+        the bench's stream)."""
+        stream = st if st is not None else stream0
         if f8 is not None and not args.separate_append:
             f8["step"](x["q"], x["k_new"], x["v_new"], f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt,
                        x["seq_lens"], w.scale, out=out, num_partitions=args.partitions, workspace=ws,
@@ -778,15 +781,46 @@ def run_ours(args):
         h_out.copy_(out, non_blocking=True)
         stream.synchronize()
 
-    for _ in range(3):
-        e2e_step()
-    barrier(dist)
-    t0 = time.perf_counter()
-    for _ in range(e2e_steps):
-        e2e_step()
-    e2e_s = max_over_ranks(dist, time.perf_counter() - t0)
-    barrier(dist)
+    def e2e_time(fn):
+        for _ in range(3):
+            fn()
+        barrier(dist)
+        t0 = time.perf_counter()
+        for _ in range(e2e_steps):
+            fn()
+        e2e_s = max_over_ranks(dist, time.perf_counter() - t0)
+        barrier(dist)
+        return e2e_s
+
+    e2e_eager_s = e2e_time(e2e_step)
+    # the same step as one CUDA graph: the H2D copy of the step's inputs from
+    # the pinned buffer, the library call, the D2H copy of out; each step
+    # replays it and waits for it (a decode loop refills h_buf between steps)
+    e2e_graph_s, e2e_graph_err = None, None
+    try:
+        gstream = torch.cuda.Stream()
+        gstream.wait_stream(stream)
+        e2e_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(gstream):
+            run_step(d_in, gstream)          # warm this stream once outside the capture
+            gstream.synchronize()
+            with torch.cuda.graph(e2e_graph, stream=gstream):
+                d_buf.copy_(h_buf, non_blocking=True)
+                run_step(d_in, gstream)
+                h_out.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+
+        def e2e_graph_step():
+            e2e_graph.replay()
+            stream.synchronize()
+
+        with torch.cuda.stream(stream):
+            e2e_graph_s = e2e_time(e2e_graph_step)
+    except Exception as exc:  # capture unsupported for this mode: report the eager figure only
+        e2e_graph_err = f"{type(exc).__name__}: {exc}"[:200]
+    e2e_s = e2e_graph_s if e2e_graph_s is not None else e2e_eager_s
     e2e_val = world * step_bytes * e2e_steps / e2e_s / 1e9
+    e2e_eager_val = world * step_bytes * e2e_steps / e2e_eager_s / 1e9
 
     if rank != 0:
         if dist is not None:
@@ -918,8 +952,14 @@ def run_ours(args):
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "us_per_step": round(e2e_s / e2e_steps * 1e6, 2),
-                "how": "the step's inputs in one pinned host buffer -> one H2D copy, the timed call, "
-                       "D2H of out, stream sync; wall clock"},
+                "mode": "cuda graph" if e2e_graph_s is not None else "eager",
+                "eager": {"value": round(e2e_eager_val, 2), "unit": "GB/s",
+                          "us_per_step": round(e2e_eager_s / e2e_steps * 1e6, 2)},
+                "graph_error": e2e_graph_err,
+                "how": "per step: the step's inputs in one pinned host buffer -> one H2D copy, the "
+                       "timed call, D2H of out, stream sync; wall clock, max over ranks.  mode "
+                       "'cuda graph': those three captured once as a CUDA graph and replayed each "
+                       "step (eager: issued from Python each step)"},
         "gpu_launches": (3 if (args.separate_append or sp is not None) else 2) * args.steps * per,
         "graph": ({"steps_per_graph": args.graph_steps, "replays": args.steps} if graph is not None
                   else None),
