@@ -427,21 +427,29 @@ def run_reference(args):
 
 # The workloads reported beside the headline one in a default run (workload,
 # shared-prefix mode): every synthetic configuration of the method's benchmark.
-PER_WORKLOADS = (("tiny", False), ("gqa70b", False), ("long", False), ("cbatch", False),
-                 ("cbatch", True))
+PER_WORKLOADS = (("tiny", False, None), ("gqa70b", False, None), ("long", False, None),
+                 ("cbatch", False, None), ("cbatch", True, None), ("mha7b", False, "fp8"),
+                 ("gqa70b", False, "fp8"), ("mha7b", False, "int8"), ("gqa70b", False, "int8"))
 
 
-def measure_workload(kvd, name, shared_prefix, dev, steps, warmup):
+def measure_workload(kvd, name, shared_prefix, dev, steps, warmup, fmt=None):
     """Time one workload's decode step through the call the headline uses
-    (kvd_decode_step, or the shared-prefix call with its fused append) with
-    automatic partitions: `warmup` untimed steps, then `steps` calls each
-    bracketed by CUDA events on the launching stream.  Returns (report dict,
-    RowSnapshot of sampled sequences taken before any kernel ran, the GPU's
-    output rows of those sequences as float64)."""
+    (kvd_decode_step, the shared-prefix call with its fused append, or, with
+    fmt "fp8" / "int8", kvd_decode_step_{fmt} over the pool quantised to
+    that 8-bit cache) with automatic partitions: `warmup` untimed steps, then
+    `steps` calls each bracketed by CUDA events on the launching stream.
+    Returns (report dict, RowSnapshot of sampled sequences taken before any
+    kernel ran, the GPU's output rows of those sequences as float64)."""
     w = named_config(name, device="cuda", gen_device="cuda")
     si = step_inputs(w, 0)
     snap = RowSnapshot(w, si, sample_sequences(w, 3, 77))
     kc, vc, bt = w.k_cache, w.v_cache, w.block_table.to(dev)
+    q8 = None
+    if fmt is not None:
+        quant = getattr(kvd, "kvd_quantize_" + fmt)
+        k8, ks = quant(kc)
+        v8, vs = quant(vc)
+        q8 = (k8, v8, ks, vs, getattr(kvd, "kvd_decode_step_" + fmt))
     q, k_new, v_new, seq_lens = si["q"], si["k_new"], si["v_new"], si["seq_lens"].to(dev)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
@@ -457,7 +465,10 @@ def measure_workload(kvd, name, shared_prefix, dev, steps, warmup):
         ws = kvd.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, 0, dev)
 
     def call(x_q, x_k, x_v, x_len):
-        if sp is not None:
+        if q8 is not None:
+            q8[4](x_q, x_k, x_v, q8[0], q8[1], q8[2], q8[3], bt, x_len, w.scale, out=out, workspace=ws,
+                  stream=stream)
+        elif sp is not None:
             kvd.kvd_decode_attention_shared_prefix(x_q, kc, vc, bt, x_len, sp["start"], sp["pages"],
                                                    sp["max"], w.scale, out=out, k_new=x_k, v_new=x_v,
                                                    workspace=ws, stream=stream)
@@ -492,11 +503,16 @@ def measure_workload(kvd, name, shared_prefix, dev, steps, warmup):
     if w.groups:
         a_b -= w.groups * (w.B // w.groups - 1) * w.prefix_tokens * w.H_kv * 2 * w.d * 2
     nbytes = a_b + append_bytes(w, si["slot"].cpu())
+    if q8 is not None:  # codes + scales read; appended rows read in 16 bits, written as codes + scales
+        rows = int((si["slot"] >= 0).sum().item()) * w.H_kv
+        nbytes = fp8_attention_bytes(w, si["seq_lens"].cpu()) + rows * 2 * (w.d * 2 + w.d + (w.d // 32) * 4)
     rep = {
-        "workload": name + (" --shared-prefix" if shared_prefix else ""),
+        "workload": name + (" --shared-prefix" if shared_prefix else "") + (f" --kv-{fmt}" if fmt else ""),
         "call": ("kvd_decode_attention_shared_prefix (fused append)" if sp is not None
-                 else "kvd_decode_step"),
-        "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d, "kv_dtype": w.dtype_name,
+                 else f"kvd_decode_step_{fmt} over the {'E4M3' if fmt == 'fp8' else 'INT8'} cache"
+                 if q8 is not None else "kvd_decode_step"),
+        "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
+        "kv_dtype": w.dtype_name if q8 is None else f"{fmt} codes, {w.dtype_name} q/out",
         "seq_lens": _lens_desc(w), "steps": steps, "warmup": warmup,
         "bytes_per_step": nbytes,
         "us_per_step": round(step_us, 2),
@@ -522,6 +538,7 @@ def measure_workload(kvd, name, shared_prefix, dev, steps, warmup):
         rep["consecutive_steps"] = {"steps": w.steps,
                                     "us_per_step": round(c0.elapsed_time(c1) * 1e3 / w.steps, 2)}
         del sets
+    rep["fmt"] = fmt
     return rep, snap, gpu_rows
 
 
@@ -832,8 +849,8 @@ def run_ours(args):
     default_run = (args.workload == "mha7b" and f8 is None and sp is None and not args.separate_append
                    and graph is None and args.scale_down == 1)
     if world == 1 and (args.per_workload == "on" or (args.per_workload == "auto" and default_run)):
-        for name, shared in PER_WORKLOADS:
-            per_wl.append(measure_workload(kvd, name, shared, dev, args.per_workload_steps, 5))
+        for name, shared, fmt in PER_WORKLOADS:
+            per_wl.append(measure_workload(kvd, name, shared, dev, args.per_workload_steps, 5, fmt))
             torch.cuda.empty_cache()
 
     peak, peak_kind = peaks()
@@ -860,7 +877,7 @@ def run_ours(args):
     per_report = []
     for rep, psnap, prows in per_wl:
         ptol = 1e-2 if psnap.bf16 else 2e-3
-        perr, pspent, pgbs, pthr = oracle_parity(psnap, prows)
+        perr, pspent, pgbs, pthr = oracle_parity(psnap, prows, fmt=rep["fmt"])
         ach = rep["bytes_per_step"] / (rep["timed_call_us"] * 1e-6) / 1e9
         rep["roofline"] = {"achieved": round(ach, 2), "frac": round(ach / peak, 4),
                            "frac_of_read_only_peak": round(ach / read_peak, 4)}
