@@ -169,8 +169,12 @@ class RowSnapshot:
         self.scale = w.scale
         self.bf16 = w.dtype == torch.bfloat16
         tokens = int(self.seq_lens.astype(np.int64).sum())
+        appended = int((self.slot >= 0).sum()) * w.H_kv
         self.nbytes = (tokens * w.H_kv * 2 * w.d * 2 + 2 * len(rows) * w.H_q * w.d * 2
-                       + int((self.slot >= 0).sum()) * w.H_kv * w.d * 2 * 2 * 2)
+                       + appended * w.d * 2 * 2 * 2)
+        # over an 8-bit cache: codes + per-32-channel fp32 scales
+        self.nbytes_q8 = (tokens * w.H_kv * 2 * (w.d + (w.d // 32) * 4) + 2 * len(rows) * w.H_q * w.d * 2
+                          + appended * 2 * (w.d * 2 + w.d + (w.d // 32) * 4))
 
     def describe(self, w):
         return (f"sequences {self.rows} of {w.B} (lengths {self.seq_lens.tolist()}), all "
@@ -360,21 +364,23 @@ def oracle_parity(snap, gpu_rows, threads=0, fmt=None):
     import oracle
     dt = oracle.BF16 if snap.bf16 else oracle.F16
     threads = threads if threads > 0 else oracle.max_threads()
-    t0 = time.perf_counter()
     if fmt is None:
+        t0 = time.perf_counter()
         kc, vc = snap.k.copy(), snap.v.copy()
         oracle.append(kc, vc, snap.bt, snap.slot, snap.k_new, snap.v_new)
         ref, _ = oracle.attend(snap.q, kc, vc, snap.bt, snap.seq_lens, snap.scale, dt, nthreads=threads)
     else:
+        # the 8-bit pool is quantised once (setup, as on the GPU), then timed
         quant = getattr(oracle, "quantize_" + fmt)
         k8, ks = quant(snap.k, dt)
         v8, vs = quant(snap.v, dt)
+        t0 = time.perf_counter()
         getattr(oracle, "append_" + fmt)(k8, v8, ks, vs, snap.bt, snap.slot, snap.k_new, snap.v_new, dt)
         ref, _ = getattr(oracle, "attend_" + fmt)(snap.q, k8, v8, ks, vs, snap.bt, snap.seq_lens,
                                                   snap.scale, dt, nthreads=threads)
     spent = time.perf_counter() - t0
     err = float(np.max(np.abs(gpu_rows - ref))) if ref.size else 0.0
-    return err, spent, snap.nbytes / spent / 1e9, threads
+    return err, spent, (snap.nbytes if fmt is None else snap.nbytes_q8) / spent / 1e9, threads
 
 
 ONE_THREAD_WORKLOADS = ("tiny", "long")
