@@ -202,7 +202,7 @@ size_t kvd_shared_prefix_workspace_size(int B, int H_q, int H_kv, int d, int n_g
  *                    k_new/v_new [B][H_kv][d] into row slot % 16 of page
  *                    block_table[b][slot / 16] of codes and scales.
  * kvd_decode_attention_fp8
- *                    kvd_decode_attention over the 8-bit cache (d = 128):
+ *                    kvd_decode_attention over the 8-bit cache (d = 64 or 128):
  *                    softmax(scale q K^T) V with K, V the dequantised values;
  *                    q and out in dtype; workspace as kvd_decode_attention.
  */
@@ -257,7 +257,7 @@ kvd_status kvd_decode_attention_int8(const void *q, const int8_t *k_codes, const
  *
  *   k_new, v_new     device, [B][H_kv][d] in dtype, 16-byte aligned
  *   k_codes, v_codes, k_scale, v_scale  the 8-bit cache, written in place
- *   other arguments as kvd_decode_attention_{fp8,int8} (d = 128)
+ *   other arguments as kvd_decode_attention_{fp8,int8} (d = 64 or 128)
  * Every sequence b with seq_lens[b] >= 1 appends its new token at position
  * seq_lens[b] - 1; seq_lens[b] = 0 appends nothing.  The codes and scales
  * written are bit-identical to kvd_append_{fp8,int8} with slot =

@@ -291,7 +291,6 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   if (!(scale == scale)) return fail(KVD_ERR_INVALID, "scale is NaN");
   if (num_partitions < 0) return fail(KVD_ERR_INVALID, "num_partitions < 0");
   if (q8) {
-    if (d != 128) return fail(KVD_ERR_UNSUPPORTED, "the 8-bit cache supports d = 128 only");
     if (!v_scale) return fail(KVD_ERR_INVALID, "v_scale is NULL");
     if (n_groups > 0) return fail(KVD_ERR_UNSUPPORTED, "the 8-bit cache has no shared-prefix mode");
     if (!aligned(k_scale, 16) || !aligned(v_scale, 16))
@@ -339,14 +338,17 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   for (int i = 0; i < 2; ++i) {
     CUresult r;
     if (q8) {
-      // E4M3 code pools as 2-D byte tensors {128, num_blocks*H_kv*16 rows};
-      // one box = the 16 rows of one page of one head, 128-byte swizzled.
-      cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(num_blocks) * H_kv * KVD_PAGE_TOKENS};
-      cuuint64_t strides[1] = {128};
-      cuuint32_t box[2] = {128, KVD_PAGE_TOKENS};
+      // 8-bit code pools as 2-D byte tensors {d, num_blocks*H_kv*16 rows};
+      // one box = the 16 rows of one page of one head, with the 128-byte
+      // (d = 128) or 64-byte (d = 64) swizzle.
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>(d),
+                            static_cast<cuuint64_t>(num_blocks) * H_kv * KVD_PAGE_TOKENS};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>(d)};
+      cuuint32_t box[2] = {static_cast<cuuint32_t>(d), KVD_PAGE_TOKENS};
       cuuint32_t estr[2] = {1, 1};
       r = encode(&tm[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(pools[i]), dims,
-                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                 d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     } else {
       // K and V pools as 3-D tensors {64 elements, d/64 units, num_blocks*H_kv*16
@@ -438,7 +440,7 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
     a.pre_lse = pa.pre_lse;
     a.pre_chunks = PL.chunks;
   }
-  e = q8 ? kvd::launch_decode_q8(a, dt, fmt, tm[0], tm[1], s, N)
+  e = q8 ? kvd::launch_decode_q8(a, d, dt, fmt, tm[0], tm[1], s, N)
           : kvd::launch_decode(a, d, dt, tm[0], tm[1], s, N);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   e = kvd::launch_decode_merge(a, d, dt, s);

@@ -131,65 +131,72 @@ struct Page16 {
   }
 };
 
-// 8-bit pages (d = 128; E4M3 or INT8 codes): codes [16][128] per (page, head)
-// in one swizzled box, fp32 scales [16][4] per (page, head) copied alongside;
+// 8-bit pages (d = D = 64 or 128; E4M3 or INT8 codes): codes [16][D] per
+// (page, head) in one box with the 128-byte (D = 128) or 64-byte (D = 64)
+// swizzle, fp32 scales [16][D / 32] per (page, head) copied alongside;
 // output dtype T.
-template <int NT, typename T, Code8 kFmt>
+template <int D, int NT, typename T, Code8 kFmt>
 struct Page8 {
   using Out = T;
-  static constexpr int kPageBytes = kPage * 128;             // codes of K (or V)
-  static constexpr int kScaleBytes = kPage * 4 * 4;          // scales of K (or V)
+  static constexpr int kG = D / 32;                          // scale groups of a token
+  static constexpr int kPageBytes = kPage * D;               // codes of K (or V)
+  static constexpr int kScaleBytes = kPage * kG * 4;         // scales of K (or V)
   static constexpr int kCopyBytes = 2 * kPageBytes + 2 * kScaleBytes;
   static constexpr int kStride = 2 * kPageBytes;             // codes only: 1024-aligned stages
   static constexpr int kAuxBytes = 2 * kScaleBytes;          // scales, in their own area
+  static_assert(kScaleBytes % 16 == 0, "scale rows are bulk copies of whole 16-byte units");
   static __device__ __forceinline__ void issue(uint32_t dst, uint32_t aux, uint32_t bar,
                                                const CUtensorMap *tmK, const CUtensorMap *tmV,
                                                int row, uint64_t policy, const DecodeArgs &a) {
     mbar_arrive_expect_tx(bar, kCopyBytes);
     tma_load_2d(dst, tmK, 0, row, bar, policy);
     tma_load_2d(dst + kPageBytes, tmV, 0, row, bar, policy);
-    bulk_load(aux, a.k_scale + static_cast<size_t>(row) * 4, kScaleBytes, bar);
-    bulk_load(aux + kScaleBytes, a.v_scale + static_cast<size_t>(row) * 4, kScaleBytes, bar);
+    bulk_load(aux, a.k_scale + static_cast<size_t>(row) * kG, kScaleBytes, bar);
+    bulk_load(aux + kScaleBytes, a.v_scale + static_cast<size_t>(row) * kG, kScaleBytes, bar);
   }
   static __device__ __forceinline__ void zero_tail(uint8_t *st, uint8_t *aux, int ntok, int lane) {
     // V codes and V scales of masked rows (their zero weights times a NaN
     // scale would otherwise poison the PV product)
-    const int n16 = (kPage - ntok) * 128 / 16;
-    uint4 *z = reinterpret_cast<uint4 *>(st + kPageBytes + ntok * 128);
+    const int n16 = (kPage - ntok) * D / 16;
+    uint4 *z = reinterpret_cast<uint4 *>(st + kPageBytes + ntok * D);
     for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
-    uint4 *zs = reinterpret_cast<uint4 *>(aux + kScaleBytes + ntok * 16);
-    for (int i = lane; i < kPage - ntok; i += 32) zs[i] = make_uint4(0, 0, 0, 0);
+    float *zs = reinterpret_cast<float *>(aux + kScaleBytes) + ntok * kG;
+    for (int i = lane; i < (kPage - ntok) * kG; i += 32) zs[i] = 0.f;
   }
   // fused append: encode the new token of pair (b, h) exactly as the
   // quantising append does (encode_row4), put its codes and scales into row t
   // of the staged page and write them to the pools at row `row` + t
   static __device__ __forceinline__ void patch(uint8_t *st, uint8_t *aux, int t, int lane,
                                                const DecodeArgs &a, int b, int h, int row) {
-    const size_t src = (static_cast<size_t>(b) * a.H_kv + h) * 128;
+    const size_t src = (static_cast<size_t>(b) * a.H_kv + h) * D;
     const size_t dst = static_cast<size_t>(row) + t;
+    const bool live = lane * 4 < D;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       float sc;
       const uint32_t w =
-          encode_row4<T, kFmt>(static_cast<const T *>(half ? a.v_new : a.k_new) + src, true, lane, sc);
-      *reinterpret_cast<uint32_t *>(st + half * kPageBytes + swz8(t, lane >> 2) + (lane & 3) * 4) = w;
-      *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(half ? a.v_cache : a.k_cache) + dst * 128 +
-                                    lane * 4) = w;
-      if ((lane & 7) == 0) {
-        reinterpret_cast<float *>(aux + half * kScaleBytes)[t * 4 + (lane >> 3)] = sc;
-        (half ? a.v_scale : a.k_scale)[dst * 4 + (lane >> 3)] = sc;
+          encode_row4<T, kFmt>(static_cast<const T *>(half ? a.v_new : a.k_new) + src, live, lane, sc);
+      if (live) {
+        *reinterpret_cast<uint32_t *>(st + half * kPageBytes + swz_rows<D>(t, lane >> 2) +
+                                      (lane & 3) * 4) = w;
+        *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(half ? a.v_cache : a.k_cache) + dst * D +
+                                      lane * 4) = w;
+        if ((lane & 7) == 0) {
+          reinterpret_cast<float *>(aux + half * kScaleBytes)[t * kG + (lane >> 3)] = sc;
+          (half ? a.v_scale : a.k_scale)[dst * kG + (lane >> 3)] = sc;
+        }
       }
     }
   }
   static __device__ __forceinline__ void tile(uint8_t *st, uint8_t *aux, int ntok, float sl2, int lane,
-                                              const uint32_t (&qf)[NT][8][2],
-                                              float (&acc)[NT][8][4], float (&m)[NT][2],
+                                              const uint32_t (&qf)[NT][D / 16][2],
+                                              float (&acc)[NT][D / 16][4], float (&m)[NT][2],
                                               float (&l)[NT][2]) {
     const float *ks = reinterpret_cast<const float *>(aux);
-    tile_page_q8<NT, kFmt>(smem_u32(st), smem_u32(st + kPageBytes), ks, ks + kPage * 4, ntok, sl2,
-                           lane, qf, acc, m, l);
+    tile_page_q8<D, NT, kFmt>(smem_u32(st), smem_u32(st + kPageBytes), ks, ks + kPage * kG, ntok, sl2,
+                              lane, qf, acc, m, l);
   }
-  // q in f16, channel order of the E4M3 tile: k-slots 2t, 2t+1 <- channels
+  // q in f16, channel order of the 8-bit tile: k-slots 2t, 2t+1 <- channels
   // 4t, 4t+1 and k-slots 2t+8, 2t+9 <- channels 4t+2, 4t+3 of each 16
   static __device__ __forceinline__ uint32_t to_f16x2(uint32_t w) {
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
@@ -1070,8 +1077,10 @@ cudaError_t launch_generic_dt(const GenericMergeArgs &a, cudaStream_t st) {
 
 int decode_auto_parts(int sms) { return sms; }
 
-// 8-bit cache (d = 128): 4 KB code stages plus 512 B of scales; as for the
-// 16-bit pages, many warps with a short ring each keep the copies in flight.
+// 8-bit cache: d = 128 has 4 KB code stages plus 512 B of scales, d = 64
+// 2 KB stages plus 256 B; as for the 16-bit pages, many warps with a short
+// ring each keep the copies in flight (d = 64 twice as many stages, for the
+// same bytes in flight).
 #ifndef KVD_TUNE_W8_1
 #define KVD_TUNE_W8_1 16
 #endif
@@ -1084,18 +1093,49 @@ int decode_auto_parts(int sms) { return sms; }
 #ifndef KVD_TUNE_S8_2
 #define KVD_TUNE_S8_2 2
 #endif
+#ifndef KVD_TUNE_W8_64_1
+#define KVD_TUNE_W8_64_1 16
+#endif
+#ifndef KVD_TUNE_S8_64_1
+#define KVD_TUNE_S8_64_1 4
+#endif
+#ifndef KVD_TUNE_W8_64_2
+#define KVD_TUNE_W8_64_2 8
+#endif
+#ifndef KVD_TUNE_S8_64_2
+#define KVD_TUNE_S8_64_2 4
+#endif
 
 namespace {
 // Largest shared memory one CTA may opt into on sm_100 (227 KB); 1 KB of it is
 // left for the kernels' static shared variables.
 constexpr size_t kMaxCtaSmem = 232448;
 
-template <int NT, typename T, Code8 kFmt, int W, int S>
+template <int D, int NT>
+struct Tune8;
+template <>
+struct Tune8<128, 1> {
+  static constexpr int W = KVD_TUNE_W8_1, S = KVD_TUNE_S8_1;
+};
+template <>
+struct Tune8<128, 2> {
+  static constexpr int W = KVD_TUNE_W8_2, S = KVD_TUNE_S8_2;
+};
+template <>
+struct Tune8<64, 1> {
+  static constexpr int W = KVD_TUNE_W8_64_1, S = KVD_TUNE_S8_64_1;
+};
+template <>
+struct Tune8<64, 2> {
+  static constexpr int W = KVD_TUNE_W8_64_2, S = KVD_TUNE_S8_64_2;
+};
+
+template <int D, int NT, typename T, Code8 kFmt, int W, int S>
 cudaError_t launch_decode8_ws(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                               cudaStream_t st, int grid) {
-  using Pol = Page8<NT, T, kFmt>;
-  auto kern = decode_kernel<128, NT, Pol, W, S>;
-  const size_t smem = Geo<128, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B);
+  using Pol = Page8<D, NT, T, kFmt>;
+  auto kern = decode_kernel<D, NT, Pol, W, S>;
+  const size_t smem = Geo<D, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -1104,39 +1144,39 @@ cudaError_t launch_decode8_ws(const DecodeArgs &a, const CUtensorMap &tmK, const
 
 // The tuned ring depth, or one stage per warp when the batch's prefix sums
 // (4 bytes per sequence) would push the tuned layout past the CTA limit.
-template <int NT, typename T, Code8 kFmt>
+template <int D, int NT, typename T, Code8 kFmt>
 cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                              cudaStream_t st, int grid) {
-  constexpr int W = NT == 1 ? KVD_TUNE_W8_1 : KVD_TUNE_W8_2;
-  constexpr int S = NT == 1 ? KVD_TUNE_S8_1 : KVD_TUNE_S8_2;
-  using Pol = Page8<NT, T, kFmt>;
+  constexpr int W = Tune8<D, NT>::W, S = Tune8<D, NT>::S;
+  using Pol = Page8<D, NT, T, kFmt>;
   // one stage must still hold a parked accumulator tile
-  constexpr bool kCanShrink = S > 1 && 8 * NT * 128 * 4 <= Pol::kStride;
+  constexpr bool kCanShrink = S > 1 && 8 * NT * D * 4 <= Pol::kStride;
   if constexpr (kCanShrink) {
-    if (Geo<128, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B) + 1024 > kMaxCtaSmem)
-      return launch_decode8_ws<NT, T, kFmt, W, 1>(a, tmK, tmV, st, grid);
+    if (Geo<D, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B) + 1024 > kMaxCtaSmem)
+      return launch_decode8_ws<D, NT, T, kFmt, W, 1>(a, tmK, tmV, st, grid);
   }
-  return launch_decode8_ws<NT, T, kFmt, W, S>(a, tmK, tmV, st, grid);
+  return launch_decode8_ws<D, NT, T, kFmt, W, S>(a, tmK, tmV, st, grid);
 }
-}  // namespace
 
-namespace {
-template <Code8 kFmt>
+template <int D, Code8 kFmt>
 cudaError_t launch_decode_q8_fmt(const DecodeArgs &a, DType dt, const CUtensorMap &tmK,
                                  const CUtensorMap &tmV, cudaStream_t s, int grid) {
   const bool two = a.G > 8;
   if (dt == DType::BF16)
-    return two ? launch_decode8_t<2, __nv_bfloat16, kFmt>(a, tmK, tmV, s, grid)
-               : launch_decode8_t<1, __nv_bfloat16, kFmt>(a, tmK, tmV, s, grid);
-  return two ? launch_decode8_t<2, __half, kFmt>(a, tmK, tmV, s, grid)
-             : launch_decode8_t<1, __half, kFmt>(a, tmK, tmV, s, grid);
+    return two ? launch_decode8_t<D, 2, __nv_bfloat16, kFmt>(a, tmK, tmV, s, grid)
+               : launch_decode8_t<D, 1, __nv_bfloat16, kFmt>(a, tmK, tmV, s, grid);
+  return two ? launch_decode8_t<D, 2, __half, kFmt>(a, tmK, tmV, s, grid)
+             : launch_decode8_t<D, 1, __half, kFmt>(a, tmK, tmV, s, grid);
 }
 }  // namespace
 
-cudaError_t launch_decode_q8(const DecodeArgs &a, DType dt, Code8 fmt, const CUtensorMap &tmK,
+cudaError_t launch_decode_q8(const DecodeArgs &a, int d, DType dt, Code8 fmt, const CUtensorMap &tmK,
                              const CUtensorMap &tmV, cudaStream_t s, int grid) {
-  return fmt == Code8::INT8 ? launch_decode_q8_fmt<Code8::INT8>(a, dt, tmK, tmV, s, grid)
-                            : launch_decode_q8_fmt<Code8::E4M3>(a, dt, tmK, tmV, s, grid);
+  if (d == 64)
+    return fmt == Code8::INT8 ? launch_decode_q8_fmt<64, Code8::INT8>(a, dt, tmK, tmV, s, grid)
+                              : launch_decode_q8_fmt<64, Code8::E4M3>(a, dt, tmK, tmV, s, grid);
+  return fmt == Code8::INT8 ? launch_decode_q8_fmt<128, Code8::INT8>(a, dt, tmK, tmV, s, grid)
+                            : launch_decode_q8_fmt<128, Code8::E4M3>(a, dt, tmK, tmV, s, grid);
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, int d, DType dt, const CUtensorMap &tmK,

@@ -117,8 +117,8 @@ cudaError_t launch_decode(const DecodeArgs &a, int d, DType dt, const CUtensorMa
                           const CUtensorMap &tmV, cudaStream_t s, int grid);
 cudaError_t launch_decode_merge(const DecodeArgs &a, int d, DType dt, cudaStream_t s);
 cudaError_t launch_generic_merge(const GenericMergeArgs &a, DType dt, cudaStream_t s);
-cudaError_t launch_decode_q8(const DecodeArgs &a, DType dt, Code8 fmt, const CUtensorMap &tmK,
-                              const CUtensorMap &tmV, cudaStream_t s, int grid);
+cudaError_t launch_decode_q8(const DecodeArgs &a, int d, DType dt, Code8 fmt, const CUtensorMap &tmK,
+                             const CUtensorMap &tmV, cudaStream_t s, int grid);
 cudaError_t launch_quantize_q8(const QuantArgs &a, DType dt, Code8 fmt, cudaStream_t s);
 // Read-only streaming of `bytes` (a multiple of 16) from src: mode
 // KVD_READ_VECTOR or KVD_READ_BULK; XOR of every 32-bit word into *sink.

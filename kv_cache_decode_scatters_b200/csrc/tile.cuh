@@ -305,8 +305,18 @@ __device__ __forceinline__ uint32_t swz8(int t, int c) {
   return static_cast<uint32_t>(t * 128 + ((c ^ (t & 7)) << 4));
 }
 
-// One 16-token page of an 8-bit cache (d = 128; E4M3 or INT8 codes) for 8*NT
-// query rows of one warp.  Codes are exact in f16, so the tensor-core tile
+// The same for a page of D-byte rows (D = 128: the 128-byte swizzle above;
+// D = 64: the 64-byte swizzle, chunk c of row t at chunk c ^ ((t >> 1) & 3),
+// so the 8 rows an ldmatrix reads fall on distinct banks).
+template <int D>
+__device__ __forceinline__ uint32_t swz_rows(int t, int c) {
+  static_assert(D == 128 || D == 64, "8-bit pages of 64 or 128 channels");
+  if constexpr (D == 128) return swz8(t, c);
+  else return static_cast<uint32_t>(t * 64 + ((c ^ ((t >> 1) & 3)) << 4));
+}
+
+// One 16-token page of an 8-bit cache (d = D = 64 or 128; E4M3 or INT8 codes)
+// for 8*NT query rows of one warp.  Codes are exact in f16, so the tensor-core tile
 // runs in f16:
 //  * K: ldmatrix on the code bytes gives each lane four consecutive channels
 //    of a token per register; converted in pairs they fill the A fragment
@@ -317,30 +327,31 @@ __device__ __forceinline__ uint32_t swz8(int t, int c) {
 //    a byte permute splits it into the A fragments of V^T, with output slot
 //    g8 <-> channel 2*g8 and slot g8+8 <-> channel 2*g8+1 of each m-tile.
 //    The V group scales ride on the probabilities (one P^T operand per group).
-// ks, vs: the page's fp32 scales in shared memory, [16 tokens][4 groups].
-template <int NT, Code8 kFmt>
+// ks, vs: the page's fp32 scales in shared memory, [16 tokens][D / 32 groups].
+template <int D, int NT, Code8 kFmt>
 __device__ __forceinline__ void tile_page_q8(uint32_t kb, uint32_t vb, const float *ks,
                                               const float *vs, int ntok, float scale_log2,
-                                              int lane, const uint32_t (&qf)[NT][8][2],
-                                              float (&acc)[NT][8][4], float (&m_run)[NT][2],
+                                              int lane, const uint32_t (&qf)[NT][D / 16][2],
+                                              float (&acc)[NT][D / 16][4], float (&m_run)[NT][2],
                                               float (&l_run)[NT][2]) {
   using M = Mma<__half>;
+  constexpr int kG = D / 32;  // scale groups of a token
   const int g8 = lane >> 2;
   const int mi = lane >> 3, r8 = lane & 7;
   const int tok = r8 + ((mi & 1) << 3);  // row this lane addresses for ldmatrix
   const int hi16 = mi >> 1;              // second 16 bytes of a 32-channel group
 
-  float sg[4][NT][4];
+  float sg[kG][NT][4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
+  for (int j = 0; j < kG; ++j)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sg[j][nt][e] = 0.f;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < kG; ++j) {
     uint32_t R[4];
-    ldmatrix_x4(R, kb + swz8(tok, 2 * j + hi16));
+    ldmatrix_x4(R, kb + swz_rows<D>(tok, 2 * j + hi16));
     uint32_t A0[4], A1[4];
     code8x4_to_f16x2x2<kFmt>(R[0], A0[0], A0[2]);
     code8x4_to_f16x2x2<kFmt>(R[1], A0[1], A0[3]);
@@ -352,22 +363,37 @@ __device__ __forceinline__ void tile_page_q8(uint32_t kb, uint32_t vb, const flo
       M::run(sg[j][nt], A1, qf[nt][2 * j + 1][0], qf[nt][2 * j + 1][1]);
     }
   }
-  const float4 kA = *reinterpret_cast<const float4 *>(ks + g8 * 4);
-  const float4 kB = *reinterpret_cast<const float4 *>(ks + (g8 + 8) * 4);
-  const float4 vA = *reinterpret_cast<const float4 *>(vs + g8 * 4);
-  const float4 vB = *reinterpret_cast<const float4 *>(vs + (g8 + 8) * 4);
-  const float kAs[4] = {kA.x, kA.y, kA.z, kA.w}, kBs[4] = {kB.x, kB.y, kB.z, kB.w};
-  const float vAs[4] = {vA.x, vA.y, vA.z, vA.w}, vBs[4] = {vB.x, vB.y, vB.z, vB.w};
+  // the scales of this lane's two tokens (g8 and g8 + 8), K and V
+  float kAs[kG], kBs[kG], vAs[kG], vBs[kG];
+  if constexpr (kG == 4) {
+    const float4 kA = *reinterpret_cast<const float4 *>(ks + g8 * 4);
+    const float4 kB = *reinterpret_cast<const float4 *>(ks + (g8 + 8) * 4);
+    const float4 vA = *reinterpret_cast<const float4 *>(vs + g8 * 4);
+    const float4 vB = *reinterpret_cast<const float4 *>(vs + (g8 + 8) * 4);
+    kAs[0] = kA.x; kAs[1] = kA.y; kAs[2] = kA.z; kAs[3] = kA.w;
+    kBs[0] = kB.x; kBs[1] = kB.y; kBs[2] = kB.z; kBs[3] = kB.w;
+    vAs[0] = vA.x; vAs[1] = vA.y; vAs[2] = vA.z; vAs[3] = vA.w;
+    vBs[0] = vB.x; vBs[1] = vB.y; vBs[2] = vB.z; vBs[3] = vB.w;
+  } else {
+    const float2 kA = *reinterpret_cast<const float2 *>(ks + g8 * 2);
+    const float2 kB = *reinterpret_cast<const float2 *>(ks + (g8 + 8) * 2);
+    const float2 vA = *reinterpret_cast<const float2 *>(vs + g8 * 2);
+    const float2 vB = *reinterpret_cast<const float2 *>(vs + (g8 + 8) * 2);
+    kAs[0] = kA.x; kAs[1] = kA.y;
+    kBs[0] = kB.x; kBs[1] = kB.y;
+    vAs[0] = vA.x; vAs[1] = vA.y;
+    vBs[0] = vB.x; vBs[1] = vB.y;
+  }
 
   const bool v0 = g8 < ntok, v1 = g8 + 8 < ntok;
-  uint32_t pj0[4][NT], pj1[4][NT];
+  uint32_t pj0[kG][NT], pj1[kG][NT];
   float alpha[NT][2];
   bool rescale = false;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < kG; ++j) {
       s4[0] += sg[j][nt][0] * kAs[j];
       s4[1] += sg[j][nt][1] * kAs[j];
       s4[2] += sg[j][nt][2] * kBs[j];
@@ -394,7 +420,7 @@ __device__ __forceinline__ void tile_page_q8(uint32_t kb, uint32_t vb, const flo
     l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (e0 + e2);
     l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (e1 + e3);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < kG; ++j) {
       // masked tokens have e = 0 and a V scale of 0 (cleared by the caller)
       pj0[j][nt] = movmatrix_trans(f16pack(e0 * vAs[j], e1 * vAs[j]));
       pj1[j][nt] = movmatrix_trans(f16pack(e2 * vBs[j], e3 * vBs[j]));
@@ -404,7 +430,7 @@ __device__ __forceinline__ void tile_page_q8(uint32_t kb, uint32_t vb, const flo
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
+      for (int mt = 0; mt < D / 16; ++mt) {
         acc[nt][mt][0] *= alpha[nt][0];
         acc[nt][mt][1] *= alpha[nt][1];
         acc[nt][mt][2] *= alpha[nt][0];
@@ -412,9 +438,9 @@ __device__ __forceinline__ void tile_page_q8(uint32_t kb, uint32_t vb, const flo
       }
   }
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < kG; ++j) {
     uint32_t R[4];
-    ldmatrix_x4_trans(R, vb + swz8(tok, 2 * j + hi16));
+    ldmatrix_x4_trans(R, vb + swz_rows<D>(tok, 2 * j + hi16));
     // R[0]: tokens 0-7, R[1]: tokens 8-15 (channels 32j..+15); R[2], R[3]: +16
     uint32_t A[2][4];
 #pragma unroll

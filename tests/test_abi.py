@@ -203,7 +203,7 @@ def decode8(fmt, step=False, **kw):
 @pytest.mark.parametrize("fmt", ["fp8", "int8"])
 @pytest.mark.parametrize("step", [False, True])
 @pytest.mark.parametrize("kw,status", [
-    (dict(d=64), kvd.KVD_ERR_UNSUPPORTED),                 # the 8-bit tile is d = 128 only
+    (dict(d=96), kvd.KVD_ERR_UNSUPPORTED),                 # the 8-bit tile is d = 64 or 128
     (dict(ks=NULL), kvd.KVD_ERR_INVALID),
     (dict(vs=NULL), kvd.KVD_ERR_INVALID),
     (dict(ks=ctypes.c_void_p(256 + 8)), kvd.KVD_ERR_INVALID),   # scale pools 16-byte aligned

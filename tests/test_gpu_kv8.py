@@ -70,6 +70,64 @@ def test_quantize_bit_exact(kvd, fmt, dtype, d):
     assert np.array_equal(host(scales).view(np.uint32), os_.view(np.uint32))
 
 
+def oracle_q8(w, fmt, si=None):
+    """The oracle's own 8-bit pools: its quantisation of the workload's whole
+    16-bit pool and, with step inputs si, its quantising append of the step's
+    rows -- no input from the GPU."""
+    k8, ks = orc_fn("quantize", fmt)(to_words(w.k_cache), odt(w))
+    v8, vs = orc_fn("quantize", fmt)(to_words(w.v_cache), odt(w))
+    if si is not None:
+        orc_fn("append", fmt)(k8, v8, ks, vs, w.block_table.numpy(), si["slot"].cpu().numpy(),
+                              to_words(si["k_new"]), to_words(si["v_new"]), odt(w))
+    return k8, v8, ks, vs
+
+
+def oracle_q8_rows(w, fmt, si, rows):
+    """oracle_q8 for a few sequences of a large workload: only the pages
+    they use, renumbered (returns the pools, their block table and the page
+    list, so the GPU's pools can be compared page for page)."""
+    bt = w.block_table.cpu()
+    n = si["seq_lens"].cpu()
+    npg = [(int(n[b]) + 15) // 16 for b in rows]
+    pages = sorted({int(p) for b, m in zip(rows, npg) for p in bt[b, :m].tolist()})
+    remap = {p: i for i, p in enumerate(pages)}
+    bts = np.zeros((len(rows), max(npg)), dtype=np.int32)
+    for i, (b, m) in enumerate(zip(rows, npg)):
+        bts[i, :m] = [remap[p] for p in bt[b, :m].tolist()]
+    idx = torch.tensor(pages, dtype=torch.long, device=w.k_cache.device)
+    kw, vw = to_words(w.k_cache.index_select(0, idx)), to_words(w.v_cache.index_select(0, idx))
+    k8, ks = orc_fn("quantize", fmt)(kw, odt(w))
+    v8, vs = orc_fn("quantize", fmt)(vw, odt(w))
+    sel = torch.tensor(rows, dtype=torch.long)
+    orc_fn("append", fmt)(k8, v8, ks, vs, bts, si["slot"].cpu()[sel].numpy(),
+                          to_words(si["k_new"].cpu()[sel]), to_words(si["v_new"].cpu()[sel]), odt(w))
+    return (k8, v8, ks, vs), bts, pages
+
+
+def data_rows(k_cache, v_cache, block_table=None, si=None):
+    """Bool [NB, H_kv, 16]: pool rows holding data -- rows of the 16-bit pool
+    that are not the NaN canary of never-written slots, plus the rows the
+    step appends.  The canary's 8-bit encoding (which NaN code, which NaN
+    scale) is a convention nothing reads, so pools are compared on these."""
+    m = (torch.isfinite(k_cache.float()).all(-1) & torch.isfinite(v_cache.float()).all(-1)).cpu().numpy()
+    if si is not None:
+        slot = si["slot"].cpu().numpy()
+        bt = block_table.cpu().numpy() if torch.is_tensor(block_table) else block_table
+        for b, pos in enumerate(slot):
+            if pos >= 0:
+                m[bt[b, pos // 16], :, pos % 16] = True
+    return m
+
+
+def assert_pools_equal(gpu, orc, rows):
+    """8-bit codes and fp32 scales, bit for bit, on the rows holding data."""
+    for g, o in zip(gpu, orc):
+        g = host(g) if torch.is_tensor(g) else g
+        if g.dtype == np.float32:
+            g, o = g.view(np.uint32), o.view(np.uint32)
+        assert np.array_equal(g[rows], o[rows])
+
+
 def q8_state(kvd, w, fmt):
     """Quantise the workload's 16-bit pools on the GPU."""
     k8, ks = gpu_fn(kvd, "quantize", fmt)(w.k_cache.cuda())
@@ -82,16 +140,13 @@ def test_append_bit_exact_whole_pool(kvd, fmt):
     w = build_workload("a8", 5, 8, 4, 128, "bf16", [1, 16, 17, 40, 0], seed=1201, spare_pages=3)
     si = step_inputs(w, 0)
     k8, v8, ks, vs = q8_state(kvd, w, fmt)
-    hk8, hv8, hks, hvs = host(k8), host(v8), host(ks), host(vs)
     bt = w.block_table.cuda()
     gpu_fn(kvd, "append", fmt)(k8, v8, ks, vs, bt, si["slot"].cuda(), si["k_new"].cuda(),
                                si["v_new"].cuda())
     torch.cuda.synchronize()
-    orc_fn("append", fmt)(hk8, hv8, hks, hvs, w.block_table.numpy(), si["slot"].numpy(),
-                          to_words(si["k_new"]), to_words(si["v_new"]), oracle.BF16)
-    assert np.array_equal(host(k8), hk8) and np.array_equal(host(v8), hv8)
-    assert np.array_equal(host(ks).view(np.uint32), hks.view(np.uint32))
-    assert np.array_equal(host(vs).view(np.uint32), hvs.view(np.uint32))
+    hk8, hv8, hks, hvs = oracle_q8(w, fmt, si)
+    assert_pools_equal((k8, v8, ks, vs), (hk8, hv8, hks, hvs),
+                       data_rows(w.k_cache, w.v_cache, w.block_table, si))
     assert kvd.kvd_read_device_error() == 0
 
 
@@ -119,7 +174,10 @@ def test_decode_matches_oracle(kvd, fmt, case):
     out = gpu_fn(kvd, "decode_attention", fmt)(si["q"].cuda(), k8, v8, ks, vs, bt, si["seq_lens"].cuda(),
                                                w.scale, num_partitions=parts, lse_out=lse)
     torch.cuda.synchronize()
-    ref, ref_lse = orc_fn("attend", fmt)(to_words(si["q"]), host(k8), host(v8), host(ks), host(vs),
+    hk8, hv8, hks, hvs = oracle_q8(w, fmt, si)
+    assert_pools_equal((k8, v8, ks, vs), (hk8, hv8, hks, hvs),
+                       data_rows(w.k_cache, w.v_cache, w.block_table, si))
+    ref, ref_lse = orc_fn("attend", fmt)(to_words(si["q"]), hk8, hv8, hks, hvs,
                                          w.block_table.numpy(), si["seq_lens"].numpy(), w.scale, odt(w))
     g = out.float().cpu().double().numpy()
     err = float(np.max(np.abs(g - ref)))
@@ -156,15 +214,16 @@ def test_decode_full_size_gqa70b(kvd, fmt):
     assert torch.isfinite(out.float()).all()
     lens = w.seq_lens0.numpy()
     rows = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 5, 40})
-    hk8, hv8, hks, hvs = host(k8), host(v8), host(ks), host(vs)
-    q = to_words(si["q"])
-    sl = si["seq_lens"].cpu().numpy()
-    btn = w.block_table.numpy()
-    worst = 0.0
-    for b in rows:
-        ref, _ = orc_fn("attend", fmt)(q[b:b + 1], hk8, hv8, hks, hvs, btn[b:b + 1], sl[b:b + 1],
-                                       w.scale, oracle.BF16)
-        worst = max(worst, float(np.max(np.abs(out[b].float().cpu().double().numpy() - ref[0]))))
+    (hk8, hv8, hks, hvs), bts, pages = oracle_q8_rows(w, fmt, si, rows)
+    idx = torch.tensor(pages, dtype=torch.long, device="cuda")
+    sel = torch.tensor(rows, dtype=torch.long)
+    rows_ok = data_rows(w.k_cache.index_select(0, idx), w.v_cache.index_select(0, idx), bts,
+                        {"slot": si["slot"].cpu()[sel]})
+    assert_pools_equal([t.index_select(0, idx) for t in (k8, v8, ks, vs)], (hk8, hv8, hks, hvs), rows_ok)
+    sel = torch.tensor(rows, dtype=torch.long)
+    ref, _ = orc_fn("attend", fmt)(to_words(si["q"].cpu()[sel]), hk8, hv8, hks, hvs, bts,
+                                   si["seq_lens"].cpu()[sel].numpy(), w.scale, oracle.BF16)
+    worst = float(np.max(np.abs(out.cpu()[sel].float().double().numpy() - ref)))
     print(f"gqa70b {fmt}: max abs error {worst:.3e} over sequences {rows}")
     assert worst <= TOL[w.dtype]
     assert kvd.kvd_read_device_error() == 0
@@ -188,7 +247,6 @@ def test_fused_step_matches_oracle_and_two_calls(kvd, fmt, case):
     si = step_inputs(w, 0)
     k8, v8, ks, vs = q8_state(kvd, w, fmt)
     two = [t.clone() for t in (k8, v8, ks, vs)]
-    hk8, hv8, hks, hvs = host(k8), host(v8), host(ks), host(vs)
     bt = w.block_table.cuda()
     q, kn, vn, sl = si["q"].cuda(), si["k_new"].cuda(), si["v_new"].cuda(), si["seq_lens"].cuda()
     lse = torch.empty((B, H_q), dtype=torch.float32, device="cuda")
@@ -199,11 +257,9 @@ def test_fused_step_matches_oracle_and_two_calls(kvd, fmt, case):
     out2 = gpu_fn(kvd, "decode_attention", fmt)(q, *two, bt, sl, w.scale, num_partitions=parts,
                                                 lse_out=lse2)
     torch.cuda.synchronize()
-    orc_fn("append", fmt)(hk8, hv8, hks, hvs, w.block_table.numpy(), si["slot"].numpy(),
-                          to_words(si["k_new"]), to_words(si["v_new"]), odt(w))
-    assert np.array_equal(host(k8), hk8) and np.array_equal(host(v8), hv8)
-    assert np.array_equal(host(ks).view(np.uint32), hks.view(np.uint32))
-    assert np.array_equal(host(vs).view(np.uint32), hvs.view(np.uint32))
+    hk8, hv8, hks, hvs = oracle_q8(w, fmt, si)
+    assert_pools_equal((k8, v8, ks, vs), (hk8, hv8, hks, hvs),
+                       data_rows(w.k_cache, w.v_cache, w.block_table, si))
     ref, ref_lse = orc_fn("attend", fmt)(to_words(si["q"]), hk8, hv8, hks, hvs, w.block_table.numpy(),
                                          si["seq_lens"].numpy(), w.scale, odt(w))
     err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
@@ -237,15 +293,16 @@ def test_fused_step_full_size_gqa70b(kvd, fmt):
     del two
     lens = w.seq_lens0.numpy()
     rows = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 7, 33})
-    hk8, hv8, hks, hvs = host(k8), host(v8), host(ks), host(vs)
-    q = to_words(si["q"])
-    sl = si["seq_lens"].cpu().numpy()
-    btn = w.block_table.numpy()
-    worst = 0.0
-    for b in rows:
-        ref, _ = orc_fn("attend", fmt)(q[b:b + 1], hk8, hv8, hks, hvs, btn[b:b + 1], sl[b:b + 1],
-                                       w.scale, oracle.BF16)
-        worst = max(worst, float(np.max(np.abs(out[b].float().cpu().double().numpy() - ref[0]))))
+    (hk8, hv8, hks, hvs), bts, pages = oracle_q8_rows(w, fmt, si, rows)
+    idx = torch.tensor(pages, dtype=torch.long, device="cuda")
+    sel = torch.tensor(rows, dtype=torch.long)
+    rows_ok = data_rows(w.k_cache.index_select(0, idx), w.v_cache.index_select(0, idx), bts,
+                        {"slot": si["slot"].cpu()[sel]})
+    assert_pools_equal([t.index_select(0, idx) for t in (k8, v8, ks, vs)], (hk8, hv8, hks, hvs), rows_ok)
+    sel = torch.tensor(rows, dtype=torch.long)
+    ref, _ = orc_fn("attend", fmt)(to_words(si["q"].cpu()[sel]), hk8, hv8, hks, hvs, bts,
+                                   si["seq_lens"].cpu()[sel].numpy(), w.scale, oracle.BF16)
+    worst = float(np.max(np.abs(out.cpu()[sel].float().double().numpy() - ref)))
     assert worst <= TOL[w.dtype], f"max abs error {worst}"
     assert kvd.kvd_read_device_error() == 0
 
@@ -277,16 +334,85 @@ def test_fused_step_maximum_batch(kvd, fmt):
     w = build_workload("max8", B, 8, 2, 128, "bf16", [int(x) for x in lens], seed=1501, spare_pages=4)
     si = step_inputs(w, 0)
     k8, v8, ks, vs = q8_state(kvd, w, fmt)
-    hk8, hv8, hks, hvs = host(k8), host(v8), host(ks), host(vs)
     bt = w.block_table.cuda()
     out = gpu_fn(kvd, "decode_step", fmt)(si["q"].cuda(), si["k_new"].cuda(), si["v_new"].cuda(), k8, v8,
                                           ks, vs, bt, si["seq_lens"].cuda(), w.scale)
     torch.cuda.synchronize()
-    orc_fn("append", fmt)(hk8, hv8, hks, hvs, w.block_table.numpy(), si["slot"].numpy(),
-                          to_words(si["k_new"]), to_words(si["v_new"]), odt(w))
-    assert np.array_equal(host(k8), hk8) and np.array_equal(host(v8), hv8)
-    assert np.array_equal(host(ks).view(np.uint32), hks.view(np.uint32))
-    assert np.array_equal(host(vs).view(np.uint32), hvs.view(np.uint32))
+    hk8, hv8, hks, hvs = oracle_q8(w, fmt, si)
+    assert_pools_equal((k8, v8, ks, vs), (hk8, hv8, hks, hvs),
+                       data_rows(w.k_cache, w.v_cache, w.block_table, si))
+    ref, _ = orc_fn("attend", fmt)(to_words(si["q"]), hk8, hv8, hks, hvs, w.block_table.numpy(),
+                                   si["seq_lens"].numpy(), w.scale, odt(w))
+    err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
+    assert err <= TOL[w.dtype], f"max abs error {err}"
+    assert kvd.kvd_read_device_error() == 0
+
+
+# ------------------------------------------------- 8-bit caches at d = 64
+
+CASES64 = [
+    # B, H_q, H_kv, dtype, lens, partitions
+    (4, 16, 16, "f16", [1, 15, 16, 300], 0),     # MHA, page edges
+    (3, 32, 8, "bf16", [513, 77, 1000], 0),      # group 4
+    (2, 16, 1, "bf16", [40, 130], 0),            # MQA, group 16 (two n-tiles)
+    (5, 16, 2, "f16", [3, 0, 45, 0, 200], 7),    # group 8, empty sequences, fixed partitions
+    (2, 24, 8, "bf16", [700, 31], 1),            # group 3, one partition
+]
+
+
+@pytest.mark.parametrize("case", CASES64, ids=lambda c: f"d64_B{c[0]}_Hq{c[1]}_Hkv{c[2]}_{c[3]}_N{c[5]}")
+def test_fused_step_d64_matches_oracle_and_two_calls(kvd, fmt, case):
+    # the 8-bit cache with 64-channel heads (two scale groups per token, 64-byte
+    # code rows): pools bit-exact against the oracle's quantising append, out
+    # within tolerance of its attention over them, and both bit-identical to
+    # the two-call path
+    B, H_q, H_kv, dtype, lens, parts = case
+    w = build_workload("s8d64", B, H_q, H_kv, 64, dtype, lens, seed=1600 + CASES64.index(case),
+                       spare_pages=2)
+    si = step_inputs(w, 0)
+    k8, v8, ks, vs = q8_state(kvd, w, fmt)
+    assert ks.shape[-1] == 2
+    two = [t.clone() for t in (k8, v8, ks, vs)]
+    bt = w.block_table.cuda()
+    q, kn, vn, sl = si["q"].cuda(), si["k_new"].cuda(), si["v_new"].cuda(), si["seq_lens"].cuda()
+    lse = torch.empty((B, H_q), dtype=torch.float32, device="cuda")
+    out = gpu_fn(kvd, "decode_step", fmt)(q, kn, vn, k8, v8, ks, vs, bt, sl, w.scale,
+                                          num_partitions=parts, lse_out=lse)
+    gpu_fn(kvd, "append", fmt)(*two, bt, si["slot"].cuda(), kn, vn)
+    out2 = gpu_fn(kvd, "decode_attention", fmt)(q, *two, bt, sl, w.scale, num_partitions=parts)
+    torch.cuda.synchronize()
+    hk8, hv8, hks, hvs = oracle_q8(w, fmt, si)
+    assert_pools_equal((k8, v8, ks, vs), (hk8, hv8, hks, hvs),
+                       data_rows(w.k_cache, w.v_cache, w.block_table, si))
+    ref, ref_lse = orc_fn("attend", fmt)(to_words(si["q"]), hk8, hv8, hks, hvs, w.block_table.numpy(),
+                                         si["seq_lens"].numpy(), w.scale, odt(w))
+    err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
+    assert err <= TOL[w.dtype], f"max abs error {err}"
+    fin = np.isfinite(ref_lse)
+    gl = lse.cpu().double().numpy()
+    assert np.array_equal(np.isfinite(gl), fin)
+    assert np.max(np.abs(gl[fin] - ref_lse[fin])) <= LSE_TOL
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert torch.all(out[b] == 0)
+    for a, b in zip((k8, v8, ks, vs), two):
+        assert torch.equal(_bits(a), _bits(b))
+    assert torch.equal(_bits(out), _bits(out2))
+    assert kvd.kvd_read_device_error() == 0
+
+
+def test_decode_d64_larger_batch_every_row(kvd, fmt):
+    # 16 sequences of 64-channel heads, 32 query / 8 KV heads, lengths over
+    # many pages and ragged tails: every row against the oracle
+    lens = [2000 - 97 * i for i in range(16)]
+    w = build_workload("b8d64", 16, 32, 8, 64, "bf16", lens, seed=1650, spare_pages=3)
+    si = step_inputs(w, 0)
+    k8, v8, ks, vs = q8_state(kvd, w, fmt)
+    bt = w.block_table.cuda()
+    out = gpu_fn(kvd, "decode_step", fmt)(si["q"].cuda(), si["k_new"].cuda(), si["v_new"].cuda(), k8, v8,
+                                          ks, vs, bt, si["seq_lens"].cuda(), w.scale)
+    torch.cuda.synchronize()
+    hk8, hv8, hks, hvs = oracle_q8(w, fmt, si)
     ref, _ = orc_fn("attend", fmt)(to_words(si["q"]), hk8, hv8, hks, hvs, w.block_table.numpy(),
                                    si["seq_lens"].numpy(), w.scale, odt(w))
     err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
