@@ -74,6 +74,17 @@ def load(path):
     L.orc_attend_int8.restype = i32
     L.orc_attend_int8.argtypes = [P, P, P, P, P, P, P, ctypes.c_double, i32, i32, i32, i32, i32,
                                   i32, i32, P, P, i32]
+    L.orc_int4_decode.restype = ctypes.c_double
+    L.orc_int4_decode.argtypes = [ctypes.c_uint8]
+    L.orc_int4_encode.restype = ctypes.c_uint8
+    L.orc_int4_encode.argtypes = [ctypes.c_float]
+    L.orc_quantize_int4.restype = i32
+    L.orc_quantize_int4.argtypes = [P, i32, i32, i32, P, P]
+    L.orc_append_int4.restype = i32
+    L.orc_append_int4.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32]
+    L.orc_attend_int4.restype = i32
+    L.orc_attend_int4.argtypes = [P, P, P, P, P, P, P, ctypes.c_double, i32, i32, i32, i32, i32,
+                                  i32, i32, P, P, i32]
     return L
 
 
@@ -287,3 +298,57 @@ def attend_int8(q, k8, v8, ks, vs, block_table, seq_lens, scale, dtype, nthreads
     """Attention (binary64) over the dequantised INT8 cache -> (out, lse)."""
     return _attend8("orc_attend_int8", q, k8, v8, ks, vs, block_table, seq_lens, scale, dtype,
                     nthreads)
+
+
+# ------------------------------------------------------------ 4-bit KV cache
+
+def int4_decode(nibble):
+    return lib().orc_int4_decode(int(nibble))
+
+
+def int4_encode(x):
+    return int(lib().orc_int4_encode(float(x)))
+
+
+def quantize_int4(rows, dtype):
+    """rows [..., d] storage words -> (packed codes uint8 [..., d/2]: channel 2i
+    in the low nibble of byte i, 2i+1 in its high nibble; scales [..., d/32])."""
+    rows = _words(rows)
+    d = rows.shape[-1]
+    n = rows.size // d
+    codes = np.zeros(rows.shape[:-1] + (d // 2,), dtype=np.uint8)
+    scales = np.zeros(rows.shape[:-1] + (d // FP8_GROUP,), dtype=np.float32)
+    _check(lib().orc_quantize_int4(_ptr(rows), n, d, dtype, _ptr(codes), _ptr(scales)),
+           "orc_quantize_int4")
+    return codes, scales
+
+
+def append_int4(k4, v4, ks, vs, block_table, slot, k_new, v_new, dtype):
+    """In-place INT4 quantised scatter into packed codes [NB,H_kv,16,d/2] and
+    scales [NB,H_kv,16,d/32]."""
+    for a in (k4, v4):
+        assert a.dtype == np.uint8 and a.flags.c_contiguous
+    for a in (ks, vs):
+        assert a.dtype == np.float32 and a.flags.c_contiguous
+    k_new, v_new = _words(k_new), _words(v_new)
+    bt, sl = _i32(block_table), _i32(slot)
+    NB, H_kv, P, half = k4.shape
+    _check(lib().orc_append_int4(_ptr(k4), _ptr(v4), _ptr(ks), _ptr(vs), _ptr(bt), _ptr(sl),
+                                 _ptr(k_new), _ptr(v_new), k_new.shape[0], H_kv, 2 * half, NB,
+                                 bt.shape[1], dtype), "orc_append_int4")
+
+
+def attend_int4(q, k4, v4, ks, vs, block_table, seq_lens, scale, dtype, nthreads=0):
+    """Attention (binary64) over the dequantised INT4 cache -> (out, lse)."""
+    q = _words(q)
+    bt, sl = _i32(block_table), _i32(seq_lens)
+    B, H_q, d = q.shape
+    NB, H_kv, P, _ = k4.shape
+    out = np.zeros((B, H_q, d), dtype=np.float64)
+    lse = np.zeros((B, H_q), dtype=np.float64)
+    _check(lib().orc_attend_int4(_ptr(q), _ptr(np.ascontiguousarray(k4)), _ptr(np.ascontiguousarray(v4)),
+                                 _ptr(np.ascontiguousarray(ks)), _ptr(np.ascontiguousarray(vs)),
+                                 _ptr(bt), _ptr(sl), float(scale), B, H_q, H_kv, d, NB,
+                                 bt.shape[1], dtype, _ptr(out), _ptr(lse), int(nthreads)),
+           "orc_attend_int4")
+    return out, lse

@@ -31,6 +31,10 @@
  *   orc_quantize_int8 / orc_append_int8 / orc_attend_int8
  *                                     -- half-step round trip, extreme -> +-127,
  *                                        CPU float64 SDPA on the dequantised cache
+ *   orc_int4_decode / orc_int4_encode -- two's complement nibbles; closed-form roundings
+ *   orc_quantize_int4 / orc_append_int4 / orc_attend_int4
+ *                                     -- half-step round trip, extreme -> +-7, nibble
+ *                                        order, CPU float64 SDPA on the dequantised cache
  */
 #include <math.h>
 #include <stdint.h>
@@ -394,14 +398,16 @@ int orc_quantize_fp8(const uint16_t *rows, int n, int d, int dtype, uint8_t *cod
  * [NB][H_kv][16][d/32]). */
 typedef int (*orc_quant_fn)(const uint16_t *, int, int, int, uint8_t *, float *);
 
-static int append_kv8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t *block_table,
-                      const int32_t *slot, const uint16_t *k_new, const uint16_t *v_new, int B,
-                      int H_kv, int d, int num_blocks, int max_blocks, int dtype, orc_quant_fn quant)
+/* row_bytes: bytes of codes per cache row (d for 8-bit codes, d / 2 for 4-bit). */
+static int append_codes(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t *block_table,
+                        const int32_t *slot, const uint16_t *k_new, const uint16_t *v_new, int B,
+                        int H_kv, int d, int row_bytes, int num_blocks, int max_blocks, int dtype,
+                        orc_quant_fn quant)
 {
     if (!k8 || !v8 || !ks || !vs || !block_table || !slot || !k_new || !v_new) return ORC_ERR_ARGS;
     if (d % ORC_FP8_GROUP) return ORC_ERR_ARGS;
     const int ng = d / ORC_FP8_GROUP;
-    uint8_t *code = (uint8_t *)malloc((size_t)d);
+    uint8_t *code = (uint8_t *)malloc((size_t)row_bytes);
     float *sc = (float *)malloc((size_t)ng * sizeof(float));
     if (!code || !sc) { free(code); free(sc); return ORC_ERR_NOMEM; }
     int rc = ORC_OK;
@@ -416,16 +422,24 @@ static int append_kv8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int3
             size_t r = ((size_t)phys * H_kv + h) * ORC_PAGE_TOKENS + row;
             size_t src = ((size_t)b * H_kv + h) * (size_t)d;
             quant(k_new + src, 1, d, dtype, code, sc);
-            memcpy(k8 + r * d, code, (size_t)d);
+            memcpy(k8 + r * row_bytes, code, (size_t)row_bytes);
             memcpy(ks + r * ng, sc, (size_t)ng * sizeof(float));
             quant(v_new + src, 1, d, dtype, code, sc);
-            memcpy(v8 + r * d, code, (size_t)d);
+            memcpy(v8 + r * row_bytes, code, (size_t)row_bytes);
             memcpy(vs + r * ng, sc, (size_t)ng * sizeof(float));
         }
     }
     free(code);
     free(sc);
     return rc;
+}
+
+static int append_kv8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t *block_table,
+                      const int32_t *slot, const uint16_t *k_new, const uint16_t *v_new, int B,
+                      int H_kv, int d, int num_blocks, int max_blocks, int dtype, orc_quant_fn quant)
+{
+    return append_codes(k8, v8, ks, vs, block_table, slot, k_new, v_new, B, H_kv, d, d, num_blocks,
+                        max_blocks, dtype, quant);
 }
 
 int orc_append_fp8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t *block_table,
@@ -440,10 +454,20 @@ int orc_append_fp8(uint8_t *k8, uint8_t *v8, float *ks, float *vs, const int32_t
  * the dequantised values s * dec(code) (binary64).  q is fp16/bf16 words. */
 typedef double (*orc_dec_fn)(uint8_t);
 
+/* Value of channel i of cache row `row` (codes of `bits` bits: 8 -- one code
+ * per byte, dec(byte); 4 -- two per byte, channel i in the low nibble of
+ * byte i / 2 when i is even, in its high nibble when i is odd). */
+static double code_value(const uint8_t *codes, long long row, int d, int i, int bits, orc_dec_fn dec)
+{
+    if (bits == 8) return dec(codes[row * d + i]);
+    uint8_t byte = codes[row * (d / 2) + i / 2];
+    return dec((uint8_t)((i % 2 == 0) ? (byte & 15) : (byte >> 4)));
+}
+
 static int attend_kv8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, const float *ks,
                       const float *vs, const int32_t *block_table, const int32_t *seq_lens,
                       double scale, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks,
-                      int dtype, double *out, double *lse, int nthreads, orc_dec_fn dec)
+                      int dtype, double *out, double *lse, int nthreads, orc_dec_fn dec, int bits)
 {
     if (!q || !k8 || !v8 || !ks || !vs || !block_table || !seq_lens || !out) return ORC_ERR_ARGS;
     if (B < 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv || d <= 0 || d % ORC_FP8_GROUP) return ORC_ERR_ARGS;
@@ -473,7 +497,7 @@ static int attend_kv8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, c
             const float *sk = ks + off / d * ng;
             double dot = 0.0;
             for (int i = 0; i < d; ++i)
-                dot += qv[i] * ((double)sk[i / ORC_FP8_GROUP] * dec(k8[off + i]));
+                dot += qv[i] * ((double)sk[i / ORC_FP8_GROUP] * code_value(k8, off / d, d, i, bits, dec));
             s[j] = scale * dot;
         }
         if (bad) { free(s); free(qv); status = ORC_ERR_RANGE; continue; }
@@ -486,7 +510,7 @@ static int attend_kv8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, c
             long long off = token_offset(block_table, b, j, g, H_kv, d, num_blocks, max_blocks);
             const float *sv = vs + off / d * ng;
             for (int i = 0; i < d; ++i)
-                o[i] += w * ((double)sv[i / ORC_FP8_GROUP] * dec(v8[off + i]));
+                o[i] += w * ((double)sv[i / ORC_FP8_GROUP] * code_value(v8, off / d, d, i, bits, dec));
         }
         for (int i = 0; i < d; ++i) o[i] /= den;
         if (lse) lse[r] = m + log(den);
@@ -502,7 +526,7 @@ int orc_attend_fp8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, cons
                    int dtype, double *out, double *lse, int nthreads)
 {
     return attend_kv8(q, k8, v8, ks, vs, block_table, seq_lens, scale, B, H_q, H_kv, d, num_blocks,
-                      max_blocks, dtype, out, lse, nthreads, orc_e4m3_decode);
+                      max_blocks, dtype, out, lse, nthreads, orc_e4m3_decode, 8);
 }
 
 /* Symmetric INT8 codes.  "KV Cache:推理慢的真正原因", section "工程优化手段 /
@@ -566,7 +590,81 @@ int orc_attend_int8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, con
                     int dtype, double *out, double *lse, int nthreads)
 {
     return attend_kv8(q, k8, v8, ks, vs, block_table, seq_lens, scale, B, H_q, H_kv, d, num_blocks,
-                      max_blocks, dtype, out, lse, nthreads, orc_int8_decode);
+                      max_blocks, dtype, out, lse, nthreads, orc_int8_decode, 8);
+}
+
+/* Symmetric INT4 codes, two per byte.  "KV Cache:推理慢的真正原因", section
+ * "工程优化手段 / 量化" (int4 storage, scales per channel group because of
+ * outlier keys); "推理速度慢怎么办？KV Cache与Flash Attention如何加速大模型推理",
+ * section "三、实际落地" (the cache kept in INT8 or even INT4).  Reading taken
+ * here: the INT8 cache's definition with 7 in place of 127 -- one fp32 scale
+ * per (token, KV head, 32-channel group), s = max|x| / 7 (fp32 division),
+ * code = x / s (fp32 division) rounded to the nearest integer, ties to even,
+ * clamped to [-7, 7]; a NaN quotient gives 0; a group of zeros gets s = 0 and
+ * codes 0.  Packing: channel 2i is the low nibble of byte i and channel
+ * 2i + 1 its high nibble, each a 4-bit two's complement integer.  Dequantised
+ * value: s * code. */
+double orc_int4_decode(uint8_t nib)
+{
+    int v = nib & 15;
+    return (double)(v >= 8 ? v - 16 : v);
+}
+
+uint8_t orc_int4_encode(float x)
+{
+    if (isnan(x)) return 0;
+    double r = rint((double)x);               /* nearest, ties to even */
+    if (r > 7.0) r = 7.0;
+    if (r < -7.0) r = -7.0;
+    return (uint8_t)((int)r & 15);
+}
+
+/* Quantise n rows of d storage words into packed codes [n][d / 2] and
+ * scales [n][d / 32]. */
+int orc_quantize_int4(const uint16_t *rows, int n, int d, int dtype, uint8_t *codes, float *scales)
+{
+    if (!rows || !codes || !scales || n < 0 || d <= 0 || d % ORC_FP8_GROUP) return ORC_ERR_ARGS;
+    const int ng = d / ORC_FP8_GROUP;
+    for (long long r = 0; r < n; ++r) {
+        for (int g = 0; g < ng; ++g) {
+            const uint16_t *x = rows + r * d + g * ORC_FP8_GROUP;
+            float mx = 0.0f;
+            for (int i = 0; i < ORC_FP8_GROUP; ++i) {
+                float v = (float)fabs(decode_elem(x[i], dtype));
+                if (v > mx) mx = v;
+            }
+            volatile float s = mx / 7.0f;
+            scales[r * ng + g] = s;
+            for (int i = 0; i < ORC_FP8_GROUP; ++i) {
+                float v = (float)decode_elem(x[i], dtype);
+                volatile float qt = s == 0.0f ? 0.0f : v / s;
+                uint8_t nib = s == 0.0f ? 0 : orc_int4_encode(qt);
+                int ch = g * ORC_FP8_GROUP + i;          /* channel within the row */
+                uint8_t *byte = codes + r * (d / 2) + ch / 2;
+                if (ch % 2 == 0) *byte = (uint8_t)((*byte & 0xF0) | nib);
+                else *byte = (uint8_t)((*byte & 0x0F) | (nib << 4));
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+int orc_append_int4(uint8_t *k4, uint8_t *v4, float *ks, float *vs, const int32_t *block_table,
+                    const int32_t *slot, const uint16_t *k_new, const uint16_t *v_new, int B,
+                    int H_kv, int d, int num_blocks, int max_blocks, int dtype)
+{
+    if (d % 2) return ORC_ERR_ARGS;
+    return append_codes(k4, v4, ks, vs, block_table, slot, k_new, v_new, B, H_kv, d, d / 2,
+                        num_blocks, max_blocks, dtype, orc_quantize_int4);
+}
+
+int orc_attend_int4(const uint16_t *q, const uint8_t *k4, const uint8_t *v4, const float *ks,
+                    const float *vs, const int32_t *block_table, const int32_t *seq_lens,
+                    double scale, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks,
+                    int dtype, double *out, double *lse, int nthreads)
+{
+    return attend_kv8(q, k4, v4, ks, vs, block_table, seq_lens, scale, B, H_q, H_kv, d, num_blocks,
+                      max_blocks, dtype, out, lse, nthreads, orc_int4_decode, 4);
 }
 
 int orc_max_threads(void)

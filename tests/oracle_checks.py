@@ -577,6 +577,125 @@ def check_append_int8():
     assert not changed.any(), "int8 append touched other rows"
 
 
+# ------------------------------------------------------------ INT4 cache
+
+def _unpack4(codes):
+    """Packed INT4 bytes [..., d/2] -> code values [..., d] in float64: channel
+    2i is the low nibble of byte i, 2i+1 its high nibble, two's complement
+    (numpy only, independent of the oracle)."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    lo = (c & 15).astype(np.int64)
+    hi = (c >> 4).astype(np.int64)
+    v = np.stack([lo, hi], axis=-1).reshape(c.shape[:-1] + (2 * c.shape[-1],))
+    return np.where(v >= 8, v - 16, v).astype(np.float64)
+
+
+def check_int4_decoder():
+    got = np.array([oracle.int4_decode(n) for n in range(16)])
+    assert np.array_equal(got, np.array([0, 1, 2, 3, 4, 5, 6, 7, -8, -7, -6, -5, -4, -3, -2, -1.0])), \
+        "INT4 decoding differs from 4-bit two's complement"
+
+
+def check_int4_encoder():
+    # closed forms: nearest integer, ties to the even one, clamp at +-7, NaN -> 0
+    cases = {2.5: 2, 3.5: 4, -2.5: -2, 0.5: 0, -0.5: 0, 1.5: 2, 6.5: 6, 6.6: 7, 7.4: 7, 7.5: 7,
+             100.0: 7, -100.0: -7, -7.6: -7, -6.5: -6, 4.49: 4, -4.51: -5, 0.0: 0}
+    for x, want in cases.items():
+        n = oracle.int4_encode(x)
+        assert 0 <= n < 16, f"INT4 encode({x}) is not a nibble: {n}"
+        got = n - 16 if n >= 8 else n
+        assert got == want, f"INT4 encode({x}) = {got}, expected {want}"
+    assert oracle.int4_encode(float("nan")) == 0
+    rng = np.random.default_rng(24)
+    x = rng.uniform(-7.4, 7.4, 3000).astype(np.float32)
+    got = np.array([oracle.int4_encode(v) for v in x])
+    got = np.where(got >= 8, got - 16, got)
+    assert np.all(np.abs(got - x.astype(np.float64)) <= 0.5), "INT4 encode is not the nearest integer"
+
+
+def check_quantize_int4():
+    rng = np.random.default_rng(25)
+    for dt, tdt in ((oracle.F16, torch.float16), (oracle.BF16, torch.bfloat16)):
+        x = torch.from_numpy(rng.standard_normal((64, 128)).astype(np.float32))
+        x[3, 17] = 40.0                        # an outlier channel in group 0 of row 3
+        x[5, 64:96] = 0.0                      # an all-zero group
+        x[9, 40] = float("nan")                # a NaN element (group 1 of row 9)
+        xq = x.to(tdt)
+        codes, scales = oracle.quantize_int4(to_words(xq), dt)
+        assert codes.shape == (64, 64) and scales.shape == (64, 4)
+        rows32 = xq.to(torch.float32).numpy().astype(np.float64)
+        q = _unpack4(codes)
+        deq = (q.reshape(64, 4, 32) * scales[..., None]).reshape(64, 128)
+        fin = np.isfinite(rows32)
+        step = scales.repeat(32, axis=1).astype(np.float64)
+        bound = step * (0.5 + 8 * 2.0 ** -24)
+        assert np.all(np.abs(deq - rows32)[fin] <= bound[fin]), "INT4 round trip exceeds half a step"
+        assert np.all(np.abs(q) <= 7), "an INT4 code outside [-7, 7]"
+        # the largest magnitude of each group is the extreme code, with its sign
+        g = np.where(fin, rows32, 0).reshape(64, 4, 32)
+        i = np.abs(g).argmax(axis=2)
+        ext = np.take_along_axis(q.reshape(64, 4, 32), i[..., None], 2)[..., 0]
+        sgn = np.sign(np.take_along_axis(g, i[..., None], 2)[..., 0])
+        nz = scales > 0
+        assert np.array_equal(ext[nz], 7 * sgn[nz]), "a group's extreme is not +-7"
+        assert scales[5, 2] == 0 and np.all(q[5, 64:96] == 0)
+        assert q[9, 40] == 0 and np.isfinite(scales[9, 1]) and scales[9, 1] > 0
+        assert scales[3, 0] > 10 * np.median(scales[:, 0]) and scales[3, 1] < 3 * np.median(scales[:, 1])
+    # packing: a row whose codes are known (x = code, max 7 -> s = 1): channel
+    # 2i in the low nibble of byte i, 2i+1 in the high one
+    want = np.array([(i % 15) - 7 for i in range(64)], dtype=np.float32)
+    want[0] = 7.0
+    codes, scales = oracle.quantize_int4(to_words(torch.from_numpy(want).to(torch.float16)), oracle.F16)
+    assert np.array_equal(scales, np.ones(2, dtype=np.float32))
+    lo = np.where(want[0::2] < 0, want[0::2] + 16, want[0::2]).astype(np.uint8)
+    hi = np.where(want[1::2] < 0, want[1::2] + 16, want[1::2]).astype(np.uint8)
+    assert np.array_equal(codes, lo | (hi << 4)), "INT4 nibble order"
+
+
+def check_attend_int4_against_sdpa():
+    for (B, H_q, H_kv, d, dt, lens, seed) in [(2, 8, 2, 128, "bf16", [40, 77], 43),
+                                              (1, 4, 4, 64, "f16", [33], 44)]:
+        c = case(B, H_q, H_kv, d, dt, lens, seed)
+        k4, ks = oracle.quantize_int4(c["kc"], c["dt"])
+        v4, vs = oracle.quantize_int4(c["vc"], c["dt"])
+        out, lse = oracle.attend_int4(c["q"], k4, v4, ks, vs, c["bt"], c["sl"], c["scale"], c["dt"])
+        G = H_q // H_kv
+        for b in range(B):
+            n = int(c["sl"][b])
+            j = np.arange(n)
+            pages, rows = c["bt"][b, j // 16], j % 16
+            Kd = _unpack4(k4[pages, :, rows, :]) * np.repeat(ks[pages, :, rows, :], 32, axis=-1)
+            Vd = _unpack4(v4[pages, :, rows, :]) * np.repeat(vs[pages, :, rows, :], 32, axis=-1)
+            K = torch.from_numpy(Kd.transpose(1, 0, 2)).repeat_interleave(G, dim=0)[None]
+            V = torch.from_numpy(Vd.transpose(1, 0, 2)).repeat_interleave(G, dim=0)[None]
+            q = torch.from_numpy(f64(c["q"][b], c["dt"]))[None, :, None, :]
+            ref = F.scaled_dot_product_attention(q, K, V, scale=c["scale"])[0, :, 0, :].numpy()
+            close(out[b], ref, 1e-12, 1e-12, "int4 attention vs SDPA on dequantised K/V")
+        full, _ = run(c)
+        assert np.max(np.abs(out - full)) < 0.5, "int4 attention far from fp16/bf16 attention"
+
+
+def check_append_int4():
+    w = build_workload("pin4i", 4, 4, 2, 128, "bf16", [1, 16, 17, 40], seed=85)
+    si = step_inputs(w, 0)
+    kc, vc = to_words(w.k_cache), to_words(w.v_cache)
+    k4, ks = oracle.quantize_int4(kc, oracle.BF16)
+    v4, vs = oracle.quantize_int4(vc, oracle.BF16)
+    k4_0, v4_0 = k4.copy(), v4.copy()
+    oracle.append_int4(k4, v4, ks, vs, w.block_table.numpy(), si["slot"].numpy(),
+                       to_words(si["k_new"]), to_words(si["v_new"]), oracle.BF16)
+    kn4, kns = oracle.quantize_int4(to_words(si["k_new"]), oracle.BF16)
+    vn4, vns = oracle.quantize_int4(to_words(si["v_new"]), oracle.BF16)
+    bt = w.block_table.numpy()
+    changed = np.any(k4 != k4_0, axis=(1, 3)) | np.any(v4 != v4_0, axis=(1, 3))
+    for b, pos in enumerate(si["slot"].numpy()):
+        p, r = bt[b, pos // 16], pos % 16
+        assert np.array_equal(k4[p, :, r, :], kn4[b]) and np.array_equal(ks[p, :, r, :], kns[b])
+        assert np.array_equal(v4[p, :, r, :], vn4[b]) and np.array_equal(vs[p, :, r, :], vns[b])
+        changed[p, r] = False
+    assert not changed.any(), "int4 append touched other rows"
+
+
 ALL_CHECKS = [
     check_f16_decoder,
     check_bf16_decoder,
@@ -601,4 +720,9 @@ ALL_CHECKS = [
     check_quantize_int8,
     check_attend_int8_against_sdpa,
     check_append_int8,
+    check_int4_decoder,
+    check_int4_encoder,
+    check_quantize_int4,
+    check_attend_int4_against_sdpa,
+    check_append_int4,
 ]

@@ -44,6 +44,15 @@ MUTANTS = {
     "int8_decode_unsigned": ("return (double)(int8_t)c;", "return (double)c;"),
     "int8_clamp": ("if (r > 127.0) r = 127.0;", "if (r > 128.0) r = 128.0;"),
     "int8_nan_code": ("if (isnan(x)) return 0;", "if (isnan(x)) return 0x7F;"),
+    "int4_scale_max": ("volatile float s = mx / 7.0f;", "volatile float s = mx / 8.0f;"),
+    "int4_clamp": ("if (r > 7.0) r = 7.0;", "if (r > 8.0) r = 8.0;"),
+    "int4_round_floor": ("double r = rint((double)x);               /* nearest, ties to even */\n    if (r > 7.0)",
+                         "double r = floor((double)x);               /* nearest, ties to even */\n    if (r > 7.0)"),
+    "int4_nibble_order": ("if (ch % 2 == 0) *byte = (uint8_t)((*byte & 0xF0) | nib);",
+                          "if (ch % 2 == 1) *byte = (uint8_t)((*byte & 0xF0) | nib);"),
+    "int4_decode_unsigned": ("return (double)(v >= 8 ? v - 16 : v);", "return (double)v;"),
+    "int4_value_nibble": ("return dec((uint8_t)((i % 2 == 0) ? (byte & 15) : (byte >> 4)));",
+                          "return dec((uint8_t)((i % 2 == 0) ? (byte >> 4) : (byte & 15)));"),
     "max_skips_first": ("for (int t = 0; t < n; ++t) if (s[t] > m) m = s[t];",
                         "for (int t = 1; t < n; ++t) if (s[t] > m) m = s[t];"),
 }
