@@ -50,10 +50,25 @@ def attention_bytes(w, seq_lens) -> int:
     return kv + 2 * w.B * w.H_q * w.d * s
 
 
-def fp8_attention_bytes(w, seq_lens) -> int:
-    """Attention bytes over the 8-bit cache: codes + fp32 group scales + q + out."""
-    per_tok = w.H_kv * 2 * (w.d + (w.d // 32) * 4)
+# quantised cache formats: the name of the code type, and the bytes of one
+# stored row of d channels (codes, then its fp32 scale per 32 channels)
+QUANT_NAMES = {"fp8": "E4M3", "int8": "INT8", "int4": "INT4"}
+
+
+def quant_row_bytes(fmt, d) -> int:
+    return (d // 2 if fmt == "int4" else d) + (d // 32) * 4
+
+
+def quant_attention_bytes(w, seq_lens, fmt) -> int:
+    """Attention bytes over a quantised cache: codes + fp32 group scales + q + out."""
+    per_tok = w.H_kv * 2 * quant_row_bytes(fmt, w.d)
     return int(seq_lens.to(torch.int64).sum().item()) * per_tok + 2 * w.B * w.H_q * w.d * 2
+
+
+def quant_append_bytes(w, slot, fmt) -> int:
+    """Quantising append: each K and V row read in 16 bits, written as codes + scales."""
+    rows = int((slot >= 0).sum().item()) * w.H_kv
+    return rows * 2 * (w.d * 2 + quant_row_bytes(fmt, w.d))
 
 
 def append_bytes(w, slot) -> int:
@@ -109,8 +124,9 @@ def source_hash() -> str:
 def profile_traffic(workload: str, mode: str):
     """DRAM bytes per decode launch from a committed ncu summary under
     profiles/, if one was taken on the current decode kernel sources for this
-    workload and step mode ("fused", "separate_append", "shared_prefix", "fp8",
-    "int8", "fp8_separate_append" or "int8_separate_append")."""
+    workload and step mode ("fused", "separate_append", "shared_prefix", or a
+    quantised format "fp8" / "int8" / "int4", optionally with
+    "_separate_append")."""
     try:
         names = sorted(os.listdir(PROFILE_DIR))
     except OSError:
@@ -172,9 +188,12 @@ class RowSnapshot:
         appended = int((self.slot >= 0).sum()) * w.H_kv
         self.nbytes = (tokens * w.H_kv * 2 * w.d * 2 + 2 * len(rows) * w.H_q * w.d * 2
                        + appended * w.d * 2 * 2 * 2)
-        # over an 8-bit cache: codes + per-32-channel fp32 scales
-        self.nbytes_q8 = (tokens * w.H_kv * 2 * (w.d + (w.d // 32) * 4) + 2 * len(rows) * w.H_q * w.d * 2
-                          + appended * 2 * (w.d * 2 + w.d + (w.d // 32) * 4))
+        self._q = (tokens * w.H_kv * 2, 2 * len(rows) * w.H_q * w.d * 2, appended * 2, w.d)
+
+    def nbytes_q(self, fmt):
+        """The bytes over a quantised cache: codes + per-32-channel fp32 scales."""
+        kv_rows, qo, app_rows, d = self._q
+        return kv_rows * quant_row_bytes(fmt, d) + qo + app_rows * (d * 2 + quant_row_bytes(fmt, d))
 
     def describe(self, w):
         return (f"sequences {self.rows} of {w.B} (lengths {self.seq_lens.tolist()}), all "
@@ -380,7 +399,7 @@ def oracle_parity(snap, gpu_rows, threads=0, fmt=None):
                                                   snap.scale, dt, nthreads=threads)
     spent = time.perf_counter() - t0
     err = float(np.max(np.abs(gpu_rows - ref))) if ref.size else 0.0
-    return err, spent, (snap.nbytes if fmt is None else snap.nbytes_q8) / spent / 1e9, threads
+    return err, spent, (snap.nbytes if fmt is None else snap.nbytes_q(fmt)) / spent / 1e9, threads
 
 
 ONE_THREAD_WORKLOADS = ("tiny", "long")
@@ -435,14 +454,15 @@ def run_reference(args):
 # shared-prefix mode): every synthetic configuration of the method's benchmark.
 PER_WORKLOADS = (("tiny", False, None), ("gqa70b", False, None), ("long", False, None),
                  ("cbatch", False, None), ("cbatch", True, None), ("mha7b", False, "fp8"),
-                 ("gqa70b", False, "fp8"), ("mha7b", False, "int8"), ("gqa70b", False, "int8"))
+                 ("gqa70b", False, "fp8"), ("mha7b", False, "int8"), ("gqa70b", False, "int8"),
+                 ("mha7b", False, "int4"), ("gqa70b", False, "int4"))
 
 
 def measure_workload(kvd, name, shared_prefix, dev, steps, warmup, fmt=None):
     """Time one workload's decode step through the call the headline uses
     (kvd_decode_step, the shared-prefix call with its fused append, or, with
-    fmt "fp8" / "int8", kvd_decode_step_{fmt} over the pool quantised to
-    that 8-bit cache) with automatic partitions: `warmup` untimed steps, then
+    fmt "fp8" / "int8" / "int4", kvd_decode_step_{fmt} over the pool
+    quantised to that cache) with automatic partitions: `warmup` untimed steps, then
     `steps` calls each bracketed by CUDA events on the launching stream.
     Returns (report dict, RowSnapshot of sampled sequences taken before any
     kernel ran, the GPU's output rows of those sequences as float64)."""
@@ -510,12 +530,12 @@ def measure_workload(kvd, name, shared_prefix, dev, steps, warmup, fmt=None):
         a_b -= w.groups * (w.B // w.groups - 1) * w.prefix_tokens * w.H_kv * 2 * w.d * 2
     nbytes = a_b + append_bytes(w, si["slot"].cpu())
     if q8 is not None:  # codes + scales read; appended rows read in 16 bits, written as codes + scales
-        rows = int((si["slot"] >= 0).sum().item()) * w.H_kv
-        nbytes = fp8_attention_bytes(w, si["seq_lens"].cpu()) + rows * 2 * (w.d * 2 + w.d + (w.d // 32) * 4)
+        nbytes = (quant_attention_bytes(w, si["seq_lens"].cpu(), fmt)
+                  + quant_append_bytes(w, si["slot"].cpu(), fmt))
     rep = {
         "workload": name + (" --shared-prefix" if shared_prefix else "") + (f" --kv-{fmt}" if fmt else ""),
         "call": ("kvd_decode_attention_shared_prefix (fused append)" if sp is not None
-                 else f"kvd_decode_step_{fmt} over the {'E4M3' if fmt == 'fp8' else 'INT8'} cache"
+                 else f"kvd_decode_step_{fmt} over the {QUANT_NAMES[fmt]} cache"
                  if q8 is not None else "kvd_decode_step"),
         "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
         "kv_dtype": w.dtype_name if q8 is None else f"{fmt} codes, {w.dtype_name} q/out",
@@ -574,16 +594,16 @@ def run_ours(args):
     stream0 = stream
 
     f8 = None
-    if args.kv_fp8 or args.kv_int8:
-        # the pool stored as 8-bit codes (E4M3 or INT8) + per-32-channel fp32 scales
-        fmt = "fp8" if args.kv_fp8 else "int8"
+    if args.kv_fp8 or args.kv_int8 or args.kv_int4:
+        # the pool stored as codes (E4M3, INT8 or packed INT4) + per-32-channel fp32 scales
+        fmt = "fp8" if args.kv_fp8 else "int8" if args.kv_int8 else "int4"
         k8, ks = getattr(kvd, "kvd_quantize_" + fmt)(kc)
         v8, vs = getattr(kvd, "kvd_quantize_" + fmt)(vc)
         f8 = {"fmt": fmt, "k8": k8, "v8": v8, "ks": ks, "vs": vs,
               "append": getattr(kvd, "kvd_append_" + fmt),
               "decode": getattr(kvd, "kvd_decode_attention_" + fmt),
               "step": getattr(kvd, "kvd_decode_step_" + fmt),
-              "name": "E4M3" if fmt == "fp8" else "INT8"}
+              "name": QUANT_NAMES[fmt]}
 
     sp = None
     if args.shared_prefix:
@@ -646,9 +666,9 @@ def run_ours(args):
         p_b = append_bytes(w, x["slot"])
         kv_tok = w.H_kv * 2 * w.d * 2  # K and V bytes per token of one sequence
         if f8 is not None:
-            a_b = fp8_attention_bytes(w, x["seq_lens"])
-            p_b = int((x["slot"] >= 0).sum().item()) * w.H_kv * 2 * (w.d * 2 + w.d + (w.d // 32) * 4)
-            kv_tok = w.H_kv * 2 * (w.d + (w.d // 32) * 4)
+            a_b = quant_attention_bytes(w, x["seq_lens"], f8["fmt"])
+            p_b = quant_append_bytes(w, x["slot"], f8["fmt"])
+            kv_tok = w.H_kv * 2 * quant_row_bytes(f8["fmt"], w.d)
         a_logical = a_b
         if w.groups:
             a_b -= w.groups * (w.B // w.groups - 1) * w.prefix_tokens * kv_tok
@@ -1011,13 +1031,15 @@ def parse_args(argv=None):
                    choices=["tiny", "mha7b", "gqa70b", "long", "cbatch"])
     p.add_argument("--partitions", type=int, default=0, help="0 = automatic")
     p.add_argument("--separate-append", action="store_true",
-                   help="time kvd_append[_fp8|_int8] + kvd_decode_attention[_fp8|_int8] instead of "
-                        "the fused kvd_decode_step[_fp8|_int8]")
+                   help="time kvd_append[_fp8|_int8|_int4] + kvd_decode_attention[_fp8|_int8|_int4] "
+                        "instead of the fused kvd_decode_step[_fp8|_int8|_int4]")
     p.add_argument("--e2e-steps", type=int, default=300)
     p.add_argument("--kv-fp8", action="store_true",
                    help="store the cache as FP8 E4M3 codes with per-32-channel scales (d=128)")
     p.add_argument("--kv-int8", action="store_true",
                    help="store the cache as INT8 codes with per-32-channel scales (d=128)")
+    p.add_argument("--kv-int4", action="store_true",
+                   help="store the cache as packed INT4 codes with per-32-channel scales (d=128)")
     p.add_argument("--shared-prefix", action="store_true",
                    help="read each group's shared prefix pages once (kvd_decode_attention_shared_prefix)")
     p.add_argument("--graph", action="store_true",
@@ -1037,10 +1059,11 @@ def parse_args(argv=None):
     args = p.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.graph and (args.separate_append or args.shared_prefix or args.kv_fp8 or args.kv_int8):
+    if args.graph and (args.separate_append or args.shared_prefix or args.kv_fp8 or args.kv_int8
+                       or args.kv_int4):
         raise SystemExit("--graph times the fused step only")
-    if args.kv_fp8 and args.kv_int8:
-        raise SystemExit("--kv-fp8 and --kv-int8 are exclusive")
+    if args.kv_fp8 + args.kv_int8 + args.kv_int4 > 1:
+        raise SystemExit("--kv-fp8, --kv-int8 and --kv-int4 are exclusive")
     return args
 
 

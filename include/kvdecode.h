@@ -247,6 +247,48 @@ kvd_status kvd_decode_attention_int8(const void *q, const int8_t *k_codes, const
                                      kvd_dtype dtype, void *stream);
 
 /*
+ * 4-bit (INT4) KV cache: symmetric codes, two per byte, with the per-group
+ * scales of the 8-bit caches.
+ * [BLOG] section "工程优化手段 / 量化" (quantise the cache from fp16 to int8 or
+ * int4, with scales per channel group because of outlier keys); [KVF] section
+ * "三、实际落地" (keys and values kept in INT8 or even INT4).
+ * Format: codes uint8 [num_blocks][H_kv][16][d/2] -- channel 2i is the low
+ * nibble of byte i, channel 2i+1 its high nibble, each a 4-bit two's
+ * complement integer; scales float [num_blocks][H_kv][16][d/32] with
+ * s = max|x| / 7 over the group and code = x / s rounded to the nearest
+ * integer (ties to even) and clamped to [-7, 7] (a NaN quotient gives 0;
+ * both divisions IEEE fp32); value = s * code.  d = 64 or 128 for attention.
+ * Bytes per (token, KV head) at d = 128: 64 of codes + 16 of scales.
+ *
+ * kvd_quantize_int4     n_rows rows of d values -> codes [n_rows][d/2] and
+ *                       scales [n_rows][d/32]
+ * kvd_append_int4       the quantising append (as kvd_append_int8)
+ * kvd_decode_attention_int4, kvd_decode_step_int4
+ *                       attention (and the fused step) over the INT4 cache,
+ *                       arguments as the _int8 calls
+ */
+kvd_status kvd_quantize_int4(const void *src, uint8_t *codes, float *scales, long long n_rows,
+                             int d, kvd_dtype dtype, void *stream);
+kvd_status kvd_append_int4(uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
+                           const int32_t *block_table, const int32_t *slot, const void *k_new,
+                           const void *v_new, int B, int H_kv, int d, int num_blocks,
+                           int max_blocks_per_seq, kvd_dtype dtype, void *stream);
+kvd_status kvd_decode_attention_int4(const void *q, const uint8_t *k_codes, const uint8_t *v_codes,
+                                     const float *k_scale, const float *v_scale,
+                                     const int32_t *block_table, const int32_t *seq_lens,
+                                     float scale, void *out, int B, int H_q, int H_kv, int d,
+                                     int num_blocks, int max_blocks_per_seq, int num_partitions,
+                                     void *workspace, size_t workspace_bytes, float *lse_out,
+                                     kvd_dtype dtype, void *stream);
+kvd_status kvd_decode_step_int4(const void *q, const void *k_new, const void *v_new,
+                                uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
+                                const int32_t *block_table, const int32_t *seq_lens, float scale,
+                                void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                                int max_blocks_per_seq, int num_partitions, void *workspace,
+                                size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+                                void *stream);
+
+/*
  * kvd_decode_step_fp8, kvd_decode_step_int8 -- kvd_decode_step over an 8-bit
  * cache: the quantising append of kvd_append_{fp8,int8} followed by the
  * attention of kvd_decode_attention_{fp8,int8}, in one decode launch.

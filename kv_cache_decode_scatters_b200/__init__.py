@@ -24,7 +24,8 @@ __all__ = [
     "kvd_decode_attention_shared_prefix", "kvd_shared_prefix_workspace_size",
     "kvd_quantize_fp8", "kvd_append_fp8", "kvd_decode_attention_fp8", "kvd_decode_step_fp8",
     "kvd_quantize_int8", "kvd_append_int8", "kvd_decode_attention_int8", "kvd_decode_step_int8",
-    "kvd_merge_lse",
+    "kvd_quantize_int4", "kvd_append_int4", "kvd_decode_attention_int4", "kvd_decode_step_int4",
+    "kvd_merge_lse", "kvd_read_stream", "kvd_set_decode_wait_limit", "KVD_READ_VECTOR", "KVD_READ_BULK",
     "kvd_workspace_size", "KVD_STATIC_WORKSPACE_BYTES",
     "kvd_auto_partitions", "kvd_kv_bytes_per_token", "kvd_read_device_error",
     "kvd_last_error", "alloc_workspace", "library_path", "lib",
@@ -63,7 +64,7 @@ def _load():
     L.kvd_shared_prefix_workspace_size.restype = S
     L.kvd_shared_prefix_workspace_size.argtypes = [I, I, I, I, I, I, I]
     LL = ctypes.c_longlong
-    for fmt in ("fp8", "int8"):
+    for fmt in ("fp8", "int8", "int4"):
         getattr(L, "kvd_quantize_" + fmt).restype = I
         getattr(L, "kvd_quantize_" + fmt).argtypes = [P, P, P, LL, I, I, P]
         getattr(L, "kvd_append_" + fmt).restype = I
@@ -290,14 +291,16 @@ def kvd_decode_attention_shared_prefix(q, k_cache, v_cache, block_table, seq_len
 
 # 8-bit KV caches: E4M3 codes (torch.uint8 storage) or INT8 codes (torch.int8),
 # one fp32 scale per (token, KV head, 32 channels).
-_CODE8 = {"fp8": torch.uint8, "int8": torch.int8}
+_CODE8 = {"fp8": torch.uint8, "int8": torch.int8, "int4": torch.uint8}
+# code bytes of a row of d values
+_ROW = {"fp8": lambda d: d, "int8": lambda d: d, "int4": lambda d: d // 2}
 
 
 def _quantize8(fmt, src, codes, scales, stream):
     d = src.shape[-1]
     n = src.numel() // d
     if codes is None:
-        codes = torch.empty(src.shape, dtype=_CODE8[fmt], device=src.device)
+        codes = torch.empty(src.shape[:-1] + (_ROW[fmt](d),), dtype=_CODE8[fmt], device=src.device)
     if scales is None:
         scales = torch.empty(src.shape[:-1] + (d // 32,), dtype=torch.float32, device=src.device)
     _check(getattr(_lib, "kvd_quantize_" + fmt)(
@@ -307,7 +310,8 @@ def _quantize8(fmt, src, codes, scales, stream):
 
 
 def _append8(fmt, k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, stream):
-    NB, H_kv, P, d = k_codes.shape
+    NB, H_kv, P, _ = k_codes.shape
+    d = k_new.shape[-1]
     B = k_new.shape[0]
     c = _CODE8[fmt]
     _check(getattr(_lib, "kvd_append_" + fmt)(
@@ -321,8 +325,8 @@ def _append8(fmt, k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, 
 def _decode8(fmt, q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
              num_partitions, workspace, lse_out, stream, k_new=None, v_new=None):
     B, H_q, d = q.shape
-    NB, H_kv, P, d2 = k_codes.shape
-    if P != KVD_PAGE_TOKENS or d2 != d:
+    NB, H_kv, P, rb = k_codes.shape
+    if P != KVD_PAGE_TOKENS or rb != _ROW[fmt](d):
         raise ValueError("q / cache shape mismatch")
     step = k_new is not None
     if step and (tuple(k_new.shape) != (B, H_kv, d) or v_new is None or v_new.shape != k_new.shape):
@@ -372,6 +376,34 @@ def kvd_decode_step_fp8(q, k_new, v_new, k_codes, v_codes, k_scale, v_scale, blo
     position seq_lens[b]-1 of every non-empty sequence, then attend
     (kvd_append_fp8 + kvd_decode_attention_fp8 in one launch).  Returns out."""
     return _decode8("fp8", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
+                    num_partitions, workspace, lse_out, stream, k_new, v_new)
+
+
+def kvd_quantize_int4(src, codes=None, scales=None, stream=None):
+    """Quantise rows src [..., d] (fp16/bf16) into INT4 codes, two per byte
+    (uint8 [..., d/2], channel 2i in the low nibble of byte i), and fp32
+    scales [..., d/32].  Returns (codes, scales)."""
+    return _quantize8("int4", src, codes, scales, stream)
+
+
+def kvd_append_int4(k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, stream=None):
+    """kvd_append for the INT4 cache (codes [NB,H_kv,16,d/2], scales [NB,H_kv,16,d/32])."""
+    _append8("int4", k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, stream)
+
+
+def kvd_decode_attention_int4(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale=None,
+                              out=None, num_partitions=0, workspace=None, lse_out=None, stream=None):
+    """kvd_decode_attention over the INT4 cache (d = 64 or 128).  Returns out."""
+    return _decode8("int4", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
+                    num_partitions, workspace, lse_out, stream)
+
+
+def kvd_decode_step_int4(q, k_new, v_new, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                         scale=None, out=None, num_partitions=0, workspace=None, lse_out=None,
+                         stream=None):
+    """kvd_decode_step over the INT4 cache (kvd_append_int4 + kvd_decode_attention_int4
+    in one launch).  Returns out."""
+    return _decode8("int4", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
                     num_partitions, workspace, lse_out, stream, k_new, v_new)
 
 

@@ -338,17 +338,20 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   for (int i = 0; i < 2; ++i) {
     CUresult r;
     if (q8) {
-      // 8-bit code pools as 2-D byte tensors {d, num_blocks*H_kv*16 rows};
-      // one box = the 16 rows of one page of one head, with the 128-byte
-      // (d = 128) or 64-byte (d = 64) swizzle.
-      cuuint64_t dims[2] = {static_cast<cuuint64_t>(d),
+      // code pools as 2-D byte tensors {row bytes, num_blocks*H_kv*16 rows}
+      // (row bytes: d for 8-bit codes, d / 2 for INT4); one box = the 16 rows
+      // of one page of one head, with the swizzle of its row size (128, 64
+      // or 32 bytes).
+      const int rb = fmt == kvd::Code8::INT4 ? d / 2 : d;
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>(rb),
                             static_cast<cuuint64_t>(num_blocks) * H_kv * KVD_PAGE_TOKENS};
-      cuuint64_t strides[1] = {static_cast<cuuint64_t>(d)};
-      cuuint32_t box[2] = {static_cast<cuuint32_t>(d), KVD_PAGE_TOKENS};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>(rb)};
+      cuuint32_t box[2] = {static_cast<cuuint32_t>(rb), KVD_PAGE_TOKENS};
       cuuint32_t estr[2] = {1, 1};
       r = encode(&tm[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(pools[i]), dims,
                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                 d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                 rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                           : (rb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B),
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     } else {
       // K and V pools as 3-D tensors {64 elements, d/64 units, num_blocks*H_kv*16
@@ -619,6 +622,43 @@ kvd_status kvd_decode_step_int8(const void *q, const void *k_new, const void *v_
                  reinterpret_cast<uint8_t *>(v_codes), k_scale, v_scale, block_table, seq_lens,
                  scale, out, B, H_q, H_kv, d, num_blocks, max_blocks_per_seq, num_partitions,
                  workspace, workspace_bytes, lse_out, dtype, stream, kvd::Code8::INT8);
+}
+
+kvd_status kvd_quantize_int4(const void *src, uint8_t *codes, float *scales, long long n_rows,
+                             int d, kvd_dtype dtype, void *stream) {
+  return quantize_q8(src, codes, scales, n_rows, d, dtype, stream, kvd::Code8::INT4);
+}
+
+kvd_status kvd_append_int4(uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
+                           const int32_t *block_table, const int32_t *slot, const void *k_new,
+                           const void *v_new, int B, int H_kv, int d, int num_blocks,
+                           int max_blocks_per_seq, kvd_dtype dtype, void *stream) {
+  return append_q8(k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new, v_new, B, H_kv, d,
+                   num_blocks, max_blocks_per_seq, dtype, stream, kvd::Code8::INT4);
+}
+
+kvd_status kvd_decode_attention_int4(const void *q, const uint8_t *k_codes, const uint8_t *v_codes,
+                                     const float *k_scale, const float *v_scale,
+                                     const int32_t *block_table, const int32_t *seq_lens,
+                                     float scale, void *out, int B, int H_q, int H_kv, int d,
+                                     int num_blocks, int max_blocks_per_seq, int num_partitions,
+                                     void *workspace, size_t workspace_bytes, float *lse_out,
+                                     kvd_dtype dtype, void *stream) {
+  return decode_q8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out, B, H_q,
+                   H_kv, d, num_blocks, max_blocks_per_seq, num_partitions, workspace,
+                   workspace_bytes, lse_out, dtype, stream, kvd::Code8::INT4);
+}
+
+kvd_status kvd_decode_step_int4(const void *q, const void *k_new, const void *v_new,
+                                uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
+                                const int32_t *block_table, const int32_t *seq_lens, float scale,
+                                void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                                int max_blocks_per_seq, int num_partitions, void *workspace,
+                                size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+                                void *stream) {
+  return step_q8(q, k_new, v_new, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale,
+                 out, B, H_q, H_kv, d, num_blocks, max_blocks_per_seq, num_partitions, workspace,
+                 workspace_bytes, lse_out, dtype, stream, kvd::Code8::INT4);
 }
 
 size_t kvd_shared_prefix_workspace_size(int B, int H_q, int H_kv, int d, int n_groups,

@@ -216,6 +216,96 @@ struct Page8 {
   }
 };
 
+// 4-bit pages (d = D = 64 or 128; INT4 codes, two per byte): codes
+// [16][D / 2] per (page, head) in one box with the 64-byte (D = 128) or
+// 32-byte (D = 64) swizzle, fp32 scales [16][D / 32] per (page, head) copied
+// alongside; output dtype T.
+template <int D, int NT, typename T>
+struct Page4 {
+  using Out = T;
+  static constexpr int kG = D / 32;                          // scale groups of a token
+  static constexpr int kRow = D / 2;                         // code bytes of a token
+  static constexpr int kPageBytes = kPage * kRow;            // codes of K (or V)
+  static constexpr int kScaleBytes = kPage * kG * 4;         // scales of K (or V)
+  static constexpr int kCopyBytes = 2 * kPageBytes + 2 * kScaleBytes;
+  static constexpr int kStride = 2 * kPageBytes;             // codes only: 1024-aligned stages
+  static constexpr int kAuxBytes = 2 * kScaleBytes;          // scales, in their own area
+  static_assert(kScaleBytes % 16 == 0, "scale rows are bulk copies of whole 16-byte units");
+  static __device__ __forceinline__ void issue(uint32_t dst, uint32_t aux, uint32_t bar,
+                                               const CUtensorMap *tmK, const CUtensorMap *tmV,
+                                               int row, uint64_t policy, const DecodeArgs &a) {
+    mbar_arrive_expect_tx(bar, kCopyBytes);
+    tma_load_2d(dst, tmK, 0, row, bar, policy);
+    tma_load_2d(dst + kPageBytes, tmV, 0, row, bar, policy);
+    bulk_load(aux, a.k_scale + static_cast<size_t>(row) * kG, kScaleBytes, bar);
+    bulk_load(aux + kScaleBytes, a.v_scale + static_cast<size_t>(row) * kG, kScaleBytes, bar);
+  }
+  static __device__ __forceinline__ void zero_tail(uint8_t *st, uint8_t *aux, int ntok, int lane) {
+    // V codes and V scales of masked rows (their zero weights times a NaN
+    // scale would otherwise poison the PV product)
+    const int n16 = (kPage - ntok) * kRow / 16;
+    uint4 *z = reinterpret_cast<uint4 *>(st + kPageBytes + ntok * kRow);
+    for (int i = lane; i < n16; i += 32) z[i] = make_uint4(0, 0, 0, 0);
+    float *zs = reinterpret_cast<float *>(aux + kScaleBytes) + ntok * kG;
+    for (int i = lane; i < (kPage - ntok) * kG; i += 32) zs[i] = 0.f;
+  }
+  // fused append: encode the new token of pair (b, h) exactly as the
+  // quantising append does (encode_row4), put its codes and scales into row t
+  // of the staged page and write them to the pools at row `row` + t
+  static __device__ __forceinline__ void patch(uint8_t *st, uint8_t *aux, int t, int lane,
+                                               const DecodeArgs &a, int b, int h, int row) {
+    const size_t src = (static_cast<size_t>(b) * a.H_kv + h) * D;
+    const size_t dst = static_cast<size_t>(row) + t;
+    const bool live = lane * 4 < D;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float sc;
+      const uint32_t w = encode_row4<T, Code8::INT4>(static_cast<const T *>(half ? a.v_new : a.k_new) + src,
+                                                     live, lane, sc);
+      if (live) {
+        // the lane's 4 codes are bytes 2 lane, 2 lane + 1 of the row
+        *reinterpret_cast<uint16_t *>(st + half * kPageBytes + swz_rows<kRow>(t, (2 * lane) >> 4) +
+                                      ((2 * lane) & 15)) = static_cast<uint16_t>(w);
+        *reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(half ? a.v_cache : a.k_cache) + dst * kRow +
+                                      2 * lane) = static_cast<uint16_t>(w);
+        if ((lane & 7) == 0) {
+          reinterpret_cast<float *>(aux + half * kScaleBytes)[t * kG + (lane >> 3)] = sc;
+          (half ? a.v_scale : a.k_scale)[dst * kG + (lane >> 3)] = sc;
+        }
+      }
+    }
+  }
+  static __device__ __forceinline__ void tile(uint8_t *st, uint8_t *aux, int ntok, float sl2, int lane,
+                                              const uint32_t (&qf)[NT][D / 16][2],
+                                              float (&acc)[NT][D / 16][4], float (&m)[NT][2],
+                                              float (&l)[NT][2]) {
+    const float *ks = reinterpret_cast<const float *>(aux);
+    tile_page_q4<D, NT>(smem_u32(st), smem_u32(st + kPageBytes), ks, ks + kPage * kG, ntok, sl2, lane,
+                        qf, acc, m, l);
+  }
+  static __device__ __forceinline__ uint32_t to_f16x2(uint32_t w) {
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w));
+      return f16pack(f.x, f.y);
+    } else {
+      return w;
+    }
+  }
+  // q in f16, channel order of the INT4 tile: in k-step 2j (2j + 1) of group
+  // j, k-slots 2 tig, 2 tig + 1 <- channels 32j + 8 tig + {0, 4} ({2, 6}) and
+  // k-slots 2 tig + 8, 2 tig + 9 <- channels 32j + 8 tig + {1, 5} ({3, 7})
+  static __device__ __forceinline__ void q_words(const uint32_t *qrow, int ks, int tig,
+                                                 uint32_t &w0, uint32_t &w1) {
+    const int base = (ks >> 1) * 16 + tig * 4 + (ks & 1);  // word of channels 8 tig + {0,1} or {2,3}
+    const uint32_t lo = to_f16x2(__ldg(qrow + base)), hi = to_f16x2(__ldg(qrow + base + 2));
+    w0 = __byte_perm(lo, hi, 0x5410);
+    w1 = __byte_perm(lo, hi, 0x7632);
+  }
+  static __device__ __forceinline__ int dim(int mt, int e, int g8) {
+    return (mt >> 1) * 32 + 4 * g8 + 2 * (mt & 1) + (e >> 1);
+  }
+};
+
 namespace {
 
 // Zero one output row of d elements (16-byte stores).
@@ -1158,6 +1248,51 @@ cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const 
   return launch_decode8_ws<D, NT, T, kFmt, W, S>(a, tmK, tmV, st, grid);
 }
 
+// 4-bit cache: d = 128 has 2 KB code stages, d = 64 1 KB; a parked
+// accumulator tile (8 NT D floats) must fit in a warp's stages.
+template <int D, int NT>
+struct Tune4;
+template <>
+struct Tune4<128, 1> {
+  static constexpr int W = 16, S = 2;
+};
+template <>
+struct Tune4<128, 2> {
+  static constexpr int W = 8, S = 4;
+};
+template <>
+struct Tune4<64, 1> {
+  static constexpr int W = 16, S = 4;
+};
+template <>
+struct Tune4<64, 2> {
+  static constexpr int W = 8, S = 4;
+};
+
+template <int D, int NT, typename T>
+cudaError_t launch_decode4_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                             cudaStream_t st, int grid) {
+  constexpr int W = Tune4<D, NT>::W, S = Tune4<D, NT>::S;
+  using Pol = Page4<D, NT, T>;
+  auto kern = decode_kernel<D, NT, Pol, W, S>;
+  const size_t smem = Geo<D, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(grid), dim3(32 * W), smem, st, a, tmK, tmV);
+}
+
+template <int D>
+cudaError_t launch_decode4_d(const DecodeArgs &a, DType dt, const CUtensorMap &tmK,
+                             const CUtensorMap &tmV, cudaStream_t s, int grid) {
+  const bool two = a.G > 8;
+  if (dt == DType::BF16)
+    return two ? launch_decode4_t<D, 2, __nv_bfloat16>(a, tmK, tmV, s, grid)
+               : launch_decode4_t<D, 1, __nv_bfloat16>(a, tmK, tmV, s, grid);
+  return two ? launch_decode4_t<D, 2, __half>(a, tmK, tmV, s, grid)
+             : launch_decode4_t<D, 1, __half>(a, tmK, tmV, s, grid);
+}
+
 template <int D, Code8 kFmt>
 cudaError_t launch_decode_q8_fmt(const DecodeArgs &a, DType dt, const CUtensorMap &tmK,
                                  const CUtensorMap &tmV, cudaStream_t s, int grid) {
@@ -1172,6 +1307,9 @@ cudaError_t launch_decode_q8_fmt(const DecodeArgs &a, DType dt, const CUtensorMa
 
 cudaError_t launch_decode_q8(const DecodeArgs &a, int d, DType dt, Code8 fmt, const CUtensorMap &tmK,
                              const CUtensorMap &tmV, cudaStream_t s, int grid) {
+  if (fmt == Code8::INT4)
+    return d == 64 ? launch_decode4_d<64>(a, dt, tmK, tmV, s, grid)
+                   : launch_decode4_d<128>(a, dt, tmK, tmV, s, grid);
   if (d == 64)
     return fmt == Code8::INT8 ? launch_decode_q8_fmt<64, Code8::INT8>(a, dt, tmK, tmV, s, grid)
                               : launch_decode_q8_fmt<64, Code8::E4M3>(a, dt, tmK, tmV, s, grid);

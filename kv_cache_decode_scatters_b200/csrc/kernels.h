@@ -10,8 +10,9 @@ namespace kvd {
 
 enum class DType { F16 = 0, BF16 = 1 };
 
-// formats of an 8-bit KV cache
-enum class Code8 { E4M3 = 0, INT8 = 1 };
+// code formats of a quantised KV cache: 8-bit E4M3 or INT8 codes (one per
+// byte), or 4-bit INT4 codes (two per byte)
+enum class Code8 { E4M3 = 0, INT8 = 1, INT4 = 2 };
 
 struct AppendArgs {
   void *k_cache;

@@ -1,4 +1,5 @@
-// quant.cu -- 8-bit quantisation of K/V rows (FP8 E4M3 or INT8 codes).
+// quant.cu -- 8- and 4-bit quantisation of K/V rows (FP8 E4M3, INT8 or INT4
+// codes).
 //
 // "KV Cache:推理慢的真正原因", section 工程优化手段 / 量化: store the cache in 8 bits
 // with scales per channel group, so a few very large key channels do not
@@ -9,7 +10,9 @@
 //  * E4M3: s = max|x| / 448 (448 is the largest E4M3 value), code = E4M3(x / s)
 //    rounded to nearest even and saturated;
 //  * INT8: s = max|x| / 127, code = x / s rounded to the nearest integer (ties
-//    to even) and clamped to +-127; a NaN quotient gives 0.
+//    to even) and clamped to +-127; a NaN quotient gives 0;
+//  * INT4: the same with 7 for 127, two codes per byte (channel 2i in the low
+//    nibble of byte i).
 // Both divisions are IEEE fp32 (__fdiv_rn), so the codes are the same on
 // every run and every machine.  A group of zeros gets s = 0.
 //
@@ -56,7 +59,10 @@ __global__ void __launch_bounds__(256) quantize_q8_kernel(const QuantArgs a) {
   float sc;
   const uint32_t word = encode_row4<T, kFmt>(static_cast<const T *>(src) + r * a.d, live, lane, sc);
   if (!live) return;
-  *reinterpret_cast<uint32_t *>(codes + dst * a.d + lane * 4) = word;
+  if constexpr (kFmt == Code8::INT4)
+    *reinterpret_cast<uint16_t *>(codes + dst * (a.d / 2) + lane * 2) = static_cast<uint16_t>(word);
+  else
+    *reinterpret_cast<uint32_t *>(codes + dst * a.d + lane * 4) = word;
   if ((lane & 7) == 0) scales[dst * (a.d / 32) + (lane >> 3)] = sc;
 }
 
@@ -64,6 +70,11 @@ cudaError_t launch_quantize_q8(const QuantArgs &a, DType dt, Code8 fmt, cudaStre
   if (a.n == 0) return cudaSuccess;
   const long long rows = a.src2 ? 2 * a.n : a.n;
   const dim3 grid(static_cast<unsigned>((rows + 7) / 8));
+  if (fmt == Code8::INT4) {
+    if (dt == DType::BF16)
+      return launch_pdl(quantize_q8_kernel<__nv_bfloat16, Code8::INT4>, grid, dim3(256), 0, s, a);
+    return launch_pdl(quantize_q8_kernel<__half, Code8::INT4>, grid, dim3(256), 0, s, a);
+  }
   if (fmt == Code8::INT8) {
     if (dt == DType::BF16)
       return launch_pdl(quantize_q8_kernel<__nv_bfloat16, Code8::INT8>, grid, dim3(256), 0, s, a);

@@ -305,14 +305,29 @@ __device__ __forceinline__ uint32_t swz8(int t, int c) {
   return static_cast<uint32_t>(t * 128 + ((c ^ (t & 7)) << 4));
 }
 
-// The same for a page of D-byte rows (D = 128: the 128-byte swizzle above;
-// D = 64: the 64-byte swizzle, chunk c of row t at chunk c ^ ((t >> 1) & 3),
-// so the 8 rows an ldmatrix reads fall on distinct banks).
-template <int D>
+// The same for a page of R-byte rows (R = 128: the 128-byte swizzle above;
+// R = 64: the 64-byte swizzle, chunk c of row t at chunk c ^ ((t >> 1) & 3);
+// R = 32: the 32-byte swizzle, chunk c ^ ((t >> 2) & 1) -- in each case the
+// 8 rows an ldmatrix reads fall on distinct banks).
+template <int R>
 __device__ __forceinline__ uint32_t swz_rows(int t, int c) {
-  static_assert(D == 128 || D == 64, "8-bit pages of 64 or 128 channels");
-  if constexpr (D == 128) return swz8(t, c);
-  else return static_cast<uint32_t>(t * 64 + ((c ^ ((t >> 1) & 3)) << 4));
+  static_assert(R == 128 || R == 64 || R == 32, "code rows of 32, 64 or 128 bytes");
+  if constexpr (R == 128) return swz8(t, c);
+  else if constexpr (R == 64) return static_cast<uint32_t>(t * 64 + ((c ^ ((t >> 1) & 3)) << 4));
+  else return static_cast<uint32_t>(t * 32 + ((c ^ ((t >> 2) & 1)) << 4));
+}
+
+// Eight INT4 codes (nibbles 0..7 of `w`, two's complement) -> four f16x2:
+// out[s] holds the values of nibbles s (low half) and s + 4 (high half),
+// exact.  Each nibble n becomes the f16 with bits 0x6400 | (n + 8), that is
+// 1024 + (n + 8), and 1032 is subtracted.
+__device__ __forceinline__ void int4x8_to_f16x2x4(uint32_t w, uint32_t (&out)[4]) {
+  const uint32_t u = w ^ 0x88888888u;  // n + 8, unsigned
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const uint32_t h = ((u >> (4 * s)) & 0x000F000Fu) | 0x64006400u;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out[s]) : "r"(h), "r"(0x64086408u));
+  }
 }
 
 // One 16-token page of an 8-bit cache (d = D = 64 or 128; E4M3 or INT8 codes)
@@ -453,6 +468,155 @@ __device__ __forceinline__ void tile_page_q8(uint32_t kb, uint32_t vb, const flo
     for (int nt = 0; nt < NT; ++nt) {
       M::run(acc[nt][2 * j], A[0], pj0[j][nt], pj1[j][nt]);
       M::run(acc[nt][2 * j + 1], A[1], pj0[j][nt], pj1[j][nt]);
+    }
+  }
+}
+
+// One 16-token page of an INT4 cache (d = D = 64 or 128: code rows of D / 2
+// bytes, 32 channels per 16-byte chunk, one scale group per chunk) for 8*NT
+// query rows of one warp, on the f16 tensor-core tile.
+//  * K: ldmatrix gives each lane 8 consecutive channels 8 tig .. 8 tig + 7 of
+//    one token per register.  int4x8_to_f16x2x4 pairs channels (8 tig + s,
+//    8 tig + s + 4); pairs s = 0, 1 fill k-step 2j of group j's A operand,
+//    s = 2, 3 k-step 2j + 1 (Page4::q_words orders q the same way).  Scores
+//    are summed per group and weighted by the token's group scales.
+//  * V: ldmatrix.trans gives each lane 4 channels 4 g8 .. 4 g8 + 3 of two
+//    consecutive tokens per register; the same conversion pairs each channel
+//    across the two tokens, which is exactly an A-fragment register of V^T.
+//    Group j makes two m-tiles: rows g8, g8 + 8 <-> channels 32j + 4 g8 + 2t
+//    and 32j + 4 g8 + 2t + 1 for m-tile 2j + t (Page4::dim).  The V group
+//    scales ride on the probabilities, as in the 8-bit tile.
+template <int D, int NT>
+__device__ __forceinline__ void tile_page_q4(uint32_t kb, uint32_t vb, const float *ks,
+                                              const float *vs, int ntok, float scale_log2,
+                                              int lane, const uint32_t (&qf)[NT][D / 16][2],
+                                              float (&acc)[NT][D / 16][4], float (&m_run)[NT][2],
+                                              float (&l_run)[NT][2]) {
+  using M = Mma<__half>;
+  constexpr int kG = D / 32;  // scale groups = 16-byte chunks of a code row
+  static_assert(kG % 2 == 0, "code rows of whole chunk pairs");
+  const int g8 = lane >> 2;
+  const int mi = lane >> 3, r8 = lane & 7;
+  const int tok = r8 + ((mi & 1) << 3);  // row this lane addresses for ldmatrix
+  const int hi = mi >> 1;                // second chunk of a pair
+
+  float sg[kG][NT][4];
+#pragma unroll
+  for (int j = 0; j < kG; ++j)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sg[j][nt][e] = 0.f;
+#pragma unroll
+  for (int jj = 0; jj < kG / 2; ++jj) {
+    uint32_t R[4];  // tokens 0-7 / 8-15 of chunk 2jj, then of chunk 2jj + 1
+    ldmatrix_x4(R, kb + swz_rows<D / 2>(tok, 2 * jj + hi));
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = 2 * jj + h;
+      uint32_t p[4], q[4];  // token g8, token g8 + 8
+      int4x8_to_f16x2x4(R[2 * h], p);
+      int4x8_to_f16x2x4(R[2 * h + 1], q);
+      const uint32_t A0[4] = {p[0], q[0], p[1], q[1]};
+      const uint32_t A1[4] = {p[2], q[2], p[3], q[3]};
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        M::run(sg[j][nt], A0, qf[nt][2 * j][0], qf[nt][2 * j][1]);
+        M::run(sg[j][nt], A1, qf[nt][2 * j + 1][0], qf[nt][2 * j + 1][1]);
+      }
+    }
+  }
+  // the scales of this lane's two tokens (g8 and g8 + 8), K and V
+  float kAs[kG], kBs[kG], vAs[kG], vBs[kG];
+  if constexpr (kG == 4) {
+    const float4 kA = *reinterpret_cast<const float4 *>(ks + g8 * 4);
+    const float4 kB = *reinterpret_cast<const float4 *>(ks + (g8 + 8) * 4);
+    const float4 vA = *reinterpret_cast<const float4 *>(vs + g8 * 4);
+    const float4 vB = *reinterpret_cast<const float4 *>(vs + (g8 + 8) * 4);
+    kAs[0] = kA.x; kAs[1] = kA.y; kAs[2] = kA.z; kAs[3] = kA.w;
+    kBs[0] = kB.x; kBs[1] = kB.y; kBs[2] = kB.z; kBs[3] = kB.w;
+    vAs[0] = vA.x; vAs[1] = vA.y; vAs[2] = vA.z; vAs[3] = vA.w;
+    vBs[0] = vB.x; vBs[1] = vB.y; vBs[2] = vB.z; vBs[3] = vB.w;
+  } else {
+    const float2 kA = *reinterpret_cast<const float2 *>(ks + g8 * 2);
+    const float2 kB = *reinterpret_cast<const float2 *>(ks + (g8 + 8) * 2);
+    const float2 vA = *reinterpret_cast<const float2 *>(vs + g8 * 2);
+    const float2 vB = *reinterpret_cast<const float2 *>(vs + (g8 + 8) * 2);
+    kAs[0] = kA.x; kAs[1] = kA.y;
+    kBs[0] = kB.x; kBs[1] = kB.y;
+    vAs[0] = vA.x; vAs[1] = vA.y;
+    vBs[0] = vB.x; vBs[1] = vB.y;
+  }
+
+  const bool v0 = g8 < ntok, v1 = g8 + 8 < ntok;
+  uint32_t pj0[kG][NT], pj1[kG][NT];
+  float alpha[NT][2];
+  bool rescale = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < kG; ++j) {
+      s4[0] += sg[j][nt][0] * kAs[j];
+      s4[1] += sg[j][nt][1] * kAs[j];
+      s4[2] += sg[j][nt][2] * kBs[j];
+      s4[3] += sg[j][nt][3] * kBs[j];
+    }
+    const float x0 = v0 ? s4[0] * scale_log2 : -INFINITY;
+    const float x1 = v0 ? s4[1] * scale_log2 : -INFINITY;
+    const float x2 = v1 ? s4[2] * scale_log2 : -INFINITY;
+    const float x3 = v1 ? s4[3] * scale_log2 : -INFINITY;
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+    alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
+    alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
+    rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
+    m_run[nt][0] = mn0;
+    m_run[nt][1] = mn1;
+    const float e0 = fast_exp2(x0 - mn0), e1 = fast_exp2(x1 - mn1);
+    const float e2 = fast_exp2(x2 - mn0), e3 = fast_exp2(x3 - mn1);
+    l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (e0 + e2);
+    l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (e1 + e3);
+#pragma unroll
+    for (int j = 0; j < kG; ++j) {
+      // masked tokens have e = 0 and a V scale of 0 (cleared by the caller)
+      pj0[j][nt] = movmatrix_trans(f16pack(e0 * vAs[j], e1 * vAs[j]));
+      pj1[j][nt] = movmatrix_trans(f16pack(e2 * vBs[j], e3 * vBs[j]));
+    }
+  }
+  if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        acc[nt][mt][0] *= alpha[nt][0];
+        acc[nt][mt][1] *= alpha[nt][1];
+        acc[nt][mt][2] *= alpha[nt][0];
+        acc[nt][mt][3] *= alpha[nt][1];
+      }
+  }
+#pragma unroll
+  for (int jj = 0; jj < kG / 2; ++jj) {
+    uint32_t R[4];  // transposed: tokens 0-7 / 8-15 of chunk 2jj, then of 2jj + 1
+    ldmatrix_x4_trans(R, vb + swz_rows<D / 2>(tok, 2 * jj + hi));
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = 2 * jj + h;
+      uint32_t u[4], w[4];  // channel 4 g8 + c of tokens (2 tig, +1) / (8 + 2 tig, +1)
+      int4x8_to_f16x2x4(R[2 * h], u);
+      int4x8_to_f16x2x4(R[2 * h + 1], w);
+      const uint32_t A0[4] = {u[0], u[1], w[0], w[1]};
+      const uint32_t A1[4] = {u[2], u[3], w[2], w[3]};
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        M::run(acc[nt][2 * j], A0, pj0[j][nt], pj1[j][nt]);
+        M::run(acc[nt][2 * j + 1], A1, pj0[j][nt], pj1[j][nt]);
+      }
     }
   }
 }

@@ -56,6 +56,72 @@ def oracle_step(w, si, kc_words=None, vc_words=None, rows=None):
     return kc, vc, res
 
 
+def host(t):
+    """Device tensor -> numpy copy; 8-bit codes as their bytes (uint8)."""
+    a = t.cpu().numpy().copy()
+    return a.view(np.uint8) if a.dtype == np.int8 else a
+
+
+def oracle_q8(w, fmt, si=None):
+    """The oracle's own 8-bit pools: its quantisation of the workload's whole
+    16-bit pool and, with step inputs si, its quantising append of the step's
+    rows -- no input from the GPU."""
+    k8, ks = getattr(oracle, "quantize_" + fmt)(to_words(w.k_cache), odt(w))
+    v8, vs = getattr(oracle, "quantize_" + fmt)(to_words(w.v_cache), odt(w))
+    if si is not None:
+        getattr(oracle, "append_" + fmt)(k8, v8, ks, vs, w.block_table.numpy(), si["slot"].cpu().numpy(),
+                              to_words(si["k_new"]), to_words(si["v_new"]), odt(w))
+    return k8, v8, ks, vs
+
+
+def oracle_q8_rows(w, fmt, si, rows):
+    """oracle_q8 for a few sequences of a large workload: only the pages
+    they use, renumbered (returns the pools, their block table and the page
+    list, so the GPU's pools can be compared page for page)."""
+    bt = w.block_table.cpu()
+    n = si["seq_lens"].cpu()
+    npg = [(int(n[b]) + 15) // 16 for b in rows]
+    pages = sorted({int(p) for b, m in zip(rows, npg) for p in bt[b, :m].tolist()})
+    remap = {p: i for i, p in enumerate(pages)}
+    bts = np.zeros((len(rows), max(npg)), dtype=np.int32)
+    for i, (b, m) in enumerate(zip(rows, npg)):
+        bts[i, :m] = [remap[p] for p in bt[b, :m].tolist()]
+    idx = torch.tensor(pages, dtype=torch.long, device=w.k_cache.device)
+    kw, vw = to_words(w.k_cache.index_select(0, idx)), to_words(w.v_cache.index_select(0, idx))
+    k8, ks = getattr(oracle, "quantize_" + fmt)(kw, odt(w))
+    v8, vs = getattr(oracle, "quantize_" + fmt)(vw, odt(w))
+    sel = torch.tensor(rows, dtype=torch.long)
+    getattr(oracle, "append_" + fmt)(k8, v8, ks, vs, bts, si["slot"].cpu()[sel].numpy(),
+                          to_words(si["k_new"].cpu()[sel]), to_words(si["v_new"].cpu()[sel]), odt(w))
+    return (k8, v8, ks, vs), bts, pages
+
+
+def data_rows(k_cache, v_cache, block_table=None, si=None):
+    """Bool [NB, H_kv, 16]: pool rows holding data -- rows of the 16-bit pool
+    that are not the NaN canary of never-written slots, plus the rows the
+    step appends.  The canary's 8-bit encoding (which NaN code, which NaN
+    scale) is a convention nothing reads, so pools are compared on these."""
+    m = (torch.isfinite(k_cache.float()).all(-1) & torch.isfinite(v_cache.float()).all(-1)).cpu().numpy()
+    if si is not None:
+        slot = si["slot"].cpu().numpy()
+        bt = block_table.cpu().numpy() if torch.is_tensor(block_table) else block_table
+        for b, pos in enumerate(slot):
+            if pos >= 0:
+                m[bt[b, pos // 16], :, pos % 16] = True
+    return m
+
+
+def assert_pools_equal(gpu, orc, rows):
+    """8-bit codes and fp32 scales, bit for bit, on the rows holding data."""
+    for g, o in zip(gpu, orc):
+        g = host(g) if torch.is_tensor(g) else g
+        if g.dtype == np.float32:
+            g, o = g.view(np.uint32), o.view(np.uint32)
+        assert np.array_equal(g[rows], o[rows])
+
+
+
+
 def max_err(gpu_out, ref, rows=None):
     g = gpu_out.float().cpu().double().numpy()
     errs = []
@@ -77,9 +143,31 @@ def max_lse_err(gpu_lse, ref):
     return float(max(errs)) if errs else 0.0
 
 
+def assert_out_close(gpu_out, ref, dtype):
+    """out within TOL[dtype] (max-abs) of the fp64 oracle wherever a value of
+    the output dtype can be that close.  Where |ref| is so large that half an
+    ulp of the dtype exceeds TOL (bf16 from |ref| >= 2.56: half an ulp is
+    1/256 of the value), even the correctly rounded output misses the
+    absolute bound, so there the output must be within one ulp of ref.
+    Returns the max abs error over all outputs."""
+    g = gpu_out.float().cpu().double().numpy() if torch.is_tensor(gpu_out) else gpu_out
+    err = np.abs(g - ref)
+    mant = 8 if dtype == torch.bfloat16 else 11               # significant bits
+    mag = np.abs(ref)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(mag, 2.0 ** -14))) - (mant - 1))
+    near = ulp / 2 <= TOL[dtype]
+    if near.any():
+        assert float(err[near].max()) <= TOL[dtype], f"max abs error {float(err[near].max())}"
+    if (~near).any():
+        worst = float((err[~near] / ulp[~near]).max())
+        assert worst <= 1.0, f"error of {worst} ulp where |out| >= {float(mag[~near].min())}"
+    return float(err.max()) if err.size else 0.0
+
+
 def words(t):
     return to_words(t)
 
 
-__all__ = ["TOL", "LSE_TOL", "ERROR_REPORT", "record_error", "gpu_state", "gpu_step", "oracle_step", "max_err", "max_lse_err",
+__all__ = ["TOL", "LSE_TOL", "ERROR_REPORT", "record_error", "assert_out_close", "host", "oracle_q8", "oracle_q8_rows",
+           "data_rows", "assert_pools_equal", "odt", "gpu_state", "gpu_step", "oracle_step", "max_err", "max_lse_err",
            "words", "step_inputs"]

@@ -200,7 +200,7 @@ def decode8(fmt, step=False, **kw):
     return getattr(L, "kvd_decode_attention_" + fmt)(a["q"], *tail)
 
 
-@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "int4"])
 @pytest.mark.parametrize("step", [False, True])
 @pytest.mark.parametrize("kw,status", [
     (dict(d=96), kvd.KVD_ERR_UNSUPPORTED),                 # the 8-bit tile is d = 64 or 128
@@ -216,14 +216,14 @@ def test_decode8_validation(fmt, step, kw, status):
     assert kvd.kvd_last_error() != ""
 
 
-@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "int4"])
 def test_step8_requires_aligned_new_rows(fmt):
     assert decode8(fmt, True, kn=NULL) == kvd.KVD_ERR_INVALID
     assert decode8(fmt, True, vn=MISALIGNED) == kvd.KVD_ERR_INVALID
     assert decode8(fmt, True, B=0, q=NULL, kn=NULL, vn=NULL, out=NULL, ws=NULL) == kvd.KVD_OK
 
 
-@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "int4"])
 @pytest.mark.parametrize("kw,status", [
     (dict(d=48), kvd.KVD_ERR_UNSUPPORTED),
     (dict(d=160), kvd.KVD_ERR_UNSUPPORTED),
@@ -241,7 +241,7 @@ def test_append8_validation(fmt, kw, status):
                                             a["dt"], a["stream"]) == status
 
 
-@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "int4"])
 @pytest.mark.parametrize("kw,status", [
     (dict(d=40), kvd.KVD_ERR_UNSUPPORTED),
     (dict(n=-1), kvd.KVD_ERR_INVALID),

@@ -4,6 +4,8 @@ import json
 import os
 import sys
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
@@ -99,16 +101,36 @@ def test_row_snapshot_renumbers_pages_and_feeds_the_oracle():
     assert abs(bench.oracle_parity(snap, wrong)[0] - 0.01) < 1e-9
 
 
-def test_row_snapshot_8bit_parity_uses_the_oracles_quantisation():
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "int4"])
+def test_row_snapshot_quantised_parity_uses_the_oracles_quantisation(fmt):
     import oracle
     from synth import build_workload, step_inputs, to_words
     w = build_workload("snap8", 3, 8, 2, 128, "bf16", [40, 17, 33], seed=32, spare_pages=2)
     si = step_inputs(w, 0)
     snap = bench.RowSnapshot(w, si, [0, 1, 2])
-    k8, ks = oracle.quantize_fp8(to_words(w.k_cache), oracle.BF16)
-    v8, vs = oracle.quantize_fp8(to_words(w.v_cache), oracle.BF16)
-    oracle.append_fp8(k8, v8, ks, vs, w.block_table.numpy(), si["slot"].numpy(), to_words(si["k_new"]),
-                      to_words(si["v_new"]), oracle.BF16)
-    ref, _ = oracle.attend_fp8(to_words(si["q"]), k8, v8, ks, vs, w.block_table.numpy(),
-                               si["seq_lens"].numpy(), w.scale, oracle.BF16)
-    assert bench.oracle_parity(snap, ref, fmt="fp8")[0] == 0.0
+    quant = getattr(oracle, "quantize_" + fmt)
+    k8, ks = quant(to_words(w.k_cache), oracle.BF16)
+    v8, vs = quant(to_words(w.v_cache), oracle.BF16)
+    getattr(oracle, "append_" + fmt)(k8, v8, ks, vs, w.block_table.numpy(), si["slot"].numpy(),
+                                     to_words(si["k_new"]), to_words(si["v_new"]), oracle.BF16)
+    ref, _ = getattr(oracle, "attend_" + fmt)(to_words(si["q"]), k8, v8, ks, vs, w.block_table.numpy(),
+                                              si["seq_lens"].numpy(), w.scale, oracle.BF16)
+    assert bench.oracle_parity(snap, ref, fmt=fmt)[0] == 0.0
+
+
+def test_quantised_byte_counts():
+    # a d = 128 row: 128 code bytes (64 for INT4) + 4 fp32 scales
+    assert bench.quant_row_bytes("fp8", 128) == 144
+    assert bench.quant_row_bytes("int8", 128) == 144
+    assert bench.quant_row_bytes("int4", 128) == 80
+    assert bench.quant_row_bytes("int4", 64) == 40
+    from synth import build_workload, step_inputs
+    w = build_workload("bytes4", 2, 8, 2, 128, "bf16", [40, 17], seed=33, spare_pages=2)
+    si = step_inputs(w, 0)
+    toks = int(si["seq_lens"].sum())
+    assert bench.quant_attention_bytes(w, si["seq_lens"], "int4") == toks * 2 * 2 * 80 + 2 * 2 * 8 * 128 * 2
+    rows = int((si["slot"] >= 0).sum()) * 2
+    assert bench.quant_append_bytes(w, si["slot"], "int4") == rows * 2 * (256 + 80)
+    snap = bench.RowSnapshot(w, si, [0, 1])
+    assert snap.nbytes_q("int4") == (bench.quant_attention_bytes(w, si["seq_lens"], "int4")
+                                     + bench.quant_append_bytes(w, si["slot"], "int4"))

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import LSE_TOL, TOL
+from gpu_helpers import LSE_TOL, TOL, assert_pools_equal, data_rows, host, odt, oracle_q8, oracle_q8_rows
 from synth import build_workload, named_config, step_inputs, to_words
 
 pytestmark = pytest.mark.gpu
@@ -22,10 +22,6 @@ def kvd():
     import kv_cache_decode_scatters_b200 as m
     m.kvd_read_device_error(clear=True)
     return m
-
-
-def odt(w):
-    return oracle.BF16 if w.dtype == torch.bfloat16 else oracle.F16
 
 
 FORMATS = ["fp8", "int8"]
@@ -42,12 +38,6 @@ def gpu_fn(kvd, what, fmt):
 
 def orc_fn(what, fmt):
     return getattr(oracle, f"{what}_{fmt}")
-
-
-def host(t):
-    """Device tensor -> numpy copy; 8-bit codes as their bytes (uint8)."""
-    a = t.cpu().numpy().copy()
-    return a.view(np.uint8) if a.dtype == np.int8 else a
 
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
@@ -68,64 +58,6 @@ def test_quantize_bit_exact(kvd, fmt, dtype, d):
     oc, os_ = orc_fn("quantize", fmt)(to_words(x), oracle.BF16 if dtype == torch.bfloat16 else oracle.F16)
     assert np.array_equal(host(codes), oc)
     assert np.array_equal(host(scales).view(np.uint32), os_.view(np.uint32))
-
-
-def oracle_q8(w, fmt, si=None):
-    """The oracle's own 8-bit pools: its quantisation of the workload's whole
-    16-bit pool and, with step inputs si, its quantising append of the step's
-    rows -- no input from the GPU."""
-    k8, ks = orc_fn("quantize", fmt)(to_words(w.k_cache), odt(w))
-    v8, vs = orc_fn("quantize", fmt)(to_words(w.v_cache), odt(w))
-    if si is not None:
-        orc_fn("append", fmt)(k8, v8, ks, vs, w.block_table.numpy(), si["slot"].cpu().numpy(),
-                              to_words(si["k_new"]), to_words(si["v_new"]), odt(w))
-    return k8, v8, ks, vs
-
-
-def oracle_q8_rows(w, fmt, si, rows):
-    """oracle_q8 for a few sequences of a large workload: only the pages
-    they use, renumbered (returns the pools, their block table and the page
-    list, so the GPU's pools can be compared page for page)."""
-    bt = w.block_table.cpu()
-    n = si["seq_lens"].cpu()
-    npg = [(int(n[b]) + 15) // 16 for b in rows]
-    pages = sorted({int(p) for b, m in zip(rows, npg) for p in bt[b, :m].tolist()})
-    remap = {p: i for i, p in enumerate(pages)}
-    bts = np.zeros((len(rows), max(npg)), dtype=np.int32)
-    for i, (b, m) in enumerate(zip(rows, npg)):
-        bts[i, :m] = [remap[p] for p in bt[b, :m].tolist()]
-    idx = torch.tensor(pages, dtype=torch.long, device=w.k_cache.device)
-    kw, vw = to_words(w.k_cache.index_select(0, idx)), to_words(w.v_cache.index_select(0, idx))
-    k8, ks = orc_fn("quantize", fmt)(kw, odt(w))
-    v8, vs = orc_fn("quantize", fmt)(vw, odt(w))
-    sel = torch.tensor(rows, dtype=torch.long)
-    orc_fn("append", fmt)(k8, v8, ks, vs, bts, si["slot"].cpu()[sel].numpy(),
-                          to_words(si["k_new"].cpu()[sel]), to_words(si["v_new"].cpu()[sel]), odt(w))
-    return (k8, v8, ks, vs), bts, pages
-
-
-def data_rows(k_cache, v_cache, block_table=None, si=None):
-    """Bool [NB, H_kv, 16]: pool rows holding data -- rows of the 16-bit pool
-    that are not the NaN canary of never-written slots, plus the rows the
-    step appends.  The canary's 8-bit encoding (which NaN code, which NaN
-    scale) is a convention nothing reads, so pools are compared on these."""
-    m = (torch.isfinite(k_cache.float()).all(-1) & torch.isfinite(v_cache.float()).all(-1)).cpu().numpy()
-    if si is not None:
-        slot = si["slot"].cpu().numpy()
-        bt = block_table.cpu().numpy() if torch.is_tensor(block_table) else block_table
-        for b, pos in enumerate(slot):
-            if pos >= 0:
-                m[bt[b, pos // 16], :, pos % 16] = True
-    return m
-
-
-def assert_pools_equal(gpu, orc, rows):
-    """8-bit codes and fp32 scales, bit for bit, on the rows holding data."""
-    for g, o in zip(gpu, orc):
-        g = host(g) if torch.is_tensor(g) else g
-        if g.dtype == np.float32:
-            g, o = g.view(np.uint32), o.view(np.uint32)
-        assert np.array_equal(g[rows], o[rows])
 
 
 def q8_state(kvd, w, fmt):

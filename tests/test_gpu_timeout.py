@@ -12,7 +12,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import LSE_TOL, TOL, gpu_state, max_err, max_lse_err, oracle_step
+from gpu_helpers import (LSE_TOL, TOL, assert_pools_equal, data_rows, gpu_state, max_err, max_lse_err,
+                         oracle_q8, oracle_step)
 from synth import build_workload, step_inputs, to_words
 
 pytestmark = pytest.mark.gpu
@@ -60,8 +61,8 @@ def test_wait_timeout_flags_and_next_call_is_correct(kvd, parts):
     assert kvd.kvd_read_device_error() == 0
 
 
-@pytest.mark.parametrize("fmt", ["fp8", "int8"])
-def test_wait_timeout_in_the_8bit_decode(kvd, fmt):
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "int4"])
+def test_wait_timeout_in_the_quantised_decode(kvd, fmt):
     w = build_workload("timeout8", 2, 16, 4, 128, "f16", [300, 47], seed=951, spare_pages=2)
     si = step_inputs(w, 0)
     quant = getattr(kvd, "kvd_quantize_" + fmt)
@@ -77,27 +78,13 @@ def test_wait_timeout_in_the_8bit_decode(kvd, fmt):
     finally:
         kvd.kvd_set_decode_wait_limit(-1)
     assert kvd.kvd_read_device_error(clear=True) & kvd.KVD_DEVERR_TIMEOUT
-    # the same step with the default limit: against the oracle over the
-    # dequantised cache, after the oracle's own quantising append
-    k8b, v8b, ksb, vsb = k8.clone(), v8.clone(), ks.clone(), vs.clone()
-    out = step(*args, k8b, v8b, ksb, vsb, bt, si["seq_lens"].cuda(), w.scale)
+    # the same step with the default limit: pools bit for bit on the slots
+    # holding data, out against the oracle's attention over its own pools
+    pools = [t.clone() for t in (k8, v8, ks, vs)]
+    out = step(*args, *pools, bt, si["seq_lens"].cuda(), w.scale)
     torch.cuda.synchronize()
-    host = lambda t: (lambda a: a.view(np.uint8) if a.dtype == np.int8 else a)(t.cpu().numpy().copy())
-    # the oracle's own pools: its quantisation of the 16-bit pool, then its
-    # quantising append of the step
-    hk, hks = getattr(oracle, "quantize_" + fmt)(to_words(w.k_cache), oracle.F16)
-    hv, hvs = getattr(oracle, "quantize_" + fmt)(to_words(w.v_cache), oracle.F16)
-    getattr(oracle, "append_" + fmt)(hk, hv, hks, hvs, w.block_table.numpy(), si["slot"].numpy(),
-                                     to_words(si["k_new"]), to_words(si["v_new"]), oracle.F16)
-    # codes and scales bit for bit on the slots holding data (the encoding of
-    # the NaN canary in never-written slots is a convention nothing reads)
-    rows = (torch.isfinite(w.k_cache.float()).all(-1) & torch.isfinite(w.v_cache.float()).all(-1)).numpy()
-    btn = w.block_table.numpy()
-    for b, pos in enumerate(si["slot"].numpy()):
-        if pos >= 0:
-            rows[btn[b, pos // 16], :, pos % 16] = True
-    assert np.array_equal(host(k8b)[rows], hk[rows]) and np.array_equal(host(v8b)[rows], hv[rows])
-    assert np.array_equal(host(ksb).view(np.uint32)[rows], hks.view(np.uint32)[rows])
+    hk, hv, hks, hvs = oracle_q8(w, fmt, si)
+    assert_pools_equal(pools, (hk, hv, hks, hvs), data_rows(w.k_cache, w.v_cache, w.block_table, si))
     ref, _ = getattr(oracle, "attend_" + fmt)(to_words(si["q"]), hk, hv, hks, hvs, w.block_table.numpy(),
                                               si["seq_lens"].numpy(), w.scale, oracle.F16)
     err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
