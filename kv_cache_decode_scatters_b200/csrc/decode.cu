@@ -1250,23 +1250,48 @@ cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const 
 
 // 4-bit cache: d = 128 has 2 KB code stages, d = 64 1 KB; a parked
 // accumulator tile (8 NT D floats) must fit in a warp's stages.
+#ifndef KVD_TUNE_W4_1
+#define KVD_TUNE_W4_1 16
+#endif
+#ifndef KVD_TUNE_S4_1
+#define KVD_TUNE_S4_1 2
+#endif
+#ifndef KVD_TUNE_W4_2
+#define KVD_TUNE_W4_2 8
+#endif
+#ifndef KVD_TUNE_S4_2
+#define KVD_TUNE_S4_2 4
+#endif
+#ifndef KVD_TUNE_W4_64_1
+#define KVD_TUNE_W4_64_1 16
+#endif
+#ifndef KVD_TUNE_S4_64_1
+#define KVD_TUNE_S4_64_1 4
+#endif
+#ifndef KVD_TUNE_W4_64_2
+#define KVD_TUNE_W4_64_2 8
+#endif
+#ifndef KVD_TUNE_S4_64_2
+#define KVD_TUNE_S4_64_2 4
+#endif
+
 template <int D, int NT>
 struct Tune4;
 template <>
 struct Tune4<128, 1> {
-  static constexpr int W = 16, S = 2;
+  static constexpr int W = KVD_TUNE_W4_1, S = KVD_TUNE_S4_1;
 };
 template <>
 struct Tune4<128, 2> {
-  static constexpr int W = 8, S = 4;
+  static constexpr int W = KVD_TUNE_W4_2, S = KVD_TUNE_S4_2;
 };
 template <>
 struct Tune4<64, 1> {
-  static constexpr int W = 16, S = 4;
+  static constexpr int W = KVD_TUNE_W4_64_1, S = KVD_TUNE_S4_64_1;
 };
 template <>
 struct Tune4<64, 2> {
-  static constexpr int W = 8, S = 4;
+  static constexpr int W = KVD_TUNE_W4_64_2, S = KVD_TUNE_S4_64_2;
 };
 
 template <int D, int NT, typename T>

@@ -319,15 +319,33 @@ __device__ __forceinline__ uint32_t swz_rows(int t, int c) {
 
 // Eight INT4 codes (nibbles 0..7 of `w`, two's complement) -> four f16x2:
 // out[s] holds the values of nibbles s (low half) and s + 4 (high half),
-// exact.  Each nibble n becomes the f16 with bits 0x6400 | (n + 8), that is
-// 1024 + (n + 8), and 1032 is subtracted.
+// exact.  With the sign bit flipped a nibble n reads n + 8.  The low nibble of
+// each 16-bit half, flipped and with 0x6400 above it (one AND-XOR), is the f16
+// 1024 + (n + 8), and 1032 is subtracted; the next nibble up, masked in place,
+// is 1024 + 16 (n + 8), scaled by 1/16 with 72 subtracted in one fma.  Every
+// intermediate is an integer (or a sixteenth of one) below 2048, so both
+// steps are exact.  Nibbles 2, 3, 6, 7 do the same after one shift by 8.
+__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t f16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 __device__ __forceinline__ void int4x8_to_f16x2x4(uint32_t w, uint32_t (&out)[4]) {
-  const uint32_t u = w ^ 0x88888888u;  // n + 8, unsigned
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const uint32_t h = ((u >> (4 * s)) & 0x000F000Fu) | 0x64006400u;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out[s]) : "r"(h), "r"(0x64086408u));
-  }
+  constexpr uint32_t kLoBias = 0x64086408u;   // f16x2 (1032, 1032)
+  constexpr uint32_t kSixteenth = 0x2C002C00u;  // f16x2 (1/16, 1/16)
+  constexpr uint32_t kMinus72 = 0xD480D480u;  // f16x2 (-72, -72)
+  const uint32_t w8 = w >> 8;
+  out[0] = f16x2_sub((w & 0x000F000Fu) ^ kLoBias, kLoBias);
+  out[1] = f16x2_fma((w & 0x00F000F0u) ^ 0x64806480u, kSixteenth, kMinus72);
+  out[2] = f16x2_sub((w8 & 0x000F000Fu) ^ kLoBias, kLoBias);
+  out[3] = f16x2_fma((w8 & 0x00F000F0u) ^ 0x64806480u, kSixteenth, kMinus72);
 }
 
 // One 16-token page of an 8-bit cache (d = D = 64 or 128; E4M3 or INT8 codes)
