@@ -455,7 +455,8 @@ def run_reference(args):
 PER_WORKLOADS = (("tiny", False, None), ("gqa70b", False, None), ("long", False, None),
                  ("cbatch", False, None), ("cbatch", True, None), ("mha7b", False, "fp8"),
                  ("gqa70b", False, "fp8"), ("mha7b", False, "int8"), ("gqa70b", False, "int8"),
-                 ("mha7b", False, "int4"), ("gqa70b", False, "int4"))
+                 ("mha7b", False, "int4"), ("gqa70b", False, "int4"), ("cbatch", True, "fp8"),
+                 ("cbatch", True, "int8"), ("cbatch", True, "int4"))
 
 
 def measure_workload(kvd, name, shared_prefix, dev, steps, warmup, fmt=None):
@@ -475,7 +476,8 @@ def measure_workload(kvd, name, shared_prefix, dev, steps, warmup, fmt=None):
         quant = getattr(kvd, "kvd_quantize_" + fmt)
         k8, ks = quant(kc)
         v8, vs = quant(vc)
-        q8 = (k8, v8, ks, vs, getattr(kvd, "kvd_decode_step_" + fmt))
+        q8 = (k8, v8, ks, vs, getattr(kvd, "kvd_decode_step_" + fmt),
+              getattr(kvd, "kvd_decode_attention_shared_prefix_" + fmt))
     q, k_new, v_new, seq_lens = si["q"], si["k_new"], si["v_new"], si["seq_lens"].to(dev)
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
@@ -491,7 +493,10 @@ def measure_workload(kvd, name, shared_prefix, dev, steps, warmup, fmt=None):
         ws = kvd.alloc_workspace(w.B, w.H_q, w.H_kv, w.d, 0, dev)
 
     def call(x_q, x_k, x_v, x_len):
-        if q8 is not None:
+        if q8 is not None and sp is not None:
+            q8[5](x_q, q8[0], q8[1], q8[2], q8[3], bt, x_len, sp["start"], sp["pages"], sp["max"], w.scale,
+                  out=out, k_new=x_k, v_new=x_v, workspace=ws, stream=stream)
+        elif q8 is not None:
             q8[4](x_q, x_k, x_v, q8[0], q8[1], q8[2], q8[3], bt, x_len, w.scale, out=out, workspace=ws,
                   stream=stream)
         elif sp is not None:
@@ -530,11 +535,17 @@ def measure_workload(kvd, name, shared_prefix, dev, steps, warmup, fmt=None):
         a_b -= w.groups * (w.B // w.groups - 1) * w.prefix_tokens * w.H_kv * 2 * w.d * 2
     nbytes = a_b + append_bytes(w, si["slot"].cpu())
     if q8 is not None:  # codes + scales read; appended rows read in 16 bits, written as codes + scales
-        nbytes = (quant_attention_bytes(w, si["seq_lens"].cpu(), fmt)
-                  + quant_append_bytes(w, si["slot"].cpu(), fmt))
+        a_b = quant_attention_bytes(w, si["seq_lens"].cpu(), fmt)
+        a_logical = a_b
+        if w.groups:
+            a_b -= (w.groups * (w.B // w.groups - 1) * w.prefix_tokens * w.H_kv * 2
+                    * quant_row_bytes(fmt, w.d))
+        nbytes = a_b + quant_append_bytes(w, si["slot"].cpu(), fmt)
     rep = {
         "workload": name + (" --shared-prefix" if shared_prefix else "") + (f" --kv-{fmt}" if fmt else ""),
-        "call": ("kvd_decode_attention_shared_prefix (fused append)" if sp is not None
+        "call": (f"kvd_decode_attention_shared_prefix_{fmt} (fused quantising append) over the "
+                 f"{QUANT_NAMES[fmt]} cache" if sp is not None and q8 is not None
+                 else "kvd_decode_attention_shared_prefix (fused append)" if sp is not None
                  else f"kvd_decode_step_{fmt} over the {QUANT_NAMES[fmt]} cache"
                  if q8 is not None else "kvd_decode_step"),
         "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "d": w.d,
@@ -603,6 +614,7 @@ def run_ours(args):
               "append": getattr(kvd, "kvd_append_" + fmt),
               "decode": getattr(kvd, "kvd_decode_attention_" + fmt),
               "step": getattr(kvd, "kvd_decode_step_" + fmt),
+              "shared": getattr(kvd, "kvd_decode_attention_shared_prefix_" + fmt),
               "name": QUANT_NAMES[fmt]}
 
     sp = None
@@ -617,6 +629,15 @@ def run_ours(args):
         ws = torch.empty(n, dtype=torch.uint8, device=dev)
 
     def step(ev_a=None, ev_b=None):
+        if f8 is not None and sp is not None:
+            if ev_a is not None:
+                ev_a.record(stream)
+            f8["shared"](q, f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, seq_lens, sp["start"], sp["pages"],
+                         sp["max"], w.scale, out=out, k_new=k_new, v_new=v_new,
+                         num_partitions=args.partitions, workspace=ws, stream=stream)
+            if ev_b is not None:
+                ev_b.record(stream)
+            return
         if f8 is not None and not args.separate_append:
             if ev_a is not None:
                 ev_a.record(stream)
@@ -745,7 +766,11 @@ def run_ours(args):
         seq_lens and, for the two-call paths, slot), on stream st (default:
         the bench's stream)."""
         stream = st if st is not None else stream0
-        if f8 is not None and not args.separate_append:
+        if f8 is not None and sp is not None:
+            f8["shared"](x["q"], f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt, x["seq_lens"], sp["start"],
+                         sp["pages"], sp["max"], w.scale, out=out, k_new=x["k_new"], v_new=x["v_new"],
+                         num_partitions=args.partitions, workspace=ws, stream=stream)
+        elif f8 is not None and not args.separate_append:
             f8["step"](x["q"], x["k_new"], x["v_new"], f8["k8"], f8["v8"], f8["ks"], f8["vs"], bt,
                        x["seq_lens"], w.scale, out=out, num_partitions=args.partitions, workspace=ws,
                        stream=stream)
@@ -936,7 +961,10 @@ def run_ours(args):
             "bytes_per_step": step_bytes, "attention_bytes": a_bytes, "append_bytes": p_bytes,
             "l2": "inputs larger than L2 (KV pool %.2f GB >> 126 MB); no flush" % (
                 2 * w.k_cache.numel() * 2 / 1e9),
-            "step": ("kvd_append_%s + kvd_decode_attention_%s over an %s cache "
+            "step": ("kvd_decode_attention_shared_prefix_%s with fused quantising append over an %s "
+                     "cache (prefix tensor-core pass with dequantised tiles, decode, merge kernels)"
+                     % (f8["fmt"], f8["name"]) if f8 is not None and sp is not None else
+                     "kvd_append_%s + kvd_decode_attention_%s over an %s cache "
                      "(quantising append, decode, merge kernels)" % (f8["fmt"], f8["fmt"], f8["name"])
                      if f8 is not None and args.separate_append else
                      "kvd_decode_step_%s over an %s cache (decode kernel with fused quantising "
@@ -959,7 +987,10 @@ def run_ours(args):
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "peak_kind": peak_kind,
-            "kernel": ("kvd_decode_attention_%s call (decode_kernel over %s pages + merge)"
+            "kernel": ("kvd_decode_attention_shared_prefix_%s call (prefix_tcq_kernel + decode_kernel over "
+                       "%s pages with fused quantising append + merge)" % (f8["fmt"], f8["name"])
+                       if f8 is not None and sp is not None else
+                       "kvd_decode_attention_%s call (decode_kernel over %s pages + merge)"
                        % (f8["fmt"], f8["name"]) if f8 is not None and args.separate_append else
                        "kvd_decode_step_%s call (decode_kernel over %s pages with fused quantising "
                        "append + merge)" % (f8["fmt"], f8["name"]) if f8 is not None else
@@ -970,7 +1001,9 @@ def run_ours(args):
                        "kvd_decode_step call (decode_kernel with fused append + decode_merge_kernel)")
                       + ", CUDA events on the launching stream; achieved = its algorithmic bytes / mean duration",
             "bytes_per_launch": timed_bytes,
-            "traffic": profile_traffic(w.name, (f8["fmt"] + ("_separate_append" if args.separate_append else ""))
+            "traffic": profile_traffic(w.name, (f8["fmt"] + ("_shared_prefix" if sp is not None else
+                                                             "_separate_append" if args.separate_append
+                                                             else ""))
                                       if f8 is not None else "shared_prefix" if sp is not None
                                       else "separate_append" if args.separate_append else "fused"),
         },
@@ -1064,6 +1097,8 @@ def parse_args(argv=None):
         raise SystemExit("--graph times the fused step only")
     if args.kv_fp8 + args.kv_int8 + args.kv_int4 > 1:
         raise SystemExit("--kv-fp8, --kv-int8 and --kv-int4 are exclusive")
+    if args.shared_prefix and args.separate_append:
+        raise SystemExit("--shared-prefix always fuses the append")
     return args
 
 

@@ -289,6 +289,47 @@ kvd_status kvd_decode_step_int4(const void *q, const void *k_new, const void *v_
                                 void *stream);
 
 /*
+ * kvd_decode_attention_shared_prefix_{fp8,int8,int4} -- the shared-prefix
+ * decode of kvd_decode_attention_shared_prefix over a quantised cache.
+ * "KV缓存与Flash注意力", sections 实际应用 and 练习 (prefix caching), with the
+ * cache of "KV Cache:推理慢的真正原因", section 工程优化手段 / 量化 (codes plus
+ * one fp32 scale per token, KV head and 32 channels).
+ *
+ *   k_codes, v_codes, k_scale, v_scale
+ *                 the quantised pools of kvd_decode_step_{fp8,int8,int4}
+ *                 (written only when k_new / v_new are given: the fused
+ *                 quantising append)
+ *   d             128 only (KVD_ERR_UNSUPPORTED otherwise)
+ *   other arguments as kvd_decode_attention_shared_prefix; the workspace is
+ *   kvd_shared_prefix_workspace_size(...) bytes, as there.
+ * Each shared page is dequantised once per (group, KV head) into f16/bf16
+ * tensor-core tiles, every value as a rounded head plus a rounded remainder
+ * (about 2^-22 of the value in f16, 2^-16 in bf16, is lost), so the result is
+ * that of kvd_decode_attention_{fp8,int8,int4} up to fp32 rounding order.
+ */
+kvd_status kvd_decode_attention_shared_prefix_fp8(
+    const void *q, const void *k_new, const void *v_new, uint8_t *k_codes, uint8_t *v_codes,
+    float *k_scale, float *v_scale, const int32_t *block_table, const int32_t *seq_lens, float scale,
+    void *out, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks_per_seq,
+    const int32_t *group_start, const int32_t *group_pages, int n_groups, int max_group_size,
+    int num_partitions, void *workspace, size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+    void *stream);
+kvd_status kvd_decode_attention_shared_prefix_int8(
+    const void *q, const void *k_new, const void *v_new, int8_t *k_codes, int8_t *v_codes,
+    float *k_scale, float *v_scale, const int32_t *block_table, const int32_t *seq_lens, float scale,
+    void *out, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks_per_seq,
+    const int32_t *group_start, const int32_t *group_pages, int n_groups, int max_group_size,
+    int num_partitions, void *workspace, size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+    void *stream);
+kvd_status kvd_decode_attention_shared_prefix_int4(
+    const void *q, const void *k_new, const void *v_new, uint8_t *k_codes, uint8_t *v_codes,
+    float *k_scale, float *v_scale, const int32_t *block_table, const int32_t *seq_lens, float scale,
+    void *out, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks_per_seq,
+    const int32_t *group_start, const int32_t *group_pages, int n_groups, int max_group_size,
+    int num_partitions, void *workspace, size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+    void *stream);
+
+/*
  * kvd_decode_step_fp8, kvd_decode_step_int8 -- kvd_decode_step over an 8-bit
  * cache: the quantising append of kvd_append_{fp8,int8} followed by the
  * attention of kvd_decode_attention_{fp8,int8}, in one decode launch.

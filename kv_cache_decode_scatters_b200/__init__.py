@@ -25,6 +25,8 @@ __all__ = [
     "kvd_quantize_fp8", "kvd_append_fp8", "kvd_decode_attention_fp8", "kvd_decode_step_fp8",
     "kvd_quantize_int8", "kvd_append_int8", "kvd_decode_attention_int8", "kvd_decode_step_int8",
     "kvd_quantize_int4", "kvd_append_int4", "kvd_decode_attention_int4", "kvd_decode_step_int4",
+    "kvd_decode_attention_shared_prefix_fp8", "kvd_decode_attention_shared_prefix_int8",
+    "kvd_decode_attention_shared_prefix_int4",
     "kvd_merge_lse", "kvd_read_stream", "kvd_set_decode_wait_limit", "KVD_READ_VECTOR", "KVD_READ_BULK",
     "kvd_workspace_size", "KVD_STATIC_WORKSPACE_BYTES",
     "kvd_auto_partitions", "kvd_kv_bytes_per_token", "kvd_read_device_error",
@@ -75,6 +77,9 @@ def _load():
         getattr(L, "kvd_decode_step_" + fmt).restype = I
         getattr(L, "kvd_decode_step_" + fmt).argtypes = [P, P, P, P, P, P, P, P, P, F, P, I, I, I,
                                                          I, I, I, I, P, S, P, I, P]
+        getattr(L, "kvd_decode_attention_shared_prefix_" + fmt).restype = I
+        getattr(L, "kvd_decode_attention_shared_prefix_" + fmt).argtypes = [
+            P, P, P, P, P, P, P, P, P, F, P, I, I, I, I, I, I, P, P, I, I, I, P, S, P, I, P]
     L.kvd_decode_attention_static.restype = I
     L.kvd_decode_attention_static.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, P, I, P]
     L.kvd_merge_lse.restype = I
@@ -349,6 +354,73 @@ def _decode8(fmt, q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, 
         int(num_partitions), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         lse_ptr, _dtype_code(q), _stream(stream)), name)
     return out
+
+
+def _shared_prefix8(fmt, q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, group_start,
+                    group_pages, max_group_size, scale, out, k_new, v_new, num_partitions, workspace,
+                    lse_out, stream):
+    B, H_q, d = q.shape
+    NB, H_kv, P, rb = k_codes.shape
+    if P != KVD_PAGE_TOKENS or rb != _ROW[fmt](d):
+        raise ValueError("q / cache shape mismatch")
+    n_groups = group_pages.shape[0]
+    if group_start.shape[0] != n_groups + 1:
+        raise ValueError("group_start must have n_groups + 1 entries")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new or neither")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        n = kvd_shared_prefix_workspace_size(B, H_q, H_kv, d, n_groups, max_group_size, num_partitions)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    kn = None if k_new is None else _dev(k_new, "k_new", q.dtype)
+    vn = None if v_new is None else _dev(v_new, "v_new", q.dtype)
+    lse_ptr = None if lse_out is None else _dev(lse_out, "lse_out", torch.float32)
+    c = _CODE8[fmt]
+    name = "kvd_decode_attention_shared_prefix_" + fmt
+    _check(getattr(_lib, name)(
+        _dev(q, "q", q.dtype), kn, vn, _dev(k_codes, "k_codes", c), _dev(v_codes, "v_codes", c),
+        _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+        _dev(block_table, "block_table", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
+        float(scale), _dev(out, "out", q.dtype), B, H_q, H_kv, d, NB, block_table.shape[1],
+        _dev(group_start, "group_start", torch.int32), _dev(group_pages, "group_pages", torch.int32),
+        n_groups, int(max_group_size), int(num_partitions), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), lse_ptr, _dtype_code(q), _stream(stream)), name)
+    return out
+
+
+def kvd_decode_attention_shared_prefix_fp8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                                           group_start, group_pages, max_group_size, scale=None,
+                                           out=None, k_new=None, v_new=None, num_partitions=0,
+                                           workspace=None, lse_out=None, stream=None):
+    """kvd_decode_attention_shared_prefix over the E4M3 cache (d = 128); with
+    k_new/v_new the step's token is quantised and appended as in
+    kvd_decode_step_fp8.  Returns out."""
+    return _shared_prefix8("fp8", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                           group_start, group_pages, max_group_size, scale, out, k_new, v_new,
+                           num_partitions, workspace, lse_out, stream)
+
+
+def kvd_decode_attention_shared_prefix_int8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                                            group_start, group_pages, max_group_size, scale=None,
+                                            out=None, k_new=None, v_new=None, num_partitions=0,
+                                            workspace=None, lse_out=None, stream=None):
+    """kvd_decode_attention_shared_prefix over the INT8 cache (d = 128).  Returns out."""
+    return _shared_prefix8("int8", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                           group_start, group_pages, max_group_size, scale, out, k_new, v_new,
+                           num_partitions, workspace, lse_out, stream)
+
+
+def kvd_decode_attention_shared_prefix_int4(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                                            group_start, group_pages, max_group_size, scale=None,
+                                            out=None, k_new=None, v_new=None, num_partitions=0,
+                                            workspace=None, lse_out=None, stream=None):
+    """kvd_decode_attention_shared_prefix over the INT4 cache (d = 128).  Returns out."""
+    return _shared_prefix8("int4", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                           group_start, group_pages, max_group_size, scale, out, k_new, v_new,
+                           num_partitions, workspace, lse_out, stream)
 
 
 def kvd_quantize_fp8(src, codes=None, scales=None, stream=None):

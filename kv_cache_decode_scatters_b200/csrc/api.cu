@@ -126,7 +126,7 @@ struct PrefixLayout {
 };
 
 kvd_status prefix_layout(int B, int H_kv, int G, int d, int n_groups, int max_group_size,
-                         size_t base, PrefixLayout *out) {
+                         size_t base, PrefixLayout *out, bool quantised = false) {
   int dev, sms;
   kvd_status st = current_device(&dev);
   if (st) return st;
@@ -137,10 +137,12 @@ kvd_status prefix_layout(int B, int H_kv, int G, int d, int n_groups, int max_gr
   const long long rb = (rows + rpc - 1) / rpc;
   if (rb > 65535) return fail(KVD_ERR_UNSUPPORTED, "group of %d sequences too large", max_group_size);
   // each (group, KV head, row block) unit's pages are cut into contiguous
-  // chunks, one CTA each: at d = 128 (tensor-memory pass, two CTAs per SM)
-  // about two per SM so that all are resident at once; otherwise about four
+  // chunks, one CTA each: at d = 128 (tensor-memory pass, two CTAs per SM;
+  // one for a quantised cache) as many as are resident at once; otherwise
+  // about four per SM.  The quantised layout never needs more workspace.
   const long long units = static_cast<long long>(n_groups) * H_kv * rb;
-  long long chunks = d == 128 ? (2LL * sms) / units : (4LL * sms + units - 1) / units;
+  long long chunks = d == 128 ? ((quantised ? 1LL : 2LL) * sms) / units
+                              : (4LL * sms + units - 1) / units;
   chunks = chunks < 1 ? 1 : (chunks > 64 ? 64 : chunks);
   if (static_cast<long long>(n_groups) * chunks > 0x7fffffffLL)
     return fail(KVD_ERR_UNSUPPORTED, "too many groups");
@@ -292,7 +294,8 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   if (num_partitions < 0) return fail(KVD_ERR_INVALID, "num_partitions < 0");
   if (q8) {
     if (!v_scale) return fail(KVD_ERR_INVALID, "v_scale is NULL");
-    if (n_groups > 0) return fail(KVD_ERR_UNSUPPORTED, "the 8-bit cache has no shared-prefix mode");
+    if (n_groups > 0 && d != 128)
+      return fail(KVD_ERR_UNSUPPORTED, "the shared-prefix pass over a quantised cache needs d = 128");
     if (!aligned(k_scale, 16) || !aligned(v_scale, 16))
       return fail(KVD_ERR_INVALID, "scale pools must be 16-byte aligned");
   }
@@ -313,7 +316,7 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   if (n_groups > 0) {
     if (!group_start || !group_pages) return fail(KVD_ERR_INVALID, "group_start / group_pages is NULL");
     if (max_group_size <= 0) return fail(KVD_ERR_INVALID, "max_group_size must be positive");
-    st = prefix_layout(B, H_kv, G, d, n_groups, max_group_size, L0.total, &PL);
+    st = prefix_layout(B, H_kv, G, d, n_groups, max_group_size, L0.total, &PL, q8);
     if (st) return st;
   }
   WsLayout L = L0;
@@ -436,7 +439,10 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
     pa.chunks = PL.chunks;
     pa.fused = k_new != nullptr;
     pa.maxg = max_group_size;
-    e = kvd::launch_prefix(pa, d, dt, tm[0], tm[1], PL.row_blocks, s);
+    pa.k_scale = k_scale;
+    pa.v_scale = v_scale;
+    e = q8 ? kvd::launch_prefix_q(pa, fmt, dt, tm[0], tm[1], PL.row_blocks, s)
+           : kvd::launch_prefix(pa, d, dt, tm[0], tm[1], PL.row_blocks, s);
     if (e != cudaSuccess) return cuda_fail(e, "prefix launch");
     a.skip = pa.skip;
     a.pre_o = pa.pre_o;
@@ -694,6 +700,68 @@ kvd_status kvd_decode_attention_shared_prefix(
                      num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
                      lse_out, dtype, stream, k_new, v_new, group_start, group_pages, n_groups,
                      max_group_size);
+}
+
+// The shared-prefix decode over a quantised cache (d = 128): the prefix pass
+// dequantises each staged page once for the whole group (prefix_tcq_kernel).
+static kvd_status shared_prefix_q(const void *q, const void *k_new, const void *v_new,
+                                  uint8_t *k_codes, uint8_t *v_codes, float *k_scale, float *v_scale,
+                                  const int32_t *block_table, const int32_t *seq_lens, float scale,
+                                  void *out, int B, int H_q, int H_kv, int d, int num_blocks,
+                                  int max_blocks_per_seq, const int32_t *group_start,
+                                  const int32_t *group_pages, int n_groups, int max_group_size,
+                                  int num_partitions, void *workspace, size_t workspace_bytes,
+                                  float *lse_out, kvd_dtype dtype, void *stream, kvd::Code8 fmt) {
+  if (n_groups < 0) return fail(KVD_ERR_INVALID, "n_groups < 0");
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return fail(KVD_ERR_INVALID, "k_new and v_new must both be given or both be NULL");
+  if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16)))
+    return fail(KVD_ERR_INVALID, "k_new / v_new must be 16-byte aligned");
+  if (!k_scale) return fail(KVD_ERR_INVALID, "k_scale is NULL");
+  return decode_impl(q, k_codes, v_codes, block_table, seq_lens, scale, out, B, H_q, H_kv, d,
+                     num_blocks, max_blocks_per_seq, num_partitions, workspace, workspace_bytes,
+                     lse_out, dtype, stream, k_new, v_new, group_start, group_pages, n_groups,
+                     max_group_size, k_scale, v_scale, fmt);
+}
+
+kvd_status kvd_decode_attention_shared_prefix_fp8(
+    const void *q, const void *k_new, const void *v_new, uint8_t *k_codes, uint8_t *v_codes,
+    float *k_scale, float *v_scale, const int32_t *block_table, const int32_t *seq_lens, float scale,
+    void *out, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks_per_seq,
+    const int32_t *group_start, const int32_t *group_pages, int n_groups, int max_group_size,
+    int num_partitions, void *workspace, size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+    void *stream) {
+  return shared_prefix_q(q, k_new, v_new, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                         scale, out, B, H_q, H_kv, d, num_blocks, max_blocks_per_seq, group_start,
+                         group_pages, n_groups, max_group_size, num_partitions, workspace,
+                         workspace_bytes, lse_out, dtype, stream, kvd::Code8::E4M3);
+}
+
+kvd_status kvd_decode_attention_shared_prefix_int8(
+    const void *q, const void *k_new, const void *v_new, int8_t *k_codes, int8_t *v_codes,
+    float *k_scale, float *v_scale, const int32_t *block_table, const int32_t *seq_lens, float scale,
+    void *out, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks_per_seq,
+    const int32_t *group_start, const int32_t *group_pages, int n_groups, int max_group_size,
+    int num_partitions, void *workspace, size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+    void *stream) {
+  return shared_prefix_q(q, k_new, v_new, reinterpret_cast<uint8_t *>(k_codes),
+                         reinterpret_cast<uint8_t *>(v_codes), k_scale, v_scale, block_table,
+                         seq_lens, scale, out, B, H_q, H_kv, d, num_blocks, max_blocks_per_seq,
+                         group_start, group_pages, n_groups, max_group_size, num_partitions,
+                         workspace, workspace_bytes, lse_out, dtype, stream, kvd::Code8::INT8);
+}
+
+kvd_status kvd_decode_attention_shared_prefix_int4(
+    const void *q, const void *k_new, const void *v_new, uint8_t *k_codes, uint8_t *v_codes,
+    float *k_scale, float *v_scale, const int32_t *block_table, const int32_t *seq_lens, float scale,
+    void *out, int B, int H_q, int H_kv, int d, int num_blocks, int max_blocks_per_seq,
+    const int32_t *group_start, const int32_t *group_pages, int n_groups, int max_group_size,
+    int num_partitions, void *workspace, size_t workspace_bytes, float *lse_out, kvd_dtype dtype,
+    void *stream) {
+  return shared_prefix_q(q, k_new, v_new, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
+                         scale, out, B, H_q, H_kv, d, num_blocks, max_blocks_per_seq, group_start,
+                         group_pages, n_groups, max_group_size, num_partitions, workspace,
+                         workspace_bytes, lse_out, dtype, stream, kvd::Code8::INT4);
 }
 
 kvd_status kvd_decode_step(const void *q, const void *k_new, const void *v_new, void *k_cache,

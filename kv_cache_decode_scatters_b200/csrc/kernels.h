@@ -95,6 +95,8 @@ struct PrefixArgs {
   float scale_log2;
   int B, H_q, H_kv, G, num_blocks, maxb, n_groups, chunks, fused;
   int maxg;                    // members per group at most: a larger group is invalid
+  const float *k_scale;        // quantised cache: scales [NB][H_kv][16][d/32] (else NULL)
+  const float *v_scale;
 };
 
 struct GenericMergeArgs {
@@ -128,6 +130,10 @@ cudaError_t launch_read_stream(const void *src, size_t bytes, int mode, unsigned
 // Prefix pass of the shared-prefix decode: grid (n_groups * chunks, H_kv, row blocks).
 cudaError_t launch_prefix(const PrefixArgs &a, int d, DType dt, const CUtensorMap &tmK,
                           const CUtensorMap &tmV, int row_blocks, cudaStream_t s);
+// The same pass over a quantised cache (d = 128; tensor maps over the code
+// pools, scales in a.k_scale / a.v_scale); one CTA per SM.
+cudaError_t launch_prefix_q(const PrefixArgs &a, Code8 fmt, DType dt, const CUtensorMap &tmK,
+                            const CUtensorMap &tmV, int row_blocks, cudaStream_t s);
 // Query rows one prefix CTA handles.
 int prefix_rows_per_cta();
 

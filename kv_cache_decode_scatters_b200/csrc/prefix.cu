@@ -305,13 +305,203 @@ static_assert(2 * kTcSmem <= 227 * 1024 && 3 * kTcSmem > 228 * 1024,
               "exactly two CTAs per SM: each allocates half of TMEM");
 }  // namespace
 
+// Pages of step j of a chunk [p_begin, p_end) that exist (bit p: page p of
+// the step has a valid physical page); 0 past the last step.
+__device__ __forceinline__ uint32_t tc_step_mask(const PrefixArgs &a, const int32_t *bt, int p_begin,
+                                                 int p_end, int nsteps, int j) {
+  uint32_t m = 0;
+  if (j < nsteps) {
+    const int p0 = p_begin + j * kTcPages, np = min(kTcPages, p_end - p0);
+#pragma unroll
+    for (int p = 0; p < kTcPages; ++p) {
+      const int pb = p < np ? __ldg(bt + p0 + p) : -1;
+      if (pb >= 0 && pb < a.num_blocks) m |= 1u << p;
+    }
+  }
+  return m;
+}
+
+// The softmax role of the tensor-memory passes (4 warps, one query row per
+// thread): puts its rows of Q into the swizzled Q tile, then per step reads
+// its S row from TMEM, updates the running (max, sum), writes P over S,
+// rescales O in TMEM when the reference max moves, and finally writes the
+// normalised partial (o, lse) of its row.
+template <typename T>
+__device__ __forceinline__ void tc_softmax_role(const PrefixArgs &a, uint8_t *qs, uint32_t tbase,
+                                                uint32_t S_FULL, uint32_t P_FULL, uint32_t O_DONE,
+                                                uint32_t Q_FULL, int warp, int lane, int r0, int rows,
+                                                int s0, int h, int chunk, int nsteps,
+                                                const int32_t *bt, int p_begin, int p_end) {
+  constexpr int D = 128;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  using M = Mma<T>;
+  const int quarter = warp & 3;
+  const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
+  const int row = r0 + quarter * 32 + lane;  // row of the group: member row / G, head row % G
+  const bool live = row < rows;
+  const int b = s0 + (live ? row / a.G : 0), jr = live ? row % a.G : 0;
+  {
+    // this row of Q into the K-major, 128-byte-swizzled tile the MMA reads
+    const int r = quarter * 32 + lane;
+    const uint4 *qv = reinterpret_cast<const uint4 *>(
+        static_cast<const T *>(a.q) +
+        (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + jr) * D);
+#pragma unroll
+    for (int c = 0; c < 2 * 8; ++c) {
+      const uint4 v = live ? __ldg(qv + c) : make_uint4(0u, 0u, 0u, 0u);
+      const int half = c >> 3, cc = c & 7;
+      *reinterpret_cast<uint4 *>(qs + half * (kTcQBytes / 2) + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();  // visible to the tensor core's reads
+    __syncwarp();
+    if (lane == 0) mbar_arrive(Q_FULL);
+  }
+
+  float m_ref = -INFINITY, l = 0.f;
+  bool ok = true;
+  uint32_t next_mask = tc_step_mask(a, bt, p_begin, p_end, nsteps, 0);  // loaded one step before use
+  for (int j = 0; j < nsteps; ++j) {
+    const int bs = j & 1;
+    const uint32_t pm = next_mask;
+    next_mask = tc_step_mask(a, bt, p_begin, p_end, nsteps, j + 1);
+    const bool got = mbar_wait_bounded(S_FULL + 8 * bs, (j >> 1) & 1);
+    if (!__all_sync(0xffffffffu, got)) {
+      ok = false;
+      break;
+    }
+    tc::fence_after_sync();
+    float x[kTcTok];
+    {
+      uint32_t r0v[32], r1v[32];
+      tc::ld32(tbase + lanes + kColS + bs * kTcTok, r0v);
+      tc::ld32(tbase + lanes + kColS + bs * kTcTok + 32, r1v);
+      tc::wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        x[i] = __uint_as_float(r0v[i]);
+        x[32 + i] = __uint_as_float(r1v[i]);
+      }
+    }
+    // row maximum of the scaled scores (in log2 units): the scale is folded
+    // into the exponent below, so the raw scores are compared (their
+    // minimum when the scale is negative); masked columns are -inf
+    const float c = a.scale_log2;
+    const bool full_step = pm == (1u << kTcPages) - 1u;  // warp-uniform
+    if (!full_step) {
+#pragma unroll
+      for (int i = 0; i < kTcTok; ++i)
+        if (!((pm >> (i / kPage)) & 1u)) x[i] = c >= 0.f ? -INFINITY : INFINITY;
+    }
+    float e4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) e4[k] = x[k];
+    if (c >= 0.f) {
+#pragma unroll
+      for (int i = 4; i < kTcTok; ++i) e4[i & 3] = fmaxf(e4[i & 3], x[i]);
+    } else {
+#pragma unroll
+      for (int i = 4; i < kTcTok; ++i) e4[i & 3] = fminf(e4[i & 3], x[i]);
+    }
+    const float ext = c >= 0.f ? fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]))
+                               : fminf(fminf(e4[0], e4[1]), fminf(e4[2], e4[3]));
+    // an all-masked row keeps -inf; otherwise the largest scaled score
+    const float mx = (ext == INFINITY || ext == -INFINITY) ? -INFINITY : ext * c;
+    const float m_new = mx > m_ref + kRefSlack ? mx : m_ref;
+    const float alpha = m_new == m_ref ? 1.f : fast_exp2(m_ref - m_new);
+    const float m_use = m_new == -INFINITY ? 0.f : m_new;
+    uint32_t ph[kTcTok / 2], pl[kTcTok / 2];
+    float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+    // exp2(s * c - m) per column; masked columns (partial steps only) are 0
+    auto exps = [&](auto masked) {
+#pragma unroll
+      for (int i = 0; i < kTcTok; i += 2) {
+        float e0 = fast_exp2(fmaf(x[i], c, -m_use));
+        float e1 = fast_exp2(fmaf(x[i + 1], c, -m_use));
+        if constexpr (decltype(masked)::value) {
+          const bool v = (pm >> (i / kPage)) & 1u;  // both columns are in one page
+          e0 = v ? e0 : 0.f;
+          e1 = v ? e1 : 0.f;
+        }
+        ph[i / 2] = M::pack(e0, e1);
+        if constexpr (kBf16) {
+          const float2 r = M::unpack(ph[i / 2]);
+          pl[i / 2] = M::pack(e0 - r.x, e1 - r.y);
+        }
+        sum4[(i / 2) & 3] += e0 + e1;
+      }
+    };
+    if (full_step) exps(std::false_type{});
+    else exps(std::true_type{});
+    const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+    l = l * alpha + sum;
+    tc::st32(tbase + lanes + kColS + bs * kTcTok, ph);
+    if constexpr (kBf16) tc::st32(tbase + lanes + kColS + bs * kTcTok + kTcTok / 2, pl);
+    if (j >= 1) {
+      // O holds the product of step j-1 once its o_done phase completes
+      const bool got2 = mbar_wait_bounded(O_DONE, (j - 1) & 1);
+      if (!__all_sync(0xffffffffu, got2)) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tc::ld32(tbase + lanes + kColO + c * 32, r);
+          tc::wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tc::st32(tbase + lanes + kColO + c * 32, r);
+        }
+      }
+    }
+    m_ref = m_new;
+    tc::wait_st();
+    tc::fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(P_FULL + 8 * bs);
+  }
+  if (ok) {
+    const bool got = mbar_wait_bounded(O_DONE, (nsteps - 1) & 1);
+    ok = __all_sync(0xffffffffu, got);
+  }
+  if (!ok) {
+    if (lane == 0) flag_error(a.err, kErrTimeout);
+  } else {
+    tc::fence_after_sync();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const float lse = l > 0.f ? (m_ref + fast_log2(l)) * kLn2 : -INFINITY;
+    const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + b) * a.G + jr;
+    float4 *o = reinterpret_cast<float4 *>(a.pre_o + idx * D);
+    const uint64_t keep = l2_policy_evict_last();  // read again by the merge
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t r[32];
+      tc::ld32(tbase + lanes + kColO + c * 32, r);
+      tc::wait_ld();
+      if (live) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const float4 v = l > 0.f ? make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
+                                                 __uint_as_float(r[i + 2]) * inv,
+                                                 __uint_as_float(r[i + 3]) * inv)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+          st_keep4(o + c * 8 + i / 4, v, keep);
+        }
+      }
+      __syncwarp();
+    }
+    if (live) st_keep(a.pre_lse + idx, lse, keep);
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(32 * kTcWarps, 2)
     prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV) {
   constexpr int D = 128;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-  using M = Mma<T>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *qs = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
@@ -353,19 +543,6 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
   }
   const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
   auto step_pages = [&](int j) { return min(kTcPages, p_end - (p_begin + j * kTcPages)); };
-  // pages of step j that exist (bit p: page p of the step)
-  auto step_mask = [&](int j) -> uint32_t {
-    uint32_t m = 0;
-    if (j < nsteps) {
-      const int p0 = p_begin + j * kTcPages, np = step_pages(j);
-#pragma unroll
-      for (int p = 0; p < kTcPages; ++p) {
-        const int pb = p < np ? __ldg(bt + p0 + p) : -1;
-        if (pb >= 0 && pb < a.num_blocks) m |= 1u << p;
-      }
-    }
-    return m;
-  };
 
   const uint32_t q0 = smem_u32(qs), ring0 = smem_u32(ring), bar0 = smem_u32(bars);
   // K and V halves of a stage have their own barriers: K is released as soon
@@ -510,7 +687,8 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
                mbar_wait_bounded(FULL_V(j % kTcStages), (j / kTcStages) & 1);
       };
       for (int j = 0; ok && j < nsteps; ++j) {
-        if (j & 1) pv_mask1 = step_mask(j); else pv_mask0 = step_mask(j);
+        if (j & 1) pv_mask1 = tc_step_mask(a, bt, p_begin, p_end, nsteps, j);
+        else pv_mask0 = tc_step_mask(a, bt, p_begin, p_end, nsteps, j);
         if (!mbar_wait_bounded(FULL_K(j % kTcStages), (j / kTcStages) & 1)) {
           ok = false;
           break;
@@ -542,165 +720,380 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int quarter = warp & 3;
-    const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
-    const int row = r0 + quarter * 32 + lane;  // row of the group: member row / G, head row % G
-    const bool live = row < rows;
-    const int b = s0 + (live ? row / a.G : 0), jr = live ? row % a.G : 0;
-    {
-      // this row of Q into the K-major, 128-byte-swizzled tile the MMA reads
-      const int r = quarter * 32 + lane;
-      const uint4 *qv = reinterpret_cast<const uint4 *>(
-          static_cast<const T *>(a.q) +
-          (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + jr) * D);
-#pragma unroll
-      for (int c = 0; c < 2 * 8; ++c) {
-        const uint4 v = live ? __ldg(qv + c) : make_uint4(0u, 0u, 0u, 0u);
-        const int half = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4 *>(qs + half * (kTcQBytes / 2) + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();  // visible to the tensor core's reads
-      __syncwarp();
-      if (lane == 0) mbar_arrive(Q_FULL);
-    }
+    tc_softmax_role<T>(a, qs, tbase, S_FULL, P_FULL, O_DONE, Q_FULL, warp, lane, r0, rows, s0, h,
+                       chunk, nsteps, bt, p_begin, p_end);
+  }
 
-    float m_ref = -INFINITY, l = 0.f;
-    bool ok = true;
-    uint32_t next_mask = step_mask(0);  // loaded one step before use
-    for (int j = 0; j < nsteps; ++j) {
-      const int bs = j & 1;
-      const uint32_t pm = next_mask;
-      next_mask = step_mask(j + 1);
-      const bool got = mbar_wait_bounded(S_FULL + 8 * bs, (j >> 1) & 1);
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-      float x[kTcTok];
-      {
-        uint32_t r0v[32], r1v[32];
-        tc::ld32(tbase + lanes + kColS + bs * kTcTok, r0v);
-        tc::ld32(tbase + lanes + kColS + bs * kTcTok + 32, r1v);
-        tc::wait_ld();
+  // release TMEM once every role is done with it
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------
+// The tensor-memory pass over a quantised cache (E4M3, INT8 or INT4 codes,
+// one fp32 scale per token, KV head and 32 channels; d = 128).
+//
+// The tensor core multiplies 16-bit operands, and a cached value is s * code
+// with an fp32 scale.  Rounded once to the operand type it would be off by up
+// to half an ulp (2^-11 relative in f16), which reaches the fp16 tolerance of
+// the output.  So each value is carried as a rounded head and a rounded
+// remainder, hi = RN(s * code) and lo = RN(s * code - hi), in two operand
+// tiles, and
+//     S = Q . K_hi^T + Q . K_lo^T,      O += P . V_hi + P . V_lo
+// (bf16 adds the probability remainder times V_hi, as in the 16-bit pass).
+// What is left is about 2^-22 (f16) or 2^-16 (bf16) of each value.
+//
+// Roles (320 threads): those of the 16-bit pass plus four dequantise warps
+// (6-9).  The producer copies a step's codes (2-D TMA boxes, swizzled by the
+// code row size) and scale rows (bulk copies) into a code stage.  The
+// dequantise warps turn them into the four operand tiles -- K hi, K lo, V hi,
+// V lo, each laid out as the TMA lays out a 16-bit page (64-channel halves,
+// 128-byte rows, 128-byte swizzle) -- and hand the code stage back.  The MMA
+// issuer waits for the tiles instead of the copies.  Per stage and per K / V:
+// codes landed (TMA / bulk bytes), codes consumed and tiles written (one
+// arrive per dequantise warp), tiles read (tcgen05.commit).  About 197 KB of
+// shared memory: one CTA per SM.
+namespace {
+constexpr int kTqWarps = 10;
+constexpr int kTqStage = 8 * kTcHalf;  // K hi, K lo, V hi, V lo: two halves each (64 KB)
+constexpr int kTqScalePage = kPage * 4 * 4;  // fp32 scales of one page and head (d = 128)
+
+template <Code8 kFmt>
+struct TqGeo {
+  static constexpr int kRow = kFmt == Code8::INT4 ? 64 : 128;  // code bytes of a token (d = 128)
+  static constexpr int kCodePage = kPage * kRow;
+  static constexpr int kCodeStage = 2 * kTcPages * kCodePage;         // K then V codes of a step
+  static constexpr int kScaleStage = 2 * kTcPages * kTqScalePage;     // K then V scales
+  static constexpr int kBars = 8 * kTcStages + 7;
+  static constexpr size_t kSmem = 1024 + kTcQBytes +
+                                  (size_t)kTcStages * (kTqStage + kCodeStage + kScaleStage) +
+                                  kBars * 8 + 64;
+  static_assert(kSmem <= 227 * 1024, "one CTA per SM");
+};
+
+// Dequantise the K (or V) half of one code stage into its hi and lo operand
+// tiles; thread ct of the 128 dequantise threads.  A unit is one 16-byte
+// chunk of one token's codes: 16 channels (8-bit) or 32 (INT4), all in one
+// scale group.
+template <typename T, Code8 kFmt>
+__device__ __forceinline__ void dequant_half(const uint8_t *codes, const float *scl, uint8_t *hi,
+                                             uint8_t *lo, int ct) {
+  using M = Mma<T>;
+  constexpr int kRow = TqGeo<kFmt>::kRow;
+  constexpr int kPerRow = kRow / 16;        // chunks of a code row
+  constexpr int kChan = 128 / kPerRow;      // channels of a chunk
+  constexpr int kUnits = kTcPages * kPage * kPerRow;
+#pragma unroll 1
+  for (int u = ct; u < kUnits; u += 128) {
+    const int c = u % kPerRow, t = (u / kPerRow) % kPage, p = u / (kPerRow * kPage);
+    const uint4 w = *reinterpret_cast<const uint4 *>(codes + p * kPage * kRow + swz_rows<kRow>(t, c));
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    const int ch0 = c * kChan;
+    const float sc = scl[(p * kPage + t) * 4 + ch0 / 32];
+    float v[kChan];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          x[i] = __uint_as_float(r0v[i]);
-          x[32 + i] = __uint_as_float(r1v[i]);
+    for (int k = 0; k < 4; ++k) {
+      if constexpr (kFmt == Code8::INT4) {
+        uint32_t f[4];  // f[s]: channels 8k + s (low half) and 8k + s + 4 (high half)
+        int4x8_to_f16x2x4(words[k], f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 x = __half22float2(*reinterpret_cast<const __half2 *>(&f[q]));
+          v[8 * k + q] = x.x;
+          v[8 * k + q + 4] = x.y;
         }
-      }
-      // row maximum of the scaled scores (in log2 units): the scale is folded
-      // into the exponent below, so the raw scores are compared (their
-      // minimum when the scale is negative); masked columns are -inf
-      const float c = a.scale_log2;
-      const bool full_step = pm == (1u << kTcPages) - 1u;  // warp-uniform
-      if (!full_step) {
-#pragma unroll
-        for (int i = 0; i < kTcTok; ++i)
-          if (!((pm >> (i / kPage)) & 1u)) x[i] = c >= 0.f ? -INFINITY : INFINITY;
-      }
-      float e4[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) e4[k] = x[k];
-      if (c >= 0.f) {
-#pragma unroll
-        for (int i = 4; i < kTcTok; ++i) e4[i & 3] = fmaxf(e4[i & 3], x[i]);
       } else {
-#pragma unroll
-        for (int i = 4; i < kTcTok; ++i) e4[i & 3] = fminf(e4[i & 3], x[i]);
+        uint32_t lo2, hi2;  // channels (4k, 4k + 1), (4k + 2, 4k + 3)
+        code8x4_to_f16x2x2<kFmt>(words[k], lo2, hi2);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&lo2));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&hi2));
+        v[4 * k] = a.x;
+        v[4 * k + 1] = a.y;
+        v[4 * k + 2] = b.x;
+        v[4 * k + 3] = b.y;
       }
-      const float ext = c >= 0.f ? fmaxf(fmaxf(e4[0], e4[1]), fmaxf(e4[2], e4[3]))
-                                 : fminf(fminf(e4[0], e4[1]), fminf(e4[2], e4[3]));
-      // an all-masked row keeps -inf; otherwise the largest scaled score
-      const float mx = (ext == INFINITY || ext == -INFINITY) ? -INFINITY : ext * c;
-      const float m_new = mx > m_ref + kRefSlack ? mx : m_ref;
-      const float alpha = m_new == m_ref ? 1.f : fast_exp2(m_ref - m_new);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      uint32_t ph[kTcTok / 2], pl[kTcTok / 2];
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-      // exp2(s * c - m) per column; masked columns (partial steps only) are 0
-      auto exps = [&](auto masked) {
+    }
+    const int r = p * kPage + t;  // row of the step's 64 tokens
 #pragma unroll
-        for (int i = 0; i < kTcTok; i += 2) {
-          float e0 = fast_exp2(fmaf(x[i], c, -m_use));
-          float e1 = fast_exp2(fmaf(x[i + 1], c, -m_use));
-          if constexpr (decltype(masked)::value) {
-            const bool v = (pm >> (i / kPage)) & 1u;  // both columns are in one page
-            e0 = v ? e0 : 0.f;
-            e1 = v ? e1 : 0.f;
+    for (int k = 0; k < kChan / 8; ++k) {
+      const int ch = ch0 + 8 * k, hf = ch / 64, cc = (ch % 64) / 8;
+      uint32_t h4[4], l4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float x0 = v[8 * k + 2 * i] * sc, x1 = v[8 * k + 2 * i + 1] * sc;
+        h4[i] = M::pack(x0, x1);
+        const float2 hv = M::unpack(h4[i]);
+        l4[i] = M::pack(x0 - hv.x, x1 - hv.y);
+      }
+      const int off = hf * kTcHalf + r * 128 + ((cc ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4 *>(hi + off) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+      *reinterpret_cast<uint4 *>(lo + off) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+    }
+  }
+}
+}  // namespace
+
+template <typename T, Code8 kFmt>
+__global__ void __launch_bounds__(32 * kTqWarps, 1)
+    prefix_tcq_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV) {
+  constexpr int D = 128;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  using Gq = TqGeo<kFmt>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *qs = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  uint8_t *tiles = qs + kTcQBytes;
+  uint8_t *codes = tiles + (size_t)kTcStages * kTqStage;
+  uint8_t *scl = codes + (size_t)kTcStages * Gq::kCodeStage;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(scl + (size_t)kTcStages * Gq::kScaleStage);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Gq::kBars);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cap = a.maxb * kPage;
+
+  grid_dependency_wait();
+  grid_launch_dependents();
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) write_skip(a, cap);
+
+  const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
+  const int h = blockIdx.y;
+  const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
+  const int gp = __ldg(a.group_pages + g);
+  if (!group_ok(a, s0, s1, gp)) {
+    if (tid == 0) flag_error(a.err, kErrSeqLen);
+    return;
+  }
+  const int rows = (s1 - s0) * a.G;
+  const int r0 = blockIdx.z * kRowsPerCta;
+  if (r0 >= rows || gp == 0) return;
+  const int p_begin = static_cast<int>((static_cast<long long>(chunk) * gp) / a.chunks);
+  const int p_end = static_cast<int>((static_cast<long long>(chunk + 1) * gp) / a.chunks);
+  const int nsteps = (p_end - p_begin + kTcPages - 1) / kTcPages;
+  if (nsteps == 0) {  // an empty chunk leaves empty partials
+    for (int r = tid; r < kRowsPerCta; r += blockDim.x) {
+      const int row = r0 + r;
+      if (row >= rows) continue;
+      const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + s0 + row / a.G) * a.G +
+                         row % a.G;
+      for (int c = 0; c < D; ++c) a.pre_o[idx * D + c] = 0.f;
+      a.pre_lse[idx] = -INFINITY;
+    }
+    return;
+  }
+  const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
+  auto step_pages = [&](int j) { return min(kTcPages, p_end - (p_begin + j * kTcPages)); };
+
+  const uint32_t q0 = smem_u32(qs), tiles0 = smem_u32(tiles), codes0 = smem_u32(codes);
+  const uint32_t scl0 = smem_u32(scl), bar0 = smem_u32(bars);
+  // kv = 0: K, 1: V
+  auto CFULL = [&](int kv, int s) { return bar0 + 8 * (kv * kTcStages + s); };
+  auto CFREE = [&](int kv, int s) { return bar0 + 8 * ((2 + kv) * kTcStages + s); };
+  auto TFULL = [&](int kv, int s) { return bar0 + 8 * ((4 + kv) * kTcStages + s); };
+  auto TFREE = [&](int kv, int s) { return bar0 + 8 * ((6 + kv) * kTcStages + s); };
+  const uint32_t S_FULL = bar0 + 8 * (8 * kTcStages);  // + 8 * buffer
+  const uint32_t P_FULL = S_FULL + 16;                 // + 8 * buffer
+  const uint32_t O_DONE = S_FULL + 32, Q_FULL = S_FULL + 40, DRAIN = S_FULL + 48;
+
+  if (warp == 0) {
+    __syncwarp();
+    tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  if (tid == 32) {
+    for (int kv = 0; kv < 2; ++kv)
+      for (int s = 0; s < kTcStages; ++s) {
+        mbar_init(CFULL(kv, s), 1);
+        mbar_init(CFREE(kv, s), 4);
+        mbar_init(TFULL(kv, s), 4);
+        mbar_init(TFREE(kv, s), 1);
+      }
+    mbar_init(S_FULL, 1);
+    mbar_init(S_FULL + 8, 1);
+    mbar_init(P_FULL, 4);
+    mbar_init(P_FULL + 8, 4);
+    mbar_init(O_DONE, 1);
+    mbar_init(Q_FULL, 4);
+    mbar_init(DRAIN, 1);
+    mbar_init_fence();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      const uint64_t policy = l2_policy_evict_normal();
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < nsteps && ok; ++j) {
+        const int s = j % kTcStages;
+        const uint32_t rel = ((j / kTcStages) - 1) & 1;  // phase of step j - kTcStages
+        const int p0 = p_begin + j * kTcPages, np = step_pages(j);
+        int prow[kTcPages];
+        int good = 0;
+#pragma unroll
+        for (int p = 0; p < kTcPages; ++p) {
+          prow[p] = -1;
+          if (p < np) {
+            const int pb = __ldg(bt + p0 + p);
+            if (pb >= 0 && pb < a.num_blocks) {
+              prow[p] = (pb * a.H_kv + h) * kPage;
+              ++good;
+            } else {
+              flag_error(a.err, kErrBlockTable);
+            }
           }
-          ph[i / 2] = M::pack(e0, e1);
-          if constexpr (kBf16) {
-            const float2 r = M::unpack(ph[i / 2]);
-            pl[i / 2] = M::pack(e0 - r.x, e1 - r.y);
-          }
-          sum4[(i / 2) & 3] += e0 + e1;
         }
+        const uint32_t bytes = static_cast<uint32_t>(good) * (Gq::kCodePage + kTqScalePage);
+        for (int kv = 0; kv < 2; ++kv) {
+          // the codes of step j - kTcStages have been dequantised
+          if (j >= kTcStages && !mbar_wait_bounded(CFREE(kv, s), rel)) {
+            flag_error(a.err, kErrTimeout);
+            ok = false;
+            break;
+          }
+          const uint32_t cst = codes0 + s * Gq::kCodeStage + kv * kTcPages * Gq::kCodePage;
+          const uint32_t sst = scl0 + s * Gq::kScaleStage + kv * kTcPages * kTqScalePage;
+          const float *gs = kv ? a.v_scale : a.k_scale;
+          mbar_arrive_expect_tx(CFULL(kv, s), bytes);
+#pragma unroll
+          for (int p = 0; p < kTcPages; ++p) {
+            if (prow[p] < 0) continue;
+            tma_load_2d(cst + p * Gq::kCodePage, kv ? &tmV : &tmK, 0, prow[p], CFULL(kv, s), policy);
+            bulk_load(sst + p * kTqScalePage, gs + static_cast<size_t>(prow[p]) * 4, kTqScalePage,
+                      CFULL(kv, s));
+          }
+        }
+        if (ok) issued = j + 1;
+      }
+      // the copies of the last stages have landed before the CTA exits
+      for (int j = max(0, issued - kTcStages); j < issued; ++j)
+        for (int kv = 0; kv < 2; ++kv) mbar_wait_bounded(CFULL(kv, j % kTcStages), (j / kTcStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t fmt = kBf16 ? 1u : 0u;
+      bool ok = mbar_wait_bounded(Q_FULL, 0);
+      tc::fence_after_sync();
+      bool o_started = false;
+      auto issue_qk = [&](int j) {
+        const int b = j & 1;
+        const uint32_t idesc = tc::idesc_f16(fmt, static_cast<uint32_t>(step_pages(j) * kPage), false);
+        const uint32_t kst = tiles0 + (j % kTcStages) * kTqStage;
+#pragma unroll
+        for (int part = 0; part < 2; ++part)  // K hi, then K lo
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t kaddr = kst + (2 * part + (k >> 2)) * kTcHalf + (k & 3) * 32;
+            const uint32_t qaddr = q0 + (k >> 2) * (kTcQBytes / 2) + (k & 3) * 32;
+            tc::mma_ss(tbase + kColS + b * kTcTok, tc::smem_desc(qaddr, 16, 1024),
+                       tc::smem_desc(kaddr, 16, 1024), idesc, part > 0 || k > 0);
+          }
+        tc::commit(TFREE(0, j % kTcStages));
+        tc::commit(S_FULL + 8 * b);
       };
-      if (full_step) exps(std::false_type{});
-      else exps(std::true_type{});
-      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-      l = l * alpha + sum;
-      tc::st32(tbase + lanes + kColS + bs * kTcTok, ph);
-      if constexpr (kBf16) tc::st32(tbase + lanes + kColS + bs * kTcTok + kTcTok / 2, pl);
-      if (j >= 1) {
-        // O holds the product of step j-1 once its o_done phase completes
-        const bool got2 = mbar_wait_bounded(O_DONE, (j - 1) & 1);
-        if (!__all_sync(0xffffffffu, got2)) {
+      uint32_t pv_mask0 = 0u, pv_mask1 = 0u;  // loaded one step before the PV product uses it
+      auto issue_pv = [&](int j) {
+        const int b = j & 1, s = j % kTcStages;
+        const int np = step_pages(j);
+        const uint32_t mask = (j & 1) ? pv_mask1 : pv_mask0;
+        const uint32_t idesc = tc::idesc_f16(fmt, D, true);
+        const uint32_t vhi = tiles0 + s * kTqStage + 4 * kTcHalf, vlo = vhi + 2 * kTcHalf;
+        for (int kk = 0; kk < np; ++kk) {
+          if (!((mask >> kk) & 1u)) continue;  // (its scores are masked; its tiles are stale)
+          const uint64_t dh = tc::smem_desc(vhi + kk * kPage * 128, kTcHalf, 1024);
+          const uint64_t dl = tc::smem_desc(vlo + kk * kPage * 128, kTcHalf, 1024);
+          const uint32_t pa = tbase + kColS + b * kTcTok + kk * 8;  // P over S; remainder at +32
+          tc::mma_ts(tbase + kColO, pa, dh, idesc, o_started);
+          o_started = true;
+          tc::mma_ts(tbase + kColO, pa, dl, idesc, true);
+          if (kBf16) tc::mma_ts(tbase + kColO, pa + kTcTok / 2, dh, idesc, true);
+        }
+        tc::commit(TFREE(1, s));
+        tc::commit(O_DONE);
+      };
+      auto wait_pv = [&](int j) {
+        return mbar_wait_bounded(P_FULL + 8 * (j & 1), (j >> 1) & 1) &&
+               mbar_wait_bounded(TFULL(1, j % kTcStages), (j / kTcStages) & 1);
+      };
+      for (int j = 0; ok && j < nsteps; ++j) {
+        if (j & 1) pv_mask1 = tc_step_mask(a, bt, p_begin, p_end, nsteps, j);
+        else pv_mask0 = tc_step_mask(a, bt, p_begin, p_end, nsteps, j);
+        if (!mbar_wait_bounded(TFULL(0, j % kTcStages), (j / kTcStages) & 1)) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tc::ld32(tbase + lanes + kColO + c * 32, r);
-            tc::wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tc::st32(tbase + lanes + kColO + c * 32, r);
+        issue_qk(j);
+        if (j >= 1) {
+          if (!wait_pv(j - 1)) {
+            ok = false;
+            break;
           }
+          tc::fence_after_sync();
+          issue_pv(j - 1);
         }
       }
-      m_ref = m_new;
-      tc::wait_st();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(P_FULL + 8 * bs);
-    }
-    if (ok) {
-      const bool got = mbar_wait_bounded(O_DONE, (nsteps - 1) & 1);
-      ok = __all_sync(0xffffffffu, got);
-    }
-    if (!ok) {
-      if (lane == 0) flag_error(a.err, kErrTimeout);
-    } else {
-      tc::fence_after_sync();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float lse = l > 0.f ? (m_ref + fast_log2(l)) * kLn2 : -INFINITY;
-      const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + b) * a.G + jr;
-      float4 *o = reinterpret_cast<float4 *>(a.pre_o + idx * D);
-      const uint64_t keep = l2_policy_evict_last();  // read again by the merge
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tc::ld32(tbase + lanes + kColO + c * 32, r);
-        tc::wait_ld();
-        if (live) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float4 v = l > 0.f ? make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
-                                                   __uint_as_float(r[i + 2]) * inv,
-                                                   __uint_as_float(r[i + 3]) * inv)
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-            st_keep4(o + c * 8 + i / 4, v, keep);
-          }
+      if (ok) {
+        const int j = nsteps - 1;
+        if (wait_pv(j)) {
+          tc::fence_after_sync();
+          issue_pv(j);
+        } else {
+          ok = false;
         }
+      }
+      if (!ok) flag_error(a.err, kErrTimeout);
+      // every MMA issued here completes before TMEM is released
+      tc::commit(DRAIN);
+      mbar_wait_bounded(DRAIN, 0);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ softmax
+    tc_softmax_role<T>(a, qs, tbase, S_FULL, P_FULL, O_DONE, Q_FULL, warp, lane, r0, rows, s0, h,
+                       chunk, nsteps, bt, p_begin, p_end);
+  } else {
+    // ------------------------------------------------------------ dequantise
+    const int ct = tid - 6 * 32;
+    bool ok = true;
+    for (int j = 0; ok && j < nsteps; ++j) {
+      const int s = j % kTcStages;
+      const uint32_t ph = (j / kTcStages) & 1, rel = ((j / kTcStages) - 1) & 1;
+      for (int kv = 0; kv < 2; ++kv) {
+        // this step's codes have landed, and the MMAs of step j - kTcStages
+        // have finished reading the tiles they are about to overwrite
+        bool got = mbar_wait_bounded(CFULL(kv, s), ph);
+        if (j >= kTcStages) got = got && mbar_wait_bounded(TFREE(kv, s), rel);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        uint8_t *hi = tiles + (size_t)s * kTqStage + kv * 4 * kTcHalf;
+        dequant_half<T, kFmt>(codes + (size_t)s * Gq::kCodeStage + kv * kTcPages * Gq::kCodePage,
+                              reinterpret_cast<const float *>(scl + (size_t)s * Gq::kScaleStage +
+                                                              kv * kTcPages * kTqScalePage),
+                              hi, hi + 2 * kTcHalf, ct);
+        fence_proxy_async_smem();  // tiles visible to the tensor core; codes read before refill
         __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(TFULL(kv, s));
+          mbar_arrive(CFREE(kv, s));
+        }
       }
-      if (live) st_keep(a.pre_lse + idx, lse, keep);
     }
+    if (!ok && lane == 0) flag_error(a.err, kErrTimeout);
   }
 
   // release TMEM once every role is done with it
@@ -739,6 +1132,37 @@ cudaError_t launch_prefix_t(const PrefixArgs &a, const CUtensorMap &tmK, const C
   return launch_pdl(kern, grid, dim3(32 * kWarps), smem, st, a, tmK, tmV);
 }
 }  // namespace
+
+namespace {
+template <typename T, Code8 kFmt>
+cudaError_t launch_prefix_q_t(const PrefixArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                              int row_blocks, cudaStream_t st) {
+  auto kern = prefix_tcq_kernel<T, kFmt>;
+  constexpr size_t smem = TqGeo<kFmt>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.n_groups * a.chunks, a.H_kv, row_blocks);
+  return launch_pdl(kern, grid, dim3(32 * kTqWarps), smem, st, a, tmK, tmV);
+}
+
+template <typename T>
+cudaError_t launch_prefix_q_d(const PrefixArgs &a, Code8 fmt, const CUtensorMap &tmK,
+                              const CUtensorMap &tmV, int row_blocks, cudaStream_t st) {
+  switch (fmt) {
+    case Code8::E4M3: return launch_prefix_q_t<T, Code8::E4M3>(a, tmK, tmV, row_blocks, st);
+    case Code8::INT8: return launch_prefix_q_t<T, Code8::INT8>(a, tmK, tmV, row_blocks, st);
+    default: return launch_prefix_q_t<T, Code8::INT4>(a, tmK, tmV, row_blocks, st);
+  }
+}
+}  // namespace
+
+cudaError_t launch_prefix_q(const PrefixArgs &a, Code8 fmt, DType dt, const CUtensorMap &tmK,
+                            const CUtensorMap &tmV, int row_blocks, cudaStream_t s) {
+  if (a.n_groups == 0 || a.B == 0) return cudaSuccess;
+  return dt == DType::BF16 ? launch_prefix_q_d<__nv_bfloat16>(a, fmt, tmK, tmV, row_blocks, s)
+                           : launch_prefix_q_d<__half>(a, fmt, tmK, tmV, row_blocks, s);
+}
 
 cudaError_t launch_prefix(const PrefixArgs &a, int d, DType dt, const CUtensorMap &tmK,
                           const CUtensorMap &tmV, int row_blocks, cudaStream_t s) {

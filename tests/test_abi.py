@@ -280,6 +280,31 @@ def test_shared_prefix_validation(kw, status):
     assert kvd.kvd_last_error() != ""
 
 
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "int4"])
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=64), kvd.KVD_ERR_UNSUPPORTED),                # the quantised prefix pass is d = 128
+    (dict(ng=-1), kvd.KVD_ERR_INVALID),
+    (dict(kn=DUMMY, vn=NULL), kvd.KVD_ERR_INVALID),       # both or neither
+    (dict(kn=MISALIGNED, vn=DUMMY), kvd.KVD_ERR_INVALID),
+    (dict(ks=NULL), kvd.KVD_ERR_INVALID),
+    (dict(vs=NULL), kvd.KVD_ERR_INVALID),
+    (dict(ks=ctypes.c_void_p(256 + 8)), kvd.KVD_ERR_INVALID),
+    (dict(gs=NULL), kvd.KVD_ERR_INVALID),
+    (dict(mg=0), kvd.KVD_ERR_INVALID),
+])
+def test_shared_prefix_quantised_validation(fmt, kw, status):
+    a = dict(q=DUMMY, kn=NULL, vn=NULL, k=DUMMY, v=DUMMY, ks=DUMMY, vs=DUMMY, bt=DUMMY, sl=DUMMY,
+             scale=0.125, out=DUMMY, B=4, H_q=8, H_kv=2, d=128, NB=16, maxb=4, gs=DUMMY, gp=DUMMY, ng=2,
+             mg=2, parts=4, ws=DUMMY, wsb=1 << 30, lse=NULL, dt=kvd.KVD_F16, stream=NULL)
+    a.update(kw)
+    st = getattr(L, "kvd_decode_attention_shared_prefix_" + fmt)(
+        a["q"], a["kn"], a["vn"], a["k"], a["v"], a["ks"], a["vs"], a["bt"], a["sl"], a["scale"],
+        a["out"], a["B"], a["H_q"], a["H_kv"], a["d"], a["NB"], a["maxb"], a["gs"], a["gp"], a["ng"],
+        a["mg"], a["parts"], a["ws"], a["wsb"], a["lse"], a["dt"], a["stream"])
+    assert st == status
+    assert kvd.kvd_last_error() != ""
+
+
 @pytest.mark.parametrize("kw,status", [
     (dict(mode=2), kvd.KVD_ERR_INVALID),
     (dict(nbytes=24), kvd.KVD_ERR_INVALID),
