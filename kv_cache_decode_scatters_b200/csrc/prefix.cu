@@ -297,6 +297,10 @@ constexpr int kTcQBytes = kRowsPerCta * 128 * 2;  // Q tile, two 64-column halve
 constexpr uint32_t kColO = 0;                     // O: 128 fp32 columns
 constexpr uint32_t kColS = 128;                   // S: 2 x 64 fp32 columns; P overwrites S
 constexpr uint32_t kTmemCols = 256;
+// the quantised pass (one CTA per SM, all of TMEM): O, two S buffers of
+// 2 kTcTok columns (scores against the heads, then the remainders), Q
+constexpr uint32_t kColQ = kColS + 2 * 2 * kTcTok;  // 384: Q, 64 columns
+constexpr uint32_t kTmemColsQ = 512;
 constexpr float kRefSlack = 8.f;                  // log2 of the largest probability kept
 constexpr int kTcBars = 4 * kTcStages + 7;
 constexpr size_t kTcSmem = 1024 + kTcQBytes + (size_t)kTcStages * kTcStage + kTcBars * 8 + 64;
@@ -305,28 +309,37 @@ static_assert(2 * kTcSmem <= 227 * 1024 && 3 * kTcSmem > 228 * 1024,
               "exactly two CTAs per SM: each allocates half of TMEM");
 }  // namespace
 
-// Pages of step j of a chunk [p_begin, p_end) that exist (bit p: page p of
-// the step has a valid physical page); 0 past the last step.
-__device__ __forceinline__ uint32_t tc_step_mask(const PrefixArgs &a, const int32_t *bt, int p_begin,
-                                                 int p_end, int nsteps, int j) {
-  uint32_t m = 0;
-  if (j < nsteps) {
-    const int p0 = p_begin + j * kTcPages, np = min(kTcPages, p_end - p0);
+// The block-table entries of one step of a chunk [p_begin, p_end), loaded
+// a step ahead of their use so that the loads' latency is not waited for:
+// load(j) issues the loads, mask() (one step later) says which pages of the
+// step exist (bit p: page p has a valid physical page; 0 past the last step).
+struct StepPages {
+  int pb[kTcPages];
+  __device__ __forceinline__ void load(const int32_t *bt, int p_begin, int p_end, int nsteps, int j) {
+    const int p0 = p_begin + j * kTcPages, np = j < nsteps ? min(kTcPages, p_end - p0) : 0;
 #pragma unroll
-    for (int p = 0; p < kTcPages; ++p) {
-      const int pb = p < np ? __ldg(bt + p0 + p) : -1;
-      if (pb >= 0 && pb < a.num_blocks) m |= 1u << p;
-    }
+    for (int p = 0; p < kTcPages; ++p) pb[p] = p < np ? __ldg(bt + p0 + p) : -1;
   }
-  return m;
-}
+  __device__ __forceinline__ uint32_t mask(const PrefixArgs &a) const {
+    uint32_t m = 0;
+#pragma unroll
+    for (int p = 0; p < kTcPages; ++p)
+      if (pb[p] >= 0 && pb[p] < a.num_blocks) m |= 1u << p;
+    return m;
+  }
+};
 
 // The softmax role of the tensor-memory passes (4 warps, one query row per
-// thread): puts its rows of Q into the swizzled Q tile, then per step reads
-// its S row from TMEM, updates the running (max, sum), writes P over S,
+// thread): puts its rows of Q where the QK^T MMAs read them, then per step
+// reads its S row from TMEM, updates the running (max, sum), writes P over S,
 // rescales O in TMEM when the reference max moves, and finally writes the
 // normalised partial (o, lse) of its row.
-template <typename T>
+//  * kSplit = false (16-bit pages): Q into the K-major, 128-byte-swizzled
+//    shared-memory tile qs; S buffers of kTcTok columns.
+//  * kSplit = true (quantised pages, head + remainder operands): Q into TMEM
+//    columns kColQ.. (the MMA's A operand); S buffers of 2 kTcTok columns,
+//    the scores against the heads then against the remainders, summed here.
+template <typename T, bool kSplit = false>
 __device__ __forceinline__ void tc_softmax_role(const PrefixArgs &a, uint8_t *qs, uint32_t tbase,
                                                 uint32_t S_FULL, uint32_t P_FULL, uint32_t O_DONE,
                                                 uint32_t Q_FULL, int warp, int lane, int r0, int rows,
@@ -340,30 +353,54 @@ __device__ __forceinline__ void tc_softmax_role(const PrefixArgs &a, uint8_t *qs
   const int row = r0 + quarter * 32 + lane;  // row of the group: member row / G, head row % G
   const bool live = row < rows;
   const int b = s0 + (live ? row / a.G : 0), jr = live ? row % a.G : 0;
+  constexpr int kSb = kSplit ? 2 * kTcTok : kTcTok;  // TMEM columns of one S buffer
   {
-    // this row of Q into the K-major, 128-byte-swizzled tile the MMA reads
-    const int r = quarter * 32 + lane;
     const uint4 *qv = reinterpret_cast<const uint4 *>(
         static_cast<const T *>(a.q) +
         (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + jr) * D);
+    if constexpr (kSplit) {
+      // this row of Q into its TMEM lane: column c holds channels 2c, 2c + 1
 #pragma unroll
-    for (int c = 0; c < 2 * 8; ++c) {
-      const uint4 v = live ? __ldg(qv + c) : make_uint4(0u, 0u, 0u, 0u);
-      const int half = c >> 3, cc = c & 7;
-      *reinterpret_cast<uint4 *>(qs + half * (kTcQBytes / 2) + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = live ? __ldg(qv + hf * 8 + c) : make_uint4(0u, 0u, 0u, 0u);
+          r[4 * c] = v.x;
+          r[4 * c + 1] = v.y;
+          r[4 * c + 2] = v.z;
+          r[4 * c + 3] = v.w;
+        }
+        tc::st32(tbase + lanes + kColQ + hf * 32, r);
+      }
+      tc::wait_st();
+      tc::fence_before_sync();
+    } else {
+      // this row of Q into the K-major, 128-byte-swizzled tile the MMA reads
+      const int r = quarter * 32 + lane;
+#pragma unroll
+      for (int c = 0; c < 2 * 8; ++c) {
+        const uint4 v = live ? __ldg(qv + c) : make_uint4(0u, 0u, 0u, 0u);
+        const int half = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4 *>(qs + half * (kTcQBytes / 2) + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();  // visible to the tensor core's reads
     }
-    fence_proxy_async_smem();  // visible to the tensor core's reads
     __syncwarp();
     if (lane == 0) mbar_arrive(Q_FULL);
   }
 
   float m_ref = -INFINITY, l = 0.f;
   bool ok = true;
-  uint32_t next_mask = tc_step_mask(a, bt, p_begin, p_end, nsteps, 0);  // loaded one step before use
+  StepPages ahead;
+  ahead.load(bt, p_begin, p_end, nsteps, 0);
+  uint32_t next_mask = ahead.mask(a);  // the mask of step j + 1 during step j
+  ahead.load(bt, p_begin, p_end, nsteps, 1);
   for (int j = 0; j < nsteps; ++j) {
     const int bs = j & 1;
     const uint32_t pm = next_mask;
-    next_mask = tc_step_mask(a, bt, p_begin, p_end, nsteps, j + 1);
+    next_mask = ahead.mask(a);
+    ahead.load(bt, p_begin, p_end, nsteps, j + 2);
     const bool got = mbar_wait_bounded(S_FULL + 8 * bs, (j >> 1) & 1);
     if (!__all_sync(0xffffffffu, got)) {
       ok = false;
@@ -373,13 +410,23 @@ __device__ __forceinline__ void tc_softmax_role(const PrefixArgs &a, uint8_t *qs
     float x[kTcTok];
     {
       uint32_t r0v[32], r1v[32];
-      tc::ld32(tbase + lanes + kColS + bs * kTcTok, r0v);
-      tc::ld32(tbase + lanes + kColS + bs * kTcTok + 32, r1v);
+      tc::ld32(tbase + lanes + kColS + bs * kSb, r0v);
+      tc::ld32(tbase + lanes + kColS + bs * kSb + 32, r1v);
       tc::wait_ld();
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         x[i] = __uint_as_float(r0v[i]);
         x[32 + i] = __uint_as_float(r1v[i]);
+      }
+      if constexpr (kSplit) {
+        tc::ld32(tbase + lanes + kColS + bs * kSb + kTcTok, r0v);
+        tc::ld32(tbase + lanes + kColS + bs * kSb + kTcTok + 32, r1v);
+        tc::wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          x[i] += __uint_as_float(r0v[i]);
+          x[32 + i] += __uint_as_float(r1v[i]);
+        }
       }
     }
     // row maximum of the scaled scores (in log2 units): the scale is folded
@@ -434,8 +481,8 @@ __device__ __forceinline__ void tc_softmax_role(const PrefixArgs &a, uint8_t *qs
     else exps(std::true_type{});
     const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
     l = l * alpha + sum;
-    tc::st32(tbase + lanes + kColS + bs * kTcTok, ph);
-    if constexpr (kBf16) tc::st32(tbase + lanes + kColS + bs * kTcTok + kTcTok / 2, pl);
+    tc::st32(tbase + lanes + kColS + bs * kSb, ph);
+    if constexpr (kBf16) tc::st32(tbase + lanes + kColS + bs * kSb + kTcTok / 2, pl);
     if (j >= 1) {
       // O holds the product of step j-1 once its o_done phase completes
       const bool got2 = mbar_wait_bounded(O_DONE, (j - 1) & 1);
@@ -686,9 +733,12 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
         return mbar_wait_bounded(P_FULL + 8 * (j & 1), (j >> 1) & 1) &&
                mbar_wait_bounded(FULL_V(j % kTcStages), (j / kTcStages) & 1);
       };
+      StepPages ahead;  // the block-table entries of step j, loaded during step j - 1
+      ahead.load(bt, p_begin, p_end, nsteps, 0);
       for (int j = 0; ok && j < nsteps; ++j) {
-        if (j & 1) pv_mask1 = tc_step_mask(a, bt, p_begin, p_end, nsteps, j);
-        else pv_mask0 = tc_step_mask(a, bt, p_begin, p_end, nsteps, j);
+        if (j & 1) pv_mask1 = ahead.mask(a);
+        else pv_mask0 = ahead.mask(a);
+        ahead.load(bt, p_begin, p_end, nsteps, j + 1);
         if (!mbar_wait_bounded(FULL_K(j % kTcStages), (j / kTcStages) & 1)) {
           ok = false;
           break;
@@ -748,19 +798,29 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
 // (bf16 adds the probability remainder times V_hi, as in the 16-bit pass).
 // What is left is about 2^-22 (f16) or 2^-16 (bf16) of each value.
 //
-// Roles (320 threads): those of the 16-bit pass plus four dequantise warps
-// (6-9).  The producer copies a step's codes (2-D TMA boxes, swizzled by the
-// code row size) and scale rows (bulk copies) into a code stage.  The
-// dequantise warps turn them into the four operand tiles -- K hi, K lo, V hi,
-// V lo, each laid out as the TMA lays out a 16-bit page (64-channel halves,
-// 128-byte rows, 128-byte swizzle) -- and hand the code stage back.  The MMA
-// issuer waits for the tiles instead of the copies.  Per stage and per K / V:
-// codes landed (TMA / bulk bytes), codes consumed and tiles written (one
-// arrive per dequantise warp), tiles read (tcgen05.commit).  About 197 KB of
-// shared memory: one CTA per SM.
+// Roles (384 threads): those of the 16-bit pass plus six dequantise warps,
+// three for K (6-8) and three for V (9-11), so that the K and V tiles of a
+// step are made in parallel and each group waits only on its own barriers.
+// The producer copies a step's codes (2-D TMA boxes, swizzled by the code row
+// size) and scale rows (bulk copies) into a code stage.  The dequantise warps
+// turn them into the four operand tiles -- K hi, K lo, V hi, V lo, each laid
+// out as the TMA lays out a 16-bit page (64-channel halves, 128-byte rows,
+// 128-byte swizzle) -- and hand the code stage back.  The MMA issuer waits for
+// the tiles instead of the copies.  Per stage and per K / V: codes landed
+// (TMA / bulk bytes), codes consumed and tiles written (one arrive per
+// dequantise warp of the group), tiles read (tcgen05.commit).  The codes ring
+// is deeper (kTqCodeStages) than the tile ring, so the copies of the next two
+// steps are in flight while a step is dequantised.  About 214 KB of shared
+// memory: one CTA per SM.
 namespace {
-constexpr int kTqWarps = 10;
-constexpr int kTqStage = 8 * kTcHalf;  // K hi, K lo, V hi, V lo: two halves each (64 KB)
+constexpr int kTqWarps = 12;
+constexpr int kTqDqWarps = 3;                // dequantise warps per K / V group
+constexpr int kTqDqThreads = 32 * kTqDqWarps;
+constexpr int kTqCodeStages = 3;             // steps of codes in flight (operand tiles: kTcStages)
+// one tile stage (64 KB): K as two 64-channel halves of 128 rows each (the
+// step's 64 tokens' heads, then their remainders: one N = 128 operand), then
+// V hi (two halves), V lo (two halves)
+constexpr int kTqStage = 8 * kTcHalf;
 constexpr int kTqScalePage = kPage * 4 * 4;  // fp32 scales of one page and head (d = 128)
 
 template <Code8 kFmt>
@@ -769,53 +829,89 @@ struct TqGeo {
   static constexpr int kCodePage = kPage * kRow;
   static constexpr int kCodeStage = 2 * kTcPages * kCodePage;         // K then V codes of a step
   static constexpr int kScaleStage = 2 * kTcPages * kTqScalePage;     // K then V scales
-  static constexpr int kBars = 8 * kTcStages + 7;
-  static constexpr size_t kSmem = 1024 + kTcQBytes +
-                                  (size_t)kTcStages * (kTqStage + kCodeStage + kScaleStage) +
-                                  kBars * 8 + 64;
+  static constexpr int kBars = 4 * kTqCodeStages + 4 * kTcStages + 7;
+  static constexpr size_t kSmem = 1024 + (size_t)kTcStages * kTqStage +
+                                  (size_t)kTqCodeStages * (kCodeStage + kScaleStage) + kBars * 8 + 64;
   static_assert(kSmem <= 227 * 1024, "one CTA per SM");
 };
 
+// Packed pair arithmetic of the operand type (f16x2 / bf16x2), one rounding each.
+template <typename T>
+__device__ __forceinline__ uint32_t x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value)
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  else
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+template <typename T>
+__device__ __forceinline__ uint32_t x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value)
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  else
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 // Dequantise the K (or V) half of one code stage into its hi and lo operand
-// tiles; thread ct of the 128 dequantise threads.  A unit is one 16-byte
-// chunk of one token's codes: 16 channels (8-bit) or 32 (INT4), all in one
-// scale group.
+// tiles; thread ct of the group's kTqDqThreads.  A unit is one 16-byte chunk
+// of one token's codes: 16 channels (8-bit) or 32 (INT4), all in one scale
+// group; several units are in flight per thread.
+//
+// Every code value v is exact in the operand type T.  The fp32 scale is split
+// once per unit into s = s_hi + s_lo + d with s_hi = RN_T(s) and
+// s_lo = RN_T(s - s_hi).  Then, in packed T arithmetic,
+//   hi = RN(v s_hi),  e = v s_hi - hi (one fma: the error of a product of a
+//   code (at most 8 significant bits) and s_hi fits in T, so it is exact),
+//   lo = RN(v s_lo + e),
+// and hi + lo is v s to about 2^-15 relative in bf16.  In f16, s_lo is a
+// subnormal once s < 2^-3 (typical for E4M3 and INT8 scales), and then the
+// error is absolute, at most about |v| 2^-25 per value (1.4e-5 for the largest
+// E4M3 code) -- below the f16 rounding of the probabilities in the PV product
+// (2^-11 relative) that the 16-bit pass already makes.
 template <typename T, Code8 kFmt>
 __device__ __forceinline__ void dequant_half(const uint8_t *codes, const float *scl, uint8_t *hi,
-                                             uint8_t *lo, int ct) {
+                                             uint8_t *lo, int half_stride, int ct) {
   using M = Mma<T>;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr int kRow = TqGeo<kFmt>::kRow;
   constexpr int kPerRow = kRow / 16;        // chunks of a code row
   constexpr int kChan = 128 / kPerRow;      // channels of a chunk
   constexpr int kUnits = kTcPages * kPage * kPerRow;
-#pragma unroll 1
-  for (int u = ct; u < kUnits; u += 128) {
+  // INT4 (at most three 32-code units a thread) unrolls fully; the 8-bit
+  // formats (five or six 16-code units) two at a time, measured faster
+#pragma unroll(kFmt == Code8::INT4 ? 4 : 2)
+  for (int u = ct; u < kUnits; u += kTqDqThreads) {
     const int c = u % kPerRow, t = (u / kPerRow) % kPage, p = u / (kPerRow * kPage);
     const uint4 w = *reinterpret_cast<const uint4 *>(codes + p * kPage * kRow + swz_rows<kRow>(t, c));
     const uint32_t words[4] = {w.x, w.y, w.z, w.w};
     const int ch0 = c * kChan;
     const float sc = scl[(p * kPage + t) * 4 + ch0 / 32];
-    float v[kChan];
+    const uint32_t shi = M::pack(sc, sc);
+    const float shf = M::unpack(shi).x;
+    const uint32_t slo = M::pack(sc - shf, sc - shf);
+    // vp[i]: channels ch0 + 2i, ch0 + 2i + 1 as an f16 pair
+    uint32_t vp[kChan / 2];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       if constexpr (kFmt == Code8::INT4) {
-        uint32_t f[4];  // f[s]: channels 8k + s (low half) and 8k + s + 4 (high half)
+        uint32_t f[4];  // f[q]: channels 8k + q (low half) and 8k + q + 4 (high half)
         int4x8_to_f16x2x4(words[k], f);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 x = __half22float2(*reinterpret_cast<const __half2 *>(&f[q]));
-          v[8 * k + q] = x.x;
-          v[8 * k + q + 4] = x.y;
-        }
+        vp[4 * k] = __byte_perm(f[0], f[1], 0x5410);
+        vp[4 * k + 1] = __byte_perm(f[2], f[3], 0x5410);
+        vp[4 * k + 2] = __byte_perm(f[0], f[1], 0x7632);
+        vp[4 * k + 3] = __byte_perm(f[2], f[3], 0x7632);
       } else {
-        uint32_t lo2, hi2;  // channels (4k, 4k + 1), (4k + 2, 4k + 3)
-        code8x4_to_f16x2x2<kFmt>(words[k], lo2, hi2);
-        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&lo2));
-        const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&hi2));
-        v[4 * k] = a.x;
-        v[4 * k + 1] = a.y;
-        v[4 * k + 2] = b.x;
-        v[4 * k + 3] = b.y;
+        code8x4_to_f16x2x2<kFmt>(words[k], vp[2 * k], vp[2 * k + 1]);
+      }
+    }
+    if constexpr (kBf16) {
+#pragma unroll
+      for (int i = 0; i < kChan / 2; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&vp[i]));
+        vp[i] = M::pack(f.x, f.y);  // exact: every code value fits in bf16
       }
     }
     const int r = p * kPage + t;  // row of the step's 64 tokens
@@ -825,12 +921,12 @@ __device__ __forceinline__ void dequant_half(const uint8_t *codes, const float *
       uint32_t h4[4], l4[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float x0 = v[8 * k + 2 * i] * sc, x1 = v[8 * k + 2 * i + 1] * sc;
-        h4[i] = M::pack(x0, x1);
-        const float2 hv = M::unpack(h4[i]);
-        l4[i] = M::pack(x0 - hv.x, x1 - hv.y);
+        const uint32_t v = vp[4 * k + i];
+        h4[i] = x2_mul<T>(v, shi);
+        const uint32_t e = x2_fma<T>(v, shi, h4[i] ^ 0x80008000u);
+        l4[i] = x2_fma<T>(v, slo, e);
       }
-      const int off = hf * kTcHalf + r * 128 + ((cc ^ (r & 7)) << 4);
+      const int off = hf * half_stride + r * 128 + ((cc ^ (r & 7)) << 4);
       *reinterpret_cast<uint4 *>(hi + off) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
       *reinterpret_cast<uint4 *>(lo + off) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
     }
@@ -846,12 +942,11 @@ __global__ void __launch_bounds__(32 * kTqWarps, 1)
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   using Gq = TqGeo<kFmt>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *qs = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                            ~static_cast<uintptr_t>(1023));
-  uint8_t *tiles = qs + kTcQBytes;
+  uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
   uint8_t *codes = tiles + (size_t)kTcStages * kTqStage;
-  uint8_t *scl = codes + (size_t)kTcStages * Gq::kCodeStage;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(scl + (size_t)kTcStages * Gq::kScaleStage);
+  uint8_t *scl = codes + (size_t)kTqCodeStages * Gq::kCodeStage;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(scl + (size_t)kTqCodeStages * Gq::kScaleStage);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Gq::kBars);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -889,30 +984,34 @@ __global__ void __launch_bounds__(32 * kTqWarps, 1)
   const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
   auto step_pages = [&](int j) { return min(kTcPages, p_end - (p_begin + j * kTcPages)); };
 
-  const uint32_t q0 = smem_u32(qs), tiles0 = smem_u32(tiles), codes0 = smem_u32(codes);
+  const uint32_t tiles0 = smem_u32(tiles), codes0 = smem_u32(codes);
   const uint32_t scl0 = smem_u32(scl), bar0 = smem_u32(bars);
-  // kv = 0: K, 1: V
-  auto CFULL = [&](int kv, int s) { return bar0 + 8 * (kv * kTcStages + s); };
-  auto CFREE = [&](int kv, int s) { return bar0 + 8 * ((2 + kv) * kTcStages + s); };
-  auto TFULL = [&](int kv, int s) { return bar0 + 8 * ((4 + kv) * kTcStages + s); };
-  auto TFREE = [&](int kv, int s) { return bar0 + 8 * ((6 + kv) * kTcStages + s); };
-  const uint32_t S_FULL = bar0 + 8 * (8 * kTcStages);  // + 8 * buffer
+  // kv = 0: K, 1: V; c: code stage (kTqCodeStages), s: tile stage (kTcStages)
+  constexpr int kT0 = 4 * kTqCodeStages;  // first tile barrier
+  auto CFULL = [&](int kv, int c) { return bar0 + 8 * (kv * kTqCodeStages + c); };
+  auto CFREE = [&](int kv, int c) { return bar0 + 8 * ((2 + kv) * kTqCodeStages + c); };
+  auto TFULL = [&](int kv, int s) { return bar0 + 8 * (kT0 + kv * kTcStages + s); };
+  auto TFREE = [&](int kv, int s) { return bar0 + 8 * (kT0 + (2 + kv) * kTcStages + s); };
+  const uint32_t S_FULL = bar0 + 8 * (kT0 + 4 * kTcStages);  // + 8 * buffer
   const uint32_t P_FULL = S_FULL + 16;                 // + 8 * buffer
   const uint32_t O_DONE = S_FULL + 32, Q_FULL = S_FULL + 40, DRAIN = S_FULL + 48;
 
   if (warp == 0) {
     __syncwarp();
-    tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tc::tmem_alloc(smem_u32(tmem_slot), kTmemColsQ);
     tc::tmem_relinquish();
   }
   if (tid == 32) {
-    for (int kv = 0; kv < 2; ++kv)
+    for (int kv = 0; kv < 2; ++kv) {
+      for (int c = 0; c < kTqCodeStages; ++c) {
+        mbar_init(CFULL(kv, c), 1);
+        mbar_init(CFREE(kv, c), kTqDqWarps);
+      }
       for (int s = 0; s < kTcStages; ++s) {
-        mbar_init(CFULL(kv, s), 1);
-        mbar_init(CFREE(kv, s), 4);
-        mbar_init(TFULL(kv, s), 4);
+        mbar_init(TFULL(kv, s), kTqDqWarps);
         mbar_init(TFREE(kv, s), 1);
       }
+    }
     mbar_init(S_FULL, 1);
     mbar_init(S_FULL + 8, 1);
     mbar_init(P_FULL, 4);
@@ -936,8 +1035,8 @@ __global__ void __launch_bounds__(32 * kTqWarps, 1)
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < nsteps && ok; ++j) {
-        const int s = j % kTcStages;
-        const uint32_t rel = ((j / kTcStages) - 1) & 1;  // phase of step j - kTcStages
+        const int c = j % kTqCodeStages;
+        const uint32_t rel = ((j / kTqCodeStages) - 1) & 1;  // phase of step j - kTqCodeStages
         const int p0 = p_begin + j * kTcPages, np = step_pages(j);
         int prow[kTcPages];
         int good = 0;
@@ -956,29 +1055,30 @@ __global__ void __launch_bounds__(32 * kTqWarps, 1)
         }
         const uint32_t bytes = static_cast<uint32_t>(good) * (Gq::kCodePage + kTqScalePage);
         for (int kv = 0; kv < 2; ++kv) {
-          // the codes of step j - kTcStages have been dequantised
-          if (j >= kTcStages && !mbar_wait_bounded(CFREE(kv, s), rel)) {
+          // the codes of step j - kTqCodeStages have been dequantised
+          if (j >= kTqCodeStages && !mbar_wait_bounded(CFREE(kv, c), rel)) {
             flag_error(a.err, kErrTimeout);
             ok = false;
             break;
           }
-          const uint32_t cst = codes0 + s * Gq::kCodeStage + kv * kTcPages * Gq::kCodePage;
-          const uint32_t sst = scl0 + s * Gq::kScaleStage + kv * kTcPages * kTqScalePage;
+          const uint32_t cst = codes0 + c * Gq::kCodeStage + kv * kTcPages * Gq::kCodePage;
+          const uint32_t sst = scl0 + c * Gq::kScaleStage + kv * kTcPages * kTqScalePage;
           const float *gs = kv ? a.v_scale : a.k_scale;
-          mbar_arrive_expect_tx(CFULL(kv, s), bytes);
+          mbar_arrive_expect_tx(CFULL(kv, c), bytes);
 #pragma unroll
           for (int p = 0; p < kTcPages; ++p) {
             if (prow[p] < 0) continue;
-            tma_load_2d(cst + p * Gq::kCodePage, kv ? &tmV : &tmK, 0, prow[p], CFULL(kv, s), policy);
+            tma_load_2d(cst + p * Gq::kCodePage, kv ? &tmV : &tmK, 0, prow[p], CFULL(kv, c), policy);
             bulk_load(sst + p * kTqScalePage, gs + static_cast<size_t>(prow[p]) * 4, kTqScalePage,
-                      CFULL(kv, s));
+                      CFULL(kv, c));
           }
         }
         if (ok) issued = j + 1;
       }
       // the copies of the last stages have landed before the CTA exits
-      for (int j = max(0, issued - kTcStages); j < issued; ++j)
-        for (int kv = 0; kv < 2; ++kv) mbar_wait_bounded(CFULL(kv, j % kTcStages), (j / kTcStages) & 1);
+      for (int j = max(0, issued - kTqCodeStages); j < issued; ++j)
+        for (int kv = 0; kv < 2; ++kv)
+          mbar_wait_bounded(CFULL(kv, j % kTqCodeStages), (j / kTqCodeStages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -987,19 +1087,19 @@ __global__ void __launch_bounds__(32 * kTqWarps, 1)
       bool ok = mbar_wait_bounded(Q_FULL, 0);
       tc::fence_after_sync();
       bool o_started = false;
+      // S[128 x (64 + 64)] = Q . [K_hi; K_lo]^T: A = Q in TMEM, B = the step's
+      // 128 K rows (heads, then remainders) of each 64-channel half; a
+      // partial step's missing rows give columns the softmax masks
       auto issue_qk = [&](int j) {
         const int b = j & 1;
-        const uint32_t idesc = tc::idesc_f16(fmt, static_cast<uint32_t>(step_pages(j) * kPage), false);
+        const uint32_t idesc = tc::idesc_f16(fmt, 2 * kTcTok, false);
         const uint32_t kst = tiles0 + (j % kTcStages) * kTqStage;
 #pragma unroll
-        for (int part = 0; part < 2; ++part)  // K hi, then K lo
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t kaddr = kst + (2 * part + (k >> 2)) * kTcHalf + (k & 3) * 32;
-            const uint32_t qaddr = q0 + (k >> 2) * (kTcQBytes / 2) + (k & 3) * 32;
-            tc::mma_ss(tbase + kColS + b * kTcTok, tc::smem_desc(qaddr, 16, 1024),
-                       tc::smem_desc(kaddr, 16, 1024), idesc, part > 0 || k > 0);
-          }
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t kaddr = kst + (k >> 2) * 2 * kTcHalf + (k & 3) * 32;
+          tc::mma_ts(tbase + kColS + b * 2 * kTcTok, tbase + kColQ + 8 * k,
+                     tc::smem_desc(kaddr, 16, 1024), idesc, k > 0);
+        }
         tc::commit(TFREE(0, j % kTcStages));
         tc::commit(S_FULL + 8 * b);
       };
@@ -1014,7 +1114,7 @@ __global__ void __launch_bounds__(32 * kTqWarps, 1)
           if (!((mask >> kk) & 1u)) continue;  // (its scores are masked; its tiles are stale)
           const uint64_t dh = tc::smem_desc(vhi + kk * kPage * 128, kTcHalf, 1024);
           const uint64_t dl = tc::smem_desc(vlo + kk * kPage * 128, kTcHalf, 1024);
-          const uint32_t pa = tbase + kColS + b * kTcTok + kk * 8;  // P over S; remainder at +32
+          const uint32_t pa = tbase + kColS + b * 2 * kTcTok + kk * 8;  // P over S; remainder at +32
           tc::mma_ts(tbase + kColO, pa, dh, idesc, o_started);
           o_started = true;
           tc::mma_ts(tbase + kColO, pa, dl, idesc, true);
@@ -1027,9 +1127,12 @@ __global__ void __launch_bounds__(32 * kTqWarps, 1)
         return mbar_wait_bounded(P_FULL + 8 * (j & 1), (j >> 1) & 1) &&
                mbar_wait_bounded(TFULL(1, j % kTcStages), (j / kTcStages) & 1);
       };
+      StepPages ahead;  // the block-table entries of step j, loaded during step j - 1
+      ahead.load(bt, p_begin, p_end, nsteps, 0);
       for (int j = 0; ok && j < nsteps; ++j) {
-        if (j & 1) pv_mask1 = tc_step_mask(a, bt, p_begin, p_end, nsteps, j);
-        else pv_mask0 = tc_step_mask(a, bt, p_begin, p_end, nsteps, j);
+        if (j & 1) pv_mask1 = ahead.mask(a);
+        else pv_mask0 = ahead.mask(a);
+        ahead.load(bt, p_begin, p_end, nsteps, j + 1);
         if (!mbar_wait_bounded(TFULL(0, j % kTcStages), (j / kTcStages) & 1)) {
           ok = false;
           break;
@@ -1061,36 +1164,37 @@ __global__ void __launch_bounds__(32 * kTqWarps, 1)
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ softmax
-    tc_softmax_role<T>(a, qs, tbase, S_FULL, P_FULL, O_DONE, Q_FULL, warp, lane, r0, rows, s0, h,
-                       chunk, nsteps, bt, p_begin, p_end);
+    tc_softmax_role<T, true>(a, nullptr, tbase, S_FULL, P_FULL, O_DONE, Q_FULL, warp, lane, r0, rows,
+                             s0, h, chunk, nsteps, bt, p_begin, p_end);
   } else {
     // ------------------------------------------------------------ dequantise
-    const int ct = tid - 6 * 32;
+    const int kv = (warp - 6) / kTqDqWarps;  // 0: K (warps 6-8), 1: V (warps 9-11)
+    const int ct = tid - (6 + kv * kTqDqWarps) * 32;
     bool ok = true;
-    for (int j = 0; ok && j < nsteps; ++j) {
-      const int s = j % kTcStages;
-      const uint32_t ph = (j / kTcStages) & 1, rel = ((j / kTcStages) - 1) & 1;
-      for (int kv = 0; kv < 2; ++kv) {
-        // this step's codes have landed, and the MMAs of step j - kTcStages
-        // have finished reading the tiles they are about to overwrite
-        bool got = mbar_wait_bounded(CFULL(kv, s), ph);
-        if (j >= kTcStages) got = got && mbar_wait_bounded(TFREE(kv, s), rel);
-        if (!__all_sync(0xffffffffu, got)) {
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
-        uint8_t *hi = tiles + (size_t)s * kTqStage + kv * 4 * kTcHalf;
-        dequant_half<T, kFmt>(codes + (size_t)s * Gq::kCodeStage + kv * kTcPages * Gq::kCodePage,
-                              reinterpret_cast<const float *>(scl + (size_t)s * Gq::kScaleStage +
-                                                              kv * kTcPages * kTqScalePage),
-                              hi, hi + 2 * kTcHalf, ct);
-        fence_proxy_async_smem();  // tiles visible to the tensor core; codes read before refill
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(TFULL(kv, s));
-          mbar_arrive(CFREE(kv, s));
-        }
+    for (int j = 0; j < nsteps; ++j) {
+      const int s = j % kTcStages, c = j % kTqCodeStages;
+      const uint32_t rel = ((j / kTcStages) - 1) & 1;
+      // this step's codes have landed, and the MMAs of step j - kTcStages
+      // have finished reading the tiles about to be overwritten
+      bool got = mbar_wait_bounded(CFULL(kv, c), (j / kTqCodeStages) & 1);
+      if (j >= kTcStages) got = got && mbar_wait_bounded(TFREE(kv, s), rel);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      // K: halves 2 kTcHalf apart, remainders kTcHalf after the heads;
+      // V: halves kTcHalf apart, remainders 2 kTcHalf after the heads
+      uint8_t *hi = tiles + (size_t)s * kTqStage + kv * 4 * kTcHalf;
+      dequant_half<T, kFmt>(codes + (size_t)c * Gq::kCodeStage + kv * kTcPages * Gq::kCodePage,
+                            reinterpret_cast<const float *>(scl + (size_t)c * Gq::kScaleStage +
+                                                            kv * kTcPages * kTqScalePage),
+                            hi, hi + (kv ? 2 : 1) * kTcHalf, (kv ? 1 : 2) * kTcHalf, ct);
+      fence_proxy_async_smem();  // tiles visible to the tensor core; codes read before refill
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(TFULL(kv, s));
+        mbar_arrive(CFREE(kv, c));
       }
     }
     if (!ok && lane == 0) flag_error(a.err, kErrTimeout);
@@ -1102,7 +1206,7 @@ __global__ void __launch_bounds__(32 * kTqWarps, 1)
   if (warp == 0) {
     __syncwarp();
     tc::fence_after_sync();
-    tc::tmem_dealloc(tbase, kTmemCols);
+    tc::tmem_dealloc(tbase, kTmemColsQ);
   }
 }
 
