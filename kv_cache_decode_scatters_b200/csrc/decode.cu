@@ -35,7 +35,9 @@
 //    operand of O^T[d x 8] += V^T[d x 16] . P^T[16 x 8] (ldmatrix.trans).
 //    G <= 8 uses one n-tile, G <= 16 two.
 //  * Softmax in base 2: scores are scaled by scale * log2(e) in fp32 and
-//    exponentiated with ex2.approx.  For fp16 the probabilities are rounded
+//    exponentiated with ex2.approx.  The running maximum is a reference that
+//    moves (with a rescale) only when a page's scores pass it by more than
+//    2^8, so most pages skip the cross-lane maximum.  For fp16 the probabilities are rounded
 //    once for the PV product and the running sum uses the same rounded
 //    values; for bf16 (8 significant bits) each probability is carried as a
 //    rounded head plus a rounded remainder in two PV products.

@@ -34,6 +34,55 @@ __device__ __forceinline__ int clamp_len(int n, int cap) { return n < 0 ? 0 : (n
 // row, probabilities to the B operand via movmatrix, O^T += V^T P^T.  kb, vb:
 // shared addresses of the staged K and V pages (d/64 swizzled 2 KB boxes);
 // tokens >= ntok are masked.  The state arrays are the warp's registers.
+// Online softmax with a reference maximum (base 2).  m_run is a reference,
+// not the exact running maximum: it moves -- to the exact maximum so far,
+// with l_run and acc rescaled -- only when a score of this step exceeds it by
+// more than kTileRefSlack; otherwise the step's probabilities are
+// exp2(x - m_run) <= 2^kTileRefSlack, exact enough in f16/bf16 (the rounding
+// is relative) and far from fp32 overflow, and the per-step row maximum (three
+// rounds of shuffles) and rescale are skipped.  x[nt][e]: this lane's scaled
+// scores, row e & 1 of n-tile nt (-inf where masked).  Warp-uniform branch.
+constexpr float kTileRefSlack = 8.f;
+template <int NT, int MT, int NX>
+__device__ __forceinline__ void ref_max_update(const float (&x)[NT][NX], float (&m_run)[NT][2],
+                                               float (&l_run)[NT][2], float (&acc)[NT][MT][4]) {
+  bool up = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < NX; ++e) up |= x[nt][e] > m_run[nt][e & 1] + kTileRefSlack;
+  if (!__any_sync(0xffffffffu, up)) return;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float mx0 = x[nt][0], mx1 = x[nt][1];
+#pragma unroll
+    for (int e = 2; e < NX; ++e) {
+      if (e & 1) mx1 = fmaxf(mx1, x[nt][e]);
+      else mx0 = fmaxf(mx0, x[nt][e]);
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
+    // a row with no finite score yet keeps its (zero) state
+    const float a0 = mn0 == -INFINITY ? 1.f : fast_exp2(m_run[nt][0] - mn0);
+    const float a1 = mn1 == -INFINITY ? 1.f : fast_exp2(m_run[nt][1] - mn1);
+    m_run[nt][0] = mn0;
+    m_run[nt][1] = mn1;
+    l_run[nt][0] *= a0;
+    l_run[nt][1] *= a1;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      acc[nt][mt][0] *= a0;
+      acc[nt][mt][1] *= a1;
+      acc[nt][mt][2] *= a0;
+      acc[nt][mt][3] *= a1;
+    }
+  }
+}
+
 template <int D, int NT, typename T>
 __device__ __forceinline__ void tile_page(uint32_t kb, uint32_t vb, int ntok, float scale_log2,
                                           int lane, const uint32_t (&qf)[NT][D / 16][2],
@@ -71,29 +120,20 @@ __device__ __forceinline__ void tile_page(uint32_t kb, uint32_t vb, int ntok, fl
   // online softmax update (base 2), probabilities rounded to T (bf16:
   // split into a rounded head and a rounded remainder, see kSplitP)
   const bool v0 = g8 < ntok, v1 = g8 + 8 < ntok;
-  uint32_t pb0[NT], pb1[NT], pc0[NT], pc1[NT];
-  float alpha[NT][2];
-  bool rescale = false;
+  float x[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const float x0 = v0 ? (s[nt][0] + s2[nt][0]) * scale_log2 : -INFINITY;
-    const float x1 = v0 ? (s[nt][1] + s2[nt][1]) * scale_log2 : -INFINITY;
-    const float x2 = v1 ? (s[nt][2] + s2[nt][2]) * scale_log2 : -INFINITY;
-    const float x3 = v1 ? (s[nt][3] + s2[nt][3]) * scale_log2 : -INFINITY;
-    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+    x[nt][0] = v0 ? (s[nt][0] + s2[nt][0]) * scale_log2 : -INFINITY;
+    x[nt][1] = v0 ? (s[nt][1] + s2[nt][1]) * scale_log2 : -INFINITY;
+    x[nt][2] = v1 ? (s[nt][2] + s2[nt][2]) * scale_log2 : -INFINITY;
+    x[nt][3] = v1 ? (s[nt][3] + s2[nt][3]) * scale_log2 : -INFINITY;
+  }
+  ref_max_update<NT, kSteps, 4>(x, m_run, l_run, acc);
+  uint32_t pb0[NT], pb1[NT], pc0[NT], pc1[NT];
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-    }
-    const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-    alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
-    alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
-    rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
-    m_run[nt][0] = mn0;
-    m_run[nt][1] = mn1;
-    const float e0 = fast_exp2(x0 - mn0), e1 = fast_exp2(x1 - mn1);
-    const float e2 = fast_exp2(x2 - mn0), e3 = fast_exp2(x3 - mn1);
+  for (int nt = 0; nt < NT; ++nt) {
+    const float e0 = fast_exp2(x[nt][0] - m_run[nt][0]), e1 = fast_exp2(x[nt][1] - m_run[nt][1]);
+    const float e2 = fast_exp2(x[nt][2] - m_run[nt][0]), e3 = fast_exp2(x[nt][3] - m_run[nt][1]);
     const uint32_t lo = M::pack(e0, e1), hi = M::pack(e2, e3);
     const float2 fl = M::unpack(lo), fh = M::unpack(hi);
     if constexpr (kSplitP) {
@@ -101,30 +141,19 @@ __device__ __forceinline__ void tile_page(uint32_t kb, uint32_t vb, int ntok, fl
       // product; the running sum uses the unrounded p to match
       const uint32_t lo2 = M::pack(e0 - fl.x, e1 - fl.y);
       const uint32_t hi2 = M::pack(e2 - fh.x, e3 - fh.y);
-      l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (e0 + e2);
-      l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (e1 + e3);
+      l_run[nt][0] += e0 + e2;
+      l_run[nt][1] += e1 + e3;
       pc0[nt] = movmatrix_trans(lo2);
       pc1[nt] = movmatrix_trans(hi2);
     } else {
       // the running sum uses the same rounded p as the PV product, so
       // the output is an exact weighted mean of V up to fp32 sums
-      l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (fl.x + fh.x);
-      l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (fl.y + fh.y);
+      l_run[nt][0] += fl.x + fh.x;
+      l_run[nt][1] += fl.y + fh.y;
       pc0[nt] = pc1[nt] = 0u;
     }
     pb0[nt] = movmatrix_trans(lo);
     pb1[nt] = movmatrix_trans(hi);
-  }
-  if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int mt = 0; mt < kSteps; ++mt) {
-        acc[nt][mt][0] *= alpha[nt][0];
-        acc[nt][mt][1] *= alpha[nt][1];
-        acc[nt][mt][2] *= alpha[nt][0];
-        acc[nt][mt][3] *= alpha[nt][1];
-      }
   }
 
   // O^T += V^T P^T
@@ -187,33 +216,21 @@ __device__ __forceinline__ void tile_page2(uint32_t kbA, uint32_t vbA, uint32_t 
 
   uint32_t pa0[NT], pa1[NT], pb0[NT], pb1[NT];
   uint32_t ra0[NT], ra1[NT], rb0[NT], rb1[NT];  // bf16 remainders
-  float alpha[NT][2];
-  bool rescale = false;
+  // row r0 = elements 0, 2 (page A), 4, 6 (page B); row r1 = 1, 3, 5, 7
+  float x[NT][8];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    float x[8];
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      x[e] = (sa[nt][e] + sa2[nt][e]) * scale_log2;
-      x[4 + e] = (sb[nt][e] + sb2[nt][e]) * scale_log2;
+      x[nt][e] = (sa[nt][e] + sa2[nt][e]) * scale_log2;
+      x[nt][4 + e] = (sb[nt][e] + sb2[nt][e]) * scale_log2;
     }
-    // row r0 = elements 0, 2 (page A), 4, 6 (page B); row r1 = 1, 3, 5, 7
-    float mx0 = fmaxf(fmaxf(x[0], x[2]), fmaxf(x[4], x[6]));
-    float mx1 = fmaxf(fmaxf(x[1], x[3]), fmaxf(x[5], x[7]));
+  ref_max_update<NT, kSteps, 8>(x, m_run, l_run, acc);
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-    }
-    const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-    alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
-    alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
-    rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
-    m_run[nt][0] = mn0;
-    m_run[nt][1] = mn1;
+  for (int nt = 0; nt < NT; ++nt) {
     float e[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) e[i] = fast_exp2(x[i] - ((i & 1) ? mn1 : mn0));
+    for (int i = 0; i < 8; ++i) e[i] = fast_exp2(x[nt][i] - m_run[nt][i & 1]);
     const uint32_t w0 = M::pack(e[0], e[1]), w1 = M::pack(e[2], e[3]);
     const uint32_t w2 = M::pack(e[4], e[5]), w3 = M::pack(e[6], e[7]);
     const float2 f0 = M::unpack(w0), f1 = M::unpack(w1), f2 = M::unpack(w2), f3 = M::unpack(w3);
@@ -222,28 +239,17 @@ __device__ __forceinline__ void tile_page2(uint32_t kbA, uint32_t vbA, uint32_t 
       ra1[nt] = movmatrix_trans(M::pack(e[2] - f1.x, e[3] - f1.y));
       rb0[nt] = movmatrix_trans(M::pack(e[4] - f2.x, e[5] - f2.y));
       rb1[nt] = movmatrix_trans(M::pack(e[6] - f3.x, e[7] - f3.y));
-      l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + ((e[0] + e[2]) + (e[4] + e[6]));
-      l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + ((e[1] + e[3]) + (e[5] + e[7]));
+      l_run[nt][0] += (e[0] + e[2]) + (e[4] + e[6]);
+      l_run[nt][1] += (e[1] + e[3]) + (e[5] + e[7]);
     } else {
       ra0[nt] = ra1[nt] = rb0[nt] = rb1[nt] = 0u;
-      l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + ((f0.x + f1.x) + (f2.x + f3.x));
-      l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + ((f0.y + f1.y) + (f2.y + f3.y));
+      l_run[nt][0] += (f0.x + f1.x) + (f2.x + f3.x);
+      l_run[nt][1] += (f0.y + f1.y) + (f2.y + f3.y);
     }
     pa0[nt] = movmatrix_trans(w0);
     pa1[nt] = movmatrix_trans(w1);
     pb0[nt] = movmatrix_trans(w2);
     pb1[nt] = movmatrix_trans(w3);
-  }
-  if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int mt = 0; mt < kSteps; ++mt) {
-        acc[nt][mt][0] *= alpha[nt][0];
-        acc[nt][mt][1] *= alpha[nt][1];
-        acc[nt][mt][2] *= alpha[nt][0];
-        acc[nt][mt][3] *= alpha[nt][1];
-      }
   }
 #pragma unroll
   for (int mt = 0; mt < kSteps; ++mt) {
@@ -419,9 +425,7 @@ __device__ __forceinline__ void tile_page_q8(uint32_t kb, uint32_t vb, const flo
   }
 
   const bool v0 = g8 < ntok, v1 = g8 + 8 < ntok;
-  uint32_t pj0[kG][NT], pj1[kG][NT];
-  float alpha[NT][2];
-  bool rescale = false;
+  float x[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     float s4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -432,43 +436,25 @@ __device__ __forceinline__ void tile_page_q8(uint32_t kb, uint32_t vb, const flo
       s4[2] += sg[j][nt][2] * kBs[j];
       s4[3] += sg[j][nt][3] * kBs[j];
     }
-    const float x0 = v0 ? s4[0] * scale_log2 : -INFINITY;
-    const float x1 = v0 ? s4[1] * scale_log2 : -INFINITY;
-    const float x2 = v1 ? s4[2] * scale_log2 : -INFINITY;
-    const float x3 = v1 ? s4[3] * scale_log2 : -INFINITY;
-    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+    x[nt][0] = v0 ? s4[0] * scale_log2 : -INFINITY;
+    x[nt][1] = v0 ? s4[1] * scale_log2 : -INFINITY;
+    x[nt][2] = v1 ? s4[2] * scale_log2 : -INFINITY;
+    x[nt][3] = v1 ? s4[3] * scale_log2 : -INFINITY;
+  }
+  ref_max_update<NT, D / 16, 4>(x, m_run, l_run, acc);
+  uint32_t pj0[kG][NT], pj1[kG][NT];
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-    }
-    const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-    alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
-    alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
-    rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
-    m_run[nt][0] = mn0;
-    m_run[nt][1] = mn1;
-    const float e0 = fast_exp2(x0 - mn0), e1 = fast_exp2(x1 - mn1);
-    const float e2 = fast_exp2(x2 - mn0), e3 = fast_exp2(x3 - mn1);
-    l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (e0 + e2);
-    l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (e1 + e3);
+  for (int nt = 0; nt < NT; ++nt) {
+    const float e0 = fast_exp2(x[nt][0] - m_run[nt][0]), e1 = fast_exp2(x[nt][1] - m_run[nt][1]);
+    const float e2 = fast_exp2(x[nt][2] - m_run[nt][0]), e3 = fast_exp2(x[nt][3] - m_run[nt][1]);
+    l_run[nt][0] += e0 + e2;
+    l_run[nt][1] += e1 + e3;
 #pragma unroll
     for (int j = 0; j < kG; ++j) {
       // masked tokens have e = 0 and a V scale of 0 (cleared by the caller)
       pj0[j][nt] = movmatrix_trans(f16pack(e0 * vAs[j], e1 * vAs[j]));
       pj1[j][nt] = movmatrix_trans(f16pack(e2 * vBs[j], e3 * vBs[j]));
     }
-  }
-  if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int mt = 0; mt < D / 16; ++mt) {
-        acc[nt][mt][0] *= alpha[nt][0];
-        acc[nt][mt][1] *= alpha[nt][1];
-        acc[nt][mt][2] *= alpha[nt][0];
-        acc[nt][mt][3] *= alpha[nt][1];
-      }
   }
 #pragma unroll
   for (int j = 0; j < kG; ++j) {
@@ -567,9 +553,7 @@ __device__ __forceinline__ void tile_page_q4(uint32_t kb, uint32_t vb, const flo
   }
 
   const bool v0 = g8 < ntok, v1 = g8 + 8 < ntok;
-  uint32_t pj0[kG][NT], pj1[kG][NT];
-  float alpha[NT][2];
-  bool rescale = false;
+  float x[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     float s4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -580,43 +564,25 @@ __device__ __forceinline__ void tile_page_q4(uint32_t kb, uint32_t vb, const flo
       s4[2] += sg[j][nt][2] * kBs[j];
       s4[3] += sg[j][nt][3] * kBs[j];
     }
-    const float x0 = v0 ? s4[0] * scale_log2 : -INFINITY;
-    const float x1 = v0 ? s4[1] * scale_log2 : -INFINITY;
-    const float x2 = v1 ? s4[2] * scale_log2 : -INFINITY;
-    const float x3 = v1 ? s4[3] * scale_log2 : -INFINITY;
-    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+    x[nt][0] = v0 ? s4[0] * scale_log2 : -INFINITY;
+    x[nt][1] = v0 ? s4[1] * scale_log2 : -INFINITY;
+    x[nt][2] = v1 ? s4[2] * scale_log2 : -INFINITY;
+    x[nt][3] = v1 ? s4[3] * scale_log2 : -INFINITY;
+  }
+  ref_max_update<NT, D / 16, 4>(x, m_run, l_run, acc);
+  uint32_t pj0[kG][NT], pj1[kG][NT];
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-    }
-    const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-    alpha[nt][0] = fast_exp2(m_run[nt][0] - mn0);
-    alpha[nt][1] = fast_exp2(m_run[nt][1] - mn1);
-    rescale |= (alpha[nt][0] != 1.f) | (alpha[nt][1] != 1.f);
-    m_run[nt][0] = mn0;
-    m_run[nt][1] = mn1;
-    const float e0 = fast_exp2(x0 - mn0), e1 = fast_exp2(x1 - mn1);
-    const float e2 = fast_exp2(x2 - mn0), e3 = fast_exp2(x3 - mn1);
-    l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (e0 + e2);
-    l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (e1 + e3);
+  for (int nt = 0; nt < NT; ++nt) {
+    const float e0 = fast_exp2(x[nt][0] - m_run[nt][0]), e1 = fast_exp2(x[nt][1] - m_run[nt][1]);
+    const float e2 = fast_exp2(x[nt][2] - m_run[nt][0]), e3 = fast_exp2(x[nt][3] - m_run[nt][1]);
+    l_run[nt][0] += e0 + e2;
+    l_run[nt][1] += e1 + e3;
 #pragma unroll
     for (int j = 0; j < kG; ++j) {
       // masked tokens have e = 0 and a V scale of 0 (cleared by the caller)
       pj0[j][nt] = movmatrix_trans(f16pack(e0 * vAs[j], e1 * vAs[j]));
       pj1[j][nt] = movmatrix_trans(f16pack(e2 * vBs[j], e3 * vBs[j]));
     }
-  }
-  if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int mt = 0; mt < D / 16; ++mt) {
-        acc[nt][mt][0] *= alpha[nt][0];
-        acc[nt][mt][1] *= alpha[nt][1];
-        acc[nt][mt][2] *= alpha[nt][0];
-        acc[nt][mt][3] *= alpha[nt][1];
-      }
   }
 #pragma unroll
   for (int jj = 0; jj < kG / 2; ++jj) {
