@@ -300,6 +300,23 @@ __device__ __forceinline__ void code8x4_to_f16x2x2(uint32_t four, uint32_t &lo, 
   }
 }
 
+// The same for the byte pairs (0, 2) and (1, 3) -- the two channels of a
+// channel pair across two tokens after ldmatrix.trans on code bytes.  INT8
+// picks those bytes in its own byte permutes; E4M3 regroups them first.
+template <Code8 kFmt>
+__device__ __forceinline__ void code8x4_to_f16x2x2_0213(uint32_t four, uint32_t &lo, uint32_t &hi) {
+  if constexpr (kFmt == Code8::E4M3) {
+    code8x4_to_f16x2x2<kFmt>(__byte_perm(four, 0, 0x3120), lo, hi);
+  } else {
+    const uint32_t u = four ^ 0x80808080u;  // b + 128, unsigned
+    const uint32_t l = __byte_perm(u, 0x64646464u, 0x4240);
+    const uint32_t h = __byte_perm(u, 0x64646464u, 0x4341);
+    const uint32_t bias = 0x64806480u;      // f16x2 (1152, 1152)
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(l), "r"(bias));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(h), "r"(bias));
+  }
+}
+
 __device__ __forceinline__ uint32_t f16pack(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
@@ -465,8 +482,8 @@ __device__ __forceinline__ void tile_page_q8(uint32_t kb, uint32_t vb, const flo
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       // bytes (0, 2) and (1, 3) of each word: the two channels of a pair
-      code8x4_to_f16x2x2<kFmt>(__byte_perm(R[2 * h], 0, 0x3120), A[h][0], A[h][1]);
-      code8x4_to_f16x2x2<kFmt>(__byte_perm(R[2 * h + 1], 0, 0x3120), A[h][2], A[h][3]);
+      code8x4_to_f16x2x2_0213<kFmt>(R[2 * h], A[h][0], A[h][1]);
+      code8x4_to_f16x2x2_0213<kFmt>(R[2 * h + 1], A[h][2], A[h][3]);
     }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
