@@ -884,7 +884,25 @@ __device__ __forceinline__ void dequant_half(const uint8_t *codes, const float *
   // formats (five or six 16-code units) two at a time, measured faster
 #pragma unroll(kFmt == Code8::INT4 ? 4 : 2)
   for (int u = ct; u < kUnits; u += kTqDqThreads) {
-    const int c = u % kPerRow, t = (u / kPerRow) % kPage, p = u / (kPerRow * kPage);
+    // unit u -> (row tr of the step's 64 tokens, chunk c).  Each 8-lane phase
+    // of a 16-byte access takes rows whose swizzles put its code reads and
+    // its tile stores on 8 distinct 16-byte bank slots (8-bit: rows r and
+    // r ^ 5, 4 chunks each; INT4: rows {0, 1, 6, 7} or {2, 3, 4, 5} of an
+    // 8-row block, 2 chunks each) -- one row's 8 chunks would store into the
+    // same slots from both 64-channel halves.
+    int tr, c;
+    {
+      const int i = u & 7, q = u >> 3, hf = q & 1, rg = q >> 1;
+      if constexpr (kFmt == Code8::INT4) {
+        constexpr uint32_t kRows = 0x54327610u;  // nibble j: row of lane pair j, two blocks
+        tr = 8 * (rg >> 1) + static_cast<int>((kRows >> (4 * (((rg & 1) << 2) | (i >> 1)))) & 7u);
+        c = hf * 2 + (i & 1);
+      } else {
+        tr = 8 * (rg >> 2) + ((rg & 3) ^ ((i >> 2) ? 5 : 0));
+        c = hf * 4 + (i & 3);
+      }
+    }
+    const int t = tr % kPage, p = tr / kPage;
     const uint4 w = *reinterpret_cast<const uint4 *>(codes + p * kPage * kRow + swz_rows<kRow>(t, c));
     const uint32_t words[4] = {w.x, w.y, w.z, w.w};
     const int ch0 = c * kChan;
@@ -914,7 +932,7 @@ __device__ __forceinline__ void dequant_half(const uint8_t *codes, const float *
         vp[i] = M::pack(f.x, f.y);  // exact: every code value fits in bf16
       }
     }
-    const int r = p * kPage + t;  // row of the step's 64 tokens
+    const int r = tr;  // row of the step's 64 tokens
 #pragma unroll
     for (int k = 0; k < kChan / 8; ++k) {
       const int ch = ch0 + 8 * k, hf = ch / 64, cc = (ch % 64) / 8;
