@@ -81,6 +81,7 @@ struct Geo {
 template <int D, int NT, typename T>
 struct Page16 {
   using Out = T;
+  static constexpr bool kPackG1 = false;  // one query row with groups in N (PackedG1)
   static constexpr int kPageBytes = kPage * D * 2;
   static constexpr int kCopyBytes = 2 * kPageBytes;
   static constexpr int kStride = kCopyBytes;
@@ -140,6 +141,7 @@ struct Page16 {
 template <int D, int NT, typename T, Code8 kFmt>
 struct Page8 {
   using Out = T;
+  static constexpr bool kPackG1 = false;  // one query row with groups in N (PackedG1)
   static constexpr int kG = D / 32;                          // scale groups of a token
   static constexpr int kPageBytes = kPage * D;               // codes of K (or V)
   static constexpr int kScaleBytes = kPage * kG * 4;         // scales of K (or V)
@@ -225,6 +227,7 @@ struct Page8 {
 template <int D, int NT, typename T>
 struct Page4 {
   using Out = T;
+  static constexpr bool kPackG1 = false;  // one query row with groups in N (PackedG1)
   static constexpr int kG = D / 32;                          // scale groups of a token
   static constexpr int kRow = D / 2;                         // code bytes of a token
   static constexpr int kPageBytes = kPage * kRow;            // codes of K (or V)
@@ -305,6 +308,24 @@ struct Page4 {
   }
   static __device__ __forceinline__ int dim(int mt, int e, int g8) {
     return (mt >> 1) * 32 + 4 * g8 + 2 * (mt & 1) + (e >> 1);
+  }
+};
+
+// A quantised page policy for KV heads with a single query row (G = 1): the
+// tile's N columns carry the 32-channel scale groups instead of idle query
+// rows (tile_page_g1).  q's fragment of k-step ks is loaded into column ks / 2
+// only, and a finished pair's state is moved back to the general layout
+// (g1_to_rows) before it is written or parked.
+template <class Base, int D, bool kInt4, Code8 kFmt>
+struct PackedG1 : Base {
+  static constexpr bool kPackG1 = true;
+  static __device__ __forceinline__ void tile(uint8_t *st, uint8_t *aux, int ntok, float sl2, int lane,
+                                              const uint32_t (&qf)[1][D / 16][2],
+                                              float (&acc)[1][D / 16][4], float (&m)[1][2],
+                                              float (&l)[1][2]) {
+    const float *ks = reinterpret_cast<const float *>(aux);
+    tile_page_g1<D, kInt4, kFmt>(smem_u32(st), smem_u32(st + Base::kPageBytes), ks,
+                                 ks + kPage * (D / 32), ntok, sl2, lane, qf, acc, m, l);
   }
 };
 
@@ -517,6 +538,7 @@ __global__ void __launch_bounds__(32 * W, 1)
   };
 
   auto finish_pair = [&](int seg, bool last) {
+    if constexpr (Pol::kPackG1) g1_to_rows(acc, lane);
     sum_l();
     long long s0, s1;
     pair_range(seg, s0, s1);
@@ -640,8 +662,11 @@ __global__ void __launch_bounds__(32 * W, 1)
         const int r = nt * 8 + g8;
 #pragma unroll
         for (int ks = 0; ks < Gm::kSteps; ++ks) {
-          if (r < a.G) {
-            Pol::q_words(qw + r * (D / 2), ks, tig, qf[nt][ks][0], qf[nt][ks][1]);
+          // one query row with the scale groups in N: k-step ks of row 0 in
+          // column (group) ks / 2
+          const bool mine = Pol::kPackG1 ? g8 == (ks >> 1) : r < a.G;
+          if (mine) {
+            Pol::q_words(qw + (Pol::kPackG1 ? 0 : r) * (D / 2), ks, tig, qf[nt][ks][0], qf[nt][ks][1]);
           } else {
             qf[nt][ks][0] = 0u;
             qf[nt][ks][1] = 0u;
@@ -1222,10 +1247,15 @@ struct Tune8<64, 2> {
   static constexpr int W = KVD_TUNE_W8_64_2, S = KVD_TUNE_S8_64_2;
 };
 
-template <int D, int NT, typename T, Code8 kFmt, int W, int S>
+// Page policy of an 8-bit launch: one query row per KV head (kG1) packs the
+// scale groups into the tile's N columns.
+template <int D, int NT, typename T, Code8 kFmt, bool kG1>
+using Pol8 = std::conditional_t<kG1, PackedG1<Page8<D, 1, T, kFmt>, D, false, kFmt>, Page8<D, NT, T, kFmt>>;
+
+template <int D, int NT, typename T, Code8 kFmt, int W, int S, bool kG1>
 cudaError_t launch_decode8_ws(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                               cudaStream_t st, int grid) {
-  using Pol = Page8<D, NT, T, kFmt>;
+  using Pol = Pol8<D, NT, T, kFmt, kG1>;
   auto kern = decode_kernel<D, NT, Pol, W, S>;
   const size_t smem = Geo<D, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1236,18 +1266,27 @@ cudaError_t launch_decode8_ws(const DecodeArgs &a, const CUtensorMap &tmK, const
 
 // The tuned ring depth, or one stage per warp when the batch's prefix sums
 // (4 bytes per sequence) would push the tuned layout past the CTA limit.
-template <int D, int NT, typename T, Code8 kFmt>
-cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
-                             cudaStream_t st, int grid) {
+template <int D, int NT, typename T, Code8 kFmt, bool kG1>
+cudaError_t launch_decode8_tg(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                              cudaStream_t st, int grid) {
   constexpr int W = Tune8<D, NT>::W, S = Tune8<D, NT>::S;
-  using Pol = Page8<D, NT, T, kFmt>;
+  using Pol = Pol8<D, NT, T, kFmt, kG1>;
   // one stage must still hold a parked accumulator tile
   constexpr bool kCanShrink = S > 1 && 8 * NT * D * 4 <= Pol::kStride;
   if constexpr (kCanShrink) {
     if (Geo<D, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B) + 1024 > kMaxCtaSmem)
-      return launch_decode8_ws<D, NT, T, kFmt, W, 1>(a, tmK, tmV, st, grid);
+      return launch_decode8_ws<D, NT, T, kFmt, W, 1, kG1>(a, tmK, tmV, st, grid);
   }
-  return launch_decode8_ws<D, NT, T, kFmt, W, S>(a, tmK, tmV, st, grid);
+  return launch_decode8_ws<D, NT, T, kFmt, W, S, kG1>(a, tmK, tmV, st, grid);
+}
+
+template <int D, int NT, typename T, Code8 kFmt>
+cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                             cudaStream_t st, int grid) {
+  if constexpr (NT == 1) {
+    if (a.G == 1) return launch_decode8_tg<D, 1, T, kFmt, true>(a, tmK, tmV, st, grid);
+  }
+  return launch_decode8_tg<D, NT, T, kFmt, false>(a, tmK, tmV, st, grid);
 }
 
 // 4-bit cache: d = 128 has 2 KB code stages, d = 64 1 KB; a parked
@@ -1296,17 +1335,26 @@ struct Tune4<64, 2> {
   static constexpr int W = KVD_TUNE_W4_64_2, S = KVD_TUNE_S4_64_2;
 };
 
-template <int D, int NT, typename T>
-cudaError_t launch_decode4_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
-                             cudaStream_t st, int grid) {
+template <int D, int NT, typename T, bool kG1>
+cudaError_t launch_decode4_tg(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                              cudaStream_t st, int grid) {
   constexpr int W = Tune4<D, NT>::W, S = Tune4<D, NT>::S;
-  using Pol = Page4<D, NT, T>;
+  using Pol = std::conditional_t<kG1, PackedG1<Page4<D, 1, T>, D, true, Code8::INT4>, Page4<D, NT, T>>;
   auto kern = decode_kernel<D, NT, Pol, W, S>;
   const size_t smem = Geo<D, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(32 * W), smem, st, a, tmK, tmV);
+}
+
+template <int D, int NT, typename T>
+cudaError_t launch_decode4_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                             cudaStream_t st, int grid) {
+  if constexpr (NT == 1) {
+    if (a.G == 1) return launch_decode4_tg<D, 1, T, true>(a, tmK, tmV, st, grid);
+  }
+  return launch_decode4_tg<D, NT, T, false>(a, tmK, tmV, st, grid);
 }
 
 template <int D>

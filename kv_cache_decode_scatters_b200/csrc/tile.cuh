@@ -622,4 +622,161 @@ __device__ __forceinline__ void tile_page_q4(uint32_t kb, uint32_t vb, const flo
   }
 }
 
+// ------------------------------------------------------------ one query row
+//
+// A quantised page for a KV head with a single query row (G = 1), on the
+// tensor-core tile whose N dimension would otherwise hold 7 idle rows.  The
+// N columns carry the 32-channel scale groups instead:
+//  * K: q's fragment of k-step ks is placed in column ks / 2 only (the
+//    caller loads it so), so S^T[token][group] -- each group's partial score
+//    -- builds up in ONE accumulator; lanes with columns 2 tig, 2 tig + 1
+//    weigh them by the token's K scales and a shuffle with the neighbour
+//    lane completes the score.
+//  * V: the B operand is X[token][group] = p_token * v_scale[token][group],
+//    one operand for all groups; O^T[channel][group] accumulates, and each
+//    channel's value is the entry of its own group's column.
+// `g1_to_rows` moves those entries to the layout of the general tile (row 0
+// in lanes tig == 0) when a pair is finished.  m_run / l_run use row 0; the
+// running sum counts each token once (lanes tig == 0).  The code layouts and
+// conversions are those of tile_page_q8 (8-bit) and tile_page_q4 (INT4).
+template <int D, bool kInt4, Code8 kFmt>
+__device__ __forceinline__ void tile_page_g1(uint32_t kb, uint32_t vb, const float *ks,
+                                             const float *vs, int ntok, float scale_log2, int lane,
+                                             const uint32_t (&qf)[1][D / 16][2],
+                                             float (&acc)[1][D / 16][4], float (&m_run)[1][2],
+                                             float (&l_run)[1][2]) {
+  using M = Mma<__half>;
+  constexpr int kG = D / 32;
+  const int g8 = lane >> 2, tig = lane & 3;
+  const int mi = lane >> 3, r8 = lane & 7;
+  const int tok = r8 + ((mi & 1) << 3);
+  const int hi = mi >> 1;
+
+  // S^T[token][group], two independent chains (even / odd groups)
+  float s[2][4];
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[c][e] = 0.f;
+  if constexpr (kInt4) {
+#pragma unroll
+    for (int jj = 0; jj < kG / 2; ++jj) {
+      uint32_t R[4];
+      ldmatrix_x4(R, kb + swz_rows<D / 2>(tok, 2 * jj + hi));
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = 2 * jj + h;
+        uint32_t p[4], q[4];
+        int4x8_to_f16x2x4(R[2 * h], p);
+        int4x8_to_f16x2x4(R[2 * h + 1], q);
+        const uint32_t A0[4] = {p[0], q[0], p[1], q[1]};
+        const uint32_t A1[4] = {p[2], q[2], p[3], q[3]};
+        M::run(s[h], A0, qf[0][2 * j][0], qf[0][2 * j][1]);
+        M::run(s[h], A1, qf[0][2 * j + 1][0], qf[0][2 * j + 1][1]);
+      }
+    }
+  } else {
+    const int hi16 = hi;
+#pragma unroll
+    for (int j = 0; j < kG; ++j) {
+      uint32_t R[4];
+      ldmatrix_x4(R, kb + swz_rows<D>(tok, 2 * j + hi16));
+      uint32_t A0[4], A1[4];
+      code8x4_to_f16x2x2<kFmt>(R[0], A0[0], A0[2]);
+      code8x4_to_f16x2x2<kFmt>(R[1], A0[1], A0[3]);
+      code8x4_to_f16x2x2<kFmt>(R[2], A1[0], A1[2]);
+      code8x4_to_f16x2x2<kFmt>(R[3], A1[1], A1[3]);
+      M::run(s[j & 1], A0, qf[0][2 * j][0], qf[0][2 * j][1]);
+      M::run(s[j & 1], A1, qf[0][2 * j + 1][0], qf[0][2 * j + 1][1]);
+    }
+  }
+  // this lane's columns 2 tig, 2 tig + 1 are groups when 2 tig < kG
+  const bool cols = 2 * tig < kG;
+  const int cg = cols ? 2 * tig : 0;
+  const float2 kA = *reinterpret_cast<const float2 *>(ks + g8 * kG + cg);
+  const float2 kB = *reinterpret_cast<const float2 *>(ks + (g8 + 8) * kG + cg);
+  const float2 vA = *reinterpret_cast<const float2 *>(vs + g8 * kG + cg);
+  const float2 vB = *reinterpret_cast<const float2 *>(vs + (g8 + 8) * kG + cg);
+  float p0 = (s[0][0] + s[1][0]) * kA.x + (s[0][1] + s[1][1]) * kA.y;  // token g8
+  float p8 = (s[0][2] + s[1][2]) * kB.x + (s[0][3] + s[1][3]) * kB.y;  // token g8 + 8
+  p0 = cols ? p0 : 0.f;
+  p8 = cols ? p8 : 0.f;
+  p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
+  p8 += __shfl_xor_sync(0xffffffffu, p8, 1);
+  const float x0 = (cols && g8 < ntok) ? p0 * scale_log2 : -INFINITY;
+  const float x8 = (cols && g8 + 8 < ntok) ? p8 * scale_log2 : -INFINITY;
+
+  // reference maximum of the single row (see ref_max_update)
+  float &m = m_run[0][0];
+  const bool up = (x0 > m + kTileRefSlack) | (x8 > m + kTileRefSlack);
+  if (__any_sync(0xffffffffu, up)) {
+    float mx = fmaxf(x0, x8);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float mn = fmaxf(m, mx);
+    const float al = mn == -INFINITY ? 1.f : fast_exp2(m - mn);
+    m = mn;
+    l_run[0][0] *= al;
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[0][mt][e] *= al;
+  }
+  const float e0 = fast_exp2(x0 - m), e8 = fast_exp2(x8 - m);
+  if (tig == 0) l_run[0][0] += e0 + e8;
+  // X[token][group]: masked tokens have e = 0 and V scales of 0 (cleared by
+  // the caller); non-group columns have scales read as 0 products of e = 0
+  const uint32_t pj0 = movmatrix_trans(f16pack(e0 * vA.x, e0 * vA.y));
+  const uint32_t pj1 = movmatrix_trans(f16pack(e8 * vB.x, e8 * vB.y));
+
+  if constexpr (kInt4) {
+#pragma unroll
+    for (int jj = 0; jj < kG / 2; ++jj) {
+      uint32_t R[4];
+      ldmatrix_x4_trans(R, vb + swz_rows<D / 2>(tok, 2 * jj + hi));
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = 2 * jj + h;
+        uint32_t u[4], w[4];
+        int4x8_to_f16x2x4(R[2 * h], u);
+        int4x8_to_f16x2x4(R[2 * h + 1], w);
+        const uint32_t A0[4] = {u[0], u[1], w[0], w[1]};
+        const uint32_t A1[4] = {u[2], u[3], w[2], w[3]};
+        M::run(acc[0][2 * j], A0, pj0, pj1);
+        M::run(acc[0][2 * j + 1], A1, pj0, pj1);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kG; ++j) {
+      uint32_t R[4];
+      ldmatrix_x4_trans(R, vb + swz_rows<D>(tok, 2 * j + hi));
+      uint32_t A[2][4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        code8x4_to_f16x2x2_0213<kFmt>(R[2 * h], A[h][0], A[h][1]);
+        code8x4_to_f16x2x2_0213<kFmt>(R[2 * h + 1], A[h][2], A[h][3]);
+      }
+      M::run(acc[0][2 * j], A[0], pj0, pj1);
+      M::run(acc[0][2 * j + 1], A[1], pj0, pj1);
+    }
+  }
+}
+
+// The state of tile_page_g1 in the layout of the general tile: the value of
+// m-tile mt (group mt / 2) moves from column mt / 2 -- lane tig = mt / 4,
+// element (mt / 2) & 1 (+ 2 for the second channel row) -- to column 0.
+template <int MT>
+__device__ __forceinline__ void g1_to_rows(float (&acc)[1][MT][4], int lane) {
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const int j = mt >> 1;
+    const int src = (lane & ~3) | (j >> 1);
+    const float v0 = __shfl_sync(0xffffffffu, acc[0][mt][j & 1], src);
+    const float v2 = __shfl_sync(0xffffffffu, acc[0][mt][2 + (j & 1)], src);
+    acc[0][mt][0] = v0;
+    acc[0][mt][2] = v2;
+  }
+}
+
 }  // namespace kvd
