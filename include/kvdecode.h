@@ -299,13 +299,15 @@ kvd_status kvd_decode_step_int4(const void *q, const void *k_new, const void *v_
  *                 the quantised pools of kvd_decode_step_{fp8,int8,int4}
  *                 (written only when k_new / v_new are given: the fused
  *                 quantising append)
- *   d             128 only (KVD_ERR_UNSUPPORTED otherwise)
+ *   d             64 or 128 (KVD_ERR_UNSUPPORTED otherwise)
  *   other arguments as kvd_decode_attention_shared_prefix; the workspace is
  *   kvd_shared_prefix_workspace_size(...) bytes, as there.
- * Each shared page is dequantised once per (group, KV head) into f16/bf16
- * tensor-core tiles, every value as a rounded head plus a rounded remainder
- * (about 2^-22 of the value in f16, 2^-16 in bf16, is lost), so the result is
- * that of kvd_decode_attention_{fp8,int8,int4} up to fp32 rounding order.
+ * At d = 128 each shared page is dequantised once per (group, KV head) into
+ * f16/bf16 tensor-core tiles, every value as a rounded head plus a rounded
+ * remainder (in f16 with an error of at most about |code| 2^-25 per value; in
+ * bf16 about 2^-15 of it); at d = 64 every warp runs the decode kernel's
+ * quantised tile on the staged page.  The result is that of
+ * kvd_decode_attention_{fp8,int8,int4} up to that and fp32 rounding order.
  */
 kvd_status kvd_decode_attention_shared_prefix_fp8(
     const void *q, const void *k_new, const void *v_new, uint8_t *k_codes, uint8_t *v_codes,

@@ -395,7 +395,7 @@ def kvd_decode_attention_shared_prefix_fp8(q, k_codes, v_codes, k_scale, v_scale
                                            group_start, group_pages, max_group_size, scale=None,
                                            out=None, k_new=None, v_new=None, num_partitions=0,
                                            workspace=None, lse_out=None, stream=None):
-    """kvd_decode_attention_shared_prefix over the E4M3 cache (d = 128); with
+    """kvd_decode_attention_shared_prefix over the E4M3 cache (d = 64 or 128); with
     k_new/v_new the step's token is quantised and appended as in
     kvd_decode_step_fp8.  Returns out."""
     return _shared_prefix8("fp8", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
@@ -407,7 +407,7 @@ def kvd_decode_attention_shared_prefix_int8(q, k_codes, v_codes, k_scale, v_scal
                                             group_start, group_pages, max_group_size, scale=None,
                                             out=None, k_new=None, v_new=None, num_partitions=0,
                                             workspace=None, lse_out=None, stream=None):
-    """kvd_decode_attention_shared_prefix over the INT8 cache (d = 128).  Returns out."""
+    """kvd_decode_attention_shared_prefix over the INT8 cache (d = 64 or 128).  Returns out."""
     return _shared_prefix8("int8", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
                            group_start, group_pages, max_group_size, scale, out, k_new, v_new,
                            num_partitions, workspace, lse_out, stream)
@@ -417,7 +417,7 @@ def kvd_decode_attention_shared_prefix_int4(q, k_codes, v_codes, k_scale, v_scal
                                             group_start, group_pages, max_group_size, scale=None,
                                             out=None, k_new=None, v_new=None, num_partitions=0,
                                             workspace=None, lse_out=None, stream=None):
-    """kvd_decode_attention_shared_prefix over the INT4 cache (d = 128).  Returns out."""
+    """kvd_decode_attention_shared_prefix over the INT4 cache (d = 64 or 128).  Returns out."""
     return _shared_prefix8("int4", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens,
                            group_start, group_pages, max_group_size, scale, out, k_new, v_new,
                            num_partitions, workspace, lse_out, stream)

@@ -294,8 +294,6 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   if (num_partitions < 0) return fail(KVD_ERR_INVALID, "num_partitions < 0");
   if (q8) {
     if (!v_scale) return fail(KVD_ERR_INVALID, "v_scale is NULL");
-    if (n_groups > 0 && d != 128)
-      return fail(KVD_ERR_UNSUPPORTED, "the shared-prefix pass over a quantised cache needs d = 128");
     if (!aligned(k_scale, 16) || !aligned(v_scale, 16))
       return fail(KVD_ERR_INVALID, "scale pools must be 16-byte aligned");
   }
@@ -441,7 +439,7 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
     pa.maxg = max_group_size;
     pa.k_scale = k_scale;
     pa.v_scale = v_scale;
-    e = q8 ? kvd::launch_prefix_q(pa, fmt, dt, tm[0], tm[1], PL.row_blocks, s)
+    e = q8 ? kvd::launch_prefix_q(pa, d, fmt, dt, tm[0], tm[1], PL.row_blocks, s)
            : kvd::launch_prefix(pa, d, dt, tm[0], tm[1], PL.row_blocks, s);
     if (e != cudaSuccess) return cuda_fail(e, "prefix launch");
     a.skip = pa.skip;

@@ -202,22 +202,11 @@ struct Page8 {
   }
   // q in f16, channel order of the 8-bit tile: k-slots 2t, 2t+1 <- channels
   // 4t, 4t+1 and k-slots 2t+8, 2t+9 <- channels 4t+2, 4t+3 of each 16
-  static __device__ __forceinline__ uint32_t to_f16x2(uint32_t w) {
-    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w));
-      return f16pack(f.x, f.y);
-    } else {
-      return w;
-    }
-  }
   static __device__ __forceinline__ void q_words(const uint32_t *qrow, int ks, int tig,
                                                  uint32_t &w0, uint32_t &w1) {
-    w0 = to_f16x2(__ldg(qrow + ks * 8 + 2 * tig));
-    w1 = to_f16x2(__ldg(qrow + ks * 8 + 2 * tig + 1));
+    q_words_q8<T>(qrow, ks, tig, w0, w1);
   }
-  static __device__ __forceinline__ int dim(int mt, int e, int g8) {
-    return mt * 16 + 2 * g8 + (e >> 1);
-  }
+  static __device__ __forceinline__ int dim(int mt, int e, int g8) { return dim_q8(mt, e, g8); }
 };
 
 // 4-bit pages (d = D = 64 or 128; INT4 codes, two per byte): codes
@@ -288,27 +277,14 @@ struct Page4 {
     tile_page_q4<D, NT>(smem_u32(st), smem_u32(st + kPageBytes), ks, ks + kPage * kG, ntok, sl2, lane,
                         qf, acc, m, l);
   }
-  static __device__ __forceinline__ uint32_t to_f16x2(uint32_t w) {
-    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w));
-      return f16pack(f.x, f.y);
-    } else {
-      return w;
-    }
-  }
   // q in f16, channel order of the INT4 tile: in k-step 2j (2j + 1) of group
   // j, k-slots 2 tig, 2 tig + 1 <- channels 32j + 8 tig + {0, 4} ({2, 6}) and
   // k-slots 2 tig + 8, 2 tig + 9 <- channels 32j + 8 tig + {1, 5} ({3, 7})
   static __device__ __forceinline__ void q_words(const uint32_t *qrow, int ks, int tig,
                                                  uint32_t &w0, uint32_t &w1) {
-    const int base = (ks >> 1) * 16 + tig * 4 + (ks & 1);  // word of channels 8 tig + {0,1} or {2,3}
-    const uint32_t lo = to_f16x2(__ldg(qrow + base)), hi = to_f16x2(__ldg(qrow + base + 2));
-    w0 = __byte_perm(lo, hi, 0x5410);
-    w1 = __byte_perm(lo, hi, 0x7632);
+    q_words_q4<T>(qrow, ks, tig, w0, w1);
   }
-  static __device__ __forceinline__ int dim(int mt, int e, int g8) {
-    return (mt >> 1) * 32 + 4 * g8 + 2 * (mt & 1) + (e >> 1);
-  }
+  static __device__ __forceinline__ int dim(int mt, int e, int g8) { return dim_q4(mt, e, g8); }
 };
 
 // A quantised page policy for KV heads with a single query row (G = 1): the

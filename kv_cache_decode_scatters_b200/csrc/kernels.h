@@ -130,9 +130,10 @@ cudaError_t launch_read_stream(const void *src, size_t bytes, int mode, unsigned
 // Prefix pass of the shared-prefix decode: grid (n_groups * chunks, H_kv, row blocks).
 cudaError_t launch_prefix(const PrefixArgs &a, int d, DType dt, const CUtensorMap &tmK,
                           const CUtensorMap &tmV, int row_blocks, cudaStream_t s);
-// The same pass over a quantised cache (d = 128; tensor maps over the code
-// pools, scales in a.k_scale / a.v_scale); one CTA per SM.
-cudaError_t launch_prefix_q(const PrefixArgs &a, Code8 fmt, DType dt, const CUtensorMap &tmK,
+// The same pass over a quantised cache (tensor maps over the code pools,
+// scales in a.k_scale / a.v_scale): d = 128 on the tensor-memory pass (one
+// CTA per SM), d = 64 on the warp-level one.
+cudaError_t launch_prefix_q(const PrefixArgs &a, int d, Code8 fmt, DType dt, const CUtensorMap &tmK,
                             const CUtensorMap &tmV, int row_blocks, cudaStream_t s);
 // Query rows one prefix CTA handles.
 int prefix_rows_per_cta();

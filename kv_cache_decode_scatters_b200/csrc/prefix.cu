@@ -253,6 +253,194 @@ __global__ void __launch_bounds__(32 * kWarps, 1)
 }
 
 // ------------------------------------------------------------------------
+// The warp-level pass over a quantised cache (E4M3, INT8 or INT4 codes with
+// one fp32 scale per token, KV head and 32 channels), used at d = 64 where the
+// tensor-memory pass does not apply.  Same structure as prefix_kernel: a
+// CTA-wide ring of kStages pages, warp 0's lane 0 copying each page's K and V
+// code boxes (2-D TMA, swizzled by the code row size) and its two scale rows
+// (bulk copies) onto the stage's "full" mbarrier, every warp running the
+// quantised tile (tile_page_q8 / tile_page_q4, exact code values, fp32
+// scales) for its 8 query rows, one page at a time.
+namespace {
+template <int D, Code8 kFmt>
+struct PQGeo {
+  static constexpr int kRow = kFmt == Code8::INT4 ? D / 2 : D;  // code bytes of a token
+  static constexpr int kCodePage = kPage * kRow;
+  static constexpr int kScalePage = kPage * (D / 32) * 4;
+  // codes of K then V, then the scales of K then V, padded to keep the
+  // code boxes on their swizzle alignment
+  static constexpr int kStageBytes = ((2 * kCodePage + 2 * kScalePage + 1023) / 1024) * 1024;
+  static constexpr size_t smem() { return 1024 + (size_t)kStages * kStageBytes + 2 * kStages * 8; }
+};
+}  // namespace
+
+template <int D, typename T, Code8 kFmt>
+__global__ void __launch_bounds__(32 * kWarps, 1)
+    prefix_q_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV) {
+  using Pg = PQGeo<D, kFmt>;
+  constexpr int kSteps = D / 16;
+  constexpr bool kInt4 = kFmt == Code8::INT4;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)kStages * Pg::kStageBytes);
+  uint64_t *empty = full + kStages;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g8 = lane >> 2, tig = lane & 3;
+  const int cap = a.maxb * kPage;
+
+  grid_dependency_wait();
+  grid_launch_dependents();
+
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) write_skip(a, cap);
+
+  const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
+  const int h = blockIdx.y;
+  const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
+  const int gp = __ldg(a.group_pages + g);
+  if (!group_ok(a, s0, s1, gp)) {
+    if (tid == 0) flag_error(a.err, kErrSeqLen);
+    return;
+  }
+  const int rows = (s1 - s0) * a.G;
+  const int r0 = blockIdx.z * kRowsPerCta;
+  if (r0 >= rows || gp == 0) return;  // (rows of ineligible members are ignored by the merge)
+  const int p_begin = static_cast<int>((static_cast<long long>(chunk) * gp) / a.chunks);
+  const int p_end = static_cast<int>((static_cast<long long>(chunk + 1) * gp) / a.chunks);
+  const int npages = p_end - p_begin;
+
+  // this warp's 8 query rows: row -> member m = row / G, head row j = row % G
+  uint32_t qf[1][kSteps][2];
+  float acc[1][kSteps][4];
+  float m_run[1][2], l_run[1][2];
+  {
+    const int row = r0 + warp * 8 + g8;
+    const bool live = row < rows;
+    const int b = s0 + (live ? row / a.G : 0), j = live ? row % a.G : 0;
+    const uint32_t *qw = reinterpret_cast<const uint32_t *>(a.q) +
+                         (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + j) * (D / 2);
+#pragma unroll
+    for (int ks = 0; ks < kSteps; ++ks) {
+      if (live) {
+        if constexpr (kInt4) q_words_q4<T>(qw, ks, tig, qf[0][ks][0], qf[0][ks][1]);
+        else q_words_q8<T>(qw, ks, tig, qf[0][ks][0], qf[0][ks][1]);
+      } else {
+        qf[0][ks][0] = qf[0][ks][1] = 0u;
+      }
+    }
+#pragma unroll
+    for (int mt = 0; mt < kSteps; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[0][mt][e] = 0.f;
+    m_run[0][0] = m_run[0][1] = -INFINITY;
+    l_run[0][0] = l_run[0][1] = 0.f;
+  }
+
+  const uint32_t st0 = smem_u32(smem);
+  const uint32_t full0 = smem_u32(full), empty0 = smem_u32(empty);
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kWarps);
+    }
+    mbar_init_fence();
+  }
+  __syncthreads();
+
+  const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
+  const uint64_t policy = l2_policy_evict_normal();
+  constexpr int kG = D / 32;
+  // producer: page k of the chunk into stage k % kStages (warp 0, lane 0)
+  auto produce = [&](int k) {
+    const int s = k % kStages;
+    const uint32_t bar = full0 + 8 * s;
+    const int pb = __ldg(bt + p_begin + k);
+    if (pb < 0 || pb >= a.num_blocks) {
+      flag_error(a.err, kErrBlockTable);
+      mbar_arrive(bar);  // completes the phase with no bytes; consumers skip the page
+      return;
+    }
+    const int row = (pb * a.H_kv + h) * kPage;
+    const uint32_t dst = st0 + s * Pg::kStageBytes;
+    mbar_arrive_expect_tx(bar, 2 * Pg::kCodePage + 2 * Pg::kScalePage);
+    tma_load_2d(dst, &tmK, 0, row, bar, policy);
+    tma_load_2d(dst + Pg::kCodePage, &tmV, 0, row, bar, policy);
+    bulk_load(dst + 2 * Pg::kCodePage, a.k_scale + static_cast<size_t>(row) * kG, Pg::kScalePage, bar);
+    bulk_load(dst + 2 * Pg::kCodePage + Pg::kScalePage, a.v_scale + static_cast<size_t>(row) * kG,
+              Pg::kScalePage, bar);
+  };
+  if (tid == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+    for (int k = 0; k < kStages && k < npages; ++k) produce(k);
+  }
+
+  bool failed = false;
+  int k = 0;
+  for (; k < npages; ++k) {
+    const int s = k % kStages;
+    const uint32_t ph = (k / kStages) & 1;
+    const bool ok = mbar_wait_bounded(full0 + 8 * s, ph);
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) flag_error(a.err, kErrTimeout);
+      failed = true;
+      break;
+    }
+    const int pb = __ldg(bt + p_begin + k);
+    if (pb >= 0 && pb < a.num_blocks) {  // (a page outside the pool was flagged and not copied)
+      uint8_t *st = smem + (size_t)s * Pg::kStageBytes;
+      const float *ks = reinterpret_cast<const float *>(st + 2 * Pg::kCodePage);
+      if constexpr (kInt4)
+        tile_page_q4<D, 1>(smem_u32(st), smem_u32(st + Pg::kCodePage), ks, ks + kPage * kG, kPage,
+                           a.scale_log2, lane, qf, acc, m_run, l_run);
+      else
+        tile_page_q8<D, 1, kFmt>(smem_u32(st), smem_u32(st + Pg::kCodePage), ks, ks + kPage * kG,
+                                 kPage, a.scale_log2, lane, qf, acc, m_run, l_run);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * s);
+    if (tid == 0 && k + kStages < npages) {
+      // every warp has released stage s before it is refilled
+      if (mbar_wait_bounded(empty0 + 8 * s, ph)) produce(k + kStages);
+      else flag_error(a.err, kErrTimeout);
+    }
+  }
+  if (failed) {
+    // let the copies in flight land before the CTA exits
+    for (int kk = k; kk < npages && kk < k + kStages; ++kk)
+      mbar_wait_bounded(full0 + 8 * (kk % kStages), (kk / kStages) & 1);
+    return;
+  }
+
+  // normalised partial (o, lse) of this chunk for each live row
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    float l = l_run[0][i];
+    l += __shfl_xor_sync(0xffffffffu, l, 4);
+    l += __shfl_xor_sync(0xffffffffu, l, 8);
+    l += __shfl_xor_sync(0xffffffffu, l, 16);
+    const int row = r0 + warp * 8 + 2 * tig + i;
+    if (row >= rows) continue;
+    const int b = s0 + row / a.G, j = row % a.G;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const float lse = l > 0.f ? (m_run[0][i] + fast_log2(l)) * kLn2 : -INFINITY;
+    const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + b) * a.G + j;
+    float *o = a.pre_o + idx * D;
+    const uint64_t keep = l2_policy_evict_last();  // read again by the merge
+#pragma unroll
+    for (int mt = 0; mt < kSteps; ++mt) {
+      const int c0 = kInt4 ? dim_q4(mt, i, g8) : dim_q8(mt, i, g8);
+      const int c2 = kInt4 ? dim_q4(mt, 2 + i, g8) : dim_q8(mt, 2 + i, g8);
+      st_keep(o + c0, acc[0][mt][i] * inv, keep);
+      st_keep(o + c2, acc[0][mt][2 + i] * inv, keep);
+    }
+    if (g8 == 0) st_keep(a.pre_lse + idx, lse, keep);
+  }
+}
+
+// ------------------------------------------------------------------------
 // The same pass on the 5th-generation tensor cores (d = 128).
 //
 // The 128 query rows of a CTA are the M dimension of tcgen05.mma, so every
@@ -1268,9 +1456,29 @@ cudaError_t launch_prefix_q_t(const PrefixArgs &a, const CUtensorMap &tmK, const
   return launch_pdl(kern, grid, dim3(32 * kTqWarps), smem, st, a, tmK, tmV);
 }
 
+// d = 64: the warp-level pass
+template <typename T, Code8 kFmt>
+cudaError_t launch_prefix_q64_t(const PrefixArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                                int row_blocks, cudaStream_t st) {
+  auto kern = prefix_q_kernel<64, T, kFmt>;
+  const size_t smem = PQGeo<64, kFmt>::smem();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.n_groups * a.chunks, a.H_kv, row_blocks);
+  return launch_pdl(kern, grid, dim3(32 * kWarps), smem, st, a, tmK, tmV);
+}
+
 template <typename T>
-cudaError_t launch_prefix_q_d(const PrefixArgs &a, Code8 fmt, const CUtensorMap &tmK,
+cudaError_t launch_prefix_q_d(const PrefixArgs &a, int d, Code8 fmt, const CUtensorMap &tmK,
                               const CUtensorMap &tmV, int row_blocks, cudaStream_t st) {
+  if (d == 64) {
+    switch (fmt) {
+      case Code8::E4M3: return launch_prefix_q64_t<T, Code8::E4M3>(a, tmK, tmV, row_blocks, st);
+      case Code8::INT8: return launch_prefix_q64_t<T, Code8::INT8>(a, tmK, tmV, row_blocks, st);
+      default: return launch_prefix_q64_t<T, Code8::INT4>(a, tmK, tmV, row_blocks, st);
+    }
+  }
   switch (fmt) {
     case Code8::E4M3: return launch_prefix_q_t<T, Code8::E4M3>(a, tmK, tmV, row_blocks, st);
     case Code8::INT8: return launch_prefix_q_t<T, Code8::INT8>(a, tmK, tmV, row_blocks, st);
@@ -1279,11 +1487,11 @@ cudaError_t launch_prefix_q_d(const PrefixArgs &a, Code8 fmt, const CUtensorMap 
 }
 }  // namespace
 
-cudaError_t launch_prefix_q(const PrefixArgs &a, Code8 fmt, DType dt, const CUtensorMap &tmK,
+cudaError_t launch_prefix_q(const PrefixArgs &a, int d, Code8 fmt, DType dt, const CUtensorMap &tmK,
                             const CUtensorMap &tmV, int row_blocks, cudaStream_t s) {
   if (a.n_groups == 0 || a.B == 0) return cudaSuccess;
-  return dt == DType::BF16 ? launch_prefix_q_d<__nv_bfloat16>(a, fmt, tmK, tmV, row_blocks, s)
-                           : launch_prefix_q_d<__half>(a, fmt, tmK, tmV, row_blocks, s);
+  return dt == DType::BF16 ? launch_prefix_q_d<__nv_bfloat16>(a, d, fmt, tmK, tmV, row_blocks, s)
+                           : launch_prefix_q_d<__half>(a, d, fmt, tmK, tmV, row_blocks, s);
 }
 
 cudaError_t launch_prefix(const PrefixArgs &a, int d, DType dt, const CUtensorMap &tmK,

@@ -322,6 +322,46 @@ __device__ __forceinline__ uint32_t f16pack(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// A q word (two channels, storage dtype T) as an f16 pair: the quantised
+// tiles multiply in f16 (inputs beyond the f16 range are not supported).
+template <typename T>
+__device__ __forceinline__ uint32_t q_to_f16x2(uint32_t w) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w));
+    return f16pack(f.x, f.y);
+  } else {
+    return w;
+  }
+}
+
+// q's B fragment of k-step ks for the 8-bit tile: k-slots 2 tig, 2 tig + 1
+// <- channels 16 ks + 4 tig, + 1 and k-slots 2 tig + 8, + 9 <- channels
+// 16 ks + 4 tig + 2, + 3 (the order ldmatrix gives the code bytes).
+template <typename T>
+__device__ __forceinline__ void q_words_q8(const uint32_t *qrow, int ks, int tig, uint32_t &w0,
+                                           uint32_t &w1) {
+  w0 = q_to_f16x2<T>(__ldg(qrow + ks * 8 + 2 * tig));
+  w1 = q_to_f16x2<T>(__ldg(qrow + ks * 8 + 2 * tig + 1));
+}
+// Output channel of accumulator element e of m-tile mt (8-bit tile).
+__device__ __forceinline__ int dim_q8(int mt, int e, int g8) { return mt * 16 + 2 * g8 + (e >> 1); }
+
+// q's B fragment for the INT4 tile: in k-step 2j (2j + 1) of group j, k-slots
+// 2 tig, 2 tig + 1 <- channels 32j + 8 tig + {0, 4} ({2, 6}) and k-slots
+// 2 tig + 8, + 9 <- channels 32j + 8 tig + {1, 5} ({3, 7}).
+template <typename T>
+__device__ __forceinline__ void q_words_q4(const uint32_t *qrow, int ks, int tig, uint32_t &w0,
+                                           uint32_t &w1) {
+  const int base = (ks >> 1) * 16 + tig * 4 + (ks & 1);  // word of channels 8 tig + {0,1} or {2,3}
+  const uint32_t lo = q_to_f16x2<T>(__ldg(qrow + base)), hi = q_to_f16x2<T>(__ldg(qrow + base + 2));
+  w0 = __byte_perm(lo, hi, 0x5410);
+  w1 = __byte_perm(lo, hi, 0x7632);
+}
+// Output channel of accumulator element e of m-tile mt (INT4 tile).
+__device__ __forceinline__ int dim_q4(int mt, int e, int g8) {
+  return (mt >> 1) * 32 + 4 * g8 + 2 * (mt & 1) + (e >> 1);
+}
+
 // Byte offset of 16-byte chunk c of token row t in a 16-row page of 128-byte
 // rows staged by one 128B-swizzled TMA box.
 __device__ __forceinline__ uint32_t swz8(int t, int c) {

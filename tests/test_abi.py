@@ -282,7 +282,7 @@ def test_shared_prefix_validation(kw, status):
 
 @pytest.mark.parametrize("fmt", ["fp8", "int8", "int4"])
 @pytest.mark.parametrize("kw,status", [
-    (dict(d=64), kvd.KVD_ERR_UNSUPPORTED),                # the quantised prefix pass is d = 128
+    (dict(d=96), kvd.KVD_ERR_UNSUPPORTED),                # quantised prefix passes: d = 64 or 128
     (dict(ng=-1), kvd.KVD_ERR_INVALID),
     (dict(kn=DUMMY, vn=NULL), kvd.KVD_ERR_INVALID),       # both or neither
     (dict(kn=MISALIGNED, vn=DUMMY), kvd.KVD_ERR_INVALID),

@@ -350,3 +350,40 @@ def test_decode_d64_larger_batch_every_row(kvd, fmt):
     err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
     assert err <= TOL[w.dtype], f"max abs error {err}"
     assert kvd.kvd_read_device_error() == 0
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8", "int4"])
+def test_fused_step_full_size_mha7b_one_query_row(kvd, fmt):
+    # the benchmark's 7B-shape MHA step (one query row per KV head, the
+    # quantised tile with the scale groups in its N columns) over each
+    # quantised cache: pools and out bit-identical to the two-call path,
+    # sampled sequences against the oracle
+    w = named_config("mha7b", device="cuda", gen_device="cuda")
+    si = step_inputs(w, 0)
+    quant = getattr(kvd, "kvd_quantize_" + fmt)
+    k8, ks = quant(w.k_cache)
+    v8, vs = quant(w.v_cache)
+    pools = [k8, v8, ks, vs]
+    two = [t.clone() for t in pools]
+    bt = w.block_table.cuda()
+    out = getattr(kvd, "kvd_decode_step_" + fmt)(si["q"], si["k_new"], si["v_new"], *pools, bt,
+                                                  si["seq_lens"], w.scale)
+    getattr(kvd, "kvd_append_" + fmt)(*two, bt, si["slot"], si["k_new"], si["v_new"])
+    out2 = getattr(kvd, "kvd_decode_attention_" + fmt)(si["q"], *two, bt, si["seq_lens"], w.scale)
+    torch.cuda.synchronize()
+    for a, b in zip(pools, two):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+    del two
+    rows = [0, 13, 31]
+    (hk, hv, hks, hvs), bts, pages = oracle_q8_rows(w, fmt, si, rows)
+    idx = torch.tensor(pages, dtype=torch.long, device="cuda")
+    sel = torch.tensor(rows, dtype=torch.long)
+    rows_ok = data_rows(w.k_cache.index_select(0, idx), w.v_cache.index_select(0, idx), bts,
+                        {"slot": si["slot"].cpu()[sel]})
+    assert_pools_equal([t.index_select(0, idx) for t in pools], (hk, hv, hks, hvs), rows_ok)
+    ref, _ = getattr(oracle, "attend_" + fmt)(to_words(si["q"].cpu()[sel]), hk, hv, hks, hvs, bts,
+                                              si["seq_lens"].cpu()[sel].numpy(), w.scale, odt(w))
+    err = float(np.max(np.abs(out.cpu()[sel].float().double().numpy() - ref)))
+    assert err <= TOL[w.dtype], f"max abs error {err}"
+    assert kvd.kvd_read_device_error() == 0

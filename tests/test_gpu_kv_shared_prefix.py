@@ -1,5 +1,6 @@
 """GPU parity of the shared-prefix decode over quantised caches (E4M3, INT8,
-INT4; d = 128) against the oracle.
+INT4; d = 128 on the tensor-memory prefix pass, d = 64 on the warp-level one)
+against the oracle.
 
 The oracle's pools are its own quantisation of the 16-bit pool plus its own
 quantising append of the step; the GPU's pools after the fused append must
@@ -54,22 +55,27 @@ def oracle_attend(w, si, pools, fmt, rows=None):
 
 
 CASES = [
-    # B, H_q, H_kv, dtype, lens, groups, prefix tokens, partitions
-    (8, 32, 8, "f16", [300, 257, 520, 999, 290, 400, 700, 266], 2, 256, 0),
-    (6, 64, 8, "bf16", [40, 33, 90, 49, 34, 70], 3, 32, 0),
-    (4, 16, 1, "bf16", [200, 145, 160, 300], 2, 144, 5),                 # MQA, group 16
+    # B, H_q, H_kv, d, dtype, lens, groups, prefix tokens, partitions
+    (8, 32, 8, 128, "f16", [300, 257, 520, 999, 290, 400, 700, 266], 2, 256, 0),
+    (6, 64, 8, 128, "bf16", [40, 33, 90, 49, 34, 70], 3, 32, 0),
+    (4, 16, 1, 128, "bf16", [200, 145, 160, 300], 2, 144, 5),                 # MQA, group 16
     # one group of 40 members x 4 rows = 160 query rows: two 128-row blocks
-    (40, 32, 8, "f16", [530 + 7 * i for i in range(40)], 1, 512, 0),
+    (40, 32, 8, 128, "f16", [530 + 7 * i for i in range(40)], 1, 512, 0),
     # a long shared prefix: several 64-token steps per chunk and a ragged last step
-    (16, 64, 8, "bf16", [2100 + 13 * i for i in range(16)], 2, 2048, 0),
+    (16, 64, 8, 128, "bf16", [2100 + 13 * i for i in range(16)], 2, 2048, 0),
+    # d = 64: the warp-level prefix pass
+    (8, 16, 4, 64, "f16", [300, 257, 520, 999, 290, 400, 700, 266], 2, 256, 0),
+    (4, 8, 8, 64, "f16", [600, 513, 530, 1000], 1, 512, 5),                  # MHA
+    (6, 32, 8, 64, "bf16", [40, 33, 90, 49, 34, 70], 3, 32, 0),
+    (40, 32, 8, 64, "bf16", [530 + 7 * i for i in range(40)], 1, 512, 0),    # two row blocks
 ]
 
 
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_{c[3]}_g{c[5]}_p{c[6]}")
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c[0]}_Hq{c[1]}_Hkv{c[2]}_d{c[3]}_{c[4]}_g{c[6]}_p{c[7]}")
 def test_fused_shared_prefix_matches_oracle_and_plain_step(kvd, fmt, case):
-    B, H_q, H_kv, dtype, lens, groups, prefix, parts = case
-    w = build_workload("spq", B, H_q, H_kv, 128, dtype, lens, seed=2100 + CASES.index(case),
+    B, H_q, H_kv, hd, dtype, lens, groups, prefix, parts = case
+    w = build_workload("spq", B, H_q, H_kv, hd, dtype, lens, seed=2100 + CASES.index(case),
                        prefix_groups=groups, prefix_tokens=prefix)
     si = step_inputs(w, 0)
     pools = q_state(kvd, w, fmt)
@@ -123,13 +129,15 @@ def test_shared_prefix_attention_only_after_append(kvd, fmt):
     assert kvd.kvd_read_device_error() == 0
 
 
+@pytest.mark.parametrize("hd", [128, 64])
 @pytest.mark.parametrize("fmt", FMTS)
-def test_shared_prefix_bad_page_is_flagged_and_contained(kvd, fmt):
+def test_shared_prefix_bad_page_is_flagged_and_contained(kvd, fmt, hd):
     # a block-table entry inside group 0's shared prefix points outside the
-    # pool: the prefix pass skips that page's copies (its tiles hold stale
-    # values, masked), the error word says so, and group 1 is still right
+    # pool: the prefix pass skips that page (d = 128: its tiles hold stale
+    # values, masked; d = 64: no warp attends it), the error word says so, and
+    # group 1 is still right
     lens = [300, 257, 520, 999, 290, 400, 700, 266]
-    w = build_workload("spqbad", 8, 32, 8, 128, "f16", lens, seed=2161, prefix_groups=2, prefix_tokens=256)
+    w = build_workload("spqbad", 8, 32, 8, hd, "f16", lens, seed=2161, prefix_groups=2, prefix_tokens=256)
     si = step_inputs(w, 0)
     pools = q_state(kvd, w, fmt)
     bt = w.block_table.cuda()
