@@ -4,7 +4,7 @@ import numpy as np
 import torch
 
 import oracle
-from synth import step_inputs, to_words
+from synth import build_workload, step_inputs, to_words
 
 TOL = {torch.float16: 2e-3, torch.bfloat16: 1e-2}   # max-abs error vs the fp64 oracle
 LSE_TOL = 1e-3
@@ -164,10 +164,34 @@ def assert_out_close(gpu_out, ref, dtype):
     return float(err.max()) if err.size else 0.0
 
 
+def uneven_groups_case(d, dtype, H_q, H_kv, seed):
+    """Groups of different sizes and shared page counts, made by pointing
+    each member's first pages at its group's first member's pages."""
+    sizes = [5, 40, 1, 3, 7]
+    gpages = [4, 10, 2, 0, 6]
+    rng = np.random.default_rng(seed)
+    lens, starts = [], [0]
+    for sz, gp in zip(sizes, gpages):
+        for i in range(sz):
+            lens.append(int(gp * 16 + 1 + rng.integers(0, 90)))
+        starts.append(starts[-1] + sz)
+    lens[starts[1] + 3] = 10 * 16      # exactly the shared prefix: no private page
+    lens[starts[4] + 2] = 40           # shorter than its group's 6 shared pages
+    w = build_workload("spu", len(lens), H_q, H_kv, d, dtype, lens, seed=seed, spare_pages=4)
+    bt2 = w.block_table.clone()
+    for g, gp in enumerate(gpages):
+        s0, s1 = starts[g], starts[g + 1]
+        for b in range(s0 + 1, s1):
+            bt2[b, :gp] = w.block_table[s0, :gp]
+    gs = torch.tensor(starts, dtype=torch.int32)
+    gpg = torch.tensor(gpages, dtype=torch.int32)
+    return w, bt2, gs, gpg, max(sizes)
+
+
 def words(t):
     return to_words(t)
 
 
-__all__ = ["TOL", "LSE_TOL", "ERROR_REPORT", "record_error", "assert_out_close", "host", "oracle_q8", "oracle_q8_rows",
+__all__ = ["TOL", "LSE_TOL", "ERROR_REPORT", "record_error", "assert_out_close", "uneven_groups_case", "host", "oracle_q8", "oracle_q8_rows",
            "data_rows", "assert_pools_equal", "odt", "gpu_state", "gpu_step", "oracle_step", "max_err", "max_lse_err",
            "words", "step_inputs"]

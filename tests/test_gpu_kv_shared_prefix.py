@@ -15,7 +15,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import LSE_TOL, TOL, assert_out_close, assert_pools_equal, data_rows, odt, oracle_q8, oracle_q8_rows
+from gpu_helpers import (LSE_TOL, TOL, assert_out_close, assert_pools_equal, data_rows, odt, oracle_q8,
+                         oracle_q8_rows, uneven_groups_case)
 from synth import build_workload, named_config, step_inputs, to_words
 
 pytestmark = pytest.mark.gpu
@@ -153,6 +154,52 @@ def test_shared_prefix_bad_page_is_flagged_and_contained(kvd, fmt, hd):
     assert kvd.kvd_read_device_error(clear=True) & kvd.KVD_DEVERR_BLOCK_TABLE
     ref, _ = oracle_attend(w, si, oracle_q8(w, fmt, si), fmt)
     assert_out_close(out[per:], ref[per:], w.dtype)
+
+
+@pytest.mark.parametrize("hd,dtype,H_q,H_kv", [(128, "f16", 32, 8), (64, "bf16", 16, 4)])
+@pytest.mark.parametrize("fmt", FMTS)
+def test_uneven_groups(kvd, fmt, hd, dtype, H_q, H_kv):
+    # groups of 5, 40, 1, 3 and 7 members sharing 4, 10, 2, 0 and 6 pages:
+    # different page counts and row blocks per unit, one member exactly as
+    # long as its prefix, one shorter than it (attended whole).  The step's
+    # rows are appended through each member's own pages, attention runs on
+    # the shared table; the oracle does the same
+    w, bt2, gs, gpg, maxg = uneven_groups_case(hd, dtype, H_q, H_kv, seed=2201)
+    si = step_inputs(w, 0)
+    pools = q_state(kvd, w, fmt)
+    d = {k: v.cuda() for k, v in si.items()}
+    getattr(kvd, "kvd_append_" + fmt)(*pools, w.block_table.cuda(), d["slot"], d["k_new"], d["v_new"])
+    kvd.kvd_read_device_error(clear=True)
+    lse = torch.empty((w.B, w.H_q), dtype=torch.float32, device="cuda")
+    out = getattr(kvd, "kvd_decode_attention_shared_prefix_" + fmt)(
+        d["q"], *pools, bt2.cuda(), d["seq_lens"], gs.cuda(), gpg.cuda(), maxg, w.scale, lse_out=lse)
+    torch.cuda.synchronize()
+    assert kvd.kvd_read_device_error() == 0
+    hk, hv, hks, hvs = oracle_q8(w, fmt, si)
+    ref, ref_lse = getattr(oracle, "attend_" + fmt)(to_words(si["q"]), hk, hv, hks, hvs, bt2.numpy(),
+                                                    si["seq_lens"].numpy(), w.scale, odt(w))
+    assert_out_close(out, ref, w.dtype)
+    assert float(np.max(np.abs(lse.cpu().double().numpy() - ref_lse))) <= LSE_TOL
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_group_larger_than_declared_is_flagged_and_attended_whole(kvd, fmt):
+    # max_group_size below the 40-member group: that group is invalid (its
+    # members are attended whole, the error word says so), the others share
+    w, bt2, gs, gpg, maxg = uneven_groups_case(128, "f16", 32, 8, seed=2202)
+    si = step_inputs(w, 0)
+    pools = q_state(kvd, w, fmt)
+    d = {k: v.cuda() for k, v in si.items()}
+    getattr(kvd, "kvd_append_" + fmt)(*pools, w.block_table.cuda(), d["slot"], d["k_new"], d["v_new"])
+    kvd.kvd_read_device_error(clear=True)
+    out = getattr(kvd, "kvd_decode_attention_shared_prefix_" + fmt)(
+        d["q"], *pools, bt2.cuda(), d["seq_lens"], gs.cuda(), gpg.cuda(), 8, w.scale)
+    torch.cuda.synchronize()
+    assert kvd.kvd_read_device_error(clear=True) & kvd.KVD_DEVERR_SEQ_LEN
+    hk, hv, hks, hvs = oracle_q8(w, fmt, si)
+    ref, _ = getattr(oracle, "attend_" + fmt)(to_words(si["q"]), hk, hv, hks, hvs, bt2.numpy(),
+                                              si["seq_lens"].numpy(), w.scale, odt(w))
+    assert_out_close(out, ref, w.dtype)
 
 
 @pytest.mark.parametrize("fmt", FMTS)

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from gpu_helpers import (LSE_TOL, TOL, gpu_state, gpu_step, max_err, max_lse_err, oracle_step,
-                         words)
+                         uneven_groups_case, words)
 from synth import CANARY_WORD, build_workload, step_inputs, to_words
 
 pytestmark = pytest.mark.gpu
@@ -479,30 +479,6 @@ def test_shared_prefix_member_shorter_than_prefix_is_attended_whole(kvd):
                            si["seq_lens"].numpy(), w.scale, oracle.F16)
     err = float(np.max(np.abs(out.float().cpu().double().numpy() - ref)))
     assert err <= TOL[w.dtype]
-
-
-def uneven_groups_case(d, dtype, H_q, H_kv, seed):
-    """Groups of different sizes and shared page counts, made by pointing
-    each member's first pages at its group's first member's pages."""
-    sizes = [5, 40, 1, 3, 7]
-    gpages = [4, 10, 2, 0, 6]
-    rng = np.random.default_rng(seed)
-    lens, starts = [], [0]
-    for sz, gp in zip(sizes, gpages):
-        for i in range(sz):
-            lens.append(int(gp * 16 + 1 + rng.integers(0, 90)))
-        starts.append(starts[-1] + sz)
-    lens[starts[1] + 3] = 10 * 16      # exactly the shared prefix: no private page
-    lens[starts[4] + 2] = 40           # shorter than its group's 6 shared pages
-    w = build_workload("spu", len(lens), H_q, H_kv, d, dtype, lens, seed=seed, spare_pages=4)
-    bt2 = w.block_table.clone()
-    for g, gp in enumerate(gpages):
-        s0, s1 = starts[g], starts[g + 1]
-        for b in range(s0 + 1, s1):
-            bt2[b, :gp] = w.block_table[s0, :gp]
-    gs = torch.tensor(starts, dtype=torch.int32)
-    gpg = torch.tensor(gpages, dtype=torch.int32)
-    return w, bt2, gs, gpg, max(sizes)
 
 
 @pytest.mark.parametrize("d,dtype,H_q,H_kv", [(128, "f16", 32, 8), (128, "bf16", 64, 8), (64, "f16", 16, 4)])
