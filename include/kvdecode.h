@@ -482,7 +482,7 @@ kvd_status kvd_read_device_error(unsigned int *flags, int clear);
  * land (with the full limit) and leaves the launch, whose output is then
  * undefined.  This call sets the poll limit of those page waits for every
  * later decode launch of the process (kvd_decode_attention, kvd_decode_step,
- * the shared-prefix call's decode pass and the 8-bit calls): 0 makes every
+ * the shared-prefix calls' decode pass and the quantised calls): 0 makes every
  * first wait give up at once, a negative value restores the default.  The
  * waits that drain copies in flight always keep the full limit, so a lowered
  * limit ends the launch early and never leaves a copy behind.  Always returns

@@ -294,8 +294,9 @@ def kvd_decode_attention_shared_prefix(q, k_cache, v_cache, block_table, seq_len
     return out
 
 
-# 8-bit KV caches: E4M3 codes (torch.uint8 storage) or INT8 codes (torch.int8),
-# one fp32 scale per (token, KV head, 32 channels).
+# Quantised KV caches: E4M3 codes (torch.uint8 storage), INT8 codes (torch.int8)
+# or INT4 codes two per byte (torch.uint8), one fp32 scale per (token, KV head,
+# 32 channels).
 _CODE8 = {"fp8": torch.uint8, "int8": torch.int8, "int4": torch.uint8}
 # code bytes of a row of d values
 _ROW = {"fp8": lambda d: d, "int8": lambda d: d, "int4": lambda d: d // 2}
@@ -436,7 +437,7 @@ def kvd_append_fp8(k_codes, v_codes, k_scale, v_scale, block_table, slot, k_new,
 
 def kvd_decode_attention_fp8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale=None,
                              out=None, num_partitions=0, workspace=None, lse_out=None, stream=None):
-    """kvd_decode_attention over the 8-bit cache (d = 128).  Returns out (q's dtype)."""
+    """kvd_decode_attention over the E4M3 cache (d = 64 or 128).  Returns out (q's dtype)."""
     return _decode8("fp8", q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale, out,
                     num_partitions, workspace, lse_out, stream)
 
