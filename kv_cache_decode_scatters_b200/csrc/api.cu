@@ -119,9 +119,10 @@ WsLayout ws_layout(int B, int G, int d, long long slots) {
 }
 
 // Shared-prefix scratch after the decode workspace: per-sequence skipped
-// pages, then the prefix chunks' partial lse and o.
+// pages, the plan (partitions of the suffix decode, the prefix pass's exit
+// count), then the prefix chunks' partial lse and o.
 struct PrefixLayout {
-  size_t skip, pre_lse, pre_o, total;
+  size_t skip, plan, pre_lse, pre_o, total;
   int chunks, row_blocks;
 };
 
@@ -150,7 +151,8 @@ kvd_status prefix_layout(int B, int H_kv, int G, int d, int n_groups, int max_gr
   L.chunks = static_cast<int>(chunks);
   L.row_blocks = static_cast<int>(rb);
   L.skip = round_up(base, 256);
-  L.pre_lse = L.skip + round_up(static_cast<size_t>(B) * 4, 256);
+  L.plan = L.skip + round_up(static_cast<size_t>(B) * 4, 256);
+  L.pre_lse = L.plan + 256;
   const size_t n = static_cast<size_t>(chunks) * H_kv * B * G;
   L.pre_o = L.pre_lse + round_up(n * 4, 256);
   L.total = L.pre_o + n * d * 4;
@@ -373,7 +375,7 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   }
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  kvd::DecodeArgs a;
+  kvd::DecodeArgs a{};
   a.q = q;
   a.block_table = block_table;
   a.seq_lens = seq_lens;
@@ -411,12 +413,13 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
   // which take them writable)
   a.k_scale = const_cast<float *>(k_scale);
   a.v_scale = const_cast<float *>(v_scale);
+  a.plan = nullptr;
 
   const kvd::DType dt = dtype == KVD_BF16 ? kvd::DType::BF16 : kvd::DType::F16;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (n_groups > 0) {
-    kvd::PrefixArgs pa;
+    kvd::PrefixArgs pa{};
     pa.q = q;
     pa.block_table = block_table;
     pa.seq_lens = seq_lens;
@@ -439,17 +442,34 @@ static kvd_status decode_impl(const void *q, const void *k_cache, const void *v_
     pa.maxg = max_group_size;
     pa.k_scale = k_scale;
     pa.v_scale = v_scale;
-    e = q8 ? kvd::launch_prefix_q(pa, d, fmt, dt, tm[0], tm[1], PL.row_blocks, s)
-           : kvd::launch_prefix(pa, d, dt, tm[0], tm[1], PL.row_blocks, s);
-    if (e != cudaSuccess) return cuda_fail(e, "prefix launch");
+    pa.plan = reinterpret_cast<int32_t *>(ws + PL.plan);
+    // automatic partitions: the suffix decode leaves the prefix pass its
+    // share of the SMs and the two run side by side; a caller's explicit
+    // count is kept as given
+    kvd::prefix_split(pa, d, q8, fmt, num_partitions == 0);
+    pa.nparts = N;
+    pa.min_pages = a.min_pages;
+    pa.row_blocks = PL.row_blocks;
     a.skip = pa.skip;
     a.pre_o = pa.pre_o;
     a.pre_lse = pa.pre_lse;
     a.pre_chunks = PL.chunks;
+    a.plan = pa.plan;
+    // plan (skip, partitions) -> suffix decode -> prefix pass, scheduled as
+    // the decode starts and run on the SMs it leaves -> merge
+    e = kvd::launch_prefix_plan(pa, s);
+    if (e != cudaSuccess) return cuda_fail(e, "prefix plan launch");
+    e = q8 ? kvd::launch_decode_q8(a, d, dt, fmt, tm[0], tm[1], s, N)
+           : kvd::launch_decode(a, d, dt, tm[0], tm[1], s, N);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    e = q8 ? kvd::launch_prefix_q(pa, d, fmt, dt, tm[0], tm[1], PL.row_blocks, s)
+           : kvd::launch_prefix(pa, d, dt, tm[0], tm[1], PL.row_blocks, s);
+    if (e != cudaSuccess) return cuda_fail(e, "prefix launch");
+  } else {
+    e = q8 ? kvd::launch_decode_q8(a, d, dt, fmt, tm[0], tm[1], s, N)
+           : kvd::launch_decode(a, d, dt, tm[0], tm[1], s, N);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   }
-  e = q8 ? kvd::launch_decode_q8(a, d, dt, fmt, tm[0], tm[1], s, N)
-          : kvd::launch_decode(a, d, dt, tm[0], tm[1], s, N);
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   e = kvd::launch_decode_merge(a, d, dt, s);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return KVD_OK;

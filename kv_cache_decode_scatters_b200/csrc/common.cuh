@@ -156,7 +156,9 @@ __device__ __forceinline__ void grid_launch_dependents() {
 
 // Launch with programmatic stream serialisation: the grid may be scheduled
 // while the previous kernel in the stream is still finishing.  Every kernel
-// launched this way calls grid_dependency_wait() before touching memory.
+// launched this way calls grid_dependency_wait() before touching memory,
+// except the shared-prefix pass, which shares no buffer with the decode
+// launch before it and waits for it only as its last warp exits.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t st, Args &&...args) {

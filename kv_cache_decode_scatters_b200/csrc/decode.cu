@@ -68,6 +68,14 @@ struct Geo {
   }
 };
 
+// Partitions a launch over P pages uses: the automatic bound, capped in a
+// shared-prefix call by its plan, which leaves the other SMs to the prefix
+// pass running beside the decode.  The merge derives the same count.
+__device__ __forceinline__ int used_parts(const DecodeArgs &a, long long P) {
+  const int N = effective_parts(P, a.nparts, a.min_pages);
+  return a.plan ? min(N, max(1, __ldcg(a.plan))) : N;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------- page formats
@@ -399,7 +407,7 @@ __global__ void __launch_bounds__(32 * W, 1)
     __syncthreads();
   }
   const long long P = static_cast<long long>(cum[a.B]) * a.H_kv;
-  const int N = effective_parts(P, a.nparts, a.min_pages);
+  const int N = used_parts(a, P);
   if (blockIdx.x == 0)
     for (int i = tid; i <= a.B; i += Gm::kThreads) a.ws_cum[i] = cum[i];
 
@@ -1027,7 +1035,7 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeArgs a) {
   long long slot0 = 0;
   int count = 0;
   if (np > 0) {
-    const int N = effective_parts(P, a.nparts, a.min_pages);
+    const int N = used_parts(a, P);
     const long long s0 = static_cast<long long>(c0) * a.H_kv + static_cast<long long>(h) * np;
     const long long wf = part_of(s0, P, N), wl = part_of(s0 + np - 1, P, N);
     if (wf == wl && skip == 0) return;  // written directly by its only CTA

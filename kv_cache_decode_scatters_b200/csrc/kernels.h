@@ -61,6 +61,9 @@ struct DecodeArgs {
   // (k_cache / v_cache are then the code pools); written only by the fused append
   float *k_scale;
   float *v_scale;
+  // shared-prefix mode (null otherwise): plan[0] caps the partitions used, so
+  // that the prefix pass, running beside this launch, keeps the other SMs
+  const int32_t *plan;
 };
 
 // Quantise rows of d fp16/bf16 words into E4M3 codes + fp32 per-32-channel
@@ -97,6 +100,13 @@ struct PrefixArgs {
   int maxg;                    // members per group at most: a larger group is invalid
   const float *k_scale;        // quantised cache: scales [NB][H_kv][16][d/32] (else NULL)
   const float *v_scale;
+  // plan[0]: partitions the suffix decode uses; plan[2..3]: 64-bit count of
+  // the prefix pass's finished warps (zeroed by the plan launch)
+  int32_t *plan;
+  float weight;                // cost of a prefix page relative to a decode page (0: no split)
+  int nparts, min_pages;       // the decode launch's partition bound and minimum pages
+  int row_blocks;              // query-row blocks of the prefix launch (grid z)
+  int ctas_per_sm;             // prefix CTAs resident on one SM
 };
 
 struct GenericMergeArgs {
@@ -137,5 +147,15 @@ cudaError_t launch_prefix_q(const PrefixArgs &a, int d, Code8 fmt, DType dt, con
                             const CUtensorMap &tmV, int row_blocks, cudaStream_t s);
 // Query rows one prefix CTA handles.
 int prefix_rows_per_cta();
+// Plan of the shared-prefix call (one CTA, before the decode launch): writes
+// the per-sequence skip, the decode's partition count and clears the prefix
+// pass's exit count.
+cudaError_t launch_prefix_plan(const PrefixArgs &a, cudaStream_t s);
+// Sets a.weight, the time of one prefix page (one KV head, one row block)
+// relative to one decode page on one SM, which sizes the split of the SMs
+// between the two passes (0 without `split`, or where no split pays), and
+// a.ctas_per_sm, the prefix CTAs resident per SM, for a 16-bit cache or a
+// quantised one of format fmt.
+void prefix_split(PrefixArgs &a, int d, bool quantised, Code8 fmt, bool split);
 
 }  // namespace kvd

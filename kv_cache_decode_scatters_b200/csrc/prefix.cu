@@ -17,6 +17,12 @@
 // regular decode kernel (its per-sequence `skip`), and the merge kernel folds
 // suffix and prefix partials.
 //
+// Scheduling: a one-CTA plan launch writes `skip` and the suffix decode's
+// partition count; the decode runs next and leaves the prefix pass a share
+// of the SMs sized by the two passes' page counts and costs; this pass is
+// launched after the decode, scheduled as soon as the decode has started, so
+// the two stream side by side; the merge comes last.
+//
 // Staging: a CTA-wide ring of kStages pages.  Warp 0's lane 0 issues the TMA
 // loads (K and V boxes as in the decode kernel) on a "full" mbarrier per
 // stage; every warp arrives on the stage's "empty" mbarrier when done with
@@ -50,8 +56,8 @@ __device__ __forceinline__ bool group_ok(const PrefixArgs &a, int s0, int s1, in
   return s0 >= 0 && s1 <= a.B && s1 >= s0 && s1 - s0 <= a.maxg && gp >= 0 && gp <= a.maxb;
 }
 
-// Per-sequence shared pages for the suffix pass (CTA (0,0,0) of the prefix
-// launch writes them, all its threads).  A member whose length does not cover
+// Per-sequence shared pages for the suffix pass (the plan launch writes
+// them, all threads of its one CTA).  A member whose length does not cover
 // the group's pages keeps no shared pages and is attended whole by the decode
 // kernel; so do the members of an invalid group.
 __device__ void write_skip(const PrefixArgs &a, int cap) {
@@ -74,7 +80,90 @@ __device__ void write_skip(const PrefixArgs &a, int cap) {
   }
 }
 
+// Counts a warp of the prefix pass as finished; the last one waits for the
+// decode grid launched before this pass.  The pass does not wait for that
+// grid at its start (the two share no buffer, so they run side by side), but
+// the merge launched after the pass reads the decode's partials too: it
+// waits for this grid, which then cannot complete before the decode has.
+__device__ __forceinline__ void prefix_exit(const PrefixArgs &a) {
+  if ((threadIdx.x & 31) == 0) {
+    const unsigned long long warps = static_cast<unsigned long long>(gridDim.x) * gridDim.y *
+                                     gridDim.z * (blockDim.x >> 5);
+    unsigned long long *done = reinterpret_cast<unsigned long long *>(a.plan + 2);
+    if (atomicAdd(done, 1ull) + 1ull == warps) grid_dependency_wait();
+  }
+}
+
+constexpr int kPlanThreads = 256;
+
+// Sum of v over the CTA (kPlanThreads threads); every thread gets it.
+__device__ long long plan_sum(long long v, long long *red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  long long t = 0;
+  for (int w = 0; w < kPlanThreads / 32; ++w) t += red[w];
+  return t;
+}
+
 }  // namespace
+
+// The plan of a shared-prefix call, one CTA ahead of the decode launch:
+//  * skip[b], the shared pages of sequence b the prefix pass attends;
+//  * plan[0], the partitions the suffix decode uses.  With weight w > 0 the
+//    decode takes the share of the nparts SMs that its pages are of the
+//    whole work, P / (P + w * Pp), with P the suffix pages and Pp the prefix
+//    pages (per KV head and row block); its other CTAs exit at once and the
+//    prefix pass, launched next, runs on their SMs meanwhile.  The prefix
+//    SMs are then adjusted so that the pass's CTAs fill whole waves there:
+//    a part-filled last wave would leave them idle while the decode runs;
+//  * plan[2..3] = 0, the prefix pass's count of finished warps.
+__global__ void __launch_bounds__(kPlanThreads) prefix_plan_kernel(const PrefixArgs a) {
+  __shared__ long long red[kPlanThreads / 32];
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int tid = threadIdx.x;
+  const int cap = a.maxb * kPage;
+  write_skip(a, cap);
+  __syncthreads();  // skip[] of every sequence written (by other threads too)
+  long long sp = 0, pp = 0, cp = 0;  // suffix pages, prefix pages, prefix row blocks
+  for (int b = tid; b < a.B; b += kPlanThreads) {
+    const int np = (clamp_len(__ldcg(a.seq_lens + b), cap) + kPage - 1) / kPage;
+    sp += max(0, np - __ldcg(a.skip + b));
+  }
+  for (int g = tid; g < a.n_groups; g += kPlanThreads) {
+    const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
+    const int gp = __ldg(a.group_pages + g);
+    if (!group_ok(a, s0, s1, gp) || gp == 0) continue;
+    const long long rows = static_cast<long long>(s1 - s0) * a.G;
+    const long long rb = (rows + kRowsPerCta - 1) / kRowsPerCta;
+    pp += gp * rb;
+    cp += rb;
+  }
+  sp = plan_sum(sp, red);
+  pp = plan_sum(pp, red);
+  cp = plan_sum(cp, red);
+  if (tid == 0) {
+    const long long P = sp * a.H_kv, Pp = pp * a.H_kv;
+    int N = effective_parts(P, a.nparts, a.min_pages);
+    if (a.weight > 0.f && Pp > 0 && a.nparts > 1) {
+      const double dp = static_cast<double>(P);
+      const double share = dp / (dp + a.weight * static_cast<double>(Pp));
+      const double k_raw = fmax(1.0, a.nparts * (1.0 - share));  // SMs for the prefix pass
+      const long long ctas = cp * a.chunks * a.H_kv;               // its CTAs with work
+      const long long slots = a.ctas_per_sm;                        // resident per SM
+      const long long waves = max(1LL, llround(static_cast<double>(ctas) / (slots * k_raw)));
+      const long long k =
+          min(static_cast<long long>(a.nparts - 1), (ctas + slots * waves - 1) / (slots * waves));
+      N = min(N, max(1, a.nparts - static_cast<int>(k)));
+    }
+    a.plan[0] = N;
+    a.plan[1] = 0;
+    *reinterpret_cast<unsigned long long *>(a.plan + 2) = 0ull;
+  }
+}
 
 template <int D, typename T>
 __global__ void __launch_bounds__(32 * kWarps, 1)
@@ -91,165 +180,165 @@ __global__ void __launch_bounds__(32 * kWarps, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, tig = lane & 3;
-  const int cap = a.maxb * kPage;
 
-  grid_dependency_wait();
+  // no wait for the decode launch before this pass (prefix_exit); every
+  // return of the body below still passes through prefix_exit
   grid_launch_dependents();
-
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) write_skip(a, cap);
-
-  const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
-  const int h = blockIdx.y;
-  const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
-  int gp = __ldg(a.group_pages + g);
-  if (!group_ok(a, s0, s1, gp)) {
-    if (tid == 0) flag_error(a.err, kErrSeqLen);
-    return;
-  }
-  const int rows = (s1 - s0) * a.G;
-  const int r0 = blockIdx.z * kRowsPerCta;
-  if (r0 >= rows || gp == 0) return;  // (rows of ineligible members are ignored by the merge)
-  const int p_begin = static_cast<int>((static_cast<long long>(chunk) * gp) / a.chunks);
-  const int p_end = static_cast<int>((static_cast<long long>(chunk + 1) * gp) / a.chunks);
-  const int npages = p_end - p_begin;
-
-  // this warp's 8 query rows: row -> member m = row / G, head row j = row % G
-  uint32_t qf[NT][kSteps][2];
-  float acc[NT][kSteps][4];
-  float m_run[NT][2], l_run[NT][2];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int row = r0 + warp * 8 + nt * 8 + g8;
-    const bool live = row < rows;
-    const int b = s0 + (live ? row / a.G : 0), j = live ? row % a.G : 0;
-    const uint32_t *qw = reinterpret_cast<const uint32_t *>(a.q) +
-                         (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + j) * (D / 2);
-#pragma unroll
-    for (int ks = 0; ks < kSteps; ++ks) {
-      qf[nt][ks][0] = live ? __ldg(qw + ks * 8 + tig) : 0u;
-      qf[nt][ks][1] = live ? __ldg(qw + ks * 8 + 4 + tig) : 0u;
-    }
-#pragma unroll
-    for (int mt = 0; mt < kSteps; ++mt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
-    m_run[nt][0] = m_run[nt][1] = -INFINITY;
-    l_run[nt][0] = l_run[nt][1] = 0.f;
-  }
-
-  const uint32_t st0 = smem_u32(smem);
-  const uint32_t full0 = smem_u32(full), empty0 = smem_u32(empty);
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, kWarps);
-    }
-    mbar_init_fence();
-  }
-  __syncthreads();
-
-  const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
-  const uint64_t policy = l2_policy_evict_normal();
-  // producer: page k of the chunk into stage k % kStages (warp 0, lane 0)
-  auto produce = [&](int k) {
-    const int s = k % kStages;
-    const uint32_t bar = full0 + 8 * s;
-    const int pb = __ldg(bt + p_begin + k);
-    if (pb < 0 || pb >= a.num_blocks) {
-      flag_error(a.err, kErrBlockTable);
-      mbar_arrive(bar);  // completes the phase with no bytes; consumers see a zero page
+  [&] {
+    const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
+    const int h = blockIdx.y;
+    const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
+    int gp = __ldg(a.group_pages + g);
+    if (!group_ok(a, s0, s1, gp)) {
+      if (tid == 0) flag_error(a.err, kErrSeqLen);
       return;
     }
-    const int row = (pb * a.H_kv + h) * kPage;
-    const uint32_t dst = st0 + s * Pg::kStageBytes;
-    mbar_arrive_expect_tx(bar, Pg::kStageBytes);
-#pragma unroll
-    for (int hf = 0; hf < D / 64; ++hf) {
-      tma_load_3d(dst + hf * kPage * 128, &tmK, 0, hf, row, bar, policy);
-      tma_load_3d(dst + Pg::kPageBytes + hf * kPage * 128, &tmV, 0, hf, row, bar, policy);
-    }
-  };
-  if (tid == 0) {
-    prefetch_tensormap(&tmK);
-    prefetch_tensormap(&tmV);
-    for (int k = 0; k < kStages && k < npages; ++k) produce(k);
-  }
+    const int rows = (s1 - s0) * a.G;
+    const int r0 = blockIdx.z * kRowsPerCta;
+    if (r0 >= rows || gp == 0) return;  // (rows of ineligible members are ignored by the merge)
+    const int p_begin = static_cast<int>((static_cast<long long>(chunk) * gp) / a.chunks);
+    const int p_end = static_cast<int>((static_cast<long long>(chunk + 1) * gp) / a.chunks);
+    const int npages = p_end - p_begin;
 
-  // every warp has released stage s (use `ph`) before it is refilled with page kn
-  auto refill = [&](int s, uint32_t ph, int kn) {
-    if (kn >= npages) return;
-    if (!mbar_wait_bounded(empty0 + 8 * s, ph)) {
-      flag_error(a.err, kErrTimeout);
-      return;
-    }
-    produce(kn);
-  };
-
-  bool failed = false;
-  int k = 0;
-  while (k < npages) {
-    const bool two = k + 1 < npages;
-    const int sA = k % kStages, sB = (k + 1) % kStages;
-    const uint32_t phA = (k / kStages) & 1, phB = ((k + 1) / kStages) & 1;
-    bool ok = mbar_wait_bounded(full0 + 8 * sA, phA);
-    if (two) ok = ok && mbar_wait_bounded(full0 + 8 * sB, phB);
-    if (!__all_sync(0xffffffffu, ok)) {
-      if (lane == 0) flag_error(a.err, kErrTimeout);
-      failed = true;
-      break;
-    }
-    uint8_t *kA = smem + (size_t)sA * Pg::kStageBytes;
-    uint8_t *kB = smem + (size_t)sB * Pg::kStageBytes;
-    if (two)
-      tile_page2<D, NT, T>(smem_u32(kA), smem_u32(kA + Pg::kPageBytes), smem_u32(kB),
-                           smem_u32(kB + Pg::kPageBytes), a.scale_log2, lane, qf, acc, m_run, l_run);
-    else
-      tile_page<D, NT, T>(smem_u32(kA), smem_u32(kA + Pg::kPageBytes), kPage, a.scale_log2, lane,
-                          qf, acc, m_run, l_run);
-    __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(empty0 + 8 * sA);
-      if (two) mbar_arrive(empty0 + 8 * sB);
-    }
-    if (tid == 0) {
-      refill(sA, phA, k + kStages);
-      if (two) refill(sB, phB, k + 1 + kStages);
-    }
-    __syncwarp();
-    k += two ? 2 : 1;
-  }
-  if (failed) {
-    // let the copies in flight land before the CTA exits
-    for (int kk = k; kk < npages && kk < k + kStages; ++kk)
-      mbar_wait_bounded(full0 + 8 * (kk % kStages), (kk / kStages) & 1);
-    return;
-  }
-
-  // normalised partial (o, lse) of this chunk for each live row
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      float l = l_run[nt][i];
-      l += __shfl_xor_sync(0xffffffffu, l, 4);
-      l += __shfl_xor_sync(0xffffffffu, l, 8);
-      l += __shfl_xor_sync(0xffffffffu, l, 16);
-      const int row = r0 + warp * 8 + nt * 8 + 2 * tig + i;
-      if (row >= rows) continue;
-      const int b = s0 + row / a.G, j = row % a.G;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float lse = l > 0.f ? (m_run[nt][i] + fast_log2(l)) * kLn2 : -INFINITY;
-      const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + b) * a.G + j;
-      float *o = a.pre_o + idx * D;
-      const uint64_t keep = l2_policy_evict_last();  // read again by the merge
-#pragma unroll
-      for (int mt = 0; mt < kSteps; ++mt) {
-        st_keep(o + mt * 16 + g8, acc[nt][mt][i] * inv, keep);
-        st_keep(o + mt * 16 + 8 + g8, acc[nt][mt][2 + i] * inv, keep);
+    // this warp's 8 query rows: row -> member m = row / G, head row j = row % G
+    uint32_t qf[NT][kSteps][2];
+    float acc[NT][kSteps][4];
+    float m_run[NT][2], l_run[NT][2];
+  #pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int row = r0 + warp * 8 + nt * 8 + g8;
+      const bool live = row < rows;
+      const int b = s0 + (live ? row / a.G : 0), j = live ? row % a.G : 0;
+      const uint32_t *qw = reinterpret_cast<const uint32_t *>(a.q) +
+                           (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + j) * (D / 2);
+  #pragma unroll
+      for (int ks = 0; ks < kSteps; ++ks) {
+        qf[nt][ks][0] = live ? __ldg(qw + ks * 8 + tig) : 0u;
+        qf[nt][ks][1] = live ? __ldg(qw + ks * 8 + 4 + tig) : 0u;
       }
-      if (g8 == 0) st_keep(a.pre_lse + idx, lse, keep);
+  #pragma unroll
+      for (int mt = 0; mt < kSteps; ++mt)
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][mt][e] = 0.f;
+      m_run[nt][0] = m_run[nt][1] = -INFINITY;
+      l_run[nt][0] = l_run[nt][1] = 0.f;
     }
-  }
+
+    const uint32_t st0 = smem_u32(smem);
+    const uint32_t full0 = smem_u32(full), empty0 = smem_u32(empty);
+    if (tid == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(full0 + 8 * s, 1);
+        mbar_init(empty0 + 8 * s, kWarps);
+      }
+      mbar_init_fence();
+    }
+    __syncthreads();
+
+    const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
+    const uint64_t policy = l2_policy_evict_normal();
+    // producer: page k of the chunk into stage k % kStages (warp 0, lane 0)
+    auto produce = [&](int k) {
+      const int s = k % kStages;
+      const uint32_t bar = full0 + 8 * s;
+      const int pb = __ldg(bt + p_begin + k);
+      if (pb < 0 || pb >= a.num_blocks) {
+        flag_error(a.err, kErrBlockTable);
+        mbar_arrive(bar);  // completes the phase with no bytes; consumers see a zero page
+        return;
+      }
+      const int row = (pb * a.H_kv + h) * kPage;
+      const uint32_t dst = st0 + s * Pg::kStageBytes;
+      mbar_arrive_expect_tx(bar, Pg::kStageBytes);
+  #pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf) {
+        tma_load_3d(dst + hf * kPage * 128, &tmK, 0, hf, row, bar, policy);
+        tma_load_3d(dst + Pg::kPageBytes + hf * kPage * 128, &tmV, 0, hf, row, bar, policy);
+      }
+    };
+    if (tid == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      for (int k = 0; k < kStages && k < npages; ++k) produce(k);
+    }
+
+    // every warp has released stage s (use `ph`) before it is refilled with page kn
+    auto refill = [&](int s, uint32_t ph, int kn) {
+      if (kn >= npages) return;
+      if (!mbar_wait_bounded(empty0 + 8 * s, ph)) {
+        flag_error(a.err, kErrTimeout);
+        return;
+      }
+      produce(kn);
+    };
+
+    bool failed = false;
+    int k = 0;
+    while (k < npages) {
+      const bool two = k + 1 < npages;
+      const int sA = k % kStages, sB = (k + 1) % kStages;
+      const uint32_t phA = (k / kStages) & 1, phB = ((k + 1) / kStages) & 1;
+      bool ok = mbar_wait_bounded(full0 + 8 * sA, phA);
+      if (two) ok = ok && mbar_wait_bounded(full0 + 8 * sB, phB);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) flag_error(a.err, kErrTimeout);
+        failed = true;
+        break;
+      }
+      uint8_t *kA = smem + (size_t)sA * Pg::kStageBytes;
+      uint8_t *kB = smem + (size_t)sB * Pg::kStageBytes;
+      if (two)
+        tile_page2<D, NT, T>(smem_u32(kA), smem_u32(kA + Pg::kPageBytes), smem_u32(kB),
+                             smem_u32(kB + Pg::kPageBytes), a.scale_log2, lane, qf, acc, m_run, l_run);
+      else
+        tile_page<D, NT, T>(smem_u32(kA), smem_u32(kA + Pg::kPageBytes), kPage, a.scale_log2, lane,
+                            qf, acc, m_run, l_run);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(empty0 + 8 * sA);
+        if (two) mbar_arrive(empty0 + 8 * sB);
+      }
+      if (tid == 0) {
+        refill(sA, phA, k + kStages);
+        if (two) refill(sB, phB, k + 1 + kStages);
+      }
+      __syncwarp();
+      k += two ? 2 : 1;
+    }
+    if (failed) {
+      // let the copies in flight land before the CTA exits
+      for (int kk = k; kk < npages && kk < k + kStages; ++kk)
+        mbar_wait_bounded(full0 + 8 * (kk % kStages), (kk / kStages) & 1);
+      return;
+    }
+
+    // normalised partial (o, lse) of this chunk for each live row
+  #pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+  #pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        float l = l_run[nt][i];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        const int row = r0 + warp * 8 + nt * 8 + 2 * tig + i;
+        if (row >= rows) continue;
+        const int b = s0 + row / a.G, j = row % a.G;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float lse = l > 0.f ? (m_run[nt][i] + fast_log2(l)) * kLn2 : -INFINITY;
+        const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + b) * a.G + j;
+        float *o = a.pre_o + idx * D;
+        const uint64_t keep = l2_policy_evict_last();  // read again by the merge
+  #pragma unroll
+        for (int mt = 0; mt < kSteps; ++mt) {
+          st_keep(o + mt * 16 + g8, acc[nt][mt][i] * inv, keep);
+          st_keep(o + mt * 16 + 8 + g8, acc[nt][mt][2 + i] * inv, keep);
+        }
+        if (g8 == 0) st_keep(a.pre_lse + idx, lse, keep);
+      }
+    }
+  }();
+  prefix_exit(a);
 }
 
 // ------------------------------------------------------------------------
@@ -289,155 +378,155 @@ __global__ void __launch_bounds__(32 * kWarps, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g8 = lane >> 2, tig = lane & 3;
-  const int cap = a.maxb * kPage;
 
-  grid_dependency_wait();
+  // no wait for the decode launch before this pass (prefix_exit); every
+  // return of the body below still passes through prefix_exit
   grid_launch_dependents();
-
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) write_skip(a, cap);
-
-  const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
-  const int h = blockIdx.y;
-  const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
-  const int gp = __ldg(a.group_pages + g);
-  if (!group_ok(a, s0, s1, gp)) {
-    if (tid == 0) flag_error(a.err, kErrSeqLen);
-    return;
-  }
-  const int rows = (s1 - s0) * a.G;
-  const int r0 = blockIdx.z * kRowsPerCta;
-  if (r0 >= rows || gp == 0) return;  // (rows of ineligible members are ignored by the merge)
-  const int p_begin = static_cast<int>((static_cast<long long>(chunk) * gp) / a.chunks);
-  const int p_end = static_cast<int>((static_cast<long long>(chunk + 1) * gp) / a.chunks);
-  const int npages = p_end - p_begin;
-
-  // this warp's 8 query rows: row -> member m = row / G, head row j = row % G
-  uint32_t qf[1][kSteps][2];
-  float acc[1][kSteps][4];
-  float m_run[1][2], l_run[1][2];
-  {
-    const int row = r0 + warp * 8 + g8;
-    const bool live = row < rows;
-    const int b = s0 + (live ? row / a.G : 0), j = live ? row % a.G : 0;
-    const uint32_t *qw = reinterpret_cast<const uint32_t *>(a.q) +
-                         (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + j) * (D / 2);
-#pragma unroll
-    for (int ks = 0; ks < kSteps; ++ks) {
-      if (live) {
-        if constexpr (kInt4) q_words_q4<T>(qw, ks, tig, qf[0][ks][0], qf[0][ks][1]);
-        else q_words_q8<T>(qw, ks, tig, qf[0][ks][0], qf[0][ks][1]);
-      } else {
-        qf[0][ks][0] = qf[0][ks][1] = 0u;
-      }
-    }
-#pragma unroll
-    for (int mt = 0; mt < kSteps; ++mt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[0][mt][e] = 0.f;
-    m_run[0][0] = m_run[0][1] = -INFINITY;
-    l_run[0][0] = l_run[0][1] = 0.f;
-  }
-
-  const uint32_t st0 = smem_u32(smem);
-  const uint32_t full0 = smem_u32(full), empty0 = smem_u32(empty);
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, kWarps);
-    }
-    mbar_init_fence();
-  }
-  __syncthreads();
-
-  const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
-  const uint64_t policy = l2_policy_evict_normal();
-  constexpr int kG = D / 32;
-  // producer: page k of the chunk into stage k % kStages (warp 0, lane 0)
-  auto produce = [&](int k) {
-    const int s = k % kStages;
-    const uint32_t bar = full0 + 8 * s;
-    const int pb = __ldg(bt + p_begin + k);
-    if (pb < 0 || pb >= a.num_blocks) {
-      flag_error(a.err, kErrBlockTable);
-      mbar_arrive(bar);  // completes the phase with no bytes; consumers skip the page
+  [&] {
+    const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
+    const int h = blockIdx.y;
+    const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
+    const int gp = __ldg(a.group_pages + g);
+    if (!group_ok(a, s0, s1, gp)) {
+      if (tid == 0) flag_error(a.err, kErrSeqLen);
       return;
     }
-    const int row = (pb * a.H_kv + h) * kPage;
-    const uint32_t dst = st0 + s * Pg::kStageBytes;
-    mbar_arrive_expect_tx(bar, 2 * Pg::kCodePage + 2 * Pg::kScalePage);
-    tma_load_2d(dst, &tmK, 0, row, bar, policy);
-    tma_load_2d(dst + Pg::kCodePage, &tmV, 0, row, bar, policy);
-    bulk_load(dst + 2 * Pg::kCodePage, a.k_scale + static_cast<size_t>(row) * kG, Pg::kScalePage, bar);
-    bulk_load(dst + 2 * Pg::kCodePage + Pg::kScalePage, a.v_scale + static_cast<size_t>(row) * kG,
-              Pg::kScalePage, bar);
-  };
-  if (tid == 0) {
-    prefetch_tensormap(&tmK);
-    prefetch_tensormap(&tmV);
-    for (int k = 0; k < kStages && k < npages; ++k) produce(k);
-  }
+    const int rows = (s1 - s0) * a.G;
+    const int r0 = blockIdx.z * kRowsPerCta;
+    if (r0 >= rows || gp == 0) return;  // (rows of ineligible members are ignored by the merge)
+    const int p_begin = static_cast<int>((static_cast<long long>(chunk) * gp) / a.chunks);
+    const int p_end = static_cast<int>((static_cast<long long>(chunk + 1) * gp) / a.chunks);
+    const int npages = p_end - p_begin;
 
-  bool failed = false;
-  int k = 0;
-  for (; k < npages; ++k) {
-    const int s = k % kStages;
-    const uint32_t ph = (k / kStages) & 1;
-    const bool ok = mbar_wait_bounded(full0 + 8 * s, ph);
-    if (!__all_sync(0xffffffffu, ok)) {
-      if (lane == 0) flag_error(a.err, kErrTimeout);
-      failed = true;
-      break;
+    // this warp's 8 query rows: row -> member m = row / G, head row j = row % G
+    uint32_t qf[1][kSteps][2];
+    float acc[1][kSteps][4];
+    float m_run[1][2], l_run[1][2];
+    {
+      const int row = r0 + warp * 8 + g8;
+      const bool live = row < rows;
+      const int b = s0 + (live ? row / a.G : 0), j = live ? row % a.G : 0;
+      const uint32_t *qw = reinterpret_cast<const uint32_t *>(a.q) +
+                           (static_cast<size_t>(b) * a.H_q + static_cast<size_t>(h) * a.G + j) * (D / 2);
+  #pragma unroll
+      for (int ks = 0; ks < kSteps; ++ks) {
+        if (live) {
+          if constexpr (kInt4) q_words_q4<T>(qw, ks, tig, qf[0][ks][0], qf[0][ks][1]);
+          else q_words_q8<T>(qw, ks, tig, qf[0][ks][0], qf[0][ks][1]);
+        } else {
+          qf[0][ks][0] = qf[0][ks][1] = 0u;
+        }
+      }
+  #pragma unroll
+      for (int mt = 0; mt < kSteps; ++mt)
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) acc[0][mt][e] = 0.f;
+      m_run[0][0] = m_run[0][1] = -INFINITY;
+      l_run[0][0] = l_run[0][1] = 0.f;
     }
-    const int pb = __ldg(bt + p_begin + k);
-    if (pb >= 0 && pb < a.num_blocks) {  // (a page outside the pool was flagged and not copied)
-      uint8_t *st = smem + (size_t)s * Pg::kStageBytes;
-      const float *ks = reinterpret_cast<const float *>(st + 2 * Pg::kCodePage);
-      if constexpr (kInt4)
-        tile_page_q4<D, 1>(smem_u32(st), smem_u32(st + Pg::kCodePage), ks, ks + kPage * kG, kPage,
-                           a.scale_log2, lane, qf, acc, m_run, l_run);
-      else
-        tile_page_q8<D, 1, kFmt>(smem_u32(st), smem_u32(st + Pg::kCodePage), ks, ks + kPage * kG,
-                                 kPage, a.scale_log2, lane, qf, acc, m_run, l_run);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8 * s);
-    if (tid == 0 && k + kStages < npages) {
-      // every warp has released stage s before it is refilled
-      if (mbar_wait_bounded(empty0 + 8 * s, ph)) produce(k + kStages);
-      else flag_error(a.err, kErrTimeout);
-    }
-  }
-  if (failed) {
-    // let the copies in flight land before the CTA exits
-    for (int kk = k; kk < npages && kk < k + kStages; ++kk)
-      mbar_wait_bounded(full0 + 8 * (kk % kStages), (kk / kStages) & 1);
-    return;
-  }
 
-  // normalised partial (o, lse) of this chunk for each live row
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    float l = l_run[0][i];
-    l += __shfl_xor_sync(0xffffffffu, l, 4);
-    l += __shfl_xor_sync(0xffffffffu, l, 8);
-    l += __shfl_xor_sync(0xffffffffu, l, 16);
-    const int row = r0 + warp * 8 + 2 * tig + i;
-    if (row >= rows) continue;
-    const int b = s0 + row / a.G, j = row % a.G;
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    const float lse = l > 0.f ? (m_run[0][i] + fast_log2(l)) * kLn2 : -INFINITY;
-    const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + b) * a.G + j;
-    float *o = a.pre_o + idx * D;
-    const uint64_t keep = l2_policy_evict_last();  // read again by the merge
-#pragma unroll
-    for (int mt = 0; mt < kSteps; ++mt) {
-      const int c0 = kInt4 ? dim_q4(mt, i, g8) : dim_q8(mt, i, g8);
-      const int c2 = kInt4 ? dim_q4(mt, 2 + i, g8) : dim_q8(mt, 2 + i, g8);
-      st_keep(o + c0, acc[0][mt][i] * inv, keep);
-      st_keep(o + c2, acc[0][mt][2 + i] * inv, keep);
+    const uint32_t st0 = smem_u32(smem);
+    const uint32_t full0 = smem_u32(full), empty0 = smem_u32(empty);
+    if (tid == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(full0 + 8 * s, 1);
+        mbar_init(empty0 + 8 * s, kWarps);
+      }
+      mbar_init_fence();
     }
-    if (g8 == 0) st_keep(a.pre_lse + idx, lse, keep);
-  }
+    __syncthreads();
+
+    const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
+    const uint64_t policy = l2_policy_evict_normal();
+    constexpr int kG = D / 32;
+    // producer: page k of the chunk into stage k % kStages (warp 0, lane 0)
+    auto produce = [&](int k) {
+      const int s = k % kStages;
+      const uint32_t bar = full0 + 8 * s;
+      const int pb = __ldg(bt + p_begin + k);
+      if (pb < 0 || pb >= a.num_blocks) {
+        flag_error(a.err, kErrBlockTable);
+        mbar_arrive(bar);  // completes the phase with no bytes; consumers skip the page
+        return;
+      }
+      const int row = (pb * a.H_kv + h) * kPage;
+      const uint32_t dst = st0 + s * Pg::kStageBytes;
+      mbar_arrive_expect_tx(bar, 2 * Pg::kCodePage + 2 * Pg::kScalePage);
+      tma_load_2d(dst, &tmK, 0, row, bar, policy);
+      tma_load_2d(dst + Pg::kCodePage, &tmV, 0, row, bar, policy);
+      bulk_load(dst + 2 * Pg::kCodePage, a.k_scale + static_cast<size_t>(row) * kG, Pg::kScalePage, bar);
+      bulk_load(dst + 2 * Pg::kCodePage + Pg::kScalePage, a.v_scale + static_cast<size_t>(row) * kG,
+                Pg::kScalePage, bar);
+    };
+    if (tid == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      for (int k = 0; k < kStages && k < npages; ++k) produce(k);
+    }
+
+    bool failed = false;
+    int k = 0;
+    for (; k < npages; ++k) {
+      const int s = k % kStages;
+      const uint32_t ph = (k / kStages) & 1;
+      const bool ok = mbar_wait_bounded(full0 + 8 * s, ph);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) flag_error(a.err, kErrTimeout);
+        failed = true;
+        break;
+      }
+      const int pb = __ldg(bt + p_begin + k);
+      if (pb >= 0 && pb < a.num_blocks) {  // (a page outside the pool was flagged and not copied)
+        uint8_t *st = smem + (size_t)s * Pg::kStageBytes;
+        const float *ks = reinterpret_cast<const float *>(st + 2 * Pg::kCodePage);
+        if constexpr (kInt4)
+          tile_page_q4<D, 1>(smem_u32(st), smem_u32(st + Pg::kCodePage), ks, ks + kPage * kG, kPage,
+                             a.scale_log2, lane, qf, acc, m_run, l_run);
+        else
+          tile_page_q8<D, 1, kFmt>(smem_u32(st), smem_u32(st + Pg::kCodePage), ks, ks + kPage * kG,
+                                   kPage, a.scale_log2, lane, qf, acc, m_run, l_run);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * s);
+      if (tid == 0 && k + kStages < npages) {
+        // every warp has released stage s before it is refilled
+        if (mbar_wait_bounded(empty0 + 8 * s, ph)) produce(k + kStages);
+        else flag_error(a.err, kErrTimeout);
+      }
+    }
+    if (failed) {
+      // let the copies in flight land before the CTA exits
+      for (int kk = k; kk < npages && kk < k + kStages; ++kk)
+        mbar_wait_bounded(full0 + 8 * (kk % kStages), (kk / kStages) & 1);
+      return;
+    }
+
+    // normalised partial (o, lse) of this chunk for each live row
+  #pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float l = l_run[0][i];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      const int row = r0 + warp * 8 + 2 * tig + i;
+      if (row >= rows) continue;
+      const int b = s0 + row / a.G, j = row % a.G;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float lse = l > 0.f ? (m_run[0][i] + fast_log2(l)) * kLn2 : -INFINITY;
+      const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + b) * a.G + j;
+      float *o = a.pre_o + idx * D;
+      const uint64_t keep = l2_policy_evict_last();  // read again by the merge
+  #pragma unroll
+      for (int mt = 0; mt < kSteps; ++mt) {
+        const int c0 = kInt4 ? dim_q4(mt, i, g8) : dim_q8(mt, i, g8);
+        const int c2 = kInt4 ? dim_q4(mt, 2 + i, g8) : dim_q8(mt, 2 + i, g8);
+        st_keep(o + c0, acc[0][mt][i] * inv, keep);
+        st_keep(o + c2, acc[0][mt][2 + i] * inv, keep);
+      }
+      if (g8 == 0) st_keep(a.pre_lse + idx, lse, keep);
+    }
+  }();
+  prefix_exit(a);
 }
 
 // ------------------------------------------------------------------------
@@ -745,231 +834,232 @@ __global__ void __launch_bounds__(32 * kTcWarps, 2)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kTcBars);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cap = a.maxb * kPage;
 
-  grid_dependency_wait();
+  // no wait for the decode launch before this pass (prefix_exit); every
+  // return of the body below still passes through prefix_exit
   grid_launch_dependents();
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) write_skip(a, cap);
-
-  const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
-  const int h = blockIdx.y;
-  const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
-  const int gp = __ldg(a.group_pages + g);
-  if (!group_ok(a, s0, s1, gp)) {
-    if (tid == 0) flag_error(a.err, kErrSeqLen);
-    return;
-  }
-  const int rows = (s1 - s0) * a.G;
-  const int r0 = blockIdx.z * kRowsPerCta;
-  if (r0 >= rows || gp == 0) return;
-  const int p_begin = static_cast<int>((static_cast<long long>(chunk) * gp) / a.chunks);
-  const int p_end = static_cast<int>((static_cast<long long>(chunk + 1) * gp) / a.chunks);
-  const int nsteps = (p_end - p_begin + kTcPages - 1) / kTcPages;
-  if (nsteps == 0) {  // an empty chunk leaves empty partials
-    for (int r = tid; r < kRowsPerCta; r += blockDim.x) {
-      const int row = r0 + r;
-      if (row >= rows) continue;
-      const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + s0 + row / a.G) * a.G +
-                         row % a.G;
-      for (int c = 0; c < D; ++c) a.pre_o[idx * D + c] = 0.f;
-      a.pre_lse[idx] = -INFINITY;
+  [&] {
+    const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
+    const int h = blockIdx.y;
+    const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
+    const int gp = __ldg(a.group_pages + g);
+    if (!group_ok(a, s0, s1, gp)) {
+      if (tid == 0) flag_error(a.err, kErrSeqLen);
+      return;
     }
-    return;
-  }
-  const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
-  auto step_pages = [&](int j) { return min(kTcPages, p_end - (p_begin + j * kTcPages)); };
-
-  const uint32_t q0 = smem_u32(qs), ring0 = smem_u32(ring), bar0 = smem_u32(bars);
-  // K and V halves of a stage have their own barriers: K is released as soon
-  // as QK^T has read it, V after the PV product
-  auto FULL_K = [&](int s) { return bar0 + 8 * s; };
-  auto FULL_V = [&](int s) { return bar0 + 8 * (kTcStages + s); };
-  auto EMPTY_K = [&](int s) { return bar0 + 8 * (2 * kTcStages + s); };
-  auto EMPTY_V = [&](int s) { return bar0 + 8 * (3 * kTcStages + s); };
-  const uint32_t S_FULL = bar0 + 8 * (4 * kTcStages);  // + 8 * buffer
-  const uint32_t P_FULL = S_FULL + 16;                 // + 8 * buffer
-  const uint32_t O_DONE = S_FULL + 32, Q_FULL = S_FULL + 40, DRAIN = S_FULL + 48;
-
-  if (warp == 0) {
-    __syncwarp();
-    tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tc::tmem_relinquish();
-  }
-  if (tid == 32) {
-    for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(FULL_K(s), 1);
-      mbar_init(FULL_V(s), 1);
-      mbar_init(EMPTY_K(s), 1);
-      mbar_init(EMPTY_V(s), 1);
+    const int rows = (s1 - s0) * a.G;
+    const int r0 = blockIdx.z * kRowsPerCta;
+    if (r0 >= rows || gp == 0) return;
+    const int p_begin = static_cast<int>((static_cast<long long>(chunk) * gp) / a.chunks);
+    const int p_end = static_cast<int>((static_cast<long long>(chunk + 1) * gp) / a.chunks);
+    const int nsteps = (p_end - p_begin + kTcPages - 1) / kTcPages;
+    if (nsteps == 0) {  // an empty chunk leaves empty partials
+      for (int r = tid; r < kRowsPerCta; r += blockDim.x) {
+        const int row = r0 + r;
+        if (row >= rows) continue;
+        const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + s0 + row / a.G) * a.G +
+                           row % a.G;
+        for (int c = 0; c < D; ++c) a.pre_o[idx * D + c] = 0.f;
+        a.pre_lse[idx] = -INFINITY;
+      }
+      return;
     }
-    mbar_init(S_FULL, 1);
-    mbar_init(S_FULL + 8, 1);
-    mbar_init(P_FULL, 4);
-    mbar_init(P_FULL + 8, 4);
-    mbar_init(O_DONE, 1);
-    mbar_init(Q_FULL, 4);
-    mbar_init(DRAIN, 1);
-    mbar_init_fence();
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tbase = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+    const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
+    auto step_pages = [&](int j) { return min(kTcPages, p_end - (p_begin + j * kTcPages)); };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      const uint64_t policy = l2_policy_evict_normal();
-      int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < nsteps; ++j) {
-        const int s = j % kTcStages;
-        const uint32_t rel = ((j / kTcStages) - 1) & 1;  // phase of step j - kTcStages
-        const int p0 = p_begin + j * kTcPages, np = step_pages(j);
-        int prow[kTcPages];
-        int good = 0;
-#pragma unroll
-        for (int p = 0; p < kTcPages; ++p) {
-          prow[p] = -1;
-          if (p < np) {
-            const int pb = __ldg(bt + p0 + p);
-            if (pb >= 0 && pb < a.num_blocks) {
-              prow[p] = (pb * a.H_kv + h) * kPage;
-              ++good;
-            } else {
-              flag_error(a.err, kErrBlockTable);
+    const uint32_t q0 = smem_u32(qs), ring0 = smem_u32(ring), bar0 = smem_u32(bars);
+    // K and V halves of a stage have their own barriers: K is released as soon
+    // as QK^T has read it, V after the PV product
+    auto FULL_K = [&](int s) { return bar0 + 8 * s; };
+    auto FULL_V = [&](int s) { return bar0 + 8 * (kTcStages + s); };
+    auto EMPTY_K = [&](int s) { return bar0 + 8 * (2 * kTcStages + s); };
+    auto EMPTY_V = [&](int s) { return bar0 + 8 * (3 * kTcStages + s); };
+    const uint32_t S_FULL = bar0 + 8 * (4 * kTcStages);  // + 8 * buffer
+    const uint32_t P_FULL = S_FULL + 16;                 // + 8 * buffer
+    const uint32_t O_DONE = S_FULL + 32, Q_FULL = S_FULL + 40, DRAIN = S_FULL + 48;
+
+    if (warp == 0) {
+      __syncwarp();
+      tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+      tc::tmem_relinquish();
+    }
+    if (tid == 32) {
+      for (int s = 0; s < kTcStages; ++s) {
+        mbar_init(FULL_K(s), 1);
+        mbar_init(FULL_V(s), 1);
+        mbar_init(EMPTY_K(s), 1);
+        mbar_init(EMPTY_V(s), 1);
+      }
+      mbar_init(S_FULL, 1);
+      mbar_init(S_FULL + 8, 1);
+      mbar_init(P_FULL, 4);
+      mbar_init(P_FULL + 8, 4);
+      mbar_init(O_DONE, 1);
+      mbar_init(Q_FULL, 4);
+      mbar_init(DRAIN, 1);
+      mbar_init_fence();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        const uint64_t policy = l2_policy_evict_normal();
+        int issued_k = 0, issued_v = 0;
+        for (int j = 0; j < nsteps; ++j) {
+          const int s = j % kTcStages;
+          const uint32_t rel = ((j / kTcStages) - 1) & 1;  // phase of step j - kTcStages
+          const int p0 = p_begin + j * kTcPages, np = step_pages(j);
+          int prow[kTcPages];
+          int good = 0;
+  #pragma unroll
+          for (int p = 0; p < kTcPages; ++p) {
+            prow[p] = -1;
+            if (p < np) {
+              const int pb = __ldg(bt + p0 + p);
+              if (pb >= 0 && pb < a.num_blocks) {
+                prow[p] = (pb * a.H_kv + h) * kPage;
+                ++good;
+              } else {
+                flag_error(a.err, kErrBlockTable);
+              }
             }
           }
+          const uint32_t st = ring0 + s * kTcStage;
+          const uint32_t bytes = static_cast<uint32_t>(good) * 2 * kPage * 128;
+          // K of step j, once QK^T of step j - kTcStages has read the stage's K
+          if (j >= kTcStages && !mbar_wait_bounded(EMPTY_K(s), rel)) {
+            flag_error(a.err, kErrTimeout);
+            break;
+          }
+          mbar_arrive_expect_tx(FULL_K(s), bytes);
+  #pragma unroll
+          for (int p = 0; p < kTcPages; ++p) {
+            if (prow[p] < 0) continue;
+            tma_load_3d(st + p * kPage * 128, &tmK, 0, 0, prow[p], FULL_K(s), policy);
+            tma_load_3d(st + kTcHalf + p * kPage * 128, &tmK, 0, 1, prow[p], FULL_K(s), policy);
+          }
+          issued_k = j + 1;
+          // V of step j, once the PV product of step j - kTcStages has read its V
+          if (j >= kTcStages && !mbar_wait_bounded(EMPTY_V(s), rel)) {
+            flag_error(a.err, kErrTimeout);
+            break;
+          }
+          mbar_arrive_expect_tx(FULL_V(s), bytes);
+  #pragma unroll
+          for (int p = 0; p < kTcPages; ++p) {
+            if (prow[p] < 0) continue;
+            tma_load_3d(st + 2 * kTcHalf + p * kPage * 128, &tmV, 0, 0, prow[p], FULL_V(s), policy);
+            tma_load_3d(st + 3 * kTcHalf + p * kPage * 128, &tmV, 0, 1, prow[p], FULL_V(s), policy);
+          }
+          issued_v = j + 1;
         }
-        const uint32_t st = ring0 + s * kTcStage;
-        const uint32_t bytes = static_cast<uint32_t>(good) * 2 * kPage * 128;
-        // K of step j, once QK^T of step j - kTcStages has read the stage's K
-        if (j >= kTcStages && !mbar_wait_bounded(EMPTY_K(s), rel)) {
-          flag_error(a.err, kErrTimeout);
-          break;
-        }
-        mbar_arrive_expect_tx(FULL_K(s), bytes);
-#pragma unroll
-        for (int p = 0; p < kTcPages; ++p) {
-          if (prow[p] < 0) continue;
-          tma_load_3d(st + p * kPage * 128, &tmK, 0, 0, prow[p], FULL_K(s), policy);
-          tma_load_3d(st + kTcHalf + p * kPage * 128, &tmK, 0, 1, prow[p], FULL_K(s), policy);
-        }
-        issued_k = j + 1;
-        // V of step j, once the PV product of step j - kTcStages has read its V
-        if (j >= kTcStages && !mbar_wait_bounded(EMPTY_V(s), rel)) {
-          flag_error(a.err, kErrTimeout);
-          break;
-        }
-        mbar_arrive_expect_tx(FULL_V(s), bytes);
-#pragma unroll
-        for (int p = 0; p < kTcPages; ++p) {
-          if (prow[p] < 0) continue;
-          tma_load_3d(st + 2 * kTcHalf + p * kPage * 128, &tmV, 0, 0, prow[p], FULL_V(s), policy);
-          tma_load_3d(st + 3 * kTcHalf + p * kPage * 128, &tmV, 0, 1, prow[p], FULL_V(s), policy);
-        }
-        issued_v = j + 1;
+        // the copies of the last stages have landed before the CTA exits
+        for (int j = max(0, issued_k - kTcStages); j < issued_k; ++j)
+          mbar_wait_bounded(FULL_K(j % kTcStages), (j / kTcStages) & 1);
+        for (int j = max(0, issued_v - kTcStages); j < issued_v; ++j)
+          mbar_wait_bounded(FULL_V(j % kTcStages), (j / kTcStages) & 1);
       }
-      // the copies of the last stages have landed before the CTA exits
-      for (int j = max(0, issued_k - kTcStages); j < issued_k; ++j)
-        mbar_wait_bounded(FULL_K(j % kTcStages), (j / kTcStages) & 1);
-      for (int j = max(0, issued_v - kTcStages); j < issued_v; ++j)
-        mbar_wait_bounded(FULL_V(j % kTcStages), (j / kTcStages) & 1);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t fmt = kBf16 ? 1u : 0u;
-      bool ok = mbar_wait_bounded(Q_FULL, 0);
-      tc::fence_after_sync();
-      bool o_started = false;
-      auto issue_qk = [&](int j) {
-        const int b = j & 1;
-        const uint32_t idesc = tc::idesc_f16(fmt, static_cast<uint32_t>(step_pages(j) * kPage), false);
-        const uint32_t kst = ring0 + (j % kTcStages) * kTcStage;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t kaddr = kst + (k >> 2) * kTcHalf + (k & 3) * 32;
-          const uint32_t qaddr = q0 + (k >> 2) * (kTcQBytes / 2) + (k & 3) * 32;
-          tc::mma_ss(tbase + kColS + b * kTcTok, tc::smem_desc(qaddr, 16, 1024),
-                     tc::smem_desc(kaddr, 16, 1024), idesc, k > 0);
-        }
-        tc::commit(EMPTY_K(j % kTcStages));
-        tc::commit(S_FULL + 8 * b);
-      };
-      uint32_t pv_mask0 = 0u, pv_mask1 = 0u;  // loaded one step before the PV product uses it
-      auto issue_pv = [&](int j) {
-        const int b = j & 1, s = j % kTcStages;
-        const int np = step_pages(j);
-        const uint32_t mask = (j & 1) ? pv_mask1 : pv_mask0;
-        const uint32_t idesc = tc::idesc_f16(fmt, D, true);
-        const uint32_t vst = ring0 + s * kTcStage + 2 * kTcHalf;
-        for (int kk = 0; kk < np; ++kk) {
-          if (!((mask >> kk) & 1u)) continue;  // (its scores are masked; its stage bytes are stale)
-          const uint64_t vd = tc::smem_desc(vst + kk * kPage * 128, kTcHalf, 1024);
-          const uint32_t pa = tbase + kColS + b * kTcTok + kk * 8;  // P over S; remainder at +32
-          tc::mma_ts(tbase + kColO, pa, vd, idesc, o_started);
-          o_started = true;
-          if (kBf16) tc::mma_ts(tbase + kColO, pa + kTcTok / 2, vd, idesc, true);
-        }
-        tc::commit(EMPTY_V(s));
-        tc::commit(O_DONE);
-      };
-      // the PV product of step j waits for its probabilities and its V pages
-      auto wait_pv = [&](int j) {
-        return mbar_wait_bounded(P_FULL + 8 * (j & 1), (j >> 1) & 1) &&
-               mbar_wait_bounded(FULL_V(j % kTcStages), (j / kTcStages) & 1);
-      };
-      StepPages ahead;  // the block-table entries of step j, loaded during step j - 1
-      ahead.load(bt, p_begin, p_end, nsteps, 0);
-      for (int j = 0; ok && j < nsteps; ++j) {
-        if (j & 1) pv_mask1 = ahead.mask(a);
-        else pv_mask0 = ahead.mask(a);
-        ahead.load(bt, p_begin, p_end, nsteps, j + 1);
-        if (!mbar_wait_bounded(FULL_K(j % kTcStages), (j / kTcStages) & 1)) {
-          ok = false;
-          break;
-        }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t fmt = kBf16 ? 1u : 0u;
+        bool ok = mbar_wait_bounded(Q_FULL, 0);
         tc::fence_after_sync();
-        issue_qk(j);
-        if (j >= 1) {
-          if (!wait_pv(j - 1)) {
+        bool o_started = false;
+        auto issue_qk = [&](int j) {
+          const int b = j & 1;
+          const uint32_t idesc = tc::idesc_f16(fmt, static_cast<uint32_t>(step_pages(j) * kPage), false);
+          const uint32_t kst = ring0 + (j % kTcStages) * kTcStage;
+  #pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t kaddr = kst + (k >> 2) * kTcHalf + (k & 3) * 32;
+            const uint32_t qaddr = q0 + (k >> 2) * (kTcQBytes / 2) + (k & 3) * 32;
+            tc::mma_ss(tbase + kColS + b * kTcTok, tc::smem_desc(qaddr, 16, 1024),
+                       tc::smem_desc(kaddr, 16, 1024), idesc, k > 0);
+          }
+          tc::commit(EMPTY_K(j % kTcStages));
+          tc::commit(S_FULL + 8 * b);
+        };
+        uint32_t pv_mask0 = 0u, pv_mask1 = 0u;  // loaded one step before the PV product uses it
+        auto issue_pv = [&](int j) {
+          const int b = j & 1, s = j % kTcStages;
+          const int np = step_pages(j);
+          const uint32_t mask = (j & 1) ? pv_mask1 : pv_mask0;
+          const uint32_t idesc = tc::idesc_f16(fmt, D, true);
+          const uint32_t vst = ring0 + s * kTcStage + 2 * kTcHalf;
+          for (int kk = 0; kk < np; ++kk) {
+            if (!((mask >> kk) & 1u)) continue;  // (its scores are masked; its stage bytes are stale)
+            const uint64_t vd = tc::smem_desc(vst + kk * kPage * 128, kTcHalf, 1024);
+            const uint32_t pa = tbase + kColS + b * kTcTok + kk * 8;  // P over S; remainder at +32
+            tc::mma_ts(tbase + kColO, pa, vd, idesc, o_started);
+            o_started = true;
+            if (kBf16) tc::mma_ts(tbase + kColO, pa + kTcTok / 2, vd, idesc, true);
+          }
+          tc::commit(EMPTY_V(s));
+          tc::commit(O_DONE);
+        };
+        // the PV product of step j waits for its probabilities and its V pages
+        auto wait_pv = [&](int j) {
+          return mbar_wait_bounded(P_FULL + 8 * (j & 1), (j >> 1) & 1) &&
+                 mbar_wait_bounded(FULL_V(j % kTcStages), (j / kTcStages) & 1);
+        };
+        StepPages ahead;  // the block-table entries of step j, loaded during step j - 1
+        ahead.load(bt, p_begin, p_end, nsteps, 0);
+        for (int j = 0; ok && j < nsteps; ++j) {
+          if (j & 1) pv_mask1 = ahead.mask(a);
+          else pv_mask0 = ahead.mask(a);
+          ahead.load(bt, p_begin, p_end, nsteps, j + 1);
+          if (!mbar_wait_bounded(FULL_K(j % kTcStages), (j / kTcStages) & 1)) {
             ok = false;
             break;
           }
           tc::fence_after_sync();
-          issue_pv(j - 1);
+          issue_qk(j);
+          if (j >= 1) {
+            if (!wait_pv(j - 1)) {
+              ok = false;
+              break;
+            }
+            tc::fence_after_sync();
+            issue_pv(j - 1);
+          }
         }
-      }
-      if (ok) {
-        const int j = nsteps - 1;
-        if (wait_pv(j)) {
-          tc::fence_after_sync();
-          issue_pv(j);
-        } else {
-          ok = false;
+        if (ok) {
+          const int j = nsteps - 1;
+          if (wait_pv(j)) {
+            tc::fence_after_sync();
+            issue_pv(j);
+          } else {
+            ok = false;
+          }
         }
+        if (!ok) flag_error(a.err, kErrTimeout);
+        // every MMA issued here completes before TMEM is released
+        tc::commit(DRAIN);
+        mbar_wait_bounded(DRAIN, 0);
       }
-      if (!ok) flag_error(a.err, kErrTimeout);
-      // every MMA issued here completes before TMEM is released
-      tc::commit(DRAIN);
-      mbar_wait_bounded(DRAIN, 0);
+    } else {
+      // ------------------------------------------------------------ softmax
+      tc_softmax_role<T>(a, qs, tbase, S_FULL, P_FULL, O_DONE, Q_FULL, warp, lane, r0, rows, s0, h,
+                         chunk, nsteps, bt, p_begin, p_end);
     }
-  } else {
-    // ------------------------------------------------------------ softmax
-    tc_softmax_role<T>(a, qs, tbase, S_FULL, P_FULL, O_DONE, Q_FULL, warp, lane, r0, rows, s0, h,
-                       chunk, nsteps, bt, p_begin, p_end);
-  }
 
-  // release TMEM once every role is done with it
-  tc::fence_before_sync();
-  __syncthreads();
-  if (warp == 0) {
-    __syncwarp();
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tbase, kTmemCols);
-  }
+    // release TMEM once every role is done with it
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+      __syncwarp();
+      tc::fence_after_sync();
+      tc::tmem_dealloc(tbase, kTmemCols);
+    }
+  }();
+  prefix_exit(a);
 }
 
 // ------------------------------------------------------------------------
@@ -1156,267 +1246,308 @@ __global__ void __launch_bounds__(32 * kTqWarps, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + Gq::kBars);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cap = a.maxb * kPage;
 
-  grid_dependency_wait();
+  // no wait for the decode launch before this pass (prefix_exit); every
+  // return of the body below still passes through prefix_exit
   grid_launch_dependents();
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) write_skip(a, cap);
-
-  const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
-  const int h = blockIdx.y;
-  const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
-  const int gp = __ldg(a.group_pages + g);
-  if (!group_ok(a, s0, s1, gp)) {
-    if (tid == 0) flag_error(a.err, kErrSeqLen);
-    return;
-  }
-  const int rows = (s1 - s0) * a.G;
-  const int r0 = blockIdx.z * kRowsPerCta;
-  if (r0 >= rows || gp == 0) return;
-  const int p_begin = static_cast<int>((static_cast<long long>(chunk) * gp) / a.chunks);
-  const int p_end = static_cast<int>((static_cast<long long>(chunk + 1) * gp) / a.chunks);
-  const int nsteps = (p_end - p_begin + kTcPages - 1) / kTcPages;
-  if (nsteps == 0) {  // an empty chunk leaves empty partials
-    for (int r = tid; r < kRowsPerCta; r += blockDim.x) {
-      const int row = r0 + r;
-      if (row >= rows) continue;
-      const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + s0 + row / a.G) * a.G +
-                         row % a.G;
-      for (int c = 0; c < D; ++c) a.pre_o[idx * D + c] = 0.f;
-      a.pre_lse[idx] = -INFINITY;
+  [&] {
+    const int g = blockIdx.x / a.chunks, chunk = blockIdx.x - g * a.chunks;
+    const int h = blockIdx.y;
+    const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
+    const int gp = __ldg(a.group_pages + g);
+    if (!group_ok(a, s0, s1, gp)) {
+      if (tid == 0) flag_error(a.err, kErrSeqLen);
+      return;
     }
-    return;
-  }
-  const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
-  auto step_pages = [&](int j) { return min(kTcPages, p_end - (p_begin + j * kTcPages)); };
-
-  const uint32_t tiles0 = smem_u32(tiles), codes0 = smem_u32(codes);
-  const uint32_t scl0 = smem_u32(scl), bar0 = smem_u32(bars);
-  // kv = 0: K, 1: V; c: code stage (kTqCodeStages), s: tile stage (kTcStages)
-  constexpr int kT0 = 4 * kTqCodeStages;  // first tile barrier
-  auto CFULL = [&](int kv, int c) { return bar0 + 8 * (kv * kTqCodeStages + c); };
-  auto CFREE = [&](int kv, int c) { return bar0 + 8 * ((2 + kv) * kTqCodeStages + c); };
-  auto TFULL = [&](int kv, int s) { return bar0 + 8 * (kT0 + kv * kTcStages + s); };
-  auto TFREE = [&](int kv, int s) { return bar0 + 8 * (kT0 + (2 + kv) * kTcStages + s); };
-  const uint32_t S_FULL = bar0 + 8 * (kT0 + 4 * kTcStages);  // + 8 * buffer
-  const uint32_t P_FULL = S_FULL + 16;                 // + 8 * buffer
-  const uint32_t O_DONE = S_FULL + 32, Q_FULL = S_FULL + 40, DRAIN = S_FULL + 48;
-
-  if (warp == 0) {
-    __syncwarp();
-    tc::tmem_alloc(smem_u32(tmem_slot), kTmemColsQ);
-    tc::tmem_relinquish();
-  }
-  if (tid == 32) {
-    for (int kv = 0; kv < 2; ++kv) {
-      for (int c = 0; c < kTqCodeStages; ++c) {
-        mbar_init(CFULL(kv, c), 1);
-        mbar_init(CFREE(kv, c), kTqDqWarps);
+    const int rows = (s1 - s0) * a.G;
+    const int r0 = blockIdx.z * kRowsPerCta;
+    if (r0 >= rows || gp == 0) return;
+    const int p_begin = static_cast<int>((static_cast<long long>(chunk) * gp) / a.chunks);
+    const int p_end = static_cast<int>((static_cast<long long>(chunk + 1) * gp) / a.chunks);
+    const int nsteps = (p_end - p_begin + kTcPages - 1) / kTcPages;
+    if (nsteps == 0) {  // an empty chunk leaves empty partials
+      for (int r = tid; r < kRowsPerCta; r += blockDim.x) {
+        const int row = r0 + r;
+        if (row >= rows) continue;
+        const size_t idx = ((static_cast<size_t>(chunk) * a.H_kv + h) * a.B + s0 + row / a.G) * a.G +
+                           row % a.G;
+        for (int c = 0; c < D; ++c) a.pre_o[idx * D + c] = 0.f;
+        a.pre_lse[idx] = -INFINITY;
       }
-      for (int s = 0; s < kTcStages; ++s) {
-        mbar_init(TFULL(kv, s), kTqDqWarps);
-        mbar_init(TFREE(kv, s), 1);
-      }
+      return;
     }
-    mbar_init(S_FULL, 1);
-    mbar_init(S_FULL + 8, 1);
-    mbar_init(P_FULL, 4);
-    mbar_init(P_FULL + 8, 4);
-    mbar_init(O_DONE, 1);
-    mbar_init(Q_FULL, 4);
-    mbar_init(DRAIN, 1);
-    mbar_init_fence();
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tbase = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+    const int32_t *bt = a.block_table + static_cast<size_t>(s0) * a.maxb;  // first member's row
+    auto step_pages = [&](int j) { return min(kTcPages, p_end - (p_begin + j * kTcPages)); };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmK);
-      prefetch_tensormap(&tmV);
-      const uint64_t policy = l2_policy_evict_normal();
-      int issued = 0;
-      bool ok = true;
-      for (int j = 0; j < nsteps && ok; ++j) {
-        const int c = j % kTqCodeStages;
-        const uint32_t rel = ((j / kTqCodeStages) - 1) & 1;  // phase of step j - kTqCodeStages
-        const int p0 = p_begin + j * kTcPages, np = step_pages(j);
-        int prow[kTcPages];
-        int good = 0;
-#pragma unroll
-        for (int p = 0; p < kTcPages; ++p) {
-          prow[p] = -1;
-          if (p < np) {
-            const int pb = __ldg(bt + p0 + p);
-            if (pb >= 0 && pb < a.num_blocks) {
-              prow[p] = (pb * a.H_kv + h) * kPage;
-              ++good;
-            } else {
-              flag_error(a.err, kErrBlockTable);
+    const uint32_t tiles0 = smem_u32(tiles), codes0 = smem_u32(codes);
+    const uint32_t scl0 = smem_u32(scl), bar0 = smem_u32(bars);
+    // kv = 0: K, 1: V; c: code stage (kTqCodeStages), s: tile stage (kTcStages)
+    constexpr int kT0 = 4 * kTqCodeStages;  // first tile barrier
+    auto CFULL = [&](int kv, int c) { return bar0 + 8 * (kv * kTqCodeStages + c); };
+    auto CFREE = [&](int kv, int c) { return bar0 + 8 * ((2 + kv) * kTqCodeStages + c); };
+    auto TFULL = [&](int kv, int s) { return bar0 + 8 * (kT0 + kv * kTcStages + s); };
+    auto TFREE = [&](int kv, int s) { return bar0 + 8 * (kT0 + (2 + kv) * kTcStages + s); };
+    const uint32_t S_FULL = bar0 + 8 * (kT0 + 4 * kTcStages);  // + 8 * buffer
+    const uint32_t P_FULL = S_FULL + 16;                 // + 8 * buffer
+    const uint32_t O_DONE = S_FULL + 32, Q_FULL = S_FULL + 40, DRAIN = S_FULL + 48;
+
+    if (warp == 0) {
+      __syncwarp();
+      tc::tmem_alloc(smem_u32(tmem_slot), kTmemColsQ);
+      tc::tmem_relinquish();
+    }
+    if (tid == 32) {
+      for (int kv = 0; kv < 2; ++kv) {
+        for (int c = 0; c < kTqCodeStages; ++c) {
+          mbar_init(CFULL(kv, c), 1);
+          mbar_init(CFREE(kv, c), kTqDqWarps);
+        }
+        for (int s = 0; s < kTcStages; ++s) {
+          mbar_init(TFULL(kv, s), kTqDqWarps);
+          mbar_init(TFREE(kv, s), 1);
+        }
+      }
+      mbar_init(S_FULL, 1);
+      mbar_init(S_FULL + 8, 1);
+      mbar_init(P_FULL, 4);
+      mbar_init(P_FULL + 8, 4);
+      mbar_init(O_DONE, 1);
+      mbar_init(Q_FULL, 4);
+      mbar_init(DRAIN, 1);
+      mbar_init_fence();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        const uint64_t policy = l2_policy_evict_normal();
+        int issued = 0;
+        bool ok = true;
+        for (int j = 0; j < nsteps && ok; ++j) {
+          const int c = j % kTqCodeStages;
+          const uint32_t rel = ((j / kTqCodeStages) - 1) & 1;  // phase of step j - kTqCodeStages
+          const int p0 = p_begin + j * kTcPages, np = step_pages(j);
+          int prow[kTcPages];
+          int good = 0;
+  #pragma unroll
+          for (int p = 0; p < kTcPages; ++p) {
+            prow[p] = -1;
+            if (p < np) {
+              const int pb = __ldg(bt + p0 + p);
+              if (pb >= 0 && pb < a.num_blocks) {
+                prow[p] = (pb * a.H_kv + h) * kPage;
+                ++good;
+              } else {
+                flag_error(a.err, kErrBlockTable);
+              }
             }
           }
+          const uint32_t bytes = static_cast<uint32_t>(good) * (Gq::kCodePage + kTqScalePage);
+          for (int kv = 0; kv < 2; ++kv) {
+            // the codes of step j - kTqCodeStages have been dequantised
+            if (j >= kTqCodeStages && !mbar_wait_bounded(CFREE(kv, c), rel)) {
+              flag_error(a.err, kErrTimeout);
+              ok = false;
+              break;
+            }
+            const uint32_t cst = codes0 + c * Gq::kCodeStage + kv * kTcPages * Gq::kCodePage;
+            const uint32_t sst = scl0 + c * Gq::kScaleStage + kv * kTcPages * kTqScalePage;
+            const float *gs = kv ? a.v_scale : a.k_scale;
+            mbar_arrive_expect_tx(CFULL(kv, c), bytes);
+  #pragma unroll
+            for (int p = 0; p < kTcPages; ++p) {
+              if (prow[p] < 0) continue;
+              tma_load_2d(cst + p * Gq::kCodePage, kv ? &tmV : &tmK, 0, prow[p], CFULL(kv, c), policy);
+              bulk_load(sst + p * kTqScalePage, gs + static_cast<size_t>(prow[p]) * 4, kTqScalePage,
+                        CFULL(kv, c));
+            }
+          }
+          if (ok) issued = j + 1;
         }
-        const uint32_t bytes = static_cast<uint32_t>(good) * (Gq::kCodePage + kTqScalePage);
-        for (int kv = 0; kv < 2; ++kv) {
-          // the codes of step j - kTqCodeStages have been dequantised
-          if (j >= kTqCodeStages && !mbar_wait_bounded(CFREE(kv, c), rel)) {
-            flag_error(a.err, kErrTimeout);
+        // the copies of the last stages have landed before the CTA exits
+        for (int j = max(0, issued - kTqCodeStages); j < issued; ++j)
+          for (int kv = 0; kv < 2; ++kv)
+            mbar_wait_bounded(CFULL(kv, j % kTqCodeStages), (j / kTqCodeStages) & 1);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t fmt = kBf16 ? 1u : 0u;
+        bool ok = mbar_wait_bounded(Q_FULL, 0);
+        tc::fence_after_sync();
+        bool o_started = false;
+        // S[128 x (64 + 64)] = Q . [K_hi; K_lo]^T: A = Q in TMEM, B = the step's
+        // 128 K rows (heads, then remainders) of each 64-channel half; a
+        // partial step's missing rows give columns the softmax masks
+        auto issue_qk = [&](int j) {
+          const int b = j & 1;
+          const uint32_t idesc = tc::idesc_f16(fmt, 2 * kTcTok, false);
+          const uint32_t kst = tiles0 + (j % kTcStages) * kTqStage;
+  #pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t kaddr = kst + (k >> 2) * 2 * kTcHalf + (k & 3) * 32;
+            tc::mma_ts(tbase + kColS + b * 2 * kTcTok, tbase + kColQ + 8 * k,
+                       tc::smem_desc(kaddr, 16, 1024), idesc, k > 0);
+          }
+          tc::commit(TFREE(0, j % kTcStages));
+          tc::commit(S_FULL + 8 * b);
+        };
+        uint32_t pv_mask0 = 0u, pv_mask1 = 0u;  // loaded one step before the PV product uses it
+        auto issue_pv = [&](int j) {
+          const int b = j & 1, s = j % kTcStages;
+          const int np = step_pages(j);
+          const uint32_t mask = (j & 1) ? pv_mask1 : pv_mask0;
+          const uint32_t idesc = tc::idesc_f16(fmt, D, true);
+          const uint32_t vhi = tiles0 + s * kTqStage + 4 * kTcHalf, vlo = vhi + 2 * kTcHalf;
+          for (int kk = 0; kk < np; ++kk) {
+            if (!((mask >> kk) & 1u)) continue;  // (its scores are masked; its tiles are stale)
+            const uint64_t dh = tc::smem_desc(vhi + kk * kPage * 128, kTcHalf, 1024);
+            const uint64_t dl = tc::smem_desc(vlo + kk * kPage * 128, kTcHalf, 1024);
+            const uint32_t pa = tbase + kColS + b * 2 * kTcTok + kk * 8;  // P over S; remainder at +32
+            tc::mma_ts(tbase + kColO, pa, dh, idesc, o_started);
+            o_started = true;
+            tc::mma_ts(tbase + kColO, pa, dl, idesc, true);
+            if (kBf16) tc::mma_ts(tbase + kColO, pa + kTcTok / 2, dh, idesc, true);
+          }
+          tc::commit(TFREE(1, s));
+          tc::commit(O_DONE);
+        };
+        auto wait_pv = [&](int j) {
+          return mbar_wait_bounded(P_FULL + 8 * (j & 1), (j >> 1) & 1) &&
+                 mbar_wait_bounded(TFULL(1, j % kTcStages), (j / kTcStages) & 1);
+        };
+        StepPages ahead;  // the block-table entries of step j, loaded during step j - 1
+        ahead.load(bt, p_begin, p_end, nsteps, 0);
+        for (int j = 0; ok && j < nsteps; ++j) {
+          if (j & 1) pv_mask1 = ahead.mask(a);
+          else pv_mask0 = ahead.mask(a);
+          ahead.load(bt, p_begin, p_end, nsteps, j + 1);
+          if (!mbar_wait_bounded(TFULL(0, j % kTcStages), (j / kTcStages) & 1)) {
             ok = false;
             break;
           }
-          const uint32_t cst = codes0 + c * Gq::kCodeStage + kv * kTcPages * Gq::kCodePage;
-          const uint32_t sst = scl0 + c * Gq::kScaleStage + kv * kTcPages * kTqScalePage;
-          const float *gs = kv ? a.v_scale : a.k_scale;
-          mbar_arrive_expect_tx(CFULL(kv, c), bytes);
-#pragma unroll
-          for (int p = 0; p < kTcPages; ++p) {
-            if (prow[p] < 0) continue;
-            tma_load_2d(cst + p * Gq::kCodePage, kv ? &tmV : &tmK, 0, prow[p], CFULL(kv, c), policy);
-            bulk_load(sst + p * kTqScalePage, gs + static_cast<size_t>(prow[p]) * 4, kTqScalePage,
-                      CFULL(kv, c));
+          tc::fence_after_sync();
+          issue_qk(j);
+          if (j >= 1) {
+            if (!wait_pv(j - 1)) {
+              ok = false;
+              break;
+            }
+            tc::fence_after_sync();
+            issue_pv(j - 1);
           }
         }
-        if (ok) issued = j + 1;
+        if (ok) {
+          const int j = nsteps - 1;
+          if (wait_pv(j)) {
+            tc::fence_after_sync();
+            issue_pv(j);
+          } else {
+            ok = false;
+          }
+        }
+        if (!ok) flag_error(a.err, kErrTimeout);
+        // every MMA issued here completes before TMEM is released
+        tc::commit(DRAIN);
+        mbar_wait_bounded(DRAIN, 0);
       }
-      // the copies of the last stages have landed before the CTA exits
-      for (int j = max(0, issued - kTqCodeStages); j < issued; ++j)
-        for (int kv = 0; kv < 2; ++kv)
-          mbar_wait_bounded(CFULL(kv, j % kTqCodeStages), (j / kTqCodeStages) & 1);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t fmt = kBf16 ? 1u : 0u;
-      bool ok = mbar_wait_bounded(Q_FULL, 0);
-      tc::fence_after_sync();
-      bool o_started = false;
-      // S[128 x (64 + 64)] = Q . [K_hi; K_lo]^T: A = Q in TMEM, B = the step's
-      // 128 K rows (heads, then remainders) of each 64-channel half; a
-      // partial step's missing rows give columns the softmax masks
-      auto issue_qk = [&](int j) {
-        const int b = j & 1;
-        const uint32_t idesc = tc::idesc_f16(fmt, 2 * kTcTok, false);
-        const uint32_t kst = tiles0 + (j % kTcStages) * kTqStage;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t kaddr = kst + (k >> 2) * 2 * kTcHalf + (k & 3) * 32;
-          tc::mma_ts(tbase + kColS + b * 2 * kTcTok, tbase + kColQ + 8 * k,
-                     tc::smem_desc(kaddr, 16, 1024), idesc, k > 0);
-        }
-        tc::commit(TFREE(0, j % kTcStages));
-        tc::commit(S_FULL + 8 * b);
-      };
-      uint32_t pv_mask0 = 0u, pv_mask1 = 0u;  // loaded one step before the PV product uses it
-      auto issue_pv = [&](int j) {
-        const int b = j & 1, s = j % kTcStages;
-        const int np = step_pages(j);
-        const uint32_t mask = (j & 1) ? pv_mask1 : pv_mask0;
-        const uint32_t idesc = tc::idesc_f16(fmt, D, true);
-        const uint32_t vhi = tiles0 + s * kTqStage + 4 * kTcHalf, vlo = vhi + 2 * kTcHalf;
-        for (int kk = 0; kk < np; ++kk) {
-          if (!((mask >> kk) & 1u)) continue;  // (its scores are masked; its tiles are stale)
-          const uint64_t dh = tc::smem_desc(vhi + kk * kPage * 128, kTcHalf, 1024);
-          const uint64_t dl = tc::smem_desc(vlo + kk * kPage * 128, kTcHalf, 1024);
-          const uint32_t pa = tbase + kColS + b * 2 * kTcTok + kk * 8;  // P over S; remainder at +32
-          tc::mma_ts(tbase + kColO, pa, dh, idesc, o_started);
-          o_started = true;
-          tc::mma_ts(tbase + kColO, pa, dl, idesc, true);
-          if (kBf16) tc::mma_ts(tbase + kColO, pa + kTcTok / 2, dh, idesc, true);
-        }
-        tc::commit(TFREE(1, s));
-        tc::commit(O_DONE);
-      };
-      auto wait_pv = [&](int j) {
-        return mbar_wait_bounded(P_FULL + 8 * (j & 1), (j >> 1) & 1) &&
-               mbar_wait_bounded(TFULL(1, j % kTcStages), (j / kTcStages) & 1);
-      };
-      StepPages ahead;  // the block-table entries of step j, loaded during step j - 1
-      ahead.load(bt, p_begin, p_end, nsteps, 0);
-      for (int j = 0; ok && j < nsteps; ++j) {
-        if (j & 1) pv_mask1 = ahead.mask(a);
-        else pv_mask0 = ahead.mask(a);
-        ahead.load(bt, p_begin, p_end, nsteps, j + 1);
-        if (!mbar_wait_bounded(TFULL(0, j % kTcStages), (j / kTcStages) & 1)) {
+    } else if (warp < 6) {
+      // ------------------------------------------------------------ softmax
+      tc_softmax_role<T, true>(a, nullptr, tbase, S_FULL, P_FULL, O_DONE, Q_FULL, warp, lane, r0, rows,
+                               s0, h, chunk, nsteps, bt, p_begin, p_end);
+    } else {
+      // ------------------------------------------------------------ dequantise
+      const int kv = (warp - 6) / kTqDqWarps;  // 0: K (warps 6-8), 1: V (warps 9-11)
+      const int ct = tid - (6 + kv * kTqDqWarps) * 32;
+      bool ok = true;
+      for (int j = 0; j < nsteps; ++j) {
+        const int s = j % kTcStages, c = j % kTqCodeStages;
+        const uint32_t rel = ((j / kTcStages) - 1) & 1;
+        // this step's codes have landed, and the MMAs of step j - kTcStages
+        // have finished reading the tiles about to be overwritten
+        bool got = mbar_wait_bounded(CFULL(kv, c), (j / kTqCodeStages) & 1);
+        if (j >= kTcStages) got = got && mbar_wait_bounded(TFREE(kv, s), rel);
+        if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        issue_qk(j);
-        if (j >= 1) {
-          if (!wait_pv(j - 1)) {
-            ok = false;
-            break;
-          }
-          tc::fence_after_sync();
-          issue_pv(j - 1);
+        // K: halves 2 kTcHalf apart, remainders kTcHalf after the heads;
+        // V: halves kTcHalf apart, remainders 2 kTcHalf after the heads
+        uint8_t *hi = tiles + (size_t)s * kTqStage + kv * 4 * kTcHalf;
+        dequant_half<T, kFmt>(codes + (size_t)c * Gq::kCodeStage + kv * kTcPages * Gq::kCodePage,
+                              reinterpret_cast<const float *>(scl + (size_t)c * Gq::kScaleStage +
+                                                              kv * kTcPages * kTqScalePage),
+                              hi, hi + (kv ? 2 : 1) * kTcHalf, (kv ? 1 : 2) * kTcHalf, ct);
+        fence_proxy_async_smem();  // tiles visible to the tensor core; codes read before refill
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(TFULL(kv, s));
+          mbar_arrive(CFREE(kv, c));
         }
       }
-      if (ok) {
-        const int j = nsteps - 1;
-        if (wait_pv(j)) {
-          tc::fence_after_sync();
-          issue_pv(j);
-        } else {
-          ok = false;
-        }
-      }
-      if (!ok) flag_error(a.err, kErrTimeout);
-      // every MMA issued here completes before TMEM is released
-      tc::commit(DRAIN);
-      mbar_wait_bounded(DRAIN, 0);
+      if (!ok && lane == 0) flag_error(a.err, kErrTimeout);
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------------------ softmax
-    tc_softmax_role<T, true>(a, nullptr, tbase, S_FULL, P_FULL, O_DONE, Q_FULL, warp, lane, r0, rows,
-                             s0, h, chunk, nsteps, bt, p_begin, p_end);
-  } else {
-    // ------------------------------------------------------------ dequantise
-    const int kv = (warp - 6) / kTqDqWarps;  // 0: K (warps 6-8), 1: V (warps 9-11)
-    const int ct = tid - (6 + kv * kTqDqWarps) * 32;
-    bool ok = true;
-    for (int j = 0; j < nsteps; ++j) {
-      const int s = j % kTcStages, c = j % kTqCodeStages;
-      const uint32_t rel = ((j / kTcStages) - 1) & 1;
-      // this step's codes have landed, and the MMAs of step j - kTcStages
-      // have finished reading the tiles about to be overwritten
-      bool got = mbar_wait_bounded(CFULL(kv, c), (j / kTqCodeStages) & 1);
-      if (j >= kTcStages) got = got && mbar_wait_bounded(TFREE(kv, s), rel);
-      if (!__all_sync(0xffffffffu, got)) {
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-      // K: halves 2 kTcHalf apart, remainders kTcHalf after the heads;
-      // V: halves kTcHalf apart, remainders 2 kTcHalf after the heads
-      uint8_t *hi = tiles + (size_t)s * kTqStage + kv * 4 * kTcHalf;
-      dequant_half<T, kFmt>(codes + (size_t)c * Gq::kCodeStage + kv * kTcPages * Gq::kCodePage,
-                            reinterpret_cast<const float *>(scl + (size_t)c * Gq::kScaleStage +
-                                                            kv * kTcPages * kTqScalePage),
-                            hi, hi + (kv ? 2 : 1) * kTcHalf, (kv ? 1 : 2) * kTcHalf, ct);
-      fence_proxy_async_smem();  // tiles visible to the tensor core; codes read before refill
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(TFULL(kv, s));
-        mbar_arrive(CFREE(kv, c));
-      }
-    }
-    if (!ok && lane == 0) flag_error(a.err, kErrTimeout);
-  }
 
-  // release TMEM once every role is done with it
-  tc::fence_before_sync();
-  __syncthreads();
-  if (warp == 0) {
-    __syncwarp();
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tbase, kTmemColsQ);
-  }
+    // release TMEM once every role is done with it
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+      __syncwarp();
+      tc::fence_after_sync();
+      tc::tmem_dealloc(tbase, kTmemColsQ);
+    }
+  }();
+  prefix_exit(a);
 }
 
 int prefix_rows_per_cta() { return kRowsPerCta; }
+
+// Time of one prefix page (one KV head, one row block of up to 128 query
+// rows) relative to one decode page, per SM, as measured on the continuous-
+// batching workload (8 groups x 32 members sharing 4096 tokens, d = 128):
+// the split pays where the suffix decode is bound by HBM (fp16 / bf16 and
+// E4M3 pages), and the two passes trade SMs for nothing where both are
+// bound by their own instructions (INT8 and INT4 pages), so those keep the
+// decode on every SM and the prefix pass only fills the SMs its tail frees.
+#ifndef KVD_PREFIX_W_TC
+#define KVD_PREFIX_W_TC 3.0f  // tensor-memory pass, fp16 / bf16 cache
+#endif
+#ifndef KVD_PREFIX_W_E4M3
+#define KVD_PREFIX_W_E4M3 6.0f  // tensor-memory pass, E4M3 cache
+#endif
+#ifndef KVD_PREFIX_W_INT8
+#define KVD_PREFIX_W_INT8 0.0f
+#endif
+#ifndef KVD_PREFIX_W_INT4
+#define KVD_PREFIX_W_INT4 0.0f
+#endif
+#ifndef KVD_PREFIX_W_WARP
+#define KVD_PREFIX_W_WARP 3.0f  // warp-level passes (d = 64)
+#endif
+void prefix_split(PrefixArgs &a, int d, bool quantised, Code8 fmt, bool split) {
+  bool tc = d == 128;
+#ifdef KVD_PREFIX_MMA_SYNC
+  if (!quantised) tc = false;
+#endif
+  a.ctas_per_sm = tc && !quantised ? 2 : 1;  // prefix_tc_kernel: two per SM
+  if (!split) a.weight = 0.f;
+  else if (!tc) a.weight = KVD_PREFIX_W_WARP;
+  else if (!quantised) a.weight = KVD_PREFIX_W_TC;
+  else if (fmt == Code8::E4M3) a.weight = KVD_PREFIX_W_E4M3;
+  else a.weight = fmt == Code8::INT8 ? KVD_PREFIX_W_INT8 : KVD_PREFIX_W_INT4;
+}
+
+cudaError_t launch_prefix_plan(const PrefixArgs &a, cudaStream_t s) {
+  if (a.n_groups == 0 || a.B == 0) return cudaSuccess;
+  return launch_pdl(prefix_plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, a);
+}
 
 namespace {
 template <typename T>

@@ -64,6 +64,8 @@ CASES = [
     (40, 32, 8, 128, "f16", [530 + 7 * i for i in range(40)], 1, 512, 0),
     # a long shared prefix: several 64-token steps per chunk and a ragged last step
     (16, 64, 8, 128, "bf16", [2100 + 13 * i for i in range(16)], 2, 2048, 0),
+    # the prefix pass outweighs the suffixes (the decode keeps few SMs)
+    (64, 32, 8, 128, "f16", [2049 + (7 * i) % 40 for i in range(64)], 8, 2048, 0),
     # d = 64: the warp-level prefix pass
     (8, 16, 4, 64, "f16", [300, 257, 520, 999, 290, 400, 700, 266], 2, 256, 0),
     (4, 8, 8, 64, "f16", [600, 513, 530, 1000], 1, 512, 5),                  # MHA

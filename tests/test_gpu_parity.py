@@ -366,6 +366,9 @@ SP_CASES = [
     (40, 32, 8, 128, "f16", [530 + 7 * i for i in range(40)], 1, 512, 0),
     # a long shared prefix: several 64-token steps per chunk and a ragged last step
     (16, 64, 8, 128, "bf16", [2100 + 13 * i for i in range(16)], 2, 2048, 0),
+    # the prefix pass outweighs the suffixes: the suffix decode keeps a few
+    # SMs and the prefix pass runs beside it on the rest
+    (64, 32, 8, 128, "f16", [2049 + (7 * i) % 40 for i in range(64)], 8, 2048, 0),
 ]
 
 
