@@ -95,17 +95,21 @@ __device__ __forceinline__ void prefix_exit(const PrefixArgs &a) {
 }
 
 constexpr int kPlanThreads = 256;
+constexpr int kPlanGroups = 2048;  // groups the plan stages in shared memory
 
-// Sum of v over the CTA (kPlanThreads threads); every thread gets it.
-__device__ long long plan_sum(long long v, long long *red) {
+// Sums of v[0..2] over the CTA (kPlanThreads threads); every thread gets them.
+__device__ void plan_sum3(long long (&v)[3], long long (*red)[3]) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+    for (int o = 16; o; o >>= 1) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+  if (lane == 0)
+    for (int i = 0; i < 3; ++i) red[warp][i] = v[i];
   __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  long long t = 0;
-  for (int w = 0; w < kPlanThreads / 32; ++w) t += red[w];
-  return t;
+  for (int i = 0; i < 3; ++i) {
+    v[i] = 0;
+    for (int w = 0; w < kPlanThreads / 32; ++w) v[i] += red[w][i];
+  }
 }
 
 }  // namespace
@@ -120,39 +124,78 @@ __device__ long long plan_sum(long long v, long long *red) {
 //    SMs are then adjusted so that the pass's CTAs fill whole waves there:
 //    a part-filled last wave would leave them idle while the decode runs;
 //  * plan[2..3] = 0, the prefix pass's count of finished warps.
+// The decode launch waits for this one, so its latency is on the step's
+// critical path: with non-decreasing group starts (and at most kPlanGroups
+// groups) every sequence finds its group by a binary search over the starts
+// staged in shared memory, all sequences at once; otherwise write_skip walks
+// the groups in order.
 __global__ void __launch_bounds__(kPlanThreads) prefix_plan_kernel(const PrefixArgs a) {
-  __shared__ long long red[kPlanThreads / 32];
+  __shared__ int g_start[kPlanGroups + 1];
+  __shared__ int g_pages[kPlanGroups];
+  __shared__ long long red[kPlanThreads / 32][3];
   grid_dependency_wait();
   grid_launch_dependents();
   const int tid = threadIdx.x;
   const int cap = a.maxb * kPage;
-  write_skip(a, cap);
-  __syncthreads();  // skip[] of every sequence written (by other threads too)
-  long long sp = 0, pp = 0, cp = 0;  // suffix pages, prefix pages, prefix row blocks
+  const bool staged = a.n_groups <= kPlanGroups;
+  int unordered = 0;
+  if (staged) {
+    for (int g = tid; g <= a.n_groups; g += kPlanThreads) g_start[g] = __ldg(a.group_start + g);
+    for (int g = tid; g < a.n_groups; g += kPlanThreads) g_pages[g] = __ldg(a.group_pages + g);
+    __syncthreads();
+    for (int g = tid; g < a.n_groups; g += kPlanThreads) unordered |= g_start[g + 1] < g_start[g];
+  }
+  const bool search = __syncthreads_or(unordered) == 0 && staged;
+  if (!search) {
+    write_skip(a, cap);
+    __syncthreads();  // skip[] of every sequence written (by other threads too)
+  }
+  long long v[3] = {0, 0, 0};  // suffix pages, prefix pages, prefix row blocks
   for (int b = tid; b < a.B; b += kPlanThreads) {
-    const int np = (clamp_len(__ldcg(a.seq_lens + b), cap) + kPage - 1) / kPage;
-    sp += max(0, np - __ldcg(a.skip + b));
+    const int n = clamp_len(__ldcg(a.seq_lens + b), cap);
+    int sk;
+    if (search) {
+      // the last group starting at or before b holds it, if b is below its end
+      int lo = 0, hi = a.n_groups;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (g_start[mid] <= b) lo = mid + 1; else hi = mid;
+      }
+      const int g = lo - 1;
+      sk = 0;
+      if (g >= 0 && b < g_start[g + 1]) {
+        const int gp = g_pages[g];
+        if (group_ok(a, g_start[g], g_start[g + 1], gp) && gp > 0 && gp * kPage <= n) {
+          sk = gp;
+          // the step's new token must land in a private page
+          if (a.fused && gp * kPage == n) flag_error(a.err, kErrSlot);
+        }
+      }
+      a.skip[b] = sk;
+    } else {
+      sk = __ldcg(a.skip + b);
+    }
+    v[0] += max(0, (n + kPage - 1) / kPage - sk);
   }
   for (int g = tid; g < a.n_groups; g += kPlanThreads) {
-    const int s0 = __ldg(a.group_start + g), s1 = __ldg(a.group_start + g + 1);
-    const int gp = __ldg(a.group_pages + g);
+    const int s0 = staged ? g_start[g] : __ldg(a.group_start + g);
+    const int s1 = staged ? g_start[g + 1] : __ldg(a.group_start + g + 1);
+    const int gp = staged ? g_pages[g] : __ldg(a.group_pages + g);
     if (!group_ok(a, s0, s1, gp) || gp == 0) continue;
     const long long rows = static_cast<long long>(s1 - s0) * a.G;
     const long long rb = (rows + kRowsPerCta - 1) / kRowsPerCta;
-    pp += gp * rb;
-    cp += rb;
+    v[1] += gp * rb;
+    v[2] += rb;
   }
-  sp = plan_sum(sp, red);
-  pp = plan_sum(pp, red);
-  cp = plan_sum(cp, red);
+  plan_sum3(v, red);
   if (tid == 0) {
-    const long long P = sp * a.H_kv, Pp = pp * a.H_kv;
+    const long long P = v[0] * a.H_kv, Pp = v[1] * a.H_kv;
     int N = effective_parts(P, a.nparts, a.min_pages);
     if (a.weight > 0.f && Pp > 0 && a.nparts > 1) {
       const double dp = static_cast<double>(P);
       const double share = dp / (dp + a.weight * static_cast<double>(Pp));
       const double k_raw = fmax(1.0, a.nparts * (1.0 - share));  // SMs for the prefix pass
-      const long long ctas = cp * a.chunks * a.H_kv;               // its CTAs with work
+      const long long ctas = v[2] * a.chunks * a.H_kv;             // its CTAs with work
       const long long slots = a.ctas_per_sm;                        // resident per SM
       const long long waves = max(1LL, llround(static_cast<double>(ctas) / (slots * k_raw)));
       const long long k =

@@ -507,6 +507,29 @@ def test_shared_prefix_uneven_groups(kvd, d, dtype, H_q, H_kv):
     assert float(np.max(np.abs(lse.cpu().double().numpy() - ref_lse))) <= LSE_TOL
 
 
+@pytest.mark.parametrize("starts", [[4, 8, 0, 4], [0, 4, 4, 8]], ids=["unordered", "empty_group"])
+def test_shared_prefix_group_starts_in_any_order(kvd, starts):
+    # Decreasing group starts make the plan walk the groups in order instead
+    # of searching them: [4, 8, 0, 4] names the workload's two groups in
+    # reverse order around an invalid group [8, 0), which is flagged.  With
+    # [0, 4, 4, 8] the search skips the empty middle group.
+    w = build_workload("spo", 8, 32, 8, 128, "f16", [300, 257, 520, 999, 290, 400, 700, 266],
+                       seed=1403, prefix_groups=2, prefix_tokens=256)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    kvd.kvd_append(kc, vc, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    kvd.kvd_read_device_error(clear=True)
+    gs = torch.tensor(starts, dtype=torch.int32, device="cuda")
+    gp = torch.full((3,), 16, dtype=torch.int32, device="cuda")
+    out = kvd.kvd_decode_attention_shared_prefix(si["q"].cuda(), kc, vc, bt, si["seq_lens"].cuda(),
+                                                 gs, gp, 4, w.scale)
+    torch.cuda.synchronize()
+    flagged = kvd.kvd_read_device_error(clear=True)
+    assert bool(flagged & kvd.KVD_DEVERR_SEQ_LEN) == (starts[1] > starts[2])
+    _, _, ref = oracle_step(w, si)
+    assert max_err(out, ref) <= TOL[w.dtype]
+
+
 def test_shared_prefix_group_larger_than_declared_is_flagged_and_attended_whole(kvd):
     # max_group_size below the 40-member group: that group is invalid (its
     # members are attended whole, the error word says so), the others share
