@@ -138,12 +138,18 @@ kvd_status prefix_layout(int B, int H_kv, int G, int d, int n_groups, int max_gr
   const long long rb = (rows + rpc - 1) / rpc;
   if (rb > 65535) return fail(KVD_ERR_UNSUPPORTED, "group of %d sequences too large", max_group_size);
   // each (group, KV head, row block) unit's pages are cut into contiguous
-  // chunks, one CTA each: at d = 128 (tensor-memory pass, two CTAs per SM;
-  // one for a quantised cache) as many as are resident at once; otherwise
-  // about four per SM.  The quantised layout never needs more workspace.
+  // chunks, one CTA each.  At d = 128 (tensor-memory passes) about one CTA
+  // per SM for a quantised cache (one resident per SM) and one per two SMs
+  // for fp16 / bf16 (two resident per SM): the pass streams beside the
+  // suffix decode on the SMs the plan leaves it, where fewer, longer CTAs
+  // pay the Q load and the pipeline fill less often and leave the merge
+  // fewer partials (measured on the continuous-batching workload: 4 chunks
+  // 295.2 us a call, 2 chunks 290.6, 1 chunk 289.5; the quantised pass with
+  // 1 chunk instead of 2 lost 39 us, its 64 CTAs filling too few waves).
+  // At d = 64 about four per SM.
   const long long units = static_cast<long long>(n_groups) * H_kv * rb;
-  long long chunks = d == 128 ? ((quantised ? 1LL : 2LL) * sms) / units
-                              : (4LL * sms + units - 1) / units;
+  long long chunks = d != 128 ? (4LL * sms + units - 1) / units
+                              : (quantised ? sms / units : sms / (2 * units));
   chunks = chunks < 1 ? 1 : (chunks > 64 ? 64 : chunks);
   if (static_cast<long long>(n_groups) * chunks > 0x7fffffffLL)
     return fail(KVD_ERR_UNSUPPORTED, "too many groups");
@@ -697,10 +703,13 @@ size_t kvd_shared_prefix_workspace_size(int B, int H_q, int H_kv, int d, int n_g
   const long long slots = static_cast<long long>(N) + static_cast<long long>(B) * H_kv;
   const WsLayout L0 = ws_layout(B, H_q / H_kv, d, slots);
   if (n_groups == 0) return L0.total;
-  PrefixLayout PL;
-  if (prefix_layout(B, H_kv, H_q / H_kv, d, n_groups, max_group_size, L0.total, &PL) != KVD_OK)
+  // the larger of the fp16 / bf16 and the quantised layouts, so that one
+  // size serves every shared-prefix call
+  PrefixLayout PL, PQ;
+  if (prefix_layout(B, H_kv, H_q / H_kv, d, n_groups, max_group_size, L0.total, &PL) != KVD_OK ||
+      prefix_layout(B, H_kv, H_q / H_kv, d, n_groups, max_group_size, L0.total, &PQ, true) != KVD_OK)
     return 0;
-  return PL.total;
+  return PL.total > PQ.total ? PL.total : PQ.total;
 }
 
 kvd_status kvd_decode_attention_shared_prefix(
