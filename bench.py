@@ -962,7 +962,7 @@ def run_ours(args):
             "l2": "inputs larger than L2 (KV pool %.2f GB >> 126 MB); no flush" % (
                 2 * w.k_cache.numel() * 2 / 1e9),
             "step": ("kvd_decode_attention_shared_prefix_%s with fused quantising append over an %s "
-                     "cache (prefix tensor-core pass with dequantised tiles, decode, merge kernels)"
+                     "cache (plan, decode, prefix tensor-core pass with dequantised tiles beside it, merge kernels)"
                      % (f8["fmt"], f8["name"]) if f8 is not None and sp is not None else
                      "kvd_append_%s + kvd_decode_attention_%s over an %s cache "
                      "(quantising append, decode, merge kernels)" % (f8["fmt"], f8["fmt"], f8["name"])
@@ -970,7 +970,8 @@ def run_ours(args):
                      "kvd_decode_step_%s over an %s cache (decode kernel with fused quantising "
                      "append, merge kernel)" % (f8["fmt"], f8["name"])
                      if f8 is not None else
-                     "kvd_decode_attention_shared_prefix with fused append (prefix, decode, merge kernels)"
+                     "kvd_decode_attention_shared_prefix with fused append (plan, decode, prefix pass beside it, "
+                     "merge kernels)"
                      if sp is not None else
                      "kvd_append + kvd_decode_attention (append, decode, merge kernels)"
                      if args.separate_append else
@@ -987,15 +988,16 @@ def run_ours(args):
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "peak_kind": peak_kind,
-            "kernel": ("kvd_decode_attention_shared_prefix_%s call (prefix_tcq_kernel + decode_kernel over "
-                       "%s pages with fused quantising append + merge)" % (f8["fmt"], f8["name"])
+            "kernel": ("kvd_decode_attention_shared_prefix_%s call (prefix_plan_kernel + decode_kernel over "
+                       "%s pages with fused quantising append + prefix_tcq_kernel + merge)"
+                       % (f8["fmt"], f8["name"])
                        if f8 is not None and sp is not None else
                        "kvd_decode_attention_%s call (decode_kernel over %s pages + merge)"
                        % (f8["fmt"], f8["name"]) if f8 is not None and args.separate_append else
                        "kvd_decode_step_%s call (decode_kernel over %s pages with fused quantising "
                        "append + merge)" % (f8["fmt"], f8["name"]) if f8 is not None else
-                       "kvd_decode_attention_shared_prefix call (prefix_kernel + decode_kernel with fused "
-                       "append + merge)" if sp is not None else
+                       "kvd_decode_attention_shared_prefix call (prefix_plan_kernel + decode_kernel with "
+                       "fused append + prefix_tc_kernel + merge)" if sp is not None else
                        "kvd_decode_attention call (decode_kernel + decode_merge_kernel)"
                        if args.separate_append else
                        "kvd_decode_step call (decode_kernel with fused append + decode_merge_kernel)")
@@ -1036,7 +1038,7 @@ def run_ours(args):
                        "timed call, D2H of out, stream sync; wall clock, max over ranks.  mode "
                        "'cuda graph': those three captured once as a CUDA graph and replayed each "
                        "step (eager: issued from Python each step)"},
-        "gpu_launches": (3 if (args.separate_append or sp is not None) else 2) * args.steps * per,
+        "gpu_launches": (4 if sp is not None else 3 if args.separate_append else 2) * args.steps * per,
         "graph": ({"steps_per_graph": args.graph_steps, "replays": args.steps} if graph is not None
                   else None),
         "clocks": clocks,
