@@ -59,11 +59,15 @@ struct Geo {
   static constexpr int kThreads = 32 * W;
   static constexpr int kSteps = D / 16;                 // k-steps of S, m-tiles of O
   static constexpr int kEdgeFloats = 8 * NT * D;        // one parked accumulator tile
+  // one 8-byte mbarrier per stage, padded so that the 16-byte page
+  // descriptors after them stay aligned whatever W * S is
+  static constexpr int kBarBytes = (W * S * 8 + 15) / 16 * 16;
   static_assert(kEdgeFloats * 4 <= S * kStageBytes, "a parked tile must fit in a warp's ring");
   static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+  static_assert(kAux % 16 == 0, "side data must keep the barriers and descriptors aligned");
   static size_t smem(int B) {
     return 1024 + (size_t)W * S * kStageBytes + (size_t)W * kEdgeFloats * 4 + (size_t)W * S * kAux +
-           (size_t)W * S * 24 +
+           kBarBytes + (size_t)W * S * 16 +
            (size_t)W * 2 * 2 * 8 * NT * 4 + (size_t)W * 2 * 4 + (size_t)(B + 1) * 4;
   }
 };
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(32 * W, 1)
   float *edge_acc = reinterpret_cast<float *>(smem + (size_t)W * S * Gm::kStageBytes);
   uint8_t *aux = reinterpret_cast<uint8_t *>(edge_acc + (size_t)W * Gm::kEdgeFloats);
   uint64_t *bars = reinterpret_cast<uint64_t *>(aux + (size_t)W * S * Gm::kAuxBytes);
-  int4 *meta = reinterpret_cast<int4 *>(bars + W * S);
+  int4 *meta = reinterpret_cast<int4 *>(reinterpret_cast<uint8_t *>(bars) + Gm::kBarBytes);
   float *edge_ml = reinterpret_cast<float *>(meta + W * S);  // [W][2][2][kRows]: m, l
   int *edge_id = reinterpret_cast<int *>(edge_ml + W * 2 * 2 * kRows);  // [W][2]
   int *cum = edge_id + 2 * W;
@@ -1126,10 +1130,9 @@ struct Tune<64, 2> {
   static constexpr int W = KVD_TUNE_W64_2, S = KVD_TUNE_S64_2;
 };
 
-template <int D, int NT, typename T>
-cudaError_t launch_decode_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
-                            cudaStream_t st, int grid) {
-  constexpr int W = Tune<D, NT>::W, S = Tune<D, NT>::S;
+template <int D, int NT, typename T, int W, int S>
+cudaError_t launch_decode_ws(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                             cudaStream_t st, int grid) {
   using Pol = Page16<D, NT, T>;
   auto kern = decode_kernel<D, NT, Pol, W, S>;
   const size_t smem = Geo<D, NT, W, S, Pol::kStride, Pol::kAuxBytes>::smem(a.B);
@@ -1137,6 +1140,31 @@ cudaError_t launch_decode_t(const DecodeArgs &a, const CUtensorMap &tmK, const C
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(32 * W), smem, st, a, tmK, tmV);
+}
+
+// Few (sequence, KV head) pairs -- long contexts, the launches that stream
+// K/V with the evict-first hint -- take fewer warps with two stages each at
+// d = 128: each warp then streams twice the pages, its ring overlaps a
+// page's tile with the next page's copy, and the CTA's warps finish closer
+// together.  `long` (131072 tokens, 8 KV heads), same-box sweeps, us a call:
+// 16 x 1 94.9, 12 x 1 93.1, 10 x 2 93.9, 8 x 2 91.9, 7 x 2 89.9, 6 x 2 91.4,
+// 5 x 2 93.8, 8 x 3 98.7, 6 x 3 92.5, 6 x 4 97.2, 4 x 3 103.6.  The 8-bit
+// tile, bound by its instructions, keeps its 16 warps there (`long --kv-fp8`
+// 60.3 us at 16 x 2 against 64.4 at 12 x 2 and 74.6 at 8 x 4).
+#ifndef KVD_TUNE_WL
+#define KVD_TUNE_WL 7
+#endif
+#ifndef KVD_TUNE_SL
+#define KVD_TUNE_SL 2
+#endif
+template <int D, int NT, typename T>
+cudaError_t launch_decode_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                            cudaStream_t st, int grid) {
+  constexpr int W = Tune<D, NT>::W, S = Tune<D, NT>::S;
+  if constexpr (D == 128 && NT == 1 && (KVD_TUNE_WL != W || KVD_TUNE_SL != S)) {
+    if (a.evict_first) return launch_decode_ws<D, NT, T, KVD_TUNE_WL, KVD_TUNE_SL>(a, tmK, tmV, st, grid);
+  }
+  return launch_decode_ws<D, NT, T, W, S>(a, tmK, tmV, st, grid);
 }
 
 template <typename T>
