@@ -169,10 +169,17 @@ kvd_status kvd_decode_step(const void *q, const void *k_new, const void *v_new, 
  *   k_new, v_new  nullable; when given, the step's new token is appended as
  *                 in kvd_decode_step (it must land in a private page)
  *   workspace     kvd_shared_prefix_workspace_size(...) bytes, 256-aligned
+ *   num_partitions  0: the decode of the private suffixes leaves the shared
+ *                 pass a share of the SMs (sized on the device from the two
+ *                 passes' pages) and the two run side by side; > 0: exactly
+ *                 as in kvd_decode_attention, with no split
  *   other arguments as kvd_decode_attention.
  * The result equals kvd_decode_attention's up to fp32 rounding order (the
  * shared tokens are summed in a separate pass and merged by log-sum-exp).
- * A member shorter than its group's shared pages is attended whole.
+ * A member shorter than its group's shared pages is attended whole.  The
+ * call issues four launches on `stream` (plan, suffix decode, shared pass,
+ * merge); the shared pass may run while the suffix decode does, and the
+ * merge runs after both.
  */
 kvd_status kvd_decode_attention_shared_prefix(
     const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
