@@ -50,7 +50,7 @@ struct DecodeArgs {
   void *k_cache;
   void *v_cache;
   // shared-prefix mode (all null otherwise): skip[b] leading pages of
-  // sequence b were attended by the prefix kernel; those pairs always leave
+  // sequence b are attended by the prefix pass; those pairs always leave
   // partials, and the merge adds the prefix partials pre_o / pre_lse
   // ([pre_chunks][H_kv][B][G][d] and [pre_chunks][H_kv][B][G])
   const int32_t *skip;
@@ -91,7 +91,7 @@ struct PrefixArgs {
   const int32_t *seq_lens;
   const int32_t *group_start;  // [n_groups + 1]: group g = sequences [start[g], start[g+1])
   const int32_t *group_pages;  // [n_groups]: leading pages every member shares
-  int32_t *skip;               // [B] out: shared pages attended here per sequence (0 = none)
+  int32_t *skip;               // [B], written by the plan: shared pages per sequence (0 = none)
   float *pre_o;                // [chunks][H_kv][B][G][d] normalised partial outputs
   float *pre_lse;              // [chunks][H_kv][B][G]
   unsigned *err;
