@@ -393,6 +393,30 @@ def test_shared_prefix_matches_oracle_and_plain_decode(kvd, case):
     assert kvd.kvd_read_device_error() == 0
 
 
+def test_shared_prefix_side_by_side_is_bit_reproducible(kvd):
+    # The prefix pass runs beside the suffix decode, and the split of the SMs
+    # between them is computed on the device.  Neither the split nor the
+    # order in which the two passes finish may change a bit of the output.
+    B = 64
+    w = build_workload("spr", B, 32, 8, 128, "f16", [2049 + (13 * i) % 300 for i in range(B)],
+                       seed=1404, prefix_groups=8, prefix_tokens=2048)
+    si = step_inputs(w, 0)
+    kc, vc, bt = gpu_state(w)
+    kvd.kvd_append(kc, vc, bt, si["slot"].cuda(), si["k_new"].cuda(), si["v_new"].cuda())
+    gs, gp, per = groups_of(w)
+    outs = []
+    for _ in range(3):
+        lse = torch.empty((B, 32), dtype=torch.float32, device="cuda")
+        out = kvd.kvd_decode_attention_shared_prefix(si["q"].cuda(), kc, vc, bt, si["seq_lens"].cuda(),
+                                                     gs, gp, per, w.scale, lse_out=lse)
+        outs.append((out, lse))
+    torch.cuda.synchronize()
+    for o, l in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0][0].view(torch.int16))
+        assert torch.equal(l, outs[0][1])
+    assert kvd.kvd_read_device_error() == 0
+
+
 @pytest.mark.parametrize("scale", [-0.09, 0.0])
 def test_shared_prefix_any_scale(kvd, scale):
     # a negative scale turns the row maximum into a minimum of the raw scores;
