@@ -1142,15 +1142,22 @@ cudaError_t launch_decode_ws(const DecodeArgs &a, const CUtensorMap &tmK, const 
   return launch_pdl(kern, dim3(grid), dim3(32 * W), smem, st, a, tmK, tmV);
 }
 
-// Few (sequence, KV head) pairs -- long contexts, the launches that stream
-// K/V with the evict-first hint -- take fewer warps with two stages each at
-// d = 128: each warp then streams twice the pages, its ring overlaps a
-// page's tile with the next page's copy, and the CTA's warps finish closer
-// together.  `long` (131072 tokens, 8 KV heads), same-box sweeps, us a call:
-// 16 x 1 94.9, 12 x 1 93.1, 10 x 2 93.9, 8 x 2 91.9, 7 x 2 89.9, 6 x 2 91.4,
-// 5 x 2 93.8, 8 x 3 98.7, 6 x 3 92.5, 6 x 4 97.2, 4 x 3 103.6.  The 8-bit
-// tile, bound by its instructions, keeps its 16 warps there (`long --kv-fp8`
-// 60.3 us at 16 x 2 against 64.4 at 12 x 2 and 74.6 at 8 x 4).
+// Launches with at most one (sequence, KV head) pair per warp at 7 warps
+// per CTA take 7 warps with two stages each at d = 128 instead of 16 with
+// one: each warp streams twice the pages, its ring overlaps a page's tile
+// with the next page's copy, and the CTA's warps finish closer together.
+// With more pairs than that, the pair changes (q loads, partial writes)
+// sit on fewer warps' serial paths and 16 x 1 is faster.  Same-box sweeps,
+// us a call:
+//   long (8 pairs): 16 x 1 94.9, 12 x 1 93.1, 10 x 2 93.9, 8 x 2 91.9,
+//     7 x 2 89.9, 6 x 2 91.4, 5 x 2 93.8, 8 x 3 98.7, 6 x 3 92.5, 6 x 4
+//     97.2, 4 x 3 103.6;
+//   gqa70b (512 pairs): 16 x 1 669.8, 7 x 2 652.0, 8 x 2 658.7, 10 x 2 678.0;
+//   mha7b (1024 pairs): 16 x 1 325.6, 7 x 2 322.1, 8 x 2 332.3, 10 x 2 330.3;
+//   cbatch (2048 pairs): 16 x 1 552.5, 7 x 2 674.3; its shared-prefix
+//     suffix decode 291.6 against 306.7.
+// The 8-bit tile, bound by its instructions, keeps its 16 warps (`long
+// --kv-fp8` 60.3 us at 16 x 2 against 64.4 at 12 x 2 and 74.6 at 8 x 4).
 #ifndef KVD_TUNE_WL
 #define KVD_TUNE_WL 7
 #endif
@@ -1162,7 +1169,9 @@ cudaError_t launch_decode_t(const DecodeArgs &a, const CUtensorMap &tmK, const C
                             cudaStream_t st, int grid) {
   constexpr int W = Tune<D, NT>::W, S = Tune<D, NT>::S;
   if constexpr (D == 128 && NT == 1 && (KVD_TUNE_WL != W || KVD_TUNE_SL != S)) {
-    if (a.evict_first) return launch_decode_ws<D, NT, T, KVD_TUNE_WL, KVD_TUNE_SL>(a, tmK, tmV, st, grid);
+    const long long pairs = static_cast<long long>(a.B) * a.H_kv;
+    if (pairs <= static_cast<long long>(KVD_TUNE_WL) * grid)
+      return launch_decode_ws<D, NT, T, KVD_TUNE_WL, KVD_TUNE_SL>(a, tmK, tmV, st, grid);
   }
   return launch_decode_ws<D, NT, T, W, S>(a, tmK, tmV, st, grid);
 }
