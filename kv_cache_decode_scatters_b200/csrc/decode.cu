@@ -25,8 +25,9 @@
 //    TMA tile loads for each page (K and V, each as d/64 boxes of 16 x 64
 //    elements with the 128-byte swizzle) that complete on the stage's
 //    mbarrier; the whole warp waits, computes, and hands the stage back to
-//    the next page.  Latency is hidden by many warps (12-16 per SM) rather
-//    than by deep per-warp rings.
+//    the next page.  Latency is hidden by many warps (12-16 per SM, one
+//    or two stages each; 7 with two stages where the pairs fit one per
+//    warp) rather than by deep per-warp rings.
 //  * Every KV byte is read once per GQA group: the G query rows of a KV head
 //    ride along as the N dimension of the tensor-core tile.  Per page,
 //    S^T[16 tokens x 8 rows] = K[16 x d] . Q^T uses mma.m16n8k16 with the K

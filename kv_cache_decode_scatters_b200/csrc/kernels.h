@@ -119,7 +119,7 @@ struct GenericMergeArgs {
 };
 
 // Partitions used when the caller asks for the automatic count: one CTA per
-// SM of a device with `sms` SMs (each CTA runs 12-16 worker warps).
+// SM of a device with `sms` SMs (each CTA runs 7-16 worker warps).
 int decode_auto_parts(int sms);
 
 // Set the text returned by kvd_last_error on this host thread.
