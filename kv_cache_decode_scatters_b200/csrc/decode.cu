@@ -1288,10 +1288,10 @@ cudaError_t launch_decode8_ws(const DecodeArgs &a, const CUtensorMap &tmK, const
 
 // The tuned ring depth, or one stage per warp when the batch's prefix sums
 // (4 bytes per sequence) would push the tuned layout past the CTA limit.
-template <int D, int NT, typename T, Code8 kFmt, bool kG1>
+template <int D, int NT, typename T, Code8 kFmt, bool kG1, int W = Tune8<D, NT>::W,
+          int S = Tune8<D, NT>::S>
 cudaError_t launch_decode8_tg(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                               cudaStream_t st, int grid) {
-  constexpr int W = Tune8<D, NT>::W, S = Tune8<D, NT>::S;
   using Pol = Pol8<D, NT, T, kFmt, kG1>;
   // one stage must still hold a parked accumulator tile
   constexpr bool kCanShrink = S > 1 && 8 * NT * D * 4 <= Pol::kStride;
@@ -1302,10 +1302,20 @@ cudaError_t launch_decode8_tg(const DecodeArgs &a, const CUtensorMap &tmK, const
   return launch_decode8_ws<D, NT, T, kFmt, W, S, kG1>(a, tmK, tmV, st, grid);
 }
 
+// One query row per KV head (G = 1) over E4M3 pages at d = 128 takes 12
+// warps x 2 stages: its hardware conversion leaves the tile few enough
+// instructions that fewer warps hide them, and each keeps its own pages in
+// flight.  INT8's conversion runs on the ALU and keeps 16 warps.
+// `mha7b` (G = 1), same box, us a call, E4M3 / INT8: 16 x 2 201.6 / 196.5,
+// 12 x 2 196.1 / 205.7, 14 x 2 197.9 / 208.2, 12 x 3 198.5 / 204.1,
+// 10 x 2 212.7 / 240.0.
 template <int D, int NT, typename T, Code8 kFmt>
 cudaError_t launch_decode8_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                              cudaStream_t st, int grid) {
   if constexpr (NT == 1) {
+    if constexpr (D == 128 && kFmt == Code8::E4M3) {
+      if (a.G == 1) return launch_decode8_tg<D, 1, T, kFmt, true, 12, 2>(a, tmK, tmV, st, grid);
+    }
     if (a.G == 1) return launch_decode8_tg<D, 1, T, kFmt, true>(a, tmK, tmV, st, grid);
   }
   return launch_decode8_tg<D, NT, T, kFmt, false>(a, tmK, tmV, st, grid);
